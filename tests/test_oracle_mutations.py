@@ -1,0 +1,128 @@
+"""Planted mistakes: each plausible bug in the oracle must fail at least one pin.
+
+Mistakes are planted in the CPU oracle only (monkeypatched module globals).
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle.model as om
+from tests import oracle_pins as pins
+
+TOL = 1e-6
+
+# originals, captured before any test patches the module
+ORIG = {n: getattr(om, n) for n in ("rotary", "layer_norm", "gelu", "attend",
+                                    "embed_blocks", "prefix_projection",
+                                    "pythia_layer")}
+
+
+def _first_failing_pin(mod):
+    """Name of the first pin the module fails, or None. Exceptions propagate:
+    a mutation that merely crashes does not count as caught."""
+    checks = [
+        ("layer_norm", lambda: pins.pin_layer_norm(mod) < TOL),
+        ("gelu", lambda: pins.pin_gelu(mod) < TOL),
+        ("attend", lambda: pins.pin_attend(mod) < TOL),
+        ("rotary", lambda: pins.pin_rotary(mod) < TOL),
+        ("embedder", lambda: pins.pin_embedder_bruteforce(mod) == 0.0),
+        ("identity_prefix", lambda: pins.pin_identity_prefix(mod) < TOL),
+        ("single_row", lambda: pins.pin_single_row_token_decoder(mod) < TOL),
+        ("future_invisible", lambda: pins.pin_future_tokens_invisible(mod)),
+        ("locality_nb0", lambda: pins.pin_locality_without_block_layers(mod)),
+        ("incremental", lambda: pins.pin_incremental_equals_full(mod) < TOL),
+        ("hf_vanilla", lambda: pins.pin_vanilla_vs_hf(mod) < TOL),
+        ("hf_block_model", lambda: pins.pin_block_model_vs_hf(mod) < TOL),
+    ]
+    for name, c in checks:
+        if not c():
+            return name
+    return None
+
+
+def _rotary_wrong_sign(x, pos, r, base):
+    return ORIG["rotary"](x, -pos, r, base)
+
+
+def _rotary_wrong_freq(x, pos, r, base):
+    # exponent over the head dim instead of the rotary dims
+    return ORIG["rotary"](x, pos, r, base ** 2)
+
+
+def _ln_unbiased(x, g, b, eps):
+    mu = x.mean(-1, keepdims=True)
+    var = ((x - mu) ** 2).sum(-1, keepdims=True) / (x.shape[-1] - 1)
+    return (x - mu) / np.sqrt(var + eps) * g + b
+
+
+def _gelu_tanh(x):
+    return 0.5 * x * (1 + np.tanh(math.sqrt(2 / math.pi) * (x + 0.044715 * x ** 3)))
+
+
+def _attend_no_mask(q, k, v, q_pos, k_pos):
+    return ORIG["attend"](q, k, v, np.full_like(q_pos, 10 ** 9), k_pos)
+
+
+def _attend_scale_d(q, k, v, q_pos, k_pos):
+    return ORIG["attend"](q / math.sqrt(q.shape[-1]), k, v, q_pos, k_pos)
+
+
+def _embed_reversed(tokens, table, L):
+    return ORIG["embed_blocks"](tokens[:, ::-1].copy(), table, L)[:, ::-1]
+
+
+def _embed_reversed_within_block(tokens, table, L):
+    B, S = tokens.shape
+    n = S // L
+    t = tokens[:, :n * L].reshape(B, n, L)[:, :, ::-1].reshape(B, n * L)
+    return ORIG["embed_blocks"](t, table, L)
+
+
+def _prefix_colmajor(c, w, b, P):
+    D = c.shape[-1]
+    out = c @ w.T + b
+    return np.swapaxes(out.reshape(*c.shape[:-1], D, P), -1, -2)
+
+
+def _layer_drop_bias_o(h, p, pos, cache, H, r, eps, base):
+    p2 = dict(p)
+    p2["b_o"] = np.zeros_like(p["b_o"])
+    return ORIG["pythia_layer"](h, p2, pos, cache, H, r, eps, base)
+
+
+def _layer_serial_residual(h, p, pos, cache, H, r, eps, base):
+    # GPT-2 style sequential residual instead of Pythia's parallel form
+    p_att = dict(p)
+    for n in ("w_1", "b_1", "w_2", "b_2"):
+        p_att[n] = np.zeros_like(p[n])
+    h1 = ORIG["pythia_layer"](h, p_att, pos, cache, H, r, eps, base)
+    m = ORIG["layer_norm"](h1, p["ln2_g"], p["ln2_b"], eps)
+    return h1 + ORIG["gelu"](m @ p["w_1"].T + p["b_1"]) @ p["w_2"].T + p["b_2"]
+
+
+MUTATIONS = {
+    "rotary_sign": ("rotary", _rotary_wrong_sign),
+    "rotary_freq": ("rotary", _rotary_wrong_freq),
+    "ln_unbiased": ("layer_norm", _ln_unbiased),
+    "gelu_tanh": ("gelu", _gelu_tanh),
+    "attend_no_mask": ("attend", _attend_no_mask),
+    "attend_scale_d": ("attend", _attend_scale_d),
+    "embed_reversed": ("embed_blocks", _embed_reversed_within_block),
+    "prefix_colmajor": ("prefix_projection", _prefix_colmajor),
+    "drop_b_o": ("pythia_layer", _layer_drop_bias_o),
+    "serial_residual": ("pythia_layer", _layer_serial_residual),
+}
+
+
+def test_unmutated_oracle_passes_every_pin():
+    assert _first_failing_pin(om) is None
+
+
+@pytest.mark.parametrize("mutation", sorted(MUTATIONS))
+def test_planted_mistake_is_caught(mutation, monkeypatch):
+    name, fn = MUTATIONS[mutation]
+    monkeypatch.setattr(om, name, fn)
+    caught_by = _first_failing_pin(om)
+    print(f"{mutation}: caught by {caught_by}")
+    assert caught_by is not None, f"no pin caught the planted mistake {mutation}"
