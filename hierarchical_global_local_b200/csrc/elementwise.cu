@@ -1,0 +1,363 @@
+// elementwise.cu -- embedder, decode ingest, LayerNorm, rotary + KV append,
+// argmax and small conversions for the Block Transformer (sm_100a).
+//
+// Model: "Block Transformer: Global-to-Local Language Modeling for Fast
+// Inference" (explainer page of arXiv 2406.02657). Embedder: §3.4 "The
+// Embedder" [orig. §2.2] -- L_B lookups of width D/L_B concatenated, token j
+// of a block in dims [j*D/L_B, (j+1)*D/L_B). Layer pieces follow the Pythia
+// architecture named in §5 "Experimental setup" (LayerNorm with biased
+// variance, rotate-half rotary on the first 25% of each head).
+#include "common.cuh"
+#include "kernels.h"
+
+namespace bt {
+
+// ---------------------------------------------------------------------------
+// embedder
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void embed_prompt_kernel(const int32_t* __restrict__ tokens, int T_len, int n, int L_B,
+                                    const T* __restrict__ table, int V, int D,
+                                    float* __restrict__ h, int* status) {
+  const int r = blockIdx.x;  // row = b * n + i
+  const int b = r / n, i = r % n;
+  const int De = D / L_B;
+  for (int x = threadIdx.x; x < D; x += blockDim.x) {
+    const int j = x / De, e = x - j * De;
+    int tok = tokens[(size_t)b * T_len + (size_t)i * L_B + j];
+    if (tok < 0 || tok >= V) {
+      set_status(status, ST_BAD_TOKEN);
+      tok = 0;
+    }
+    h[(size_t)r * D + x] = to_f(table[(size_t)tok * De + e]);
+  }
+}
+
+template <typename T>
+__global__ void ingest_kernel(const int32_t* __restrict__ src, int32_t* __restrict__ block_tok,
+                              const int* __restrict__ dstate, int L_B, int V, int D,
+                              int block_step, const T* __restrict__ blk_emb,
+                              const T* __restrict__ tok_emb, float* __restrict__ h,
+                              int* status) {
+  const int b = blockIdx.x;
+  const int j = dstate[1];
+  int tok = src[b];
+  if (tok < 0 || tok >= V) {
+    if (threadIdx.x == 0) set_status(status, ST_BAD_TOKEN);
+    tok = 0;
+  }
+  if (threadIdx.x == 0) block_tok[b * L_B + j] = tok;
+  if (!block_step) {
+    for (int x = threadIdx.x; x < D; x += blockDim.x)
+      h[(size_t)b * D + x] = to_f(tok_emb[(size_t)tok * D + x]);
+  } else {
+    const int De = D / L_B;
+    for (int x = threadIdx.x; x < D; x += blockDim.x) {
+      const int jj = x / De, e = x - jj * De;
+      int t = (jj == j) ? tok : block_tok[b * L_B + jj];
+      if (t < 0 || t >= V) t = 0;
+      h[(size_t)b * D + x] = to_f(blk_emb[(size_t)t * De + e]);
+    }
+  }
+}
+
+__global__ void set_state_kernel(int* dstate, int t, int L_B) {
+  dstate[0] = t;
+  dstate[1] = t % L_B;
+  dstate[2] = t / L_B;
+}
+
+__global__ void advance_kernel(int* dstate, int L_B) {
+  const int t = dstate[0] + 1;
+  dstate[0] = t;
+  dstate[1] = t % L_B;
+  dstate[2] = t / L_B;
+}
+
+cudaError_t launch_embed_prompt(int dt, const int32_t* tokens, int B, int T, int L_B,
+                                const void* blk_emb, int V, int D, float* h, int* status,
+                                cudaStream_t s) {
+  const int n = T / L_B;
+  if (B * n == 0) return cudaSuccess;
+  if (dt == DT_BF16)
+    embed_prompt_kernel<bf16><<<B * n, 256, 0, s>>>(tokens, T, n, L_B, (const bf16*)blk_emb, V, D,
+                                                    h, status);
+  else
+    embed_prompt_kernel<float><<<B * n, 256, 0, s>>>(tokens, T, n, L_B, (const float*)blk_emb, V,
+                                                     D, h, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ingest(int dt, const int32_t* src, int32_t* block_tok, const int* dstate,
+                          int B, int L_B, int V, int D, int block_step, const void* blk_emb,
+                          const void* tok_emb, float* h, int* status, cudaStream_t s) {
+  if (dt == DT_BF16)
+    ingest_kernel<bf16><<<B, 256, 0, s>>>(src, block_tok, dstate, L_B, V, D, block_step,
+                                          (const bf16*)blk_emb, (const bf16*)tok_emb, h, status);
+  else
+    ingest_kernel<float><<<B, 256, 0, s>>>(src, block_tok, dstate, L_B, V, D, block_step,
+                                           (const float*)blk_emb, (const float*)tok_emb, h,
+                                           status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_set_state(int* dstate, int t, int L_B, cudaStream_t s) {
+  set_state_kernel<<<1, 1, 0, s>>>(dstate, t, L_B);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_advance(int* dstate, int L_B, cudaStream_t s) {
+  advance_kernel<<<1, 1, 0, s>>>(dstate, L_B);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// LayerNorm: one warp per row, two-pass (mean, then centred variance) in fp32
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void row_stats(const float* __restrict__ x, int D, float& mu,
+                                          float& rstd, float eps) {
+  const int lane = threadIdx.x & 31;
+  float s = 0.f;
+  for (int i = lane * 4; i < D; i += 128) {
+    float4 v = *reinterpret_cast<const float4*>(x + i);
+    s += (v.x + v.y) + (v.z + v.w);
+  }
+  mu = warp_sum(s) / (float)D;
+  float q = 0.f;
+  for (int i = lane * 4; i < D; i += 128) {
+    float4 v = *reinterpret_cast<const float4*>(x + i);
+    float a = v.x - mu, b = v.y - mu, c = v.z - mu, d = v.w - mu;
+    q += (a * a + b * b) + (c * c + d * d);
+  }
+  rstd = rsqrtf(warp_sum(q) / (float)D + eps);
+}
+
+template <typename T>
+__device__ __forceinline__ void store4(T* out, int i, float a, float b, float c, float d);
+template <>
+__device__ __forceinline__ void store4<float>(float* out, int i, float a, float b, float c, float d) {
+  *reinterpret_cast<float4*>(out + i) = make_float4(a, b, c, d);
+}
+template <>
+__device__ __forceinline__ void store4<bf16>(bf16* out, int i, float a, float b, float c, float d) {
+  __nv_bfloat162 lo = __floats2bfloat162_rn(a, b), hi = __floats2bfloat162_rn(c, d);
+  uint2 u;
+  u.x = *reinterpret_cast<uint32_t*>(&lo);
+  u.y = *reinterpret_cast<uint32_t*>(&hi);
+  *reinterpret_cast<uint2*>(out + i) = u;
+}
+
+template <typename T>
+__global__ void ln_dual_kernel(const float* __restrict__ h, int M, int D,
+                               const float* __restrict__ g1, const float* __restrict__ b1,
+                               const float* __restrict__ g2, const float* __restrict__ b2,
+                               float eps, T* __restrict__ x1) {
+  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (row >= M) return;
+  const int lane = threadIdx.x & 31;
+  const float* x = h + (size_t)row * D;
+  float mu, rstd;
+  row_stats(x, D, mu, rstd, eps);
+  T* o = x1 + (size_t)row * 2 * D;
+  for (int i = lane * 4; i < D; i += 128) {
+    float4 v = *reinterpret_cast<const float4*>(x + i);
+    float n0 = (v.x - mu) * rstd, n1 = (v.y - mu) * rstd, n2 = (v.z - mu) * rstd,
+          n3 = (v.w - mu) * rstd;
+    float4 ga = *reinterpret_cast<const float4*>(g1 + i), ba = *reinterpret_cast<const float4*>(b1 + i);
+    float4 gb = *reinterpret_cast<const float4*>(g2 + i), bb = *reinterpret_cast<const float4*>(b2 + i);
+    store4<T>(o, i, n0 * ga.x + ba.x, n1 * ga.y + ba.y, n2 * ga.z + ba.z, n3 * ga.w + ba.w);
+    store4<T>(o + D, i, n0 * gb.x + bb.x, n1 * gb.y + bb.y, n2 * gb.z + bb.z, n3 * gb.w + bb.w);
+  }
+}
+
+template <typename T>
+__global__ void ln_rows_kernel(const float* __restrict__ h, int R, int row_step, int row_off,
+                               int D, const float* __restrict__ g, const float* __restrict__ b,
+                               float eps, T* __restrict__ out) {
+  const int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (r >= R) return;
+  const int lane = threadIdx.x & 31;
+  const float* x = h + ((size_t)r * row_step + row_off) * D;
+  float mu, rstd;
+  row_stats(x, D, mu, rstd, eps);
+  T* o = out + (size_t)r * D;
+  for (int i = lane * 4; i < D; i += 128) {
+    float4 v = *reinterpret_cast<const float4*>(x + i);
+    float4 ga = *reinterpret_cast<const float4*>(g + i), ba = *reinterpret_cast<const float4*>(b + i);
+    store4<T>(o, i, (v.x - mu) * rstd * ga.x + ba.x, (v.y - mu) * rstd * ga.y + ba.y,
+              (v.z - mu) * rstd * ga.z + ba.z, (v.w - mu) * rstd * ga.w + ba.w);
+  }
+}
+
+cudaError_t launch_ln_dual(int dt, const float* h, int M, int D, const float* g1,
+                           const float* b1, const float* g2, const float* b2, float eps,
+                           void* x1, cudaStream_t s) {
+  if (M == 0) return cudaSuccess;
+  const int rows_per_cta = 8;
+  dim3 grid((M + rows_per_cta - 1) / rows_per_cta);
+  if (dt == DT_BF16)
+    ln_dual_kernel<bf16><<<grid, 256, 0, s>>>(h, M, D, g1, b1, g2, b2, eps, (bf16*)x1);
+  else
+    ln_dual_kernel<float><<<grid, 256, 0, s>>>(h, M, D, g1, b1, g2, b2, eps, (float*)x1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ln_rows(int dt, const float* h, int R, int row_step, int row_off, int D,
+                           const float* g, const float* b, float eps, void* out, cudaStream_t s) {
+  if (R == 0) return cudaSuccess;
+  dim3 grid((R + 7) / 8);
+  if (dt == DT_BF16)
+    ln_rows_kernel<bf16><<<grid, 256, 0, s>>>(h, R, row_step, row_off, D, g, b, eps, (bf16*)out);
+  else
+    ln_rows_kernel<float><<<grid, 256, 0, s>>>(h, R, row_step, row_off, D, g, b, eps, (float*)out);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// rotary table + rotary/append
+// ---------------------------------------------------------------------------
+__global__ void rope_table_kernel(float2* tab, int n_pos, int half, double base) {
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= n_pos * half) return;
+  const int p = idx / half, i = idx - p * half;
+  // angle = p * base^(-2i/rot), rot = 2*half
+  const double inv = pow(base, -(double)(2 * i) / (double)(2 * half));
+  double sn, cs;
+  sincos((double)p * inv, &sn, &cs);
+  tab[idx] = make_float2((float)cs, (float)sn);
+}
+
+cudaError_t launch_rope_table(float2* tab, int n_pos, int rot, float base, cudaStream_t s) {
+  const int half = rot / 2;
+  if (half == 0 || n_pos == 0) return cudaSuccess;
+  const int total = n_pos * half;
+  rope_table_kernel<<<(total + 255) / 256, 256, 0, s>>>(tab, n_pos, half, (double)base);
+  return cudaGetLastError();
+}
+
+template <typename T>
+__global__ void rope_append_kernel(const T* __restrict__ qkv, int D, int H, int rot,
+                                   const float2* __restrict__ tab, PosSpec ps,
+                                   T* __restrict__ q_out, T* __restrict__ kc,
+                                   T* __restrict__ vc, int cap) {
+  const int m = blockIdx.x;
+  const int d = D / H;
+  const int half = rot >> 1;
+  const int b = m / ps.rows_per_seq;
+  const int pos = pos_base(ps) + (m - b * ps.rows_per_seq);
+  const T* row = qkv + (size_t)m * 3 * D;
+  for (int x = threadIdx.x; x < 3 * D; x += blockDim.x) {
+    const int part = x / D;  // 0 q, 1 k, 2 v
+    const int c = x - part * D;
+    const int hh = c / d, e = c - hh * d;
+    float v = to_f(row[x]);
+    if (part < 2 && e < rot) {
+      const int i = (e < half) ? e : e - half;
+      const float2 cs = tab[(size_t)pos * half + i];
+      if (e < half) v = v * cs.x - to_f(row[x + half]) * cs.y;
+      else v = v * cs.x + to_f(row[x - half]) * cs.y;
+    }
+    if (part == 0) {
+      q_out[(size_t)m * D + c] = from_f<T>(v);
+    } else {
+      T* cache = (part == 1) ? kc : vc;
+      cache[(((size_t)b * H + hh) * cap + pos) * d + e] = from_f<T>(v);
+    }
+  }
+}
+
+cudaError_t launch_rope_append(int dt, const void* qkv, int M, int D, int H, int rot,
+                               const float2* rope_tab, PosSpec pos, void* q_out, void* k_cache,
+                               void* v_cache, int cap, cudaStream_t s) {
+  if (M == 0) return cudaSuccess;
+  if (dt == DT_BF16)
+    rope_append_kernel<bf16><<<M, 256, 0, s>>>((const bf16*)qkv, D, H, rot, rope_tab, pos,
+                                               (bf16*)q_out, (bf16*)k_cache, (bf16*)v_cache, cap);
+  else
+    rope_append_kernel<float><<<M, 256, 0, s>>>((const float*)qkv, D, H, rot, rope_tab, pos,
+                                                (float*)q_out, (float*)k_cache, (float*)v_cache,
+                                                cap);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// argmax over the vocabulary (lowest id among ties)
+// ---------------------------------------------------------------------------
+__global__ void argmax_kernel(const float* __restrict__ logits, int V, int ld,
+                              int32_t* __restrict__ next) {
+  const int b = blockIdx.x;
+  const float* z = logits + (size_t)b * ld;
+  float best = -INFINITY;
+  int bi = 0x7fffffff;
+  for (int v = threadIdx.x; v < V; v += blockDim.x) {
+    const float x = z[v];
+    if (x > best || (x == best && v < bi)) { best = x; bi = v; }
+  }
+  __shared__ float sv[32];
+  __shared__ int si[32];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float ov = __shfl_xor_sync(0xffffffffu, best, o);
+    const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+    if (ov > best || (ov == best && oi < bi)) { best = ov; bi = oi; }
+  }
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) { sv[w] = best; si[w] = bi; }
+  __syncthreads();
+  if (w == 0) {
+    const int nw = blockDim.x >> 5;
+    best = lane < nw ? sv[lane] : -INFINITY;
+    bi = lane < nw ? si[lane] : 0x7fffffff;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, best, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ov > best || (ov == best && oi < bi)) { best = ov; bi = oi; }
+    }
+    if (lane == 0) next[b] = (bi == 0x7fffffff) ? 0 : bi;
+  }
+}
+
+cudaError_t launch_argmax(const float* logits, int B, int V, int ld, int32_t* next,
+                          cudaStream_t s) {
+  if (B == 0) return cudaSuccess;
+  argmax_kernel<<<B, 1024, 0, s>>>(logits, V, ld, next);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// conversions used when the model is created
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void convert_kernel(const T* __restrict__ src, float* __restrict__ dst, size_t n) {
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n;
+       i += (size_t)gridDim.x * blockDim.x)
+    dst[i] = to_f(src[i]);
+}
+
+template <typename T>
+__global__ void add_kernel(const T* __restrict__ a, const T* __restrict__ b,
+                           float* __restrict__ dst, size_t n) {
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n;
+       i += (size_t)gridDim.x * blockDim.x)
+    dst[i] = to_f(a[i]) + to_f(b[i]);
+}
+
+cudaError_t launch_convert_to_f32(int dt, const void* src, float* dst, size_t n, cudaStream_t s) {
+  if (n == 0) return cudaSuccess;
+  const int grid = (int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
+  if (dt == DT_BF16) convert_kernel<bf16><<<grid, 256, 0, s>>>((const bf16*)src, dst, n);
+  else convert_kernel<float><<<grid, 256, 0, s>>>((const float*)src, dst, n);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_add_to_f32(int dt, const void* a, const void* b, float* dst, size_t n,
+                              cudaStream_t s) {
+  if (n == 0) return cudaSuccess;
+  const int grid = (int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
+  if (dt == DT_BF16) add_kernel<bf16><<<grid, 256, 0, s>>>((const bf16*)a, (const bf16*)b, dst, n);
+  else add_kernel<float><<<grid, 256, 0, s>>>((const float*)a, (const float*)b, dst, n);
+  return cudaGetLastError();
+}
+
+}  // namespace bt

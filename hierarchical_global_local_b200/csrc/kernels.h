@@ -1,0 +1,122 @@
+// kernels.h -- host-side launchers of the Block Transformer kernels.
+// Every launcher enqueues on the given stream and returns the launch's
+// cudaError_t (cudaSuccess when nothing was launched).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace bt {
+
+enum DType : int { DT_F32 = 0, DT_BF16 = 1 };
+inline size_t dt_size(int dt) { return dt == DT_F32 ? 4 : 2; }
+
+// ---- embedder / token ingest / step state --------------------------------
+// Prompt embedder: h[b*n + i, :] = concat_j blk_emb[tokens[b, i*L_B + j]].
+cudaError_t launch_embed_prompt(int dt, const int32_t* tokens, int B, int T, int L_B,
+                                const void* blk_emb, int V, int D, float* h, int* status,
+                                cudaStream_t s);
+// Decode ingest of the fed token src[b] at position t = dstate[0]:
+// records it in block_tok[b, t % L_B]; block_step = 0 gathers
+// h[b] = tok_emb[src[b]]; block_step = 1 (the token completes its block)
+// gathers h[b] = concat_j blk_emb[block_tok[b, j]].
+cudaError_t launch_ingest(int dt, const int32_t* src, int32_t* block_tok, const int* dstate,
+                          int B, int L_B, int V, int D, int block_step, const void* blk_emb,
+                          const void* tok_emb, float* h, int* status, cudaStream_t s);
+// dstate <- position t (t, t % L_B, t / L_B).
+cudaError_t launch_set_state(int* dstate, int t, int L_B, cudaStream_t s);
+// dstate <- dstate[0] + 1.
+cudaError_t launch_advance(int* dstate, int L_B, cudaStream_t s);
+
+// ---- LayerNorm ------------------------------------------------------------
+// x1[m, 0:D] = LN(h[m]; g1, b1), x1[m, D:2D] = LN(h[m]; g2, b2) (act dtype).
+cudaError_t launch_ln_dual(int dt, const float* h, int M, int D, const float* g1,
+                           const float* b1, const float* g2, const float* b2, float eps,
+                           void* x1, cudaStream_t s);
+// out[r] = LN(h[r * row_step + row_off]; g, b) for r < R (act dtype).
+cudaError_t launch_ln_rows(int dt, const float* h, int R, int row_step, int row_off, int D,
+                           const float* g, const float* b, float eps, void* out, cudaStream_t s);
+
+// ---- rotary + KV append ---------------------------------------------------
+// Row m of qkv [M, 3D] belongs to sequence m / rows_per_seq at position
+// pos_base(pos) + m % rows_per_seq. Writes rotated q to q_out [M, D] and
+// rotated k, v to the caches [B][H][cap][d] at that position.
+// rope_tab[p * (rot/2) + i] = (cos, sin) of p * base^(-2i/rot).
+cudaError_t launch_rope_append(int dt, const void* qkv, int M, int D, int H, int rot,
+                               const float2* rope_tab, PosSpec pos, void* q_out, void* k_cache,
+                               void* v_cache, int cap, cudaStream_t s);
+cudaError_t launch_rope_table(float2* tab, int n_pos, int rot, float base, cudaStream_t s);
+
+// ---- attention --------------------------------------------------------------
+// Split-K flash decoding: one query per (b, h) (q row b of q [B, ldq]) over
+// the first n = pos_base(kvlen) + 1 cache entries; out[b, h*d:(h+1)*d].
+// part / counters: scratch of attn_decode_scratch_bytes(); counters must be
+// zero before the first launch and are left zero.
+size_t attn_decode_scratch_bytes(int B, int H, int d, int cap, int dt);
+int attn_decode_max_splits(int d, int cap, int dt);
+cudaError_t launch_attn_decode(int dt, const void* q, int ldq, const void* k_cache,
+                               const void* v_cache, int B, int H, int d, int cap,
+                               PosSpec kvlen, void* out, int ld_out, void* scratch,
+                               int* status, cudaStream_t s);
+// Small causal attention: rows_per_seq queries per sequence at positions
+// pos_base(qpos) + i; query at position p attends to cache entries 0..p.
+cudaError_t launch_attn_small(int dt, const void* q, int ldq, const void* k_cache,
+                              const void* v_cache, int B, int H, int d, int cap, PosSpec qpos,
+                              void* out, int ld_out, cudaStream_t s);
+// Prefill causal attention over n positions 0..n-1 of every sequence:
+// q rows b*n + i of q [B*n, ldq]; out rows likewise.
+cudaError_t launch_attn_prefill(int dt, const void* q, int ldq, const void* k_cache,
+                                const void* v_cache, int B, int H, int d, int cap, int n,
+                                void* out, int ld_out, cudaStream_t s);
+
+// ---- GEMM -----------------------------------------------------------------
+enum EpiKind : int {
+  EPI_QKV1 = 0,   // n < split_n: out0[m, n] = acc + bias[n] (act);
+                  // n >= split_n: out1[m, D + n - split_n] = gelu(acc + bias[n]) (act)
+  EPI_RESID = 1,  // out0 (fp32) [m, n] += acc + bias[n]
+  EPI_F32 = 2,    // out0 (fp32) [m, n] = acc (+ bias[n] if bias)
+  EPI_ACT = 3,    // out0 (act)  [m, n] = acc (+ bias[n] if bias)
+};
+
+struct Epi {
+  int kind;
+  void* out0;
+  int ld0;
+  void* out1;
+  int ld1;
+  const float* bias;
+  int split_n;
+  int D;
+};
+
+// out = X [M, K] (row stride ldx) . W [N, K]^T (row stride ldw), fp32
+// accumulation; for output columns n >= xk_split the X columns read are
+// shifted by xk_off. scratch: split-K partials (gemm_scratch_bytes).
+struct GemmScratch {
+  float* part;        // split-K partial tiles
+  size_t part_bytes;
+  int* counters;      // per output tile, zero between launches
+  int n_counters;
+};
+size_t gemm_scratch_bytes(int max_M, int max_N);
+int gemm_counter_count(int max_N);
+cudaError_t launch_gemm(int dt, const void* X, int ldx, const void* W, int ldw, int M, int N,
+                        int K, int xk_split, int xk_off, const Epi& e, const GemmScratch& scr,
+                        int* status, cudaStream_t s);
+// 0 = automatic, 1 = force the SIMT path, 2 = force the tensor-core path.
+void gemm_set_path(int path);
+int gemm_tc_supported(int dt, int M, int N, int K, int xk_split, int xk_off);
+
+// ---- LM head argmax ---------------------------------------------------------
+// next[b] = argmax_v logits[b, v] (lowest id among ties).
+cudaError_t launch_argmax(const float* logits, int B, int V, int ld, int32_t* next,
+                          cudaStream_t s);
+
+// ---- misc -----------------------------------------------------------------
+cudaError_t launch_convert_to_f32(int dt, const void* src, float* dst, size_t n, cudaStream_t s);
+cudaError_t launch_add_to_f32(int dt, const void* a, const void* b, float* dst, size_t n,
+                              cudaStream_t s);
+
+}  // namespace bt

@@ -1,0 +1,508 @@
+// runtime.cu -- the bt_* C-ABI: model creation, prefill and decode schedules.
+//
+// Schedules follow the inference stages of "Block Transformer: Global-to-Local
+// Language Modeling for Fast Inference" (§3.4 "Prefill vs. decode" and the
+// per-component cost analyses):
+//   prefill  embed all prompt blocks, run the block decoder over them (KV
+//            cache filled), then only the last block's context enters the
+//            token decoder (prefix rows) -> logits for the next token;
+//   decode   every call feeds one token; a token that completes its block
+//            triggers one block-decoder step (one new cache entry) and a new
+//            token-decoder block from the fresh context; other tokens append
+//            one row to the token decoder's local cache.
+// Each decode call is one CUDA-graph launch (graphs captured lazily per step
+// kind); the step position lives in device memory so graphs are reusable.
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <string>
+#include <vector>
+
+#include "../../include/bt.h"
+#include "common.cuh"
+#include "kernels.h"
+
+using namespace bt;
+
+static thread_local std::string g_last_cuda;
+
+#define BT_CUDA(call)                                      \
+  do {                                                     \
+    cudaError_t e__ = (call);                              \
+    if (e__ != cudaSuccess) {                              \
+      g_last_cuda = std::string(#call) + ": " + cudaGetErrorString(e__); \
+      return BT_ECUDA;                                     \
+    }                                                      \
+  } while (0)
+
+namespace {
+
+struct LayerW {
+  void* w_qkv1 = nullptr;  // [7D, D]   rows q | k | v | fc1
+  void* w_o2 = nullptr;    // [D, 5D]   cols W_o | W_2
+  float* b_qkv1 = nullptr; // [7D]
+  float* b_o2 = nullptr;   // [D]       b_o + b_2
+  float *ln1_g = nullptr, *ln1_b = nullptr, *ln2_g = nullptr, *ln2_b = nullptr;
+};
+
+// Bump allocator over the caller's workspace (dry run when base == nullptr).
+struct Carver {
+  uint8_t* base;
+  size_t off = 0;
+  explicit Carver(void* b) : base(static_cast<uint8_t*>(b)) {}
+  void* take(size_t bytes) {
+    off = (off + 255) & ~(size_t)255;
+    void* p = base ? base + off : nullptr;
+    off += bytes;
+    return p;
+  }
+};
+
+struct Dims {
+  int V, D, H, d, L, Nb, Nt, P, rot, Bmax, max_seq, dt, tokdec;
+  size_t eb;
+  int n_cap;   // block-cache entries per sequence
+  int l_cap;   // local-cache rows per sequence
+  int R;       // activation rows
+  int tab_pos; // rotary table positions
+};
+
+int dims_of(const bt_config* c, Dims* o) {
+  if (!c) return BT_EINVAL;
+  Dims d{};
+  d.V = c->vocab; d.D = c->d_model; d.H = c->n_heads; d.L = c->block_len;
+  d.Nb = c->n_block_layers; d.tokdec = c->use_token_decoder ? 1 : 0;
+  d.Nt = d.tokdec ? c->n_token_layers : 0;
+  d.P = d.tokdec ? c->prefix_len : 0;
+  d.rot = c->rotary_dims; d.Bmax = c->max_batch; d.max_seq = c->max_seq; d.dt = c->dtype;
+  if (d.V <= 0 || d.D <= 0 || d.H <= 0 || d.L <= 0 || d.Nb < 0 || d.Nt < 0 || d.Bmax <= 0 ||
+      d.max_seq <= 0)
+    return BT_EINVAL;
+  if (d.dt != BT_FP32 && d.dt != BT_BF16) return BT_EINVAL;
+  if (d.D % d.H || d.D % d.L || d.D % 8) return BT_EINVAL;
+  d.d = d.D / d.H;
+  if (d.d != 32 && d.d != 64 && d.d != 128) return BT_ENOTSUP;
+  if (d.rot < 0 || d.rot > d.d || (d.rot & 1)) return BT_EINVAL;
+  if ((d.D / d.L) * (int)dt_size(d.dt) % 4) return BT_ENOTSUP;
+  if (d.tokdec) {
+    if (d.P < 1) return BT_EINVAL;
+  } else if (d.L != 1) {
+    return BT_EINVAL;  // vanilla mode is the L_B = 1 special case
+  }
+  if (!(c->ln_eps > 0.f) || !(c->rope_base > 0.f)) return BT_EINVAL;
+  d.eb = dt_size(d.dt);
+  d.n_cap = (d.max_seq + d.L - 1) / d.L;
+  d.l_cap = d.tokdec ? d.P + d.L - 1 : 1;
+  const int rows_blk = d.Bmax * d.n_cap;
+  const int rows_tok = d.Bmax * (d.P > 1 ? d.P : 1);
+  d.R = rows_blk > rows_tok ? rows_blk : rows_tok;
+  d.tab_pos = d.n_cap > d.l_cap ? d.n_cap : d.l_cap;
+  *o = d;
+  return BT_OK;
+}
+
+}  // namespace
+
+struct bt_model {
+  bt_config cfg;
+  Dims d;
+  cudaStream_t stream = nullptr;      // caller's
+  cudaStream_t cap_stream = nullptr;  // private, for graph capture
+  std::vector<LayerW> blk, tok;
+  void *blk_emb = nullptr, *tok_emb = nullptr, *w_prefix = nullptr, *w_lm = nullptr;
+  float *b_prefix = nullptr, *lnf_b_g = nullptr, *lnf_b_b = nullptr, *lnf_t_g = nullptr,
+        *lnf_t_b = nullptr;
+  void *kb = nullptr, *vb = nullptr, *kt = nullptr, *vt = nullptr;
+  size_t kb_layer = 0, kt_layer = 0;  // elements per layer
+  float *h_b = nullptr, *h_t = nullptr, *logits = nullptr;
+  void *x1 = nullptr, *qkv = nullptr, *qrot = nullptr, *a2 = nullptr, *xf = nullptr;
+  int32_t *next = nullptr, *fed = nullptr, *block_tok = nullptr;
+  int *dstate = nullptr, *status = nullptr;
+  float2* rope_tab = nullptr;
+  void* attn_scratch = nullptr;
+  GemmScratch gs{};
+  int B = 0, t = 0;
+  bool prefilled = false;
+  bool use_graphs = true;
+  cudaGraphExec_t graphs[2][2] = {{nullptr, nullptr}, {nullptr, nullptr}};  // [block_step][greedy]
+  int graph_B = 0;
+};
+
+static size_t carve(bt_model* m, const Dims& d, void* ws) {
+  Carver c(ws);
+  const size_t eb = d.eb;
+  const size_t D = d.D;
+  auto layer = [&](LayerW& w) {
+    w.w_qkv1 = c.take(7 * D * D * eb);
+    w.w_o2 = c.take(5 * D * D * eb);
+    w.b_qkv1 = (float*)c.take(7 * D * 4);
+    w.b_o2 = (float*)c.take(D * 4);
+    w.ln1_g = (float*)c.take(D * 4); w.ln1_b = (float*)c.take(D * 4);
+    w.ln2_g = (float*)c.take(D * 4); w.ln2_b = (float*)c.take(D * 4);
+  };
+  m->blk.assign(d.Nb, LayerW());
+  m->tok.assign(d.Nt, LayerW());
+  for (auto& w : m->blk) layer(w);
+  for (auto& w : m->tok) layer(w);
+  m->blk_emb = c.take((size_t)d.V * (D / d.L) * eb);
+  m->lnf_b_g = (float*)c.take(D * 4); m->lnf_b_b = (float*)c.take(D * 4);
+  if (d.tokdec) {
+    m->tok_emb = c.take((size_t)d.V * D * eb);
+    m->w_prefix = c.take((size_t)d.P * D * D * eb);
+    m->b_prefix = (float*)c.take((size_t)d.P * D * 4);
+    m->lnf_t_g = (float*)c.take(D * 4); m->lnf_t_b = (float*)c.take(D * 4);
+  }
+  m->w_lm = c.take((size_t)d.V * D * eb);
+  // caches: [layer][B][H][cap][d]
+  m->kb_layer = (size_t)d.Bmax * D * d.n_cap;
+  m->kb = c.take(m->kb_layer * d.Nb * eb);
+  m->vb = c.take(m->kb_layer * d.Nb * eb);
+  m->kt_layer = (size_t)d.Bmax * D * d.l_cap;
+  m->kt = c.take(m->kt_layer * (d.Nt > 0 ? d.Nt : 0) * eb);
+  m->vt = c.take(m->kt_layer * (d.Nt > 0 ? d.Nt : 0) * eb);
+  // activations
+  const size_t R = d.R;
+  m->h_b = (float*)c.take(R * D * 4);
+  m->h_t = (float*)c.take((size_t)d.Bmax * (d.P > 1 ? d.P : 1) * D * 4);
+  m->x1 = c.take(R * 2 * D * eb);
+  m->qkv = c.take(R * 3 * D * eb);
+  m->qrot = c.take(R * D * eb);
+  m->a2 = c.take(R * 5 * D * eb);
+  m->xf = c.take((size_t)d.Bmax * D * eb);
+  m->logits = (float*)c.take((size_t)d.Bmax * d.V * 4);
+  m->next = (int32_t*)c.take((size_t)d.Bmax * 4);
+  m->fed = (int32_t*)c.take((size_t)d.Bmax * 4);
+  m->block_tok = (int32_t*)c.take((size_t)d.Bmax * d.L * 4);
+  m->dstate = (int*)c.take(64);
+  m->status = (int*)c.take(64);
+  m->rope_tab = (float2*)c.take((size_t)d.tab_pos * (d.rot / 2 > 0 ? d.rot / 2 : 1) * 8);
+  m->attn_scratch = c.take(attn_decode_scratch_bytes(d.Bmax, d.H, d.d, d.n_cap, d.dt));
+  const int maxN = 7 * d.D > d.V ? 7 * d.D : d.V;
+  m->gs.part_bytes = gemm_scratch_bytes(d.Bmax, maxN);
+  m->gs.part = (float*)c.take(m->gs.part_bytes);
+  m->gs.n_counters = gemm_counter_count(maxN);
+  m->gs.counters = (int*)c.take((size_t)m->gs.n_counters * 4);
+  return c.off + 256;
+}
+
+extern "C" {
+
+const char* bt_strerror(int s) {
+  switch (s) {
+    case BT_OK: return "ok";
+    case BT_EINVAL: return "invalid argument or configuration";
+    case BT_EWORKSPACE: return "workspace missing, misaligned or too small";
+    case BT_ECAPACITY: return "batch or sequence capacity exceeded";
+    case BT_ESTATE: return "decode before prefill";
+    case BT_ECUDA: return "CUDA runtime error";
+    case BT_EDEVICE: return "device-side failure reported through the status word";
+    case BT_ENOTSUP: return "unsupported shape";
+    default: return "unknown status";
+  }
+}
+
+const char* bt_last_cuda_error(void) { return g_last_cuda.c_str(); }
+
+size_t bt_workspace_bytes(const bt_config* cfg) {
+  Dims d;
+  if (dims_of(cfg, &d) != BT_OK) return 0;
+  bt_model tmp;
+  return carve(&tmp, d, nullptr);
+}
+
+static int copy_layer(bt_model* m, const LayerW& w, const bt_layer_weights& s) {
+  const Dims& d = m->d;
+  const size_t D = d.D, eb = d.eb;
+  cudaStream_t st = m->stream;
+  if (!s.w_qkv_dev || !s.w_o_dev || !s.w_1_dev || !s.w_2_dev || !s.b_qkv_dev || !s.b_o_dev ||
+      !s.b_1_dev || !s.b_2_dev || !s.ln1_g_dev || !s.ln1_b_dev || !s.ln2_g_dev || !s.ln2_b_dev)
+    return BT_EINVAL;
+  uint8_t* q1 = (uint8_t*)w.w_qkv1;
+  BT_CUDA(cudaMemcpyAsync(q1, s.w_qkv_dev, 3 * D * D * eb, cudaMemcpyDeviceToDevice, st));
+  BT_CUDA(cudaMemcpyAsync(q1 + 3 * D * D * eb, s.w_1_dev, 4 * D * D * eb,
+                          cudaMemcpyDeviceToDevice, st));
+  uint8_t* o2 = (uint8_t*)w.w_o2;
+  BT_CUDA(cudaMemcpy2DAsync(o2, 5 * D * eb, s.w_o_dev, D * eb, D * eb, D,
+                            cudaMemcpyDeviceToDevice, st));
+  BT_CUDA(cudaMemcpy2DAsync(o2 + D * eb, 5 * D * eb, s.w_2_dev, 4 * D * eb, 4 * D * eb, D,
+                            cudaMemcpyDeviceToDevice, st));
+  BT_CUDA(launch_convert_to_f32(d.dt, s.b_qkv_dev, w.b_qkv1, 3 * D, st));
+  BT_CUDA(launch_convert_to_f32(d.dt, s.b_1_dev, w.b_qkv1 + 3 * D, 4 * D, st));
+  BT_CUDA(launch_add_to_f32(d.dt, s.b_o_dev, s.b_2_dev, w.b_o2, D, st));
+  BT_CUDA(launch_convert_to_f32(d.dt, s.ln1_g_dev, w.ln1_g, D, st));
+  BT_CUDA(launch_convert_to_f32(d.dt, s.ln1_b_dev, w.ln1_b, D, st));
+  BT_CUDA(launch_convert_to_f32(d.dt, s.ln2_g_dev, w.ln2_g, D, st));
+  BT_CUDA(launch_convert_to_f32(d.dt, s.ln2_b_dev, w.ln2_b, D, st));
+  return BT_OK;
+}
+
+int bt_create(const bt_config* cfg, const bt_weights* w, void* ws, size_t ws_bytes, void* stream,
+              bt_model** out) {
+  if (!out || !w) return BT_EINVAL;
+  *out = nullptr;
+  Dims d;
+  int rc = dims_of(cfg, &d);
+  if (rc != BT_OK) return rc;
+  if (!ws || ((uintptr_t)ws & 255)) return BT_EWORKSPACE;
+  bt_model* m = new bt_model();
+  m->cfg = *cfg;
+  m->d = d;
+  m->stream = (cudaStream_t)stream;
+  const size_t need = carve(m, d, ws);
+  if (ws_bytes < need) { delete m; return BT_EWORKSPACE; }
+  const char* ng = getenv("BT_NO_GRAPH");
+  m->use_graphs = !(ng && ng[0] == '1');
+  if (!w->blk_emb_dev || !w->lnf_b_g_dev || !w->lnf_b_b_dev || !w->w_lm_dev ||
+      (d.Nb > 0 && !w->block_layers) || (d.Nt > 0 && !w->token_layers) ||
+      (d.tokdec && (!w->w_prefix_dev || !w->b_prefix_dev || !w->tok_emb_dev ||
+                    !w->lnf_t_g_dev || !w->lnf_t_b_dev))) {
+    delete m;
+    return BT_EINVAL;
+  }
+  cudaStream_t st = m->stream;
+  auto fail = [&](int code) { delete m; return code; };
+#define BT_TRY(x) do { int r__ = (x); if (r__ != BT_OK) return fail(r__); } while (0)
+#define BT_TRYC(x) do { cudaError_t e__ = (x); if (e__ != cudaSuccess) { g_last_cuda = std::string(#x) + ": " + cudaGetErrorString(e__); return fail(BT_ECUDA); } } while (0)
+  for (int l = 0; l < d.Nb; ++l) BT_TRY(copy_layer(m, m->blk[l], w->block_layers[l]));
+  for (int l = 0; l < d.Nt; ++l) BT_TRY(copy_layer(m, m->tok[l], w->token_layers[l]));
+  const size_t D = d.D, eb = d.eb;
+  BT_TRYC(cudaMemcpyAsync(m->blk_emb, w->blk_emb_dev, (size_t)d.V * (D / d.L) * eb,
+                          cudaMemcpyDeviceToDevice, st));
+  BT_TRYC(launch_convert_to_f32(d.dt, w->lnf_b_g_dev, m->lnf_b_g, D, st));
+  BT_TRYC(launch_convert_to_f32(d.dt, w->lnf_b_b_dev, m->lnf_b_b, D, st));
+  if (d.tokdec) {
+    BT_TRYC(cudaMemcpyAsync(m->tok_emb, w->tok_emb_dev, (size_t)d.V * D * eb,
+                            cudaMemcpyDeviceToDevice, st));
+    BT_TRYC(cudaMemcpyAsync(m->w_prefix, w->w_prefix_dev, (size_t)d.P * D * D * eb,
+                            cudaMemcpyDeviceToDevice, st));
+    BT_TRYC(launch_convert_to_f32(d.dt, w->b_prefix_dev, m->b_prefix, (size_t)d.P * D, st));
+    BT_TRYC(launch_convert_to_f32(d.dt, w->lnf_t_g_dev, m->lnf_t_g, D, st));
+    BT_TRYC(launch_convert_to_f32(d.dt, w->lnf_t_b_dev, m->lnf_t_b, D, st));
+  }
+  BT_TRYC(cudaMemcpyAsync(m->w_lm, w->w_lm_dev, (size_t)d.V * D * eb, cudaMemcpyDeviceToDevice, st));
+  BT_TRYC(launch_rope_table(m->rope_tab, d.tab_pos, d.rot, cfg->rope_base, st));
+  BT_TRYC(cudaMemsetAsync(m->status, 0, 64, st));
+  BT_TRYC(cudaMemsetAsync(m->dstate, 0, 64, st));
+  BT_TRYC(cudaMemsetAsync(m->attn_scratch, 0, attn_decode_scratch_bytes(d.Bmax, d.H, d.d, d.n_cap, d.dt), st));
+  BT_TRYC(cudaMemsetAsync(m->gs.counters, 0, (size_t)m->gs.n_counters * 4, st));
+  BT_TRYC(cudaMemsetAsync(m->block_tok, 0, (size_t)d.Bmax * d.L * 4, st));
+  BT_TRYC(cudaStreamCreateWithFlags(&m->cap_stream, cudaStreamNonBlocking));
+#undef BT_TRY
+#undef BT_TRYC
+  *out = m;
+  return BT_OK;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// schedule pieces
+// ---------------------------------------------------------------------------
+enum AttnKind { ATT_PREFILL, ATT_DECODE, ATT_LOCAL };
+
+static int run_layer(bt_model* m, const LayerW& w, float* h, int M, PosSpec pos, void* kc,
+                     void* vc, int cap, AttnKind ak, int n_prefill, cudaStream_t s) {
+  const Dims& d = m->d;
+  const int D = d.D;
+  BT_CUDA(launch_ln_dual(d.dt, h, M, D, w.ln1_g, w.ln1_b, w.ln2_g, w.ln2_b, m->cfg.ln_eps, m->x1, s));
+  Epi e1{EPI_QKV1, m->qkv, 3 * D, m->a2, 5 * D, w.b_qkv1, 3 * D, D};
+  BT_CUDA(launch_gemm(d.dt, m->x1, 2 * D, w.w_qkv1, D, M, 7 * D, D, 3 * D, D, e1, m->gs, m->status, s));
+  BT_CUDA(launch_rope_append(d.dt, m->qkv, M, D, d.H, d.rot, m->rope_tab, pos, m->qrot, kc, vc, cap, s));
+  const int Bseq = M / pos.rows_per_seq;
+  if (ak == ATT_PREFILL) {
+    BT_CUDA(launch_attn_prefill(d.dt, m->qrot, D, kc, vc, Bseq, d.H, d.d, cap, n_prefill, m->a2, 5 * D, s));
+  } else if (ak == ATT_DECODE) {
+    BT_CUDA(launch_attn_decode(d.dt, m->qrot, D, kc, vc, Bseq, d.H, d.d, cap, pos, m->a2, 5 * D,
+                               m->attn_scratch, m->status, s));
+  } else {
+    BT_CUDA(launch_attn_small(d.dt, m->qrot, D, kc, vc, Bseq, d.H, d.d, cap, pos, m->a2, 5 * D, s));
+  }
+  Epi e2{EPI_RESID, h, D, nullptr, 0, w.b_o2, 0, D};
+  BT_CUDA(launch_gemm(d.dt, m->a2, 5 * D, w.w_o2, 5 * D, M, D, 5 * D, 1 << 30, 0, e2, m->gs, m->status, s));
+  return BT_OK;
+}
+
+static void* layer_ptr(void* base, size_t layer_elems, int l, size_t eb) {
+  return (uint8_t*)base + (size_t)l * layer_elems * eb;
+}
+
+// token decoder over rows_per_seq rows per sequence, then LN_t of the last
+// of them into xf
+static int run_token_decoder(bt_model* m, int B, PosSpec pos, cudaStream_t s) {
+  const Dims& d = m->d;
+  const int M = B * pos.rows_per_seq;
+  for (int l = 0; l < d.Nt; ++l) {
+    int rc = run_layer(m, m->tok[l], m->h_t, M, pos, layer_ptr(m->kt, m->kt_layer, l, d.eb),
+                       layer_ptr(m->vt, m->kt_layer, l, d.eb), d.l_cap, ATT_LOCAL, 0, s);
+    if (rc != BT_OK) return rc;
+  }
+  BT_CUDA(launch_ln_rows(d.dt, m->h_t, B, pos.rows_per_seq, pos.rows_per_seq - 1, d.D, m->lnf_t_g,
+                         m->lnf_t_b, m->cfg.ln_eps, m->xf, s));
+  return BT_OK;
+}
+
+// context rows (B rows of h_b, row r*row_step + row_off) -> LN_b -> either the
+// prefix projection and the token decoder over P rows, or (vanilla) xf.
+static int run_context_to_head_input(bt_model* m, int B, int row_step, int row_off, cudaStream_t s) {
+  const Dims& d = m->d;
+  BT_CUDA(launch_ln_rows(d.dt, m->h_b, B, row_step, row_off, d.D, m->lnf_b_g, m->lnf_b_b,
+                         m->cfg.ln_eps, m->xf, s));
+  if (!d.tokdec) return BT_OK;
+  // prefix rows: h_t[b*P + p, :] = (W_p c_b + b_p)[p*D:(p+1)*D]
+  Epi ep{EPI_F32, m->h_t, d.P * d.D, nullptr, 0, m->b_prefix, 0, d.D};
+  BT_CUDA(launch_gemm(d.dt, m->xf, d.D, m->w_prefix, d.D, B, d.P * d.D, d.D, 1 << 30, 0, ep, m->gs,
+                      m->status, s));
+  PosSpec pos{nullptr, POS_ZERO, 0, d.P};
+  return run_token_decoder(m, B, pos, s);
+}
+
+static int run_head(bt_model* m, int B, cudaStream_t s) {
+  const Dims& d = m->d;
+  Epi el{EPI_F32, m->logits, d.V, nullptr, 0, nullptr, 0, d.D};
+  BT_CUDA(launch_gemm(d.dt, m->xf, d.D, m->w_lm, d.D, B, d.V, d.D, 1 << 30, 0, el, m->gs, m->status, s));
+  BT_CUDA(launch_argmax(m->logits, B, d.V, d.V, m->next, s));
+  return BT_OK;
+}
+
+static int copy_outputs(bt_model* m, float* logits, int32_t* next) {
+  const Dims& d = m->d;
+  if (logits)
+    BT_CUDA(cudaMemcpyAsync(logits, m->logits, (size_t)m->B * d.V * 4, cudaMemcpyDeviceToDevice, m->stream));
+  if (next)
+    BT_CUDA(cudaMemcpyAsync(next, m->next, (size_t)m->B * 4, cudaMemcpyDeviceToDevice, m->stream));
+  return BT_OK;
+}
+
+// the body of one decode call (captured into a graph or run directly)
+static int enqueue_decode(bt_model* m, bool block_step, bool greedy, cudaStream_t s) {
+  const Dims& d = m->d;
+  const int B = m->B;
+  const int32_t* src = greedy ? m->next : m->fed;
+  BT_CUDA(launch_ingest(d.dt, src, m->block_tok, m->dstate, B, d.L, d.V, d.D, block_step ? 1 : 0,
+                        m->blk_emb, m->tok_emb, block_step ? m->h_b : m->h_t, m->status, s));
+  int rc;
+  if (block_step) {
+    PosSpec pos{m->dstate, POS_BLOCK, 0, 1};
+    for (int l = 0; l < d.Nb; ++l) {
+      rc = run_layer(m, m->blk[l], m->h_b, B, pos, layer_ptr(m->kb, m->kb_layer, l, d.eb),
+                     layer_ptr(m->vb, m->kb_layer, l, d.eb), d.n_cap, ATT_DECODE, 0, s);
+      if (rc != BT_OK) return rc;
+    }
+    rc = run_context_to_head_input(m, B, 1, 0, s);
+    if (rc != BT_OK) return rc;
+  } else {
+    PosSpec pos{m->dstate, POS_LOCAL, d.P, 1};
+    rc = run_token_decoder(m, B, pos, s);
+    if (rc != BT_OK) return rc;
+  }
+  rc = run_head(m, B, s);
+  if (rc != BT_OK) return rc;
+  BT_CUDA(launch_advance(m->dstate, d.L, s));
+  return BT_OK;
+}
+
+static void drop_graphs(bt_model* m) {
+  for (auto& a : m->graphs)
+    for (auto& g : a)
+      if (g) { cudaGraphExecDestroy(g); g = nullptr; }
+}
+
+extern "C" {
+
+int bt_prefill(bt_model* m, const int32_t* tokens, int32_t B, int32_t T, float* logits,
+               int32_t* next) {
+  if (!m || !tokens) return BT_EINVAL;
+  const Dims& d = m->d;
+  if (B < 1 || B > d.Bmax) return BT_ECAPACITY;
+  if (T < d.L || T % d.L) return BT_EINVAL;
+  if (T >= d.max_seq) return BT_ECAPACITY;
+  cudaStream_t s = m->stream;
+  m->B = B;
+  m->t = T;
+  const int n = T / d.L;
+  const int M = B * n;
+  BT_CUDA(launch_set_state(m->dstate, T, d.L, s));
+  BT_CUDA(launch_embed_prompt(d.dt, tokens, B, T, d.L, m->blk_emb, d.V, d.D, m->h_b, m->status, s));
+  PosSpec pos{nullptr, POS_ZERO, 0, n};
+  for (int l = 0; l < d.Nb; ++l) {
+    int rc = run_layer(m, m->blk[l], m->h_b, M, pos, layer_ptr(m->kb, m->kb_layer, l, d.eb),
+                       layer_ptr(m->vb, m->kb_layer, l, d.eb), d.n_cap, ATT_PREFILL, n, s);
+    if (rc != BT_OK) return rc;
+  }
+  int rc = run_context_to_head_input(m, B, n, n - 1, s);
+  if (rc != BT_OK) return rc;
+  rc = run_head(m, B, s);
+  if (rc != BT_OK) return rc;
+  m->prefilled = true;
+  if (m->graph_B != B) { drop_graphs(m); m->graph_B = B; }
+  return copy_outputs(m, logits, next);
+}
+
+int bt_decode_step(bt_model* m, const int32_t* tokens, float* logits, int32_t* next) {
+  if (!m) return BT_EINVAL;
+  if (!m->prefilled) return BT_ESTATE;
+  const Dims& d = m->d;
+  if (m->t + 1 > d.max_seq) return BT_ECAPACITY;
+  const bool block_step = (m->t % d.L) == d.L - 1;
+  const bool greedy = tokens == nullptr;
+  if (!greedy)
+    BT_CUDA(cudaMemcpyAsync(m->fed, tokens, (size_t)m->B * 4, cudaMemcpyDeviceToDevice, m->stream));
+  if (m->use_graphs) {
+    cudaGraphExec_t& g = m->graphs[block_step ? 1 : 0][greedy ? 1 : 0];
+    if (!g) {
+      // capture on the private stream, ordered after the caller's stream
+      cudaEvent_t ev;
+      BT_CUDA(cudaEventCreateWithFlags(&ev, cudaEventDisableTiming));
+      BT_CUDA(cudaEventRecord(ev, m->stream));
+      BT_CUDA(cudaStreamWaitEvent(m->cap_stream, ev, 0));
+      BT_CUDA(cudaStreamSynchronize(m->cap_stream));
+      cudaEventDestroy(ev);
+      cudaGraph_t graph;
+      BT_CUDA(cudaStreamBeginCapture(m->cap_stream, cudaStreamCaptureModeThreadLocal));
+      int rc = enqueue_decode(m, block_step, greedy, m->cap_stream);
+      cudaError_t ce = cudaStreamEndCapture(m->cap_stream, &graph);
+      if (rc != BT_OK) return rc;
+      BT_CUDA(ce);
+      BT_CUDA(cudaGraphInstantiate(&g, graph, 0));
+      cudaGraphDestroy(graph);
+    }
+    BT_CUDA(cudaGraphLaunch(g, m->stream));
+  } else {
+    int rc = enqueue_decode(m, block_step, greedy, m->stream);
+    if (rc != BT_OK) return rc;
+  }
+  m->t += 1;
+  return copy_outputs(m, logits, next);
+}
+
+int bt_sync(bt_model* m) {
+  if (!m) return BT_EINVAL;
+  BT_CUDA(cudaStreamSynchronize(m->stream));
+  int st = 0;
+  BT_CUDA(cudaMemcpy(&st, m->status, sizeof(int), cudaMemcpyDeviceToHost));
+  if (st) {
+    BT_CUDA(cudaMemsetAsync(m->status, 0, sizeof(int), m->stream));
+    BT_CUDA(cudaStreamSynchronize(m->stream));
+    return BT_EDEVICE;
+  }
+  return BT_OK;
+}
+
+int bt_position(const bt_model* m) {
+  if (!m) return BT_EINVAL;
+  if (!m->prefilled) return BT_ESTATE;
+  return m->t;
+}
+
+int bt_destroy(bt_model* m) {
+  if (!m) return BT_EINVAL;
+  cudaStreamSynchronize(m->stream);
+  drop_graphs(m);
+  if (m->cap_stream) cudaStreamDestroy(m->cap_stream);
+  delete m;
+  return BT_OK;
+}
+
+}  // extern "C"

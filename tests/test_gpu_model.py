@@ -1,0 +1,129 @@
+"""Whole-model parity: CUDA path through the C-ABI vs the CPU oracle.
+
+Tolerances: fp32 workloads, max |logit difference| <= 1e-4 at every
+teacher-forced step; bf16 workloads, per-step relative L2 error of the
+[B, V] logits <= 2e-2.
+"""
+import numpy as np
+import pytest
+
+import synth
+from tests import gpu_helpers as gh
+
+pytestmark = pytest.mark.gpu
+
+FP32_TOL = 1e-4
+BF16_REL = 2e-2
+
+
+def _run(shape, B, T, G, seed=3, rows=None, kind="uniform"):
+    w = synth.make_weights(shape, seed=1000 + seed)
+    toks = synth.make_tokens(batch=B, length=T + G, vocab=shape.vocab, kind=kind, seed=2000 + seed)
+    model = gh.build_model(shape, w, max_batch=B, max_seq=T + G)
+    gl, gn = gh.gpu_teacher_forced(model, toks, T, G)
+    model.close()
+    ol = gh.oracle_teacher_forced(shape, w, toks, T, G, rows=rows)
+    if rows is not None:
+        gl, gn = gl[:, rows], gn[:, rows]
+    return gl, gn, ol
+
+
+def test_tiny_fp32_workload_teacher_forced():
+    wl = synth.WORKLOADS["tiny_fp32"]
+    w = synth.make_weights(wl)
+    toks = synth.make_tokens(wl)
+    model = gh.build_model(wl.shape, w, wl.batch, wl.max_seq)
+    gl, gn = gh.gpu_teacher_forced(model, toks, wl.prompt_len, wl.gen_len)
+    model.close()
+    ol = gh.oracle_teacher_forced(wl.shape, w, toks, wl.prompt_len, wl.gen_len)
+    err = np.abs(gl - ol).max(axis=(1, 2))
+    assert err.max() <= FP32_TOL, err
+    # greedy ids are the argmax of the returned logits (lowest id on ties)
+    assert np.array_equal(gn, gl.argmax(axis=-1))
+
+
+@pytest.mark.parametrize("lb,P", [(4, 1), (2, 2), (8, 1)])
+def test_small_bf16_block_transformer(lb, P):
+    shape = synth.ModelShape(vocab=1000, d_model=256, n_heads=4, block_len=lb,
+                             n_block_layers=2, n_token_layers=2, prefix_len=P)
+    T = 12 * lb
+    gl, gn, ol = _run(shape, B=3, T=T, G=3 * lb + 2)
+    for s in range(gl.shape[0]):
+        assert gh.rel_l2(gl[s], ol[s]) <= BF16_REL, (s, gh.rel_l2(gl[s], ol[s]))
+
+
+def test_small_bf16_vanilla_lb1():
+    shape = synth.ModelShape(vocab=700, d_model=256, n_heads=2, block_len=1,
+                             n_block_layers=3, n_token_layers=0, prefix_len=0,
+                             use_token_decoder=False)
+    gl, gn, ol = _run(shape, B=2, T=40, G=6)
+    for s in range(gl.shape[0]):
+        assert gh.rel_l2(gl[s], ol[s]) <= BF16_REL
+
+
+def test_head_dim_128_bf16():
+    shape = synth.ModelShape(vocab=500, d_model=512, n_heads=4, block_len=4,
+                             n_block_layers=2, n_token_layers=1, prefix_len=1)
+    gl, gn, ol = _run(shape, B=2, T=64, G=9)
+    for s in range(gl.shape[0]):
+        assert gh.rel_l2(gl[s], ol[s]) <= BF16_REL
+
+
+def test_fp32_small_exact_tolerance_multi_prefix():
+    shape = synth.ModelShape(vocab=300, d_model=128, n_heads=2, block_len=4,
+                             n_block_layers=2, n_token_layers=2, prefix_len=3, dtype="fp32")
+    gl, gn, ol = _run(shape, B=3, T=20, G=11)
+    assert np.abs(gl - ol).max() <= FP32_TOL
+
+
+def test_greedy_generation_feeds_own_argmax():
+    shape = synth.ModelShape(vocab=300, d_model=128, n_heads=2, block_len=4,
+                             n_block_layers=1, n_token_layers=1, prefix_len=1, dtype="fp32")
+    torch = gh.torch_mod()
+    w = synth.make_weights(shape, seed=77)
+    B, T, G = 2, 16, 9
+    toks = synth.make_tokens(batch=B, length=T, vocab=shape.vocab, seed=5)
+    model = gh.build_model(shape, w, B, T + G)
+    t = torch.from_numpy(toks).cuda()
+    _, nxt = model.prefill(t)
+    seq = [nxt.clone()]
+    for _ in range(G - 1):
+        _, nxt = model.decode(None)
+        seq.append(nxt.clone())
+    model.sync()
+    gen = torch.stack(seq, 1).cpu().numpy()              # [B, G]
+    model.close()
+    full = np.concatenate([toks, gen], axis=1)
+    ol = gh.oracle_teacher_forced(shape, w, full, T, G)  # oracle fed the same ids
+    assert np.array_equal(ol.argmax(-1).T, gen)
+
+
+def test_rows_are_independent_bitwise():
+    shape = synth.ModelShape(vocab=512, d_model=256, n_heads=4, block_len=4,
+                             n_block_layers=2, n_token_layers=2, prefix_len=1)
+    w = synth.make_weights(shape, seed=11)
+    B, T, G = 4, 32, 6
+    toks = synth.make_tokens(batch=B, length=T + G, vocab=shape.vocab, seed=12)
+    m = gh.build_model(shape, w, B, T + G)
+    a, _ = gh.gpu_teacher_forced(m, toks, T, G)
+    toks2 = toks.copy()
+    toks2[2] = (toks2[2] + 17) % shape.vocab
+    b, _ = gh.gpu_teacher_forced(m, toks2, T, G)
+    m.close()
+    assert np.array_equal(a[:, [0, 1, 3]], b[:, [0, 1, 3]])
+    assert not np.array_equal(a[:, 2], b[:, 2])
+
+
+def test_pythia160m_shape_sampled_rows():
+    """Full-width Pythia-160M-scale model (V 50304, D 768, 6+6 layers) at a
+    small batch and prompt; every step compared on all rows."""
+    wl = synth.WORKLOADS["pythia160m_decode_heavy"]
+    B, T, G = 3, 64, 10
+    w = synth.make_weights(wl)
+    toks = synth.make_tokens(wl, batch=B, length=T + G)
+    m = gh.build_model(wl.shape, w, B, T + G)
+    gl, _ = gh.gpu_teacher_forced(m, toks, T, G)
+    m.close()
+    ol = gh.oracle_teacher_forced(wl.shape, w, toks, T, G, dtype=np.float32)
+    for s in range(G):
+        assert gh.rel_l2(gl[s], ol[s]) <= BF16_REL, (s, gh.rel_l2(gl[s], ol[s]))
