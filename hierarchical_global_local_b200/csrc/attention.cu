@@ -109,17 +109,23 @@ attn_decode_kernel(const T* __restrict__ q, int ldq, const T* __restrict__ kc,
     return;
   }
 
-  // scores s_r = q . k_r (log2 domain)
-  for (int r = g; r < rows; r += C::RPP) {
-    const uint4 u = *reinterpret_cast<const uint4*>(sK + r * DH + e0);
-    float kf[C::EPT];
-    unpack16(u, kf, (const T*)nullptr);
+  // scores s_r = q . k_r (log2 domain). The trip count is the same for every
+  // thread of the CTA (rows and RPP are uniform) so the full-warp shuffles
+  // below never see a partial warp; rows past the end contribute nothing.
+  for (int rb = 0; rb < rows; rb += C::RPP) {
+    const int r = rb + g;
+    const bool valid = r < rows;
     float s = 0.f;
+    if (valid) {
+      const uint4 u = *reinterpret_cast<const uint4*>(sK + r * DH + e0);
+      float kf[C::EPT];
+      unpack16(u, kf, (const T*)nullptr);
 #pragma unroll
-    for (int i = 0; i < C::EPT; ++i) s = fmaf(qf[i], kf[i], s);
+      for (int i = 0; i < C::EPT; ++i) s = fmaf(qf[i], kf[i], s);
+    }
 #pragma unroll
     for (int o = C::TPR / 2; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    if ((tid % C::TPR) == 0) sS[r] = s;
+    if (valid && (tid % C::TPR) == 0) sS[r] = s;
   }
   __syncthreads();
   float mx = -FLT_MAX;
