@@ -1,0 +1,427 @@
+"""Benchmark: generated tokens/s of Block Transformer inference on B200.
+
+One step = the two runs of the Pythia-160M-scale Block Transformer workload
+(d_model 768, 12 heads, V 50304, L_B 4, 6 + 6 layers, prefix 1, bf16,
+random-init weights, Zipf(1.1) token ids), on one model instance:
+  prefill-heavy  batch 64, prompt 2048, 128 generated tokens;
+  decode-heavy   batch 64, prompt 128, 2048 generated tokens.
+Each run is a prefill plus greedy decode steps through the C-ABI (G tokens
+generated per sequence = 1 prefill + G - 1 decode calls). value = generated
+tokens of both runs / their device time, summed over ranks (replicas).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0). --impl reference times the CPU oracle on a
+bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synth  # noqa: E402
+
+RUNS = ("pythia160m_prefill_heavy", "pythia160m_decode_heavy")
+METRIC = "generated tokens/s at 1 B200 (prefill- & decode-heavy); % HBM roofline"
+UNIT = "tokens/s"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d["bf16_tflops_sustained"]), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# --------------------------------------------------------------------------
+# clocks during the timed region
+# --------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append(ln.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------
+# our arm
+# --------------------------------------------------------------------------
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def build(rank: int):
+    import torch
+    from tests.gpu_helpers import build_model
+    wl = synth.WORKLOADS[RUNS[0]]
+    w = synth.make_weights(wl)
+    max_seq = max(synth.WORKLOADS[r].max_seq for r in RUNS)
+    B = max(synth.WORKLOADS[r].batch for r in RUNS)
+    model = build_model(wl.shape, w, B, max_seq)
+    prompts = {}
+    for r in RUNS:
+        x = synth.WORKLOADS[r]
+        toks = synth.make_tokens(x, seed=x.token_seed + 100 * rank)
+        prompts[r] = torch.from_numpy(np.ascontiguousarray(toks[:, :x.prompt_len])).cuda()
+    return model, prompts
+
+
+def generate(model, prompt, G, out):
+    """Prefill + G - 1 greedy decode calls; generated ids land in out [G, B]."""
+    model.prefill(prompt, next_tokens=out[0])
+    for i in range(1, G):
+        model.decode(None, next_tokens=out[i])
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    from hierarchical_global_local_b200 import costmodel as cm
+    from hierarchical_global_local_b200 import native
+
+    ws, rank, local = _dist()
+    torch.cuda.set_device(local)
+    if ws > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=600))
+    model, prompts = build(rank)
+    gens = {r: torch.empty(synth.WORKLOADS[r].gen_len, synth.WORKLOADS[r].batch,
+                           dtype=torch.int32, device="cuda") for r in RUNS}
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if ws > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def one_step(times):
+        for r in RUNS:
+            x = synth.WORKLOADS[r]
+            flush.fill_(rank & 0xFF)          # L2 flush between timed runs (untimed)
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            generate(model, prompts[r], x.gen_len, gens[r])
+            b.record(stream)
+            times.append((r, a, b))
+
+    for _ in range(args.warmup):
+        one_step([])
+    model.sync()
+    k0 = native.lib().bt_kernel_launches(model._h)
+    times = []
+    barrier()
+    with ClockSampler(local) as clk:
+        for _ in range(args.steps):
+            one_step(times)
+        barrier()
+    k1 = native.lib().bt_kernel_launches(model._h)
+    model.sync()
+    per_run = {r: 0.0 for r in RUNS}
+    for r, a, b in times:
+        per_run[r] += a.elapsed_time(b)
+    total_ms = sum(per_run.values())
+    tmax = torch.tensor([total_ms] + [per_run[r] for r in RUNS], dtype=torch.float64, device="cuda")
+    if ws > 1:
+        dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
+    total_ms = float(tmax[0])
+    per_run_max = {r: float(tmax[1 + i]) for i, r in enumerate(RUNS)}
+    tokens_per_step = sum(synth.WORKLOADS[r].batch * synth.WORKLOADS[r].gen_len for r in RUNS)
+    value = ws * tokens_per_step * args.steps / (total_ms / 1e3)
+
+    # ---- end to end through the public API, host buffers -------------------
+    e2e = None
+    if not args.no_e2e:
+        host_prompts = {r: prompts[r].cpu().pin_memory() for r in RUNS}
+        host_out = {r: torch.empty_like(gens[r], device="cpu").pin_memory() for r in RUNS}
+        dev_prompts = {r: torch.empty_like(prompts[r]) for r in RUNS}
+        e_times = []
+        barrier()
+        for _ in range(args.steps):
+            for r in RUNS:
+                x = synth.WORKLOADS[r]
+                flush.fill_(1)
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                dev_prompts[r].copy_(host_prompts[r], non_blocking=True)
+                generate(model, dev_prompts[r], x.gen_len, gens[r])
+                host_out[r].copy_(gens[r], non_blocking=True)
+                b.record(stream)
+                e_times.append((a, b))
+        barrier()
+        e_ms = sum(a.elapsed_time(b) for a, b in e_times)
+        et = torch.tensor([e_ms], dtype=torch.float64, device="cuda")
+        if ws > 1:
+            dist.all_reduce(et, op=dist.ReduceOp.MAX)
+        h2d = sum(int(prompts[r].numel()) * 4 for r in RUNS)
+        d2h = sum(int(gens[r].numel()) * 4 for r in RUNS)
+        e2e = {"value": ws * tokens_per_step * args.steps / (float(et[0]) / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    # ---- profiled pass: event pair around every kernel of one step ---------
+    hbm, tf_burst, tf_sus, peak_src = _peaks()
+    prof = profile_step(model, prompts, gens, flush) if not args.no_profile else None
+
+    # ---- bytes / FLOPs roofline of the whole generate runs ------------------
+    s = cm.Shape.of(synth.WORKLOADS[RUNS[0]].shape)
+    roof = {}
+    for r in RUNS:
+        x = synth.WORKLOADS[r]
+        g = cm.generate(s, x.batch, x.prompt_len, x.gen_len)
+        t_roof = g.roofline_seconds(hbm, tf_sus)
+        t_meas = per_run_max[r] / args.steps / 1e3
+        roof[r] = {"ms": per_run_max[r] / args.steps, "tokens_per_s": ws * x.batch * x.gen_len / t_meas,
+                   "roofline_ms": t_roof * 1e3, "frac_of_roofline": t_roof / t_meas,
+                   "decode_bytes_per_step_GB": g.decode.bytes / 1e9,
+                   "prefill_tflop": g.prefill.flops / 1e12}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "pythia160m-scale Block Transformer L_B=4 6+6 layers P=1: "
+                               "prefill-heavy B64 2048/128 + decode-heavy B64 128/2048",
+                   "global_batch": 64 * ws, "seq_len": 2176, "parallelism": f"replicas{ws}",
+                   "l2": "flushed (256 MiB write) before each timed run; weights + KV > L2",
+                   "tokens": "Zipf(1.1) ids, greedy generation"},
+        "runs": roof,
+        "gpu_launches": int(k1 - k0),
+        "clocks": clk.summary(),
+        "e2e": e2e,
+    }
+    if prof:
+        line["roofline"] = prof["dominant"]
+        line["roofline_decode_attention"] = prof.get("attn_decode")
+        line["kernel_time_shares"] = prof["shares"]
+        line["roofline"]["peak_source"] = peak_src
+    if rank == 0 and ws == 1 and not args.no_cpu:
+        line["cpu_baseline"] = cpu_baseline(budget_s=args.cpu_seconds)
+    if ws > 1:
+        dist.barrier()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    model.close()
+    if ws > 1:
+        dist.destroy_process_group()
+
+
+def profile_step(model, prompts, gens, flush):
+    """One step with an event pair around every kernel; per-kind time shares
+    and the roofline of the dominant kernel class."""
+    import torch
+    from hierarchical_global_local_b200 import native
+    L = native.lib()
+    cap = 400000
+    _check = native._check
+    _check(L.bt_profile_begin(model._h, cap), "bt_profile_begin")
+    for r in RUNS:
+        flush.fill_(2)
+        generate(model, prompts[r], synth.WORKLOADS[r].gen_len, gens[r])
+    recs = (native_record() * cap)()
+    n = native.ctypes.c_int32()
+    _check(L.bt_profile_end(model._h, native.ctypes.cast(recs, native.ctypes.c_void_p), cap,
+                           native.ctypes.byref(n)), "bt_profile_end")
+    hbm, tf_burst, tf_sus, _ = _peaks()
+    kinds = {0: "gemm", 1: "attn_decode", 2: "attn_prefill", 3: "attn_local", 4: "layernorm",
+             5: "rope_append", 6: "embed", 7: "argmax", 8: "other"}
+    D = synth.WORKLOADS[RUNS[0]].shape.d_model
+    cls = {}
+    for i in range(n.value):
+        rc = recs[i]
+        k = kinds.get(rc.kind, "other")
+        if k == "gemm":
+            k = "gemm_decode" if rc.m <= 256 else "gemm_prefill"
+        c = cls.setdefault(k, {"ms": 0.0, "launches": 0, "bytes": 0.0, "flops": 0.0})
+        c["ms"] += rc.ms
+        c["launches"] += 1
+        if k.startswith("gemm"):
+            # output: bf16 q|k|v|GELU(fc1); fp32 residual read + write; fp32 logits / prefix rows
+            out_b = 2 if rc.n == 7 * D else (8 if rc.k == 5 * D else 4)
+            c["bytes"] += 2.0 * (rc.n * rc.k + rc.m * rc.k) + out_b * rc.m * rc.n
+            c["flops"] += 2.0 * rc.m * rc.n * rc.k
+        elif k == "attn_decode":
+            c["bytes"] += rc.m * (2.0 * rc.n * rc.k * 2 + 2.0 * rc.k * 2)
+    total = sum(c["ms"] for c in cls.values())
+    shares = {k: round(c["ms"] / total, 4) for k, c in sorted(cls.items(), key=lambda kv: -kv[1]["ms"])}
+    dom_name = max(cls, key=lambda k: cls[k]["ms"])
+
+    def roof(k):
+        c = cls[k]
+        per = c["ms"] / c["launches"] / 1e3
+        if k == "gemm_prefill":
+            ach = c["flops"] / c["launches"] / per / 1e12
+            return {"kernel": k, "bound": "tensor", "achieved": ach, "peak": tf_sus, "unit": "TFLOP/s",
+                    "frac": ach / tf_sus, "traffic": None, "launches": c["launches"],
+                    "avg_launch_us": per * 1e6}
+        ach = c["bytes"] / c["launches"] / per / 1e9
+        return {"kernel": k, "bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s",
+                "frac": ach / hbm, "traffic": None, "launches": c["launches"],
+                "avg_launch_us": per * 1e6}
+
+    out = {"dominant": roof(dom_name) if dom_name in ("gemm_decode", "gemm_prefill", "attn_decode")
+           else {"kernel": dom_name, "bound": "hbm", "achieved": None, "peak": hbm, "unit": "GB/s",
+                 "frac": None, "traffic": None},
+           "shares": shares}
+    if "attn_decode" in cls:
+        out["attn_decode"] = roof("attn_decode")
+    return out
+
+
+def native_record():
+    from hierarchical_global_local_b200 import native
+    import ctypes
+
+    class Rec(ctypes.Structure):
+        _fields_ = [("kind", ctypes.c_int32), ("m", ctypes.c_int32), ("n", ctypes.c_int32),
+                    ("k", ctypes.c_int32), ("ms", ctypes.c_float)]
+    return Rec
+
+
+# --------------------------------------------------------------------------
+# oracle on the host cores (baseline / reference arm)
+# --------------------------------------------------------------------------
+
+def _threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(budget_s: float = 20.0):
+    """The oracle (fp64 numpy), as it stands, on a bounded sample of the same
+    workload: 1 sequence of each run, the full prompt, and as many generated
+    tokens as fit in the time budget (split between the runs)."""
+    from oracle.model import BlockTransformerOracle
+    wl = synth.WORKLOADS[RUNS[0]]
+    w = synth.make_weights(wl)
+    params = {n: w.values(n) for n in w.names()}
+    o = BlockTransformerOracle(wl.shape, params)
+    gen_total, t_total, parts = 0, 0.0, []
+    for r in RUNS:
+        x = synth.WORKLOADS[r]
+        toks = synth.make_tokens(x, batch=1)
+        sess = o.session()
+        t0 = time.perf_counter()
+        z = sess.prefill(toks[:, :x.prompt_len])
+        g = 1
+        while g < x.gen_len and time.perf_counter() - t0 < budget_s / len(RUNS):
+            z = sess.decode(z.argmax(-1))
+            g += 1
+        dt = time.perf_counter() - t0
+        gen_total += g
+        t_total += dt
+        parts.append(f"{r}: 1 sequence, prompt {x.prompt_len}, {g} of {x.gen_len} tokens, {dt:.1f}s")
+    return {"value": gen_total / t_total, "unit": UNIT, "cores": _threads(), "kind": "oracle",
+            "sample": "; ".join(parts)}
+
+
+def run_reference(args):
+    ws, rank, _ = _dist()
+    if rank != 0:
+        return
+    per_step = []
+    for _ in range(args.warmup + args.steps):
+        per_step.append(cpu_baseline(budget_s=max(5.0, 60.0 / (args.warmup + args.steps))))
+    timed = per_step[args.warmup:]
+    v = statistics.mean(s["value"] for s in timed)
+    line = {"metric": METRIC, "value": v, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": "pythia160m-scale Block Transformer L_B=4 6+6 layers P=1: "
+                                   "prefill-heavy B64 2048/128 + decode-heavy B64 128/2048",
+                       "parallelism": "host cores"},
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": timed[0]["cores"], "kind": "oracle",
+                             "sample": timed[0]["sample"]},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-profile", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -216,7 +216,7 @@ static cudaError_t launch_dec(const void* q, int ldq, const void* kc, const void
   const float qscale = 1.4426950408889634f / sqrtf((float)DH);
   attn_decode_kernel<T, DH><<<grid, C::THREADS, C::SMEM, s>>>(
       (const T*)q, ldq, (const T*)kc, (const T*)vc, H, cap, kvlen, (T*)out, ld_out, partp,
-      counters, ms, status, qscale);
+      counters, ms, status, qscale); note_launch();
   return cudaGetLastError();
 }
 
@@ -291,7 +291,7 @@ cudaError_t launch_attn_small(int dt, const void* q, int ldq, const void* k_cach
 #define BT_SMALL(T, DHV)                                                                      \
   attn_small_kernel<T, DHV><<<grid, 128, 0, s>>>((const T*)q, ldq, (const T*)k_cache,        \
                                                   (const T*)v_cache, B, H, cap, qpos, (T*)out, \
-                                                  ld_out, scale);                             \
+                                                  ld_out, scale); note_launch();                             \
   return cudaGetLastError()
   if (dt == DT_BF16) {
     if (d == 32) { BT_SMALL(bf16, 32); }

@@ -12,6 +12,10 @@
 
 namespace bt {
 
+static long long g_launches = 0;
+void note_launch() { __atomic_add_fetch(&g_launches, 1, __ATOMIC_RELAXED); }
+long long launch_count() { return __atomic_load_n(&g_launches, __ATOMIC_RELAXED); }
+
 // ---------------------------------------------------------------------------
 // embedder
 // ---------------------------------------------------------------------------
@@ -79,35 +83,39 @@ cudaError_t launch_embed_prompt(int dt, const int32_t* tokens, int B, int T, int
                                 cudaStream_t s) {
   const int n = T / L_B;
   if (B * n == 0) return cudaSuccess;
-  if (dt == DT_BF16)
+  if (dt == DT_BF16) {
     embed_prompt_kernel<bf16><<<B * n, 256, 0, s>>>(tokens, T, n, L_B, (const bf16*)blk_emb, V, D,
-                                                    h, status);
-  else
+                                                    h, status); note_launch();
+  }
+  else {
     embed_prompt_kernel<float><<<B * n, 256, 0, s>>>(tokens, T, n, L_B, (const float*)blk_emb, V,
-                                                     D, h, status);
+                                                     D, h, status); note_launch();
+  }
   return cudaGetLastError();
 }
 
 cudaError_t launch_ingest(int dt, const int32_t* src, int32_t* block_tok, const int* dstate,
                           int B, int L_B, int V, int D, int block_step, const void* blk_emb,
                           const void* tok_emb, float* h, int* status, cudaStream_t s) {
-  if (dt == DT_BF16)
+  if (dt == DT_BF16) {
     ingest_kernel<bf16><<<B, 256, 0, s>>>(src, block_tok, dstate, L_B, V, D, block_step,
-                                          (const bf16*)blk_emb, (const bf16*)tok_emb, h, status);
-  else
+                                          (const bf16*)blk_emb, (const bf16*)tok_emb, h, status); note_launch();
+  }
+  else {
     ingest_kernel<float><<<B, 256, 0, s>>>(src, block_tok, dstate, L_B, V, D, block_step,
                                            (const float*)blk_emb, (const float*)tok_emb, h,
-                                           status);
+                                           status); note_launch();
+  }
   return cudaGetLastError();
 }
 
 cudaError_t launch_set_state(int* dstate, int t, int L_B, cudaStream_t s) {
-  set_state_kernel<<<1, 1, 0, s>>>(dstate, t, L_B);
+  set_state_kernel<<<1, 1, 0, s>>>(dstate, t, L_B); note_launch();
   return cudaGetLastError();
 }
 
 cudaError_t launch_advance(int* dstate, int L_B, cudaStream_t s) {
-  advance_kernel<<<1, 1, 0, s>>>(dstate, L_B);
+  advance_kernel<<<1, 1, 0, s>>>(dstate, L_B); note_launch();
   return cudaGetLastError();
 }
 
@@ -195,10 +203,12 @@ cudaError_t launch_ln_dual(int dt, const float* h, int M, int D, const float* g1
   if (M == 0) return cudaSuccess;
   const int rows_per_cta = 8;
   dim3 grid((M + rows_per_cta - 1) / rows_per_cta);
-  if (dt == DT_BF16)
-    ln_dual_kernel<bf16><<<grid, 256, 0, s>>>(h, M, D, g1, b1, g2, b2, eps, (bf16*)x1);
-  else
-    ln_dual_kernel<float><<<grid, 256, 0, s>>>(h, M, D, g1, b1, g2, b2, eps, (float*)x1);
+  if (dt == DT_BF16) {
+    ln_dual_kernel<bf16><<<grid, 256, 0, s>>>(h, M, D, g1, b1, g2, b2, eps, (bf16*)x1); note_launch();
+  }
+  else {
+    ln_dual_kernel<float><<<grid, 256, 0, s>>>(h, M, D, g1, b1, g2, b2, eps, (float*)x1); note_launch();
+  }
   return cudaGetLastError();
 }
 
@@ -206,10 +216,12 @@ cudaError_t launch_ln_rows(int dt, const float* h, int R, int row_step, int row_
                            const float* g, const float* b, float eps, void* out, cudaStream_t s) {
   if (R == 0) return cudaSuccess;
   dim3 grid((R + 7) / 8);
-  if (dt == DT_BF16)
-    ln_rows_kernel<bf16><<<grid, 256, 0, s>>>(h, R, row_step, row_off, D, g, b, eps, (bf16*)out);
-  else
-    ln_rows_kernel<float><<<grid, 256, 0, s>>>(h, R, row_step, row_off, D, g, b, eps, (float*)out);
+  if (dt == DT_BF16) {
+    ln_rows_kernel<bf16><<<grid, 256, 0, s>>>(h, R, row_step, row_off, D, g, b, eps, (bf16*)out); note_launch();
+  }
+  else {
+    ln_rows_kernel<float><<<grid, 256, 0, s>>>(h, R, row_step, row_off, D, g, b, eps, (float*)out); note_launch();
+  }
   return cudaGetLastError();
 }
 
@@ -231,7 +243,7 @@ cudaError_t launch_rope_table(float2* tab, int n_pos, int rot, float base, cudaS
   const int half = rot / 2;
   if (half == 0 || n_pos == 0) return cudaSuccess;
   const int total = n_pos * half;
-  rope_table_kernel<<<(total + 255) / 256, 256, 0, s>>>(tab, n_pos, half, (double)base);
+  rope_table_kernel<<<(total + 255) / 256, 256, 0, s>>>(tab, n_pos, half, (double)base); note_launch();
   return cudaGetLastError();
 }
 
@@ -270,13 +282,15 @@ cudaError_t launch_rope_append(int dt, const void* qkv, int M, int D, int H, int
                                const float2* rope_tab, PosSpec pos, void* q_out, void* k_cache,
                                void* v_cache, int cap, cudaStream_t s) {
   if (M == 0) return cudaSuccess;
-  if (dt == DT_BF16)
+  if (dt == DT_BF16) {
     rope_append_kernel<bf16><<<M, 256, 0, s>>>((const bf16*)qkv, D, H, rot, rope_tab, pos,
-                                               (bf16*)q_out, (bf16*)k_cache, (bf16*)v_cache, cap);
-  else
+                                               (bf16*)q_out, (bf16*)k_cache, (bf16*)v_cache, cap); note_launch();
+  }
+  else {
     rope_append_kernel<float><<<M, 256, 0, s>>>((const float*)qkv, D, H, rot, rope_tab, pos,
                                                 (float*)q_out, (float*)k_cache, (float*)v_cache,
-                                                cap);
+                                                cap); note_launch();
+  }
   return cudaGetLastError();
 }
 
@@ -321,7 +335,7 @@ __global__ void argmax_kernel(const float* __restrict__ logits, int V, int ld,
 cudaError_t launch_argmax(const float* logits, int B, int V, int ld, int32_t* next,
                           cudaStream_t s) {
   if (B == 0) return cudaSuccess;
-  argmax_kernel<<<B, 1024, 0, s>>>(logits, V, ld, next);
+  argmax_kernel<<<B, 1024, 0, s>>>(logits, V, ld, next); note_launch();
   return cudaGetLastError();
 }
 
@@ -348,6 +362,7 @@ cudaError_t launch_convert_to_f32(int dt, const void* src, float* dst, size_t n,
   const int grid = (int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
   if (dt == DT_BF16) convert_kernel<bf16><<<grid, 256, 0, s>>>((const bf16*)src, dst, n);
   else convert_kernel<float><<<grid, 256, 0, s>>>((const float*)src, dst, n);
+  note_launch();
   return cudaGetLastError();
 }
 
@@ -357,6 +372,7 @@ cudaError_t launch_add_to_f32(int dt, const void* a, const void* b, float* dst, 
   const int grid = (int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
   if (dt == DT_BF16) add_kernel<bf16><<<grid, 256, 0, s>>>((const bf16*)a, (const bf16*)b, dst, n);
   else add_kernel<float><<<grid, 256, 0, s>>>((const float*)a, (const float*)b, dst, n);
+  note_launch();
   return cudaGetLastError();
 }
 

@@ -110,12 +110,14 @@ cudaError_t launch_gemm(int dt, const void* X, int ldx, const void* W, int ldw, 
     const uint8_t* Xp = (const uint8_t*)X + (part ? (size_t)xk_off * es : 0);
     const uint8_t* Wp = (const uint8_t*)W + (size_t)nb * ldw * es;
     dim3 grid((nn + 63) / 64, (M + 63) / 64);
-    if (dt == DT_BF16)
+    if (dt == DT_BF16) {
       gemm_simt_kernel<bf16><<<grid, 256, 0, s>>>((const bf16*)Xp, ldx, (const bf16*)Wp, ldw, M,
-                                                  nn, K, nb, e);
-    else
+                                                  nn, K, nb, e); note_launch();
+    }
+    else {
       gemm_simt_kernel<float><<<grid, 256, 0, s>>>((const float*)Xp, ldx, (const float*)Wp, ldw,
-                                                   M, nn, K, nb, e);
+                                                   M, nn, K, nb, e); note_launch();
+    }
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return err;
   }

@@ -114,6 +114,12 @@ int gemm_tc_supported(int dt, int M, int N, int K, int xk_split, int xk_off);
 cudaError_t launch_argmax(const float* logits, int B, int V, int ld, int32_t* next,
                           cudaStream_t s);
 
+// ---- launch accounting ------------------------------------------------------
+// Every kernel launch site calls note_launch(); launch_count() is the running
+// total for this process (graph captures count when captured).
+void note_launch();
+long long launch_count();
+
 // ---- misc -----------------------------------------------------------------
 cudaError_t launch_convert_to_f32(int dt, const void* src, float* dst, size_t n, cudaStream_t s);
 cudaError_t launch_add_to_f32(int dt, const void* a, const void* b, float* dst, size_t n,

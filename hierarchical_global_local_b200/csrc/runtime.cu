@@ -127,7 +127,31 @@ struct bt_model {
   bool prefilled = false;
   bool use_graphs = true;
   cudaGraphExec_t graphs[2][2] = {{nullptr, nullptr}, {nullptr, nullptr}};  // [block_step][greedy]
+  long long graph_kernels[2][2] = {{0, 0}, {0, 0}};
   int graph_B = 0;
+  long long kernels = 0;  // kernels enqueued for execution
+  // profiler
+  bool prof = false;
+  bool capturing = false;
+  std::vector<cudaEvent_t> ev;
+  std::vector<bt_profile_record> rec;
+  int cap_records = 0;
+};
+
+// Event pair around one kernel launch while the profiler is on.
+struct ProfScope {
+  bt_model* m;
+  cudaStream_t s;
+  int idx = -1;
+  ProfScope(bt_model* m_, cudaStream_t s_, int kind, int M, int N, int K) : m(m_), s(s_) {
+    if (!m->prof || m->capturing || (int)m->rec.size() >= m->cap_records) return;
+    idx = (int)m->rec.size();
+    m->rec.push_back(bt_profile_record{kind, M, N, K, 0.f});
+    cudaEventRecord(m->ev[2 * idx], s);
+  }
+  ~ProfScope() {
+    if (idx >= 0) cudaEventRecord(m->ev[2 * idx + 1], s);
+  }
 };
 
 static size_t carve(bt_model* m, const Dims& d, void* ws) {
@@ -306,21 +330,37 @@ static int run_layer(bt_model* m, const LayerW& w, float* h, int M, PosSpec pos,
                      void* vc, int cap, AttnKind ak, int n_prefill, cudaStream_t s) {
   const Dims& d = m->d;
   const int D = d.D;
-  BT_CUDA(launch_ln_dual(d.dt, h, M, D, w.ln1_g, w.ln1_b, w.ln2_g, w.ln2_b, m->cfg.ln_eps, m->x1, s));
-  Epi e1{EPI_QKV1, m->qkv, 3 * D, m->a2, 5 * D, w.b_qkv1, 3 * D, D};
-  BT_CUDA(launch_gemm(d.dt, m->x1, 2 * D, w.w_qkv1, D, M, 7 * D, D, 3 * D, D, e1, m->gs, m->status, s));
-  BT_CUDA(launch_rope_append(d.dt, m->qkv, M, D, d.H, d.rot, m->rope_tab, pos, m->qrot, kc, vc, cap, s));
+  {
+    ProfScope p(m, s, BT_K_LAYERNORM, M, D, 0);
+    BT_CUDA(launch_ln_dual(d.dt, h, M, D, w.ln1_g, w.ln1_b, w.ln2_g, w.ln2_b, m->cfg.ln_eps, m->x1, s));
+  }
+  {
+    ProfScope p(m, s, BT_K_GEMM, M, 7 * D, D);
+    Epi e1{EPI_QKV1, m->qkv, 3 * D, m->a2, 5 * D, w.b_qkv1, 3 * D, D};
+    BT_CUDA(launch_gemm(d.dt, m->x1, 2 * D, w.w_qkv1, D, M, 7 * D, D, 3 * D, D, e1, m->gs, m->status, s));
+  }
+  {
+    ProfScope p(m, s, BT_K_ROPE_APPEND, M, 3 * D, 0);
+    BT_CUDA(launch_rope_append(d.dt, m->qkv, M, D, d.H, d.rot, m->rope_tab, pos, m->qrot, kc, vc, cap, s));
+  }
   const int Bseq = M / pos.rows_per_seq;
   if (ak == ATT_PREFILL) {
+    ProfScope p(m, s, BT_K_ATTN_PREFILL, Bseq * d.H, n_prefill, d.d);
     BT_CUDA(launch_attn_prefill(d.dt, m->qrot, D, kc, vc, Bseq, d.H, d.d, cap, n_prefill, m->a2, 5 * D, s));
   } else if (ak == ATT_DECODE) {
+    // entries read: the block index of the fed token + 1 (known on the host)
+    ProfScope p(m, s, BT_K_ATTN_DECODE, Bseq * d.H, m->t / d.L + 1, d.d);
     BT_CUDA(launch_attn_decode(d.dt, m->qrot, D, kc, vc, Bseq, d.H, d.d, cap, pos, m->a2, 5 * D,
                                m->attn_scratch, m->status, s));
   } else {
+    ProfScope p(m, s, BT_K_ATTN_LOCAL, M * d.H, cap, d.d);
     BT_CUDA(launch_attn_small(d.dt, m->qrot, D, kc, vc, Bseq, d.H, d.d, cap, pos, m->a2, 5 * D, s));
   }
-  Epi e2{EPI_RESID, h, D, nullptr, 0, w.b_o2, 0, D};
-  BT_CUDA(launch_gemm(d.dt, m->a2, 5 * D, w.w_o2, 5 * D, M, D, 5 * D, 1 << 30, 0, e2, m->gs, m->status, s));
+  {
+    ProfScope p(m, s, BT_K_GEMM, M, D, 5 * D);
+    Epi e2{EPI_RESID, h, D, nullptr, 0, w.b_o2, 0, D};
+    BT_CUDA(launch_gemm(d.dt, m->a2, 5 * D, w.w_o2, 5 * D, M, D, 5 * D, 1 << 30, 0, e2, m->gs, m->status, s));
+  }
   return BT_OK;
 }
 
@@ -338,6 +378,7 @@ static int run_token_decoder(bt_model* m, int B, PosSpec pos, cudaStream_t s) {
                        layer_ptr(m->vt, m->kt_layer, l, d.eb), d.l_cap, ATT_LOCAL, 0, s);
     if (rc != BT_OK) return rc;
   }
+  ProfScope p(m, s, BT_K_LAYERNORM, B, d.D, 0);
   BT_CUDA(launch_ln_rows(d.dt, m->h_t, B, pos.rows_per_seq, pos.rows_per_seq - 1, d.D, m->lnf_t_g,
                          m->lnf_t_b, m->cfg.ln_eps, m->xf, s));
   return BT_OK;
@@ -347,22 +388,34 @@ static int run_token_decoder(bt_model* m, int B, PosSpec pos, cudaStream_t s) {
 // prefix projection and the token decoder over P rows, or (vanilla) xf.
 static int run_context_to_head_input(bt_model* m, int B, int row_step, int row_off, cudaStream_t s) {
   const Dims& d = m->d;
-  BT_CUDA(launch_ln_rows(d.dt, m->h_b, B, row_step, row_off, d.D, m->lnf_b_g, m->lnf_b_b,
-                         m->cfg.ln_eps, m->xf, s));
+  {
+    ProfScope p(m, s, BT_K_LAYERNORM, B, d.D, 0);
+    BT_CUDA(launch_ln_rows(d.dt, m->h_b, B, row_step, row_off, d.D, m->lnf_b_g, m->lnf_b_b,
+                           m->cfg.ln_eps, m->xf, s));
+  }
   if (!d.tokdec) return BT_OK;
-  // prefix rows: h_t[b*P + p, :] = (W_p c_b + b_p)[p*D:(p+1)*D]
-  Epi ep{EPI_F32, m->h_t, d.P * d.D, nullptr, 0, m->b_prefix, 0, d.D};
-  BT_CUDA(launch_gemm(d.dt, m->xf, d.D, m->w_prefix, d.D, B, d.P * d.D, d.D, 1 << 30, 0, ep, m->gs,
-                      m->status, s));
+  {
+    // prefix rows: h_t[b*P + p, :] = (W_p c_b + b_p)[p*D:(p+1)*D]
+    ProfScope p(m, s, BT_K_GEMM, B, d.P * d.D, d.D);
+    Epi ep{EPI_F32, m->h_t, d.P * d.D, nullptr, 0, m->b_prefix, 0, d.D};
+    BT_CUDA(launch_gemm(d.dt, m->xf, d.D, m->w_prefix, d.D, B, d.P * d.D, d.D, 1 << 30, 0, ep, m->gs,
+                        m->status, s));
+  }
   PosSpec pos{nullptr, POS_ZERO, 0, d.P};
   return run_token_decoder(m, B, pos, s);
 }
 
 static int run_head(bt_model* m, int B, cudaStream_t s) {
   const Dims& d = m->d;
-  Epi el{EPI_F32, m->logits, d.V, nullptr, 0, nullptr, 0, d.D};
-  BT_CUDA(launch_gemm(d.dt, m->xf, d.D, m->w_lm, d.D, B, d.V, d.D, 1 << 30, 0, el, m->gs, m->status, s));
-  BT_CUDA(launch_argmax(m->logits, B, d.V, d.V, m->next, s));
+  {
+    ProfScope p(m, s, BT_K_GEMM, B, d.V, d.D);
+    Epi el{EPI_F32, m->logits, d.V, nullptr, 0, nullptr, 0, d.D};
+    BT_CUDA(launch_gemm(d.dt, m->xf, d.D, m->w_lm, d.D, B, d.V, d.D, 1 << 30, 0, el, m->gs, m->status, s));
+  }
+  {
+    ProfScope p(m, s, BT_K_ARGMAX, B, d.V, 0);
+    BT_CUDA(launch_argmax(m->logits, B, d.V, d.V, m->next, s));
+  }
   return BT_OK;
 }
 
@@ -380,8 +433,11 @@ static int enqueue_decode(bt_model* m, bool block_step, bool greedy, cudaStream_
   const Dims& d = m->d;
   const int B = m->B;
   const int32_t* src = greedy ? m->next : m->fed;
-  BT_CUDA(launch_ingest(d.dt, src, m->block_tok, m->dstate, B, d.L, d.V, d.D, block_step ? 1 : 0,
-                        m->blk_emb, m->tok_emb, block_step ? m->h_b : m->h_t, m->status, s));
+  {
+    ProfScope p(m, s, BT_K_EMBED, B, d.D, 0);
+    BT_CUDA(launch_ingest(d.dt, src, m->block_tok, m->dstate, B, d.L, d.V, d.D, block_step ? 1 : 0,
+                          m->blk_emb, m->tok_emb, block_step ? m->h_b : m->h_t, m->status, s));
+  }
   int rc;
   if (block_step) {
     PosSpec pos{m->dstate, POS_BLOCK, 0, 1};
@@ -399,7 +455,10 @@ static int enqueue_decode(bt_model* m, bool block_step, bool greedy, cudaStream_
   }
   rc = run_head(m, B, s);
   if (rc != BT_OK) return rc;
-  BT_CUDA(launch_advance(m->dstate, d.L, s));
+  {
+    ProfScope p(m, s, BT_K_OTHER, 1, 0, 0);
+    BT_CUDA(launch_advance(m->dstate, d.L, s));
+  }
   return BT_OK;
 }
 
@@ -423,8 +482,12 @@ int bt_prefill(bt_model* m, const int32_t* tokens, int32_t B, int32_t T, float* 
   m->t = T;
   const int n = T / d.L;
   const int M = B * n;
+  const long long k0 = launch_count();
   BT_CUDA(launch_set_state(m->dstate, T, d.L, s));
-  BT_CUDA(launch_embed_prompt(d.dt, tokens, B, T, d.L, m->blk_emb, d.V, d.D, m->h_b, m->status, s));
+  {
+    ProfScope p(m, s, BT_K_EMBED, M, d.D, 0);
+    BT_CUDA(launch_embed_prompt(d.dt, tokens, B, T, d.L, m->blk_emb, d.V, d.D, m->h_b, m->status, s));
+  }
   PosSpec pos{nullptr, POS_ZERO, 0, n};
   for (int l = 0; l < d.Nb; ++l) {
     int rc = run_layer(m, m->blk[l], m->h_b, M, pos, layer_ptr(m->kb, m->kb_layer, l, d.eb),
@@ -435,6 +498,7 @@ int bt_prefill(bt_model* m, const int32_t* tokens, int32_t B, int32_t T, float* 
   if (rc != BT_OK) return rc;
   rc = run_head(m, B, s);
   if (rc != BT_OK) return rc;
+  m->kernels += launch_count() - k0;
   m->prefilled = true;
   if (m->graph_B != B) { drop_graphs(m); m->graph_B = B; }
   return copy_outputs(m, logits, next);
@@ -449,8 +513,9 @@ int bt_decode_step(bt_model* m, const int32_t* tokens, float* logits, int32_t* n
   const bool greedy = tokens == nullptr;
   if (!greedy)
     BT_CUDA(cudaMemcpyAsync(m->fed, tokens, (size_t)m->B * 4, cudaMemcpyDeviceToDevice, m->stream));
-  if (m->use_graphs) {
+  if (m->use_graphs && !m->prof) {
     cudaGraphExec_t& g = m->graphs[block_step ? 1 : 0][greedy ? 1 : 0];
+    long long& gk = m->graph_kernels[block_step ? 1 : 0][greedy ? 1 : 0];
     if (!g) {
       // capture on the private stream, ordered after the caller's stream
       cudaEvent_t ev;
@@ -461,7 +526,11 @@ int bt_decode_step(bt_model* m, const int32_t* tokens, float* logits, int32_t* n
       cudaEventDestroy(ev);
       cudaGraph_t graph;
       BT_CUDA(cudaStreamBeginCapture(m->cap_stream, cudaStreamCaptureModeThreadLocal));
+      const long long c0 = launch_count();
+      m->capturing = true;
       int rc = enqueue_decode(m, block_step, greedy, m->cap_stream);
+      m->capturing = false;
+      gk = launch_count() - c0;
       cudaError_t ce = cudaStreamEndCapture(m->cap_stream, &graph);
       if (rc != BT_OK) return rc;
       BT_CUDA(ce);
@@ -469,9 +538,12 @@ int bt_decode_step(bt_model* m, const int32_t* tokens, float* logits, int32_t* n
       cudaGraphDestroy(graph);
     }
     BT_CUDA(cudaGraphLaunch(g, m->stream));
+    m->kernels += gk;
   } else {
+    const long long c0 = launch_count();
     int rc = enqueue_decode(m, block_step, greedy, m->stream);
     if (rc != BT_OK) return rc;
+    m->kernels += launch_count() - c0;
   }
   m->t += 1;
   return copy_outputs(m, logits, next);
@@ -496,9 +568,45 @@ int bt_position(const bt_model* m) {
   return m->t;
 }
 
+int64_t bt_kernel_launches(const bt_model* m) { return m ? (int64_t)m->kernels : -1; }
+
+static void free_events(bt_model* m) {
+  for (auto e : m->ev) cudaEventDestroy(e);
+  m->ev.clear();
+}
+
+int bt_profile_begin(bt_model* m, int32_t capacity) {
+  if (!m || capacity <= 0) return BT_EINVAL;
+  free_events(m);
+  m->rec.clear();
+  m->rec.reserve(capacity);
+  m->ev.resize(2 * (size_t)capacity);
+  for (auto& e : m->ev) BT_CUDA(cudaEventCreate(&e));
+  m->cap_records = capacity;
+  m->prof = true;
+  return BT_OK;
+}
+
+int bt_profile_end(bt_model* m, bt_profile_record* out, int32_t capacity, int32_t* n_out) {
+  if (!m || !m->prof) return BT_EINVAL;
+  m->prof = false;
+  BT_CUDA(cudaStreamSynchronize(m->stream));
+  const int n = (int)m->rec.size() < capacity ? (int)m->rec.size() : capacity;
+  for (int i = 0; i < n; ++i) {
+    float ms = 0.f;
+    BT_CUDA(cudaEventElapsedTime(&ms, m->ev[2 * i], m->ev[2 * i + 1]));
+    m->rec[i].ms = ms;
+    if (out) out[i] = m->rec[i];
+  }
+  if (n_out) *n_out = n;
+  free_events(m);
+  return BT_OK;
+}
+
 int bt_destroy(bt_model* m) {
   if (!m) return BT_EINVAL;
   cudaStreamSynchronize(m->stream);
+  free_events(m);
   drop_graphs(m);
   if (m->cap_stream) cudaStreamDestroy(m->cap_stream);
   delete m;

@@ -77,6 +77,9 @@ def lib() -> ctypes.CDLL:
             "bt_destroy": (c_int, [c_void_p]),
             "bt_strerror": (ctypes.c_char_p, [c_int]),
             "bt_last_cuda_error": (ctypes.c_char_p, []),
+            "bt_kernel_launches": (ctypes.c_int64, [c_void_p]),
+            "bt_profile_begin": (c_int, [c_void_p, c_int32]),
+            "bt_profile_end": (c_int, [c_void_p, c_void_p, c_int32, c_void_p]),
             "bt_op_decode_attention_scratch_bytes": (c_size_t, [c_int] * 5),
             "bt_op_decode_attention": (c_int, [c_int, c_void_p, c_int, c_void_p, c_void_p, c_int,
                                                c_int, c_int, c_int, c_int, c_void_p, c_int,
@@ -105,6 +108,7 @@ def exported_symbols():
     return [
         "bt_workspace_bytes", "bt_create", "bt_prefill", "bt_decode_step", "bt_sync",
         "bt_position", "bt_destroy", "bt_strerror", "bt_last_cuda_error",
+        "bt_kernel_launches", "bt_profile_begin", "bt_profile_end",
         "bt_op_decode_attention_scratch_bytes", "bt_op_decode_attention",
         "bt_op_prefill_attention", "bt_op_linear_scratch_bytes", "bt_op_linear",
         "bt_op_layernorm", "bt_op_embed_prompt"]

@@ -25,7 +25,8 @@
  *     call returns after enqueueing. Outputs are valid once that stream has
  *     reached them (bt_sync, or any later stream-ordered consumer).
  *   - The library never allocates device memory: all device state lives in
- *     the caller's workspace. It creates two CUDA streams for graph capture.
+ *     the caller's workspace. It creates one private CUDA stream (graph
+ *     capture) per model.
  *   - Errors are returned as negative bt_status codes; the library never
  *     aborts the process and never traps the device. Device-side failures
  *     (a token id outside [0, vocab), a bounded wait that ran out) set a
@@ -166,6 +167,35 @@ BT_API int bt_position(const bt_model *m);
 /* Release host-side resources (graphs, streams). Does not free the caller's
  * workspace. Waits for the model's outstanding work first. */
 BT_API int bt_destroy(bt_model *m);
+
+/* ---- measurement support ------------------------------------------------
+ * Kernel kinds reported by the profiler. */
+enum {
+  BT_K_GEMM = 0, BT_K_ATTN_DECODE = 1, BT_K_ATTN_PREFILL = 2, BT_K_ATTN_LOCAL = 3,
+  BT_K_LAYERNORM = 4, BT_K_ROPE_APPEND = 5, BT_K_EMBED = 6, BT_K_ARGMAX = 7, BT_K_OTHER = 8
+};
+
+/* One timed kernel launch: kind, shape (GEMM: M, N, K; decode attention:
+ * B*H, cached entries read, d_head; others: rows, width, 0) and its duration
+ * from a pair of CUDA events recorded on the model's stream around it. */
+typedef struct bt_profile_record {
+  int32_t kind, m, n, k;
+  float ms;
+} bt_profile_record;
+
+/* Number of this model's kernels that have been enqueued for execution so
+ * far (each replay of a captured decode graph counts its kernel nodes). */
+BT_API int64_t bt_kernel_launches(const bt_model *m);
+
+/* Start recording an event pair around every kernel launch, for at most
+ * `capacity` launches. While recording, decode steps are enqueued kernel by
+ * kernel instead of as graph replays. Creates 2*capacity CUDA events. */
+BT_API int bt_profile_begin(bt_model *m, int32_t capacity);
+
+/* Stop recording, wait for the stream, and copy up to `capacity` records
+ * into out (host array); *n_out receives the number copied. */
+BT_API int bt_profile_end(bt_model *m, bt_profile_record *out, int32_t capacity,
+                          int32_t *n_out);
 
 /* Static, human-readable name of a status code. */
 BT_API const char *bt_strerror(int status);
