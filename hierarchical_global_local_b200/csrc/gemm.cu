@@ -11,36 +11,10 @@
 // The SIMT path serves fp32 workloads (FFMA, no TF32) and any shape the
 // tensor-core path does not take.
 #include "common.cuh"
+#include "epilogue.cuh"
 #include "kernels.h"
 
 namespace bt {
-
-template <typename T>
-__device__ __forceinline__ void epi_apply(const Epi& e, int m, int n, float acc) {
-  switch (e.kind) {
-    case EPI_QKV1: {
-      const float v = acc + e.bias[n];
-      if (n < e.split_n)
-        reinterpret_cast<T*>(e.out0)[(size_t)m * e.ld0 + n] = from_f<T>(v);
-      else
-        reinterpret_cast<T*>(e.out1)[(size_t)m * e.ld1 + e.D + (n - e.split_n)] =
-            from_f<T>(gelu_erf(v));
-      break;
-    }
-    case EPI_RESID: {
-      float* o = reinterpret_cast<float*>(e.out0) + (size_t)m * e.ld0 + n;
-      *o = *o + (acc + e.bias[n]);
-      break;
-    }
-    case EPI_F32:
-      reinterpret_cast<float*>(e.out0)[(size_t)m * e.ld0 + n] = acc + (e.bias ? e.bias[n] : 0.f);
-      break;
-    default:
-      reinterpret_cast<T*>(e.out0)[(size_t)m * e.ld0 + n] =
-          from_f<T>(acc + (e.bias ? e.bias[n] : 0.f));
-      break;
-  }
-}
 
 // 64x64 output tile, K step 16, 256 threads, 4x4 outputs per thread.
 template <typename T>

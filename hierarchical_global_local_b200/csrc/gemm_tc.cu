@@ -1,18 +1,357 @@
-// gemm_tc.cu -- tensor-core (tcgen05) GEMM path. Placeholder until the
-// kernel lands: reports no supported shapes, so the SIMT path runs.
+// gemm_tc.cu -- bf16 dense projections on the 5th-generation tensor cores
+// (tcgen05 + TMEM), sm_100a.
+//
+// D[r, c] = sum_k A[r, k] * B[c, k]; A and B K-major bf16 in global memory,
+// fp32 accumulation in tensor memory. One CTA per 128 x BN output tile (and
+// per K split):
+//   * one thread issues TMA tile loads (128-byte swizzle, no multicast) into a
+//     4-stage shared-memory ring guarded by full/empty mbarriers;
+//   * one thread issues tcgen05.mma (M = 128, N = BN, K = 16) per 16-wide K
+//     slice and commits each stage back to its empty barrier;
+//   * all four warps read the accumulator with tcgen05.ld (warp w owns TMEM
+//     lanes 32w..32w+31) and apply the fused epilogue.
+// Two orientations:
+//   decode ("weights as A"): A = W [N, K] (128 output features per tile),
+//     B = X [M, K] (the M <= 256 tokens of the batch, padded to BN by TMA
+//     zero fill). K is split across CTAs so that every SM streams weights;
+//     each split writes an fp32 partial tile and the last CTA of a tile (an
+//     atomic counter, no waiting) sums the partials in split order and runs
+//     the epilogue, so results do not depend on CTA timing.
+//   prefill ("activations as A"): A = X (128 tokens per tile), B = W (BN
+//     features per tile), one K split.
+// Every mbarrier wait is bounded; a wait that runs out sets a status bit.
+#include <cuda.h>
+#include <stdio.h>
+
 #include "common.cuh"
+#include "epilogue.cuh"
 #include "kernels.h"
 
 namespace bt {
 
-size_t gemm_scratch_bytes(int max_M, int max_N) { return 256; }
-int gemm_counter_count(int max_N) { return 64; }
-int gemm_tc_supported(int dt, int M, int N, int K, int xk_split, int xk_off) { return 0; }
+namespace {
+
+constexpr int BM = 128;  // MMA M (TMEM lanes)
+constexpr int BK = 64;   // K elements per stage = one 128-byte swizzle row
+constexpr int STAGES = 4;
+constexpr size_t PART_BUDGET = 64ull << 20;
+
+// ---- tcgen05 / TMA wrappers --------------------------------------------------
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
+  // K-major, 128-byte swizzle: rows of 128 B, 8-row groups 1024 B apart.
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFF) >> 4);          // start address
+  d |= (uint64_t)(16 >> 4) << 16;                   // leading byte offset (unused)
+  d |= (uint64_t)(1024 >> 4) << 32;                 // stride byte offset
+  d |= (uint64_t)1 << 46;                           // descriptor version
+  d |= (uint64_t)2 << 61;                           // SWIZZLE_128B
+  return d;
+}
+
+template <int BN>
+__device__ __forceinline__ constexpr uint32_t instr_desc() {
+  // kind::f16: D fp32, A bf16, B bf16, both K-major, M = 128, N = BN.
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+         ((uint32_t)(BM >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc,
+                                         uint32_t accum) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
+      "l"(a), "l"(b), "r"(idesc), "r"(accum));
+}
+
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
+      "%4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15}, [%16];\n"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+template <int BN>
+__host__ __device__ constexpr int tmem_cols() {
+  return BN < 32 ? 32 : BN;
+}
+
+template <int BN>
+__host__ __device__ constexpr size_t smem_bytes() {
+  return (size_t)STAGES * (BM * BK * 2 + BN * BK * 2) + 1024;  // + alignment slack
+}
+
+// ---- the kernel ---------------------------------------------------------------
+// SWAP = true: A = weights (rows = output features), B = activations (rows =
+// tokens). SWAP = false: A = activations, B = weights.
+template <int BN, bool SWAP>
+__global__ void __launch_bounds__(128, 1)
+gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
+               int M, int N, int nkb, int ks, int xk_split, int xk_off, Epi e,
+               float* __restrict__ part, int* __restrict__ counters, int* status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~(uintptr_t)1023);
+  bf16* sA = reinterpret_cast<bf16*>(smem);
+  bf16* sB = reinterpret_cast<bf16*>(smem + (size_t)STAGES * BM * BK * 2);
+  __shared__ __align__(8) uint64_t full[STAGES], empty[STAGES], done;
+  __shared__ uint32_t tmem_slot;
+  __shared__ int s_last;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // tile coordinates: rows of A (BM) and rows of B (BN)
+  const int a0 = blockIdx.x * BM;
+  const int b0 = blockIdx.y * BN;
+  const int z = blockIdx.z;
+  const int feat0 = SWAP ? a0 : b0;
+  const int koff = (feat0 >= xk_split) ? xk_off : 0;
+  const int kb_begin = (int)(((long long)z * nkb) / ks);
+  const int kb_end = (int)(((long long)(z + 1) * nkb) / ks);
+  const int nloc = kb_end - kb_begin;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    mbar_init(&done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&tmem_slot)),
+                 "r"(tmem_cols<BN>()));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    // ---- producer: TMA loads ----
+    const uint32_t bytes = (uint32_t)(BM * BK * 2 + BN * BK * 2);
+    for (int i = 0; i < nloc; ++i) {
+      const int s = i % STAGES;
+      if (i >= STAGES) mbar_wait_bounded(&empty[s], ((i / STAGES) + 1) & 1, status);
+      mbar_arrive_expect_tx(&full[s], bytes);
+      const int k = (kb_begin + i) * BK;
+      tma_load_2d(sA + (size_t)s * BM * BK, &mapA, k + (SWAP ? 0 : koff), a0, &full[s]);
+      tma_load_2d(sB + (size_t)s * BN * BK, &mapB, k + (SWAP ? koff : 0), b0, &full[s]);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---- MMA issuer ----
+    constexpr uint32_t idesc = instr_desc<BN>();
+    for (int i = 0; i < nloc; ++i) {
+      const int s = i % STAGES;
+      mbar_wait_bounded(&full[s], (i / STAGES) & 1, status);
+      tc_fence_after();
+      const uint64_t da = smem_desc_sw128(smem_u32(sA + (size_t)s * BM * BK));
+      const uint64_t db = smem_desc_sw128(smem_u32(sB + (size_t)s * BN * BK));
+#pragma unroll
+      for (int kk = 0; kk < BK / 16; ++kk)  // 32 bytes per K slice: +2 in 16-byte units
+        mma_bf16(tmem, da + 2 * kk, db + 2 * kk, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+      mma_commit(&empty[s]);
+    }
+    mma_commit(&done);
+  }
+  __syncwarp();
+
+  // ---- epilogue ----
+  mbar_wait_bounded(&done, 0, status);
+  tc_fence_after();
+  const int r = warp * 32 + lane;  // TMEM lane = row of A
+  const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+  const int tile = blockIdx.x + gridDim.x * blockIdx.y;
+
+  if (ks == 1) {
+    for (int c0 = 0; c0 < BN; c0 += 16) {
+      float v[16];
+      tmem_ld16(trow + c0, v);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int m = SWAP ? (b0 + c0 + j) : (a0 + r);
+        const int n = SWAP ? (a0 + r) : (b0 + c0 + j);
+        if (m < M && n < N) epi_apply<bf16>(e, m, n, v[j]);
+      }
+    }
+  } else {
+    // partial tile [BN][BM] of this split (row index fastest: coalesced)
+    float* my = part + ((size_t)tile * ks + z) * BN * BM;
+    for (int c0 = 0; c0 < BN; c0 += 16) {
+      float v[16];
+      tmem_ld16(trow + c0, v);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) my[(size_t)(c0 + j) * BM + r] = v[j];
+    }
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_last = (atomicAdd(&counters[tile], 1) == ks - 1);
+    __syncthreads();
+    if (s_last) {
+      __threadfence();
+      const float* tp = part + (size_t)tile * ks * BN * BM;
+      for (int c = 0; c < BN; ++c) {
+        const int m = SWAP ? (b0 + c) : (a0 + r);
+        const int n = SWAP ? (a0 + r) : (b0 + c);
+        if (m >= M || n >= N) continue;
+        float acc = 0.f;
+        for (int zz = 0; zz < ks; ++zz) acc += __ldcg(tp + ((size_t)zz * BN + c) * BM + r);
+        epi_apply<bf16>(e, m, n, acc);
+      }
+      if (threadIdx.x == 0) counters[tile] = 0;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(tmem_cols<BN>()));
+}
+
+// ---- host side -------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encoder() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// Row-major bf16 matrix [rows, cols] with row stride ld (elements); box of
+// 64 columns x box_rows rows, 128-byte swizzle, zero fill out of bounds.
+bool make_map(CUtensorMap* map, const void* base, int rows, int cols, int ld, int box_rows) {
+  EncodeTiledFn enc = encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
+  cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BN, bool SWAP>
+cudaError_t prepare_one() {
+  return cudaFuncSetAttribute(gemm_tc_kernel<BN, SWAP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)smem_bytes<BN>());
+}
+
+template <int BN, bool SWAP>
+cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& mb, dim3 grid, int M, int N,
+                       int nkb, int ks, int xk_split, int xk_off, const Epi& e,
+                       const GemmScratch& scr, int* status, cudaStream_t s) {
+  gemm_tc_kernel<BN, SWAP><<<grid, 128, smem_bytes<BN>(), s>>>(
+      ma, mb, M, N, nkb, ks, xk_split, xk_off, e, scr.part, scr.counters, status);
+  note_launch();
+  return cudaGetLastError();
+}
+
+int swap_bn(int M) {
+  int bn = 32;
+  while (bn < M) bn <<= 1;
+  return bn;
+}
+
+}  // namespace
+
+cudaError_t gemm_tc_prepare() {
+  static bool done = false;
+  if (done) return cudaSuccess;
+  cudaError_t e;
+  if ((e = prepare_one<32, true>()) != cudaSuccess) return e;
+  if ((e = prepare_one<64, true>()) != cudaSuccess) return e;
+  if ((e = prepare_one<128, true>()) != cudaSuccess) return e;
+  if ((e = prepare_one<256, true>()) != cudaSuccess) return e;
+  if ((e = prepare_one<256, false>()) != cudaSuccess) return e;
+  done = true;
+  return cudaSuccess;
+}
+
+size_t gemm_scratch_bytes(int max_M, int max_N) { return PART_BUDGET; }
+int gemm_counter_count(int max_N) { return (max_N + BM - 1) / BM + 64; }
+
+int gemm_tc_supported(int dt, int M, int N, int K, int xk_split, int xk_off) {
+  if (dt != DT_BF16 || M < 1 || N < 1 || K < BK || (K % BK)) return 0;
+  if (encoder() == nullptr) return 0;
+  const int ftile = (M <= 256) ? BM : 256;
+  if (xk_split < N && (xk_split % ftile)) return 0;
+  if (xk_off % 8) return 0;
+  return 1;
+}
 
 cudaError_t launch_gemm_tc(int dt, const void* X, int ldx, const void* W, int ldw, int M, int N,
                            int K, int xk_split, int xk_off, const Epi& e,
                            const GemmScratch& scr, int* status, cudaStream_t s) {
-  return cudaErrorNotSupported;
+  cudaError_t err = gemm_tc_prepare();
+  if (err != cudaSuccess) return err;
+  const int nkb = K / BK;
+  const int xcols = (xk_split < N) ? xk_off + K : K;  // columns of X any tile reads
+  CUtensorMap ma, mb;
+  if (M <= 256) {
+    const int BN = swap_bn(M);
+    const int nt = (N + BM - 1) / BM;
+    if (!make_map(&ma, W, N, K, ldw, BM) || !make_map(&mb, X, M, xcols, ldx, BN))
+      return cudaErrorInvalidValue;
+    // K splits: aim for ~2 CTAs per SM, >= 2 K blocks per split, within budget
+    int ks = (2 * 148 + nt - 1) / nt;
+    if (ks > nkb / 2) ks = nkb / 2;
+    if (ks > 8) ks = 8;  // the last CTA of a tile sums the splits serially
+    if (ks < 1) ks = 1;
+    while (ks > 1 && ((size_t)nt * ks * BN * BM * 4 > scr.part_bytes || nt > scr.n_counters)) --ks;
+    dim3 grid(nt, 1, ks);
+    switch (BN) {
+      case 32: return launch_one<32, true>(ma, mb, grid, M, N, nkb, ks, xk_split, xk_off, e, scr, status, s);
+      case 64: return launch_one<64, true>(ma, mb, grid, M, N, nkb, ks, xk_split, xk_off, e, scr, status, s);
+      case 128: return launch_one<128, true>(ma, mb, grid, M, N, nkb, ks, xk_split, xk_off, e, scr, status, s);
+      default: return launch_one<256, true>(ma, mb, grid, M, N, nkb, ks, xk_split, xk_off, e, scr, status, s);
+    }
+  }
+  constexpr int BNP = 256;
+  if (!make_map(&ma, X, M, xcols, ldx, BM) || !make_map(&mb, W, N, K, ldw, BNP))
+    return cudaErrorInvalidValue;
+  dim3 grid((M + BM - 1) / BM, (N + BNP - 1) / BNP, 1);
+  return launch_one<BNP, false>(ma, mb, grid, M, N, nkb, 1, xk_split, xk_off, e, scr, status, s);
 }
 
 }  // namespace bt

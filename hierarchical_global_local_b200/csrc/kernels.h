@@ -105,6 +105,8 @@ int gemm_counter_count(int max_N);
 cudaError_t launch_gemm(int dt, const void* X, int ldx, const void* W, int ldw, int M, int N,
                         int K, int xk_split, int xk_off, const Epi& e, const GemmScratch& scr,
                         int* status, cudaStream_t s);
+// One-time setup of the tensor-core kernels (shared-memory limits).
+cudaError_t gemm_tc_prepare();
 // 0 = automatic, 1 = force the SIMT path, 2 = force the tensor-core path.
 void gemm_set_path(int path);
 int gemm_tc_supported(int dt, int M, int N, int K, int xk_split, int xk_off);

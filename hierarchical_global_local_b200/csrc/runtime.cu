@@ -313,6 +313,7 @@ int bt_create(const bt_config* cfg, const bt_weights* w, void* ws, size_t ws_byt
   BT_TRYC(cudaMemsetAsync(m->gs.counters, 0, (size_t)m->gs.n_counters * 4, st));
   BT_TRYC(cudaMemsetAsync(m->block_tok, 0, (size_t)d.Bmax * d.L * 4, st));
   BT_TRYC(cudaStreamCreateWithFlags(&m->cap_stream, cudaStreamNonBlocking));
+  if (d.dt == BT_BF16) BT_TRYC(gemm_tc_prepare());
 #undef BT_TRY
 #undef BT_TRYC
   *out = m;
