@@ -13,13 +13,15 @@
 // Two orientations:
 //   decode ("weights as A"): A = W [N, K] (128 output features per tile),
 //     B = X [M, K] (the M <= 256 tokens of the batch, padded to BN by TMA
-//     zero fill). K is split across CTAs so that every SM streams weights;
-//     each split writes an fp32 partial tile and the last CTA of a tile (an
-//     atomic counter, no waiting) sums the partials in split order and runs
-//     the epilogue, so results do not depend on CTA timing.
+//     zero fill). K is split across the ks CTAs of a thread-block cluster so
+//     that enough SMs stream weights; each CTA parks its fp32 partial tile in
+//     its own shared memory and the cluster reduce-scatters over distributed
+//     shared memory: rank q sums columns [q*BN/ks, (q+1)*BN/ks) of all ks
+//     partials in rank order (deterministic) and runs the epilogue on them.
 //   prefill ("activations as A"): A = X (128 tokens per tile), B = W (BN
 //     features per tile), one K split.
 // Every mbarrier wait is bounded; a wait that runs out sets a status bit.
+#include <cooperative_groups.h>
 #include <cuda.h>
 #include <stdio.h>
 
@@ -33,8 +35,7 @@ namespace {
 
 constexpr int BM = 128;  // MMA M (TMEM lanes)
 constexpr int BK = 64;   // K elements per stage = one 128-byte swizzle row
-constexpr int STAGES = 4;
-constexpr size_t PART_BUDGET = 64ull << 20;
+constexpr size_t PART_BUDGET = 256;  // split-K no longer needs global scratch
 
 // ---- tcgen05 / TMA wrappers --------------------------------------------------
 __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
@@ -104,9 +105,15 @@ __host__ __device__ constexpr int tmem_cols() {
   return BN < 32 ? 32 : BN;
 }
 
+// pipeline depth: ~192 KB of operands in flight per CTA
+template <int BN>
+__host__ __device__ constexpr int stages() {
+  return BN <= 64 ? 8 : (BN == 128 ? 6 : 4);
+}
+
 template <int BN>
 __host__ __device__ constexpr size_t smem_bytes() {
-  return (size_t)STAGES * (BM * BK * 2 + BN * BK * 2) + 1024;  // + alignment slack
+  return (size_t)stages<BN>() * (BM * BK * 2 + BN * BK * 2) + 1024;  // + alignment slack
 }
 
 // ---- the kernel ---------------------------------------------------------------
@@ -115,8 +122,8 @@ __host__ __device__ constexpr size_t smem_bytes() {
 template <int BN, bool SWAP>
 __global__ void __launch_bounds__(128, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
-               int M, int N, int nkb, int ks, int xk_split, int xk_off, Epi e,
-               float* __restrict__ part, int* __restrict__ counters, int* status) {
+               int M, int N, int nkb, int ks, int xk_split, int xk_off, Epi e, int* status) {
+  constexpr int STAGES = stages<BN>();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~(uintptr_t)1023);
@@ -124,7 +131,6 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
   bf16* sB = reinterpret_cast<bf16*>(smem + (size_t)STAGES * BM * BK * 2);
   __shared__ __align__(8) uint64_t full[STAGES], empty[STAGES], done;
   __shared__ uint32_t tmem_slot;
-  __shared__ int s_last;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // tile coordinates: rows of A (BM) and rows of B (BN)
@@ -190,8 +196,6 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
   tc_fence_after();
   const int r = warp * 32 + lane;  // TMEM lane = row of A
   const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
-  const int tile = blockIdx.x + gridDim.x * blockIdx.y;
-
   if (ks == 1) {
     for (int c0 = 0; c0 < BN; c0 += 16) {
       float v[16];
@@ -204,31 +208,34 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
       }
     }
   } else {
-    // partial tile [BN][BM] of this split (row index fastest: coalesced)
-    float* my = part + ((size_t)tile * ks + z) * BN * BM;
+    // Split K across the cluster (ks = cluster size along z, rank = z):
+    // park this CTA's partial tile [BN][BM] in its own (now idle) operand
+    // buffers, then reduce-scatter over distributed shared memory.
+    namespace cg = cooperative_groups;
+    cg::cluster_group cluster = cg::this_cluster();
+    float* red = reinterpret_cast<float*>(smem);
     for (int c0 = 0; c0 < BN; c0 += 16) {
       float v[16];
       tmem_ld16(trow + c0, v);
 #pragma unroll
-      for (int j = 0; j < 16; ++j) my[(size_t)(c0 + j) * BM + r] = v[j];
+      for (int j = 0; j < 16; ++j) red[(c0 + j) * BM + r] = v[j];
     }
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) s_last = (atomicAdd(&counters[tile], 1) == ks - 1);
-    __syncthreads();
-    if (s_last) {
-      __threadfence();
-      const float* tp = part + (size_t)tile * ks * BN * BM;
-      for (int c = 0; c < BN; ++c) {
-        const int m = SWAP ? (b0 + c) : (a0 + r);
-        const int n = SWAP ? (a0 + r) : (b0 + c);
-        if (m >= M || n >= N) continue;
-        float acc = 0.f;
-        for (int zz = 0; zz < ks; ++zz) acc += __ldcg(tp + ((size_t)zz * BN + c) * BM + r);
-        epi_apply<bf16>(e, m, n, acc);
-      }
-      if (threadIdx.x == 0) counters[tile] = 0;
+    cluster.sync();
+    const int cpr = BN / ks;  // columns reduced by this rank
+    const int cbeg = (int)cluster.block_rank() * cpr;
+    for (int c = cbeg; c < cbeg + cpr; ++c) {
+      float part[8];
+#pragma unroll
+      for (int p = 0; p < 8; ++p)
+        part[p] = (p < ks) ? cluster.map_shared_rank(red, p)[c * BM + r] : 0.f;
+      float acc = 0.f;
+#pragma unroll
+      for (int p = 0; p < 8; ++p) acc += part[p];   // rank order: deterministic
+      const int m = SWAP ? (b0 + c) : (a0 + r);
+      const int n = SWAP ? (a0 + r) : (b0 + c);
+      if (m < M && n < N) epi_apply<bf16>(e, m, n, acc);
     }
+    cluster.sync();  // no CTA leaves while another still reads its partial
   }
 
   tc_fence_before();
@@ -279,12 +286,24 @@ cudaError_t prepare_one() {
 
 template <int BN, bool SWAP>
 cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& mb, dim3 grid, int M, int N,
-                       int nkb, int ks, int xk_split, int xk_off, const Epi& e,
-                       const GemmScratch& scr, int* status, cudaStream_t s) {
-  gemm_tc_kernel<BN, SWAP><<<grid, 128, smem_bytes<BN>(), s>>>(
-      ma, mb, M, N, nkb, ks, xk_split, xk_off, e, scr.part, scr.counters, status);
+                       int nkb, int ks, int xk_split, int xk_off, const Epi& e, int* status,
+                       cudaStream_t s) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(128, 1, 1);
+  cfg.dynamicSmemBytes = smem_bytes<BN>();
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = ks;  // the K splits of one tile form a cluster
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t err = cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN, SWAP>, ma, mb, M, N, nkb, ks,
+                                       xk_split, xk_off, e, status);
   note_launch();
-  return cudaGetLastError();
+  return err;
 }
 
 int swap_bn(int M) {
@@ -333,25 +352,23 @@ cudaError_t launch_gemm_tc(int dt, const void* X, int ldx, const void* W, int ld
     const int nt = (N + BM - 1) / BM;
     if (!make_map(&ma, W, N, K, ldw, BM) || !make_map(&mb, X, M, xcols, ldx, BN))
       return cudaErrorInvalidValue;
-    // K splits: aim for ~2 CTAs per SM, >= 2 K blocks per split, within budget
-    int ks = (2 * 148 + nt - 1) / nt;
-    if (ks > nkb / 2) ks = nkb / 2;
-    if (ks > 8) ks = 8;  // the last CTA of a tile sums the splits serially
-    if (ks < 1) ks = 1;
-    while (ks > 1 && ((size_t)nt * ks * BN * BM * 4 > scr.part_bytes || nt > scr.n_counters)) --ks;
+    // K splits (a power of two <= 8, the portable cluster size): the fewest
+    // that put a CTA on every SM, each split keeping >= 1 K block.
+    int ks = 1;
+    while (ks < 8 && nt * ks < 148 && nkb / (ks * 2) >= 1) ks *= 2;
     dim3 grid(nt, 1, ks);
     switch (BN) {
-      case 32: return launch_one<32, true>(ma, mb, grid, M, N, nkb, ks, xk_split, xk_off, e, scr, status, s);
-      case 64: return launch_one<64, true>(ma, mb, grid, M, N, nkb, ks, xk_split, xk_off, e, scr, status, s);
-      case 128: return launch_one<128, true>(ma, mb, grid, M, N, nkb, ks, xk_split, xk_off, e, scr, status, s);
-      default: return launch_one<256, true>(ma, mb, grid, M, N, nkb, ks, xk_split, xk_off, e, scr, status, s);
+      case 32: return launch_one<32, true>(ma, mb, grid, M, N, nkb, ks, xk_split, xk_off, e, status, s);
+      case 64: return launch_one<64, true>(ma, mb, grid, M, N, nkb, ks, xk_split, xk_off, e, status, s);
+      case 128: return launch_one<128, true>(ma, mb, grid, M, N, nkb, ks, xk_split, xk_off, e, status, s);
+      default: return launch_one<256, true>(ma, mb, grid, M, N, nkb, ks, xk_split, xk_off, e, status, s);
     }
   }
   constexpr int BNP = 256;
   if (!make_map(&ma, X, M, xcols, ldx, BM) || !make_map(&mb, W, N, K, ldw, BNP))
     return cudaErrorInvalidValue;
   dim3 grid((M + BM - 1) / BM, (N + BNP - 1) / BNP, 1);
-  return launch_one<BNP, false>(ma, mb, grid, M, N, nkb, 1, xk_split, xk_off, e, scr, status, s);
+  return launch_one<BNP, false>(ma, mb, grid, M, N, nkb, 1, xk_split, xk_off, e, status, s);
 }
 
 }  // namespace bt
