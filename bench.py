@@ -179,9 +179,11 @@ def run_ours(args):
     times = []
     barrier()
     with ClockSampler(local) as clk:
+        torch.cuda.nvtx.range_push("timed")      # ncu --nvtx-include timed/
         for _ in range(args.steps):
             one_step(times)
         barrier()
+        torch.cuda.nvtx.range_pop()
     k1 = native.lib().bt_kernel_launches(model._h)
     model.sync()
     per_run = {r: 0.0 for r in RUNS}

@@ -120,24 +120,42 @@ cudaError_t launch_advance(int* dstate, int L_B, cudaStream_t s) {
 }
 
 // ---------------------------------------------------------------------------
-// LayerNorm: one warp per row, two-pass (mean, then centred variance) in fp32
+// LayerNorm: one CTA (128 threads) per row, the row held in registers;
+// two-pass statistics (mean, then centred variance) in fp32.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void row_stats(const float* __restrict__ x, int D, float& mu,
-                                          float& rstd, float eps) {
-  const int lane = threadIdx.x & 31;
+constexpr int LN_THREADS = 128;
+constexpr int LN_MAXV = 4;  // float4 per thread: D <= 2048
+
+__device__ __forceinline__ float ln_block_sum(float v, float* red) {
+  v = warp_sum(v);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  v = (red[0] + red[1]) + (red[2] + red[3]);
+  __syncthreads();
+  return v;
+}
+
+// Loads row x (D floats) into v[]; returns mean and 1/sqrt(var + eps).
+__device__ __forceinline__ void ln_row(const float* __restrict__ x, int D, float eps, float4* v,
+                                       float& mu, float& rstd, float* red) {
   float s = 0.f;
-  for (int i = lane * 4; i < D; i += 128) {
-    float4 v = *reinterpret_cast<const float4*>(x + i);
-    s += (v.x + v.y) + (v.z + v.w);
+#pragma unroll
+  for (int u = 0; u < LN_MAXV; ++u) {
+    const int i = (threadIdx.x + u * LN_THREADS) * 4;
+    v[u] = (i < D) ? *reinterpret_cast<const float4*>(x + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+    s += (v[u].x + v[u].y) + (v[u].z + v[u].w);
   }
-  mu = warp_sum(s) / (float)D;
+  mu = ln_block_sum(s, red) / (float)D;
   float q = 0.f;
-  for (int i = lane * 4; i < D; i += 128) {
-    float4 v = *reinterpret_cast<const float4*>(x + i);
-    float a = v.x - mu, b = v.y - mu, c = v.z - mu, d = v.w - mu;
-    q += (a * a + b * b) + (c * c + d * d);
+#pragma unroll
+  for (int u = 0; u < LN_MAXV; ++u) {
+    const int i = (threadIdx.x + u * LN_THREADS) * 4;
+    if (i < D) {
+      const float a = v[u].x - mu, b = v[u].y - mu, c = v[u].z - mu, d = v[u].w - mu;
+      q += (a * a + b * b) + (c * c + d * d);
+    }
   }
-  rstd = rsqrtf(warp_sum(q) / (float)D + eps);
+  rstd = rsqrtf(ln_block_sum(q, red) / (float)D + eps);
 }
 
 template <typename T>
@@ -156,44 +174,50 @@ __device__ __forceinline__ void store4<bf16>(bf16* out, int i, float a, float b,
 }
 
 template <typename T>
-__global__ void ln_dual_kernel(const float* __restrict__ h, int M, int D,
-                               const float* __restrict__ g1, const float* __restrict__ b1,
-                               const float* __restrict__ g2, const float* __restrict__ b2,
-                               float eps, T* __restrict__ x1) {
-  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (row >= M) return;
-  const int lane = threadIdx.x & 31;
-  const float* x = h + (size_t)row * D;
+__device__ __forceinline__ void ln_store(T* o, const float4& v, int i, float mu, float rstd,
+                                         const float* __restrict__ g, const float* __restrict__ b) {
+  const float4 ga = *reinterpret_cast<const float4*>(g + i);
+  const float4 ba = *reinterpret_cast<const float4*>(b + i);
+  store4<T>(o, i, (v.x - mu) * rstd * ga.x + ba.x, (v.y - mu) * rstd * ga.y + ba.y,
+            (v.z - mu) * rstd * ga.z + ba.z, (v.w - mu) * rstd * ga.w + ba.w);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(LN_THREADS)
+ln_dual_kernel(const float* __restrict__ h, int D, const float* __restrict__ g1,
+               const float* __restrict__ b1, const float* __restrict__ g2,
+               const float* __restrict__ b2, float eps, T* __restrict__ x1) {
+  __shared__ float red[4];
+  const int row = blockIdx.x;
+  float4 v[LN_MAXV];
   float mu, rstd;
-  row_stats(x, D, mu, rstd, eps);
+  ln_row(h + (size_t)row * D, D, eps, v, mu, rstd, red);
   T* o = x1 + (size_t)row * 2 * D;
-  for (int i = lane * 4; i < D; i += 128) {
-    float4 v = *reinterpret_cast<const float4*>(x + i);
-    float n0 = (v.x - mu) * rstd, n1 = (v.y - mu) * rstd, n2 = (v.z - mu) * rstd,
-          n3 = (v.w - mu) * rstd;
-    float4 ga = *reinterpret_cast<const float4*>(g1 + i), ba = *reinterpret_cast<const float4*>(b1 + i);
-    float4 gb = *reinterpret_cast<const float4*>(g2 + i), bb = *reinterpret_cast<const float4*>(b2 + i);
-    store4<T>(o, i, n0 * ga.x + ba.x, n1 * ga.y + ba.y, n2 * ga.z + ba.z, n3 * ga.w + ba.w);
-    store4<T>(o + D, i, n0 * gb.x + bb.x, n1 * gb.y + bb.y, n2 * gb.z + bb.z, n3 * gb.w + bb.w);
+#pragma unroll
+  for (int u = 0; u < LN_MAXV; ++u) {
+    const int i = (threadIdx.x + u * LN_THREADS) * 4;
+    if (i < D) {
+      ln_store<T>(o, v[u], i, mu, rstd, g1, b1);
+      ln_store<T>(o + D, v[u], i, mu, rstd, g2, b2);
+    }
   }
 }
 
 template <typename T>
-__global__ void ln_rows_kernel(const float* __restrict__ h, int R, int row_step, int row_off,
-                               int D, const float* __restrict__ g, const float* __restrict__ b,
-                               float eps, T* __restrict__ out) {
-  const int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (r >= R) return;
-  const int lane = threadIdx.x & 31;
-  const float* x = h + ((size_t)r * row_step + row_off) * D;
+__global__ void __launch_bounds__(LN_THREADS)
+ln_rows_kernel(const float* __restrict__ h, int row_step, int row_off, int D,
+               const float* __restrict__ g, const float* __restrict__ b, float eps,
+               T* __restrict__ out) {
+  __shared__ float red[4];
+  const int r = blockIdx.x;
+  float4 v[LN_MAXV];
   float mu, rstd;
-  row_stats(x, D, mu, rstd, eps);
+  ln_row(h + ((size_t)r * row_step + row_off) * D, D, eps, v, mu, rstd, red);
   T* o = out + (size_t)r * D;
-  for (int i = lane * 4; i < D; i += 128) {
-    float4 v = *reinterpret_cast<const float4*>(x + i);
-    float4 ga = *reinterpret_cast<const float4*>(g + i), ba = *reinterpret_cast<const float4*>(b + i);
-    store4<T>(o, i, (v.x - mu) * rstd * ga.x + ba.x, (v.y - mu) * rstd * ga.y + ba.y,
-              (v.z - mu) * rstd * ga.z + ba.z, (v.w - mu) * rstd * ga.w + ba.w);
+#pragma unroll
+  for (int u = 0; u < LN_MAXV; ++u) {
+    const int i = (threadIdx.x + u * LN_THREADS) * 4;
+    if (i < D) ln_store<T>(o, v[u], i, mu, rstd, g, b);
   }
 }
 
@@ -201,27 +225,24 @@ cudaError_t launch_ln_dual(int dt, const float* h, int M, int D, const float* g1
                            const float* b1, const float* g2, const float* b2, float eps,
                            void* x1, cudaStream_t s) {
   if (M == 0) return cudaSuccess;
-  const int rows_per_cta = 8;
-  dim3 grid((M + rows_per_cta - 1) / rows_per_cta);
-  if (dt == DT_BF16) {
-    ln_dual_kernel<bf16><<<grid, 256, 0, s>>>(h, M, D, g1, b1, g2, b2, eps, (bf16*)x1); note_launch();
-  }
-  else {
-    ln_dual_kernel<float><<<grid, 256, 0, s>>>(h, M, D, g1, b1, g2, b2, eps, (float*)x1); note_launch();
-  }
+  if (D > LN_THREADS * 4 * LN_MAXV || (D % 4)) return cudaErrorInvalidValue;
+  if (dt == DT_BF16)
+    ln_dual_kernel<bf16><<<M, LN_THREADS, 0, s>>>(h, D, g1, b1, g2, b2, eps, (bf16*)x1);
+  else
+    ln_dual_kernel<float><<<M, LN_THREADS, 0, s>>>(h, D, g1, b1, g2, b2, eps, (float*)x1);
+  note_launch();
   return cudaGetLastError();
 }
 
 cudaError_t launch_ln_rows(int dt, const float* h, int R, int row_step, int row_off, int D,
                            const float* g, const float* b, float eps, void* out, cudaStream_t s) {
   if (R == 0) return cudaSuccess;
-  dim3 grid((R + 7) / 8);
-  if (dt == DT_BF16) {
-    ln_rows_kernel<bf16><<<grid, 256, 0, s>>>(h, R, row_step, row_off, D, g, b, eps, (bf16*)out); note_launch();
-  }
-  else {
-    ln_rows_kernel<float><<<grid, 256, 0, s>>>(h, R, row_step, row_off, D, g, b, eps, (float*)out); note_launch();
-  }
+  if (D > LN_THREADS * 4 * LN_MAXV || (D % 4)) return cudaErrorInvalidValue;
+  if (dt == DT_BF16)
+    ln_rows_kernel<bf16><<<R, LN_THREADS, 0, s>>>(h, row_step, row_off, D, g, b, eps, (bf16*)out);
+  else
+    ln_rows_kernel<float><<<R, LN_THREADS, 0, s>>>(h, row_step, row_off, D, g, b, eps, (float*)out);
+  note_launch();
   return cudaGetLastError();
 }
 

@@ -34,4 +34,35 @@ __device__ __forceinline__ void epi_apply(const Epi& e, int m, int n, float acc)
   }
 }
 
+// EPI_QKV1_ROPE for one element; `partner` is the value of feature n ^ (rot/2)
+// (its rotate-half pair) of the same token, fetched by the caller.
+template <typename T>
+__device__ __forceinline__ void epi_apply_rope(const Epi& e, int m, int n, float acc,
+                                               float partner) {
+  const float v = acc + e.bias[n];
+  const int D = e.D;
+  if (n >= 3 * D) {
+    reinterpret_cast<T*>(e.out1)[(size_t)m * e.ld1 + D + (n - 3 * D)] = from_f<T>(gelu_erf(v));
+    return;
+  }
+  const int part = n / D, c = n - part * D;
+  const int d = D / e.H;
+  const int hh = c / d, dim = c - hh * d;
+  const int b = m / e.pos.rows_per_seq;
+  const int pos = pos_base(e.pos) + (m - b * e.pos.rows_per_seq);
+  float out = v;
+  if (part < 2 && dim < e.rot) {
+    const int half = e.rot >> 1;
+    const float pv = partner + e.bias[n ^ half];
+    const float2 cs = e.rope_tab[(size_t)pos * half + (dim & (half - 1))];
+    out = (dim < half) ? v * cs.x - pv * cs.y : v * cs.x + pv * cs.y;
+  }
+  if (part == 0) {
+    reinterpret_cast<T*>(e.out0)[(size_t)m * e.ld0 + c] = from_f<T>(out);
+  } else {
+    T* cache = reinterpret_cast<T*>(part == 1 ? e.kc : e.vc);
+    cache[(((size_t)b * e.H + hh) * e.cap + pos) * d + dim] = from_f<T>(out);
+  }
+}
+
 }  // namespace bt

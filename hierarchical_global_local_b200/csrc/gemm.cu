@@ -69,6 +69,8 @@ cudaError_t launch_gemm(int dt, const void* X, int ldx, const void* W, int ldw, 
                         int K, int xk_split, int xk_off, const Epi& e, const GemmScratch& scr,
                         int* status, cudaStream_t s) {
   if (M == 0 || N == 0) return cudaSuccess;
+  if (e.kind == EPI_QKV1_ROPE && (g_gemm_path == 1 || !gemm_rope_fusable(dt, M, N, K, xk_split, xk_off, e.D / e.H, e.rot)))
+    return cudaErrorNotSupported;  // the caller runs EPI_QKV1 + the rotary kernel instead
   const bool tc_ok = gemm_tc_supported(dt, M, N, K, xk_split, xk_off) != 0;
   if (g_gemm_path != 1 && tc_ok)
     return launch_gemm_tc(dt, X, ldx, W, ldw, M, N, K, xk_split, xk_off, e, scr, status, s);

@@ -196,6 +196,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
   tc_fence_after();
   const int r = warp * 32 + lane;  // TMEM lane = row of A
   const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+  // fused rotary: the rotate-half partner of feature f is f ^ (rot/2), held
+  // by lane ^ (rot/2) of the same warp (heads are 32-feature aligned)
+  const bool rope = SWAP && e.kind == EPI_QKV1_ROPE;
+  const int rhalf = e.rot >> 1;
   if (ks == 1) {
     for (int c0 = 0; c0 < BN; c0 += 16) {
       float v[16];
@@ -204,7 +208,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
       for (int j = 0; j < 16; ++j) {
         const int m = SWAP ? (b0 + c0 + j) : (a0 + r);
         const int n = SWAP ? (a0 + r) : (b0 + c0 + j);
-        if (m < M && n < N) epi_apply<bf16>(e, m, n, v[j]);
+        if (rope) {
+          const float pv = __shfl_xor_sync(0xffffffffu, v[j], rhalf);
+          if (m < M && n < N) epi_apply_rope<bf16>(e, m, n, v[j], pv);
+        } else if (m < M && n < N) {
+          epi_apply<bf16>(e, m, n, v[j]);
+        }
       }
     }
   } else {
@@ -233,7 +242,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
       for (int p = 0; p < 8; ++p) acc += part[p];   // rank order: deterministic
       const int m = SWAP ? (b0 + c) : (a0 + r);
       const int n = SWAP ? (a0 + r) : (b0 + c);
-      if (m < M && n < N) epi_apply<bf16>(e, m, n, acc);
+      if (rope) {
+        const float pv = __shfl_xor_sync(0xffffffffu, acc, rhalf);
+        if (m < M && n < N) epi_apply_rope<bf16>(e, m, n, acc, pv);
+      } else if (m < M && n < N) {
+        epi_apply<bf16>(e, m, n, acc);
+      }
     }
     cluster.sync();  // no CTA leaves while another still reads its partial
   }
@@ -329,6 +343,15 @@ cudaError_t gemm_tc_prepare() {
 
 size_t gemm_scratch_bytes(int max_M, int max_N) { return PART_BUDGET; }
 int gemm_counter_count(int max_N) { return (max_N + BM - 1) / BM + 64; }
+
+int gemm_rope_fusable(int dt, int M, int N, int K, int xk_split, int xk_off, int d_head, int rot) {
+  if (!gemm_tc_supported(dt, M, N, K, xk_split, xk_off) || M > 256) return 0;
+  const int half = rot / 2;
+  // partner lane = lane ^ half inside a warp: half a power of two <= 16,
+  // heads at least one warp (32 features) wide
+  if (d_head < 32 || half < 1 || half > 16 || (half & (half - 1))) return 0;
+  return 1;
+}
 
 int gemm_tc_supported(int dt, int M, int N, int K, int xk_split, int xk_off) {
   if (dt != DT_BF16 || M < 1 || N < 1 || K < BK || (K % BK)) return 0;

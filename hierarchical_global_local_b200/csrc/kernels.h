@@ -78,6 +78,10 @@ enum EpiKind : int {
   EPI_RESID = 1,  // out0 (fp32) [m, n] += acc + bias[n]
   EPI_F32 = 2,    // out0 (fp32) [m, n] = acc (+ bias[n] if bias)
   EPI_ACT = 3,    // out0 (act)  [m, n] = acc (+ bias[n] if bias)
+  EPI_QKV1_ROPE = 4,  // as EPI_QKV1, with rotary + KV-cache append fused:
+                      // q (rotated) -> out0 [m, n]; k (rotated), v -> the
+                      // caches at the token's position (tensor-core decode
+                      // orientation only, see gemm_rope_fusable)
 };
 
 struct Epi {
@@ -89,7 +93,17 @@ struct Epi {
   const float* bias;
   int split_n;
   int D;
+  // EPI_QKV1_ROPE only
+  const float2* rope_tab;
+  int rot;
+  int H;
+  void* kc;
+  void* vc;
+  int cap;
+  PosSpec pos;
 };
+// True when launch_gemm will run EPI_QKV1_ROPE fused for this shape.
+int gemm_rope_fusable(int dt, int M, int N, int K, int xk_split, int xk_off, int d_head, int rot);
 
 // out = X [M, K] (row stride ldx) . W [N, K]^T (row stride ldw), fp32
 // accumulation; for output columns n >= xk_split the X columns read are

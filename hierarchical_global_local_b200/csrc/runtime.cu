@@ -135,7 +135,15 @@ struct bt_model {
   bool capturing = false;
   std::vector<cudaEvent_t> ev;
   std::vector<bt_profile_record> rec;
+  std::vector<int> rec_direct;  // per record: event-pair index (direct launch) or -1
+  int n_direct = 0;
   int cap_records = 0;
+  // profiled decode graphs: event-record nodes around every kernel
+  struct Pair { bt_profile_record r; cudaEvent_t a, b; };
+  cudaGraphExec_t pgraphs[2][2] = {{nullptr, nullptr}, {nullptr, nullptr}};
+  long long pgraph_kernels[2][2] = {{0, 0}, {0, 0}};
+  std::vector<Pair> pairs[2][2];
+  std::vector<Pair>* cap_pairs = nullptr;  // list being captured into
 };
 
 // Event pair around one kernel launch while the profiler is on.
@@ -143,14 +151,28 @@ struct ProfScope {
   bt_model* m;
   cudaStream_t s;
   int idx = -1;
+  cudaEvent_t end = nullptr;
   ProfScope(bt_model* m_, cudaStream_t s_, int kind, int M, int N, int K) : m(m_), s(s_) {
-    if (!m->prof || m->capturing || (int)m->rec.size() >= m->cap_records) return;
-    idx = (int)m->rec.size();
+    if (!m->prof) return;
+    if (m->capturing) {
+      // inside a profiled graph: the pair becomes two event-record nodes
+      if (!m->cap_pairs) return;
+      bt_model::Pair p{bt_profile_record{kind, M, N, K, 0.f}, nullptr, nullptr};
+      if (cudaEventCreate(&p.a) != cudaSuccess || cudaEventCreate(&p.b) != cudaSuccess) return;
+      cudaEventRecord(p.a, s);
+      end = p.b;
+      m->cap_pairs->push_back(p);
+      return;
+    }
+    if ((int)m->rec.size() >= m->cap_records || 2 * (m->n_direct + 1) > (int)m->ev.size()) return;
+    idx = m->n_direct++;
     m->rec.push_back(bt_profile_record{kind, M, N, K, 0.f});
+    m->rec_direct.push_back(idx);
     cudaEventRecord(m->ev[2 * idx], s);
   }
   ~ProfScope() {
-    if (idx >= 0) cudaEventRecord(m->ev[2 * idx + 1], s);
+    if (end) cudaEventRecord(end, s);
+    else if (idx >= 0) cudaEventRecord(m->ev[2 * idx + 1], s);
   }
 };
 
@@ -335,12 +357,18 @@ static int run_layer(bt_model* m, const LayerW& w, float* h, int M, PosSpec pos,
     ProfScope p(m, s, BT_K_LAYERNORM, M, D, 0);
     BT_CUDA(launch_ln_dual(d.dt, h, M, D, w.ln1_g, w.ln1_b, w.ln2_g, w.ln2_b, m->cfg.ln_eps, m->x1, s));
   }
-  {
+  if (gemm_rope_fusable(d.dt, M, 7 * D, D, 3 * D, D, d.d, d.rot)) {
+    // q|k|v|fc1 GEMM with rotary and the KV-cache append in its epilogue
     ProfScope p(m, s, BT_K_GEMM, M, 7 * D, D);
-    Epi e1{EPI_QKV1, m->qkv, 3 * D, m->a2, 5 * D, w.b_qkv1, 3 * D, D};
+    Epi e1{EPI_QKV1_ROPE, m->qrot, D, m->a2, 5 * D, w.b_qkv1, 3 * D, D,
+           m->rope_tab, d.rot, d.H, kc, vc, cap, pos};
     BT_CUDA(launch_gemm(d.dt, m->x1, 2 * D, w.w_qkv1, D, M, 7 * D, D, 3 * D, D, e1, m->gs, m->status, s));
-  }
-  {
+  } else {
+    {
+      ProfScope p(m, s, BT_K_GEMM, M, 7 * D, D);
+      Epi e1{EPI_QKV1, m->qkv, 3 * D, m->a2, 5 * D, w.b_qkv1, 3 * D, D};
+      BT_CUDA(launch_gemm(d.dt, m->x1, 2 * D, w.w_qkv1, D, M, 7 * D, D, 3 * D, D, e1, m->gs, m->status, s));
+    }
     ProfScope p(m, s, BT_K_ROPE_APPEND, M, 3 * D, 0);
     BT_CUDA(launch_rope_append(d.dt, m->qkv, M, D, d.H, d.rot, m->rope_tab, pos, m->qrot, kc, vc, cap, s));
   }
@@ -514,9 +542,10 @@ int bt_decode_step(bt_model* m, const int32_t* tokens, float* logits, int32_t* n
   const bool greedy = tokens == nullptr;
   if (!greedy)
     BT_CUDA(cudaMemcpyAsync(m->fed, tokens, (size_t)m->B * 4, cudaMemcpyDeviceToDevice, m->stream));
-  if (m->use_graphs && !m->prof) {
-    cudaGraphExec_t& g = m->graphs[block_step ? 1 : 0][greedy ? 1 : 0];
-    long long& gk = m->graph_kernels[block_step ? 1 : 0][greedy ? 1 : 0];
+  if (m->use_graphs) {
+    const int bi = block_step ? 1 : 0, gi = greedy ? 1 : 0;
+    cudaGraphExec_t& g = m->prof ? m->pgraphs[bi][gi] : m->graphs[bi][gi];
+    long long& gk = m->prof ? m->pgraph_kernels[bi][gi] : m->graph_kernels[bi][gi];
     if (!g) {
       // capture on the private stream, ordered after the caller's stream
       cudaEvent_t ev;
@@ -529,8 +558,10 @@ int bt_decode_step(bt_model* m, const int32_t* tokens, float* logits, int32_t* n
       BT_CUDA(cudaStreamBeginCapture(m->cap_stream, cudaStreamCaptureModeThreadLocal));
       const long long c0 = launch_count();
       m->capturing = true;
+      m->cap_pairs = m->prof ? &m->pairs[bi][gi] : nullptr;
       int rc = enqueue_decode(m, block_step, greedy, m->cap_stream);
       m->capturing = false;
+      m->cap_pairs = nullptr;
       gk = launch_count() - c0;
       cudaError_t ce = cudaStreamEndCapture(m->cap_stream, &graph);
       if (rc != BT_OK) return rc;
@@ -540,6 +571,18 @@ int bt_decode_step(bt_model* m, const int32_t* tokens, float* logits, int32_t* n
     }
     BT_CUDA(cudaGraphLaunch(g, m->stream));
     m->kernels += gk;
+    if (m->prof) {
+      // read this replay's event pairs
+      BT_CUDA(cudaStreamSynchronize(m->stream));
+      for (auto& p : m->pairs[bi][gi]) {
+        if ((int)m->rec.size() >= m->cap_records) break;
+        bt_profile_record r = p.r;
+        if (r.kind == BT_K_ATTN_DECODE) r.n = m->t / d.L + 1;
+        BT_CUDA(cudaEventElapsedTime(&r.ms, p.a, p.b));
+        m->rec.push_back(r);
+        m->rec_direct.push_back(-1);
+      }
+    }
   } else {
     const long long c0 = launch_count();
     int rc = enqueue_decode(m, block_step, greedy, m->stream);
@@ -576,12 +619,25 @@ static void free_events(bt_model* m) {
   m->ev.clear();
 }
 
+static void drop_pgraphs(bt_model* m) {
+  for (int i = 0; i < 2; ++i)
+    for (int j = 0; j < 2; ++j) {
+      if (m->pgraphs[i][j]) { cudaGraphExecDestroy(m->pgraphs[i][j]); m->pgraphs[i][j] = nullptr; }
+      for (auto& p : m->pairs[i][j]) { cudaEventDestroy(p.a); cudaEventDestroy(p.b); }
+      m->pairs[i][j].clear();
+    }
+}
+
 int bt_profile_begin(bt_model* m, int32_t capacity) {
   if (!m || capacity <= 0) return BT_EINVAL;
   free_events(m);
+  drop_pgraphs(m);
   m->rec.clear();
+  m->rec_direct.clear();
+  m->n_direct = 0;
   m->rec.reserve(capacity);
-  m->ev.resize(2 * (size_t)capacity);
+  // event pairs for direct launches (prefill); decode graphs carry their own
+  m->ev.resize(2 * (size_t)(capacity < 8192 ? capacity : 8192));
   for (auto& e : m->ev) BT_CUDA(cudaEventCreate(&e));
   m->cap_records = capacity;
   m->prof = true;
@@ -594,13 +650,16 @@ int bt_profile_end(bt_model* m, bt_profile_record* out, int32_t capacity, int32_
   BT_CUDA(cudaStreamSynchronize(m->stream));
   const int n = (int)m->rec.size() < capacity ? (int)m->rec.size() : capacity;
   for (int i = 0; i < n; ++i) {
-    float ms = 0.f;
-    BT_CUDA(cudaEventElapsedTime(&ms, m->ev[2 * i], m->ev[2 * i + 1]));
-    m->rec[i].ms = ms;
+    if (m->rec_direct[i] >= 0) {
+      float ms = 0.f;
+      BT_CUDA(cudaEventElapsedTime(&ms, m->ev[2 * m->rec_direct[i]], m->ev[2 * m->rec_direct[i] + 1]));
+      m->rec[i].ms = ms;
+    }
     if (out) out[i] = m->rec[i];
   }
   if (n_out) *n_out = n;
   free_events(m);
+  drop_pgraphs(m);
   return BT_OK;
 }
 
@@ -608,6 +667,7 @@ int bt_destroy(bt_model* m) {
   if (!m) return BT_EINVAL;
   cudaStreamSynchronize(m->stream);
   free_events(m);
+  drop_pgraphs(m);
   drop_graphs(m);
   if (m->cap_stream) cudaStreamDestroy(m->cap_stream);
   delete m;
