@@ -159,7 +159,8 @@ struct ProfScope {
       if (!m->cap_pairs) return;
       bt_model::Pair p{bt_profile_record{kind, M, N, K, 0.f}, nullptr, nullptr};
       if (cudaEventCreate(&p.a) != cudaSuccess || cudaEventCreate(&p.b) != cudaSuccess) return;
-      cudaEventRecord(p.a, s);
+      // external record nodes: real timestamps on every replay
+      cudaEventRecordWithFlags(p.a, s, cudaEventRecordExternal);
       end = p.b;
       m->cap_pairs->push_back(p);
       return;
@@ -171,7 +172,7 @@ struct ProfScope {
     cudaEventRecord(m->ev[2 * idx], s);
   }
   ~ProfScope() {
-    if (end) cudaEventRecord(end, s);
+    if (end) cudaEventRecordWithFlags(end, s, cudaEventRecordExternal);
     else if (idx >= 0) cudaEventRecord(m->ev[2 * idx + 1], s);
   }
 };
