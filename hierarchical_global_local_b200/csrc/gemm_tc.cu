@@ -35,7 +35,7 @@ namespace {
 
 constexpr int BM = 128;  // MMA M (TMEM lanes)
 constexpr int BK = 64;   // K elements per stage = one 128-byte swizzle row
-constexpr size_t PART_BUDGET = 256;  // split-K no longer needs global scratch
+constexpr size_t PART_BUDGET = 256;  // split-K reduces in distributed shared memory
 
 // ---- tcgen05 / TMA wrappers --------------------------------------------------
 __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
@@ -100,55 +100,58 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
+constexpr int MAX_STAGES = 8;
+constexpr int THREADS = 192;  // warps 0-3 epilogue, warp 4 TMA producer, warp 5 MMA issuer
+
+template <int BN>
+__host__ __device__ constexpr size_t stage_bytes() {
+  return (size_t)(BM * BK * 2 + BN * BK * 2);
+}
+
+// TMEM columns: two fp32 accumulators of BN columns (double buffer)
 template <int BN>
 __host__ __device__ constexpr int tmem_cols() {
-  return BN < 32 ? 32 : BN;
-}
-
-// pipeline depth: ~192 KB of operands in flight per CTA
-template <int BN>
-__host__ __device__ constexpr int stages() {
-  return BN <= 64 ? 8 : (BN == 128 ? 6 : 4);
-}
-
-template <int BN>
-__host__ __device__ constexpr size_t smem_bytes() {
-  return (size_t)stages<BN>() * (BM * BK * 2 + BN * BK * 2) + 1024;  // + alignment slack
+  return 2 * BN < 32 ? 32 : 2 * BN;
 }
 
 // ---- the kernel ---------------------------------------------------------------
 // SWAP = true: A = weights (rows = output features), B = activations (rows =
 // tokens). SWAP = false: A = activations, B = weights.
+// ks == 1: persistent; CTA c handles tiles c, c + gridDim.x, ... with a
+//   continuous TMA ring across tiles and two TMEM accumulators, so the
+//   epilogue of one tile overlaps the loads and MMAs of the next.
+// ks > 1: one tile per CTA, K split over the cluster's ks CTAs, partial
+//   tiles reduce-scattered over distributed shared memory.
 template <int BN, bool SWAP>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(THREADS, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
-               int M, int N, int nkb, int ks, int xk_split, int xk_off, Epi e, int* status) {
-  constexpr int STAGES = stages<BN>();
+               int M, int N, int nkb, int ks, int stages, int ntA, int ntB, int xk_split,
+               int xk_off, Epi e, int* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~(uintptr_t)1023);
   bf16* sA = reinterpret_cast<bf16*>(smem);
-  bf16* sB = reinterpret_cast<bf16*>(smem + (size_t)STAGES * BM * BK * 2);
-  __shared__ __align__(8) uint64_t full[STAGES], empty[STAGES], done;
+  bf16* sB = reinterpret_cast<bf16*>(smem + (size_t)stages * BM * BK * 2);
+  __shared__ __align__(8) uint64_t full[MAX_STAGES], empty[MAX_STAGES], acc_full[2], acc_empty[2];
   __shared__ uint32_t tmem_slot;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // tile coordinates: rows of A (BM) and rows of B (BN)
-  const int a0 = blockIdx.x * BM;
-  const int b0 = blockIdx.y * BN;
+  const int ntiles = ntA * ntB;
+  const int t_first = blockIdx.x;
+  const int t_step = (ks == 1) ? gridDim.x : ntiles;  // split mode: exactly one tile
   const int z = blockIdx.z;
-  const int feat0 = SWAP ? a0 : b0;
-  const int koff = (feat0 >= xk_split) ? xk_off : 0;
   const int kb_begin = (int)(((long long)z * nkb) / ks);
   const int kb_end = (int)(((long long)(z + 1) * nkb) / ks);
-  const int nloc = kb_end - kb_begin;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < STAGES; ++i) {
+    for (int i = 0; i < stages; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
     }
-    mbar_init(&done, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 128);
+    }
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -162,91 +165,143 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
 
-  if (warp == 0 && lane == 0) {
-    // ---- producer: TMA loads ----
-    const uint32_t bytes = (uint32_t)(BM * BK * 2 + BN * BK * 2);
-    for (int i = 0; i < nloc; ++i) {
-      const int s = i % STAGES;
-      if (i >= STAGES) mbar_wait_bounded(&empty[s], ((i / STAGES) + 1) & 1, status);
-      mbar_arrive_expect_tx(&full[s], bytes);
-      const int k = (kb_begin + i) * BK;
-      tma_load_2d(sA + (size_t)s * BM * BK, &mapA, k + (SWAP ? 0 : koff), a0, &full[s]);
-      tma_load_2d(sB + (size_t)s * BN * BK, &mapB, k + (SWAP ? koff : 0), b0, &full[s]);
-    }
-  } else if (warp == 1 && lane == 0) {
-    // ---- MMA issuer ----
-    constexpr uint32_t idesc = instr_desc<BN>();
-    for (int i = 0; i < nloc; ++i) {
-      const int s = i % STAGES;
-      mbar_wait_bounded(&full[s], (i / STAGES) & 1, status);
-      tc_fence_after();
-      const uint64_t da = smem_desc_sw128(smem_u32(sA + (size_t)s * BM * BK));
-      const uint64_t db = smem_desc_sw128(smem_u32(sB + (size_t)s * BN * BK));
-#pragma unroll
-      for (int kk = 0; kk < BK / 16; ++kk)  // 32 bytes per K slice: +2 in 16-byte units
-        mma_bf16(tmem, da + 2 * kk, db + 2 * kk, idesc, (i > 0 || kk > 0) ? 1u : 0u);
-      mma_commit(&empty[s]);
-    }
-    mma_commit(&done);
-  }
-  __syncwarp();
-
-  // ---- epilogue ----
-  mbar_wait_bounded(&done, 0, status);
-  tc_fence_after();
-  const int r = warp * 32 + lane;  // TMEM lane = row of A
-  const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
-  // fused rotary: the rotate-half partner of feature f is f ^ (rot/2), held
-  // by lane ^ (rot/2) of the same warp (heads are 32-feature aligned)
-  const bool rope = SWAP && e.kind == EPI_QKV1_ROPE;
-  const int rhalf = e.rot >> 1;
-  if (ks == 1) {
-    for (int c0 = 0; c0 < BN; c0 += 16) {
-      float v[16];
-      tmem_ld16(trow + c0, v);
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const int m = SWAP ? (b0 + c0 + j) : (a0 + r);
-        const int n = SWAP ? (a0 + r) : (b0 + c0 + j);
-        if (rope) {
-          const float pv = __shfl_xor_sync(0xffffffffu, v[j], rhalf);
-          if (m < M && n < N) epi_apply_rope<bf16>(e, m, n, v[j], pv);
-        } else if (m < M && n < N) {
-          epi_apply<bf16>(e, m, n, v[j]);
+  if (warp == 4) {
+    // ---- TMA producer ----
+    if (lane == 0) {
+      const uint32_t bytes = (uint32_t)stage_bytes<BN>();
+      int it = 0;
+      for (int t = t_first; t < ntiles; t += t_step) {
+        const int a0 = (t % ntA) * BM, b0 = (t / ntA) * BN;
+        const int koff = ((SWAP ? a0 : b0) >= xk_split) ? xk_off : 0;
+        for (int kb = kb_begin; kb < kb_end; ++kb, ++it) {
+          const int s = it % stages;
+          if (it >= stages) mbar_wait_bounded(&empty[s], ((it / stages) + 1) & 1, status);
+          mbar_arrive_expect_tx(&full[s], bytes);
+          const int k = kb * BK;
+          tma_load_2d(sA + (size_t)s * BM * BK, &mapA, k + (SWAP ? 0 : koff), a0, &full[s]);
+          tma_load_2d(sB + (size_t)s * BN * BK, &mapB, k + (SWAP ? koff : 0), b0, &full[s]);
         }
       }
     }
+  } else if (warp == 5) {
+    // ---- MMA issuer ----
+    if (lane == 0) {
+      constexpr uint32_t idesc = instr_desc<BN>();
+      int it = 0, tl = 0;
+      for (int t = t_first; t < ntiles; t += t_step, ++tl) {
+        const int buf = tl & 1;
+        if (tl >= 2) mbar_wait_bounded(&acc_empty[buf], ((tl >> 1) + 1) & 1, status);
+        tc_fence_after();
+        const uint32_t dt = tmem + (uint32_t)(buf * BN);
+        for (int kb = kb_begin; kb < kb_end; ++kb, ++it) {
+          const int s = it % stages;
+          mbar_wait_bounded(&full[s], (it / stages) & 1, status);
+          tc_fence_after();
+          const uint64_t da = smem_desc_sw128(smem_u32(sA + (size_t)s * BM * BK));
+          const uint64_t db = smem_desc_sw128(smem_u32(sB + (size_t)s * BN * BK));
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)  // 32 bytes per K slice: +2 in 16-byte units
+            mma_bf16(dt, da + 2 * kk, db + 2 * kk, idesc, (kb > kb_begin || kk > 0) ? 1u : 0u);
+          mma_commit(&empty[s]);
+        }
+        mma_commit(&acc_full[buf]);
+      }
+    }
   } else {
-    // Split K across the cluster (ks = cluster size along z, rank = z):
-    // park this CTA's partial tile [BN][BM] in its own (now idle) operand
-    // buffers, then reduce-scatter over distributed shared memory.
+    // ---- epilogue warps 0-3: TMEM lanes 32w..32w+31 ----
+    const int r = warp * 32 + lane;  // row of A = TMEM lane
+    const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+    // fused rotary: the rotate-half partner of feature f is f ^ (rot/2), held
+    // by lane ^ (rot/2) of the same warp (heads are 32-feature aligned)
+    const bool rope = SWAP && e.kind == EPI_QKV1_ROPE;
+    const int rhalf = e.rot >> 1;
+    int tl = 0;
+    for (int t = t_first; t < ntiles; t += t_step, ++tl) {
+      const int buf = tl & 1;
+      const int a0 = (t % ntA) * BM, b0 = (t / ntA) * BN;
+      mbar_wait_bounded(&acc_full[buf], (tl >> 1) & 1, status);
+      tc_fence_after();
+      const uint32_t tb = trow + (uint32_t)(buf * BN);
+      if (ks > 1) {
+        // park the partial tile [BN][BM] in the (idle) operand buffers
+        float* red = reinterpret_cast<float*>(smem);
+        for (int c0 = 0; c0 < BN; c0 += 16) {
+          float v[16];
+          tmem_ld16(tb + c0, v);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) red[(c0 + j) * BM + r] = v[j];
+        }
+      } else if (BN <= 64) {
+        // drain the whole accumulator first, release it, then store
+        float v[BN];
+#pragma unroll
+        for (int c0 = 0; c0 < BN; c0 += 16) tmem_ld16(tb + c0, v + c0);
+        tc_fence_before();
+        mbar_arrive(&acc_empty[buf]);
+#pragma unroll
+        for (int c = 0; c < BN; ++c) {
+          const int m = SWAP ? (b0 + c) : (a0 + r);
+          const int n = SWAP ? (a0 + r) : (b0 + c);
+          if (rope) {
+            const float pv = __shfl_xor_sync(0xffffffffu, v[c], rhalf);
+            if (m < M && n < N) epi_apply_rope<bf16>(e, m, n, v[c], pv);
+          } else if (m < M && n < N) {
+            epi_apply<bf16>(e, m, n, v[c]);
+          }
+        }
+      } else {
+        for (int c0 = 0; c0 < BN; c0 += 16) {
+          float v[16];
+          tmem_ld16(tb + c0, v);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int m = SWAP ? (b0 + c0 + j) : (a0 + r);
+            const int n = SWAP ? (a0 + r) : (b0 + c0 + j);
+            if (rope) {
+              const float pv = __shfl_xor_sync(0xffffffffu, v[j], rhalf);
+              if (m < M && n < N) epi_apply_rope<bf16>(e, m, n, v[j], pv);
+            } else if (m < M && n < N) {
+              epi_apply<bf16>(e, m, n, v[j]);
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&acc_empty[buf]);
+      }
+    }
+  }
+
+  if (ks > 1) {
+    // reduce-scatter over the cluster: rank q sums columns [q*BN/ks, ...)
+    // of all ks partial tiles in rank order (deterministic). Every thread of
+    // every CTA takes part in both cluster barriers.
     namespace cg = cooperative_groups;
     cg::cluster_group cluster = cg::this_cluster();
-    float* red = reinterpret_cast<float*>(smem);
-    for (int c0 = 0; c0 < BN; c0 += 16) {
-      float v[16];
-      tmem_ld16(trow + c0, v);
-#pragma unroll
-      for (int j = 0; j < 16; ++j) red[(c0 + j) * BM + r] = v[j];
-    }
     cluster.sync();
-    const int cpr = BN / ks;  // columns reduced by this rank
-    const int cbeg = (int)cluster.block_rank() * cpr;
-    for (int c = cbeg; c < cbeg + cpr; ++c) {
-      float part[8];
+    if (warp < 4) {
+      const int r = warp * 32 + lane;
+      const bool rope = SWAP && e.kind == EPI_QKV1_ROPE;
+      const int rhalf = e.rot >> 1;
+      const int a0 = (t_first % ntA) * BM, b0 = (t_first / ntA) * BN;
+      float* red = reinterpret_cast<float*>(smem);
+      const int cpr = BN / ks;
+      const int cbeg = (int)cluster.block_rank() * cpr;
+      for (int c = cbeg; c < cbeg + cpr; ++c) {
+        float part[8];
 #pragma unroll
-      for (int p = 0; p < 8; ++p)
-        part[p] = (p < ks) ? cluster.map_shared_rank(red, p)[c * BM + r] : 0.f;
-      float acc = 0.f;
+        for (int p = 0; p < 8; ++p)
+          part[p] = (p < ks) ? cluster.map_shared_rank(red, p)[c * BM + r] : 0.f;
+        float acc = 0.f;
 #pragma unroll
-      for (int p = 0; p < 8; ++p) acc += part[p];   // rank order: deterministic
-      const int m = SWAP ? (b0 + c) : (a0 + r);
-      const int n = SWAP ? (a0 + r) : (b0 + c);
-      if (rope) {
-        const float pv = __shfl_xor_sync(0xffffffffu, acc, rhalf);
-        if (m < M && n < N) epi_apply_rope<bf16>(e, m, n, acc, pv);
-      } else if (m < M && n < N) {
-        epi_apply<bf16>(e, m, n, acc);
+        for (int p = 0; p < 8; ++p) acc += part[p];
+        const int m = SWAP ? (b0 + c) : (a0 + r);
+        const int n = SWAP ? (a0 + r) : (b0 + c);
+        if (rope) {
+          const float pv = __shfl_xor_sync(0xffffffffu, acc, rhalf);
+          if (m < M && n < N) epi_apply_rope<bf16>(e, m, n, acc, pv);
+        } else if (m < M && n < N) {
+          epi_apply<bf16>(e, m, n, acc);
+        }
       }
     }
     cluster.sync();  // no CTA leaves while another still reads its partial
@@ -292,20 +347,58 @@ bool make_map(CUtensorMap* map, const void* base, int rows, int cols, int ld, in
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+constexpr size_t SMEM_MAX = 227 * 1024;
+
 template <int BN, bool SWAP>
 cudaError_t prepare_one() {
-  return cudaFuncSetAttribute(gemm_tc_kernel<BN, SWAP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              (int)smem_bytes<BN>());
+  cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, SWAP>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_MAX);
+  return e;
+}
+
+int sm_count() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
 }
 
 template <int BN, bool SWAP>
-cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& mb, dim3 grid, int M, int N,
-                       int nkb, int ks, int xk_split, int xk_off, const Epi& e, int* status,
-                       cudaStream_t s) {
+cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& mb, int M, int N, int nkb,
+                       int ks, int ntA, int ntB, int xk_split, int xk_off, const Epi& e,
+                       int* status, cudaStream_t s) {
+  constexpr size_t SB = stage_bytes<BN>();
+  const int nloc = (nkb + ks - 1) / ks;
+  int stages = (int)((SMEM_MAX - 1024) / SB);
+  if (stages > MAX_STAGES) stages = MAX_STAGES;
+  if (ks > 1) {
+    // one tile per CTA: no deeper ring than its K blocks, but room for the
+    // [BN][BM] fp32 partial tile
+    const int need = (int)((BN * BM * 4 + SB - 1) / SB);
+    stages = nloc < stages ? nloc : stages;
+    if (stages < need) stages = need;
+  }
+  if (stages < 2) stages = 2;
+  const size_t smem = (size_t)stages * SB + 1024;
+  const int ntiles = ntA * ntB;
+  dim3 grid;
+  if (ks > 1) {
+    grid = dim3(ntiles, 1, ks);
+  } else {
+    int per_sm = 0;
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gemm_tc_kernel<BN, SWAP>, THREADS, smem);
+    if (per_sm < 1) per_sm = 1;
+    const int slots = sm_count() * per_sm;
+    grid = dim3(ntiles < slots ? ntiles : slots, 1, 1);
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
-  cfg.blockDim = dim3(128, 1, 1);
-  cfg.dynamicSmemBytes = smem_bytes<BN>();
+  cfg.blockDim = dim3(THREADS, 1, 1);
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -315,7 +408,7 @@ cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& mb, dim3 grid, 
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   cudaError_t err = cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN, SWAP>, ma, mb, M, N, nkb, ks,
-                                       xk_split, xk_off, e, status);
+                                       stages, ntA, ntB, xk_split, xk_off, e, status);
   note_launch();
   return err;
 }
@@ -337,6 +430,7 @@ cudaError_t gemm_tc_prepare() {
   if ((e = prepare_one<128, true>()) != cudaSuccess) return e;
   if ((e = prepare_one<256, true>()) != cudaSuccess) return e;
   if ((e = prepare_one<256, false>()) != cudaSuccess) return e;
+  sm_count();
   done = true;
   return cudaSuccess;
 }
@@ -376,22 +470,22 @@ cudaError_t launch_gemm_tc(int dt, const void* X, int ldx, const void* W, int ld
     if (!make_map(&ma, W, N, K, ldw, BM) || !make_map(&mb, X, M, xcols, ldx, BN))
       return cudaErrorInvalidValue;
     // K splits (a power of two <= 8, the portable cluster size): the fewest
-    // that put a CTA on every SM, each split keeping >= 1 K block.
+    // that put a CTA on every SM, each split keeping >= 2 K blocks. Without
+    // a split the kernel runs persistent over the tiles.
     int ks = 1;
-    while (ks < 8 && nt * ks < 148 && nkb / (ks * 2) >= 1) ks *= 2;
-    dim3 grid(nt, 1, ks);
+    while (ks < 8 && nt * ks < sm_count() && nkb / (ks * 2) >= 2) ks *= 2;
     switch (BN) {
-      case 32: return launch_one<32, true>(ma, mb, grid, M, N, nkb, ks, xk_split, xk_off, e, status, s);
-      case 64: return launch_one<64, true>(ma, mb, grid, M, N, nkb, ks, xk_split, xk_off, e, status, s);
-      case 128: return launch_one<128, true>(ma, mb, grid, M, N, nkb, ks, xk_split, xk_off, e, status, s);
-      default: return launch_one<256, true>(ma, mb, grid, M, N, nkb, ks, xk_split, xk_off, e, status, s);
+      case 32: return launch_one<32, true>(ma, mb, M, N, nkb, ks, nt, 1, xk_split, xk_off, e, status, s);
+      case 64: return launch_one<64, true>(ma, mb, M, N, nkb, ks, nt, 1, xk_split, xk_off, e, status, s);
+      case 128: return launch_one<128, true>(ma, mb, M, N, nkb, ks, nt, 1, xk_split, xk_off, e, status, s);
+      default: return launch_one<256, true>(ma, mb, M, N, nkb, ks, nt, 1, xk_split, xk_off, e, status, s);
     }
   }
   constexpr int BNP = 256;
   if (!make_map(&ma, X, M, xcols, ldx, BM) || !make_map(&mb, W, N, K, ldw, BNP))
     return cudaErrorInvalidValue;
-  dim3 grid((M + BM - 1) / BM, (N + BNP - 1) / BNP, 1);
-  return launch_one<BNP, false>(ma, mb, grid, M, N, nkb, 1, xk_split, xk_off, e, status, s);
+  return launch_one<BNP, false>(ma, mb, M, N, nkb, 1, (M + BM - 1) / BM, (N + BNP - 1) / BNP,
+                                xk_split, xk_off, e, status, s);
 }
 
 }  // namespace bt

@@ -135,7 +135,8 @@ def test_embedder_flags_bad_token():
 
 @pytest.mark.parametrize("M,N,K", [(1, 128, 64), (2, 384, 128), (33, 768, 768), (64, 5376, 768),
                                    (64, 768, 3840), (100, 1000, 256), (256, 2048, 1024),
-                                   (257, 768, 768), (1000, 2304, 768), (4096, 512, 192)])
+                                   (257, 768, 768), (1000, 2304, 768), (4096, 512, 192),
+                                   (64, 50304, 768), (32, 4096, 512), (128, 9000, 1024)])
 def test_linear_tensor_cores_match_fp64(M, N, K):
     """tcgen05 path (weights-as-A for M <= 256 with split K; activations-as-A
     above) against an fp64 product of the same bf16 operands."""
