@@ -347,7 +347,9 @@ bool make_map(CUtensorMap* map, const void* base, int rows, int cols, int ld, in
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-constexpr size_t SMEM_MAX = 227 * 1024;
+// dynamic shared memory ceiling: the 227 KB opt-in less room for the
+// kernel's static shared memory (barriers)
+constexpr size_t SMEM_MAX = 227 * 1024 - 1024;
 
 template <int BN, bool SWAP>
 cudaError_t prepare_one() {

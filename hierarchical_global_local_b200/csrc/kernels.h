@@ -130,6 +130,9 @@ int gemm_tc_supported(int dt, int M, int N, int K, int xk_split, int xk_off);
 cudaError_t launch_argmax(const float* logits, int B, int V, int ld, int32_t* next,
                           cudaStream_t s);
 
+// Record a failed CUDA call for bt_last_cuda_error (per thread).
+void note_cuda_error(const char* what, cudaError_t e);
+
 // ---- launch accounting ------------------------------------------------------
 // Every kernel launch site calls note_launch(); launch_count() is the running
 // total for this process (graph captures count when captured).

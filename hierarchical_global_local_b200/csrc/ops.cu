@@ -7,7 +7,11 @@
 
 using namespace bt;
 
-static int status_of(cudaError_t e) { return e == cudaSuccess ? BT_OK : BT_ECUDA; }
+static int status_of(cudaError_t e) {
+  if (e == cudaSuccess) return BT_OK;
+  note_cuda_error("kernel launch", e);
+  return BT_ECUDA;
+}
 
 extern "C" {
 

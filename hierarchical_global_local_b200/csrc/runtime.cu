@@ -28,6 +28,10 @@ using namespace bt;
 
 static thread_local std::string g_last_cuda;
 
+void bt::note_cuda_error(const char* what, cudaError_t e) {
+  g_last_cuda = std::string(what) + ": " + cudaGetErrorString(e);
+}
+
 #define BT_CUDA(call)                                      \
   do {                                                     \
     cudaError_t e__ = (call);                              \
