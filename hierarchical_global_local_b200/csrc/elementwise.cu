@@ -360,6 +360,42 @@ cudaError_t launch_argmax(const float* logits, int B, int V, int ld, int32_t* ne
   return cudaGetLastError();
 }
 
+__global__ void argmax_reduce_kernel(const float2* __restrict__ part, int n_tiles, int M,
+                                     int32_t* __restrict__ next) {
+  const int m = blockIdx.x;
+  float best = -INFINITY;
+  int bi = 0x7fffffff;
+  for (int t = threadIdx.x; t < n_tiles; t += blockDim.x) {
+    const float2 p = part[(size_t)t * M + m];
+    const int i = __float_as_int(p.y);
+    if (p.x > best || (p.x == best && i < bi)) { best = p.x; bi = i; }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float ov = __shfl_xor_sync(0xffffffffu, best, o);
+    const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+    if (ov > best || (ov == best && oi < bi)) { best = ov; bi = oi; }
+  }
+  __shared__ float sv[8];
+  __shared__ int si[8];
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) { sv[w] = best; si[w] = bi; }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int k = 1; k < (int)(blockDim.x >> 5); ++k)
+      if (sv[k] > best || (sv[k] == best && si[k] < bi)) { best = sv[k]; bi = si[k]; }
+    next[m] = (bi == 0x7fffffff) ? 0 : bi;
+  }
+}
+
+cudaError_t launch_argmax_reduce(const float2* part, int n_tiles, int M, int32_t* next,
+                                 cudaStream_t s) {
+  if (M == 0) return cudaSuccess;
+  argmax_reduce_kernel<<<M, 256, 0, s>>>(part, n_tiles, M, next);
+  note_launch();
+  return cudaGetLastError();
+}
+
 // ---------------------------------------------------------------------------
 // conversions used when the model is created
 // ---------------------------------------------------------------------------

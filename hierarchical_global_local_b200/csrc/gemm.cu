@@ -71,6 +71,8 @@ cudaError_t launch_gemm(int dt, const void* X, int ldx, const void* W, int ldw, 
   if (M == 0 || N == 0) return cudaSuccess;
   if (e.kind == EPI_QKV1_ROPE && (g_gemm_path == 1 || !gemm_rope_fusable(dt, M, N, K, xk_split, xk_off, e.D / e.H, e.rot)))
     return cudaErrorNotSupported;  // the caller runs EPI_QKV1 + the rotary kernel instead
+  if (e.kind == EPI_LOGITS_ARGMAX && (g_gemm_path == 1 || !gemm_argmax_fusable(dt, M, N, K)))
+    return cudaErrorNotSupported;  // the caller runs EPI_F32 + the argmax kernel instead
   const bool tc_ok = gemm_tc_supported(dt, M, N, K, xk_split, xk_off) != 0;
   if (g_gemm_path != 1 && tc_ok)
     return launch_gemm_tc(dt, X, ldx, W, ldw, M, N, K, xk_split, xk_off, e, scr, status, s);

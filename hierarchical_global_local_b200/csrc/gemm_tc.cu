@@ -93,6 +93,17 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// cluster barrier halves (per thread, not warp-aligned)
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_arrive_release() {
+  asm volatile("barrier.cluster.arrive.release;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire() {
+  asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
+}
+
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
@@ -134,6 +145,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
   bf16* sB = reinterpret_cast<bf16*>(smem + (size_t)stages * BM * BK * 2);
   __shared__ __align__(8) uint64_t full[MAX_STAGES], empty[MAX_STAGES], acc_full[2], acc_empty[2];
   __shared__ uint32_t tmem_slot;
+  __shared__ float2 s_arg[4][BN <= 64 ? BN : 1];  // fused argmax: per warp, per column
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ntiles = ntA * ntB;
@@ -164,6 +176,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
+  // split K: announce that this CTA is running; peers wait on it before
+  // their first store into this CTA's shared memory
+  if (ks > 1) cluster_arrive_relaxed();
 
   if (warp == 4) {
     // ---- TMA producer ----
@@ -223,14 +238,62 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
       tc_fence_after();
       const uint32_t tb = trow + (uint32_t)(buf * BN);
       if (ks > 1) {
-        // park the partial tile [BN][BM] in the (idle) operand buffers
-        float* red = reinterpret_cast<float*>(smem);
+        // push this CTA's partial columns to their owners: column c goes to
+        // rank c / (BN/ks), slot [my rank][c % (BN/ks)] of its receive
+        // buffer (remote stores do not wait for a round trip)
+        namespace cg = cooperative_groups;
+        cg::cluster_group cluster = cg::this_cluster();
+        float* recv = reinterpret_cast<float*>(smem + (size_t)stages * stage_bytes<BN>());
+        const int cpr = BN / ks;
+        const int me = (int)cluster.block_rank();
+        cluster_wait_acquire();  // every CTA of the cluster has started
         for (int c0 = 0; c0 < BN; c0 += 16) {
           float v[16];
           tmem_ld16(tb + c0, v);
 #pragma unroll
-          for (int j = 0; j < 16; ++j) red[(c0 + j) * BM + r] = v[j];
+          for (int j = 0; j < 16; ++j) {
+            const int c = c0 + j;
+            float* dst = cluster.map_shared_rank(recv, c / cpr);
+            dst[((size_t)me * cpr + (c % cpr)) * BM + r] = v[j];
+          }
         }
+      } else if (SWAP && BN <= 64 && e.kind == EPI_LOGITS_ARGMAX) {
+        // LM head: logits (optional) and the tile's argmax per token column:
+        // warp shuffles, then the four warps through shared memory
+        const int n = a0 + r;
+        float* logits = reinterpret_cast<float*>(e.out0);
+        for (int c0 = 0; c0 < BN; c0 += 16) {
+          float v[16];
+          tmem_ld16(tb + c0, v);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int m = b0 + c0 + j;
+            if (logits && m < M && n < N) logits[(size_t)m * e.ld0 + n] = v[j];
+            float bv = (n < N) ? v[j] : -INFINITY;
+            int bi = n;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+              const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+              const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+              if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+            }
+            if (lane == 0) s_arg[warp][c0 + j] = make_float2(bv, __int_as_float(bi));
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&acc_empty[buf]);
+        asm volatile("bar.sync 1, 128;" ::: "memory");  // the four epilogue warps
+        if (r < BN && b0 + r < M) {
+          float2 best = s_arg[0][r];
+#pragma unroll
+          for (int w = 1; w < 4; ++w) {
+            const float2 o = s_arg[w][r];
+            if (o.x > best.x || (o.x == best.x && __float_as_int(o.y) < __float_as_int(best.y)))
+              best = o;
+          }
+          reinterpret_cast<float2*>(e.aux)[(size_t)(t % ntA) * M + b0 + r] = best;
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");  // s_arg reused by the next tile
       } else if (BN <= 64) {
         // drain the whole accumulator first, release it, then store
         float v[BN];
@@ -272,28 +335,28 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
   }
 
   if (ks > 1) {
-    // reduce-scatter over the cluster: rank q sums columns [q*BN/ks, ...)
-    // of all ks partial tiles in rank order (deterministic). Every thread of
-    // every CTA takes part in both cluster barriers.
+    // every partial has been pushed once all ranks pass this barrier (every
+    // thread of every CTA takes part); then rank q sums, in rank order
+    // (deterministic), the ks slices of its columns [q*BN/ks, (q+1)*BN/ks)
+    // from its own shared memory. Nobody touches another CTA's shared
+    // memory after the barrier, so no second barrier is needed.
     namespace cg = cooperative_groups;
     cg::cluster_group cluster = cg::this_cluster();
-    cluster.sync();
+    if (warp >= 4) cluster_wait_acquire();  // producer / MMA warps: first phase
+    cluster_arrive_release();               // second phase: all pushes done
+    cluster_wait_acquire();
     if (warp < 4) {
       const int r = warp * 32 + lane;
       const bool rope = SWAP && e.kind == EPI_QKV1_ROPE;
       const int rhalf = e.rot >> 1;
       const int a0 = (t_first % ntA) * BM, b0 = (t_first / ntA) * BN;
-      float* red = reinterpret_cast<float*>(smem);
+      const float* recv = reinterpret_cast<const float*>(smem + (size_t)stages * stage_bytes<BN>());
       const int cpr = BN / ks;
       const int cbeg = (int)cluster.block_rank() * cpr;
-      for (int c = cbeg; c < cbeg + cpr; ++c) {
-        float part[8];
-#pragma unroll
-        for (int p = 0; p < 8; ++p)
-          part[p] = (p < ks) ? cluster.map_shared_rank(red, p)[c * BM + r] : 0.f;
+      for (int cc = 0; cc < cpr; ++cc) {
         float acc = 0.f;
-#pragma unroll
-        for (int p = 0; p < 8; ++p) acc += part[p];
+        for (int p = 0; p < ks; ++p) acc += recv[((size_t)p * cpr + cc) * BM + r];
+        const int c = cbeg + cc;
         const int m = SWAP ? (b0 + c) : (a0 + r);
         const int n = SWAP ? (a0 + r) : (b0 + c);
         if (rope) {
@@ -304,7 +367,6 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
         }
       }
     }
-    cluster.sync();  // no CTA leaves while another still reads its partial
   }
 
   tc_fence_before();
@@ -377,15 +439,17 @@ cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& mb, int M, int 
   const int nloc = (nkb + ks - 1) / ks;
   int stages = (int)((SMEM_MAX - 1024) / SB);
   if (stages > MAX_STAGES) stages = MAX_STAGES;
+  size_t recv_bytes = 0;
   if (ks > 1) {
-    // one tile per CTA: no deeper ring than its K blocks, but room for the
-    // [BN][BM] fp32 partial tile
-    const int need = (int)((BN * BM * 4 + SB - 1) / SB);
+    // one tile per CTA: no deeper ring than its K blocks, plus a receive
+    // buffer for the [BN][BM] fp32 partials pushed by the cluster
+    recv_bytes = (size_t)BN * BM * 4;
+    int fit = (int)((SMEM_MAX - 1024 - recv_bytes) / SB);
     stages = nloc < stages ? nloc : stages;
-    if (stages < need) stages = need;
+    if (stages > fit) stages = fit;
   }
   if (stages < 2) stages = 2;
-  const size_t smem = (size_t)stages * SB + 1024;
+  const size_t smem = (size_t)stages * SB + recv_bytes + 1024;
   const int ntiles = ntA * ntB;
   dim3 grid;
   if (ks > 1) {
@@ -449,6 +513,10 @@ int gemm_rope_fusable(int dt, int M, int N, int K, int xk_split, int xk_off, int
   return 1;
 }
 
+int gemm_argmax_fusable(int dt, int M, int N, int K) {
+  return (gemm_tc_supported(dt, M, N, K, 1 << 30, 0) && M <= 64) ? 1 : 0;
+}
+
 int gemm_tc_supported(int dt, int M, int N, int K, int xk_split, int xk_off) {
   if (dt != DT_BF16 || M < 1 || N < 1 || K < BK || (K % BK)) return 0;
   if (encoder() == nullptr) return 0;
@@ -476,6 +544,7 @@ cudaError_t launch_gemm_tc(int dt, const void* X, int ldx, const void* W, int ld
     // a split the kernel runs persistent over the tiles.
     int ks = 1;
     while (ks < 8 && nt * ks < sm_count() && nkb / (ks * 2) >= 2) ks *= 2;
+    if (e.kind == EPI_LOGITS_ARGMAX) ks = 1;  // the argmax epilogue needs whole tiles
     switch (BN) {
       case 32: return launch_one<32, true>(ma, mb, M, N, nkb, ks, nt, 1, xk_split, xk_off, e, status, s);
       case 64: return launch_one<64, true>(ma, mb, M, N, nkb, ks, nt, 1, xk_split, xk_off, e, status, s);

@@ -82,6 +82,10 @@ enum EpiKind : int {
                       // q (rotated) -> out0 [m, n]; k (rotated), v -> the
                       // caches at the token's position (tensor-core decode
                       // orientation only, see gemm_rope_fusable)
+  EPI_LOGITS_ARGMAX = 5,  // LM head: logits -> out0 [m, n] fp32 if out0 != null;
+                          // per 128-row tile t, the (max, lowest argmax) of
+                          // column m -> aux[t * M + m] (float2: value, index
+                          // bits); tensor-core decode orientation only
 };
 
 struct Epi {
@@ -101,7 +105,15 @@ struct Epi {
   void* vc;
   int cap;
   PosSpec pos;
+  // EPI_LOGITS_ARGMAX only
+  void* aux;
 };
+// True when launch_gemm runs EPI_LOGITS_ARGMAX for this shape.
+int gemm_argmax_fusable(int dt, int M, int N, int K);
+// next[m] = index of the best of the n_tiles partial (value, index) pairs
+// part[t * M + m] (lowest index among equal values).
+cudaError_t launch_argmax_reduce(const float2* part, int n_tiles, int M, int32_t* next,
+                                 cudaStream_t s);
 // True when launch_gemm will run EPI_QKV1_ROPE fused for this shape.
 int gemm_rope_fusable(int dt, int M, int N, int K, int xk_split, int xk_off, int d_head, int rot);
 

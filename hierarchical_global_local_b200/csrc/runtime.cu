@@ -126,12 +126,13 @@ struct bt_model {
   int *dstate = nullptr, *status = nullptr;
   float2* rope_tab = nullptr;
   void* attn_scratch = nullptr;
+  float2* arg_part = nullptr;  // LM-head per-tile argmax partials
   GemmScratch gs{};
   int B = 0, t = 0;
   bool prefilled = false;
   bool use_graphs = true;
-  cudaGraphExec_t graphs[2][2] = {{nullptr, nullptr}, {nullptr, nullptr}};  // [block_step][greedy]
-  long long graph_kernels[2][2] = {{0, 0}, {0, 0}};
+  cudaGraphExec_t graphs[2][2][2] = {};  // [block_step][greedy][logits wanted]
+  long long graph_kernels[2][2][2] = {};
   int graph_B = 0;
   long long kernels = 0;  // kernels enqueued for execution
   // profiler
@@ -144,9 +145,9 @@ struct bt_model {
   int cap_records = 0;
   // profiled decode graphs: event-record nodes around every kernel
   struct Pair { bt_profile_record r; cudaEvent_t a, b; };
-  cudaGraphExec_t pgraphs[2][2] = {{nullptr, nullptr}, {nullptr, nullptr}};
-  long long pgraph_kernels[2][2] = {{0, 0}, {0, 0}};
-  std::vector<Pair> pairs[2][2];
+  cudaGraphExec_t pgraphs[2][2][2] = {};
+  long long pgraph_kernels[2][2][2] = {};
+  std::vector<Pair> pairs[2][2][2];
   std::vector<Pair>* cap_pairs = nullptr;  // list being captured into
 };
 
@@ -230,6 +231,7 @@ static size_t carve(bt_model* m, const Dims& d, void* ws) {
   m->status = (int*)c.take(64);
   m->rope_tab = (float2*)c.take((size_t)d.tab_pos * (d.rot / 2 > 0 ? d.rot / 2 : 1) * 8);
   m->attn_scratch = c.take(attn_decode_scratch_bytes(d.Bmax, d.H, d.d, d.n_cap, d.dt));
+  m->arg_part = (float2*)c.take((size_t)((d.V + 127) / 128) * d.Bmax * sizeof(float2));
   const int maxN = 7 * d.D > d.V ? 7 * d.D : d.V;
   m->gs.part_bytes = gemm_scratch_bytes(d.Bmax, maxN);
   m->gs.part = (float*)c.take(m->gs.part_bytes);
@@ -439,8 +441,21 @@ static int run_context_to_head_input(bt_model* m, int B, int row_step, int row_o
   return run_token_decoder(m, B, pos, s);
 }
 
-static int run_head(bt_model* m, int B, cudaStream_t s) {
+static int run_head(bt_model* m, int B, bool want_logits, cudaStream_t s) {
   const Dims& d = m->d;
+  if (gemm_argmax_fusable(d.dt, B, d.V, d.D)) {
+    // LM head with the greedy argmax in its epilogue; logits stored only
+    // when the caller asked for them
+    {
+      ProfScope p(m, s, BT_K_GEMM, B, d.V, d.D);
+      Epi el{EPI_LOGITS_ARGMAX, want_logits ? m->logits : nullptr, d.V, nullptr, 0, nullptr, 0, d.D};
+      el.aux = m->arg_part;
+      BT_CUDA(launch_gemm(d.dt, m->xf, d.D, m->w_lm, d.D, B, d.V, d.D, 1 << 30, 0, el, m->gs, m->status, s));
+    }
+    ProfScope p(m, s, BT_K_ARGMAX, B, d.V, 0);
+    BT_CUDA(launch_argmax_reduce(m->arg_part, (d.V + 127) / 128, B, m->next, s));
+    return BT_OK;
+  }
   {
     ProfScope p(m, s, BT_K_GEMM, B, d.V, d.D);
     Epi el{EPI_F32, m->logits, d.V, nullptr, 0, nullptr, 0, d.D};
@@ -463,7 +478,8 @@ static int copy_outputs(bt_model* m, float* logits, int32_t* next) {
 }
 
 // the body of one decode call (captured into a graph or run directly)
-static int enqueue_decode(bt_model* m, bool block_step, bool greedy, cudaStream_t s) {
+static int enqueue_decode(bt_model* m, bool block_step, bool greedy, bool want_logits,
+                          cudaStream_t s) {
   const Dims& d = m->d;
   const int B = m->B;
   const int32_t* src = greedy ? m->next : m->fed;
@@ -487,7 +503,7 @@ static int enqueue_decode(bt_model* m, bool block_step, bool greedy, cudaStream_
     rc = run_token_decoder(m, B, pos, s);
     if (rc != BT_OK) return rc;
   }
-  rc = run_head(m, B, s);
+  rc = run_head(m, B, want_logits, s);
   if (rc != BT_OK) return rc;
   {
     ProfScope p(m, s, BT_K_OTHER, 1, 0, 0);
@@ -498,8 +514,9 @@ static int enqueue_decode(bt_model* m, bool block_step, bool greedy, cudaStream_
 
 static void drop_graphs(bt_model* m) {
   for (auto& a : m->graphs)
-    for (auto& g : a)
-      if (g) { cudaGraphExecDestroy(g); g = nullptr; }
+    for (auto& b : a)
+      for (auto& g : b)
+        if (g) { cudaGraphExecDestroy(g); g = nullptr; }
 }
 
 extern "C" {
@@ -530,7 +547,7 @@ int bt_prefill(bt_model* m, const int32_t* tokens, int32_t B, int32_t T, float* 
   }
   int rc = run_context_to_head_input(m, B, n, n - 1, s);
   if (rc != BT_OK) return rc;
-  rc = run_head(m, B, s);
+  rc = run_head(m, B, logits != nullptr, s);
   if (rc != BT_OK) return rc;
   m->kernels += launch_count() - k0;
   m->prefilled = true;
@@ -548,9 +565,9 @@ int bt_decode_step(bt_model* m, const int32_t* tokens, float* logits, int32_t* n
   if (!greedy)
     BT_CUDA(cudaMemcpyAsync(m->fed, tokens, (size_t)m->B * 4, cudaMemcpyDeviceToDevice, m->stream));
   if (m->use_graphs) {
-    const int bi = block_step ? 1 : 0, gi = greedy ? 1 : 0;
-    cudaGraphExec_t& g = m->prof ? m->pgraphs[bi][gi] : m->graphs[bi][gi];
-    long long& gk = m->prof ? m->pgraph_kernels[bi][gi] : m->graph_kernels[bi][gi];
+    const int bi = block_step ? 1 : 0, gi = greedy ? 1 : 0, li = logits ? 1 : 0;
+    cudaGraphExec_t& g = m->prof ? m->pgraphs[bi][gi][li] : m->graphs[bi][gi][li];
+    long long& gk = m->prof ? m->pgraph_kernels[bi][gi][li] : m->graph_kernels[bi][gi][li];
     if (!g) {
       // capture on the private stream, ordered after the caller's stream
       cudaEvent_t ev;
@@ -563,8 +580,8 @@ int bt_decode_step(bt_model* m, const int32_t* tokens, float* logits, int32_t* n
       BT_CUDA(cudaStreamBeginCapture(m->cap_stream, cudaStreamCaptureModeThreadLocal));
       const long long c0 = launch_count();
       m->capturing = true;
-      m->cap_pairs = m->prof ? &m->pairs[bi][gi] : nullptr;
-      int rc = enqueue_decode(m, block_step, greedy, m->cap_stream);
+      m->cap_pairs = m->prof ? &m->pairs[bi][gi][li] : nullptr;
+      int rc = enqueue_decode(m, block_step, greedy, logits != nullptr, m->cap_stream);
       m->capturing = false;
       m->cap_pairs = nullptr;
       gk = launch_count() - c0;
@@ -579,7 +596,7 @@ int bt_decode_step(bt_model* m, const int32_t* tokens, float* logits, int32_t* n
     if (m->prof) {
       // read this replay's event pairs
       BT_CUDA(cudaStreamSynchronize(m->stream));
-      for (auto& p : m->pairs[bi][gi]) {
+      for (auto& p : m->pairs[bi][gi][li]) {
         if ((int)m->rec.size() >= m->cap_records) break;
         bt_profile_record r = p.r;
         if (r.kind == BT_K_ATTN_DECODE) r.n = m->t / d.L + 1;
@@ -590,7 +607,7 @@ int bt_decode_step(bt_model* m, const int32_t* tokens, float* logits, int32_t* n
     }
   } else {
     const long long c0 = launch_count();
-    int rc = enqueue_decode(m, block_step, greedy, m->stream);
+    int rc = enqueue_decode(m, block_step, greedy, logits != nullptr, m->stream);
     if (rc != BT_OK) return rc;
     m->kernels += launch_count() - c0;
   }
@@ -626,11 +643,12 @@ static void free_events(bt_model* m) {
 
 static void drop_pgraphs(bt_model* m) {
   for (int i = 0; i < 2; ++i)
-    for (int j = 0; j < 2; ++j) {
-      if (m->pgraphs[i][j]) { cudaGraphExecDestroy(m->pgraphs[i][j]); m->pgraphs[i][j] = nullptr; }
-      for (auto& p : m->pairs[i][j]) { cudaEventDestroy(p.a); cudaEventDestroy(p.b); }
-      m->pairs[i][j].clear();
-    }
+    for (int j = 0; j < 2; ++j)
+      for (int k = 0; k < 2; ++k) {
+        if (m->pgraphs[i][j][k]) { cudaGraphExecDestroy(m->pgraphs[i][j][k]); m->pgraphs[i][j][k] = nullptr; }
+        for (auto& p : m->pairs[i][j][k]) { cudaEventDestroy(p.a); cudaEventDestroy(p.b); }
+        m->pairs[i][j][k].clear();
+      }
 }
 
 int bt_profile_begin(bt_model* m, int32_t capacity) {

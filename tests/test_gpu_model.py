@@ -127,3 +127,17 @@ def test_pythia160m_shape_sampled_rows():
     ol = gh.oracle_teacher_forced(wl.shape, w, toks, T, G, dtype=np.float32)
     for s in range(G):
         assert gh.rel_l2(gl[s], ol[s]) <= BF16_REL, (s, gh.rel_l2(gl[s], ol[s]))
+
+
+def test_fused_argmax_matches_returned_logits_bf16():
+    """bf16 LM head: the greedy id computed in the GEMM epilogue equals the
+    argmax of the logits the same call returns, at every step."""
+    shape = synth.ModelShape(vocab=5000, d_model=256, n_heads=4, block_len=4,
+                             n_block_layers=1, n_token_layers=1, prefix_len=1)
+    w = synth.make_weights(shape, seed=21)
+    B, T, G = 5, 24, 9
+    toks = synth.make_tokens(batch=B, length=T + G, vocab=shape.vocab, seed=22)
+    m = gh.build_model(shape, w, B, T + G)
+    gl, gn = gh.gpu_teacher_forced(m, toks, T, G)
+    m.close()
+    assert np.array_equal(gn, gl.argmax(-1))
