@@ -409,14 +409,26 @@ bool make_map(CUtensorMap* map, const void* base, int rows, int cols, int ld, in
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// dynamic shared memory ceiling: the 227 KB opt-in less room for the
-// kernel's static shared memory (barriers)
-constexpr size_t SMEM_MAX = 227 * 1024 - 1024;
+// Dynamic shared memory ceiling of one instantiation: the device's opt-in
+// per-block limit less the kernel's static shared memory.
+template <int BN, bool SWAP>
+size_t& dyn_smem_max() {
+  static size_t v = 0;
+  return v;
+}
 
 template <int BN, bool SWAP>
 cudaError_t prepare_one() {
-  cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, SWAP>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_MAX);
+  int dev = 0, optin = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  cudaFuncAttributes fa;
+  if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, gemm_tc_kernel<BN, SWAP>);
+  if (e != cudaSuccess) return e;
+  const size_t mx = (size_t)optin - fa.sharedSizeBytes;
+  e = cudaFuncSetAttribute(gemm_tc_kernel<BN, SWAP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)mx);
+  if (e == cudaSuccess) dyn_smem_max<BN, SWAP>() = mx;
   return e;
 }
 
@@ -436,6 +448,8 @@ cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& mb, int M, int 
                        int ks, int ntA, int ntB, int xk_split, int xk_off, const Epi& e,
                        int* status, cudaStream_t s) {
   constexpr size_t SB = stage_bytes<BN>();
+  const size_t SMEM_MAX = dyn_smem_max<BN, SWAP>();
+  if (SMEM_MAX < 3 * SB) return cudaErrorInvalidConfiguration;
   const int nloc = (nkb + ks - 1) / ks;
   int stages = (int)((SMEM_MAX - 1024) / SB);
   if (stages > MAX_STAGES) stages = MAX_STAGES;
