@@ -60,6 +60,8 @@ attn_decode_kernel(const T* __restrict__ q, int ldq, const T* __restrict__ kc,
                    const T* __restrict__ vc, int H, int cap, PosSpec kvlen, T* __restrict__ out,
                    int ld_out, float* __restrict__ part, int* __restrict__ counters,
                    int max_splits, int* status, float qscale) {
+  pdl_trigger();
+  pdl_wait();
   using C = DecCfg<T, DH>;
   const int pair = blockIdx.x;  // b * H + h
   const int split = blockIdx.y;
@@ -214,9 +216,9 @@ static cudaError_t launch_dec(const void* q, int ldq, const void* kc, const void
                                          ((part + 255) & ~(size_t)255));
   dim3 grid(B * H, ms);
   const float qscale = 1.4426950408889634f / sqrtf((float)DH);
-  attn_decode_kernel<T, DH><<<grid, C::THREADS, C::SMEM, s>>>(
+  BT_LAUNCH(attn_decode_kernel<T, DH>, dim3(grid), dim3(C::THREADS), C::SMEM, s, 
       (const T*)q, ldq, (const T*)kc, (const T*)vc, H, cap, kvlen, (T*)out, ld_out, partp,
-      counters, ms, status, qscale); note_launch();
+      counters, ms, status, qscale);
   return cudaGetLastError();
 }
 
@@ -247,6 +249,8 @@ template <typename T, int DH>
 __global__ void attn_small_kernel(const T* __restrict__ q, int ldq, const T* __restrict__ kc,
                                   const T* __restrict__ vc, int B, int H, int cap, PosSpec qpos,
                                   T* __restrict__ out, int ld_out, float scale) {
+  pdl_trigger();
+  pdl_wait();
   constexpr int EPL = DH / 32;  // elements per lane
   const int warp = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -289,9 +293,9 @@ cudaError_t launch_attn_small(int dt, const void* q, int ldq, const void* k_cach
   const int grid = (warps + 3) / 4;
   const float scale = 1.4426950408889634f / sqrtf((float)d);
 #define BT_SMALL(T, DHV)                                                                      \
-  attn_small_kernel<T, DHV><<<grid, 128, 0, s>>>((const T*)q, ldq, (const T*)k_cache,        \
+  BT_LAUNCH(attn_small_kernel<T, DHV>, dim3(grid), dim3(128), 0, s, (const T*)q, ldq, (const T*)k_cache,        \
                                                   (const T*)v_cache, B, H, cap, qpos, (T*)out, \
-                                                  ld_out, scale); note_launch();                             \
+                                                  ld_out, scale);                             \
   return cudaGetLastError()
   if (dt == DT_BF16) {
     if (d == 32) { BT_SMALL(bf16, 32); }

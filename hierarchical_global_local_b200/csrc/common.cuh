@@ -133,6 +133,17 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       : "memory");
 }
 
+// ---- programmatic dependent launch ------------------------------------------
+// Every kernel of the library calls pdl_trigger() first (its dependents may be
+// scheduled as soon as all of its CTAs are running) and pdl_wait() before it
+// reads or writes anything an earlier kernel in the stream touches (returns
+// once the preceding grid has completed and its writes are visible). Without
+// the launch attribute both are no-ops.
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

@@ -7,6 +7,8 @@
 // of a block in dims [j*D/L_B, (j+1)*D/L_B). Layer pieces follow the Pythia
 // architecture named in §5 "Experimental setup" (LayerNorm with biased
 // variance, rotate-half rotary on the first 25% of each head).
+#include <stdlib.h>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -16,6 +18,15 @@ static long long g_launches = 0;
 void note_launch() { __atomic_add_fetch(&g_launches, 1, __ATOMIC_RELAXED); }
 long long launch_count() { return __atomic_load_n(&g_launches, __ATOMIC_RELAXED); }
 
+bool pdl_enabled() {
+  static int on = -1;
+  if (on < 0) {
+    const char* e = getenv("BT_NO_PDL");
+    on = (e && e[0] == '1') ? 0 : 1;
+  }
+  return on == 1;
+}
+
 // ---------------------------------------------------------------------------
 // embedder
 // ---------------------------------------------------------------------------
@@ -23,6 +34,8 @@ template <typename T>
 __global__ void embed_prompt_kernel(const int32_t* __restrict__ tokens, int T_len, int n, int L_B,
                                     const T* __restrict__ table, int V, int D,
                                     float* __restrict__ h, int* status) {
+  pdl_trigger();
+  pdl_wait();
   const int r = blockIdx.x;  // row = b * n + i
   const int b = r / n, i = r % n;
   const int De = D / L_B;
@@ -43,6 +56,8 @@ __global__ void ingest_kernel(const int32_t* __restrict__ src, int32_t* __restri
                               int block_step, const T* __restrict__ blk_emb,
                               const T* __restrict__ tok_emb, float* __restrict__ h,
                               int* status) {
+  pdl_trigger();
+  pdl_wait();
   const int b = blockIdx.x;
   const int j = dstate[1];
   int tok = src[b];
@@ -66,12 +81,16 @@ __global__ void ingest_kernel(const int32_t* __restrict__ src, int32_t* __restri
 }
 
 __global__ void set_state_kernel(int* dstate, int t, int L_B) {
+  pdl_trigger();
+  pdl_wait();
   dstate[0] = t;
   dstate[1] = t % L_B;
   dstate[2] = t / L_B;
 }
 
 __global__ void advance_kernel(int* dstate, int L_B) {
+  pdl_trigger();
+  pdl_wait();
   const int t = dstate[0] + 1;
   dstate[0] = t;
   dstate[1] = t % L_B;
@@ -84,12 +103,12 @@ cudaError_t launch_embed_prompt(int dt, const int32_t* tokens, int B, int T, int
   const int n = T / L_B;
   if (B * n == 0) return cudaSuccess;
   if (dt == DT_BF16) {
-    embed_prompt_kernel<bf16><<<B * n, 256, 0, s>>>(tokens, T, n, L_B, (const bf16*)blk_emb, V, D,
-                                                    h, status); note_launch();
+    BT_LAUNCH(embed_prompt_kernel<bf16>, dim3(B * n), dim3(256), 0, s, tokens, T, n, L_B, (const bf16*)blk_emb, V, D,
+                                                    h, status);
   }
   else {
-    embed_prompt_kernel<float><<<B * n, 256, 0, s>>>(tokens, T, n, L_B, (const float*)blk_emb, V,
-                                                     D, h, status); note_launch();
+    BT_LAUNCH(embed_prompt_kernel<float>, dim3(B * n), dim3(256), 0, s, tokens, T, n, L_B, (const float*)blk_emb, V,
+                                                     D, h, status);
   }
   return cudaGetLastError();
 }
@@ -98,24 +117,24 @@ cudaError_t launch_ingest(int dt, const int32_t* src, int32_t* block_tok, const 
                           int B, int L_B, int V, int D, int block_step, const void* blk_emb,
                           const void* tok_emb, float* h, int* status, cudaStream_t s) {
   if (dt == DT_BF16) {
-    ingest_kernel<bf16><<<B, 256, 0, s>>>(src, block_tok, dstate, L_B, V, D, block_step,
-                                          (const bf16*)blk_emb, (const bf16*)tok_emb, h, status); note_launch();
+    BT_LAUNCH(ingest_kernel<bf16>, dim3(B), dim3(256), 0, s, src, block_tok, dstate, L_B, V, D, block_step,
+                                          (const bf16*)blk_emb, (const bf16*)tok_emb, h, status);
   }
   else {
-    ingest_kernel<float><<<B, 256, 0, s>>>(src, block_tok, dstate, L_B, V, D, block_step,
+    BT_LAUNCH(ingest_kernel<float>, dim3(B), dim3(256), 0, s, src, block_tok, dstate, L_B, V, D, block_step,
                                            (const float*)blk_emb, (const float*)tok_emb, h,
-                                           status); note_launch();
+                                           status);
   }
   return cudaGetLastError();
 }
 
 cudaError_t launch_set_state(int* dstate, int t, int L_B, cudaStream_t s) {
-  set_state_kernel<<<1, 1, 0, s>>>(dstate, t, L_B); note_launch();
+  BT_LAUNCH(set_state_kernel, dim3(1), dim3(1), 0, s, dstate, t, L_B);
   return cudaGetLastError();
 }
 
 cudaError_t launch_advance(int* dstate, int L_B, cudaStream_t s) {
-  advance_kernel<<<1, 1, 0, s>>>(dstate, L_B); note_launch();
+  BT_LAUNCH(advance_kernel, dim3(1), dim3(1), 0, s, dstate, L_B);
   return cudaGetLastError();
 }
 
@@ -187,6 +206,8 @@ __global__ void __launch_bounds__(LN_THREADS)
 ln_dual_kernel(const float* __restrict__ h, int D, const float* __restrict__ g1,
                const float* __restrict__ b1, const float* __restrict__ g2,
                const float* __restrict__ b2, float eps, T* __restrict__ x1) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float red[4];
   const int row = blockIdx.x;
   float4 v[LN_MAXV];
@@ -208,6 +229,8 @@ __global__ void __launch_bounds__(LN_THREADS)
 ln_rows_kernel(const float* __restrict__ h, int row_step, int row_off, int D,
                const float* __restrict__ g, const float* __restrict__ b, float eps,
                T* __restrict__ out) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float red[4];
   const int r = blockIdx.x;
   float4 v[LN_MAXV];
@@ -227,10 +250,9 @@ cudaError_t launch_ln_dual(int dt, const float* h, int M, int D, const float* g1
   if (M == 0) return cudaSuccess;
   if (D > LN_THREADS * 4 * LN_MAXV || (D % 4)) return cudaErrorInvalidValue;
   if (dt == DT_BF16)
-    ln_dual_kernel<bf16><<<M, LN_THREADS, 0, s>>>(h, D, g1, b1, g2, b2, eps, (bf16*)x1);
+    BT_LAUNCH(ln_dual_kernel<bf16>, dim3(M), dim3(LN_THREADS), 0, s, h, D, g1, b1, g2, b2, eps, (bf16*)x1);
   else
-    ln_dual_kernel<float><<<M, LN_THREADS, 0, s>>>(h, D, g1, b1, g2, b2, eps, (float*)x1);
-  note_launch();
+    BT_LAUNCH(ln_dual_kernel<float>, dim3(M), dim3(LN_THREADS), 0, s, h, D, g1, b1, g2, b2, eps, (float*)x1);
   return cudaGetLastError();
 }
 
@@ -239,10 +261,9 @@ cudaError_t launch_ln_rows(int dt, const float* h, int R, int row_step, int row_
   if (R == 0) return cudaSuccess;
   if (D > LN_THREADS * 4 * LN_MAXV || (D % 4)) return cudaErrorInvalidValue;
   if (dt == DT_BF16)
-    ln_rows_kernel<bf16><<<R, LN_THREADS, 0, s>>>(h, row_step, row_off, D, g, b, eps, (bf16*)out);
+    BT_LAUNCH(ln_rows_kernel<bf16>, dim3(R), dim3(LN_THREADS), 0, s, h, row_step, row_off, D, g, b, eps, (bf16*)out);
   else
-    ln_rows_kernel<float><<<R, LN_THREADS, 0, s>>>(h, row_step, row_off, D, g, b, eps, (float*)out);
-  note_launch();
+    BT_LAUNCH(ln_rows_kernel<float>, dim3(R), dim3(LN_THREADS), 0, s, h, row_step, row_off, D, g, b, eps, (float*)out);
   return cudaGetLastError();
 }
 
@@ -250,6 +271,8 @@ cudaError_t launch_ln_rows(int dt, const float* h, int R, int row_step, int row_
 // rotary table + rotary/append
 // ---------------------------------------------------------------------------
 __global__ void rope_table_kernel(float2* tab, int n_pos, int half, double base) {
+  pdl_trigger();
+  pdl_wait();
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= n_pos * half) return;
   const int p = idx / half, i = idx - p * half;
@@ -264,7 +287,7 @@ cudaError_t launch_rope_table(float2* tab, int n_pos, int rot, float base, cudaS
   const int half = rot / 2;
   if (half == 0 || n_pos == 0) return cudaSuccess;
   const int total = n_pos * half;
-  rope_table_kernel<<<(total + 255) / 256, 256, 0, s>>>(tab, n_pos, half, (double)base); note_launch();
+  BT_LAUNCH(rope_table_kernel, dim3((total + 255) / 256), dim3(256), 0, s, tab, n_pos, half, (double)base);
   return cudaGetLastError();
 }
 
@@ -273,6 +296,8 @@ __global__ void rope_append_kernel(const T* __restrict__ qkv, int D, int H, int 
                                    const float2* __restrict__ tab, PosSpec ps,
                                    T* __restrict__ q_out, T* __restrict__ kc,
                                    T* __restrict__ vc, int cap) {
+  pdl_trigger();
+  pdl_wait();
   const int m = blockIdx.x;
   const int d = D / H;
   const int half = rot >> 1;
@@ -304,13 +329,13 @@ cudaError_t launch_rope_append(int dt, const void* qkv, int M, int D, int H, int
                                void* v_cache, int cap, cudaStream_t s) {
   if (M == 0) return cudaSuccess;
   if (dt == DT_BF16) {
-    rope_append_kernel<bf16><<<M, 256, 0, s>>>((const bf16*)qkv, D, H, rot, rope_tab, pos,
-                                               (bf16*)q_out, (bf16*)k_cache, (bf16*)v_cache, cap); note_launch();
+    BT_LAUNCH(rope_append_kernel<bf16>, dim3(M), dim3(256), 0, s, (const bf16*)qkv, D, H, rot, rope_tab, pos,
+                                               (bf16*)q_out, (bf16*)k_cache, (bf16*)v_cache, cap);
   }
   else {
-    rope_append_kernel<float><<<M, 256, 0, s>>>((const float*)qkv, D, H, rot, rope_tab, pos,
+    BT_LAUNCH(rope_append_kernel<float>, dim3(M), dim3(256), 0, s, (const float*)qkv, D, H, rot, rope_tab, pos,
                                                 (float*)q_out, (float*)k_cache, (float*)v_cache,
-                                                cap); note_launch();
+                                                cap);
   }
   return cudaGetLastError();
 }
@@ -320,6 +345,8 @@ cudaError_t launch_rope_append(int dt, const void* qkv, int M, int D, int H, int
 // ---------------------------------------------------------------------------
 __global__ void argmax_kernel(const float* __restrict__ logits, int V, int ld,
                               int32_t* __restrict__ next) {
+  pdl_trigger();
+  pdl_wait();
   const int b = blockIdx.x;
   const float* z = logits + (size_t)b * ld;
   float best = -INFINITY;
@@ -356,12 +383,14 @@ __global__ void argmax_kernel(const float* __restrict__ logits, int V, int ld,
 cudaError_t launch_argmax(const float* logits, int B, int V, int ld, int32_t* next,
                           cudaStream_t s) {
   if (B == 0) return cudaSuccess;
-  argmax_kernel<<<B, 1024, 0, s>>>(logits, V, ld, next); note_launch();
+  BT_LAUNCH(argmax_kernel, dim3(B), dim3(1024), 0, s, logits, V, ld, next);
   return cudaGetLastError();
 }
 
 __global__ void argmax_reduce_kernel(const float2* __restrict__ part, int n_tiles, int M,
                                      int32_t* __restrict__ next) {
+  pdl_trigger();
+  pdl_wait();
   const int m = blockIdx.x;
   float best = -INFINITY;
   int bi = 0x7fffffff;
@@ -391,8 +420,7 @@ __global__ void argmax_reduce_kernel(const float2* __restrict__ part, int n_tile
 cudaError_t launch_argmax_reduce(const float2* part, int n_tiles, int M, int32_t* next,
                                  cudaStream_t s) {
   if (M == 0) return cudaSuccess;
-  argmax_reduce_kernel<<<M, 256, 0, s>>>(part, n_tiles, M, next);
-  note_launch();
+  BT_LAUNCH(argmax_reduce_kernel, dim3(M), dim3(256), 0, s, part, n_tiles, M, next);
   return cudaGetLastError();
 }
 
@@ -401,6 +429,8 @@ cudaError_t launch_argmax_reduce(const float2* part, int n_tiles, int M, int32_t
 // ---------------------------------------------------------------------------
 template <typename T>
 __global__ void convert_kernel(const T* __restrict__ src, float* __restrict__ dst, size_t n) {
+  pdl_trigger();
+  pdl_wait();
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n;
        i += (size_t)gridDim.x * blockDim.x)
     dst[i] = to_f(src[i]);
@@ -409,6 +439,8 @@ __global__ void convert_kernel(const T* __restrict__ src, float* __restrict__ ds
 template <typename T>
 __global__ void add_kernel(const T* __restrict__ a, const T* __restrict__ b,
                            float* __restrict__ dst, size_t n) {
+  pdl_trigger();
+  pdl_wait();
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n;
        i += (size_t)gridDim.x * blockDim.x)
     dst[i] = to_f(a[i]) + to_f(b[i]);
@@ -417,9 +449,8 @@ __global__ void add_kernel(const T* __restrict__ a, const T* __restrict__ b,
 cudaError_t launch_convert_to_f32(int dt, const void* src, float* dst, size_t n, cudaStream_t s) {
   if (n == 0) return cudaSuccess;
   const int grid = (int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
-  if (dt == DT_BF16) convert_kernel<bf16><<<grid, 256, 0, s>>>((const bf16*)src, dst, n);
-  else convert_kernel<float><<<grid, 256, 0, s>>>((const float*)src, dst, n);
-  note_launch();
+  if (dt == DT_BF16) BT_LAUNCH(convert_kernel<bf16>, dim3(grid), dim3(256), 0, s, (const bf16*)src, dst, n);
+  else BT_LAUNCH(convert_kernel<float>, dim3(grid), dim3(256), 0, s, (const float*)src, dst, n);
   return cudaGetLastError();
 }
 
@@ -427,9 +458,8 @@ cudaError_t launch_add_to_f32(int dt, const void* a, const void* b, float* dst, 
                               cudaStream_t s) {
   if (n == 0) return cudaSuccess;
   const int grid = (int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
-  if (dt == DT_BF16) add_kernel<bf16><<<grid, 256, 0, s>>>((const bf16*)a, (const bf16*)b, dst, n);
-  else add_kernel<float><<<grid, 256, 0, s>>>((const float*)a, (const float*)b, dst, n);
-  note_launch();
+  if (dt == DT_BF16) BT_LAUNCH(add_kernel<bf16>, dim3(grid), dim3(256), 0, s, (const bf16*)a, (const bf16*)b, dst, n);
+  else BT_LAUNCH(add_kernel<float>, dim3(grid), dim3(256), 0, s, (const float*)a, (const float*)b, dst, n);
   return cudaGetLastError();
 }
 

@@ -21,6 +21,8 @@ template <typename T>
 __global__ void __launch_bounds__(256)
 gemm_simt_kernel(const T* __restrict__ X, int ldx, const T* __restrict__ W, int ldw, int M,
                  int N, int K, int n_base, Epi e) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float sX[16][64 + 4];
   __shared__ float sW[16][64 + 4];
   const int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
@@ -89,12 +91,12 @@ cudaError_t launch_gemm(int dt, const void* X, int ldx, const void* W, int ldw, 
     const uint8_t* Wp = (const uint8_t*)W + (size_t)nb * ldw * es;
     dim3 grid((nn + 63) / 64, (M + 63) / 64);
     if (dt == DT_BF16) {
-      gemm_simt_kernel<bf16><<<grid, 256, 0, s>>>((const bf16*)Xp, ldx, (const bf16*)Wp, ldw, M,
-                                                  nn, K, nb, e); note_launch();
+      BT_LAUNCH(gemm_simt_kernel<bf16>, dim3(grid), dim3(256), 0, s, (const bf16*)Xp, ldx, (const bf16*)Wp, ldw, M,
+                                                  nn, K, nb, e);
     }
     else {
-      gemm_simt_kernel<float><<<grid, 256, 0, s>>>((const float*)Xp, ldx, (const float*)Wp, ldw,
-                                                   M, nn, K, nb, e); note_launch();
+      BT_LAUNCH(gemm_simt_kernel<float>, dim3(grid), dim3(256), 0, s, (const float*)Xp, ldx, (const float*)Wp, ldw,
+                                                   M, nn, K, nb, e);
     }
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return err;

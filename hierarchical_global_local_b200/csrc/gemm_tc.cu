@@ -180,26 +180,54 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
   // their first store into this CTA's shared memory
   if (ks > 1) cluster_arrive_relaxed();
 
+  pdl_trigger();
   if (warp == 4) {
     // ---- TMA producer ----
     if (lane == 0) {
       const uint32_t bytes = (uint32_t)stage_bytes<BN>();
-      int it = 0;
-      for (int t = t_first; t < ntiles; t += t_step) {
-        const int a0 = (t % ntA) * BM, b0 = (t / ntA) * BN;
-        const int koff = ((SWAP ? a0 : b0) >= xk_split) ? xk_off : 0;
-        for (int kb = kb_begin; kb < kb_end; ++kb, ++it) {
-          const int s = it % stages;
-          if (it >= stages) mbar_wait_bounded(&empty[s], ((it / stages) + 1) & 1, status);
-          mbar_arrive_expect_tx(&full[s], bytes);
-          const int k = kb * BK;
-          tma_load_2d(sA + (size_t)s * BM * BK, &mapA, k + (SWAP ? 0 : koff), a0, &full[s]);
-          tma_load_2d(sB + (size_t)s * BN * BK, &mapB, k + (SWAP ? koff : 0), b0, &full[s]);
-        }
+      const int nloc = kb_end - kb_begin;
+      const int my_tiles = (t_first < ntiles) ? (ntiles - t_first + t_step - 1) / t_step : 0;
+      const int total = my_tiles * nloc;
+      // load iteration -> (A row, B row, K column of the weights, activation K offset)
+      auto coords = [&](int it, int& a0, int& b0, int& k, int& koff) {
+        const int t = t_first + (it / nloc) * t_step;
+        a0 = (t % ntA) * BM;
+        b0 = (t / ntA) * BN;
+        k = (kb_begin + it % nloc) * BK;
+        koff = ((SWAP ? a0 : b0) >= xk_split) ? xk_off : 0;
+      };
+      auto load_w = [&](int it, int s) {  // the weight operand
+        int a0, b0, k, koff;
+        coords(it, a0, b0, k, koff);
+        if (SWAP) tma_load_2d(sA + (size_t)s * BM * BK, &mapA, k, a0, &full[s]);
+        else tma_load_2d(sB + (size_t)s * BN * BK, &mapB, k, b0, &full[s]);
+      };
+      auto load_x = [&](int it, int s) {  // the activation operand
+        int a0, b0, k, koff;
+        coords(it, a0, b0, k, koff);
+        if (SWAP) tma_load_2d(sB + (size_t)s * BN * BK, &mapB, k + koff, b0, &full[s]);
+        else tma_load_2d(sA + (size_t)s * BM * BK, &mapA, k + koff, a0, &full[s]);
+      };
+      // weights do not depend on earlier kernels: fill the first ring with
+      // them while the previous kernel finishes, then wait for it
+      const int pre = total < stages ? total : stages;
+      for (int it = 0; it < pre; ++it) {
+        mbar_arrive_expect_tx(&full[it], bytes);
+        load_w(it, it);
+      }
+      pdl_wait();
+      for (int it = 0; it < pre; ++it) load_x(it, it);
+      for (int it = pre; it < total; ++it) {
+        const int s = it % stages;
+        mbar_wait_bounded(&empty[s], ((it / stages) + 1) & 1, status);
+        mbar_arrive_expect_tx(&full[s], bytes);
+        load_w(it, s);
+        load_x(it, s);
       }
     }
   } else if (warp == 5) {
     // ---- MMA issuer ----
+    pdl_wait();
     if (lane == 0) {
       constexpr uint32_t idesc = instr_desc<BN>();
       int it = 0, tl = 0;
@@ -224,6 +252,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
     }
   } else {
     // ---- epilogue warps 0-3: TMEM lanes 32w..32w+31 ----
+    pdl_wait();  // outputs may still be read by earlier kernels
     const int r = warp * 32 + lane;  // row of A = TMEM lane
     const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
     // fused rotary: the rotate-half partner of feature f is f ^ (rot/2), held
@@ -480,13 +509,15 @@ cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& mb, int M, int 
   cfg.blockDim = dim3(THREADS, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 1;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = ks;  // the K splits of one tile form a cluster
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = pdl_enabled() ? 2 : 1;
   cudaError_t err = cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN, SWAP>, ma, mb, M, N, nkb, ks,
                                        stages, ntA, ntB, xk_split, xk_off, e, status);
   note_launch();

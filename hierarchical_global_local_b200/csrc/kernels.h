@@ -151,6 +151,36 @@ void note_cuda_error(const char* what, cudaError_t e);
 void note_launch();
 long long launch_count();
 
+// Programmatic dependent launch on every kernel (on unless BT_NO_PDL=1).
+bool pdl_enabled();
+
+// Launch through cudaLaunchKernelEx with the programmatic-serialization
+// attribute (the kernel overlaps its prologue with the previous kernel's
+// tail; see pdl_trigger / pdl_wait) and count it.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                      cudaStream_t s, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
+  note_launch();
+  return e;
+}
+
+#define BT_LAUNCH(...)                               \
+  do {                                               \
+    cudaError_t e_ = ::bt::launch_ex(__VA_ARGS__);   \
+    if (e_ != cudaSuccess) return e_;                \
+  } while (0)
+
 // ---- misc -----------------------------------------------------------------
 cudaError_t launch_convert_to_f32(int dt, const void* src, float* dst, size_t n, cudaStream_t s);
 cudaError_t launch_add_to_f32(int dt, const void* a, const void* b, float* dst, size_t n,
