@@ -23,17 +23,26 @@ namespace bt {
 // ---------------------------------------------------------------------------
 // split-K decode attention
 // ---------------------------------------------------------------------------
+// A work unit is one (sequence, head) pair and a contiguous range of its
+// cached rows, streamed in CHUNK-row pieces (8 KB of K + 8 KB of V) through a
+// STAGES-deep ring of 1-D bulk copies, with an online softmax across chunks.
+// Pairs are split into several units only when there are too few pairs to
+// keep every SM busy; split units are merged by the last one to finish.
 template <typename T, int DH>
 struct DecCfg {
   static constexpr int ROW_BYTES = DH * (int)sizeof(T);
-  static constexpr int CHUNK = 16384 / ROW_BYTES;        // rows per split (16 KB of K)
+  static constexpr int CHUNK = 8192 / ROW_BYTES;         // rows per chunk (8 KB of K)
+  static constexpr int STAGES = 4;
   static constexpr int TPR = ROW_BYTES / 16;             // threads per row, 16 B each
   static constexpr int THREADS = 128;
   static constexpr int RPP = THREADS / TPR;              // rows per pass
   static constexpr int EPT = 16 / (int)sizeof(T);        // elements per thread
-  static constexpr int SMEM = 2 * CHUNK * ROW_BYTES + CHUNK * 4 + RPP * DH * 4;
+  static constexpr int SMEM = STAGES * 2 * CHUNK * ROW_BYTES + CHUNK * 4 + RPP * DH * 4;
   static_assert(TPR >= 1 && TPR <= 32 && (32 % TPR) == 0, "row split");
+  static_assert(DH <= THREADS, "one thread per output dim in the final reduction");
 };
+
+constexpr int DEC_UNITS_SLACK = 4096;  // work units beyond one per pair (scratch sizing)
 
 __device__ __forceinline__ float block_reduce_max128(float v, float* red) {
   v = warp_max(v);
@@ -59,45 +68,50 @@ __global__ void __launch_bounds__(128)
 attn_decode_kernel(const T* __restrict__ q, int ldq, const T* __restrict__ kc,
                    const T* __restrict__ vc, int H, int cap, PosSpec kvlen, T* __restrict__ out,
                    int ld_out, float* __restrict__ part, int* __restrict__ counters,
-                   int max_splits, int* status, float qscale) {
+                   int splits, int* status, float qscale) {
   pdl_trigger();
   pdl_wait();
   using C = DecCfg<T, DH>;
   const int pair = blockIdx.x;  // b * H + h
-  const int split = blockIdx.y;
+  const int z = blockIdx.y;
   const int b = pair / H, h = pair - b * H;
   const int n = pos_base(kvlen) + 1;
-  const int nsplit = (n + C::CHUNK - 1) / C::CHUNK;
-  if (split >= nsplit) return;
-  const int r0 = split * C::CHUNK;
-  const int rows = min(C::CHUNK, n - r0);
+  const int nchunks = (n + C::CHUNK - 1) / C::CHUNK;
+  const int S = splits < nchunks ? splits : nchunks;  // non-empty units of this pair
+  if (z >= S) return;
+  const int c_begin = (int)(((long long)z * nchunks) / S);
+  const int c_end = (int)(((long long)(z + 1) * nchunks) / S);
+  const int nc = c_end - c_begin;
 
   extern __shared__ __align__(128) uint8_t smem[];
-  T* sK = reinterpret_cast<T*>(smem);
-  T* sV = reinterpret_cast<T*>(smem + C::CHUNK * C::ROW_BYTES);
-  float* sS = reinterpret_cast<float*>(smem + 2 * C::CHUNK * C::ROW_BYTES);
+  T* sKV = reinterpret_cast<T*>(smem);  // [STAGES][K chunk | V chunk]
+  float* sS = reinterpret_cast<float*>(smem + C::STAGES * 2 * C::CHUNK * C::ROW_BYTES);
   float* sO = sS + C::CHUNK;
-  __shared__ __align__(8) uint64_t bar;
+  __shared__ __align__(8) uint64_t full[C::STAGES];
   __shared__ float red[4];
   __shared__ int s_last;
 
   const int tid = threadIdx.x;
-  const size_t base = ((size_t)pair * cap + r0) * DH;
-  if (tid == 0) {
-    mbar_init(&bar, 1);
-    fence_mbar_init();
-  }
-  __syncthreads();
-  if (tid == 0) {
+  const size_t pair_base = (size_t)pair * cap * DH;
+  auto issue = [&](int i, int s) {  // chunk c_begin + i -> stage s
+    const int r0 = (c_begin + i) * C::CHUNK;
+    const int rows = min(C::CHUNK, n - r0);
     const uint32_t bytes = (uint32_t)rows * C::ROW_BYTES;
-    mbar_arrive_expect_tx(&bar, 2 * bytes);
-    bulk_g2s(sK, kc + base, bytes, &bar);
-    bulk_g2s(sV, vc + base, bytes, &bar);
+    T* dk = sKV + (size_t)s * 2 * C::CHUNK * DH;
+    mbar_arrive_expect_tx(&full[s], 2 * bytes);
+    bulk_g2s(dk, kc + pair_base + (size_t)r0 * DH, bytes, &full[s]);
+    bulk_g2s(dk + C::CHUNK * DH, vc + pair_base + (size_t)r0 * DH, bytes, &full[s]);
+  };
+  if (tid == 0) {
+    for (int s = 0; s < C::STAGES; ++s) mbar_init(&full[s], 1);
+    fence_mbar_init();
+    for (int i = 0; i < nc && i < C::STAGES; ++i) issue(i, i);
   }
 
   // this thread's slice of q (16 bytes), scaled by log2(e)/sqrt(d)
   const int g = tid / C::TPR;
   const int e0 = (tid % C::TPR) * C::EPT;
+  const bool row_leader = (tid % C::TPR) == 0;
   float qf[C::EPT];
   {
     const uint4 u = *reinterpret_cast<const uint4*>(q + (size_t)b * ldq + h * DH + e0);
@@ -105,80 +119,88 @@ attn_decode_kernel(const T* __restrict__ q, int ldq, const T* __restrict__ kc,
 #pragma unroll
     for (int i = 0; i < C::EPT; ++i) qf[i] *= qscale;
   }
+  __syncthreads();  // barriers initialised before anyone waits on them
 
-  if (!mbar_wait_bounded(&bar, 0, status)) {
-    mbar_wait_bounded(&bar, 0, status);  // second bounded wait for the copies in flight
-    return;
-  }
-
-  // scores s_r = q . k_r (log2 domain). The trip count is the same for every
-  // thread of the CTA (rows and RPP are uniform) so the full-warp shuffles
-  // below never see a partial warp; rows past the end contribute nothing.
-  for (int rb = 0; rb < rows; rb += C::RPP) {
-    const int r = rb + g;
-    const bool valid = r < rows;
-    float s = 0.f;
-    if (valid) {
-      const uint4 u = *reinterpret_cast<const uint4*>(sK + r * DH + e0);
-      float kf[C::EPT];
-      unpack16(u, kf, (const T*)nullptr);
-#pragma unroll
-      for (int i = 0; i < C::EPT; ++i) s = fmaf(qf[i], kf[i], s);
-    }
-#pragma unroll
-    for (int o = C::TPR / 2; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    if (valid && (tid % C::TPR) == 0) sS[r] = s;
-  }
-  __syncthreads();
-  float mx = -FLT_MAX;
-  for (int r = tid; r < rows; r += C::THREADS) mx = fmaxf(mx, sS[r]);
-  const float M = block_reduce_max128(mx, red);
-  float l = 0.f;
-  for (int r = tid; r < rows; r += C::THREADS) {
-    const float p = exp2f(sS[r] - M);
-    sS[r] = p;
-    l += p;
-  }
-  const float L = block_reduce_sum128(l, red);  // contains __syncthreads: sS visible
-
+  float M = -FLT_MAX, l = 0.f;
   float of[C::EPT];
 #pragma unroll
   for (int i = 0; i < C::EPT; ++i) of[i] = 0.f;
-  for (int r = g; r < rows; r += C::RPP) {
-    const float p = sS[r];
-    const uint4 u = *reinterpret_cast<const uint4*>(sV + r * DH + e0);
-    float vf[C::EPT];
-    unpack16(u, vf, (const T*)nullptr);
+  bool ok = true;
+
+  for (int i = 0; i < nc; ++i) {
+    const int s = i % C::STAGES;
+    if (!mbar_wait_bounded(&full[s], (i / C::STAGES) & 1, status)) ok = false;
+    const T* sK = sKV + (size_t)s * 2 * C::CHUNK * DH;
+    const T* sV = sK + C::CHUNK * DH;
+    const int rows = min(C::CHUNK, n - (c_begin + i) * C::CHUNK);
+    // scores s_r = q . k_r (log2 domain); the trip count is uniform across the
+    // CTA so every full-warp shuffle sees the whole warp
+    float cmax = -FLT_MAX;
+    for (int rb = 0; rb < rows; rb += C::RPP) {
+      const int r = rb + g;
+      const bool valid = r < rows;
+      float sc = 0.f;
+      if (valid) {
+        const uint4 u = *reinterpret_cast<const uint4*>(sK + r * DH + e0);
+        float kf[C::EPT];
+        unpack16(u, kf, (const T*)nullptr);
 #pragma unroll
-    for (int i = 0; i < C::EPT; ++i) of[i] = fmaf(p, vf[i], of[i]);
+        for (int e = 0; e < C::EPT; ++e) sc = fmaf(qf[e], kf[e], sc);
+      }
+#pragma unroll
+      for (int o = C::TPR / 2; o > 0; o >>= 1) sc += __shfl_xor_sync(0xffffffffu, sc, o);
+      if (valid) {
+        cmax = fmaxf(cmax, sc);
+        if (row_leader) sS[r] = sc;
+      }
+    }
+    const float Mn = fmaxf(M, block_reduce_max128(cmax, red));  // syncs: sS complete
+    const float scale = exp2f(M - Mn);
+    l *= scale;
+#pragma unroll
+    for (int e = 0; e < C::EPT; ++e) of[e] *= scale;
+    for (int r = g; r < rows; r += C::RPP) {
+      const float p = exp2f(sS[r] - Mn);
+      if (row_leader) l += p;
+      const uint4 u = *reinterpret_cast<const uint4*>(sV + r * DH + e0);
+      float vf[C::EPT];
+      unpack16(u, vf, (const T*)nullptr);
+#pragma unroll
+      for (int e = 0; e < C::EPT; ++e) of[e] = fmaf(p, vf[e], of[e]);
+    }
+    M = Mn;
+    __syncthreads();  // stage s and sS free again
+    if (tid == 0 && i + C::STAGES < nc) issue(i + C::STAGES, s);
   }
+  if (!ok) return;  // a copy never arrived: status is set, output left as is
+
+  // combine the RPP row groups: o per dim, l over the CTA
 #pragma unroll
-  for (int i = 0; i < C::EPT; ++i) sO[g * DH + e0 + i] = of[i];
-  __syncthreads();
+  for (int e = 0; e < C::EPT; ++e) sO[g * DH + e0 + e] = of[e];
+  const float L = block_reduce_sum128(l, red);  // contains the barrier for sO
   float o_d = 0.f;
   if (tid < DH) {
     for (int gg = 0; gg < C::RPP; ++gg) o_d += sO[gg * DH + tid];
   }
-
-  if (nsplit == 1) {
+  if (S == 1) {
     if (tid < DH) out[(size_t)b * ld_out + h * DH + tid] = from_f<T>(o_d / L);
     return;
   }
-  float* my = part + ((size_t)pair * max_splits + split) * (DH + 2);
+  float* my = part + ((size_t)pair * splits + z) * (DH + 2);
   if (tid < DH) my[2 + tid] = o_d;
   if (tid == 0) { my[0] = M; my[1] = L; }
   __threadfence();
   __syncthreads();
-  if (tid == 0) s_last = (atomicAdd(&counters[pair], 1) == nsplit - 1);
+  if (tid == 0) s_last = (atomicAdd(&counters[pair], 1) == S - 1);
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  const float* pp = part + (size_t)pair * max_splits * (DH + 2);
+  const float* pp = part + (size_t)pair * splits * (DH + 2);
   float Mg = -FLT_MAX;
-  for (int s = 0; s < nsplit; ++s) Mg = fmaxf(Mg, __ldcg(pp + (size_t)s * (DH + 2)));
+  for (int u = 0; u < S; ++u) Mg = fmaxf(Mg, __ldcg(pp + (size_t)u * (DH + 2)));
   float Lg = 0.f, og = 0.f;
-  for (int s = 0; s < nsplit; ++s) {
-    const float* ps = pp + (size_t)s * (DH + 2);
+  for (int u = 0; u < S; ++u) {
+    const float* ps = pp + (size_t)u * (DH + 2);
     const float w = exp2f(__ldcg(ps) - Mg);
     Lg = fmaf(w, __ldcg(ps + 1), Lg);
     if (tid < DH) og = fmaf(w, __ldcg(ps + 2 + tid), og);
@@ -187,21 +209,63 @@ attn_decode_kernel(const T* __restrict__ q, int ldq, const T* __restrict__ kc,
   if (tid == 0) counters[pair] = 0;
 }
 
+static int dec_sm_count() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
 template <typename T>
 static int dec_chunk(int d) {
-  return 16384 / (d * (int)sizeof(T));
+  return 8192 / (d * (int)sizeof(T));
 }
 
-int attn_decode_max_splits(int d, int cap, int dt) {
+// Units per pair: about two work units per resident CTA slot (3 per SM),
+// never more than the pair has chunks.
+static int dec_splits(int pairs, int d, int cap, int dt) {
   const int chunk = dt == DT_BF16 ? dec_chunk<bf16>(d) : dec_chunk<float>(d);
-  return (cap + chunk - 1) / chunk;
+  const int max_chunks = (cap + chunk - 1) / chunk;
+  const int target = 2 * 3 * dec_sm_count();
+  int sp = (target + pairs - 1) / pairs;
+  if (sp > max_chunks) sp = max_chunks;
+  if ((long long)pairs * sp > (long long)pairs + DEC_UNITS_SLACK) sp = 1 + DEC_UNITS_SLACK / pairs;
+  return sp < 1 ? 1 : sp;
 }
 
+int attn_decode_max_splits(int d, int cap, int dt) { return dec_splits(1, d, cap, dt); }
+
+// scratch layout: [merge counters: B*H ints, 256-aligned][partials:
+// (B*H + slack) units x (d + 2) floats]; counters sit at offset 0 for any B.
 size_t attn_decode_scratch_bytes(int B, int H, int d, int cap, int dt) {
-  const size_t ms = (size_t)attn_decode_max_splits(d, cap, dt);
-  const size_t part = (size_t)B * H * ms * (d + 2) * sizeof(float);
-  const size_t part_al = (part + 255) & ~(size_t)255;
-  return part_al + (size_t)B * H * sizeof(int);
+  const size_t cnt = ((size_t)B * H * sizeof(int) + 255) & ~(size_t)255;
+  const size_t units = (size_t)B * H + DEC_UNITS_SLACK;
+  return cnt + units * (d + 2) * sizeof(float);
+}
+
+template <typename T, int DH>
+static cudaError_t dec_prepare() {
+  static bool done = false;
+  if (done) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(attn_decode_kernel<T, DH>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       DecCfg<T, DH>::SMEM);
+  if (e == cudaSuccess) done = true;
+  return e;
+}
+
+cudaError_t attn_prepare() {
+  cudaError_t e;
+  if ((e = dec_prepare<bf16, 32>()) != cudaSuccess) return e;
+  if ((e = dec_prepare<bf16, 64>()) != cudaSuccess) return e;
+  if ((e = dec_prepare<bf16, 128>()) != cudaSuccess) return e;
+  if ((e = dec_prepare<float, 32>()) != cudaSuccess) return e;
+  if ((e = dec_prepare<float, 64>()) != cudaSuccess) return e;
+  return dec_prepare<float, 128>();
 }
 
 template <typename T, int DH>
@@ -209,17 +273,19 @@ static cudaError_t launch_dec(const void* q, int ldq, const void* kc, const void
                               int H, int cap, PosSpec kvlen, void* out, int ld_out,
                               void* scratch, int* status, cudaStream_t s) {
   using C = DecCfg<T, DH>;
-  const int ms = (cap + C::CHUNK - 1) / C::CHUNK;
-  const size_t part = (size_t)B * H * ms * (DH + 2) * sizeof(float);
-  float* partp = reinterpret_cast<float*>(scratch);
-  int* counters = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(scratch) +
-                                         ((part + 255) & ~(size_t)255));
-  dim3 grid(B * H, ms);
+  cudaError_t e = dec_prepare<T, DH>();
+  if (e != cudaSuccess) return e;
+  const int pairs = B * H;
+  const int sp = dec_splits(pairs, DH, cap, sizeof(T) == 2 ? DT_BF16 : DT_F32);
+  int* counters = reinterpret_cast<int*>(scratch);
+  float* partp = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(scratch) +
+                                          (((size_t)pairs * sizeof(int) + 255) & ~(size_t)255));
+  dim3 grid(pairs, sp);
   const float qscale = 1.4426950408889634f / sqrtf((float)DH);
-  BT_LAUNCH(attn_decode_kernel<T, DH>, dim3(grid), dim3(C::THREADS), C::SMEM, s, 
-      (const T*)q, ldq, (const T*)kc, (const T*)vc, H, cap, kvlen, (T*)out, ld_out, partp,
-      counters, ms, status, qscale);
-  return cudaGetLastError();
+  BT_LAUNCH(attn_decode_kernel<T, DH>, grid, dim3(C::THREADS), C::SMEM, s, (const T*)q, ldq,
+            (const T*)kc, (const T*)vc, H, cap, kvlen, (T*)out, ld_out, partp, counters, sp,
+            status, qscale);
+  return cudaSuccess;
 }
 
 cudaError_t launch_attn_decode(int dt, const void* q, int ldq, const void* k_cache,

@@ -55,6 +55,8 @@ cudaError_t launch_rope_table(float2* tab, int n_pos, int rot, float base, cudaS
 // part / counters: scratch of attn_decode_scratch_bytes(); counters must be
 // zero before the first launch and are left zero.
 size_t attn_decode_scratch_bytes(int B, int H, int d, int cap, int dt);
+// One-time setup of the decode-attention kernels (shared-memory limits).
+cudaError_t attn_prepare();
 int attn_decode_max_splits(int d, int cap, int dt);
 cudaError_t launch_attn_decode(int dt, const void* q, int ldq, const void* k_cache,
                                const void* v_cache, int B, int H, int d, int cap,

@@ -343,6 +343,7 @@ int bt_create(const bt_config* cfg, const bt_weights* w, void* ws, size_t ws_byt
   BT_TRYC(cudaMemsetAsync(m->block_tok, 0, (size_t)d.Bmax * d.L * 4, st));
   BT_TRYC(cudaStreamCreateWithFlags(&m->cap_stream, cudaStreamNonBlocking));
   if (d.dt == BT_BF16) BT_TRYC(gemm_tc_prepare());
+  BT_TRYC(attn_prepare());
 #undef BT_TRY
 #undef BT_TRYC
   *out = m;
@@ -533,6 +534,9 @@ int bt_prefill(bt_model* m, const int32_t* tokens, int32_t B, int32_t T, float* 
   m->t = T;
   const int n = T / d.L;
   const int M = B * n;
+  // a new session: merge counters of the decode attention start from zero
+  BT_CUDA(cudaMemsetAsync(m->attn_scratch, 0,
+                          attn_decode_scratch_bytes(d.Bmax, d.H, d.d, d.n_cap, d.dt), s));
   const long long k0 = launch_count();
   BT_CUDA(launch_set_state(m->dstate, T, d.L, s));
   {

@@ -30,7 +30,8 @@ extern "C" {
  *   out_dev     [B, ld_out] dtype; out[b*ld_out + h*d + e]
  *   softmax(q k^T / sqrt(d)) v over the n entries, per (b, h).
  *   scratch_dev >= bt_op_decode_attention_scratch_bytes(...) bytes, 256-byte
- *   aligned, zero-filled before its first use (the call leaves it reusable).
+ *   aligned, zero-filled before its first use; the call leaves it ready for
+ *   further calls with the same B and H (re-zero it when B or H changes).
  * Requires d in {32, 64, 128}, 1 <= n <= cap, 16-byte aligned rows.
  * Calls that share a scratch buffer must not overlap on the GPU. */
 BT_API size_t bt_op_decode_attention_scratch_bytes(int dtype, int B, int H, int d, int cap);
