@@ -63,25 +63,36 @@ __device__ __forceinline__ float block_reduce_sum128(float v, float* red) {
   return v;
 }
 
+// Persistent, stream-K over the flattened list of (pair, chunk) work: CTA c of
+// G handles chunks [floor(c*T/G), floor((c+1)*T/G)) of the T = pairs * nch
+// chunks, its copy ring running straight across pair boundaries. A pair whose
+// chunks span several CTAs gets one partial (m, l, o) from each; the last to
+// finish (atomic counter, no waiting) merges them in CTA order.
+__device__ __forceinline__ int dec_owner(long long x, int G, long long T) {
+  // the CTA whose chunk range contains chunk x
+  return (int)(((x + 1) * G + T - 1) / T) - 1;
+}
+
 template <typename T, int DH>
 __global__ void __launch_bounds__(128)
 attn_decode_kernel(const T* __restrict__ q, int ldq, const T* __restrict__ kc,
-                   const T* __restrict__ vc, int H, int cap, PosSpec kvlen, T* __restrict__ out,
-                   int ld_out, float* __restrict__ part, int* __restrict__ counters,
-                   int splits, int* status, float qscale) {
+                   const T* __restrict__ vc, int pairs, int H, int cap, PosSpec kvlen,
+                   T* __restrict__ out, int ld_out, float* __restrict__ part,
+                   int* __restrict__ counters, int* status, float qscale) {
   pdl_trigger();
   pdl_wait();
   using C = DecCfg<T, DH>;
-  const int pair = blockIdx.x;  // b * H + h
-  const int z = blockIdx.y;
-  const int b = pair / H, h = pair - b * H;
   const int n = pos_base(kvlen) + 1;
-  const int nchunks = (n + C::CHUNK - 1) / C::CHUNK;
-  const int S = splits < nchunks ? splits : nchunks;  // non-empty units of this pair
-  if (z >= S) return;
-  const int c_begin = (int)(((long long)z * nchunks) / S);
-  const int c_end = (int)(((long long)(z + 1) * nchunks) / S);
-  const int nc = c_end - c_begin;
+  const int nch = (n + C::CHUNK - 1) / C::CHUNK;
+  const long long Ttot = (long long)pairs * nch;
+  // effective grid <= chunks, so that every CTA's range is non-empty and the
+  // CTAs sharing a pair are consecutive
+  const int G = (int)((long long)gridDim.x < Ttot ? (long long)gridDim.x : Ttot);
+  const int c = blockIdx.x;
+  if (c >= G) return;
+  const long long x0 = (long long)c * Ttot / G, x1 = (long long)(c + 1) * Ttot / G;
+  const int nc = (int)(x1 - x0);
+  if (nc <= 0) return;
 
   extern __shared__ __align__(128) uint8_t smem[];
   T* sKV = reinterpret_cast<T*>(smem);  // [STAGES][K chunk | V chunk]
@@ -92,121 +103,135 @@ attn_decode_kernel(const T* __restrict__ q, int ldq, const T* __restrict__ kc,
   __shared__ int s_last;
 
   const int tid = threadIdx.x;
-  const size_t pair_base = (size_t)pair * cap * DH;
-  auto issue = [&](int i, int s) {  // chunk c_begin + i -> stage s
-    const int r0 = (c_begin + i) * C::CHUNK;
+  auto issue = [&](int i, int s) {  // chunk x0 + i -> stage s
+    const long long x = x0 + i;
+    const int pr = (int)(x / nch), ci = (int)(x - (long long)pr * nch);
+    const int r0 = ci * C::CHUNK;
     const int rows = min(C::CHUNK, n - r0);
     const uint32_t bytes = (uint32_t)rows * C::ROW_BYTES;
+    const size_t off = ((size_t)pr * cap + r0) * DH;
     T* dk = sKV + (size_t)s * 2 * C::CHUNK * DH;
     mbar_arrive_expect_tx(&full[s], 2 * bytes);
-    bulk_g2s(dk, kc + pair_base + (size_t)r0 * DH, bytes, &full[s]);
-    bulk_g2s(dk + C::CHUNK * DH, vc + pair_base + (size_t)r0 * DH, bytes, &full[s]);
+    bulk_g2s(dk, kc + off, bytes, &full[s]);
+    bulk_g2s(dk + C::CHUNK * DH, vc + off, bytes, &full[s]);
   };
   if (tid == 0) {
     for (int s = 0; s < C::STAGES; ++s) mbar_init(&full[s], 1);
     fence_mbar_init();
     for (int i = 0; i < nc && i < C::STAGES; ++i) issue(i, i);
   }
+  __syncthreads();  // barriers initialised before anyone waits on them
 
-  // this thread's slice of q (16 bytes), scaled by log2(e)/sqrt(d)
   const int g = tid / C::TPR;
   const int e0 = (tid % C::TPR) * C::EPT;
   const bool row_leader = (tid % C::TPR) == 0;
-  float qf[C::EPT];
-  {
-    const uint4 u = *reinterpret_cast<const uint4*>(q + (size_t)b * ldq + h * DH + e0);
-    unpack16(u, qf, (const T*)nullptr);
-#pragma unroll
-    for (int i = 0; i < C::EPT; ++i) qf[i] *= qscale;
-  }
-  __syncthreads();  // barriers initialised before anyone waits on them
-
-  float M = -FLT_MAX, l = 0.f;
-  float of[C::EPT];
-#pragma unroll
-  for (int i = 0; i < C::EPT; ++i) of[i] = 0.f;
+  const int first_pair = (int)(x0 / nch);
   bool ok = true;
-
-  for (int i = 0; i < nc; ++i) {
-    const int s = i % C::STAGES;
-    if (!mbar_wait_bounded(&full[s], (i / C::STAGES) & 1, status)) ok = false;
-    const T* sK = sKV + (size_t)s * 2 * C::CHUNK * DH;
-    const T* sV = sK + C::CHUNK * DH;
-    const int rows = min(C::CHUNK, n - (c_begin + i) * C::CHUNK);
-    // scores s_r = q . k_r (log2 domain); the trip count is uniform across the
-    // CTA so every full-warp shuffle sees the whole warp
-    float cmax = -FLT_MAX;
-    for (int rb = 0; rb < rows; rb += C::RPP) {
-      const int r = rb + g;
-      const bool valid = r < rows;
-      float sc = 0.f;
-      if (valid) {
-        const uint4 u = *reinterpret_cast<const uint4*>(sK + r * DH + e0);
-        float kf[C::EPT];
-        unpack16(u, kf, (const T*)nullptr);
+  int i = 0;
+  for (int pr = first_pair; i < nc; ++pr) {
+    // chunks of pair pr inside this CTA's range: [i, i + cnt)
+    const long long pend = (long long)(pr + 1) * nch;
+    const int cnt = (int)((pend < x1 ? pend : x1) - (x0 + i));
+    const int b = pr / H, h = pr - b * H;
+    float qf[C::EPT];
+    {
+      const uint4 u = *reinterpret_cast<const uint4*>(q + (size_t)b * ldq + h * DH + e0);
+      unpack16(u, qf, (const T*)nullptr);
 #pragma unroll
-        for (int e = 0; e < C::EPT; ++e) sc = fmaf(qf[e], kf[e], sc);
+      for (int e = 0; e < C::EPT; ++e) qf[e] *= qscale;
+    }
+    float M = -FLT_MAX, l = 0.f;
+    float of[C::EPT];
+#pragma unroll
+    for (int e = 0; e < C::EPT; ++e) of[e] = 0.f;
+    for (int k = 0; k < cnt; ++k, ++i) {
+      const int s = i % C::STAGES;
+      if (!mbar_wait_bounded(&full[s], (i / C::STAGES) & 1, status)) ok = false;
+      const T* sK = sKV + (size_t)s * 2 * C::CHUNK * DH;
+      const T* sV = sK + C::CHUNK * DH;
+      const long long x = x0 + i;
+      const int rows = min(C::CHUNK, n - (int)(x - (long long)pr * nch) * C::CHUNK);
+      // scores (log2 domain); uniform trip count -> whole-warp shuffles
+      float cmax = -FLT_MAX;
+      for (int rb = 0; rb < rows; rb += C::RPP) {
+        const int r = rb + g;
+        const bool valid = r < rows;
+        float sc = 0.f;
+        if (valid) {
+          const uint4 u = *reinterpret_cast<const uint4*>(sK + r * DH + e0);
+          float kf[C::EPT];
+          unpack16(u, kf, (const T*)nullptr);
+#pragma unroll
+          for (int e = 0; e < C::EPT; ++e) sc = fmaf(qf[e], kf[e], sc);
+        }
+#pragma unroll
+        for (int o = C::TPR / 2; o > 0; o >>= 1) sc += __shfl_xor_sync(0xffffffffu, sc, o);
+        if (valid) {
+          cmax = fmaxf(cmax, sc);
+          if (row_leader) sS[r] = sc;
+        }
       }
+      const float Mn = fmaxf(M, block_reduce_max128(cmax, red));  // syncs: sS complete
+      const float scale = exp2f(M - Mn);
+      l *= scale;
 #pragma unroll
-      for (int o = C::TPR / 2; o > 0; o >>= 1) sc += __shfl_xor_sync(0xffffffffu, sc, o);
-      if (valid) {
-        cmax = fmaxf(cmax, sc);
-        if (row_leader) sS[r] = sc;
+      for (int e = 0; e < C::EPT; ++e) of[e] *= scale;
+      for (int r = g; r < rows; r += C::RPP) {
+        const float p = exp2f(sS[r] - Mn);
+        if (row_leader) l += p;
+        const uint4 u = *reinterpret_cast<const uint4*>(sV + r * DH + e0);
+        float vf[C::EPT];
+        unpack16(u, vf, (const T*)nullptr);
+#pragma unroll
+        for (int e = 0; e < C::EPT; ++e) of[e] = fmaf(p, vf[e], of[e]);
+      }
+      M = Mn;
+      __syncthreads();  // stage s and sS free again
+      if (tid == 0 && i + C::STAGES < nc) issue(i + C::STAGES, s);
+    }
+    // this CTA's share of pair pr: combine the row groups
+#pragma unroll
+    for (int e = 0; e < C::EPT; ++e) sO[g * DH + e0 + e] = of[e];
+    const float L = block_reduce_sum128(l, red);  // barrier for sO
+    float o_d = 0.f;
+    if (tid < DH) {
+      for (int gg = 0; gg < C::RPP; ++gg) o_d += sO[gg * DH + tid];
+    }
+    const long long pbeg = (long long)pr * nch;
+    const int first = dec_owner(pbeg, G, Ttot), last = dec_owner(pbeg + nch - 1, G, Ttot);
+    if (first == last) {
+      if (ok && tid < DH) out[(size_t)b * ld_out + h * DH + tid] = from_f<T>(o_d / L);
+    } else {
+      // partial slot: 2c if pair pr is where this CTA's range starts, else 2c + 1
+      float* my = part + ((size_t)2 * c + (pr == first_pair ? 0 : 1)) * (DH + 2);
+      if (tid < DH) my[2 + tid] = o_d;
+      if (tid == 0) { my[0] = M; my[1] = L; }
+      __threadfence();
+      __syncthreads();
+      if (tid == 0) s_last = (atomicAdd(&counters[pr], 1) == last - first);
+      __syncthreads();
+      if (s_last) {
+        __threadfence();
+        float Mg = -FLT_MAX;
+        for (int cc = first; cc <= last; ++cc) {
+          const int first_of_cc = (int)(((long long)cc * Ttot / G) / nch);
+          const float* ps = part + ((size_t)2 * cc + (pr == first_of_cc ? 0 : 1)) * (DH + 2);
+          Mg = fmaxf(Mg, __ldcg(ps));
+        }
+        float Lg = 0.f, og = 0.f;
+        for (int cc = first; cc <= last; ++cc) {
+          const int first_of_cc = (int)(((long long)cc * Ttot / G) / nch);
+          const float* ps = part + ((size_t)2 * cc + (pr == first_of_cc ? 0 : 1)) * (DH + 2);
+          const float w = exp2f(__ldcg(ps) - Mg);
+          Lg = fmaf(w, __ldcg(ps + 1), Lg);
+          if (tid < DH) og = fmaf(w, __ldcg(ps + 2 + tid), og);
+        }
+        if (ok && tid < DH) out[(size_t)b * ld_out + h * DH + tid] = from_f<T>(og / Lg);
+        if (tid == 0) counters[pr] = 0;
       }
     }
-    const float Mn = fmaxf(M, block_reduce_max128(cmax, red));  // syncs: sS complete
-    const float scale = exp2f(M - Mn);
-    l *= scale;
-#pragma unroll
-    for (int e = 0; e < C::EPT; ++e) of[e] *= scale;
-    for (int r = g; r < rows; r += C::RPP) {
-      const float p = exp2f(sS[r] - Mn);
-      if (row_leader) l += p;
-      const uint4 u = *reinterpret_cast<const uint4*>(sV + r * DH + e0);
-      float vf[C::EPT];
-      unpack16(u, vf, (const T*)nullptr);
-#pragma unroll
-      for (int e = 0; e < C::EPT; ++e) of[e] = fmaf(p, vf[e], of[e]);
-    }
-    M = Mn;
-    __syncthreads();  // stage s and sS free again
-    if (tid == 0 && i + C::STAGES < nc) issue(i + C::STAGES, s);
+    __syncthreads();  // sO / s_last reused for the next pair
   }
-  if (!ok) return;  // a copy never arrived: status is set, output left as is
-
-  // combine the RPP row groups: o per dim, l over the CTA
-#pragma unroll
-  for (int e = 0; e < C::EPT; ++e) sO[g * DH + e0 + e] = of[e];
-  const float L = block_reduce_sum128(l, red);  // contains the barrier for sO
-  float o_d = 0.f;
-  if (tid < DH) {
-    for (int gg = 0; gg < C::RPP; ++gg) o_d += sO[gg * DH + tid];
-  }
-  if (S == 1) {
-    if (tid < DH) out[(size_t)b * ld_out + h * DH + tid] = from_f<T>(o_d / L);
-    return;
-  }
-  float* my = part + ((size_t)pair * splits + z) * (DH + 2);
-  if (tid < DH) my[2 + tid] = o_d;
-  if (tid == 0) { my[0] = M; my[1] = L; }
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) s_last = (atomicAdd(&counters[pair], 1) == S - 1);
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  const float* pp = part + (size_t)pair * splits * (DH + 2);
-  float Mg = -FLT_MAX;
-  for (int u = 0; u < S; ++u) Mg = fmaxf(Mg, __ldcg(pp + (size_t)u * (DH + 2)));
-  float Lg = 0.f, og = 0.f;
-  for (int u = 0; u < S; ++u) {
-    const float* ps = pp + (size_t)u * (DH + 2);
-    const float w = exp2f(__ldcg(ps) - Mg);
-    Lg = fmaf(w, __ldcg(ps + 1), Lg);
-    if (tid < DH) og = fmaf(w, __ldcg(ps + 2 + tid), og);
-  }
-  if (tid < DH) out[(size_t)b * ld_out + h * DH + tid] = from_f<T>(og / Lg);
-  if (tid == 0) counters[pair] = 0;
 }
 
 static int dec_sm_count() {
@@ -225,26 +250,23 @@ static int dec_chunk(int d) {
   return 8192 / (d * (int)sizeof(T));
 }
 
-// Units per pair: about two work units per resident CTA slot (3 per SM),
-// never more than the pair has chunks.
-static int dec_splits(int pairs, int d, int cap, int dt) {
+constexpr int DEC_CTAS_PER_SM = 3;
+
+// Persistent grid: DEC_CTAS_PER_SM CTAs per SM, never more than the chunks.
+static int dec_grid(int pairs, int d, int cap, int dt) {
   const int chunk = dt == DT_BF16 ? dec_chunk<bf16>(d) : dec_chunk<float>(d);
-  const int max_chunks = (cap + chunk - 1) / chunk;
-  const int target = 2 * 3 * dec_sm_count();
-  int sp = (target + pairs - 1) / pairs;
-  if (sp > max_chunks) sp = max_chunks;
-  if ((long long)pairs * sp > (long long)pairs + DEC_UNITS_SLACK) sp = 1 + DEC_UNITS_SLACK / pairs;
-  return sp < 1 ? 1 : sp;
+  const long long max_chunks = (long long)pairs * ((cap + chunk - 1) / chunk);
+  const long long g = (long long)DEC_CTAS_PER_SM * dec_sm_count();
+  return (int)(g < max_chunks ? g : max_chunks);
 }
 
-int attn_decode_max_splits(int d, int cap, int dt) { return dec_splits(1, d, cap, dt); }
+int attn_decode_max_splits(int d, int cap, int dt) { return dec_grid(1, d, cap, dt); }
 
-// scratch layout: [merge counters: B*H ints, 256-aligned][partials:
-// (B*H + slack) units x (d + 2) floats]; counters sit at offset 0 for any B.
+// scratch layout: [merge counters: B*H ints, 256-aligned][partials: two
+// slots of (d + 2) floats per CTA of the grid]; counters sit at offset 0.
 size_t attn_decode_scratch_bytes(int B, int H, int d, int cap, int dt) {
   const size_t cnt = ((size_t)B * H * sizeof(int) + 255) & ~(size_t)255;
-  const size_t units = (size_t)B * H + DEC_UNITS_SLACK;
-  return cnt + units * (d + 2) * sizeof(float);
+  return cnt + (size_t)2 * DEC_UNITS_SLACK * (d + 2) * sizeof(float);
 }
 
 template <typename T, int DH>
@@ -276,14 +298,14 @@ static cudaError_t launch_dec(const void* q, int ldq, const void* kc, const void
   cudaError_t e = dec_prepare<T, DH>();
   if (e != cudaSuccess) return e;
   const int pairs = B * H;
-  const int sp = dec_splits(pairs, DH, cap, sizeof(T) == 2 ? DT_BF16 : DT_F32);
+  int G = dec_grid(pairs, DH, cap, sizeof(T) == 2 ? DT_BF16 : DT_F32);
+  if (G > DEC_UNITS_SLACK) G = DEC_UNITS_SLACK;  // partial slots in the scratch
   int* counters = reinterpret_cast<int*>(scratch);
   float* partp = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(scratch) +
                                           (((size_t)pairs * sizeof(int) + 255) & ~(size_t)255));
-  dim3 grid(pairs, sp);
   const float qscale = 1.4426950408889634f / sqrtf((float)DH);
-  BT_LAUNCH(attn_decode_kernel<T, DH>, grid, dim3(C::THREADS), C::SMEM, s, (const T*)q, ldq,
-            (const T*)kc, (const T*)vc, H, cap, kvlen, (T*)out, ld_out, partp, counters, sp,
+  BT_LAUNCH(attn_decode_kernel<T, DH>, dim3(G), dim3(C::THREADS), C::SMEM, s, (const T*)q, ldq,
+            (const T*)kc, (const T*)vc, pairs, H, cap, kvlen, (T*)out, ld_out, partp, counters,
             status, qscale);
   return cudaSuccess;
 }

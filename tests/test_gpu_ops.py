@@ -153,3 +153,22 @@ def test_linear_tensor_cores_match_fp64(M, N, K):
     # deterministic: a second call gives the same bits
     out2 = native.linear(xt, wt, bt, path=2).cpu().numpy()
     assert np.array_equal(out, out2)
+
+
+@pytest.mark.parametrize("B,H,d,n,cap", [(64, 12, 64, 300, 544), (8, 16, 128, 2100, 2176),
+                                         (256, 16, 64, 37, 544), (1, 1, 64, 1, 8)])
+def test_decode_attention_bench_shapes(B, H, d, n, cap):
+    """Stream-K decode attention at the workloads' shapes (pairs split across
+    CTAs and merged) against the oracle's attention in fp64."""
+    from hierarchical_global_local_b200 import native
+    torch = gh.torch_mod()
+    g = torch.Generator(device="cuda").manual_seed(B * 7 + n)
+    q = torch.randn(B, H * d, device="cuda", generator=g).bfloat16()
+    k = torch.randn(B, H, cap, d, device="cuda", generator=g).bfloat16()
+    v = torch.randn(B, H, cap, d, device="cuda", generator=g).bfloat16()
+    out = native.decode_attention(q, k, v, n).float().cpu().numpy()
+    qr = q.double().cpu().numpy().reshape(B, 1, H, d)
+    kr = k[:, :, :n].double().cpu().numpy().transpose(0, 2, 1, 3)
+    vr = v[:, :, :n].double().cpu().numpy().transpose(0, 2, 1, 3)
+    ref = om.attend(qr, kr, vr, np.array([n - 1]), np.arange(n)).reshape(B, H * d)
+    assert np.abs(out - ref).max() <= 2e-2
