@@ -117,6 +117,23 @@ def _dist():
     return ws, rank, local
 
 
+def allreduce_max(values, device: str = "cuda"):
+    """Element-wise max of per-rank timings over all ranks (identity when
+    torch.distributed is not initialised)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def job_throughput(tokens_per_rank_step: int, steps: int, world: int, max_ms: float) -> float:
+    """Whole-job tokens/s: every rank generates the same tokens per step;
+    the job lasts as long as the slowest rank."""
+    return world * tokens_per_rank_step * steps / (max_ms / 1e3)
+
+
 def build(rank: int):
     import torch
     from tests.gpu_helpers import build_model
@@ -190,13 +207,11 @@ def run_ours(args):
     for r, a, b in times:
         per_run[r] += a.elapsed_time(b)
     total_ms = sum(per_run.values())
-    tmax = torch.tensor([total_ms] + [per_run[r] for r in RUNS], dtype=torch.float64, device="cuda")
-    if ws > 1:
-        dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
-    total_ms = float(tmax[0])
-    per_run_max = {r: float(tmax[1 + i]) for i, r in enumerate(RUNS)}
+    tmax = allreduce_max([total_ms] + [per_run[r] for r in RUNS])
+    total_ms = tmax[0]
+    per_run_max = {r: tmax[1 + i] for i, r in enumerate(RUNS)}
     tokens_per_step = sum(synth.WORKLOADS[r].batch * synth.WORKLOADS[r].gen_len for r in RUNS)
-    value = ws * tokens_per_step * args.steps / (total_ms / 1e3)
+    value = job_throughput(tokens_per_step, args.steps, ws, total_ms)
 
     # ---- end to end through the public API, host buffers -------------------
     e2e = None
@@ -219,13 +234,10 @@ def run_ours(args):
                 b.record(stream)
                 e_times.append((a, b))
         barrier()
-        e_ms = sum(a.elapsed_time(b) for a, b in e_times)
-        et = torch.tensor([e_ms], dtype=torch.float64, device="cuda")
-        if ws > 1:
-            dist.all_reduce(et, op=dist.ReduceOp.MAX)
+        e_ms = allreduce_max([sum(a.elapsed_time(b) for a, b in e_times)])[0]
         h2d = sum(int(prompts[r].numel()) * 4 for r in RUNS)
         d2h = sum(int(gens[r].numel()) * 4 for r in RUNS)
-        e2e = {"value": ws * tokens_per_step * args.steps / (float(et[0]) / 1e3), "unit": UNIT,
+        e2e = {"value": job_throughput(tokens_per_step, args.steps, ws, e_ms), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     # ---- profiled pass: event pair around every kernel of one step ---------
