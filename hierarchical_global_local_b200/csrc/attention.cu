@@ -32,14 +32,15 @@ template <typename T, int DH>
 struct DecCfg {
   static constexpr int ROW_BYTES = DH * (int)sizeof(T);
   static constexpr int CHUNK = 8192 / ROW_BYTES;         // rows per chunk (8 KB of K)
-  static constexpr int STAGES = 4;
+  static constexpr int STAGES = 3;
   static constexpr int TPR = ROW_BYTES / 16;             // threads per row, 16 B each
-  static constexpr int THREADS = 128;
-  static constexpr int RPP = THREADS / TPR;              // rows per pass
+  static constexpr int CWARPS = 4;                       // consumer warps
+  static constexpr int THREADS = (CWARPS + 1) * 32;      // + one producer warp
+  static constexpr int GROUPS = CWARPS * 32 / TPR;       // row groups (each owns rows)
   static constexpr int EPT = 16 / (int)sizeof(T);        // elements per thread
-  static constexpr int SMEM = STAGES * 2 * CHUNK * ROW_BYTES + CHUNK * 4 + RPP * DH * 4;
+  static constexpr int SMEM = STAGES * 2 * CHUNK * ROW_BYTES + GROUPS * (DH + 2) * 4;
   static_assert(TPR >= 1 && TPR <= 32 && (32 % TPR) == 0, "row split");
-  static_assert(DH <= THREADS, "one thread per output dim in the final reduction");
+  static_assert(DH <= CWARPS * 32, "one thread per output dim in the final reduction");
 };
 
 constexpr int DEC_UNITS_SLACK = 4096;  // work units beyond one per pair (scratch sizing)
@@ -73,8 +74,12 @@ __device__ __forceinline__ int dec_owner(long long x, int G, long long T) {
   return (int)(((x + 1) * G + T - 1) / T) - 1;
 }
 
+// barrier among the consumer warps only (the producer warp may still be
+// waiting for a free stage, or gone)
+__device__ __forceinline__ void cons_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
 template <typename T, int DH>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(DecCfg<T, DH>::THREADS)
 attn_decode_kernel(const T* __restrict__ q, int ldq, const T* __restrict__ kc,
                    const T* __restrict__ vc, int pairs, int H, int cap, PosSpec kvlen,
                    T* __restrict__ out, int ld_out, float* __restrict__ part,
@@ -92,145 +97,159 @@ attn_decode_kernel(const T* __restrict__ q, int ldq, const T* __restrict__ kc,
   if (c >= G) return;
   const long long x0 = (long long)c * Ttot / G, x1 = (long long)(c + 1) * Ttot / G;
   const int nc = (int)(x1 - x0);
-  if (nc <= 0) return;
 
   extern __shared__ __align__(128) uint8_t smem[];
   T* sKV = reinterpret_cast<T*>(smem);  // [STAGES][K chunk | V chunk]
-  float* sS = reinterpret_cast<float*>(smem + C::STAGES * 2 * C::CHUNK * C::ROW_BYTES);
-  float* sO = sS + C::CHUNK;
-  __shared__ __align__(8) uint64_t full[C::STAGES];
-  __shared__ float red[4];
+  float* sR = reinterpret_cast<float*>(smem + C::STAGES * 2 * C::CHUNK * C::ROW_BYTES);
+  __shared__ __align__(8) uint64_t full[C::STAGES], empty[C::STAGES];
   __shared__ int s_last;
 
   const int tid = threadIdx.x;
-  auto issue = [&](int i, int s) {  // chunk x0 + i -> stage s
-    const long long x = x0 + i;
-    const int pr = (int)(x / nch), ci = (int)(x - (long long)pr * nch);
-    const int r0 = ci * C::CHUNK;
-    const int rows = min(C::CHUNK, n - r0);
-    const uint32_t bytes = (uint32_t)rows * C::ROW_BYTES;
-    const size_t off = ((size_t)pr * cap + r0) * DH;
-    T* dk = sKV + (size_t)s * 2 * C::CHUNK * DH;
-    mbar_arrive_expect_tx(&full[s], 2 * bytes);
-    bulk_g2s(dk, kc + off, bytes, &full[s]);
-    bulk_g2s(dk + C::CHUNK * DH, vc + off, bytes, &full[s]);
-  };
+  const int warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
-    for (int s = 0; s < C::STAGES; ++s) mbar_init(&full[s], 1);
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], C::CWARPS);
+    }
     fence_mbar_init();
-    for (int i = 0; i < nc && i < C::STAGES; ++i) issue(i, i);
   }
-  __syncthreads();  // barriers initialised before anyone waits on them
+  __syncthreads();
 
-  const int g = tid / C::TPR;
-  const int e0 = (tid % C::TPR) * C::EPT;
-  const bool row_leader = (tid % C::TPR) == 0;
-  const int first_pair = (int)(x0 / nch);
   bool ok = true;
+  if (warp == C::CWARPS) {
+    // ---- producer warp: one lane streams chunks x0 .. x1 through the ring ----
+    if (lane == 0) {
+      for (int i = 0; i < nc; ++i) {
+        const int s = i % C::STAGES;
+        if (i >= C::STAGES) mbar_wait_bounded(&empty[s], ((i / C::STAGES) + 1) & 1, status);
+        const long long x = x0 + i;
+        const int pr = (int)(x / nch), ci = (int)(x - (long long)pr * nch);
+        const int r0 = ci * C::CHUNK;
+        const int rows = min(C::CHUNK, n - r0);
+        const uint32_t bytes = (uint32_t)rows * C::ROW_BYTES;
+        const size_t off = ((size_t)pr * cap + r0) * DH;
+        T* dk = sKV + (size_t)s * 2 * C::CHUNK * DH;
+        mbar_arrive_expect_tx(&full[s], 2 * bytes);
+        bulk_g2s(dk, kc + off, bytes, &full[s]);
+        bulk_g2s(dk + C::CHUNK * DH, vc + off, bytes, &full[s]);
+      }
+    }
+    return;  // the copies complete on the mbarriers; consumers sync among themselves
+  }
+
+  // ---- consumers: row group g (TPR lanes) owns rows g, g + GROUPS, ... of
+  // every chunk, with its own running max, sum and output slice ----
+  const int g = tid / C::TPR;  // valid for consumer warps
+  const int e0 = (tid % C::TPR) * C::EPT;
+  const int first_pair = (int)(x0 / nch);
   int i = 0;
   for (int pr = first_pair; i < nc; ++pr) {
-    // chunks of pair pr inside this CTA's range: [i, i + cnt)
     const long long pend = (long long)(pr + 1) * nch;
     const int cnt = (int)((pend < x1 ? pend : x1) - (x0 + i));
     const int b = pr / H, h = pr - b * H;
-    float qf[C::EPT];
-    {
-      const uint4 u = *reinterpret_cast<const uint4*>(q + (size_t)b * ldq + h * DH + e0);
-      unpack16(u, qf, (const T*)nullptr);
-#pragma unroll
-      for (int e = 0; e < C::EPT; ++e) qf[e] *= qscale;
-    }
     float M = -FLT_MAX, l = 0.f;
     float of[C::EPT];
 #pragma unroll
     for (int e = 0; e < C::EPT; ++e) of[e] = 0.f;
-    for (int k = 0; k < cnt; ++k, ++i) {
-      const int s = i % C::STAGES;
-      if (!mbar_wait_bounded(&full[s], (i / C::STAGES) & 1, status)) ok = false;
-      const T* sK = sKV + (size_t)s * 2 * C::CHUNK * DH;
-      const T* sV = sK + C::CHUNK * DH;
-      const long long x = x0 + i;
-      const int rows = min(C::CHUNK, n - (int)(x - (long long)pr * nch) * C::CHUNK);
-      // scores (log2 domain); uniform trip count -> whole-warp shuffles
-      float cmax = -FLT_MAX;
-      for (int rb = 0; rb < rows; rb += C::RPP) {
-        const int r = rb + g;
-        const bool valid = r < rows;
-        float sc = 0.f;
-        if (valid) {
-          const uint4 u = *reinterpret_cast<const uint4*>(sK + r * DH + e0);
-          float kf[C::EPT];
-          unpack16(u, kf, (const T*)nullptr);
+    {
+      float qf[C::EPT];
+      {
+        const uint4 u = *reinterpret_cast<const uint4*>(q + (size_t)b * ldq + h * DH + e0);
+        unpack16(u, qf, (const T*)nullptr);
 #pragma unroll
-          for (int e = 0; e < C::EPT; ++e) sc = fmaf(qf[e], kf[e], sc);
-        }
-#pragma unroll
-        for (int o = C::TPR / 2; o > 0; o >>= 1) sc += __shfl_xor_sync(0xffffffffu, sc, o);
-        if (valid) {
-          cmax = fmaxf(cmax, sc);
-          if (row_leader) sS[r] = sc;
-        }
+        for (int e = 0; e < C::EPT; ++e) qf[e] *= qscale;
       }
-      const float Mn = fmaxf(M, block_reduce_max128(cmax, red));  // syncs: sS complete
-      const float scale = exp2f(M - Mn);
-      l *= scale;
+      for (int k = 0; k < cnt; ++k) {
+        const int ii = i + k;
+        const int s = ii % C::STAGES;
+        if (!mbar_wait_bounded(&full[s], (ii / C::STAGES) & 1, status)) ok = false;
+        const T* sK = sKV + (size_t)s * 2 * C::CHUNK * DH;
+        const T* sV = sK + C::CHUNK * DH;
+        const long long x = x0 + ii;
+        const int rows = min(C::CHUNK, n - (int)(x - (long long)pr * nch) * C::CHUNK);
+        // uniform trip count over the warp: the row-group shuffles always
+        // see the whole warp
+        for (int rb = 0; rb < rows; rb += C::GROUPS) {
+          const int r = rb + g;
+          const bool valid = r < rows;
+          float sc = 0.f;
+          float vf[C::EPT];
+          if (valid) {
+            const uint4 uk = *reinterpret_cast<const uint4*>(sK + r * DH + e0);
+            const uint4 uv = *reinterpret_cast<const uint4*>(sV + r * DH + e0);
+            float kf[C::EPT];
+            unpack16(uk, kf, (const T*)nullptr);
+            unpack16(uv, vf, (const T*)nullptr);
 #pragma unroll
-      for (int e = 0; e < C::EPT; ++e) of[e] *= scale;
-      for (int r = g; r < rows; r += C::RPP) {
-        const float p = exp2f(sS[r] - Mn);
-        if (row_leader) l += p;
-        const uint4 u = *reinterpret_cast<const uint4*>(sV + r * DH + e0);
-        float vf[C::EPT];
-        unpack16(u, vf, (const T*)nullptr);
+            for (int e = 0; e < C::EPT; ++e) sc = fmaf(qf[e], kf[e], sc);
+          }
 #pragma unroll
-        for (int e = 0; e < C::EPT; ++e) of[e] = fmaf(p, vf[e], of[e]);
+          for (int o = C::TPR / 2; o > 0; o >>= 1) sc += __shfl_xor_sync(0xffffffffu, sc, o);
+          if (valid) {
+            const float Mn = fmaxf(M, sc);
+            const float cs = exp2f(M - Mn), p = exp2f(sc - Mn);
+            l = l * cs + p;
+#pragma unroll
+            for (int e = 0; e < C::EPT; ++e) of[e] = fmaf(p, vf[e], of[e] * cs);
+            M = Mn;
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);  // this warp is done with stage s
       }
-      M = Mn;
-      __syncthreads();  // stage s and sS free again
-      if (tid == 0 && i + C::STAGES < nc) issue(i + C::STAGES, s);
+      // park this group's (M, l, o slice) for the combination
+      float* gr = sR + (size_t)g * (DH + 2);
+#pragma unroll
+      for (int e = 0; e < C::EPT; ++e) gr[2 + e0 + e] = of[e];
+      if ((tid % C::TPR) == 0) { gr[0] = M; gr[1] = l; }
     }
-    // this CTA's share of pair pr: combine the row groups
-#pragma unroll
-    for (int e = 0; e < C::EPT; ++e) sO[g * DH + e0 + e] = of[e];
-    const float L = block_reduce_sum128(l, red);  // barrier for sO
-    float o_d = 0.f;
+    i += cnt;
+    cons_sync();
+    // combine the groups: thread t < DH owns output dim t
+    float Mg = -FLT_MAX, Lg = 0.f, og = 0.f;
     if (tid < DH) {
-      for (int gg = 0; gg < C::RPP; ++gg) o_d += sO[gg * DH + tid];
+      for (int gg = 0; gg < C::GROUPS; ++gg) Mg = fmaxf(Mg, sR[(size_t)gg * (DH + 2)]);
+      for (int gg = 0; gg < C::GROUPS; ++gg) {
+        const float* gr = sR + (size_t)gg * (DH + 2);
+        const float w = exp2f(gr[0] - Mg);
+        Lg = fmaf(w, gr[1], Lg);
+        og = fmaf(w, gr[2 + tid], og);
+      }
     }
     const long long pbeg = (long long)pr * nch;
     const int first = dec_owner(pbeg, G, Ttot), last = dec_owner(pbeg + nch - 1, G, Ttot);
     if (first == last) {
-      if (ok && tid < DH) out[(size_t)b * ld_out + h * DH + tid] = from_f<T>(o_d / L);
+      if (ok && tid < DH) out[(size_t)b * ld_out + h * DH + tid] = from_f<T>(og / Lg);
     } else {
       // partial slot: 2c if pair pr is where this CTA's range starts, else 2c + 1
       float* my = part + ((size_t)2 * c + (pr == first_pair ? 0 : 1)) * (DH + 2);
-      if (tid < DH) my[2 + tid] = o_d;
-      if (tid == 0) { my[0] = M; my[1] = L; }
+      if (tid < DH) my[2 + tid] = og;
+      if (tid == 0) { my[0] = Mg; my[1] = Lg; }
       __threadfence();
-      __syncthreads();
+      cons_sync();
       if (tid == 0) s_last = (atomicAdd(&counters[pr], 1) == last - first);
-      __syncthreads();
+      cons_sync();
       if (s_last) {
         __threadfence();
-        float Mg = -FLT_MAX;
+        float M2 = -FLT_MAX;
         for (int cc = first; cc <= last; ++cc) {
           const int first_of_cc = (int)(((long long)cc * Ttot / G) / nch);
           const float* ps = part + ((size_t)2 * cc + (pr == first_of_cc ? 0 : 1)) * (DH + 2);
-          Mg = fmaxf(Mg, __ldcg(ps));
+          M2 = fmaxf(M2, __ldcg(ps));
         }
-        float Lg = 0.f, og = 0.f;
+        float L2 = 0.f, o2 = 0.f;
         for (int cc = first; cc <= last; ++cc) {
           const int first_of_cc = (int)(((long long)cc * Ttot / G) / nch);
           const float* ps = part + ((size_t)2 * cc + (pr == first_of_cc ? 0 : 1)) * (DH + 2);
-          const float w = exp2f(__ldcg(ps) - Mg);
-          Lg = fmaf(w, __ldcg(ps + 1), Lg);
-          if (tid < DH) og = fmaf(w, __ldcg(ps + 2 + tid), og);
+          const float w = exp2f(__ldcg(ps) - M2);
+          L2 = fmaf(w, __ldcg(ps + 1), L2);
+          if (tid < DH) o2 = fmaf(w, __ldcg(ps + 2 + tid), o2);
         }
-        if (ok && tid < DH) out[(size_t)b * ld_out + h * DH + tid] = from_f<T>(og / Lg);
+        if (ok && tid < DH) out[(size_t)b * ld_out + h * DH + tid] = from_f<T>(o2 / L2);
         if (tid == 0) counters[pr] = 0;
       }
     }
-    __syncthreads();  // sO / s_last reused for the next pair
+    cons_sync();  // sR / s_last reused for the next pair
   }
 }
 
@@ -250,7 +269,7 @@ static int dec_chunk(int d) {
   return 8192 / (d * (int)sizeof(T));
 }
 
-constexpr int DEC_CTAS_PER_SM = 3;
+constexpr int DEC_CTAS_PER_SM = 4;
 
 // Persistent grid: DEC_CTAS_PER_SM CTAs per SM, never more than the chunks.
 static int dec_grid(int pairs, int d, int cap, int dt) {
