@@ -84,6 +84,9 @@ def lib() -> ctypes.CDLL:
             "bt_op_decode_attention": (c_int, [c_int, c_void_p, c_int, c_void_p, c_void_p, c_int,
                                                c_int, c_int, c_int, c_int, c_void_p, c_int,
                                                c_void_p, c_size_t, c_void_p]),
+            "bt_op_decode_attention_noalloc": (c_int, [c_int, c_void_p, c_int, c_void_p, c_void_p,
+                                                       c_int, c_int, c_int, c_int, c_int,
+                                                       c_void_p, c_int, c_void_p]),
             "bt_op_prefill_attention": (c_int, [c_int, c_void_p, c_int, c_void_p, c_void_p, c_int,
                                                 c_int, c_int, c_int, c_int, c_void_p, c_int,
                                                 c_void_p]),
@@ -110,6 +113,7 @@ def exported_symbols():
         "bt_position", "bt_destroy", "bt_strerror", "bt_last_cuda_error",
         "bt_kernel_launches", "bt_profile_begin", "bt_profile_end",
         "bt_op_decode_attention_scratch_bytes", "bt_op_decode_attention",
+        "bt_op_decode_attention_noalloc",
         "bt_op_prefill_attention", "bt_op_linear_scratch_bytes", "bt_op_linear",
         "bt_op_layernorm", "bt_op_embed_prompt"]
 
@@ -277,6 +281,20 @@ def decode_attention(q, k, v, n: int, out=None, scratch=None):
                                         v.data_ptr(), B, H, d, cap, n, out.data_ptr(),
                                         out.stride(0), scratch.data_ptr(), scratch.numel(),
                                         _stream()), "bt_op_decode_attention")
+    return out
+
+
+def decode_attention_noalloc(q, k, v, n: int, out=None):
+    """Decode attention through the entry point that takes no scratch and
+    allocates nothing (fixed array inside the library; see bt_ops.h)."""
+    import torch
+    B, H, cap, d = k.shape
+    if out is None:
+        out = torch.empty(B, H * d, dtype=q.dtype, device="cuda")
+    _check(lib().bt_op_decode_attention_noalloc(_dt(q), q.data_ptr(), q.stride(0), k.data_ptr(),
+                                                v.data_ptr(), B, H, d, cap, n, out.data_ptr(),
+                                                out.stride(0), _stream()),
+           "bt_op_decode_attention_noalloc")
     return out
 
 

@@ -39,6 +39,27 @@ BT_API int bt_op_decode_attention(int dtype, const void *q_dev, int ldq, const v
                            const void *v_dev, int B, int H, int d, int cap, int n, void *out_dev,
                            int ld_out, void *scratch_dev, size_t scratch_bytes, void *stream);
 
+/* bt_op_decode_attention without a scratch argument, for callers that cannot
+ * allocate device memory at the time they run it (for example while recording
+ * a CUDA graph, where cudaMalloc is not a capturable operation, or inside a
+ * runtime whose device memory is a fixed pool carved at start-up). The paper
+ * has no counterpart: this is an integration convenience of this library.
+ *   Arguments and result as bt_op_decode_attention (q, k, v, out are still the
+ *   caller's). The split-K merge state lives in one fixed array compiled into
+ *   the library (about 4.3 MB, held on every GPU that loads the library until
+ *   the process exits), so it allocates nothing: it calls no cudaMalloc,
+ *   cudaFree or allocating library routine.
+ *   Limits: B*H <= 8192 and d <= 128; larger problems return BT_ECAPACITY.
+ *   The first call on each device looks up the array's device address (with
+ *   that device current) and caches it; make that first call before any
+ *   stream capture. Every call zeroes the merge counters it uses on `stream`.
+ *   All calls share the one array: calls that may overlap on the GPU (other
+ *   streams, other threads) race and must be serialised by the caller. */
+BT_API int bt_op_decode_attention_noalloc(int dtype, const void *q_dev, int ldq,
+                                          const void *k_dev, const void *v_dev, int B, int H,
+                                          int d, int cap, int n, void *out_dev, int ld_out,
+                                          void *stream);
+
 /* Causal attention of the block decoder at prefill: queries are the n rows
  * b*n + i of q_dev [B*n, ldq]; query i attends to cache entries 0..i of
  * k_dev/v_dev [B, H, cap, d]; out rows likewise. */
