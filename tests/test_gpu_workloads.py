@@ -1,0 +1,81 @@
+"""Parity at the workloads' full sizes (full batch, full prompt, the launch
+configuration the benchmark times), checked on sampled rows.
+
+The GPU runs the whole batch; the oracle recomputes only the sampled rows
+(sequences are independent -- checked bitwise in test_gpu_model -- so a row
+of a full-batch run equals that row run alone). The oracle runs in fp32 for
+these sizes to keep the CPU time bounded; its rounding error is orders of
+magnitude below the bf16 tolerance (per-step relative L2 <= 2e-2 over the
+sampled rows' logits). Decode-heavy runs are checked on a stride of steps
+that crosses many block boundaries.
+"""
+import numpy as np
+import pytest
+
+import synth
+from tests import gpu_helpers as gh
+
+pytestmark = pytest.mark.gpu
+
+BF16_REL = 2e-2
+
+
+def _rows(B, n, seed):
+    g = np.random.default_rng(seed)
+    extra = [int(x) for x in g.choice(np.arange(1, B - 1), size=max(0, n - 2), replace=False)] if B > 2 else []
+    return sorted(set([0, B - 1] + extra))[:n] if n >= 2 else [B - 1]
+
+
+def _run(name, G, check, n_rows, **over):
+    torch = gh.torch_mod()
+    wl = synth.workload(name, **over) if over else synth.WORKLOADS[name]
+    B, T = wl.batch, wl.prompt_len
+    w = synth.make_weights(wl)
+    toks = synth.make_tokens(wl, length=T + G)
+    rows = _rows(B, n_rows, 17)
+    model = gh.build_model(wl.shape, w, B, wl.max_seq)
+    tok = torch.from_numpy(np.ascontiguousarray(toks)).cuda()
+    logits = torch.empty(B, wl.shape.vocab, dtype=torch.float32, device="cuda")
+    ridx = torch.tensor(rows, device="cuda")
+    got = {}
+    model.prefill(tok[:, :T].contiguous(), logits=logits)
+    if 0 in check:
+        got[0] = logits.index_select(0, ridx).cpu().numpy()
+    for i in range(1, G):
+        model.decode(tok[:, T + i - 1].contiguous(), logits=logits if i in check else None)
+        if i in check:
+            got[i] = logits.index_select(0, ridx).cpu().numpy()
+    model.sync()
+    model.close()
+    del model
+    torch.cuda.empty_cache()
+    ol = gh.oracle_teacher_forced(wl.shape, w, toks, T, G, rows=rows, dtype=np.float32)
+    worst = 0.0
+    for i, g in got.items():
+        e = gh.rel_l2(g, ol[i])
+        worst = max(worst, e)
+        assert e <= BF16_REL, (name, i, e)
+    return worst
+
+
+def test_pythia160m_prefill_heavy_full_batch_and_prompt():
+    _run("pythia160m_prefill_heavy", G=9, check=set(range(9)), n_rows=4)
+
+
+def test_pythia160m_decode_heavy_first_257_steps():
+    G = 257
+    _run("pythia160m_decode_heavy", G=G, check=set(range(0, G, 16)) | {1, 2, 3, 4, G - 1}, n_rows=4)
+
+
+def test_pythia410m_decode_heavy_full_batch():
+    G = 129
+    _run("pythia410m_decode_heavy", G=G, check=set(range(0, G, 16)) | {1, 2, 3, G - 1}, n_rows=3)
+
+
+@pytest.mark.parametrize("lb", [1, 2, 4, 8])
+def test_lb_sweep_full_batch_and_prompt(lb):
+    _run(f"lb_sweep_L{lb}", G=2 * max(lb, 2) + 1, check=set(range(2 * max(lb, 2) + 1)), n_rows=1)
+
+
+def test_long_context_full_batch_and_prompt():
+    _run("long_context", G=5, check=set(range(5)), n_rows=1)
