@@ -1,0 +1,366 @@
+// attn_prefill_tc.cu -- causal attention of the block decoder at prefill on
+// the 5th-generation tensor cores (tcgen05 + TMEM), sm_100a.
+//
+// "Block Transformer: Global-to-Local Language Modeling for Fast Inference",
+// §3.4 "The Block Decoder": standard causal self-attention over the n block
+// embeddings of the prompt (n = T / L_B).
+//
+// One CTA per (sequence, head, 128-query tile), flash-attention style:
+//   S = Q K^T           tcgen05.mma, M = 128 queries, N = 128 keys, into TMEM
+//   P = softmax pieces  4 warps, one query row per thread (tcgen05.ld), online
+//                       max / sum, causal + tail masking, P written to shared
+//                       memory in the 128-byte-swizzled K-major layout
+//   O_j = P V           tcgen05.mma, M = 128, N = d, K = 128 keys, into TMEM;
+//                       accumulated (with the softmax rescale) in registers
+// Operands come in by TMA with 3-D tensor maps bounded per (sequence, head),
+// so keys / queries past n read as zeros (no stale cache bytes reach the
+// products). V is read through its transpose V^T [B*H][d][n_pad] (written
+// next to the cache during prefill), so both MMAs take K-major operands.
+// Warps: 0-3 softmax/epilogue, 4 TMA producer, 5 MMA issuer. All waits are
+// bounded.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace bt {
+
+namespace {
+
+constexpr int QT = 128;   // queries per CTA (MMA M)
+constexpr int KT = 128;   // keys per tile (MMA N of S, K of P V)
+constexpr int THREADS = 192;
+
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFF) >> 4);
+  d |= (uint64_t)(16 >> 4) << 16;
+  d |= (uint64_t)(1024 >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+
+__device__ __forceinline__ constexpr uint32_t idesc_bf16(int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(QT >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc));
+}
+
+__device__ __forceinline__ void commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tma3(void* dst, const CUtensorMap* m, int x, int y, int z, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
+      "%4, %5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
+__device__ __forceinline__ void ld32(uint32_t taddr, float* v) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
+      "%30, %31}, [%32];\n"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
+        "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
+        "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// shared memory plan (bytes), all tiles 1024-aligned
+template <int DH>
+struct Plan {
+  static constexpr int KB = DH / 64;                  // 64-wide K blocks of Q and K
+  static constexpr int Q_BYTES = QT * DH * 2;         // KB blocks of [128 x 64]
+  static constexpr int K_BYTES = KT * DH * 2;         // per stage
+  static constexpr int VT_BYTES = DH * KT * 2;        // per stage: 2 blocks of [DH x 64 keys]
+  static constexpr int P_BYTES = QT * KT * 2;         // 2 blocks of [128 x 64 keys]
+  static constexpr int STAGES = 2;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + Q_BYTES;
+  static constexpr int OFF_VT = OFF_K + STAGES * K_BYTES;
+  static constexpr int OFF_P = OFF_VT + STAGES * VT_BYTES;
+  static constexpr int BYTES = OFF_P + P_BYTES + 1024;  // + alignment slack
+  static constexpr int TMEM_COLS = 256;               // S: 128 columns, O: DH columns
+};
+
+template <int DH>
+__global__ void __launch_bounds__(THREADS, 1)
+attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
+                       const __grid_constant__ CUtensorMap mVt, int H, int n, bf16* __restrict__ out,
+                       int ld_out, float scale_log2, int* status) {
+  using PL = Plan<DH>;
+  pdl_trigger();
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  __shared__ __align__(8) uint64_t q_full, kv_full[PL::STAGES], kv_empty[PL::STAGES], s_full, p_full, o_full;
+  __shared__ uint32_t tmem_slot;
+
+  const int nqt = (n + QT - 1) / QT;
+  const int qt = blockIdx.x % nqt;
+  const int bh = blockIdx.x / nqt;  // b * H + h
+  const int b = bh / H, h = bh - b * H;
+  const int q0 = qt * QT;
+  const int ntiles = (q0 + QT - 1) / KT + 1;  // key tiles intersecting the causal band
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&q_full, 1);
+    for (int s = 0; s < PL::STAGES; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    mbar_init(&s_full, 1);
+    mbar_init(&p_full, 128);
+    mbar_init(&o_full, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&tmem_slot)),
+                 "r"(PL::TMEM_COLS));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem = tmem_slot;
+  const uint32_t tS = tmem, tO = tmem + KT;
+  pdl_wait();
+
+  if (warp == 4) {
+    if (lane == 0) {
+      // Q tile (KB blocks of 64 dims), then K / V^T tiles through the ring
+      mbar_arrive_expect_tx(&q_full, PL::Q_BYTES);
+      for (int kb = 0; kb < PL::KB; ++kb)
+        tma3(sm + PL::OFF_Q + kb * QT * 128, &mQ, h * DH + kb * 64, q0, b, &q_full);
+      for (int j = 0; j < ntiles; ++j) {
+        const int s = j % PL::STAGES;
+        if (j >= PL::STAGES) mbar_wait_bounded(&kv_empty[s], ((j / PL::STAGES) + 1) & 1, status);
+        mbar_arrive_expect_tx(&kv_full[s], PL::K_BYTES + PL::VT_BYTES);
+        for (int kb = 0; kb < PL::KB; ++kb)
+          tma3(sm + PL::OFF_K + s * PL::K_BYTES + kb * KT * 128, &mK, kb * 64, j * KT, bh, &kv_full[s]);
+        for (int kb = 0; kb < KT / 64; ++kb)
+          tma3(sm + PL::OFF_VT + s * PL::VT_BYTES + kb * DH * 128, &mVt, j * KT + kb * 64, 0, bh,
+               &kv_full[s]);
+      }
+    }
+  } else if (warp == 5) {
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16(KT), idO = idesc_bf16(DH);
+      mbar_wait_bounded(&q_full, 0, status);
+      for (int j = 0; j < ntiles; ++j) {
+        const int s = j % PL::STAGES;
+        // (S of tile j-1 was consumed before P of tile j-1 was published,
+        // which this thread waited for before the previous P V)
+        mbar_wait_bounded(&kv_full[s], (j / PL::STAGES) & 1, status);
+        fence_after();
+        // S = Q K^T over DH (KB blocks x 4 slices of 16)
+        for (int kb = 0; kb < PL::KB; ++kb) {
+          const uint64_t dq = desc_sw128(smem_u32(sm + PL::OFF_Q + kb * QT * 128));
+          const uint64_t dk = desc_sw128(smem_u32(sm + PL::OFF_K + s * PL::K_BYTES + kb * KT * 128));
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) mma(tS, dq + 2 * kk, dk + 2 * kk, idS, (kb | kk) ? 1u : 0u);
+        }
+        commit(&s_full);
+        // O_j = P V over the 128 keys (2 blocks x 4 slices of 16), once P is written
+        mbar_wait_bounded(&p_full, j & 1, status);
+        fence_after();
+        for (int kb = 0; kb < KT / 64; ++kb) {
+          const uint64_t dp = desc_sw128(smem_u32(sm + PL::OFF_P + kb * QT * 128));
+          const uint64_t dv = desc_sw128(smem_u32(sm + PL::OFF_VT + s * PL::VT_BYTES + kb * DH * 128));
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) mma(tO, dp + 2 * kk, dv + 2 * kk, idO, (kb | kk) ? 1u : 0u);
+        }
+        commit(&o_full);
+        commit(&kv_empty[s]);
+      }
+    }
+  } else {
+    // ---- softmax / epilogue: thread r owns query row q0 + r ----
+    const int r = warp * 32 + lane;
+    const int qi = q0 + r;
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    float m = -INFINITY, l = 0.f;
+    float o[DH];
+#pragma unroll
+    for (int e = 0; e < DH; ++e) o[e] = 0.f;
+    uint8_t* prow = sm + PL::OFF_P;
+    for (int j = 0; j < ntiles; ++j) {
+      mbar_wait_bounded(&s_full, j & 1, status);
+      fence_after();
+      const int k0 = j * KT;
+      // pass 1: row max over this tile (masked keys excluded), 32 columns at a time
+      float tmax = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < KT; c += 32) {
+        float sv[32];
+        ld32(tS + lane_base + c, sv);
+#pragma unroll
+        for (int u = 0; u < 32; ++u) {
+          const int kj = k0 + c + u;
+          if (kj <= qi && kj < n) tmax = fmaxf(tmax, sv[u] * scale_log2);
+        }
+      }
+      const float mn = fmaxf(m, tmax);
+      const float corr = (mn == -INFINITY) ? 1.f : exp2f(m - mn);
+      // pass 2: P = exp2(s - mn) as bf16 into the swizzled K-major tile
+      float lt = 0.f;
+#pragma unroll
+      for (int c = 0; c < KT; c += 32) {
+        float sv[32];
+        ld32(tS + lane_base + c, sv);
+#pragma unroll
+        for (int c8 = 0; c8 < 4; ++c8) {
+          float p[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int kj = k0 + c + c8 * 8 + u;
+            p[u] = (kj <= qi && kj < n) ? exp2f(sv[c8 * 8 + u] * scale_log2 - mn) : 0.f;
+            lt += p[u];
+          }
+          __nv_bfloat162 h0 = __floats2bfloat162_rn(p[0], p[1]), h1 = __floats2bfloat162_rn(p[2], p[3]);
+          __nv_bfloat162 h2 = __floats2bfloat162_rn(p[4], p[5]), h3 = __floats2bfloat162_rn(p[6], p[7]);
+          uint4 w;
+          w.x = *reinterpret_cast<uint32_t*>(&h0); w.y = *reinterpret_cast<uint32_t*>(&h1);
+          w.z = *reinterpret_cast<uint32_t*>(&h2); w.w = *reinterpret_cast<uint32_t*>(&h3);
+          const int col8 = (c >> 3) + c8;          // 8-key chunk index within the 128 keys
+          const int kb = col8 >> 3, chunk = col8 & 7;  // 64-key block, 16-byte chunk in the row
+          uint8_t* dst = prow + kb * QT * 128 + r * 128 + ((chunk ^ (r & 7)) << 4);
+          *reinterpret_cast<uint4*>(dst) = w;
+        }
+      }
+      fence_proxy_async();  // P visible to the tensor core
+      fence_before();
+      mbar_arrive(&p_full);
+      // accumulate O_j with the rescale
+      mbar_wait_bounded(&o_full, j & 1, status);
+      fence_after();
+#pragma unroll
+      for (int c = 0; c < DH; c += 32) {
+        float ov[32];
+        ld32(tO + lane_base + c, ov);
+#pragma unroll
+        for (int u = 0; u < 32; ++u) o[c + u] = o[c + u] * corr + ov[u];
+      }
+      l = l * corr + lt;
+      m = mn;
+    }
+    if (qi < n) {
+      const float inv = 1.f / l;
+      bf16* dst = out + ((size_t)b * n + qi) * ld_out + h * DH;
+#pragma unroll
+      for (int e = 0; e < DH; e += 8) {
+        __nv_bfloat162 h0 = __floats2bfloat162_rn(o[e] * inv, o[e + 1] * inv);
+        __nv_bfloat162 h1 = __floats2bfloat162_rn(o[e + 2] * inv, o[e + 3] * inv);
+        __nv_bfloat162 h2 = __floats2bfloat162_rn(o[e + 4] * inv, o[e + 5] * inv);
+        __nv_bfloat162 h3 = __floats2bfloat162_rn(o[e + 6] * inv, o[e + 7] * inv);
+        uint4 w;
+        w.x = *reinterpret_cast<uint32_t*>(&h0); w.y = *reinterpret_cast<uint32_t*>(&h1);
+        w.z = *reinterpret_cast<uint32_t*>(&h2); w.w = *reinterpret_cast<uint32_t*>(&h3);
+        *reinterpret_cast<uint4*>(dst + e) = w;
+      }
+    }
+  }
+  fence_before();
+  __syncthreads();
+  if (warp == 0)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(PL::TMEM_COLS));
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn enc3() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 3-D bf16 map {x (contiguous), y, z}, strides in elements for y and z, box
+// {64, by, 1}, 128-byte swizzle, zero fill outside [0, dims).
+bool map3(CUtensorMap* m, const void* base, long long x, long long y, long long z, long long sy,
+          long long sz, int by) {
+  EncodeTiledFn f = enc3();
+  if (!f) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)x, (cuuint64_t)y, (cuuint64_t)z};
+  cuuint64_t str[2] = {(cuuint64_t)sy * 2, (cuuint64_t)sz * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)by, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, str, box, es,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int DH>
+cudaError_t launch_tc(const void* q, int ldq, const void* kc, const void* vt, int vt_ld, int B,
+                      int H, int cap, int n, void* out, int ld_out, int* status, cudaStream_t s) {
+  static bool prepared = false;
+  if (!prepared) {
+    cudaError_t e = cudaFuncSetAttribute(attn_prefill_tc_kernel<DH>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Plan<DH>::BYTES);
+    if (e != cudaSuccess) return e;
+    prepared = true;
+  }
+  CUtensorMap mQ, mK, mVt;
+  // Q rows b*n + i, dims (h*d + e): {ldq cols, n rows, B}
+  if (!map3(&mQ, q, ldq, n, B, ldq, (long long)n * ldq, QT)) return cudaErrorInvalidValue;
+  // K cache [B*H][cap][d], valid rows < n
+  if (!map3(&mK, kc, DH, n, (long long)B * H, DH, (long long)cap * DH, KT)) return cudaErrorInvalidValue;
+  // V^T [B*H][d][vt_ld], valid keys < n
+  if (!map3(&mVt, vt, n, DH, (long long)B * H, vt_ld, (long long)DH * vt_ld, DH)) return cudaErrorInvalidValue;
+  const int nqt = (n + QT - 1) / QT;
+  const float scale = 1.4426950408889634f / sqrtf((float)DH);
+  BT_LAUNCH(attn_prefill_tc_kernel<DH>, dim3(B * H * nqt), dim3(THREADS), Plan<DH>::BYTES, s, mQ, mK,
+            mVt, H, n, (bf16*)out, ld_out, scale, status);
+  return cudaSuccess;
+}
+
+}  // namespace
+
+int attn_prefill_tc_supported(int dt, int d, int ldq, int vt_ld) {
+  return (dt == DT_BF16 && (d == 64 || d == 128) && (ldq % 8) == 0 && (vt_ld % 8) == 0 &&
+          enc3() != nullptr)
+             ? 1
+             : 0;
+}
+
+cudaError_t launch_attn_prefill_tc(const void* q, int ldq, const void* k_cache, const void* vt,
+                                   int vt_ld, int B, int H, int d, int cap, int n, void* out,
+                                   int ld_out, int* status, cudaStream_t s) {
+  if (B * H * n == 0) return cudaSuccess;
+  if (d == 64) return launch_tc<64>(q, ldq, k_cache, vt, vt_ld, B, H, cap, n, out, ld_out, status, s);
+  if (d == 128) return launch_tc<128>(q, ldq, k_cache, vt, vt_ld, B, H, cap, n, out, ld_out, status, s);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace bt

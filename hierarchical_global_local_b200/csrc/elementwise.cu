@@ -295,7 +295,7 @@ template <typename T>
 __global__ void rope_append_kernel(const T* __restrict__ qkv, int D, int H, int rot,
                                    const float2* __restrict__ tab, PosSpec ps,
                                    T* __restrict__ q_out, T* __restrict__ kc,
-                                   T* __restrict__ vc, int cap) {
+                                   T* __restrict__ vc, int cap, T* __restrict__ vt, int vt_ld) {
   pdl_trigger();
   pdl_wait();
   const int m = blockIdx.x;
@@ -320,22 +320,23 @@ __global__ void rope_append_kernel(const T* __restrict__ qkv, int D, int H, int 
     } else {
       T* cache = (part == 1) ? kc : vc;
       cache[(((size_t)b * H + hh) * cap + pos) * d + e] = from_f<T>(v);
+      if (part == 2 && vt) vt[(((size_t)b * H + hh) * d + e) * vt_ld + pos] = from_f<T>(v);
     }
   }
 }
 
 cudaError_t launch_rope_append(int dt, const void* qkv, int M, int D, int H, int rot,
                                const float2* rope_tab, PosSpec pos, void* q_out, void* k_cache,
-                               void* v_cache, int cap, cudaStream_t s) {
+                               void* v_cache, int cap, cudaStream_t s, void* vt, int vt_ld) {
   if (M == 0) return cudaSuccess;
   if (dt == DT_BF16) {
     BT_LAUNCH(rope_append_kernel<bf16>, dim3(M), dim3(256), 0, s, (const bf16*)qkv, D, H, rot, rope_tab, pos,
-                                               (bf16*)q_out, (bf16*)k_cache, (bf16*)v_cache, cap);
+                                               (bf16*)q_out, (bf16*)k_cache, (bf16*)v_cache, cap, (bf16*)vt, vt_ld);
   }
   else {
     BT_LAUNCH(rope_append_kernel<float>, dim3(M), dim3(256), 0, s, (const float*)qkv, D, H, rot, rope_tab, pos,
                                                 (float*)q_out, (float*)k_cache, (float*)v_cache,
-                                                cap);
+                                                cap, (float*)vt, vt_ld);
   }
   return cudaGetLastError();
 }

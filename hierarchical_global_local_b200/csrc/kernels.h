@@ -44,9 +44,11 @@ cudaError_t launch_ln_rows(int dt, const float* h, int R, int row_step, int row_
 // pos_base(pos) + m % rows_per_seq. Writes rotated q to q_out [M, D] and
 // rotated k, v to the caches [B][H][cap][d] at that position.
 // rope_tab[p * (rot/2) + i] = (cos, sin) of p * base^(-2i/rot).
+// vt (optional, may be null): also write V transposed, vt[(b*H + h)*d + e][pos].
 cudaError_t launch_rope_append(int dt, const void* qkv, int M, int D, int H, int rot,
                                const float2* rope_tab, PosSpec pos, void* q_out, void* k_cache,
-                               void* v_cache, int cap, cudaStream_t s);
+                               void* v_cache, int cap, cudaStream_t s, void* vt = nullptr,
+                               int vt_ld = 0);
 cudaError_t launch_rope_table(float2* tab, int n_pos, int rot, float base, cudaStream_t s);
 
 // ---- attention --------------------------------------------------------------
@@ -67,6 +69,12 @@ cudaError_t launch_attn_decode(int dt, const void* q, int ldq, const void* k_cac
 cudaError_t launch_attn_small(int dt, const void* q, int ldq, const void* k_cache,
                               const void* v_cache, int B, int H, int d, int cap, PosSpec qpos,
                               void* out, int ld_out, cudaStream_t s);
+// Tensor-core prefill attention (bf16, d in {64, 128}): as launch_attn_prefill
+// but V is read through its transpose vt [B*H][d][vt_ld] (keys contiguous).
+int attn_prefill_tc_supported(int dt, int d, int ldq, int vt_ld);
+cudaError_t launch_attn_prefill_tc(const void* q, int ldq, const void* k_cache, const void* vt,
+                                   int vt_ld, int B, int H, int d, int cap, int n, void* out,
+                                   int ld_out, int* status, cudaStream_t s);
 // Prefill causal attention over n positions 0..n-1 of every sequence:
 // q rows b*n + i of q [B*n, ldq]; out rows likewise.
 cudaError_t launch_attn_prefill(int dt, const void* q, int ldq, const void* k_cache,

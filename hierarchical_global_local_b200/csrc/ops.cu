@@ -43,6 +43,15 @@ int bt_op_prefill_attention(int dtype, const void* q, int ldq, const void* k, co
                                        (cudaStream_t)stream));
 }
 
+int bt_op_prefill_attention_tc(const void* q, int ldq, const void* k, const void* vt, int vt_ld,
+                               int B, int H, int d, int cap, int n, void* out, int ld_out,
+                               void* stream) {
+  if (!q || !k || !vt || !out || B <= 0 || H <= 0 || n < 1 || n > cap || vt_ld < n) return BT_EINVAL;
+  if (!attn_prefill_tc_supported(BT_BF16, d, ldq, vt_ld)) return BT_ENOTSUP;
+  return status_of(launch_attn_prefill_tc(q, ldq, k, vt, vt_ld, B, H, d, cap, n, out, ld_out,
+                                          nullptr, (cudaStream_t)stream));
+}
+
 size_t bt_op_linear_scratch_bytes(int M, int N) {
   if (M <= 0 || N <= 0) return 0;
   return gemm_scratch_bytes(M, N) + 256 + (size_t)gemm_counter_count(N) * 4;

@@ -126,6 +126,8 @@ struct bt_model {
   int *dstate = nullptr, *status = nullptr;
   float2* rope_tab = nullptr;
   void* attn_scratch = nullptr;
+  void* vtr = nullptr;         // V transposed [B_max*H*d][vt_ld] for the prefill attention
+  int vt_ld = 0;
   float2* arg_part = nullptr;  // LM-head per-tile argmax partials
   GemmScratch gs{};
   int B = 0, t = 0;
@@ -232,6 +234,8 @@ static size_t carve(bt_model* m, const Dims& d, void* ws) {
   m->rope_tab = (float2*)c.take((size_t)d.tab_pos * (d.rot / 2 > 0 ? d.rot / 2 : 1) * 8);
   m->attn_scratch = c.take(attn_decode_scratch_bytes(d.Bmax, d.H, d.d, d.n_cap, d.dt));
   m->arg_part = (float2*)c.take((size_t)((d.V + 127) / 128) * d.Bmax * sizeof(float2));
+  m->vt_ld = (d.n_cap + 63) / 64 * 64;
+  m->vtr = c.take((size_t)d.Bmax * D * m->vt_ld * eb);
   const int maxN = 7 * d.D > d.V ? 7 * d.D : d.V;
   m->gs.part_bytes = gemm_scratch_bytes(d.Bmax, maxN);
   m->gs.part = (float*)c.take(m->gs.part_bytes);
@@ -378,12 +382,19 @@ static int run_layer(bt_model* m, const LayerW& w, float* h, int M, PosSpec pos,
       BT_CUDA(launch_gemm(d.dt, m->x1, 2 * D, w.w_qkv1, D, M, 7 * D, D, 3 * D, D, e1, m->gs, m->status, s));
     }
     ProfScope p(m, s, BT_K_ROPE_APPEND, M, 3 * D, 0);
-    BT_CUDA(launch_rope_append(d.dt, m->qkv, M, D, d.H, d.rot, m->rope_tab, pos, m->qrot, kc, vc, cap, s));
+    // the tensor-core prefill attention reads V through its transpose
+    const bool vt = ak == ATT_PREFILL && attn_prefill_tc_supported(d.dt, d.d, D, m->vt_ld);
+    BT_CUDA(launch_rope_append(d.dt, m->qkv, M, D, d.H, d.rot, m->rope_tab, pos, m->qrot, kc, vc,
+                               cap, s, vt ? m->vtr : nullptr, m->vt_ld));
   }
   const int Bseq = M / pos.rows_per_seq;
   if (ak == ATT_PREFILL) {
     ProfScope p(m, s, BT_K_ATTN_PREFILL, Bseq * d.H, n_prefill, d.d);
-    BT_CUDA(launch_attn_prefill(d.dt, m->qrot, D, kc, vc, Bseq, d.H, d.d, cap, n_prefill, m->a2, 5 * D, s));
+    if (attn_prefill_tc_supported(d.dt, d.d, D, m->vt_ld))
+      BT_CUDA(launch_attn_prefill_tc(m->qrot, D, kc, m->vtr, m->vt_ld, Bseq, d.H, d.d, cap, n_prefill,
+                                     m->a2, 5 * D, m->status, s));
+    else
+      BT_CUDA(launch_attn_prefill(d.dt, m->qrot, D, kc, vc, Bseq, d.H, d.d, cap, n_prefill, m->a2, 5 * D, s));
   } else if (ak == ATT_DECODE) {
     // entries read: the block index of the fed token + 1 (known on the host)
     ProfScope p(m, s, BT_K_ATTN_DECODE, Bseq * d.H, m->t / d.L + 1, d.d);

@@ -90,6 +90,9 @@ def lib() -> ctypes.CDLL:
             "bt_op_prefill_attention": (c_int, [c_int, c_void_p, c_int, c_void_p, c_void_p, c_int,
                                                 c_int, c_int, c_int, c_int, c_void_p, c_int,
                                                 c_void_p]),
+            "bt_op_prefill_attention_tc": (c_int, [c_void_p, c_int, c_void_p, c_void_p, c_int, c_int,
+                                                   c_int, c_int, c_int, c_int, c_void_p, c_int,
+                                                   c_void_p]),
             "bt_op_linear_scratch_bytes": (c_size_t, [c_int, c_int]),
             "bt_op_linear": (c_int, [c_int, c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_int,
                                      c_int, c_int, c_int, c_int, c_void_p, c_size_t, c_void_p]),
@@ -114,7 +117,8 @@ def exported_symbols():
         "bt_kernel_launches", "bt_profile_begin", "bt_profile_end",
         "bt_op_decode_attention_scratch_bytes", "bt_op_decode_attention",
         "bt_op_decode_attention_noalloc",
-        "bt_op_prefill_attention", "bt_op_linear_scratch_bytes", "bt_op_linear",
+        "bt_op_prefill_attention", "bt_op_prefill_attention_tc",
+        "bt_op_linear_scratch_bytes", "bt_op_linear",
         "bt_op_layernorm", "bt_op_embed_prompt"]
 
 
@@ -307,6 +311,21 @@ def prefill_attention(q, k, v, n: int, out=None):
     _check(lib().bt_op_prefill_attention(_dt(q), q.data_ptr(), q.stride(0), k.data_ptr(),
                                          v.data_ptr(), B, H, d, cap, n, out.data_ptr(),
                                          out.stride(0), _stream()), "bt_op_prefill_attention")
+    return out
+
+
+def prefill_attention_tc(q, k, v, n: int, out=None):
+    """Tensor-core prefill attention; builds V^T [B*H][d][vt_ld] from v."""
+    import torch
+    B, H, cap, d = k.shape
+    vt_ld = (cap + 63) // 64 * 64
+    vt = torch.zeros(B * H * d, vt_ld, dtype=v.dtype, device="cuda")
+    vt[:, :cap] = v.permute(0, 1, 3, 2).reshape(B * H * d, cap)
+    if out is None:
+        out = torch.empty(B * n, H * d, dtype=q.dtype, device="cuda")
+    _check(lib().bt_op_prefill_attention_tc(q.data_ptr(), q.stride(0), k.data_ptr(), vt.data_ptr(),
+                                            vt_ld, B, H, d, cap, n, out.data_ptr(), out.stride(0),
+                                            _stream()), "bt_op_prefill_attention_tc")
     return out
 
 

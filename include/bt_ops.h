@@ -67,6 +67,14 @@ BT_API int bt_op_prefill_attention(int dtype, const void *q_dev, int ldq, const 
                             const void *v_dev, int B, int H, int d, int cap, int n,
                             void *out_dev, int ld_out, void *stream);
 
+/* Tensor-core form of bt_op_prefill_attention (bf16, d in {64, 128}): the same
+ * causal attention, with V read through its transpose vt_dev [B*H][d][vt_ld]
+ * (vt[(b*H + h)*d + e][i] = V[b][h][i][e]); vt_ld a multiple of 8. Returns
+ * BT_ENOTSUP for other types or head sizes. */
+BT_API int bt_op_prefill_attention_tc(const void *q_dev, int ldq, const void *k_dev,
+                                      const void *vt_dev, int vt_ld, int B, int H, int d, int cap,
+                                      int n, void *out_dev, int ld_out, void *stream);
+
 /* Dense projection out = X W^T (+ bias): X [M, ldx] dtype, W [N, K] dtype
  * row-major, bias fp32 [N] or NULL, out fp32 [M, ld_out]. path: 0 automatic
  * (tensor cores when the shape allows), 1 SIMT FFMA, 2 tensor cores only

@@ -172,3 +172,27 @@ def test_decode_attention_bench_shapes(B, H, d, n, cap):
     vr = v[:, :, :n].double().cpu().numpy().transpose(0, 2, 1, 3)
     ref = om.attend(qr, kr, vr, np.array([n - 1]), np.arange(n)).reshape(B, H * d)
     assert np.abs(out - ref).max() <= 2e-2
+
+
+@pytest.mark.parametrize("B,H,d,n,cap", [(2, 3, 64, 1, 8), (2, 2, 64, 37, 40), (1, 2, 64, 128, 128),
+                                         (2, 2, 64, 300, 320), (1, 2, 128, 129, 136),
+                                         (2, 1, 128, 513, 520)])
+def test_prefill_attention_tensor_cores_matches_oracle(B, H, d, n, cap):
+    """tcgen05 flash-attention prefill (query tiles of 128, causal and tail
+    masking) against the oracle's causal attention in fp64."""
+    from hierarchical_global_local_b200 import native
+    torch = gh.torch_mod()
+    g = torch.Generator(device="cuda").manual_seed(n * 13 + d)
+    q = torch.randn(B * n, H * d, device="cuda", generator=g).bfloat16()
+    k = torch.randn(B, H, cap, d, device="cuda", generator=g).bfloat16()
+    v = torch.randn(B, H, cap, d, device="cuda", generator=g).bfloat16()
+    # rows past n hold garbage in a real cache: make them huge to catch leaks
+    k[:, :, n:] = 3e4
+    v[:, :, n:] = float("nan")
+    out = native.prefill_attention_tc(q, k, v, n).float().cpu().numpy()
+    qr = q.double().cpu().numpy().reshape(B, n, H, d)
+    kr = k[:, :, :n].double().cpu().numpy().transpose(0, 2, 1, 3)
+    vr = v[:, :, :n].double().cpu().numpy().transpose(0, 2, 1, 3)
+    ref = om.attend(qr, kr, vr, np.arange(n), np.arange(n)).reshape(B * n, H * d)
+    assert np.isfinite(out).all()
+    assert np.abs(out - ref).max() <= 3e-2
