@@ -369,7 +369,10 @@ static int run_layer(bt_model* m, const LayerW& w, float* h, int M, PosSpec pos,
     ProfScope p(m, s, BT_K_LAYERNORM, M, D, 0);
     BT_CUDA(launch_ln_dual(d.dt, h, M, D, w.ln1_g, w.ln1_b, w.ln2_g, w.ln2_b, m->cfg.ln_eps, m->x1, s));
   }
-  if (gemm_rope_fusable(d.dt, M, 7 * D, D, 3 * D, D, d.d, d.rot)) {
+  // the fused rotary epilogue does not write V^T, which the tensor-core
+  // prefill attention reads: prefill takes the separate rotary kernel then
+  const bool pf_tc = ak == ATT_PREFILL && attn_prefill_tc_supported(d.dt, d.d, D, m->vt_ld);
+  if (!pf_tc && gemm_rope_fusable(d.dt, M, 7 * D, D, 3 * D, D, d.d, d.rot)) {
     // q|k|v|fc1 GEMM with rotary and the KV-cache append in its epilogue
     ProfScope p(m, s, BT_K_GEMM, M, 7 * D, D);
     Epi e1{EPI_QKV1_ROPE, m->qrot, D, m->a2, 5 * D, w.b_qkv1, 3 * D, D,
@@ -383,9 +386,8 @@ static int run_layer(bt_model* m, const LayerW& w, float* h, int M, PosSpec pos,
     }
     ProfScope p(m, s, BT_K_ROPE_APPEND, M, 3 * D, 0);
     // the tensor-core prefill attention reads V through its transpose
-    const bool vt = ak == ATT_PREFILL && attn_prefill_tc_supported(d.dt, d.d, D, m->vt_ld);
     BT_CUDA(launch_rope_append(d.dt, m->qkv, M, D, d.H, d.rot, m->rope_tab, pos, m->qrot, kc, vc,
-                               cap, s, vt ? m->vtr : nullptr, m->vt_ld));
+                               cap, s, pf_tc ? m->vtr : nullptr, m->vt_ld));
   }
   const int Bseq = M / pos.rows_per_seq;
   if (ak == ATT_PREFILL) {
