@@ -80,6 +80,77 @@ __global__ void ingest_kernel(const int32_t* __restrict__ src, int32_t* __restri
   }
 }
 
+// ingest + LayerNorm of the gathered row (one CTA of 128 threads per row)
+__global__ void __launch_bounds__(128)
+ingest_ln_kernel(const int32_t* __restrict__ src, int32_t* __restrict__ block_tok,
+                 const int* __restrict__ dstate, int L_B, int V, int D, int block_step,
+                 const bf16* __restrict__ blk_emb, const bf16* __restrict__ tok_emb,
+                 float* __restrict__ h, const float* __restrict__ g1, const float* __restrict__ b1,
+                 const float* __restrict__ g2, const float* __restrict__ b2, float eps,
+                 bf16* __restrict__ x, int* status) {
+  pdl_trigger();
+  pdl_wait();
+  __shared__ float row[2048];
+  __shared__ float red[4];
+  const int b = blockIdx.x;
+  const int j = dstate[1];
+  int tok = src[b];
+  if (tok < 0 || tok >= V) {
+    if (threadIdx.x == 0) set_status(status, ST_BAD_TOKEN);
+    tok = 0;
+  }
+  if (threadIdx.x == 0) block_tok[b * L_B + j] = tok;
+  const int De = D / L_B;
+  float s1 = 0.f;
+  for (int c = threadIdx.x; c < D; c += 128) {
+    float v;
+    if (!block_step) {
+      v = __bfloat162float(tok_emb[(size_t)tok * D + c]);
+    } else {
+      const int jj = c / De, e = c - jj * De;
+      int t = (jj == j) ? tok : block_tok[b * L_B + jj];
+      if (t < 0 || t >= V) t = 0;
+      v = __bfloat162float(blk_emb[(size_t)t * De + e]);
+    }
+    row[c] = v;
+    h[(size_t)b * D + c] = v;
+    s1 += v;
+  }
+  s1 = warp_sum(s1);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s1;
+  __syncthreads();
+  const float mu = ((red[0] + red[1]) + (red[2] + red[3])) / (float)D;
+  __syncthreads();
+  float s2 = 0.f;
+  for (int c = threadIdx.x; c < D; c += 128) {
+    const float d = row[c] - mu;
+    s2 += d * d;
+  }
+  s2 = warp_sum(s2);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s2;
+  __syncthreads();
+  const float rstd = rsqrtf(((red[0] + red[1]) + (red[2] + red[3])) / (float)D + eps);
+  const bool dual = g2 != nullptr;
+  bf16* o = x + (size_t)b * (dual ? 2 * D : D);
+  for (int c = threadIdx.x; c < D; c += 128) {
+    const float nv = (row[c] - mu) * rstd;
+    o[c] = __float2bfloat16_rn(nv * g1[c] + b1[c]);
+    if (dual) o[D + c] = __float2bfloat16_rn(nv * g2[c] + b2[c]);
+  }
+}
+
+cudaError_t launch_ingest_ln(const int32_t* src, int32_t* block_tok, const int* dstate, int B,
+                             int L_B, int V, int D, int block_step, const void* blk_emb,
+                             const void* tok_emb, float* h, const float* g1, const float* b1,
+                             const float* g2, const float* b2, float eps, void* x, int* status,
+                             cudaStream_t s) {
+  if (D > 2048) return cudaErrorInvalidValue;
+  BT_LAUNCH(ingest_ln_kernel, dim3(B), dim3(128), 0, s, src, block_tok, dstate, L_B, V, D,
+            block_step, (const bf16*)blk_emb, (const bf16*)tok_emb, h, g1, b1, g2, b2, eps,
+            (bf16*)x, status);
+  return cudaSuccess;
+}
+
 __global__ void set_state_kernel(int* dstate, int t, int L_B) {
   pdl_trigger();
   pdl_wait();
@@ -389,7 +460,7 @@ cudaError_t launch_argmax(const float* logits, int B, int V, int ld, int32_t* ne
 }
 
 __global__ void argmax_reduce_kernel(const float2* __restrict__ part, int n_tiles, int M,
-                                     int32_t* __restrict__ next) {
+                                     int32_t* __restrict__ next, int* dstate, int L_B) {
   pdl_trigger();
   pdl_wait();
   const int m = blockIdx.x;
@@ -415,13 +486,19 @@ __global__ void argmax_reduce_kernel(const float2* __restrict__ part, int n_tile
     for (int k = 1; k < (int)(blockDim.x >> 5); ++k)
       if (sv[k] > best || (sv[k] == best && si[k] < bi)) { best = sv[k]; bi = si[k]; }
     next[m] = (bi == 0x7fffffff) ? 0 : bi;
+    if (dstate && m == 0) {  // the step is over: advance the position
+      const int t = dstate[0] + 1;
+      dstate[0] = t;
+      dstate[1] = t % L_B;
+      dstate[2] = t / L_B;
+    }
   }
 }
 
 cudaError_t launch_argmax_reduce(const float2* part, int n_tiles, int M, int32_t* next,
-                                 cudaStream_t s) {
+                                 cudaStream_t s, int* dstate, int L_B) {
   if (M == 0) return cudaSuccess;
-  BT_LAUNCH(argmax_reduce_kernel, dim3(M), dim3(256), 0, s, part, n_tiles, M, next);
+  BT_LAUNCH(argmax_reduce_kernel, dim3(M), dim3(256), 0, s, part, n_tiles, M, next, dstate, L_B);
   return cudaGetLastError();
 }
 

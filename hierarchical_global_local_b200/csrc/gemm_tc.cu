@@ -125,6 +125,74 @@ __host__ __device__ constexpr int tmem_cols() {
   return 2 * BN < 32 ? 32 : 2 * BN;
 }
 
+// Fused LayerNorm (see Epi::ln_*): called by the four epilogue warps after
+// they stored rows [m_lo, m_hi) of out0 for this feature tile. The tile that
+// completes a row (counter reaches the number of feature tiles) normalises
+// it; every other tile only counts. One warp per row.
+__device__ __forceinline__ void ep_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+__device__ void post_ln(const Epi& e, int m_lo, int m_hi, int M, int N, int nfeat_tiles,
+                        int* s_rows, int* s_n) {
+  __threadfence();
+  ep_sync();
+  if (threadIdx.x == 0) *s_n = 0;
+  ep_sync();
+  for (int m = m_lo + (int)threadIdx.x; m < m_hi && m < M; m += 128)
+    if (atomicAdd(&e.ln_cnt[m], 1) == nfeat_tiles - 1) s_rows[atomicAdd(s_n, 1)] = m;
+  ep_sync();
+  const int nrows = *s_n;
+  __threadfence();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const float* hsrc = reinterpret_cast<const float*>(e.out0);
+  for (int i = warp; i < nrows; i += 4) {
+    const int m = s_rows[i];
+    const float* x = hsrc + (size_t)m * e.ld0;
+    float sum = 0.f;
+    for (int c = lane * 4; c < N; c += 128) {
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(x + c));
+      sum += (v.x + v.y) + (v.z + v.w);
+    }
+    const float mu = warp_sum(sum) / (float)N;
+    float sq = 0.f;
+    for (int c = lane * 4; c < N; c += 128) {
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(x + c));
+      const float a = v.x - mu, b = v.y - mu, cc = v.z - mu, d = v.w - mu;
+      sq += (a * a + b * b) + (cc * cc + d * d);
+    }
+    const float rstd = rsqrtf(warp_sum(sq) / (float)N + e.ln_eps);
+    const bool dual = e.ln_g2 != nullptr;
+    const bool take = dual || (m % e.ln_step) == e.ln_off;
+    if (take) {
+      bf16* o = reinterpret_cast<bf16*>(e.ln_out) +
+                (dual ? (size_t)m * 2 * N : (size_t)(m / e.ln_step) * N);
+      for (int c = lane * 4; c < N; c += 128) {
+        const float4 v = __ldcg(reinterpret_cast<const float4*>(x + c));
+        const float n0 = (v.x - mu) * rstd, n1 = (v.y - mu) * rstd;
+        const float n2 = (v.z - mu) * rstd, n3 = (v.w - mu) * rstd;
+        const float4 g = *reinterpret_cast<const float4*>(e.ln_g1 + c);
+        const float4 bb = *reinterpret_cast<const float4*>(e.ln_b1 + c);
+        __nv_bfloat162 lo = __floats2bfloat162_rn(n0 * g.x + bb.x, n1 * g.y + bb.y);
+        __nv_bfloat162 hi = __floats2bfloat162_rn(n2 * g.z + bb.z, n3 * g.w + bb.w);
+        uint2 u;
+        u.x = *reinterpret_cast<uint32_t*>(&lo);
+        u.y = *reinterpret_cast<uint32_t*>(&hi);
+        *reinterpret_cast<uint2*>(o + c) = u;
+        if (dual) {
+          const float4 g2 = *reinterpret_cast<const float4*>(e.ln_g2 + c);
+          const float4 b2 = *reinterpret_cast<const float4*>(e.ln_b2 + c);
+          lo = __floats2bfloat162_rn(n0 * g2.x + b2.x, n1 * g2.y + b2.y);
+          hi = __floats2bfloat162_rn(n2 * g2.z + b2.z, n3 * g2.w + b2.w);
+          u.x = *reinterpret_cast<uint32_t*>(&lo);
+          u.y = *reinterpret_cast<uint32_t*>(&hi);
+          *reinterpret_cast<uint2*>(o + N + c) = u;
+        }
+      }
+    }
+    if (lane == 0) e.ln_cnt[m] = 0;
+  }
+  ep_sync();  // s_rows / s_n reused by the next tile
+}
+
 // ---- the kernel ---------------------------------------------------------------
 // SWAP = true: A = weights (rows = output features), B = activations (rows =
 // tokens). SWAP = false: A = activations, B = weights.
@@ -146,6 +214,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
   __shared__ __align__(8) uint64_t full[MAX_STAGES], empty[MAX_STAGES], acc_full[2], acc_empty[2];
   __shared__ uint32_t tmem_slot;
   __shared__ float2 s_arg[4][BN <= 64 ? BN : 1];  // fused argmax: per warp, per column
+  __shared__ int s_rows[256];                      // fused LayerNorm: rows completed here
+  __shared__ int s_nrows;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ntiles = ntA * ntB;
@@ -341,6 +411,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
             epi_apply<bf16>(e, m, n, v[c]);
           }
         }
+        if (SWAP && e.ln_cnt) post_ln(e, b0, b0 + BN, M, N, ntA, s_rows, &s_nrows);
       } else {
         for (int c0 = 0; c0 < BN; c0 += 16) {
           float v[16];
@@ -359,6 +430,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
         }
         tc_fence_before();
         mbar_arrive(&acc_empty[buf]);
+        if (SWAP && e.ln_cnt) post_ln(e, b0, b0 + BN, M, N, ntA, s_rows, &s_nrows);
       }
     }
   }
@@ -395,6 +467,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
           epi_apply<bf16>(e, m, n, acc);
         }
       }
+      if (SWAP && e.ln_cnt) post_ln(e, b0 + cbeg, b0 + cbeg + cpr, M, N, ntA, s_rows, &s_nrows);
     }
   }
 

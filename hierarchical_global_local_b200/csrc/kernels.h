@@ -25,6 +25,13 @@ cudaError_t launch_embed_prompt(int dt, const int32_t* tokens, int B, int T, int
 cudaError_t launch_ingest(int dt, const int32_t* src, int32_t* block_tok, const int* dstate,
                           int B, int L_B, int V, int D, int block_step, const void* blk_emb,
                           const void* tok_emb, float* h, int* status, cudaStream_t s);
+// Ingest plus the first LayerNorm(s) of the gathered row (bf16): g2 != null ->
+// x[b] = [LN1 | LN2] ([B, 2D]); else x[b] = LN(h[b]) ([B, D]).
+cudaError_t launch_ingest_ln(const int32_t* src, int32_t* block_tok, const int* dstate, int B,
+                             int L_B, int V, int D, int block_step, const void* blk_emb,
+                             const void* tok_emb, float* h, const float* g1, const float* b1,
+                             const float* g2, const float* b2, float eps, void* x, int* status,
+                             cudaStream_t s);
 // dstate <- position t (t, t % L_B, t / L_B).
 cudaError_t launch_set_state(int* dstate, int t, int L_B, cudaStream_t s);
 // dstate <- dstate[0] + 1.
@@ -117,13 +124,28 @@ struct Epi {
   PosSpec pos;
   // EPI_LOGITS_ARGMAX only
   void* aux;
+  // Fused LayerNorm of completed rows (EPI_RESID / EPI_F32, tensor-core decode
+  // orientation, N = the full row width D): the feature tile that completes
+  // row m of out0 last computes LayerNorm(s) of that row. ln_g2 != null: both
+  // LN1 and LN2 -> ln_out [M, 2D]; else one LN of rows m % ln_step == ln_off
+  // -> ln_out row m / ln_step. ln_cnt: per-row counters, zero between launches.
+  const float* ln_g1;
+  const float* ln_b1;
+  const float* ln_g2;
+  const float* ln_b2;
+  void* ln_out;
+  int* ln_cnt;
+  int ln_step;
+  int ln_off;
+  float ln_eps;
 };
 // True when launch_gemm runs EPI_LOGITS_ARGMAX for this shape.
 int gemm_argmax_fusable(int dt, int M, int N, int K);
 // next[m] = index of the best of the n_tiles partial (value, index) pairs
 // part[t * M + m] (lowest index among equal values).
+// dstate (optional): advanced to the next position by the same kernel.
 cudaError_t launch_argmax_reduce(const float2* part, int n_tiles, int M, int32_t* next,
-                                 cudaStream_t s);
+                                 cudaStream_t s, int* dstate = nullptr, int L_B = 1);
 // True when launch_gemm will run EPI_QKV1_ROPE fused for this shape.
 int gemm_rope_fusable(int dt, int M, int N, int K, int xk_split, int xk_off, int d_head, int rot);
 

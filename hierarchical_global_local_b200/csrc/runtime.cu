@@ -129,6 +129,7 @@ struct bt_model {
   void* vtr = nullptr;         // V transposed [B_max*H*d][vt_ld] for the prefill attention
   int vt_ld = 0;
   float2* arg_part = nullptr;  // LM-head per-tile argmax partials
+  int* ln_cnt = nullptr;       // per-row counters of the LayerNorm fused into GEMM epilogues
   GemmScratch gs{};
   int B = 0, t = 0;
   bool prefilled = false;
@@ -234,6 +235,7 @@ static size_t carve(bt_model* m, const Dims& d, void* ws) {
   m->rope_tab = (float2*)c.take((size_t)d.tab_pos * (d.rot / 2 > 0 ? d.rot / 2 : 1) * 8);
   m->attn_scratch = c.take(attn_decode_scratch_bytes(d.Bmax, d.H, d.d, d.n_cap, d.dt));
   m->arg_part = (float2*)c.take((size_t)((d.V + 127) / 128) * d.Bmax * sizeof(float2));
+  m->ln_cnt = (int*)c.take((size_t)d.Bmax * (d.P > 1 ? d.P : 1) * sizeof(int));
   m->vt_ld = (d.n_cap + 63) / 64 * 64;
   m->vtr = c.take((size_t)d.Bmax * D * m->vt_ld * eb);
   const int maxN = 7 * d.D > d.V ? 7 * d.D : d.V;
@@ -345,6 +347,7 @@ int bt_create(const bt_config* cfg, const bt_weights* w, void* ws, size_t ws_byt
   BT_TRYC(cudaMemsetAsync(m->attn_scratch, 0, attn_decode_scratch_bytes(d.Bmax, d.H, d.d, d.n_cap, d.dt), st));
   BT_TRYC(cudaMemsetAsync(m->gs.counters, 0, (size_t)m->gs.n_counters * 4, st));
   BT_TRYC(cudaMemsetAsync(m->block_tok, 0, (size_t)d.Bmax * d.L * 4, st));
+  BT_TRYC(cudaMemsetAsync(m->ln_cnt, 0, (size_t)d.Bmax * (d.P > 1 ? d.P : 1) * sizeof(int), st));
   BT_TRYC(cudaStreamCreateWithFlags(&m->cap_stream, cudaStreamNonBlocking));
   if (d.dt == BT_BF16) BT_TRYC(gemm_tc_prepare());
   BT_TRYC(attn_prepare());
@@ -361,11 +364,47 @@ int bt_create(const bt_config* cfg, const bt_weights* w, void* ws, size_t ws_byt
 // ---------------------------------------------------------------------------
 enum AttnKind { ATT_PREFILL, ATT_DECODE, ATT_LOCAL };
 
+// LayerNorm to fuse into the epilogue of a GEMM that completes residual rows
+// (decode): dual (g2 != null) -> x1; single -> rows m % step == off of xf.
+struct NextLN {
+  const float *g1 = nullptr, *b1 = nullptr, *g2 = nullptr, *b2 = nullptr;
+  void* out = nullptr;
+  int step = 1, off = 0;
+};
+
+static void attach_ln(bt_model* m, Epi& e, const NextLN* nl) {
+  if (!nl || !nl->g1) return;
+  e.ln_g1 = nl->g1; e.ln_b1 = nl->b1; e.ln_g2 = nl->g2; e.ln_b2 = nl->b2;
+  e.ln_out = nl->out; e.ln_cnt = m->ln_cnt; e.ln_step = nl->step; e.ln_off = nl->off;
+  e.ln_eps = m->cfg.ln_eps;
+}
+
+static NextLN dual_ln(bt_model* m, const LayerW& w) {
+  NextLN n;
+  n.g1 = w.ln1_g; n.b1 = w.ln1_b; n.g2 = w.ln2_g; n.b2 = w.ln2_b; n.out = m->x1;
+  return n;
+}
+
+static NextLN single_ln(bt_model* m, const float* g, const float* b, int step, int off) {
+  NextLN n;
+  n.g1 = g; n.b1 = b; n.out = m->xf; n.step = step; n.off = off;
+  return n;
+}
+
+// The decode schedule with every LayerNorm fused (ingest and GEMM epilogues)
+// needs the tensor-core decode GEMMs and P = 1.
+static bool fused_decode(const bt_model* m, int B) {
+  const Dims& d = m->d;
+  return d.dt == BT_BF16 && B <= 256 && d.D <= 2048 && (d.D % 128) == 0 &&
+         gemm_tc_supported(d.dt, B, d.D, 5 * d.D, 1 << 30, 0) && (!d.tokdec || d.P == 1);
+}
+
 static int run_layer(bt_model* m, const LayerW& w, float* h, int M, PosSpec pos, void* kc,
-                     void* vc, int cap, AttnKind ak, int n_prefill, cudaStream_t s) {
+                     void* vc, int cap, AttnKind ak, int n_prefill, cudaStream_t s,
+                     bool ln_done = false, const NextLN* next = nullptr) {
   const Dims& d = m->d;
   const int D = d.D;
-  {
+  if (!ln_done) {
     ProfScope p(m, s, BT_K_LAYERNORM, M, D, 0);
     BT_CUDA(launch_ln_dual(d.dt, h, M, D, w.ln1_g, w.ln1_b, w.ln2_g, w.ln2_b, m->cfg.ln_eps, m->x1, s));
   }
@@ -409,6 +448,7 @@ static int run_layer(bt_model* m, const LayerW& w, float* h, int M, PosSpec pos,
   {
     ProfScope p(m, s, BT_K_GEMM, M, D, 5 * D);
     Epi e2{EPI_RESID, h, D, nullptr, 0, w.b_o2, 0, D};
+    attach_ln(m, e2, next);
     BT_CUDA(launch_gemm(d.dt, m->a2, 5 * D, w.w_o2, 5 * D, M, D, 5 * D, 1 << 30, 0, e2, m->gs, m->status, s));
   }
   return BT_OK;
@@ -491,11 +531,87 @@ static int copy_outputs(bt_model* m, float* logits, int32_t* next) {
   return BT_OK;
 }
 
+// Decode call with every LayerNorm fused: the ingest kernel normalises the
+// gathered row for the first layer, each layer's residual GEMM normalises the
+// completed rows for the next layer (or the final norm), and the argmax
+// reduction advances the position.
+static int enqueue_decode_fused(bt_model* m, bool block_step, bool greedy, bool want_logits,
+                                cudaStream_t s) {
+  const Dims& d = m->d;
+  const int B = m->B;
+  const int32_t* src = greedy ? m->next : m->fed;
+  const NextLN lnb = single_ln(m, m->lnf_b_g, m->lnf_b_b, 1, 0);
+  const NextLN lnt = d.tokdec ? single_ln(m, m->lnf_t_g, m->lnf_t_b, 1, 0) : NextLN();
+  // first LayerNorm of this call
+  NextLN first;
+  if (block_step) first = d.Nb > 0 ? dual_ln(m, m->blk[0]) : lnb;
+  else first = d.Nt > 0 ? dual_ln(m, m->tok[0]) : lnt;
+  {
+    ProfScope p(m, s, BT_K_EMBED, B, d.D, 0);
+    BT_CUDA(launch_ingest_ln(src, m->block_tok, m->dstate, B, d.L, d.V, d.D, block_step ? 1 : 0,
+                             m->blk_emb, m->tok_emb, block_step ? m->h_b : m->h_t, first.g1,
+                             first.b1, first.g2, first.b2, m->cfg.ln_eps, first.out, m->status, s));
+  }
+  int rc;
+  auto token_layers = [&](PosSpec pos) -> int {
+    for (int l = 0; l < d.Nt; ++l) {
+      const NextLN nx = (l + 1 < d.Nt) ? dual_ln(m, m->tok[l + 1]) : lnt;
+      int r = run_layer(m, m->tok[l], m->h_t, B, pos, layer_ptr(m->kt, m->kt_layer, l, d.eb),
+                        layer_ptr(m->vt, m->kt_layer, l, d.eb), d.l_cap, ATT_LOCAL, 0, s, true, &nx);
+      if (r != BT_OK) return r;
+    }
+    return BT_OK;
+  };
+  if (block_step) {
+    PosSpec pos{m->dstate, POS_BLOCK, 0, 1};
+    for (int l = 0; l < d.Nb; ++l) {
+      const NextLN nx = (l + 1 < d.Nb) ? dual_ln(m, m->blk[l + 1]) : lnb;
+      rc = run_layer(m, m->blk[l], m->h_b, B, pos, layer_ptr(m->kb, m->kb_layer, l, d.eb),
+                     layer_ptr(m->vb, m->kb_layer, l, d.eb), d.n_cap, ATT_DECODE, 0, s, true, &nx);
+      if (rc != BT_OK) return rc;
+    }
+    if (d.tokdec) {
+      // prefix rows (P = 1) with the token decoder's first LayerNorm fused
+      const NextLN nx = d.Nt > 0 ? dual_ln(m, m->tok[0]) : lnt;
+      ProfScope p(m, s, BT_K_GEMM, B, d.D, d.D);
+      Epi ep{EPI_F32, m->h_t, d.D, nullptr, 0, m->b_prefix, 0, d.D};
+      attach_ln(m, ep, &nx);
+      BT_CUDA(launch_gemm(d.dt, m->xf, d.D, m->w_prefix, d.D, B, d.D, d.D, 1 << 30, 0, ep, m->gs,
+                          m->status, s));
+    }
+    if (d.tokdec) {
+      rc = token_layers(PosSpec{nullptr, POS_ZERO, 0, 1});
+      if (rc != BT_OK) return rc;
+    }
+  } else {
+    rc = token_layers(PosSpec{m->dstate, POS_LOCAL, d.P, 1});
+    if (rc != BT_OK) return rc;
+  }
+  // LM head on xf (already normalised) + argmax; the reduction advances the step
+  if (gemm_argmax_fusable(d.dt, B, d.V, d.D)) {
+    {
+      ProfScope p(m, s, BT_K_GEMM, B, d.V, d.D);
+      Epi el{EPI_LOGITS_ARGMAX, want_logits ? m->logits : nullptr, d.V, nullptr, 0, nullptr, 0, d.D};
+      el.aux = m->arg_part;
+      BT_CUDA(launch_gemm(d.dt, m->xf, d.D, m->w_lm, d.D, B, d.V, d.D, 1 << 30, 0, el, m->gs, m->status, s));
+    }
+    ProfScope p(m, s, BT_K_ARGMAX, B, d.V, 0);
+    BT_CUDA(launch_argmax_reduce(m->arg_part, (d.V + 127) / 128, B, m->next, s, m->dstate, d.L));
+    return BT_OK;
+  }
+  rc = run_head(m, B, want_logits, s);
+  if (rc != BT_OK) return rc;
+  ProfScope p(m, s, BT_K_OTHER, 1, 0, 0);
+  BT_CUDA(launch_advance(m->dstate, d.L, s));
+  return BT_OK;
+}
+
 // the body of one decode call (captured into a graph or run directly)
 static int enqueue_decode(bt_model* m, bool block_step, bool greedy, bool want_logits,
                           cudaStream_t s) {
   const Dims& d = m->d;
   const int B = m->B;
+  if (fused_decode(m, B)) return enqueue_decode_fused(m, block_step, greedy, want_logits, s);
   const int32_t* src = greedy ? m->next : m->fed;
   {
     ProfScope p(m, s, BT_K_EMBED, B, d.D, 0);
