@@ -144,20 +144,29 @@ __device__ void post_ln(const Epi& e, int m_lo, int m_hi, int M, int N, int nfea
   __threadfence();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const float* hsrc = reinterpret_cast<const float*>(e.out0);
+  constexpr int MAXV = 16;  // float4 per lane: rows up to 2048 wide
   for (int i = warp; i < nrows; i += 4) {
     const int m = s_rows[i];
     const float* x = hsrc + (size_t)m * e.ld0;
-    float sum = 0.f;
-    for (int c = lane * 4; c < N; c += 128) {
-      const float4 v = __ldcg(reinterpret_cast<const float4*>(x + c));
-      sum += (v.x + v.y) + (v.z + v.w);
+    // the whole row in registers: one round trip to L2
+    float4 v[MAXV];
+#pragma unroll
+    for (int u = 0; u < MAXV; ++u) {
+      const int c = (lane + 32 * u) * 4;
+      v[u] = (c < N) ? __ldcg(reinterpret_cast<const float4*>(x + c)) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
+    float sum = 0.f;
+#pragma unroll
+    for (int u = 0; u < MAXV; ++u) sum += (v[u].x + v[u].y) + (v[u].z + v[u].w);
     const float mu = warp_sum(sum) / (float)N;
     float sq = 0.f;
-    for (int c = lane * 4; c < N; c += 128) {
-      const float4 v = __ldcg(reinterpret_cast<const float4*>(x + c));
-      const float a = v.x - mu, b = v.y - mu, cc = v.z - mu, d = v.w - mu;
-      sq += (a * a + b * b) + (cc * cc + d * d);
+#pragma unroll
+    for (int u = 0; u < MAXV; ++u) {
+      const int c = (lane + 32 * u) * 4;
+      if (c < N) {
+        const float a = v[u].x - mu, b = v[u].y - mu, cc = v[u].z - mu, d = v[u].w - mu;
+        sq += (a * a + b * b) + (cc * cc + d * d);
+      }
     }
     const float rstd = rsqrtf(warp_sum(sq) / (float)N + e.ln_eps);
     const bool dual = e.ln_g2 != nullptr;
@@ -165,26 +174,29 @@ __device__ void post_ln(const Epi& e, int m_lo, int m_hi, int M, int N, int nfea
     if (take) {
       bf16* o = reinterpret_cast<bf16*>(e.ln_out) +
                 (dual ? (size_t)m * 2 * N : (size_t)(m / e.ln_step) * N);
-      for (int c = lane * 4; c < N; c += 128) {
-        const float4 v = __ldcg(reinterpret_cast<const float4*>(x + c));
-        const float n0 = (v.x - mu) * rstd, n1 = (v.y - mu) * rstd;
-        const float n2 = (v.z - mu) * rstd, n3 = (v.w - mu) * rstd;
-        const float4 g = *reinterpret_cast<const float4*>(e.ln_g1 + c);
-        const float4 bb = *reinterpret_cast<const float4*>(e.ln_b1 + c);
-        __nv_bfloat162 lo = __floats2bfloat162_rn(n0 * g.x + bb.x, n1 * g.y + bb.y);
-        __nv_bfloat162 hi = __floats2bfloat162_rn(n2 * g.z + bb.z, n3 * g.w + bb.w);
-        uint2 u;
-        u.x = *reinterpret_cast<uint32_t*>(&lo);
-        u.y = *reinterpret_cast<uint32_t*>(&hi);
-        *reinterpret_cast<uint2*>(o + c) = u;
-        if (dual) {
-          const float4 g2 = *reinterpret_cast<const float4*>(e.ln_g2 + c);
-          const float4 b2 = *reinterpret_cast<const float4*>(e.ln_b2 + c);
-          lo = __floats2bfloat162_rn(n0 * g2.x + b2.x, n1 * g2.y + b2.y);
-          hi = __floats2bfloat162_rn(n2 * g2.z + b2.z, n3 * g2.w + b2.w);
-          u.x = *reinterpret_cast<uint32_t*>(&lo);
-          u.y = *reinterpret_cast<uint32_t*>(&hi);
-          *reinterpret_cast<uint2*>(o + N + c) = u;
+#pragma unroll
+      for (int u = 0; u < MAXV; ++u) {
+        const int c = (lane + 32 * u) * 4;
+        if (c < N) {
+          const float n0 = (v[u].x - mu) * rstd, n1 = (v[u].y - mu) * rstd;
+          const float n2 = (v[u].z - mu) * rstd, n3 = (v[u].w - mu) * rstd;
+          const float4 g = *reinterpret_cast<const float4*>(e.ln_g1 + c);
+          const float4 bb = *reinterpret_cast<const float4*>(e.ln_b1 + c);
+          __nv_bfloat162 lo = __floats2bfloat162_rn(n0 * g.x + bb.x, n1 * g.y + bb.y);
+          __nv_bfloat162 hi = __floats2bfloat162_rn(n2 * g.z + bb.z, n3 * g.w + bb.w);
+          uint2 w;
+          w.x = *reinterpret_cast<uint32_t*>(&lo);
+          w.y = *reinterpret_cast<uint32_t*>(&hi);
+          *reinterpret_cast<uint2*>(o + c) = w;
+          if (dual) {
+            const float4 g2 = *reinterpret_cast<const float4*>(e.ln_g2 + c);
+            const float4 b2 = *reinterpret_cast<const float4*>(e.ln_b2 + c);
+            lo = __floats2bfloat162_rn(n0 * g2.x + b2.x, n1 * g2.y + b2.y);
+            hi = __floats2bfloat162_rn(n2 * g2.z + b2.z, n3 * g2.w + b2.w);
+            w.x = *reinterpret_cast<uint32_t*>(&lo);
+            w.y = *reinterpret_cast<uint32_t*>(&hi);
+            *reinterpret_cast<uint2*>(o + N + c) = w;
+          }
         }
       }
     }

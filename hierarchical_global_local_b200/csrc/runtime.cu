@@ -393,8 +393,16 @@ static NextLN single_ln(bt_model* m, const float* g, const float* b, int step, i
 
 // The decode schedule with every LayerNorm fused (ingest and GEMM epilogues)
 // needs the tensor-core decode GEMMs and P = 1.
+// The decode step runs one LayerNorm kernel per layer by default. With
+// BT_DECODE_LN=fused (read when a step kind is first recorded) the GEMM
+// epilogues normalise instead: the last tile to finish a row normalises it.
+// That schedule has fewer launches but measured slower at batch 64 on B200:
+// one CTA then normalises a whole 64-row chunk at the end of the GEMM, where
+// the separate kernel spreads the rows over 64 CTAs.
 static bool fused_decode(const bt_model* m, int B) {
   const Dims& d = m->d;
+  const char* env = getenv("BT_DECODE_LN");
+  if (!env || strcmp(env, "fused") != 0) return false;
   return d.dt == BT_BF16 && B <= 256 && d.D <= 2048 && (d.D % 128) == 0 &&
          gemm_tc_supported(d.dt, B, d.D, 5 * d.D, 1 << 30, 0) && (!d.tokdec || d.P == 1);
 }

@@ -52,6 +52,18 @@ def test_small_bf16_block_transformer(lb, P):
         assert gh.rel_l2(gl[s], ol[s]) <= BF16_REL, (s, gh.rel_l2(gl[s], ol[s]))
 
 
+@pytest.mark.parametrize("lb", [4, 8])
+def test_small_bf16_layernorm_fused_in_gemm_epilogues(lb, monkeypatch):
+    """The decode schedule that normalises in the residual GEMMs' epilogues
+    (opt-in) gives the same logits as the oracle."""
+    monkeypatch.setenv("BT_DECODE_LN", "fused")
+    shape = synth.ModelShape(vocab=1000, d_model=256, n_heads=4, block_len=lb,
+                             n_block_layers=2, n_token_layers=2, prefix_len=1)
+    gl, gn, ol = _run(shape, B=3, T=8 * lb, G=3 * lb + 2, seed=5)
+    for s in range(gl.shape[0]):
+        assert gh.rel_l2(gl[s], ol[s]) <= BF16_REL, (s, gh.rel_l2(gl[s], ol[s]))
+
+
 def test_small_bf16_vanilla_lb1():
     shape = synth.ModelShape(vocab=700, d_model=256, n_heads=2, block_len=1,
                              n_block_layers=3, n_token_layers=0, prefix_len=0,
