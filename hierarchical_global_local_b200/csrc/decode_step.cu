@@ -1,0 +1,991 @@
+// decode_step.cu -- the token-decoder half of a decode step as one persistent
+// kernel (bf16, at most 64 sequences): every token-decoder layer, the final
+// LayerNorm, the LM head and the greedy argmax.
+//
+// Block Transformer (Ho et al., "Block Transformer: Global-to-Local Language
+// Modeling for Fast Inference"), section 2.3 (token decoder) and the Pythia
+// layer it is built from (parallel attention + MLP residual, partial rotary,
+// GELU MLP). The token decoder of one decode step reads every one of its
+// weights once for a single row per sequence: the step is a chain of small
+// weight-streaming GEMMs whose cost, launched as separate kernels, is
+// launch and pipeline-fill latency rather than bytes.
+//
+// Here one CTA per SM runs the whole chain. A producer warp streams every
+// weight tile the CTA will use, in program order, through a shared-memory
+// ring with TMA (weights do not depend on the activations, so the stream
+// runs ahead across layer boundaries and grid barriers); an MMA warp issues
+// the tensor-core work of every unit as soon as its activations are staged
+// and an accumulator is free; the four worker warps stage activations, drain
+// the accumulators and run the phases below, separated by grid-wide barriers:
+//   I   (row b per CTA)  embed the fed token (token steps), LayerNorm 1/2 of
+//                        layer 0 -> x1 = [LN1(h) | LN2(h)] bf16
+//   per layer l:
+//   G1  (tile x K-split) partial sums of x1 W_qkv1^T (q | k | v | fc1) on
+//                        tcgen05 (activation boxes by TMA), fp32 partial
+//                        tiles to L2
+//   R1                   sum the splits + bias; q, k rotary; k, v into the
+//                        local cache; attention over the local window (16
+//                        lanes per sequence and head); GELU(fc1) -> a2
+//   G2  (tile x K-split) partial sums of a2 W_o2^T ([W_o | W_2])
+//   R2  (row b per CTA)  h += splits + b_o + b_2; LayerNorm of the new row
+//                        for the next layer, or the final LayerNorm -> xf
+//   GL  (vocab tiles)    LM head on tcgen05 (two TMEM accumulators: the MMAs
+//                        of one tile overlap the epilogue of the previous);
+//                        logits (optional) and per-tile argmax partials
+//   AR                   greedy argmax per row (lowest id on ties), advance
+//                        the step state
+// The MMA orientation is "weights as A": M = 128 output features per tile,
+// N = the batch padded to a multiple of 16, K in 64-wide swizzled blocks.
+//
+// Grid barriers are a counter in global memory (release by fence + atomic
+// add, acquire by polling with ld.acquire). All CTAs must be resident at
+// once: one CTA per SM, grid = number of SMs. Every wait is bounded: a
+// barrier that runs out sets ST_WAIT_TIMEOUT and an abort word that makes
+// every CTA skip the rest of the step; the producer then waits (bounded) for
+// its copies in flight, TMEM is freed and the kernel returns.
+#include <cuda.h>
+#include <float.h>
+#include <limits.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc.cuh"
+
+namespace bt {
+
+namespace {
+
+constexpr int WORKERS = 128;                 // warps 0-3 (TMEM lanes 0-127)
+constexpr int THREADS = WORKERS + 64;        // warp 4: TMA producer, warp 5: MMA issuer
+constexpr int TILE_BYTES = 128 * 64 * 2;     // one weight box: 128 rows x 64 K (bf16)
+constexpr int MAX_STAGES = 12;
+constexpr int MAX_S1 = 4;                    // K splits of the q|k|v|fc1 GEMM
+constexpr int MAX_S2 = 16;                   // K splits of the [W_o | W_2] GEMM
+constexpr int MAX_B = 64;
+constexpr int MAX_WIN = 8;                   // local-window slots (P + L_B - 1)
+constexpr int TMEM_COLS = 128;               // two accumulators of up to 64 columns
+constexpr long long BAR_CYCLES = 2000000000LL;  // ~1 s at 1.9 GHz
+#ifndef PRODUCER_SLEEP_NS
+#define PRODUCER_SLEEP_NS 128  // back-off of the weight producer's slot waits
+#endif
+#ifndef MMA_SLEEP_NS
+#define MMA_SLEEP_NS 32        // back-off of the MMA warp's waits (on the critical path)
+#endif
+
+struct Plan {
+  int Bp;            // batch padded to a multiple of 16 (MMA N)
+  int S1, S2;        // K splits
+  int T1, T2, TL;    // feature tiles: 7D/128, D/128, ceil(V/128)
+  int nkb1, nkb2;    // 64-wide K blocks per split
+  int nkbL;          // K blocks of the LM head (D/64)
+  int stages;
+  float scale;       // log2(e) / sqrt(d_head)
+};
+
+__device__ __forceinline__ void wsync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+__device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+template <typename T>
+__device__ __forceinline__ const T* layer_ptr(const T* base, int l, long long stride) {
+  return reinterpret_cast<const T*>(reinterpret_cast<const uint8_t*>(base) + (long long)l * stride);
+}
+
+// mbarrier wait of the producer and MMA warps: backs off between polls so
+// that the worker warps sharing their SM sub-partitions keep the issue
+// slots; gives up when the CTA has aborted
+__device__ bool wait_or_abort(uint64_t* bar, uint32_t parity, int* status, volatile int* s_abort,
+                              int sleep_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  int n = 0;
+  while (!mbar_try_wait(bar, parity)) {
+    __nanosleep(sleep_ns);
+    if ((++n & 63) == 0) {
+      if (*s_abort) return false;
+      if (clock64() - t0 > BAR_CYCLES) {
+        set_status(status, ST_WAIT_TIMEOUT);
+        return false;
+      }
+    }
+  }
+  return true;
+}
+
+// Grid-wide barrier for the 128 worker threads of every CTA. `target` is
+// (barriers passed so far + 1) * gridDim.x. Returns false once the step has
+// been aborted (here or in another CTA).
+__device__ bool grid_sync(unsigned* bar, unsigned target, int* status, volatile int* s_abort) {
+  // activations written in this phase are read by TMA (async proxy) later
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+  wsync();  // this CTA's writes of the phase are issued
+  if (threadIdx.x == 0 && !*s_abort) {
+    __threadfence();
+    atomicAdd(&bar[0], 1u);
+    const long long t0 = clock64();
+    int n = 0;
+    while (ld_acquire(&bar[0]) < target) {
+      if ((++n & 63) == 0) {
+        if (ld_acquire(&bar[2]) != 0u) { *s_abort = 1; break; }
+        if (clock64() - t0 > BAR_CYCLES) {
+          atomicExch(&bar[2], 1u);
+          set_status(status, ST_WAIT_TIMEOUT);
+          *s_abort = 1;
+          break;
+        }
+      }
+    }
+    __threadfence();
+  }
+  wsync();
+  return !*s_abort;
+}
+
+// sum over the four worker warps (all 128 workers call it)
+__device__ __forceinline__ float worker_sum(float v, float* red) {
+  v = warp_sum(v);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  wsync();
+  v = (red[0] + red[1]) + (red[2] + red[3]);
+  wsync();
+  return v;
+}
+
+__device__ __forceinline__ void store_bf16x4(bf16* o, float a, float b, float c, float d) {
+  __nv_bfloat162 lo = __floats2bfloat162_rn(a, b), hi = __floats2bfloat162_rn(c, d);
+  uint2 u;
+  u.x = *reinterpret_cast<uint32_t*>(&lo);
+  u.y = *reinterpret_cast<uint32_t*>(&hi);
+  *reinterpret_cast<uint2*>(o) = u;
+}
+
+__device__ __forceinline__ float4 f4add(float4 a, float4 b) {
+  return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
+}
+
+// LayerNorm gains / biases of the features this thread holds (float4 q =
+// tid + 128u covers features 4q..4q+3), loaded with the row's other inputs
+struct LnParams {
+  float4 g1[4], b1[4], g2[4], b2[4];
+};
+__device__ __forceinline__ void ln_load(LnParams& p, int D, const float* g1, const float* b1,
+                                        const float* g2, const float* b2) {
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int f = (threadIdx.x + u * WORKERS) * 4;
+    if (f < D) {
+      p.g1[u] = *reinterpret_cast<const float4*>(g1 + f);
+      p.b1[u] = *reinterpret_cast<const float4*>(b1 + f);
+      if (g2) {
+        p.g2[u] = *reinterpret_cast<const float4*>(g2 + f);
+        p.b2[u] = *reinterpret_cast<const float4*>(b2 + f);
+      }
+    }
+  }
+}
+
+// LayerNorm of the row held in v[] (same layout), written as bf16 with
+// (g1, b1) to out1 and, if out2, (g2, b2) to out2. Two-pass statistics in fp32.
+__device__ void ln_out(const float4* v, int D, float eps, const LnParams& p, bf16* out1, bf16* out2,
+                       float* red) {
+  float s = 0.f;
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int f = (threadIdx.x + u * WORKERS) * 4;
+    if (f < D) s += (v[u].x + v[u].y) + (v[u].z + v[u].w);
+  }
+  const float mu = worker_sum(s, red) / (float)D;
+  float q = 0.f;
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int f = (threadIdx.x + u * WORKERS) * 4;
+    if (f < D) {
+      const float a = v[u].x - mu, b = v[u].y - mu, c = v[u].z - mu, d = v[u].w - mu;
+      q += (a * a + b * b) + (c * c + d * d);
+    }
+  }
+  const float rstd = rsqrtf(worker_sum(q, red) / (float)D + eps);
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int f = (threadIdx.x + u * WORKERS) * 4;
+    if (f < D) {
+      const float n0 = (v[u].x - mu) * rstd, n1 = (v[u].y - mu) * rstd;
+      const float n2 = (v[u].z - mu) * rstd, n3 = (v[u].w - mu) * rstd;
+      const float4 ga = p.g1[u], ba = p.b1[u];
+      store_bf16x4(out1 + f, n0 * ga.x + ba.x, n1 * ga.y + ba.y, n2 * ga.z + ba.z, n3 * ga.w + ba.w);
+      if (out2) {
+        const float4 gb = p.g2[u], bb = p.b2[u];
+        store_bf16x4(out2 + f, n0 * gb.x + bb.x, n1 * gb.y + bb.y, n2 * gb.z + bb.z, n3 * gb.w + bb.w);
+      }
+    }
+  }
+}
+
+// ---- TMA producer (warp 4, one thread) ----------------------------------------
+// Walks exactly the (phase, unit, K block) sequence the MMA issuer consumes.
+__device__ void producer(const CUtensorMap* mq, const CUtensorMap* mo, const CUtensorMap* ml,
+                         const Plan& P, int Nt, uint8_t* ring, uint64_t* full, uint64_t* empty,
+                         int* status, volatile int* s_abort) {
+  const int G = gridDim.x, c = blockIdx.x;
+  int it = 0;
+  bool stop = false;
+  // weights are read once per step: keep them from evicting the activations
+  // and partial sums that the phases exchange through L2
+  uint64_t policy;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(policy));
+  auto load = [&](const CUtensorMap* m, int x, int y, int z, bool three) {
+    if (stop) return;
+    const int s = it % P.stages;
+    if (it >= P.stages && !wait_or_abort(&empty[s], ((it / P.stages) + 1) & 1, status, s_abort, PRODUCER_SLEEP_NS)) {
+      stop = true;
+      return;
+    }
+    mbar_arrive_expect_tx(&full[s], TILE_BYTES);
+    if (three) tc::tma_load_3d_hint(ring + (size_t)s * TILE_BYTES, m, x, y, z, &full[s], policy);
+    else tc::tma_load_2d_hint(ring + (size_t)s * TILE_BYTES, m, x, y, &full[s], policy);
+    ++it;
+  };
+  for (int l = 0; l < Nt && !stop; ++l) {
+    for (int u = c; u < P.T1 * P.S1 && !stop; u += G) {
+      const int t = u % P.T1, sp = u / P.T1;
+      for (int kb = 0; kb < P.nkb1; ++kb) load(mq, (sp * P.nkb1 + kb) * 64, t * 128, l, true);
+    }
+    for (int u = c; u < P.T2 * P.S2 && !stop; u += G) {
+      const int t = u % P.T2, sp = u / P.T2;
+      for (int kb = 0; kb < P.nkb2; ++kb) load(mo, (sp * P.nkb2 + kb) * 64, t * 128, l, true);
+    }
+  }
+  for (int t = c; t < P.TL && !stop; t += G)
+    for (int kb = 0; kb < P.nkbL; ++kb) load(ml, kb * 64, t * 128, 0, false);
+  // copies still in flight (none on a normal run: the issuer consumed them all)
+  const int first = it > P.stages ? it - P.stages : 0;
+  for (int j = first; j < it; ++j) mbar_wait_bounded(&full[j % P.stages], (j / P.stages) & 1, status);
+}
+
+// ---- worker-side pieces ------------------------------------------------------
+// Activations for one unit: nkb boxes of Bp rows x 64 columns of a bf16
+// matrix (rows >= B read as zero), columns col0 + 64*kb, by TMA into `act`
+// (swizzled K-major blocks of Bp x 128 bytes) with completion on `bar`. One
+// thread. The rows were written by other CTAs of this kernel through the
+// generic proxy before the grid barrier; the proxy fence orders those writes
+// before this thread's asynchronous-proxy reads.
+__device__ void load_act(const CUtensorMap* map, uint8_t* act, int col0, int nkb, int Bp, uint64_t* bar) {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+  mbar_arrive_expect_tx(bar, (uint32_t)(nkb * Bp * 128));
+  for (int kb = 0; kb < nkb; ++kb)
+    tc::tma_load_2d(act + (size_t)kb * Bp * 128, map, col0 + kb * 64, 0, bar);
+}
+
+// One thread: the MMAs of one unit (nkb K blocks from the ring, activations
+// from `act`) into TMEM columns at tmem_d, then a commit to `done`.
+__device__ void issue_unit(const Plan& P, int nkb, uint8_t* ring, const uint8_t* act, uint32_t tmem_d,
+                           uint64_t* full, uint64_t* empty, uint64_t* done, int& it, int* status) {
+  const uint32_t idesc = tc::idesc_bf16_m128(P.Bp);
+  for (int kb = 0; kb < nkb; ++kb, ++it) {
+    const int s = it % P.stages;
+    mbar_wait_bounded(&full[s], (it / P.stages) & 1, status);
+    tc::fence_after();
+    const uint64_t da = tc::desc_sw128(smem_u32(ring + (size_t)s * TILE_BYTES));
+    const uint64_t db = tc::desc_sw128(smem_u32(act + (size_t)kb * P.Bp * 128));
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk)  // 16-wide K slices: +32 bytes = +2 in descriptor units
+      tc::mma_bf16(tmem_d, da + 2 * kk, db + 2 * kk, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+    tc::commit(&empty[s]);
+  }
+  tc::commit(done);
+}
+
+// fp32 partial tile (128 features x B rows) from TMEM to part[u][row][128]
+__device__ void store_partial(uint32_t tbuf, float* part, int u, int B, int Bp) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t trow = tbuf + ((uint32_t)(warp * 32) << 16);
+  float* dst = part + (size_t)u * B * 128 + warp * 32 + lane;
+  for (int c0 = 0; c0 < Bp; c0 += 16) {
+    float v[16];
+    tc::tmem_ld16(trow + c0, v);
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      if (c0 + j < B) __stcg(dst + (size_t)(c0 + j) * 128, v[j]);
+  }
+}
+
+// Shared-memory barriers of the worker / MMA hand-off.
+struct Sync {
+  uint64_t* full;       // [stages] weight tile landed
+  uint64_t* empty;      // [stages] weight tile consumed
+  uint64_t* act_full;   // activations landed (TMA transaction count)
+  uint64_t* acc_full;   // [2] accumulator ready (tcgen05.commit)
+  uint64_t* acc_empty;  // [2] accumulator drained (128 worker arrivals)
+};
+
+// Split-K GEMM phase, worker side: units u = blockIdx.x + i*gridDim.x of T
+// tiles x S splits, each nkb K blocks; activations through `map`, columns
+// col_of(tile) + split*nkb*64. `na` counts activation loads, `nu` accumulator
+// uses (both in the MMA warp's order).
+template <typename ColOf>
+__device__ void gemm_phase(const Plan& P, int T, int S, int nkb, const CUtensorMap* map, ColOf col_of,
+                           int B, float* part, uint8_t* act, uint32_t tmem, const Sync& y, int& na,
+                           int& nu, int* status) {
+  for (int u = blockIdx.x; u < T * S; u += gridDim.x) {
+    const int t = u % T, sp = u / T;
+    // act is free: the previous unit's MMAs (its last readers) completed
+    // before that unit's accumulator was drained below
+    if (threadIdx.x == 0) load_act(map, act, col_of(t) + sp * nkb * 64, nkb, P.Bp, y.act_full);
+    ++na;
+    const int buf = nu & 1;
+    mbar_wait_bounded(&y.acc_full[buf], (nu >> 1) & 1, status);
+    tc::fence_after();
+    store_partial(tmem + (uint32_t)(buf * 64), part, u, B, P.Bp);
+    tc::fence_before();
+    mbar_arrive(&y.acc_empty[buf]);
+    ++nu;
+  }
+}
+
+// MMA warp (one thread): the same unit sequence as the workers and the
+// producer. Waits for staged activations and a drained accumulator.
+__device__ void mma_issuer(const Plan& P, int Nt, uint8_t* ring, const uint8_t* act, uint32_t tmem,
+                           const Sync& y, int* status, volatile int* s_abort) {
+  const int G = gridDim.x, c = blockIdx.x;
+  int it = 0, na = 0, nu = 0;
+  auto unit = [&](int nkb, bool need_act) -> bool {
+    if (need_act) {
+      if (!wait_or_abort(y.act_full, na & 1, status, s_abort, MMA_SLEEP_NS)) return false;
+      ++na;
+    }
+    const int buf = nu & 1;
+    if (nu >= 2 && !wait_or_abort(&y.acc_empty[buf], ((nu >> 1) + 1) & 1, status, s_abort, MMA_SLEEP_NS))
+      return false;
+    tc::fence_after();
+    issue_unit(P, nkb, ring, act, tmem + (uint32_t)(buf * 64), y.full, y.empty, &y.acc_full[buf], it, status);
+    ++nu;
+    return true;
+  };
+  for (int l = 0; l < Nt; ++l) {
+    for (int u = c; u < P.T1 * P.S1; u += G)
+      if (!unit(P.nkb1, true)) return;
+    for (int u = c; u < P.T2 * P.S2; u += G)
+      if (!unit(P.nkb2, true)) return;
+  }
+  bool first = true;
+  for (int t = c; t < P.TL; t += G) {
+    if (!unit(P.nkbL, first)) return;  // every vocab tile reads the same staged input
+    first = false;
+  }
+}
+
+// R1, one half-warp (16 lanes) per (sequence, head): q|k|v from the K
+// splits + bias, rotary on q and k, k and v appended to the local cache at
+// `pos`, attention of the query over cache slots 0..pos. Lane l of the group
+// holds head dims l + 16x.
+template <int DH>
+__device__ void attend_item(const TokenStepArgs& a, const Plan& P, const float* bq, bf16* kc, bf16* vc,
+                            int b, int h, int pos, bool active) {
+  constexpr int EPL = DH / 16;
+  const int l16 = threadIdx.x & 15;
+  const int D = a.D, B = a.B;
+  const size_t split_stride = (size_t)P.T1 * B * 128;
+  float q[EPL], k[EPL], v[EPL];
+  float kw[MAX_WIN][EPL], vw[MAX_WIN][EPL];
+  const size_t base = ((size_t)b * a.H + h) * a.l_cap * DH;
+  // every load of the item in one batch: partial sums, biases, the window
+#pragma unroll
+  for (int x = 0; x < EPL; ++x) {
+    const int nq = h * DH + l16 + 16 * x, nk = D + nq, nv = 2 * D + nq;
+    float sq = 0.f, sk = 0.f, sv = 0.f;
+    if (active) {
+      sq = bq[nq]; sk = bq[nk]; sv = bq[nv];
+      const float* pq = a.p1 + ((size_t)(nq >> 7) * B + b) * 128 + (nq & 127);
+      const float* pk = a.p1 + ((size_t)(nk >> 7) * B + b) * 128 + (nk & 127);
+      const float* pv = a.p1 + ((size_t)(nv >> 7) * B + b) * 128 + (nv & 127);
+#pragma unroll
+      for (int s = 0; s < MAX_S1; ++s) {
+        if (s < P.S1) {
+          sq += __ldcg(pq + s * split_stride);
+          sk += __ldcg(pk + s * split_stride);
+          sv += __ldcg(pv + s * split_stride);
+        }
+      }
+    }
+    q[x] = sq; k[x] = sk; v[x] = sv;
+#pragma unroll
+    for (int j = 0; j < MAX_WIN; ++j) {
+      const int e = l16 + 16 * x;
+      kw[j][x] = (active && j < pos) ? __bfloat162float(kc[base + (size_t)j * DH + e]) : 0.f;
+      vw[j][x] = (active && j < pos) ? __bfloat162float(vc[base + (size_t)j * DH + e]) : 0.f;
+    }
+  }
+  if (a.rot > 0) {
+    // rotate-half pairs (e, e ^ half), e < rot: for half < 16 the pair is in
+    // lane l16 ^ half of the group, for half = 16 in this lane's register x ^ 1
+    const int half = a.rot >> 1;
+    float qp[EPL], kp[EPL];
+#pragma unroll
+    for (int x = 0; x < EPL; ++x) {
+      const float qs = __shfl_xor_sync(0xffffffffu, q[x], half < 16 ? half : 0);
+      const float ks = __shfl_xor_sync(0xffffffffu, k[x], half < 16 ? half : 0);
+      qp[x] = (half < 16) ? qs : q[x ^ 1];
+      kp[x] = (half < 16) ? ks : k[x ^ 1];
+    }
+#pragma unroll
+    for (int x = 0; x < EPL; ++x) {
+      const int e = l16 + 16 * x;
+      if (e < a.rot) {
+        const float2 cs = a.rope_tab[(size_t)pos * half + (e & (half - 1))];
+        if (e & half) {
+          q[x] = q[x] * cs.x + qp[x] * cs.y;
+          k[x] = k[x] * cs.x + kp[x] * cs.y;
+        } else {
+          q[x] = q[x] * cs.x - qp[x] * cs.y;
+          k[x] = k[x] * cs.x - kp[x] * cs.y;
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int x = 0; x < EPL; ++x) {
+    const int e = l16 + 16 * x;
+    const bf16 kb = __float2bfloat16_rn(k[x]), vb = __float2bfloat16_rn(v[x]);
+    if (active) {
+      kc[base + (size_t)pos * DH + e] = kb;
+      vc[base + (size_t)pos * DH + e] = vb;
+    }
+    k[x] = __bfloat162float(kb);  // attention reads what the cache holds
+    v[x] = __bfloat162float(vb);
+  }
+  float mrun = -FLT_MAX, lsum = 0.f, o[EPL];
+#pragma unroll
+  for (int x = 0; x < EPL; ++x) o[x] = 0.f;
+#pragma unroll
+  for (int j = 0; j < MAX_WIN; ++j) {
+    if (j > pos) break;
+    float s = 0.f;
+#pragma unroll
+    for (int x = 0; x < EPL; ++x) s = fmaf(q[x], j < pos ? kw[j][x] : k[x], s);
+#pragma unroll
+    for (int off = 8; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);  // 16-lane group
+    s *= P.scale;
+    const float mn = fmaxf(mrun, s);
+    const float cf = exp2f(mrun - mn), p = exp2f(s - mn);
+    lsum = lsum * cf + p;
+#pragma unroll
+    for (int x = 0; x < EPL; ++x) o[x] = o[x] * cf + p * (j < pos ? vw[j][x] : v[x]);
+    mrun = mn;
+  }
+  if (active) {
+    bf16* out = a.a2 + (size_t)b * 5 * D + h * DH;
+#pragma unroll
+    for (int x = 0; x < EPL; ++x) out[l16 + 16 * x] = __float2bfloat16_rn(o[x] / lsum);
+  }
+}
+
+__device__ void r1_phase(const TokenStepArgs& a, const Plan& P, int l, int pos) {
+  const int D = a.D, B = a.B;
+  const float* bq = layer_ptr(a.b_qkv1, l, a.layer_stride);
+  bf16* kc = a.kt + (size_t)l * a.kt_layer;
+  bf16* vc = a.vt + (size_t)l * a.kt_layer;
+  // (sequence, head) items over the half-warps of the grid; both halves of
+  // a warp run the shuffles together, an idle half with active = false
+  const int hw = threadIdx.x >> 4;
+  const int n_items = B * a.H;
+  for (int i0 = blockIdx.x * 8 + (hw & ~1); i0 < n_items; i0 += 8 * gridDim.x) {
+    const int i = i0 + (hw & 1);
+    const bool active = i < n_items;
+    const int b = active ? i / a.H : 0, h = active ? i - b * a.H : 0;
+    if (a.dh == 32) attend_item<32>(a, P, bq, kc, vc, b, h, pos, active);
+    else if (a.dh == 64) attend_item<64>(a, P, bq, kc, vc, b, h, pos, active);
+    else attend_item<128>(a, P, bq, kc, vc, b, h, pos, active);
+  }
+  // GELU(fc1): features 3D + c, c < 4D, of the first GEMM, four at a time
+  // (a group never crosses a 128-feature tile)
+  const int W4 = D;  // float4 groups per row
+  const int E = B * W4;
+  const int nthr = gridDim.x * WORKERS;
+  constexpr int BATCH = 4;
+  for (int e0 = blockIdx.x * WORKERS + threadIdx.x; e0 < E; e0 += BATCH * nthr) {
+    float4 acc[BATCH];
+#pragma unroll
+    for (int j = 0; j < BATCH; ++j) {
+      const int e = e0 + j * nthr;
+      if (e < E) {
+        const int b = e / W4, n = 3 * D + 4 * (e - b * W4);
+        float4 sum = *reinterpret_cast<const float4*>(bq + n);
+        const float* src = a.p1 + ((size_t)(n >> 7) * B + b) * 128 + (n & 127);
+        const size_t split_stride = (size_t)P.T1 * B * 128;
+#pragma unroll
+        for (int sp = 0; sp < MAX_S1; ++sp)
+          if (sp < P.S1) sum = f4add(sum, __ldcg(reinterpret_cast<const float4*>(src + sp * split_stride)));
+        acc[j] = sum;
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < BATCH; ++j) {
+      const int e = e0 + j * nthr;
+      if (e < E) {
+        const int b = e / W4, c = 4 * (e - b * W4);
+        store_bf16x4(a.a2 + (size_t)b * 5 * D + D + c, gelu_erf(acc[j].x), gelu_erf(acc[j].y),
+                     gelu_erf(acc[j].z), gelu_erf(acc[j].w));
+      }
+    }
+  }
+}
+
+// R2: h += sum of the K splits + (b_o + b_2); LayerNorm of the new row for
+// layer l + 1 (LN1 | LN2 -> x1) or the final LayerNorm (-> xf).
+__device__ void r2_phase(const TokenStepArgs& a, const Plan& P, int l, float* red) {
+  const int D = a.D, B = a.B;
+  const float* bo = layer_ptr(a.b_o2, l, a.layer_stride);
+  // the next LayerNorm's parameters: layer l + 1's LN1 | LN2, or the final one
+  LnParams lp;
+  if (blockIdx.x < B) {
+    if (l + 1 < a.Nt)
+      ln_load(lp, D, layer_ptr(a.ln1_g, l + 1, a.layer_stride), layer_ptr(a.ln1_b, l + 1, a.layer_stride),
+              layer_ptr(a.ln2_g, l + 1, a.layer_stride), layer_ptr(a.ln2_b, l + 1, a.layer_stride));
+    else
+      ln_load(lp, D, a.lnf_g, a.lnf_b, nullptr, nullptr);
+  }
+  for (int b = blockIdx.x; b < B; b += gridDim.x) {
+    float4 hv[4];
+    float* hrow = a.h + (size_t)b * D;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int f = (threadIdx.x + u * WORKERS) * 4;
+      hv[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (f < D) {
+        float4 acc = f4add(__ldcg(reinterpret_cast<const float4*>(hrow + f)),
+                           *reinterpret_cast<const float4*>(bo + f));
+        const int t = f >> 7, off = f & 127;
+#pragma unroll
+        for (int s = 0; s < MAX_S2; ++s)
+          if (s < P.S2)
+            acc = f4add(acc, __ldcg(reinterpret_cast<const float4*>(
+                                 a.p2 + ((size_t)(s * P.T2 + t) * B + b) * 128 + off)));
+        hv[u] = acc;
+        __stcg(reinterpret_cast<float4*>(hrow + f), acc);
+      }
+    }
+    if (l + 1 < a.Nt) {
+      bf16* o = a.x1 + (size_t)b * 2 * D;
+      ln_out(hv, D, a.eps, lp, o, o + D, red);
+    } else {
+      ln_out(hv, D, a.eps, lp, a.xf + (size_t)b * D, nullptr, red);
+    }
+  }
+}
+
+// phase I: the row of each sequence (the fed token's embedding on token
+// steps; the prefix row already in h on block steps) -> LN1 | LN2 of layer 0
+__device__ void ingest_phase(const TokenStepArgs& a, int jb, float* red) {
+  const int D = a.D;
+  LnParams lp;
+  if (blockIdx.x < a.B) ln_load(lp, D, a.ln1_g, a.ln1_b, a.ln2_g, a.ln2_b);
+  for (int b = blockIdx.x; b < a.B; b += gridDim.x) {
+    float4 hv[4];
+    float* hrow = a.h + (size_t)b * D;
+    int tok = 0;
+    if (a.ingest) {
+      tok = a.src[b];
+      if (tok < 0 || tok >= a.V) {
+        if (threadIdx.x == 0) set_status(a.status, ST_BAD_TOKEN);
+        tok = 0;
+      }
+      if (threadIdx.x == 0) a.block_tok[b * a.L_B + jb] = tok;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int f = (threadIdx.x + u * WORKERS) * 4;
+      hv[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (f < D) {
+        if (a.ingest) {
+          const uint2 w = *reinterpret_cast<const uint2*>(a.tok_emb + (size_t)tok * D + f);
+          const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w.x));
+          const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w.y));
+          hv[u] = make_float4(lo.x, lo.y, hi.x, hi.y);
+          __stcg(reinterpret_cast<float4*>(hrow + f), hv[u]);
+        } else {
+          hv[u] = __ldcg(reinterpret_cast<const float4*>(hrow + f));
+        }
+      }
+    }
+    bf16* o = a.x1 + (size_t)b * 2 * D;
+    ln_out(hv, D, a.eps, lp, o, o + D, red);
+  }
+}
+
+__device__ __forceinline__ void better(float& v, int& i, float ov, int oi) {
+  if (ov > v || (ov == v && oi < i)) { v = ov; i = oi; }
+}
+
+// Per-row argmax over the warp's 32 features for 32 rows held one per
+// register (v[r], index idx for all): a transposing butterfly -- at each of
+// the 5 levels a lane keeps half of its rows and trades the other half with
+// its partner -- leaves row `lane` reduced over the 32 lanes in 31 exchanges.
+__device__ __forceinline__ void warp_argmax32(float* v, int* ix) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int o = 16, h = 16; o > 0; o >>= 1, h >>= 1) {
+    const bool up = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < h; ++i) {
+      const float sv = up ? v[i] : v[i + h];
+      const int si = up ? ix[i] : ix[i + h];
+      const float rv = __shfl_xor_sync(0xffffffffu, sv, o);
+      const int ri = __shfl_xor_sync(0xffffffffu, si, o);
+      float kv = up ? v[i + h] : v[i];
+      int ki = up ? ix[i + h] : ix[i];
+      better(kv, ki, rv, ri);
+      v[i] = kv;
+      ix[i] = ki;
+    }
+  }
+}
+
+// GL epilogue of vocab tile t: logits (optional) and the tile's argmax per row
+__device__ void lm_epilogue(uint32_t tbuf, int t, const TokenStepArgs& a, int Bp, float2 (*s_arg)[MAX_B]) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t trow = tbuf + ((uint32_t)(warp * 32) << 16);
+  const int n = t * 128 + warp * 32 + lane;
+  for (int c0 = 0; c0 < Bp; c0 += 32) {
+    float v[32];
+    int ix[32];
+    tc::tmem_ld16(trow + c0, v);
+    if (c0 + 16 < Bp) tc::tmem_ld16(trow + c0 + 16, v + 16);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const int m = c0 + j;
+      if (a.logits && m < a.B && n < a.V) a.logits[(size_t)m * a.V + n] = v[j];
+      if (n >= a.V || m >= a.B) v[j] = -INFINITY;
+      ix[j] = n;
+    }
+    warp_argmax32(v, ix);
+    if (c0 + lane < a.B) s_arg[warp][c0 + lane] = make_float2(v[0], __int_as_float(ix[0]));
+  }
+  tc::fence_before();
+  wsync();
+  if (threadIdx.x < a.B) {
+    const int r = threadIdx.x;
+    float2 best = s_arg[0][r];
+#pragma unroll
+    for (int w = 1; w < 4; ++w) {
+      const float2 o = s_arg[w][r];
+      if (o.x > best.x || (o.x == best.x && __float_as_int(o.y) < __float_as_int(best.y))) best = o;
+    }
+    __stcg(a.arg_part + (size_t)t * a.B + r, best);
+  }
+  wsync();  // s_arg is reused by the next tile
+}
+
+__device__ void lm_phase(const TokenStepArgs& a, const Plan& P, const CUtensorMap* mxf, uint8_t* act,
+                         uint32_t tmem, const Sync& y, int& na, int& nu, float2 (*s_arg)[MAX_B]) {
+  const int G = gridDim.x;
+  if ((int)blockIdx.x >= P.TL) return;
+  if (threadIdx.x == 0) load_act(mxf, act, 0, P.nkbL, P.Bp, y.act_full);
+  ++na;
+  for (int t = blockIdx.x; t < P.TL; t += G) {
+    const int buf = nu & 1;
+    mbar_wait_bounded(&y.acc_full[buf], (nu >> 1) & 1, a.status);
+    tc::fence_after();
+    lm_epilogue(tmem + (uint32_t)(buf * 64), t, a, P.Bp, s_arg);
+    mbar_arrive(&y.acc_empty[buf]);  // lm_epilogue ended with the tcgen05 fence + barrier
+    ++nu;
+  }
+}
+
+// AR: greedy id per row from the tile partials (lowest id on ties)
+__device__ void argmax_phase(const TokenStepArgs& a, const Plan& P) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int b = blockIdx.x * 4 + warp; b < a.B; b += 4 * gridDim.x) {
+    float bv = -INFINITY;
+    int bi = INT_MAX;
+    for (int t = lane; t < P.TL; t += 32) {
+      const float2 o = __ldcg(a.arg_part + (size_t)t * a.B + b);
+      const int oi = __float_as_int(o.y);
+      if (o.x > bv || (o.x == bv && oi < bi)) { bv = o.x; bi = oi; }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+    }
+    if (lane == 0) a.next[b] = bi;
+  }
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+token_step_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mo,
+                  const __grid_constant__ CUtensorMap ml, const __grid_constant__ CUtensorMap mx1,
+                  const __grid_constant__ CUtensorMap ma2, const __grid_constant__ CUtensorMap mxf,
+                  const TokenStepArgs a, const Plan P) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~(uintptr_t)1023);
+  uint8_t* ring = smem;
+  uint8_t* act = smem + (size_t)P.stages * TILE_BYTES;
+  __shared__ __align__(8) uint64_t full[MAX_STAGES], empty[MAX_STAGES], act_full, acc_full[2], acc_empty[2];
+  __shared__ uint32_t tmem_slot;
+  __shared__ float red[4];
+  __shared__ float2 s_arg[4][MAX_B];
+  __shared__ volatile int s_abort;
+
+  const int warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < P.stages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    mbar_init(&act_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], WORKERS);
+    }
+    s_abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) tc::tmem_alloc(&tmem_slot, TMEM_COLS);
+  tc::fence_before();
+  __syncthreads();
+  tc::fence_after();
+  const uint32_t tmem = tmem_slot;
+  const Sync y{full, empty, &act_full, acc_full, acc_empty};
+  pdl_trigger();
+
+  if (warp == 4) {
+    // weights do not depend on earlier kernels: no wait before streaming them
+    if ((threadIdx.x & 31) == 0) producer(&mq, &mo, &ml, P, a.Nt, ring, full, empty, a.status, &s_abort);
+  } else if (warp == 5) {
+    if ((threadIdx.x & 31) == 0) mma_issuer(P, a.Nt, ring, act, tmem, y, a.status, &s_abort);
+  } else {
+    pdl_wait();
+    const int G = gridDim.x;
+    const int pos = pos_base(a.pos);  // read before the first barrier: the last phase advances it
+    const int jb = a.dstate[1];
+    unsigned nb = 0;
+    int na = 0, nu = 0;
+    bool ok;
+    ingest_phase(a, jb, red);
+    ok = grid_sync(a.bar, ++nb * G, a.status, &s_abort);
+    const int D = a.D;
+    for (int l = 0; ok && l < a.Nt; ++l) {
+      // G1: q|k|v tiles read LN1(h), fc1 tiles LN2(h)
+      gemm_phase(P, P.T1, P.S1, P.nkb1, &mx1, [=](int t) { return t * 128 < 3 * D ? 0 : D; }, a.B, a.p1,
+                 act, tmem, y, na, nu, a.status);
+      if (!(ok = grid_sync(a.bar, ++nb * G, a.status, &s_abort))) break;
+      r1_phase(a, P, l, pos);
+      if (!(ok = grid_sync(a.bar, ++nb * G, a.status, &s_abort))) break;
+      gemm_phase(P, P.T2, P.S2, P.nkb2, &ma2, [](int) { return 0; }, a.B, a.p2, act, tmem, y, na, nu,
+                 a.status);
+      if (!(ok = grid_sync(a.bar, ++nb * G, a.status, &s_abort))) break;
+      r2_phase(a, P, l, red);
+      ok = grid_sync(a.bar, ++nb * G, a.status, &s_abort);
+    }
+    if (ok) {
+      lm_phase(a, P, &mxf, act, tmem, y, na, nu, s_arg);
+      ok = grid_sync(a.bar, ++nb * G, a.status, &s_abort);
+    }
+    if (ok) {
+      argmax_phase(a, P);
+      if (blockIdx.x == 0 && threadIdx.x == 0) {
+        const int t = a.dstate[0] + 1;
+        a.dstate[0] = t;
+        a.dstate[1] = t % a.L_B;
+        a.dstate[2] = t / a.L_B;
+      }
+    }
+    // workers that stop early (abort) release the MMA warp's waits
+    if (!ok && threadIdx.x == 0) s_abort = 1;
+  }
+
+  tc::fence_before();
+  __syncthreads();
+  if (warp == 0) tc::tmem_free(tmem, TMEM_COLS);
+  if (threadIdx.x == 0) {
+    // the last CTA out resets the barrier counter for the next launch: every
+    // CTA counts itself here only after its last barrier wait
+    __threadfence();
+    if (atomicAdd(&a.bar[1], 1u) == gridDim.x - 1) {
+      a.bar[0] = 0u;
+      a.bar[1] = 0u;
+      __threadfence();
+    }
+  }
+}
+
+// ---- host side -----------------------------------------------------------------
+typedef CUresult (*EncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                             const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                             CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                             CUtensorMapFloatOOBfill);
+
+EncodeFn encode_fn() {
+  static EncodeFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeFn>(p);
+  }
+  return fn;
+}
+
+// bf16 weight boxes of 64 K x 128 rows, 128-byte swizzle, zero fill past the
+// last row; rank 3 adds the layer dimension (stride in bytes)
+bool weight_map(CUtensorMap* m, const void* base, long long K, long long rows, long long layers,
+                long long layer_stride) {
+  EncodeFn f = encode_fn();
+  if (!f) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)K, (cuuint64_t)rows, (cuuint64_t)layers};
+  cuuint64_t str[2] = {(cuuint64_t)K * 2, (cuuint64_t)layer_stride};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  const cuuint32_t rank = layers > 0 ? 3 : 2;
+  return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, str, box, es,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// bf16 activation rows [rows, cols] (row-major, ld = cols): boxes of 64
+// columns x box_rows rows, 128-byte swizzle, zero fill for rows >= rows
+bool act_map(CUtensorMap* m, const void* base, long long rows, long long cols, int box_rows) {
+  EncodeFn f = encode_fn();
+  if (!f) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t str[1] = {(cuuint64_t)cols * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, str, box, es,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct Device {
+  int sms = 0;
+  size_t smem_max = 0;  // dynamic shared memory per CTA
+  bool ready = false;
+};
+
+Device& device() {
+  static Device d;
+  if (!d.ready) {
+    int dev = 0, optin = 0;
+    cudaFuncAttributes fa;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
+        cudaFuncGetAttributes(&fa, token_step_kernel) != cudaSuccess)
+      return d;
+    d.smem_max = (size_t)optin - fa.sharedSizeBytes;
+    if (cudaFuncSetAttribute(token_step_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)d.smem_max) != cudaSuccess)
+      return d;
+    d.ready = true;
+  }
+  return d;
+}
+
+// largest divisor of n that is <= cap
+int divisor_at_most(int n, int cap) {
+  for (int s = cap < n ? cap : n; s > 1; --s)
+    if (n % s == 0) return s;
+  return 1;
+}
+
+bool make_plan(int B, int D, int dh, int V, int sms, size_t smem_max, Plan* P, size_t* smem) {
+  Plan p{};
+  p.Bp = (B + 15) / 16 * 16;
+  p.T1 = 7 * D / 128;
+  p.T2 = D / 128;
+  p.TL = (V + 127) / 128;
+  const int kb1 = D / 64, kb2 = 5 * D / 64;
+  int c1 = sms / p.T1;
+  if (c1 > MAX_S1) c1 = MAX_S1;
+  int c2 = sms / p.T2;
+  if (c2 > MAX_S2) c2 = MAX_S2;
+  p.S1 = divisor_at_most(kb1, c1 < 1 ? 1 : c1);
+  p.S2 = divisor_at_most(kb2, c2 < 1 ? 1 : c2);
+  p.nkb1 = kb1 / p.S1;
+  p.nkb2 = kb2 / p.S2;
+  p.nkbL = kb1;
+  // the activation buffer holds the LM head's whole input (the largest unit)
+  int act_kb = p.nkbL;
+  if (p.nkb1 > act_kb) act_kb = p.nkb1;
+  if (p.nkb2 > act_kb) act_kb = p.nkb2;
+  const size_t act = (size_t)act_kb * p.Bp * 128;
+  if (smem_max < act + 1024 + 4 * (size_t)TILE_BYTES) return false;
+  int st = (int)((smem_max - act - 1024) / TILE_BYTES);
+  p.stages = st > MAX_STAGES ? MAX_STAGES : st;
+  p.scale = 1.4426950408889634f / sqrtf((float)dh);
+  *P = p;
+  *smem = (size_t)p.stages * TILE_BYTES + act + 1024;
+  return true;
+}
+
+}  // namespace
+
+int token_step_supported(int dt, int B, int D, int H, int rot, int V, int Nt, int P_prefix, int l_cap) {
+  if (dt != DT_BF16 || B < 1 || B > MAX_B || Nt < 1 || P_prefix != 1 || V < 1 || l_cap > MAX_WIN) return 0;
+  if (D % 128 || D > 2048 || H < 1 || D % H) return 0;
+  const int dh = D / H;
+  if (dh != 32 && dh != 64 && dh != 128) return 0;
+  if (rot) {
+    const int half = rot / 2;
+    if ((rot & 1) || rot > dh || half > 16 || (half & (half - 1))) return 0;
+  }
+  if (!encode_fn()) return 0;
+  Device& d = device();
+  if (!d.ready) return 0;
+  Plan p;
+  size_t smem;
+  return make_plan(B, D, dh, V, d.sms, d.smem_max, &p, &smem) ? 1 : 0;
+}
+
+size_t token_step_scratch_floats(int B, int D, int which) {
+  // upper bounds over every plan: T1 * MAX_S1 and T2 * MAX_S2 partial tiles
+  if (B > MAX_B) B = MAX_B;
+  return which == 1 ? (size_t)(7 * D / 128) * MAX_S1 * B * 128 : (size_t)(D / 128) * MAX_S2 * B * 128;
+}
+
+cudaError_t launch_token_step(const TokenStepArgs& a, const void* w_qkv1, const void* w_o2,
+                              const void* w_lm, cudaStream_t s) {
+  if (!token_step_supported(DT_BF16, a.B, a.D, a.H, a.rot, a.V, a.Nt, 1, a.l_cap)) return cudaErrorNotSupported;
+  Device& d = device();
+  Plan P;
+  size_t smem;
+  if (!make_plan(a.B, a.D, a.dh, a.V, d.sms, d.smem_max, &P, &smem)) return cudaErrorNotSupported;
+  CUtensorMap mq, mo, ml;
+  // one layer: any stride at least the layer's own size satisfies the encoder
+  const long long lsq = a.Nt > 1 ? a.layer_stride : 14LL * a.D * a.D;
+  const long long lso = a.Nt > 1 ? a.layer_stride : 10LL * a.D * a.D;
+  if (!weight_map(&mq, w_qkv1, a.D, 7LL * a.D, a.Nt, lsq) || !weight_map(&mo, w_o2, 5LL * a.D, a.D, a.Nt, lso) ||
+      !weight_map(&ml, w_lm, a.D, a.V, 0, 0))
+    return cudaErrorInvalidValue;
+  CUtensorMap mx1, ma2, mxf;
+  if (!act_map(&mx1, a.x1, a.B, 2LL * a.D, P.Bp) || !act_map(&ma2, a.a2, a.B, 5LL * a.D, P.Bp) ||
+      !act_map(&mxf, a.xf, a.B, a.D, P.Bp))
+    return cudaErrorInvalidValue;
+  // every CTA must be resident at once (grid barriers): one per SM
+  int per_sm = 0;
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, token_step_kernel, THREADS, smem);
+  if (e != cudaSuccess) return e;
+  if (per_sm < 1) return cudaErrorNotSupported;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(d.sms, 1, 1);
+  cfg.blockDim = dim3(THREADS, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  e = cudaLaunchKernelEx(&cfg, token_step_kernel, mq, mo, ml, mx1, ma2, mxf, a, P);
+  note_launch();
+  return e;
+}
+
+}  // namespace bt

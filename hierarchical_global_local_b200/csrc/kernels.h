@@ -169,6 +169,44 @@ cudaError_t gemm_tc_prepare();
 void gemm_set_path(int path);
 int gemm_tc_supported(int dt, int M, int N, int K, int xk_split, int xk_off);
 
+// ---- fused token-decoder step -------------------------------------------------
+// One persistent kernel for the token-decoder half of a decode step (bf16,
+// B <= 64, prefix length 1): the row of each sequence through every
+// token-decoder layer (local attention over the window in the local cache,
+// the new k, v appended at `pos`), the final LayerNorm, the LM head (logits
+// -> `logits` when not null), the greedy argmax -> `next`, and the step state
+// advanced by one position. Layer l's parameters sit at layer 0's pointers
+// plus l * layer_stride bytes (weights, biases and gains alike).
+struct TokenStepArgs {
+  int B, D, H, dh, rot, V, Nt, L_B, l_cap;
+  float eps;
+  int ingest;        // 1: h = token embedding of src[b] first (block_tok updated)
+  PosSpec pos;       // position of the row in the local window
+  const int32_t* src;
+  int32_t* block_tok;
+  const bf16* tok_emb;
+  int* dstate;
+  const float *b_qkv1, *b_o2, *ln1_g, *ln1_b, *ln2_g, *ln2_b;
+  long long layer_stride;
+  bf16 *kt, *vt;     // local caches [layer][B][H][l_cap][dh]
+  long long kt_layer;
+  const float2* rope_tab;
+  const float *lnf_g, *lnf_b;
+  float* h;          // [B, D] fp32 residual rows
+  bf16 *x1, *a2, *xf;
+  float* logits;
+  int32_t* next;
+  float2* arg_part;  // [ceil(V/128), B]
+  float *p1, *p2;    // split-K partials (token_step_scratch_floats)
+  unsigned* bar;     // 3 words, zero before the first launch
+  int* status;
+};
+int token_step_supported(int dt, int B, int D, int H, int rot, int V, int Nt, int P_prefix, int l_cap);
+// which = 1: first-GEMM partials, 2: second-GEMM partials (floats, for B rows)
+size_t token_step_scratch_floats(int B, int D, int which);
+cudaError_t launch_token_step(const TokenStepArgs& a, const void* w_qkv1, const void* w_o2,
+                              const void* w_lm, cudaStream_t s);
+
 // ---- LM head argmax ---------------------------------------------------------
 // next[b] = argmax_v logits[b, v] (lowest id among ties).
 cudaError_t launch_argmax(const float* logits, int B, int V, int ld, int32_t* next,

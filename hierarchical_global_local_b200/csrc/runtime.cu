@@ -130,6 +130,8 @@ struct bt_model {
   int vt_ld = 0;
   float2* arg_part = nullptr;  // LM-head per-tile argmax partials
   int* ln_cnt = nullptr;       // per-row counters of the LayerNorm fused into GEMM epilogues
+  float *ts_p1 = nullptr, *ts_p2 = nullptr;  // fused token step: split-K partials
+  unsigned* ts_bar = nullptr;                // fused token step: grid-barrier words
   GemmScratch gs{};
   int B = 0, t = 0;
   bool prefilled = false;
@@ -236,6 +238,11 @@ static size_t carve(bt_model* m, const Dims& d, void* ws) {
   m->attn_scratch = c.take(attn_decode_scratch_bytes(d.Bmax, d.H, d.d, d.n_cap, d.dt));
   m->arg_part = (float2*)c.take((size_t)((d.V + 127) / 128) * d.Bmax * sizeof(float2));
   m->ln_cnt = (int*)c.take((size_t)d.Bmax * (d.P > 1 ? d.P : 1) * sizeof(int));
+  if (d.tokdec && d.Bmax > 0) {
+    m->ts_p1 = (float*)c.take(token_step_scratch_floats(d.Bmax, d.D, 1) * 4);
+    m->ts_p2 = (float*)c.take(token_step_scratch_floats(d.Bmax, d.D, 2) * 4);
+    m->ts_bar = (unsigned*)c.take(64);
+  }
   m->vt_ld = (d.n_cap + 63) / 64 * 64;
   m->vtr = c.take((size_t)d.Bmax * D * m->vt_ld * eb);
   const int maxN = 7 * d.D > d.V ? 7 * d.D : d.V;
@@ -348,6 +355,7 @@ int bt_create(const bt_config* cfg, const bt_weights* w, void* ws, size_t ws_byt
   BT_TRYC(cudaMemsetAsync(m->gs.counters, 0, (size_t)m->gs.n_counters * 4, st));
   BT_TRYC(cudaMemsetAsync(m->block_tok, 0, (size_t)d.Bmax * d.L * 4, st));
   BT_TRYC(cudaMemsetAsync(m->ln_cnt, 0, (size_t)d.Bmax * (d.P > 1 ? d.P : 1) * sizeof(int), st));
+  if (m->ts_bar) BT_TRYC(cudaMemsetAsync(m->ts_bar, 0, 64, st));
   BT_TRYC(cudaStreamCreateWithFlags(&m->cap_stream, cudaStreamNonBlocking));
   if (d.dt == BT_BF16) BT_TRYC(gemm_tc_prepare());
   BT_TRYC(attn_prepare());
@@ -614,11 +622,92 @@ static int enqueue_decode_fused(bt_model* m, bool block_step, bool greedy, bool 
   return BT_OK;
 }
 
+// The token-decoder half of a decode call (every token-decoder layer, the
+// final LayerNorm, the LM head, the argmax and the position advance) runs as
+// one persistent kernel where the shape allows; BT_DECODE_TOKEN_STEP=chain
+// keeps the kernel-per-operation schedule instead (read when a step kind is
+// first recorded).
+static bool token_step_fused(const bt_model* m, int B) {
+  const Dims& d = m->d;
+  const char* env = getenv("BT_DECODE_TOKEN_STEP");
+  if (env && strcmp(env, "chain") == 0) return false;
+  if (!d.tokdec || d.Nt < 1 || !m->ts_bar) return false;
+  if (!token_step_supported(d.dt, B, d.D, d.H, d.rot, d.V, d.Nt, d.P, d.l_cap)) return false;
+  // layer l's parameters at a fixed stride from layer 0's
+  const long long ls = d.Nt > 1 ? (long long)((uint8_t*)m->tok[1].w_qkv1 - (uint8_t*)m->tok[0].w_qkv1) : 0;
+  for (int l = 0; l < d.Nt; ++l) {
+    const LayerW& w = m->tok[l];
+    const LayerW& w0 = m->tok[0];
+    auto at = [&](const void* p, const void* p0) {
+      return (const uint8_t*)p == (const uint8_t*)p0 + (long long)l * ls;
+    };
+    if (!at(w.w_qkv1, w0.w_qkv1) || !at(w.w_o2, w0.w_o2) || !at(w.b_qkv1, w0.b_qkv1) ||
+        !at(w.b_o2, w0.b_o2) || !at(w.ln1_g, w0.ln1_g) || !at(w.ln1_b, w0.ln1_b) ||
+        !at(w.ln2_g, w0.ln2_g) || !at(w.ln2_b, w0.ln2_b))
+      return false;
+  }
+  return true;
+}
+
+static int run_token_step(bt_model* m, int B, bool ingest, PosSpec pos, const int32_t* src,
+                          bool want_logits, cudaStream_t s) {
+  const Dims& d = m->d;
+  const LayerW& w0 = m->tok[0];
+  TokenStepArgs a{};
+  a.B = B; a.D = d.D; a.H = d.H; a.dh = d.d; a.rot = d.rot; a.V = d.V; a.Nt = d.Nt; a.L_B = d.L;
+  a.l_cap = d.l_cap; a.eps = m->cfg.ln_eps; a.ingest = ingest ? 1 : 0; a.pos = pos;
+  a.src = src; a.block_tok = m->block_tok; a.tok_emb = (const bf16*)m->tok_emb; a.dstate = m->dstate;
+  a.b_qkv1 = w0.b_qkv1; a.b_o2 = w0.b_o2; a.ln1_g = w0.ln1_g; a.ln1_b = w0.ln1_b;
+  a.ln2_g = w0.ln2_g; a.ln2_b = w0.ln2_b;
+  a.layer_stride = d.Nt > 1 ? (long long)((uint8_t*)m->tok[1].w_qkv1 - (uint8_t*)w0.w_qkv1) : 0;
+  a.kt = (bf16*)m->kt; a.vt = (bf16*)m->vt; a.kt_layer = (long long)m->kt_layer;
+  a.rope_tab = m->rope_tab; a.lnf_g = m->lnf_t_g; a.lnf_b = m->lnf_t_b;
+  a.h = m->h_t; a.x1 = (bf16*)m->x1; a.a2 = (bf16*)m->a2; a.xf = (bf16*)m->xf;
+  a.logits = want_logits ? m->logits : nullptr; a.next = m->next; a.arg_part = m->arg_part;
+  a.p1 = m->ts_p1; a.p2 = m->ts_p2; a.bar = m->ts_bar; a.status = m->status;
+  ProfScope p(m, s, BT_K_TOKEN_STEP, B, d.V, d.D);
+  BT_CUDA(launch_token_step(a, w0.w_qkv1, w0.w_o2, m->w_lm, s));
+  return BT_OK;
+}
+
+// Decode call with the token-decoder half fused into one kernel.
+static int enqueue_decode_token_step(bt_model* m, bool block_step, bool greedy, bool want_logits,
+                                     cudaStream_t s) {
+  const Dims& d = m->d;
+  const int B = m->B;
+  const int32_t* src = greedy ? m->next : m->fed;
+  if (!block_step) return run_token_step(m, B, true, PosSpec{m->dstate, POS_LOCAL, d.P, 1}, src, want_logits, s);
+  {
+    ProfScope p(m, s, BT_K_EMBED, B, d.D, 0);
+    BT_CUDA(launch_ingest(d.dt, src, m->block_tok, m->dstate, B, d.L, d.V, d.D, 1, m->blk_emb,
+                          m->tok_emb, m->h_b, m->status, s));
+  }
+  PosSpec pos{m->dstate, POS_BLOCK, 0, 1};
+  for (int l = 0; l < d.Nb; ++l) {
+    int rc = run_layer(m, m->blk[l], m->h_b, B, pos, layer_ptr(m->kb, m->kb_layer, l, d.eb),
+                       layer_ptr(m->vb, m->kb_layer, l, d.eb), d.n_cap, ATT_DECODE, 0, s);
+    if (rc != BT_OK) return rc;
+  }
+  {
+    ProfScope p(m, s, BT_K_LAYERNORM, B, d.D, 0);
+    BT_CUDA(launch_ln_rows(d.dt, m->h_b, B, 1, 0, d.D, m->lnf_b_g, m->lnf_b_b, m->cfg.ln_eps, m->xf, s));
+  }
+  {
+    // the prefix row h_t[b] = W_p c_b + b_p, then the token decoder over it
+    ProfScope p(m, s, BT_K_GEMM, B, d.D, d.D);
+    Epi ep{EPI_F32, m->h_t, d.D, nullptr, 0, m->b_prefix, 0, d.D};
+    BT_CUDA(launch_gemm(d.dt, m->xf, d.D, m->w_prefix, d.D, B, d.D, d.D, 1 << 30, 0, ep, m->gs,
+                        m->status, s));
+  }
+  return run_token_step(m, B, false, PosSpec{nullptr, POS_ZERO, 0, 1}, src, want_logits, s);
+}
+
 // the body of one decode call (captured into a graph or run directly)
 static int enqueue_decode(bt_model* m, bool block_step, bool greedy, bool want_logits,
                           cudaStream_t s) {
   const Dims& d = m->d;
   const int B = m->B;
+  if (token_step_fused(m, B)) return enqueue_decode_token_step(m, block_step, greedy, want_logits, s);
   if (fused_decode(m, B)) return enqueue_decode_fused(m, block_step, greedy, want_logits, s);
   const int32_t* src = greedy ? m->next : m->fed;
   {
@@ -674,6 +763,8 @@ int bt_prefill(bt_model* m, const int32_t* tokens, int32_t B, int32_t T, float* 
   // a new session: merge counters of the decode attention start from zero
   BT_CUDA(cudaMemsetAsync(m->attn_scratch, 0,
                           attn_decode_scratch_bytes(d.Bmax, d.H, d.d, d.n_cap, d.dt), s));
+  // and the fused token step's barrier words (an aborted step leaves them set)
+  if (m->ts_bar) BT_CUDA(cudaMemsetAsync(m->ts_bar, 0, 64, s));
   const long long k0 = launch_count();
   BT_CUDA(launch_set_state(m->dstate, T, d.L, s));
   {

@@ -153,3 +153,42 @@ def test_fused_argmax_matches_returned_logits_bf16():
     gl, gn = gh.gpu_teacher_forced(m, toks, T, G)
     m.close()
     assert np.array_equal(gn, gl.argmax(-1))
+
+
+def _launches(model):
+    from hierarchical_global_local_b200 import native
+    return int(native.lib().bt_kernel_launches(model._h))
+
+
+@pytest.mark.parametrize("lb,B", [(4, 3), (8, 17), (2, 64)])
+def test_fused_token_step_matches_oracle_and_chain(lb, B, monkeypatch):
+    """The token-decoder half of a decode step as one persistent kernel: a
+    token step is a single launch, its logits match the oracle, and they
+    agree with the kernel-per-operation schedule on the same inputs."""
+    shape = synth.ModelShape(vocab=3000, d_model=256, n_heads=4, block_len=lb,
+                             n_block_layers=2, n_token_layers=3, prefix_len=1)
+    T, G = 6 * lb, 3 * lb + 2
+    w = synth.make_weights(shape, seed=31)
+    toks = synth.make_tokens(batch=B, length=T + G, vocab=shape.vocab, seed=32)
+    torch = gh.torch_mod()
+    m = gh.build_model(shape, w, B, T + G)
+    tok = torch.from_numpy(np.ascontiguousarray(toks)).cuda()
+    m.prefill(tok[:, :T].contiguous())
+    k0 = _launches(m)
+    m.decode(tok[:, T].contiguous())  # position T: not the last of a block
+    m.sync()
+    assert _launches(m) - k0 == 1
+    m.close()
+    m = gh.build_model(shape, w, B, T + G)
+    gl, gn = gh.gpu_teacher_forced(m, toks, T, G)
+    m.close()
+    monkeypatch.setenv("BT_DECODE_TOKEN_STEP", "chain")
+    m = gh.build_model(shape, w, B, T + G)
+    cl, cn = gh.gpu_teacher_forced(m, toks, T, G)
+    m.close()
+    ol = gh.oracle_teacher_forced(shape, w, toks, T, G)
+    for s in range(G):
+        assert gh.rel_l2(gl[s], ol[s]) <= BF16_REL, (s, gh.rel_l2(gl[s], ol[s]))
+        assert gh.rel_l2(gl[s], cl[s]) <= 1e-2, (s, gh.rel_l2(gl[s], cl[s]))
+    # greedy ids are the argmax of the returned logits (lowest id on ties)
+    assert np.array_equal(gn, gl.argmax(axis=-1))
