@@ -274,6 +274,7 @@ def run_ours(args):
     if prof:
         line["roofline"] = prof["dominant"]
         line["roofline_decode_attention"] = prof.get("attn_decode")
+        line["roofline_decode_gemm"] = prof.get("gemm_decode")
         line["kernel_time_shares"] = prof["shares"]
         line["roofline"]["peak_source"] = peak_src
     if rank == 0 and ws == 1 and not args.no_cpu:
@@ -305,8 +306,10 @@ def profile_step(model, prompts, gens, flush):
                            native.ctypes.byref(n)), "bt_profile_end")
     hbm, tf_burst, tf_sus, _ = _peaks()
     kinds = {0: "gemm", 1: "attn_decode", 2: "attn_prefill", 3: "attn_local", 4: "layernorm",
-             5: "rope_append", 6: "embed", 7: "argmax", 8: "other"}
-    D = synth.WORKLOADS[RUNS[0]].shape.d_model
+             5: "rope_append", 6: "embed", 7: "argmax", 8: "other", 9: "token_step"}
+    shape0 = synth.WORKLOADS[RUNS[0]].shape
+    D = shape0.d_model
+    Nt = shape0.n_token_layers if shape0.use_token_decoder else 0
     cls = {}
     for i in range(n.value):
         rc = recs[i]
@@ -323,6 +326,11 @@ def profile_step(model, prompts, gens, flush):
             c["flops"] += 2.0 * rc.m * rc.n * rc.k
         elif k == "attn_decode":
             c["bytes"] += rc.m * (2.0 * rc.n * rc.k * 2 + 2.0 * rc.k * 2)
+        elif k == "token_step":
+            # every token-decoder weight (q|k|v|fc1 and o|fc2: 12 D^2 per layer)
+            # and the LM head, once per launch; activations stay in L2
+            c["bytes"] += 2.0 * (Nt * 12 * rc.k * rc.k + rc.n * rc.k)
+            c["flops"] += 2.0 * rc.m * (Nt * 12 * rc.k * rc.k + rc.n * rc.k)
     total = sum(c["ms"] for c in cls.values())
     shares = {k: round(c["ms"] / total, 4) for k, c in sorted(cls.items(), key=lambda kv: -kv[1]["ms"])}
     dom_name = max(cls, key=lambda k: cls[k]["ms"])
@@ -340,12 +348,14 @@ def profile_step(model, prompts, gens, flush):
                 "frac": ach / hbm, "traffic": None, "launches": c["launches"],
                 "avg_launch_us": per * 1e6}
 
-    out = {"dominant": roof(dom_name) if dom_name in ("gemm_decode", "gemm_prefill", "attn_decode")
+    out = {"dominant": roof(dom_name) if dom_name in ("gemm_decode", "gemm_prefill", "attn_decode", "token_step")
            else {"kernel": dom_name, "bound": "hbm", "achieved": None, "peak": hbm, "unit": "GB/s",
                  "frac": None, "traffic": None},
            "shares": shares}
     if "attn_decode" in cls:
         out["attn_decode"] = roof("attn_decode")
+    if "gemm_decode" in cls:
+        out["gemm_decode"] = roof("gemm_decode")
     return out
 
 
@@ -420,6 +430,30 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_decode_case(args):
+    """A bounded decode-only case for profiler captures: the decode-heavy
+    model and batch, its 128-token prompt, then --case-steps greedy decode
+    calls (every L_B-th a block step). Prints the mean ms per decode call."""
+    import torch
+    torch.cuda.set_device(0)
+    model, prompts = build(0)
+    r = RUNS[1]
+    x = synth.WORKLOADS[r]
+    out = torch.empty(args.case_steps + 1, x.batch, dtype=torch.int32, device="cuda")
+    model.prefill(prompts[r], next_tokens=out[0])
+    model.sync()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for i in range(1, args.case_steps + 1):
+        model.decode(None, next_tokens=out[i])
+    b.record()
+    model.sync()
+    print(json.dumps({"case": "decode", "workload": r, "steps": args.case_steps,
+                      "ms_per_decode_call": a.elapsed_time(b) / args.case_steps}), flush=True)
+    model.close()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -430,7 +464,13 @@ def main():
     ap.add_argument("--no-profile", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    ap.add_argument("--case", default=None, choices=["decode"],
+                    help="run a bounded decode-only case (profiler captures) instead of the benchmark")
+    ap.add_argument("--case-steps", type=int, default=8)
     args = ap.parse_args()
+    if args.case == "decode":
+        run_decode_case(args)
+        return
     if args.impl == "reference":
         run_reference(args)
     else:

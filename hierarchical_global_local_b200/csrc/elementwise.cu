@@ -396,18 +396,60 @@ __global__ void rope_append_kernel(const T* __restrict__ qkv, int D, int H, int 
   }
 }
 
+// V^T [(b*H + h)*d + e][pos] for positions p0 + [0, 64) of one (sequence,
+// head): the tile goes through shared memory so that both the reads (along
+// the head dims of a row) and the writes (along positions) are coalesced.
+// Rows of a sequence are consecutive; row i has position pos0 + i.
+template <typename T>
+__global__ void __launch_bounds__(256)
+vt_write_kernel(const T* __restrict__ qkv, int D, int H, int d, int rows, int pos0,
+                T* __restrict__ vt, int vt_ld) {
+  pdl_trigger();
+  pdl_wait();
+  __shared__ float tile[64][65];
+  const int bh = blockIdx.y, b = bh / H, h = bh - b * H;
+  const int i0 = blockIdx.x * 64;
+  const int ec = d < 64 ? d : 64;
+  for (int e0 = 0; e0 < d; e0 += ec) {
+    for (int x = threadIdx.x; x < 64 * ec; x += blockDim.x) {
+      const int ii = x / ec, e = x - ii * ec;
+      const int i = i0 + ii;
+      tile[ii][e] = (i < rows) ? to_f(qkv[((size_t)b * rows + i) * 3 * D + 2 * D + h * d + e0 + e]) : 0.f;
+    }
+    __syncthreads();
+    for (int x = threadIdx.x; x < 64 * ec; x += blockDim.x) {
+      const int e = x / 64, ii = x - e * 64;
+      const int i = i0 + ii;
+      if (i < rows) vt[((size_t)bh * d + e0 + e) * vt_ld + pos0 + i] = from_f<T>(tile[ii][e]);
+    }
+    __syncthreads();
+  }
+}
+
 cudaError_t launch_rope_append(int dt, const void* qkv, int M, int D, int H, int rot,
                                const float2* rope_tab, PosSpec pos, void* q_out, void* k_cache,
                                void* v_cache, int cap, cudaStream_t s, void* vt, int vt_ld) {
   if (M == 0) return cudaSuccess;
+  // V^T is written for positions known on the host (prefill) only
+  if (vt && pos.mode != POS_ZERO) return cudaErrorInvalidValue;
   if (dt == DT_BF16) {
     BT_LAUNCH(rope_append_kernel<bf16>, dim3(M), dim3(256), 0, s, (const bf16*)qkv, D, H, rot, rope_tab, pos,
-                                               (bf16*)q_out, (bf16*)k_cache, (bf16*)v_cache, cap, (bf16*)vt, vt_ld);
+                                               (bf16*)q_out, (bf16*)k_cache, (bf16*)v_cache, cap, (bf16*)nullptr, 0);
   }
   else {
     BT_LAUNCH(rope_append_kernel<float>, dim3(M), dim3(256), 0, s, (const float*)qkv, D, H, rot, rope_tab, pos,
                                                 (float*)q_out, (float*)k_cache, (float*)v_cache,
-                                                cap, (float*)vt, vt_ld);
+                                                cap, (float*)nullptr, 0);
+  }
+  if (vt) {
+    const int rows = pos.rows_per_seq, B = M / rows, d = D / H;
+    const dim3 grid((rows + 63) / 64, B * H);
+    if (dt == DT_BF16)
+      BT_LAUNCH(vt_write_kernel<bf16>, grid, dim3(256), 0, s, (const bf16*)qkv, D, H, d, rows, pos.add,
+                (bf16*)vt, vt_ld);
+    else
+      BT_LAUNCH(vt_write_kernel<float>, grid, dim3(256), 0, s, (const float*)qkv, D, H, d, rows, pos.add,
+                (float*)vt, vt_ld);
   }
   return cudaGetLastError();
 }

@@ -424,6 +424,27 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
           }
         }
         if (SWAP && e.ln_cnt) post_ln(e, b0, b0 + BN, M, N, ntA, s_rows, &s_nrows);
+      } else if (!SWAP) {
+        // activations as A: TMEM lane = token row. Transpose 32 x 32 blocks
+        // through this warp's shared-memory tile so that one store
+        // instruction covers 32 consecutive output columns of one row
+        float* tile = reinterpret_cast<float*>(smem + (size_t)stages * stage_bytes<BN>()) + warp * 32 * 33;
+        for (int c0 = 0; c0 < BN; c0 += 32) {
+          float v[32];
+          tmem_ld16(tb + c0, v);
+          tmem_ld16(tb + c0 + 16, v + 16);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) tile[lane * 33 + j] = v[j];
+          __syncwarp();
+          const int n = b0 + c0 + lane;
+          for (int rr = 0; rr < 32; ++rr) {
+            const int m = a0 + warp * 32 + rr;
+            if (m < M && n < N) epi_apply<bf16>(e, m, n, tile[rr * 33 + lane]);
+          }
+          __syncwarp();
+        }
+        tc_fence_before();
+        mbar_arrive(&acc_empty[buf]);
       } else {
         for (int c0 = 0; c0 < BN; c0 += 16) {
           float v[16];
@@ -576,8 +597,14 @@ cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& mb, int M, int 
     stages = nloc < stages ? nloc : stages;
     if (stages > fit) stages = fit;
   }
+  // activations as A: per-warp 32 x 33 fp32 transpose tiles for the epilogue
+  const size_t tr_bytes = SWAP ? 0 : (size_t)4 * 32 * 33 * 4;
+  if (!SWAP) {
+    int fit = (int)((SMEM_MAX - 1024 - tr_bytes) / SB);
+    if (stages > fit) stages = fit;
+  }
   if (stages < 2) stages = 2;
-  const size_t smem = (size_t)stages * SB + recv_bytes + 1024;
+  const size_t smem = (size_t)stages * SB + recv_bytes + tr_bytes + 1024;
   const int ntiles = ntA * ntB;
   dim3 grid;
   if (ks > 1) {
