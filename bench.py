@@ -454,6 +454,36 @@ def run_decode_case(args):
     model.close()
 
 
+def run_kernel_case(args):
+    """One op of the path through the op-level C-ABI, a few launches, for
+    profiler captures: decode attention (B, H, d, n) or a dense projection
+    (M, N, K) on the tensor-core path."""
+    import torch
+    from hierarchical_global_local_b200 import native
+    torch.cuda.set_device(0)
+    dims = [int(v) for v in args.case_shape.split(",")]
+    g = torch.Generator(device="cuda").manual_seed(7)
+    if args.case == "decode_attention":
+        B, H, d, n = dims
+        q = torch.randn(B, H * d, device="cuda", generator=g).bfloat16()
+        k = torch.randn(B, H, n, d, device="cuda", generator=g).bfloat16()
+        v = torch.randn(B, H, n, d, device="cuda", generator=g).bfloat16()
+        out = torch.empty(B, H * d, device="cuda", dtype=torch.bfloat16)
+        scr = native.decode_attention_scratch(native.BT_BF16, B, H, d, n)
+        run = lambda: native.decode_attention(q, k, v, n, out=out, scratch=scr)  # noqa: E731
+    else:
+        M, N, K = dims
+        x = torch.randn(M, K, device="cuda", generator=g).bfloat16()
+        w = torch.randn(N, K, device="cuda", generator=g).bfloat16()
+        out = torch.empty(M, N, device="cuda")
+        scr = torch.zeros(native.lib().bt_op_linear_scratch_bytes(M, N), dtype=torch.uint8, device="cuda")
+        run = lambda: native.linear(x, w, None, path=2, out=out, scratch=scr)  # noqa: E731
+    for _ in range(args.case_steps):
+        run()
+    torch.cuda.synchronize()
+    print(json.dumps({"case": args.case, "shape": dims, "launches": args.case_steps}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -464,12 +494,18 @@ def main():
     ap.add_argument("--no-profile", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
-    ap.add_argument("--case", default=None, choices=["decode"],
-                    help="run a bounded decode-only case (profiler captures) instead of the benchmark")
+    ap.add_argument("--case", default=None, choices=["decode", "decode_attention", "linear"],
+                    help="instead of the benchmark, run a bounded case for profiler captures: decode "
+                         "calls of the decode-heavy workload, or one op of the path")
     ap.add_argument("--case-steps", type=int, default=8)
+    ap.add_argument("--case-shape", default="128,16,64,640",
+                    help="decode_attention: B,H,d,n; linear: M,N,K")
     args = ap.parse_args()
     if args.case == "decode":
         run_decode_case(args)
+        return
+    if args.case in ("decode_attention", "linear"):
+        run_kernel_case(args)
         return
     if args.impl == "reference":
         run_reference(args)
