@@ -37,7 +37,7 @@
 // The MMA orientation is "weights as A": M = 128 output features per tile,
 // N = the batch padded to a multiple of 16, K in 64-wide swizzled blocks.
 //
-// Grid barriers are a counter in global memory (release by fence + atomic
+// Grid barriers are a counter in global memory (release by a red.release
 // add, acquire by polling with ld.acquire). All CTAs must be resident at
 // once: one CTA per SM, grid = number of SMs. Every wait is bounded: a
 // barrier that runs out sets ST_WAIT_TIMEOUT and an abort word that makes
@@ -59,8 +59,14 @@ constexpr int WORKERS = 128;                 // warps 0-3 (TMEM lanes 0-127)
 constexpr int THREADS = WORKERS + 64;        // warp 4: TMA producer, warp 5: MMA issuer
 constexpr int TILE_BYTES = 128 * 64 * 2;     // one weight box: 128 rows x 64 K (bf16)
 constexpr int MAX_STAGES = 12;
-constexpr int MAX_S1 = 4;                    // K splits of the q|k|v|fc1 GEMM
-constexpr int MAX_S2 = 16;                   // K splits of the [W_o | W_2] GEMM
+#ifndef TS_MAX_S1
+#define TS_MAX_S1 2
+#endif
+#ifndef TS_MAX_S2
+#define TS_MAX_S2 12
+#endif
+constexpr int MAX_S1 = TS_MAX_S1;            // K splits of the q|k|v|fc1 GEMM
+constexpr int MAX_S2 = TS_MAX_S2;            // K splits of the [W_o | W_2] GEMM
 constexpr int MAX_B = 64;
 constexpr int MAX_WIN = 8;                   // local-window slots (P + L_B - 1)
 constexpr int TMEM_COLS = 128;               // two accumulators of up to 64 columns
@@ -124,8 +130,9 @@ __device__ bool grid_sync(unsigned* bar, unsigned target, int* status, volatile 
   asm volatile("fence.proxy.async.global;" ::: "memory");
   wsync();  // this CTA's writes of the phase are issued
   if (threadIdx.x == 0 && !*s_abort) {
-    __threadfence();
-    atomicAdd(&bar[0], 1u);
+    // release: this CTA's writes of the phase (ordered before by the CTA
+    // barrier above) are visible to any CTA that acquires the count
+    asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(&bar[0]) : "memory");
     const long long t0 = clock64();
     int n = 0;
     while (ld_acquire(&bar[0]) < target) {
@@ -139,7 +146,6 @@ __device__ bool grid_sync(unsigned* bar, unsigned target, int* status, volatile 
         }
       }
     }
-    __threadfence();
   }
   wsync();
   return !*s_abort;
