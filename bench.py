@@ -306,10 +306,11 @@ def profile_step(model, prompts, gens, flush):
                            native.ctypes.byref(n)), "bt_profile_end")
     hbm, tf_burst, tf_sus, _ = _peaks()
     kinds = {0: "gemm", 1: "attn_decode", 2: "attn_prefill", 3: "attn_local", 4: "layernorm",
-             5: "rope_append", 6: "embed", 7: "argmax", 8: "other", 9: "token_step"}
+             5: "rope_append", 6: "embed", 7: "argmax", 8: "other", 9: "token_step", 10: "block_step"}
     shape0 = synth.WORKLOADS[RUNS[0]].shape
     D = shape0.d_model
     Nt = shape0.n_token_layers if shape0.use_token_decoder else 0
+    Nb = shape0.n_block_layers
     cls = {}
     for i in range(n.value):
         rc = recs[i]
@@ -326,6 +327,11 @@ def profile_step(model, prompts, gens, flush):
             c["flops"] += 2.0 * rc.m * rc.n * rc.k
         elif k == "attn_decode":
             c["bytes"] += rc.m * (2.0 * rc.n * rc.k * 2 + 2.0 * rc.k * 2)
+        elif k == "block_step":
+            # block-decoder, prefix, token-decoder and LM-head weights (the
+            # block KV read is not in the record and is left out)
+            c["bytes"] += 2.0 * ((Nb + Nt) * 12 * rc.k * rc.k + rc.k * rc.k + rc.n * rc.k)
+            c["flops"] += 2.0 * rc.m * ((Nb + Nt) * 12 * rc.k * rc.k + rc.k * rc.k + rc.n * rc.k)
         elif k == "token_step":
             # every token-decoder weight (q|k|v|fc1 and o|fc2: 12 D^2 per layer)
             # and the LM head, once per launch; activations stay in L2
@@ -348,7 +354,8 @@ def profile_step(model, prompts, gens, flush):
                 "frac": ach / hbm, "traffic": None, "launches": c["launches"],
                 "avg_launch_us": per * 1e6}
 
-    out = {"dominant": roof(dom_name) if dom_name in ("gemm_decode", "gemm_prefill", "attn_decode", "token_step")
+    out = {"dominant": roof(dom_name) if dom_name in ("gemm_decode", "gemm_prefill", "attn_decode", "token_step",
+                                                     "block_step")
            else {"kernel": dom_name, "bound": "hbm", "achieved": None, "peak": hbm, "unit": "GB/s",
                  "frac": None, "traffic": None},
            "shares": shares}

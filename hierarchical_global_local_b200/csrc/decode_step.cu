@@ -70,6 +70,15 @@ constexpr int MAX_S2 = TS_MAX_S2;            // K splits of the [W_o | W_2] GEMM
 constexpr int MAX_B = 64;
 constexpr int MAX_WIN = 8;                   // local-window slots (P + L_B - 1)
 constexpr int TMEM_COLS = 128;               // two accumulators of up to 64 columns
+// block-step decode attention: units of ATT_CH cache entries of one
+// (sequence, head), d_head 64; each worker warp streams its units' K and V
+// rows through ATT_SLOTS bulk-copy slots in the (then idle) activation buffer
+constexpr int ATT_CH = 32;
+constexpr int ATT_SLOTS = 3;
+constexpr int ATT_SLOT_BYTES = 2 * ATT_CH * 64 * 2;              // K and V rows
+constexpr int ATT_BYTES = 4 * ATT_SLOTS * ATT_SLOT_BYTES;        // 96 KB
+constexpr int ATT_PART = 68;                                     // m, l, o[64], pad
+constexpr int ATT_MAX_CHUNKS = 32;                               // n_cap <= 1024
 constexpr long long BAR_CYCLES = 2000000000LL;  // ~1 s at 1.9 GHz
 #ifndef PRODUCER_SLEEP_NS
 #define PRODUCER_SLEEP_NS 128  // back-off of the weight producer's slot waits
@@ -84,6 +93,7 @@ struct Plan {
   int T1, T2, TL;    // feature tiles: 7D/128, D/128, ceil(V/128)
   int nkb1, nkb2;    // 64-wide K blocks per split
   int nkbL;          // K blocks of the LM head (D/64)
+  int Sp, nkbp;      // prefix projection (block steps): K splits, K blocks per split
   int stages;
   float scale;       // log2(e) / sqrt(d_head)
 };
@@ -234,7 +244,8 @@ __device__ void ln_out(const float4* v, int D, float eps, const LnParams& p, bf1
 // ---- TMA producer (warp 4, one thread) ----------------------------------------
 // Walks exactly the (phase, unit, K block) sequence the MMA issuer consumes.
 __device__ void producer(const CUtensorMap* mq, const CUtensorMap* mo, const CUtensorMap* ml,
-                         const Plan& P, int Nt, uint8_t* ring, uint64_t* full, uint64_t* empty,
+                         const CUtensorMap* mqb, const CUtensorMap* mob, const CUtensorMap* mp,
+                         const Plan& P, int Nt, int Nb, uint8_t* ring, uint64_t* full, uint64_t* empty,
                          int* status, volatile int* s_abort) {
   const int G = gridDim.x, c = blockIdx.x;
   int it = 0;
@@ -255,6 +266,22 @@ __device__ void producer(const CUtensorMap* mq, const CUtensorMap* mo, const CUt
     else tc::tma_load_2d_hint(ring + (size_t)s * TILE_BYTES, m, x, y, &full[s], policy);
     ++it;
   };
+  // block step: block-decoder layers and the prefix projection first
+  for (int l = 0; l < Nb && !stop; ++l) {
+    for (int u = c; u < P.T1 * P.S1 && !stop; u += G) {
+      const int t = u % P.T1, sp = u / P.T1;
+      for (int kb = 0; kb < P.nkb1; ++kb) load(mqb, (sp * P.nkb1 + kb) * 64, t * 128, l, true);
+    }
+    for (int u = c; u < P.T2 * P.S2 && !stop; u += G) {
+      const int t = u % P.T2, sp = u / P.T2;
+      for (int kb = 0; kb < P.nkb2; ++kb) load(mob, (sp * P.nkb2 + kb) * 64, t * 128, l, true);
+    }
+  }
+  if (Nb > 0)
+    for (int u = c; u < P.T2 * P.Sp && !stop; u += G) {
+      const int t = u % P.T2, sp = u / P.T2;
+      for (int kb = 0; kb < P.nkbp; ++kb) load(mp, (sp * P.nkbp + kb) * 64, t * 128, 0, false);
+    }
   for (int l = 0; l < Nt && !stop; ++l) {
     for (int u = c; u < P.T1 * P.S1 && !stop; u += G) {
       const int t = u % P.T1, sp = u / P.T1;
@@ -354,7 +381,7 @@ __device__ void gemm_phase(const Plan& P, int T, int S, int nkb, const CUtensorM
 
 // MMA warp (one thread): the same unit sequence as the workers and the
 // producer. Waits for staged activations and a drained accumulator.
-__device__ void mma_issuer(const Plan& P, int Nt, uint8_t* ring, const uint8_t* act, uint32_t tmem,
+__device__ void mma_issuer(const Plan& P, int Nt, int Nb, uint8_t* ring, const uint8_t* act, uint32_t tmem,
                            const Sync& y, int* status, volatile int* s_abort) {
   const int G = gridDim.x, c = blockIdx.x;
   int it = 0, na = 0, nu = 0;
@@ -371,6 +398,15 @@ __device__ void mma_issuer(const Plan& P, int Nt, uint8_t* ring, const uint8_t* 
     ++nu;
     return true;
   };
+  for (int l = 0; l < Nb; ++l) {
+    for (int u = c; u < P.T1 * P.S1; u += G)
+      if (!unit(P.nkb1, true)) return;
+    for (int u = c; u < P.T2 * P.S2; u += G)
+      if (!unit(P.nkb2, true)) return;
+  }
+  if (Nb > 0)
+    for (int u = c; u < P.T2 * P.Sp; u += G)
+      if (!unit(P.nkbp, true)) return;
   for (int l = 0; l < Nt; ++l) {
     for (int u = c; u < P.T1 * P.S1; u += G)
       if (!unit(P.nkb1, true)) return;
@@ -489,6 +525,8 @@ __device__ void attend_item(const TokenStepArgs& a, const Plan& P, const float* 
   }
 }
 
+__device__ void gelu_fc1(const TokenStepArgs& a, const Plan& P, const float* bq);
+
 __device__ void r1_phase(const TokenStepArgs& a, const Plan& P, int l, int pos) {
   const int D = a.D, B = a.B;
   const float* bq = layer_ptr(a.b_qkv1, l, a.layer_stride);
@@ -506,8 +544,14 @@ __device__ void r1_phase(const TokenStepArgs& a, const Plan& P, int l, int pos) 
     else if (a.dh == 64) attend_item<64>(a, P, bq, kc, vc, b, h, pos, active);
     else attend_item<128>(a, P, bq, kc, vc, b, h, pos, active);
   }
-  // GELU(fc1): features 3D + c, c < 4D, of the first GEMM, four at a time
-  // (a group never crosses a 128-feature tile)
+  gelu_fc1(a, P, bq);
+}
+
+// GELU(fc1): features 3D + c, c < 4D, of the first GEMM (its K splits + the
+// bias) -> a2[:, D + c], four at a time (a group never crosses a 128-feature
+// tile)
+__device__ void gelu_fc1(const TokenStepArgs& a, const Plan& P, const float* bq) {
+  const int D = a.D, B = a.B;
   const int W4 = D;  // float4 groups per row
   const int E = B * W4;
   const int nthr = gridDim.x * WORKERS;
@@ -622,6 +666,294 @@ __device__ void ingest_phase(const TokenStepArgs& a, int jb, float* red) {
   }
 }
 
+// Row reduction for the out|fc2 and prefix GEMMs: h[b] = (residual ? h[b] : 0)
+// + bias + the S K-split partials (T tiles), then a LayerNorm of the new row:
+// LN1 | LN2 -> out (row stride 2D) when lp holds two, else one LN -> out
+// (row stride D). One CTA per row.
+__device__ void reduce_ln(const TokenStepArgs& a, const Plan& P, float* h, const float* bias, int S,
+                          bool residual, const float* g1, const float* b1, const float* g2,
+                          const float* b2, bf16* out, float* red) {
+  const int D = a.D, B = a.B;
+  LnParams lp;
+  if (blockIdx.x < B) ln_load(lp, D, g1, b1, g2, b2);
+  for (int b = blockIdx.x; b < B; b += gridDim.x) {
+    float4 hv[4];
+    float* hrow = h + (size_t)b * D;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int f = (threadIdx.x + u * WORKERS) * 4;
+      hv[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (f < D) {
+        float4 acc = *reinterpret_cast<const float4*>(bias + f);
+        if (residual) acc = f4add(acc, __ldcg(reinterpret_cast<const float4*>(hrow + f)));
+        const int t = f >> 7, off = f & 127;
+#pragma unroll
+        for (int sp = 0; sp < MAX_S2; ++sp)
+          if (sp < S)
+            acc = f4add(acc, __ldcg(reinterpret_cast<const float4*>(
+                                 a.p2 + ((size_t)(sp * P.T2 + t) * B + b) * 128 + off)));
+        hv[u] = acc;
+        __stcg(reinterpret_cast<float4*>(hrow + f), acc);
+      }
+    }
+    if (g2) ln_out(hv, D, a.eps, lp, out + (size_t)b * 2 * D, out + (size_t)b * 2 * D + D, red);
+    else ln_out(hv, D, a.eps, lp, out + (size_t)b * D, nullptr, red);
+  }
+}
+
+// Block step, phase I: block row of each sequence = the L_B token embeddings
+// of the completed block concatenated (the fed token is its last), then
+// LN1 | LN2 of block layer 0 -> x1.
+__device__ void block_ingest_phase(const TokenStepArgs& a, int jb, float* red) {
+  const int D = a.D, De = D / a.L_B;
+  LnParams lp;
+  if (blockIdx.x < a.B) ln_load(lp, D, a.bln1_g, a.bln1_b, a.bln2_g, a.bln2_b);
+  for (int b = blockIdx.x; b < a.B; b += gridDim.x) {
+    int tok = a.src[b];
+    if (tok < 0 || tok >= a.V) {
+      if (threadIdx.x == 0) set_status(a.status, ST_BAD_TOKEN);
+      tok = 0;
+    }
+    if (threadIdx.x == 0) a.block_tok[b * a.L_B + jb] = tok;
+    float4 hv[4];
+    float* hrow = a.h_b + (size_t)b * D;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int f = (threadIdx.x + u * WORKERS) * 4;
+      hv[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (f < D) {
+        // 4 | De: a float4 group never straddles two tokens' pieces
+        const int j = f / De, e = f - j * De;
+        int t = (j == jb) ? tok : a.block_tok[b * a.L_B + j];
+        if (t < 0 || t >= a.V) t = 0;
+        const uint2 w = *reinterpret_cast<const uint2*>(a.blk_emb + (size_t)t * De + e);
+        const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w.x));
+        const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w.y));
+        hv[u] = make_float4(lo.x, lo.y, hi.x, hi.y);
+        __stcg(reinterpret_cast<float4*>(hrow + f), hv[u]);
+      }
+    }
+    bf16* o = a.x1 + (size_t)b * 2 * D;
+    ln_out(hv, D, a.eps, lp, o, o + D, red);
+  }
+}
+
+// q, k or v (part 0, 1, 2) of head h of row b, head dims lane and lane + 32
+// (d_head 64): the K splits of the first GEMM + the bias, rotary on q and k.
+__device__ __forceinline__ void head_dims64(const TokenStepArgs& a, const Plan& P, const float* bq, int b,
+                                            int h, int part, int pos, float& x0, float& x1) {
+  const int lane = threadIdx.x & 31;
+  const size_t split_stride = (size_t)P.T1 * a.B * 128;
+  const int n0 = part * a.D + h * 64 + lane, n1 = n0 + 32;
+  float s0 = bq[n0], s1 = bq[n1];
+  const float* p0 = a.p1 + ((size_t)(n0 >> 7) * a.B + b) * 128 + (n0 & 127);
+  const float* p1 = a.p1 + ((size_t)(n1 >> 7) * a.B + b) * 128 + (n1 & 127);
+#pragma unroll
+  for (int sp = 0; sp < MAX_S1; ++sp)
+    if (sp < P.S1) {
+      s0 += __ldcg(p0 + sp * split_stride);
+      s1 += __ldcg(p1 + sp * split_stride);
+    }
+  if (part < 2 && a.rot > 0) {
+    // rotate-half pairs (e, e ^ half), e < rot <= 32: the pair of dim lane
+    // is in lane ^ half of the same register
+    const int half = a.rot >> 1;
+    const float r0 = __shfl_xor_sync(0xffffffffu, s0, half < 32 ? half : 0);
+    const float r1 = __shfl_xor_sync(0xffffffffu, s1, half < 32 ? half : 0);
+    const int e0 = lane, e1 = lane + 32;
+    if (e0 < a.rot) {
+      const float2 cs = a.rope_tab[(size_t)pos * half + (e0 & (half - 1))];
+      s0 = (e0 & half) ? s0 * cs.x + r0 * cs.y : s0 * cs.x - r0 * cs.y;
+    }
+    if (e1 < a.rot) {
+      const float2 cs = a.rope_tab[(size_t)pos * half + (e1 & (half - 1))];
+      s1 = (e1 & half) ? s1 * cs.x + r1 * cs.y : s1 * cs.x - r1 * cs.y;
+    }
+  }
+  x0 = s0;
+  x1 = s1;
+}
+
+// Block step, phase R1 of block layer l: decode attention of each
+// (sequence, head) over its n = pos + 1 block-cache entries, split into
+// units of ATT_CH entries spread evenly over the grid: a CTA takes a
+// contiguous range of units and each of its warps a contiguous quarter, so a
+// warp's units are mostly consecutive chunks of one (sequence, head). A warp
+// streams its units' K and V rows with 1-D bulk copies into its ATT_SLOTS
+// slots, scores one entry per lane and folds each unit into a running
+// (max, sum, weighted V) per (sequence, head); at the end of each run it
+// writes one partial and counts the run's units on the (sequence, head)'s
+// counter. The warp that completes the count merges the partials into a2.
+// The unit holding the newest entry (position pos) computes its k and v from
+// the first GEMM's partial sums, appends them to the cache and scores them
+// from shared memory. `katt` counts this warp's units over the launch (slot
+// and parity bookkeeping). Then GELU(fc1) as in the token layers.
+__device__ void block_attention_phase(const TokenStepArgs& a, const Plan& P, int l, int pos, uint8_t* att,
+                                      uint64_t* att_bar, float* q_s, int& katt) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int H = a.H, D = a.D;
+  const float* bq = layer_ptr(a.bb_qkv1, l, a.layer_stride);
+  bf16* kc = a.kb + (size_t)l * a.kb_layer;
+  bf16* vc = a.vb + (size_t)l * a.kb_layer;
+  const int n = pos + 1;
+  const int C = (n + ATT_CH - 1) / ATT_CH;
+  const long long U = (long long)a.B * H * C;
+  const long long c0 = U * blockIdx.x / gridDim.x, c1 = U * (blockIdx.x + 1) / gridDim.x;
+  const long long per_w = (c1 - c0 + 3) / 4;
+  const long long wb = c0 + warp * per_w;
+  const long long we = (wb + per_w < c1) ? wb + per_w : c1;
+  const int nm = we > wb ? (int)(we - wb) : 0;
+  uint8_t* wslot = att + (size_t)warp * ATT_SLOTS * ATT_SLOT_BYTES;
+  uint64_t* wbar = att_bar + warp * ATT_SLOTS;
+  float* qs = q_s + warp * 64;
+  auto issue = [&](int i) {  // lane 0
+    const long long u = wb + i;
+    const int pr = (int)(u / C), j = (int)(u - (long long)pr * C);
+    const int e0 = j * ATT_CH;
+    const int rows = min(ATT_CH, n - e0);
+    const int rc = (e0 + rows == n) ? rows - 1 : rows;  // the newest entry is not in the cache yet
+    const int slot = (katt + i) % ATT_SLOTS;
+    uint8_t* ks = wslot + (size_t)slot * ATT_SLOT_BYTES;
+    const uint32_t bytes = (uint32_t)rc * 128;
+    mbar_arrive_expect_tx(&wbar[slot], 2 * bytes);
+    if (bytes) {
+      const size_t off = ((size_t)pr * a.n_cap + e0) * 64;
+      bulk_g2s(ks, kc + off, bytes, &wbar[slot]);
+      bulk_g2s(ks + ATT_CH * 128, vc + off, bytes, &wbar[slot]);
+    }
+  };
+  if (lane == 0)
+    for (int i = 0; i < nm && i < ATT_SLOTS; ++i) issue(i);
+
+  // the (sequence, head) run in progress
+  int cur = -1, run_first = 0, run_len = 0;
+  float mr = -INFINITY, lr = 0.f, or0 = 0.f, or1 = 0.f;
+  auto flush = [&]() {
+    float* part = a.att_part + ((size_t)cur * C + run_first) * ATT_PART;
+    if (lane == 0) {
+      __stcg(part, mr);
+      __stcg(part + 1, lr);
+    }
+    __stcg(reinterpret_cast<float2*>(part + 2) + lane, make_float2(or0, or1));
+    __threadfence();
+    int old = 0;
+    if (lane == 0) old = atomicAdd(&a.att_cnt[cur], run_len);
+    old = __shfl_sync(0xffffffffu, old, 0);
+    if (old + run_len == C) {
+      // every unit of (b, h) is in: merge the runs' partials (slots of units
+      // that were not the first of a run hold m = -inf and are skipped)
+      __threadfence();
+      const int b = cur / H, h = cur - b * H;
+      const float* pp = a.att_part + (size_t)cur * C * ATT_PART;
+      const float mc = (lane < C) ? __ldcg(pp + (size_t)lane * ATT_PART) : -INFINITY;
+      const float lc = (lane < C && mc != -INFINITY) ? __ldcg(pp + (size_t)lane * ATT_PART + 1) : 0.f;
+      const float M = warp_max(mc);
+      const float wc = (lane < C && mc != -INFINITY) ? exp2f(mc - M) : 0.f;
+      const float L = warp_sum(lc * wc);
+      float O0 = 0.f, O1 = 0.f;
+      for (int c = 0; c < C; ++c) {
+        const float w = __shfl_sync(0xffffffffu, wc, c);
+        if (w != 0.f) {
+          const float2 oc = __ldcg(reinterpret_cast<const float2*>(pp + (size_t)c * ATT_PART + 2) + lane);
+          O0 = fmaf(w, oc.x, O0);
+          O1 = fmaf(w, oc.y, O1);
+        }
+      }
+      const float inv = 1.f / L;
+      *reinterpret_cast<__nv_bfloat162*>(a.a2 + (size_t)b * 5 * D + h * 64 + 2 * lane) =
+          __floats2bfloat162_rn(O0 * inv, O1 * inv);
+      if (lane == 0) a.att_cnt[cur] = 0;  // ready for the next layer / step
+    }
+  };
+
+  for (int i = 0; i < nm; ++i) {
+    const long long u = wb + i;
+    const int pr = (int)(u / C), j = (int)(u - (long long)pr * C);
+    if (pr != cur) {
+      if (cur >= 0) flush();
+      cur = pr;
+      run_first = j;
+      run_len = 0;
+      mr = -INFINITY;
+      lr = or0 = or1 = 0.f;
+      float q0, q1;
+      head_dims64(a, P, bq, pr / H, pr % H, 0, pos, q0, q1);
+      __syncwarp();
+      qs[lane] = q0 * P.scale;
+      qs[lane + 32] = q1 * P.scale;
+    } else if (lane == 0) {
+      __stcg(a.att_part + ((size_t)pr * C + j) * ATT_PART, -INFINITY);  // not a run's first unit
+    }
+    const int e0 = j * ATT_CH;
+    const int rows = min(ATT_CH, n - e0);
+    const bool newest = (e0 + rows == n);
+    const int slot = (katt + i) % ATT_SLOTS;
+    uint8_t* ks = wslot + (size_t)slot * ATT_SLOT_BYTES;
+    uint8_t* vs = ks + ATT_CH * 128;
+    float k0 = 0.f, k1 = 0.f, v0 = 0.f, v1 = 0.f;
+    if (newest) {
+      head_dims64(a, P, bq, pr / H, pr % H, 1, pos, k0, k1);
+      head_dims64(a, P, bq, pr / H, pr % H, 2, pos, v0, v1);
+    }
+    mbar_wait_bounded(&wbar[slot], ((katt + i) / ATT_SLOTS) & 1, a.status);
+    if (newest) {
+      const bf16 kb0 = __float2bfloat16_rn(k0), kb1 = __float2bfloat16_rn(k1);
+      const bf16 vb0 = __float2bfloat16_rn(v0), vb1 = __float2bfloat16_rn(v1);
+      const size_t off = ((size_t)pr * a.n_cap + pos) * 64;
+      kc[off + lane] = kb0;
+      kc[off + lane + 32] = kb1;
+      vc[off + lane] = vb0;
+      vc[off + lane + 32] = vb1;
+      bf16* kr = reinterpret_cast<bf16*>(ks + (size_t)(rows - 1) * 128);
+      bf16* vr = reinterpret_cast<bf16*>(vs + (size_t)(rows - 1) * 128);
+      kr[lane] = kb0;
+      kr[lane + 32] = kb1;
+      vr[lane] = vb0;
+      vr[lane + 32] = vb1;
+    }
+    __syncwarp();
+    // scores, one entry per lane; the word order is rotated per lane so that
+    // the 32 lanes read 32 different banks
+    float sc = -INFINITY;
+    if (lane < rows) {
+      const uint32_t* kr = reinterpret_cast<const uint32_t*>(ks + (size_t)lane * 128);
+      float acc = 0.f;
+#pragma unroll 8
+      for (int w = 0; w < 32; ++w) {
+        const int ww = (w + lane) & 31;
+        const uint32_t kw = kr[ww];
+        const float2 kf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&kw));
+        acc = fmaf(qs[2 * ww], kf.x, acc);
+        acc = fmaf(qs[2 * ww + 1], kf.y, acc);
+      }
+      sc = acc;
+    }
+    const float mx = fmaxf(warp_max(sc), mr);
+    const float pj = (lane < rows) ? exp2f(sc - mx) : 0.f;
+    const float cf = exp2f(mr - mx);
+    lr = lr * cf + warp_sum(pj);
+    or0 *= cf;
+    or1 *= cf;
+    mr = mx;
+    // weighted V for head dims 2*lane, 2*lane + 1
+    for (int jj = 0; jj < rows; ++jj) {
+      const float pw = __shfl_sync(0xffffffffu, pj, jj);
+      const uint32_t vw = reinterpret_cast<const uint32_t*>(vs + (size_t)jj * 128)[lane];
+      const float2 vf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&vw));
+      or0 = fmaf(pw, vf.x, or0);
+      or1 = fmaf(pw, vf.y, or1);
+    }
+    ++run_len;
+    // this slot's generic reads are done before the next bulk copy into it
+    fence_proxy_async();
+    __syncwarp();
+    if (lane == 0 && i + ATT_SLOTS < nm) issue(i + ATT_SLOTS);
+  }
+  if (cur >= 0) flush();
+  katt += nm;
+  gelu_fc1(a, P, bq);
+}
+
 __device__ __forceinline__ void better(float& v, int& i, float ov, int oi) {
   if (ov > v || (ov == v && oi < i)) { v = ov; i = oi; }
 }
@@ -722,11 +1054,14 @@ __device__ void argmax_phase(const TokenStepArgs& a, const Plan& P) {
   }
 }
 
+// BLOCK = false: token steps only (no block-step code, fewer registers)
+template <bool BLOCK>
 __global__ void __launch_bounds__(THREADS, 1)
 token_step_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mo,
                   const __grid_constant__ CUtensorMap ml, const __grid_constant__ CUtensorMap mx1,
                   const __grid_constant__ CUtensorMap ma2, const __grid_constant__ CUtensorMap mxf,
-                  const TokenStepArgs a, const Plan P) {
+                  const __grid_constant__ CUtensorMap mqb, const __grid_constant__ CUtensorMap mob,
+                  const __grid_constant__ CUtensorMap mp, const TokenStepArgs a, const Plan P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~(uintptr_t)1023);
@@ -737,13 +1072,17 @@ token_step_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
   __shared__ float red[4];
   __shared__ float2 s_arg[4][MAX_B];
   __shared__ volatile int s_abort;
+  __shared__ __align__(8) uint64_t att_bar[4 * ATT_SLOTS];  // block-step attention slots
+  __shared__ float q_s[4 * 64];
 
   const int warp = threadIdx.x >> 5;
+  const int Nb = (BLOCK && a.block) ? a.Nb : 0;
   if (threadIdx.x == 0) {
     for (int i = 0; i < P.stages; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
     }
+    for (int i = 0; i < 4 * ATT_SLOTS; ++i) mbar_init(&att_bar[i], 1);
     mbar_init(&act_full, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&acc_full[i], 1);
@@ -762,9 +1101,10 @@ token_step_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
 
   if (warp == 4) {
     // weights do not depend on earlier kernels: no wait before streaming them
-    if ((threadIdx.x & 31) == 0) producer(&mq, &mo, &ml, P, a.Nt, ring, full, empty, a.status, &s_abort);
+    if ((threadIdx.x & 31) == 0)
+      producer(&mq, &mo, &ml, &mqb, &mob, &mp, P, a.Nt, Nb, ring, full, empty, a.status, &s_abort);
   } else if (warp == 5) {
-    if ((threadIdx.x & 31) == 0) mma_issuer(P, a.Nt, ring, act, tmem, y, a.status, &s_abort);
+    if ((threadIdx.x & 31) == 0) mma_issuer(P, a.Nt, Nb, ring, act, tmem, y, a.status, &s_abort);
   } else {
     pdl_wait();
     const int G = gridDim.x;
@@ -773,9 +1113,47 @@ token_step_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
     unsigned nb = 0;
     int na = 0, nu = 0;
     bool ok;
-    ingest_phase(a, jb, red);
-    ok = grid_sync(a.bar, ++nb * G, a.status, &s_abort);
     const int D = a.D;
+    if (BLOCK && Nb > 0) {
+      // block step: block embedding, the block-decoder layers at block
+      // position dstate[2], LN_b, the prefix projection (-> h, LN1 | LN2 of
+      // token layer 0)
+      const int bpos = a.dstate[2];
+      int katt = 0;
+      block_ingest_phase(a, jb, red);
+      ok = grid_sync(a.bar, ++nb * G, a.status, &s_abort);
+      for (int l = 0; ok && l < Nb; ++l) {
+        gemm_phase(P, P.T1, P.S1, P.nkb1, &mx1, [=](int t) { return t * 128 < 3 * D ? 0 : D; }, a.B, a.p1,
+                   act, tmem, y, na, nu, a.status);
+        if (!(ok = grid_sync(a.bar, ++nb * G, a.status, &s_abort))) break;
+        block_attention_phase(a, P, l, bpos, act, att_bar, q_s, katt);
+        if (!(ok = grid_sync(a.bar, ++nb * G, a.status, &s_abort))) break;
+        gemm_phase(P, P.T2, P.S2, P.nkb2, &ma2, [](int) { return 0; }, a.B, a.p2, act, tmem, y, na, nu,
+                   a.status);
+        if (!(ok = grid_sync(a.bar, ++nb * G, a.status, &s_abort))) break;
+        if (l + 1 < Nb)
+          reduce_ln(a, P, a.h_b, layer_ptr(a.bb_o2, l, a.layer_stride), P.S2, true,
+                    layer_ptr(a.bln1_g, l + 1, a.layer_stride), layer_ptr(a.bln1_b, l + 1, a.layer_stride),
+                    layer_ptr(a.bln2_g, l + 1, a.layer_stride), layer_ptr(a.bln2_b, l + 1, a.layer_stride),
+                    a.x1, red);
+        else
+          reduce_ln(a, P, a.h_b, layer_ptr(a.bb_o2, l, a.layer_stride), P.S2, true, a.lnb_g, a.lnb_b,
+                    nullptr, nullptr, a.xf, red);
+        ok = grid_sync(a.bar, ++nb * G, a.status, &s_abort);
+      }
+      if (ok) {
+        gemm_phase(P, P.T2, P.Sp, P.nkbp, &mxf, [](int) { return 0; }, a.B, a.p2, act, tmem, y, na, nu,
+                   a.status);
+        ok = grid_sync(a.bar, ++nb * G, a.status, &s_abort);
+      }
+      if (ok) {
+        reduce_ln(a, P, a.h, a.b_prefix, P.Sp, false, a.ln1_g, a.ln1_b, a.ln2_g, a.ln2_b, a.x1, red);
+        ok = grid_sync(a.bar, ++nb * G, a.status, &s_abort);
+      }
+    } else {
+      ingest_phase(a, jb, red);
+      ok = grid_sync(a.bar, ++nb * G, a.status, &s_abort);
+    }
     for (int l = 0; ok && l < a.Nt; ++l) {
       // G1: q|k|v tiles read LN1(h), fc1 tiles LN2(h)
       gemm_phase(P, P.T1, P.S1, P.nkb1, &mx1, [=](int t) { return t * 128 < 3 * D ? 0 : D; }, a.B, a.p1,
@@ -883,10 +1261,13 @@ Device& device() {
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
-        cudaFuncGetAttributes(&fa, token_step_kernel) != cudaSuccess)
+        cudaFuncGetAttributes(&fa, token_step_kernel<true>) != cudaSuccess)
       return d;
+    // both instantiations declare the same static shared memory
     d.smem_max = (size_t)optin - fa.sharedSizeBytes;
-    if (cudaFuncSetAttribute(token_step_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(token_step_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)d.smem_max) != cudaSuccess ||
+        cudaFuncSetAttribute(token_step_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)d.smem_max) != cudaSuccess)
       return d;
     d.ready = true;
@@ -901,7 +1282,8 @@ int divisor_at_most(int n, int cap) {
   return 1;
 }
 
-bool make_plan(int B, int D, int dh, int V, int sms, size_t smem_max, Plan* P, size_t* smem) {
+bool make_plan(int B, int D, int dh, int V, int sms, size_t smem_max, Plan* P, size_t* smem,
+               bool block = false) {
   Plan p{};
   p.Bp = (B + 15) / 16 * 16;
   p.T1 = 7 * D / 128;
@@ -917,11 +1299,18 @@ bool make_plan(int B, int D, int dh, int V, int sms, size_t smem_max, Plan* P, s
   p.nkb1 = kb1 / p.S1;
   p.nkb2 = kb2 / p.S2;
   p.nkbL = kb1;
+  // prefix projection of block steps: N = D, K = D
+  int cp = sms / p.T2;
+  if (cp > MAX_S2) cp = MAX_S2;
+  p.Sp = divisor_at_most(kb1, cp < 1 ? 1 : cp);
+  p.nkbp = kb1 / p.Sp;
   // the activation buffer holds the LM head's whole input (the largest unit)
+  // and, on block steps, the decode-attention slots of the four worker warps
   int act_kb = p.nkbL;
   if (p.nkb1 > act_kb) act_kb = p.nkb1;
   if (p.nkb2 > act_kb) act_kb = p.nkb2;
-  const size_t act = (size_t)act_kb * p.Bp * 128;
+  size_t act = (size_t)act_kb * p.Bp * 128;
+  if (block && act < (size_t)ATT_BYTES) act = ATT_BYTES;
   if (smem_max < act + 1024 + 4 * (size_t)TILE_BYTES) return false;
   int st = (int)((smem_max - act - 1024) / TILE_BYTES);
   p.stages = st > MAX_STAGES ? MAX_STAGES : st;
@@ -950,19 +1339,37 @@ int token_step_supported(int dt, int B, int D, int H, int rot, int V, int Nt, in
   return make_plan(B, D, dh, V, d.sms, d.smem_max, &p, &smem) ? 1 : 0;
 }
 
-size_t token_step_scratch_floats(int B, int D, int which) {
+int token_step_block_supported(int dt, int B, int D, int H, int rot, int V, int Nt, int Nb, int P_prefix,
+                               int l_cap, int n_cap, int L_B) {
+  if (!token_step_supported(dt, B, D, H, rot, V, Nt, P_prefix, l_cap)) return 0;
+  if (Nb < 1 || D / H != 64 || n_cap < 1 || n_cap > ATT_CH * ATT_MAX_CHUNKS) return 0;
+  // a float4 of the block embedding never straddles two tokens' pieces
+  if (L_B < 1 || D % L_B || (D / L_B) % 4) return 0;
+  return 1;
+}
+
+size_t token_step_scratch_floats(int B, int D, int which, int H, int n_cap) {
   // upper bounds over every plan: T1 * MAX_S1 and T2 * MAX_S2 partial tiles
   if (B > MAX_B) B = MAX_B;
+  if (which == 3) {
+    const int C = (n_cap + ATT_CH - 1) / ATT_CH;
+    return (size_t)B * H * C * ATT_PART;
+  }
   return which == 1 ? (size_t)(7 * D / 128) * MAX_S1 * B * 128 : (size_t)(D / 128) * MAX_S2 * B * 128;
 }
 
 cudaError_t launch_token_step(const TokenStepArgs& a, const void* w_qkv1, const void* w_o2,
-                              const void* w_lm, cudaStream_t s) {
+                              const void* w_lm, const void* w_qkv1_b, const void* w_o2_b,
+                              const void* w_prefix, cudaStream_t s) {
   if (!token_step_supported(DT_BF16, a.B, a.D, a.H, a.rot, a.V, a.Nt, 1, a.l_cap)) return cudaErrorNotSupported;
+  if (a.block && (!w_qkv1_b || !w_o2_b || !w_prefix ||
+                  !token_step_block_supported(DT_BF16, a.B, a.D, a.H, a.rot, a.V, a.Nt, a.Nb, 1, a.l_cap,
+                                              a.n_cap, a.L_B)))
+    return cudaErrorNotSupported;
   Device& d = device();
   Plan P;
   size_t smem;
-  if (!make_plan(a.B, a.D, a.dh, a.V, d.sms, d.smem_max, &P, &smem)) return cudaErrorNotSupported;
+  if (!make_plan(a.B, a.D, a.dh, a.V, d.sms, d.smem_max, &P, &smem, a.block != 0)) return cudaErrorNotSupported;
   CUtensorMap mq, mo, ml;
   // one layer: any stride at least the layer's own size satisfies the encoder
   const long long lsq = a.Nt > 1 ? a.layer_stride : 14LL * a.D * a.D;
@@ -974,9 +1381,19 @@ cudaError_t launch_token_step(const TokenStepArgs& a, const void* w_qkv1, const 
   if (!act_map(&mx1, a.x1, a.B, 2LL * a.D, P.Bp) || !act_map(&ma2, a.a2, a.B, 5LL * a.D, P.Bp) ||
       !act_map(&mxf, a.xf, a.B, a.D, P.Bp))
     return cudaErrorInvalidValue;
+  // block-step weights (token steps pass the token maps; they are not read)
+  CUtensorMap mqb = mq, mob = mo, mp = ml;
+  if (a.block) {
+    const long long bsq = a.Nb > 1 ? a.layer_stride : 14LL * a.D * a.D;
+    const long long bso = a.Nb > 1 ? a.layer_stride : 10LL * a.D * a.D;
+    if (!weight_map(&mqb, w_qkv1_b, a.D, 7LL * a.D, a.Nb, bsq) ||
+        !weight_map(&mob, w_o2_b, 5LL * a.D, a.D, a.Nb, bso) || !weight_map(&mp, w_prefix, a.D, a.D, 0, 0))
+      return cudaErrorInvalidValue;
+  }
   // every CTA must be resident at once (grid barriers): one per SM
   int per_sm = 0;
-  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, token_step_kernel, THREADS, smem);
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+      &per_sm, a.block ? token_step_kernel<true> : token_step_kernel<false>, THREADS, smem);
   if (e != cudaSuccess) return e;
   if (per_sm < 1) return cudaErrorNotSupported;
   cudaLaunchConfig_t cfg = {};
@@ -989,7 +1406,8 @@ cudaError_t launch_token_step(const TokenStepArgs& a, const void* w_qkv1, const 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl_enabled() ? 1 : 0;
-  e = cudaLaunchKernelEx(&cfg, token_step_kernel, mq, mo, ml, mx1, ma2, mxf, a, P);
+  if (a.block) e = cudaLaunchKernelEx(&cfg, token_step_kernel<true>, mq, mo, ml, mx1, ma2, mxf, mqb, mob, mp, a, P);
+  else e = cudaLaunchKernelEx(&cfg, token_step_kernel<false>, mq, mo, ml, mx1, ma2, mxf, mqb, mob, mp, a, P);
   note_launch();
   return e;
 }

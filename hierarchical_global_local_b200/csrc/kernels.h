@@ -200,12 +200,34 @@ struct TokenStepArgs {
   float *p1, *p2;    // split-K partials (token_step_scratch_floats)
   unsigned* bar;     // 3 words, zero before the first launch
   int* status;
+  // Block step (block = 1): the fed token completes a block. The block
+  // embedding, every block-decoder layer (decode attention over the block
+  // cache, the new entry appended at dstate[2]), LN_b and the prefix
+  // projection run first; the token decoder then runs over the prefix row
+  // (pos must be position 0) and no token is ingested. Block layer l's
+  // parameters sit at block layer 0's pointers plus l * layer_stride bytes.
+  int block, Nb, n_cap;
+  const bf16* blk_emb;
+  float* h_b;        // [B, D] fp32 block-decoder residual rows
+  const float *bb_qkv1, *bb_o2, *bln1_g, *bln1_b, *bln2_g, *bln2_b;
+  bf16 *kb, *vb;     // block caches [layer][B][H][n_cap][dh]
+  long long kb_layer;
+  const float *lnb_g, *lnb_b, *b_prefix;
+  float* att_part;   // decode-attention chunk partials (token_step_scratch_floats, which = 3)
+  int* att_cnt;      // [B * H] merge counters, zero between launches
 };
 int token_step_supported(int dt, int B, int D, int H, int rot, int V, int Nt, int P_prefix, int l_cap);
-// which = 1: first-GEMM partials, 2: second-GEMM partials (floats, for B rows)
-size_t token_step_scratch_floats(int B, int D, int which);
+// the block-step form as well (d_head 64, at least one block layer)
+int token_step_block_supported(int dt, int B, int D, int H, int rot, int V, int Nt, int Nb, int P_prefix,
+                               int l_cap, int n_cap, int L_B);
+// which = 1: first-GEMM partials, 2: second-GEMM partials (floats, for B rows);
+// 3: block decode-attention partials for n_cap cached entries
+size_t token_step_scratch_floats(int B, int D, int which, int H = 0, int n_cap = 0);
+// w_qkv1_b, w_o2_b, w_prefix: block layer 0's weights and the prefix
+// projection, used when a.block (may be null otherwise)
 cudaError_t launch_token_step(const TokenStepArgs& a, const void* w_qkv1, const void* w_o2,
-                              const void* w_lm, cudaStream_t s);
+                              const void* w_lm, const void* w_qkv1_b, const void* w_o2_b,
+                              const void* w_prefix, cudaStream_t s);
 
 // ---- LM head argmax ---------------------------------------------------------
 // next[b] = argmax_v logits[b, v] (lowest id among ties).

@@ -132,6 +132,8 @@ struct bt_model {
   int* ln_cnt = nullptr;       // per-row counters of the LayerNorm fused into GEMM epilogues
   float *ts_p1 = nullptr, *ts_p2 = nullptr;  // fused token step: split-K partials
   unsigned* ts_bar = nullptr;                // fused token step: grid-barrier words
+  float* ts_att = nullptr;                   // fused block step: decode-attention partials
+  int* ts_cnt = nullptr;                     // fused block step: merge counters [B_max * H]
   GemmScratch gs{};
   int B = 0, t = 0;
   bool prefilled = false;
@@ -242,6 +244,8 @@ static size_t carve(bt_model* m, const Dims& d, void* ws) {
     m->ts_p1 = (float*)c.take(token_step_scratch_floats(d.Bmax, d.D, 1) * 4);
     m->ts_p2 = (float*)c.take(token_step_scratch_floats(d.Bmax, d.D, 2) * 4);
     m->ts_bar = (unsigned*)c.take(64);
+    m->ts_att = (float*)c.take(token_step_scratch_floats(d.Bmax, d.D, 3, d.H, d.n_cap) * 4);
+    m->ts_cnt = (int*)c.take((size_t)d.Bmax * d.H * sizeof(int));
   }
   m->vt_ld = (d.n_cap + 63) / 64 * 64;
   m->vtr = c.take((size_t)d.Bmax * D * m->vt_ld * eb);
@@ -356,6 +360,7 @@ int bt_create(const bt_config* cfg, const bt_weights* w, void* ws, size_t ws_byt
   BT_TRYC(cudaMemsetAsync(m->block_tok, 0, (size_t)d.Bmax * d.L * 4, st));
   BT_TRYC(cudaMemsetAsync(m->ln_cnt, 0, (size_t)d.Bmax * (d.P > 1 ? d.P : 1) * sizeof(int), st));
   if (m->ts_bar) BT_TRYC(cudaMemsetAsync(m->ts_bar, 0, 64, st));
+  if (m->ts_cnt) BT_TRYC(cudaMemsetAsync(m->ts_cnt, 0, (size_t)d.Bmax * d.H * sizeof(int), st));
   BT_TRYC(cudaStreamCreateWithFlags(&m->cap_stream, cudaStreamNonBlocking));
   if (d.dt == BT_BF16) BT_TRYC(gemm_tc_prepare());
   BT_TRYC(attn_prepare());
@@ -649,8 +654,40 @@ static bool token_step_fused(const bt_model* m, int B) {
   return true;
 }
 
+// The block-step form of the same kernel (block embedding, block-decoder
+// layers with the decode attention as one of its phases, LN_b and the
+// prefix projection) is opt-in: BT_DECODE_BLOCK_STEP=fused. On B200 at batch
+// 64 it beats the kernel chain while the block cache is short (392 against
+// 435 us per block step at ~35 entries) but loses as the cache grows: the
+// attention phase has four worker warps per SM where the separate decode-
+// attention kernel keeps sixteen consumer warps per SM busy.
+static bool block_step_fused(const bt_model* m, int B) {
+  const Dims& d = m->d;
+  const char* env = getenv("BT_DECODE_BLOCK_STEP");
+  if (!env || strcmp(env, "fused") != 0) return false;
+  if (!m->ts_att || d.Nb < 1 || d.P != 1) return false;
+  if (!token_step_block_supported(d.dt, B, d.D, d.H, d.rot, d.V, d.Nt, d.Nb, d.P, d.l_cap, d.n_cap, d.L))
+    return false;
+  const long long ls = d.Nt > 1 ? (long long)((uint8_t*)m->tok[1].w_qkv1 - (uint8_t*)m->tok[0].w_qkv1) : 0;
+  const long long lsb = d.Nb > 1 ? (long long)((uint8_t*)m->blk[1].w_qkv1 - (uint8_t*)m->blk[0].w_qkv1) : ls;
+  if (d.Nt > 1 && d.Nb > 1 && ls != lsb) return false;
+  const long long stride = d.Nt > 1 ? ls : lsb;
+  for (int l = 0; l < d.Nb; ++l) {
+    const LayerW& w = m->blk[l];
+    const LayerW& w0 = m->blk[0];
+    auto at = [&](const void* p, const void* p0) {
+      return (const uint8_t*)p == (const uint8_t*)p0 + (long long)l * stride;
+    };
+    if (!at(w.w_qkv1, w0.w_qkv1) || !at(w.w_o2, w0.w_o2) || !at(w.b_qkv1, w0.b_qkv1) ||
+        !at(w.b_o2, w0.b_o2) || !at(w.ln1_g, w0.ln1_g) || !at(w.ln1_b, w0.ln1_b) ||
+        !at(w.ln2_g, w0.ln2_g) || !at(w.ln2_b, w0.ln2_b))
+      return false;
+  }
+  return true;
+}
+
 static int run_token_step(bt_model* m, int B, bool ingest, PosSpec pos, const int32_t* src,
-                          bool want_logits, cudaStream_t s) {
+                          bool want_logits, cudaStream_t s, bool block = false) {
   const Dims& d = m->d;
   const LayerW& w0 = m->tok[0];
   TokenStepArgs a{};
@@ -665,8 +702,22 @@ static int run_token_step(bt_model* m, int B, bool ingest, PosSpec pos, const in
   a.h = m->h_t; a.x1 = (bf16*)m->x1; a.a2 = (bf16*)m->a2; a.xf = (bf16*)m->xf;
   a.logits = want_logits ? m->logits : nullptr; a.next = m->next; a.arg_part = m->arg_part;
   a.p1 = m->ts_p1; a.p2 = m->ts_p2; a.bar = m->ts_bar; a.status = m->status;
-  ProfScope p(m, s, BT_K_TOKEN_STEP, B, d.V, d.D);
-  BT_CUDA(launch_token_step(a, w0.w_qkv1, w0.w_o2, m->w_lm, s));
+  const void *wqb = nullptr, *wob = nullptr;
+  if (block) {
+    const LayerW& b0 = m->blk[0];
+    a.block = 1; a.Nb = d.Nb; a.n_cap = d.n_cap;
+    if (d.Nt <= 1 && d.Nb > 1)
+      a.layer_stride = (long long)((uint8_t*)m->blk[1].w_qkv1 - (uint8_t*)b0.w_qkv1);
+    a.blk_emb = (const bf16*)m->blk_emb; a.h_b = m->h_b;
+    a.bb_qkv1 = b0.b_qkv1; a.bb_o2 = b0.b_o2; a.bln1_g = b0.ln1_g; a.bln1_b = b0.ln1_b;
+    a.bln2_g = b0.ln2_g; a.bln2_b = b0.ln2_b;
+    a.kb = (bf16*)m->kb; a.vb = (bf16*)m->vb; a.kb_layer = (long long)m->kb_layer;
+    a.lnb_g = m->lnf_b_g; a.lnb_b = m->lnf_b_b; a.b_prefix = m->b_prefix;
+    a.att_part = m->ts_att; a.att_cnt = m->ts_cnt;
+    wqb = b0.w_qkv1; wob = b0.w_o2;
+  }
+  ProfScope p(m, s, block ? BT_K_BLOCK_STEP : BT_K_TOKEN_STEP, B, d.V, d.D);
+  BT_CUDA(launch_token_step(a, w0.w_qkv1, w0.w_o2, m->w_lm, wqb, wob, block ? m->w_prefix : nullptr, s));
   return BT_OK;
 }
 
@@ -677,6 +728,8 @@ static int enqueue_decode_token_step(bt_model* m, bool block_step, bool greedy, 
   const int B = m->B;
   const int32_t* src = greedy ? m->next : m->fed;
   if (!block_step) return run_token_step(m, B, true, PosSpec{m->dstate, POS_LOCAL, d.P, 1}, src, want_logits, s);
+  if (block_step_fused(m, B))
+    return run_token_step(m, B, false, PosSpec{nullptr, POS_ZERO, 0, 1}, src, want_logits, s, true);
   {
     ProfScope p(m, s, BT_K_EMBED, B, d.D, 0);
     BT_CUDA(launch_ingest(d.dt, src, m->block_tok, m->dstate, B, d.L, d.V, d.D, 1, m->blk_emb,
@@ -765,6 +818,7 @@ int bt_prefill(bt_model* m, const int32_t* tokens, int32_t B, int32_t T, float* 
                           attn_decode_scratch_bytes(d.Bmax, d.H, d.d, d.n_cap, d.dt), s));
   // and the fused token step's barrier words (an aborted step leaves them set)
   if (m->ts_bar) BT_CUDA(cudaMemsetAsync(m->ts_bar, 0, 64, s));
+  if (m->ts_cnt) BT_CUDA(cudaMemsetAsync(m->ts_cnt, 0, (size_t)d.Bmax * d.H * sizeof(int), s));
   const long long k0 = launch_count();
   BT_CUDA(launch_set_state(m->dstate, T, d.L, s));
   {

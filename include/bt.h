@@ -173,7 +173,8 @@ BT_API int bt_destroy(bt_model *m);
 enum {
   BT_K_GEMM = 0, BT_K_ATTN_DECODE = 1, BT_K_ATTN_PREFILL = 2, BT_K_ATTN_LOCAL = 3,
   BT_K_LAYERNORM = 4, BT_K_ROPE_APPEND = 5, BT_K_EMBED = 6, BT_K_ARGMAX = 7, BT_K_OTHER = 8,
-  BT_K_TOKEN_STEP = 9  /* fused token decoder + LM head + argmax: m = B, n = vocab, k = d_model */
+  BT_K_TOKEN_STEP = 9,  /* fused token decoder + LM head + argmax: m = B, n = vocab, k = d_model */
+  BT_K_BLOCK_STEP = 10  /* the same kernel on a block step, block decoder and prefix included */
 };
 
 /* One timed kernel launch: kind, shape (GEMM: M, N, K; decode attention:

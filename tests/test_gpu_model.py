@@ -192,3 +192,41 @@ def test_fused_token_step_matches_oracle_and_chain(lb, B, monkeypatch):
         assert gh.rel_l2(gl[s], cl[s]) <= 1e-2, (s, gh.rel_l2(gl[s], cl[s]))
     # greedy ids are the argmax of the returned logits (lowest id on ties)
     assert np.array_equal(gn, gl.argmax(axis=-1))
+
+
+@pytest.mark.parametrize("lb,B", [(4, 5), (8, 64), (2, 33)])
+def test_fused_block_step_matches_oracle_and_chain(lb, B, monkeypatch):
+    """A block step (block decoder with decode attention over the block cache,
+    LN_b, the prefix projection, then the token decoder and the LM head) as
+    one persistent kernel (opt-in): one launch per block step, logits match
+    the oracle and agree with the kernel-per-operation block step."""
+    monkeypatch.setenv("BT_DECODE_BLOCK_STEP", "fused")
+    shape = synth.ModelShape(vocab=3000, d_model=256, n_heads=4, block_len=lb,
+                             n_block_layers=3, n_token_layers=2, prefix_len=1)
+    T, G = 12 * lb, 4 * lb + 3
+    w = synth.make_weights(shape, seed=41)
+    toks = synth.make_tokens(batch=B, length=T + G, vocab=shape.vocab, seed=42)
+    torch = gh.torch_mod()
+    m = gh.build_model(shape, w, B, T + G)
+    tok = torch.from_numpy(np.ascontiguousarray(toks)).cuda()
+    m.prefill(tok[:, :T].contiguous())
+    for i in range(lb - 1):  # token steps up to the last position of the block
+        m.decode(tok[:, T + i].contiguous())
+    m.sync()
+    k0 = _launches(m)
+    m.decode(tok[:, T + lb - 1].contiguous())  # completes the block
+    m.sync()
+    assert _launches(m) - k0 == 1
+    m.close()
+    m = gh.build_model(shape, w, B, T + G)
+    gl, gn = gh.gpu_teacher_forced(m, toks, T, G)
+    m.close()
+    monkeypatch.setenv("BT_DECODE_BLOCK_STEP", "chain")
+    m = gh.build_model(shape, w, B, T + G)
+    cl, cn = gh.gpu_teacher_forced(m, toks, T, G)
+    m.close()
+    ol = gh.oracle_teacher_forced(shape, w, toks, T, G)
+    for s in range(G):
+        assert gh.rel_l2(gl[s], ol[s]) <= BF16_REL, (s, gh.rel_l2(gl[s], ol[s]))
+        assert gh.rel_l2(gl[s], cl[s]) <= 1e-2, (s, gh.rel_l2(gl[s], cl[s]))
+    assert np.array_equal(gn, gl.argmax(axis=-1))
