@@ -288,6 +288,12 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+# DRAM bytes (read + write) per launch of the dominant kernel on this
+# workload, from the ncu capture summarised in
+# profiles/token_step_pythia160m_B64.md (the current token-step kernel)
+NCU_TRAFFIC_BYTES = {"token_step": 172.09e6}
+
+
 def profile_step(model, prompts, gens, flush):
     """One step with an event pair around every kernel; per-kind time shares
     and the roofline of the dominant kernel class."""
@@ -351,7 +357,7 @@ def profile_step(model, prompts, gens, flush):
                     "avg_launch_us": per * 1e6}
         ach = c["bytes"] / c["launches"] / per / 1e9
         return {"kernel": k, "bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s",
-                "frac": ach / hbm, "traffic": None, "launches": c["launches"],
+                "frac": ach / hbm, "traffic": NCU_TRAFFIC_BYTES.get(k), "launches": c["launches"],
                 "avg_launch_us": per * 1e6}
 
     out = {"dominant": roof(dom_name) if dom_name in ("gemm_decode", "gemm_prefill", "attn_decode", "token_step",
