@@ -39,7 +39,8 @@
 //
 // Grid barriers are a counter in global memory (release by a red.release
 // add, acquire by polling with ld.acquire). All CTAs must be resident at
-// once: one CTA per SM, grid = number of SMs. Every wait is bounded: a
+// once: one CTA per SM, grid = number of SMs, launched cooperatively so that
+// the driver guarantees it. Every wait is bounded: a
 // barrier that runs out sets ST_WAIT_TIMEOUT and an abort word that makes
 // every CTA skip the rest of the step; the producer then waits (bounded) for
 // its copies in flight, TMEM is freed and the kernel returns.
@@ -1401,11 +1402,15 @@ cudaError_t launch_token_step(const TokenStepArgs& a, const void* w_qkv1, const 
   cfg.blockDim = dim3(THREADS, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  // cooperative: the driver guarantees that every CTA is resident at once
+  // (the grid barriers rely on it) or refuses the launch
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  cfg.numAttrs = pdl_enabled() ? 2 : 1;
   if (a.block) e = cudaLaunchKernelEx(&cfg, token_step_kernel<true>, mq, mo, ml, mx1, ma2, mxf, mqb, mob, mp, a, P);
   else e = cudaLaunchKernelEx(&cfg, token_step_kernel<false>, mq, mo, ml, mx1, ma2, mxf, mqb, mob, mp, a, P);
   note_launch();
