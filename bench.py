@@ -467,6 +467,40 @@ def run_decode_case(args):
     model.close()
 
 
+def run_lb_sweep(args):
+    """The L_B sweep configurations (d_model 1024, 16 heads, 12 + 12 layers,
+    batch 128, prompt 2,048, 512 generated; L_B = 1 is the vanilla 24-layer
+    model without a token decoder, built from the same kernels): one untimed
+    generate run (graph capture), then one timed run each. One JSON line per
+    configuration; --case-steps > 0 shortens the generated length."""
+    import torch
+    from tests.gpu_helpers import build_model
+    torch.cuda.set_device(0)
+    for lb in (1, 2, 4, 8):
+        wl = synth.WORKLOADS[f"lb_sweep_L{lb}"]
+        model = build_model(wl.shape, synth.make_weights(wl), wl.batch, wl.max_seq)
+        toks = synth.make_tokens(wl)
+        prompt = torch.from_numpy(np.ascontiguousarray(toks[:, :wl.prompt_len])).cuda()
+        G = min(args.case_steps, wl.gen_len) if args.case_steps > 0 else wl.gen_len
+        out = torch.empty(G, wl.batch, dtype=torch.int32, device="cuda")
+        generate(model, prompt, G, out)
+        model.sync()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        generate(model, prompt, G, out)
+        b.record()
+        model.sync()
+        ms = a.elapsed_time(b)
+        print(json.dumps({"case": "lb_sweep", "workload": wl.name, "block_len": lb,
+                          "vanilla": not wl.shape.use_token_decoder, "batch": wl.batch,
+                          "prompt": wl.prompt_len, "generated": G, "ms": ms,
+                          "tokens_per_s": wl.batch * G / (ms / 1e3)}), flush=True)
+        model.close()
+        del model
+        torch.cuda.empty_cache()
+
+
 def run_kernel_case(args):
     """One op of the path through the op-level C-ABI, a few launches, for
     profiler captures: decode attention (B, H, d, n) or a dense projection
@@ -507,13 +541,21 @@ def main():
     ap.add_argument("--no-profile", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
-    ap.add_argument("--case", default=None, choices=["decode", "decode_attention", "linear"],
+    ap.add_argument("--case", default=None, choices=["decode", "decode_attention", "linear", "lb_sweep"],
                     help="instead of the benchmark, run a bounded case for profiler captures: decode "
                          "calls of the decode-heavy workload, or one op of the path")
-    ap.add_argument("--case-steps", type=int, default=8)
+    ap.add_argument("--case-steps", type=int, default=None,
+                    help="decode calls / launches of the case (default 8); lb_sweep: generated "
+                         "tokens (default: the configured 512)")
     ap.add_argument("--case-shape", default="128,16,64,640",
                     help="decode_attention: B,H,d,n; linear: M,N,K")
     args = ap.parse_args()
+    if args.case == "lb_sweep":
+        args.case_steps = args.case_steps or 0
+        run_lb_sweep(args)
+        return
+    if args.case is not None and args.case_steps is None:
+        args.case_steps = 8
     if args.case == "decode":
         run_decode_case(args)
         return
