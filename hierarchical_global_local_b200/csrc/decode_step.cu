@@ -1,6 +1,9 @@
 // decode_step.cu -- the token-decoder half of a decode step as one persistent
 // kernel (bf16, at most 64 sequences): every token-decoder layer, the final
-// LayerNorm, the LM head and the greedy argmax.
+// LayerNorm, the LM head and the greedy argmax. A second instance of the same
+// kernel (BLOCK = true, opt-in) runs a whole block step: the block embedding,
+// every block-decoder layer with its decode attention as a phase, LN_b and the
+// prefix projection, then the token-decoder program over the prefix row.
 //
 // Block Transformer (Ho et al., "Block Transformer: Global-to-Local Language
 // Modeling for Fast Inference"), section 2.3 (token decoder) and the Pythia
@@ -37,13 +40,22 @@
 // The MMA orientation is "weights as A": M = 128 output features per tile,
 // N = the batch padded to a multiple of 16, K in 64-wide swizzled blocks.
 //
+// Block-step phases before the token-decoder program (BLOCK = true):
+//   I_b (row b per CTA)  block row = the L_B token embeddings of the completed
+//                        block; LN1 | LN2 of block layer 0 -> x1
+//   per block layer: G1, then A (decode attention over the block cache, see
+//   block_attention_phase; GELU(fc1) -> a2), G2, then R2 into the block
+//   residual rows with the next block layer's LayerNorms or LN_b -> xf
+//   Gp / Rp              prefix projection W_p xf + b_p -> the token rows,
+//                        LN1 | LN2 of token layer 0 -> x1
+//
 // Grid barriers are a counter in global memory (release by a red.release
 // add, acquire by polling with ld.acquire). All CTAs must be resident at
 // once: one CTA per SM, grid = number of SMs, launched cooperatively so that
-// the driver guarantees it. Every wait is bounded: a
-// barrier that runs out sets ST_WAIT_TIMEOUT and an abort word that makes
-// every CTA skip the rest of the step; the producer then waits (bounded) for
-// its copies in flight, TMEM is freed and the kernel returns.
+// the driver guarantees it. Every wait is bounded: a barrier that runs out
+// sets ST_WAIT_TIMEOUT and an abort word that makes every CTA skip the rest
+// of the step; the producer then waits (bounded) for its copies in flight,
+// TMEM is freed and the kernel returns.
 #include <cuda.h>
 #include <float.h>
 #include <limits.h>
@@ -60,14 +72,11 @@ constexpr int WORKERS = 128;                 // warps 0-3 (TMEM lanes 0-127)
 constexpr int THREADS = WORKERS + 64;        // warp 4: TMA producer, warp 5: MMA issuer
 constexpr int TILE_BYTES = 128 * 64 * 2;     // one weight box: 128 rows x 64 K (bf16)
 constexpr int MAX_STAGES = 12;
-#ifndef TS_MAX_S1
-#define TS_MAX_S1 2
-#endif
-#ifndef TS_MAX_S2
-#define TS_MAX_S2 12
-#endif
-constexpr int MAX_S1 = TS_MAX_S1;            // K splits of the q|k|v|fc1 GEMM
-constexpr int MAX_S2 = TS_MAX_S2;            // K splits of the [W_o | W_2] GEMM
+// K splits: as many as fill the SMs up to these caps (fewer splits mean
+// fewer partial sums for the reduction phases; measured on B200 at D = 768:
+// 2 and 12 beat 3 / 15 and 1 / 12)
+constexpr int MAX_S1 = 2;                    // K splits of the q|k|v|fc1 GEMM
+constexpr int MAX_S2 = 12;                   // K splits of the [W_o | W_2] GEMM
 constexpr int MAX_B = 64;
 constexpr int MAX_WIN = 8;                   // local-window slots (P + L_B - 1)
 constexpr int TMEM_COLS = 128;               // two accumulators of up to 64 columns
@@ -81,12 +90,8 @@ constexpr int ATT_BYTES = 4 * ATT_SLOTS * ATT_SLOT_BYTES;        // 96 KB
 constexpr int ATT_PART = 68;                                     // m, l, o[64], pad
 constexpr int ATT_MAX_CHUNKS = 32;                               // n_cap <= 1024
 constexpr long long BAR_CYCLES = 2000000000LL;  // ~1 s at 1.9 GHz
-#ifndef PRODUCER_SLEEP_NS
-#define PRODUCER_SLEEP_NS 128  // back-off of the weight producer's slot waits
-#endif
-#ifndef MMA_SLEEP_NS
-#define MMA_SLEEP_NS 32        // back-off of the MMA warp's waits (on the critical path)
-#endif
+constexpr int PRODUCER_SLEEP_NS = 128;  // back-off of the weight producer's slot waits
+constexpr int MMA_SLEEP_NS = 32;        // back-off of the MMA warp's waits (on the critical path)
 
 struct Plan {
   int Bp;            // batch padded to a multiple of 16 (MMA N)

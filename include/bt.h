@@ -152,7 +152,14 @@ BT_API int bt_prefill(bt_model *m, const int32_t *tokens_dev, int32_t batch,
  * new token-decoder block starts from its context; otherwise the token
  * decoder appends one row to the block's local cache.
  * Errors: BT_ESTATE before a prefill, BT_ECAPACITY when t + 1 would exceed
- * max_seq. */
+ * max_seq.
+ * Execution: each call is one CUDA-graph replay on the model's stream. For
+ * bf16 models with batch <= 64 and prefix length 1 the token-decoder half of
+ * the step (all token-decoder layers, the LM head, the argmax) is a single
+ * persistent kernel launched cooperatively with one CTA on every SM: it
+ * waits for SMs held by other work on the device, and the driver refuses it
+ * if the device cannot hold one CTA per SM (the call then returns
+ * BT_ECUDA). */
 BT_API int bt_decode_step(bt_model *m, const int32_t *tokens_dev, float *logits_dev,
                    int32_t *next_tokens_dev);
 
