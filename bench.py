@@ -419,20 +419,23 @@ def cpu_baseline(budget_s: float = 20.0):
         t_total += dt
         parts.append(f"{r}: 1 sequence, prompt {x.prompt_len}, {g} of {x.gen_len} tokens, {dt:.1f}s")
     return {"value": gen_total / t_total, "unit": UNIT, "cores": _threads(), "kind": "oracle",
-            "sample": "; ".join(parts)}
+            "sample": "; ".join(parts), "seconds": t_total}
 
 
 def run_reference(args):
     ws, rank, _ = _dist()
     if rank != 0:
         return
+    # each step: a bounded sample of the workload (--ref-seconds over all steps)
     per_step = []
+    budget = max(2.0, args.ref_seconds / max(1, args.warmup + args.steps))
     for _ in range(args.warmup + args.steps):
-        per_step.append(cpu_baseline(budget_s=max(5.0, 60.0 / (args.warmup + args.steps))))
+        per_step.append(cpu_baseline(budget_s=budget))
     timed = per_step[args.warmup:]
     v = statistics.mean(s["value"] for s in timed)
+    ms = 1e3 * statistics.mean(s["seconds"] for s in timed)
     line = {"metric": METRIC, "value": v, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
-            "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
             "config": {"workload": "pythia160m-scale Block Transformer L_B=4 6+6 layers P=1: "
                                    "prefill-heavy B64 2048/128 + decode-heavy B64 128/2048",
@@ -540,7 +543,10 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-profile", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
-    ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    ap.add_argument("--cpu-seconds", type=float, default=20.0,
+                    help="time budget of the cpu_baseline leg of our arm")
+    ap.add_argument("--ref-seconds", type=float, default=60.0,
+                    help="--impl reference: oracle time budget over all warm-up and timed steps")
     ap.add_argument("--case", default=None, choices=["decode", "decode_attention", "linear", "lb_sweep"],
                     help="instead of the benchmark, run a bounded case for profiler captures: decode "
                          "calls of the decode-heavy workload, or one op of the path")
