@@ -72,3 +72,15 @@ def test_strerror_names_every_code(native):
     for code in range(0, -8, -1):
         s = L.bt_strerror(code).decode()
         assert s and s != "unknown status"
+
+
+def test_workspace_bytes_deterministic_and_monotone(native):
+    """The workspace size is a pure function of the configuration (no device
+    query) and grows with the batch and sequence capacity."""
+    from tests.gpu_helpers import model_config
+    wl = synth.WORKLOADS["pythia160m_decode_heavy"]
+    base = native.workspace_bytes(model_config(wl.shape, wl.batch, wl.max_seq))
+    assert base == native.workspace_bytes(model_config(wl.shape, wl.batch, wl.max_seq))
+    assert native.workspace_bytes(model_config(wl.shape, wl.batch + 1, wl.max_seq)) > base
+    assert native.workspace_bytes(model_config(wl.shape, wl.batch, wl.max_seq + 4 * 64)) > base
+    assert native.workspace_bytes(model_config(wl.shape, 1, wl.max_seq)) < base
