@@ -136,7 +136,7 @@ def job_throughput(tokens_per_rank_step: int, steps: int, world: int, max_ms: fl
 
 def build(rank: int):
     import torch
-    from tests.gpu_helpers import build_model
+    from hierarchical_global_local_b200.loader import build_model
     wl = synth.WORKLOADS[RUNS[0]]
     w = synth.make_weights(wl)
     max_seq = max(synth.WORKLOADS[r].max_seq for r in RUNS)
@@ -288,10 +288,30 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
-# DRAM bytes (read + write) per launch of the dominant kernel on this
-# workload, from the ncu capture summarised in
-# profiles/token_step_pythia160m_B64.md (the current token-step kernel)
-NCU_TRAFFIC_BYTES = {"token_step": 172.09e6}
+# DRAM bytes (read + write) per launch of a kernel class on this workload,
+# measured by an ncu capture, with the SHA-256 prefix of the kernel's source
+# file at the time of the capture. The bench reports the figure only while
+# the source is unchanged; after a change the traffic is null until it is
+# captured again.
+NCU_TRAFFIC = {
+    "token_step": {"bytes": 172.09e6, "source": "hierarchical_global_local_b200/csrc/decode_step.cu",
+                   "sha16": "fa7b915618c4d566"},
+}
+
+
+def ncu_traffic(kind: str):
+    """Measured DRAM bytes per launch of `kind`, or None when there is no
+    capture of the current kernel source."""
+    import hashlib
+    e = NCU_TRAFFIC.get(kind)
+    if not e:
+        return None
+    try:
+        with open(os.path.join(ROOT, e["source"]), "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()[:16]
+    except OSError:
+        return None
+    return e["bytes"] if sha == e["sha16"] else None
 
 
 def profile_step(model, prompts, gens, flush):
@@ -357,7 +377,7 @@ def profile_step(model, prompts, gens, flush):
                     "avg_launch_us": per * 1e6}
         ach = c["bytes"] / c["launches"] / per / 1e9
         return {"kernel": k, "bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s",
-                "frac": ach / hbm, "traffic": NCU_TRAFFIC_BYTES.get(k), "launches": c["launches"],
+                "frac": ach / hbm, "traffic": ncu_traffic(k), "launches": c["launches"],
                 "avg_launch_us": per * 1e6}
 
     out = {"dominant": roof(dom_name) if dom_name in ("gemm_decode", "gemm_prefill", "attn_decode", "token_step",
@@ -477,7 +497,7 @@ def run_lb_sweep(args):
     generate run (graph capture), then one timed run each. One JSON line per
     configuration; --case-steps > 0 shortens the generated length."""
     import torch
-    from tests.gpu_helpers import build_model
+    from hierarchical_global_local_b200.loader import build_model
     torch.cuda.set_device(0)
     for lb in (1, 2, 4, 8):
         wl = synth.WORKLOADS[f"lb_sweep_L{lb}"]
@@ -534,6 +554,18 @@ def run_kernel_case(args):
     print(json.dumps({"case": args.case, "shape": dims, "launches": args.case_steps}), flush=True)
 
 
+def relaunch_distributed(n: int):
+    """One process per GPU: run this script again under torch.distributed.run
+    with n ranks on this node (rendezvous on 127.0.0.1)."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__)] + sys.argv[1:]
+    os.execv(sys.executable, cmd)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -556,6 +588,11 @@ def main():
     ap.add_argument("--case-shape", default="128,16,64,640",
                     help="decode_attention: B,H,d,n; linear: M,N,K")
     args = ap.parse_args()
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ and args.case is None:
+        relaunch_distributed(args.gpus)
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    if ws != args.gpus and args.case is None:
+        print(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={ws}; timing {ws} rank(s)", file=sys.stderr)
     if args.case == "lb_sweep":
         args.case_steps = args.case_steps or 0
         run_lb_sweep(args)

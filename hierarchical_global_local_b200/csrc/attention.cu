@@ -43,7 +43,7 @@ struct DecCfg {
   static_assert(DH <= CWARPS * 32, "one thread per output dim in the final reduction");
 };
 
-constexpr int DEC_UNITS_SLACK = 4096;  // work units beyond one per pair (scratch sizing)
+constexpr int DEC_UNITS_SLACK = ATTN_DECODE_MAX_CTAS;  // partial slots in the scratch (grid cap)
 
 __device__ __forceinline__ float block_reduce_max128(float v, float* red) {
   v = warp_max(v);
@@ -253,16 +253,7 @@ attn_decode_kernel(const T* __restrict__ q, int ldq, const T* __restrict__ kc,
   }
 }
 
-static int dec_sm_count() {
-  static int n = 0;
-  if (!n) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
-  }
-  return n;
-}
+static int dec_sm_count() { return device_sm_count(); }
 
 template <typename T>
 static int dec_chunk(int d) {
@@ -284,18 +275,19 @@ int attn_decode_max_splits(int d, int cap, int dt) { return dec_grid(1, d, cap, 
 // scratch layout: [merge counters: B*H ints, 256-aligned][partials: two
 // slots of (d + 2) floats per CTA of the grid]; counters sit at offset 0.
 size_t attn_decode_scratch_bytes(int B, int H, int d, int cap, int dt) {
-  const size_t cnt = ((size_t)B * H * sizeof(int) + 255) & ~(size_t)255;
-  return cnt + (size_t)2 * DEC_UNITS_SLACK * (d + 2) * sizeof(float);
+  return attn_decode_scratch_bytes_for((long long)B * H, d);
 }
 
 template <typename T, int DH>
 static cudaError_t dec_prepare() {
-  static bool done = false;
-  if (done) return cudaSuccess;
+  // the attribute applies to the current device only
+  static bool done[MAX_DEVICES] = {};
+  const int dev = current_device();
+  if (dev >= 0 && done[dev]) return cudaSuccess;
   cudaError_t e = cudaFuncSetAttribute(attn_decode_kernel<T, DH>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        DecCfg<T, DH>::SMEM);
-  if (e == cudaSuccess) done = true;
+  if (e == cudaSuccess && dev >= 0) done[dev] = true;
   return e;
 }
 

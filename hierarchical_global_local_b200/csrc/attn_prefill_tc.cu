@@ -22,6 +22,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "tc.cuh"
 
 namespace bt {
 
@@ -30,61 +31,6 @@ namespace {
 constexpr int QT = 128;   // queries per CTA (MMA M)
 constexpr int KT = 128;   // keys per tile (MMA N of S, K of P V)
 constexpr int THREADS = 192;
-
-__device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr) {
-  uint64_t d = 0;
-  d |= (uint64_t)((saddr & 0x3FFFF) >> 4);
-  d |= (uint64_t)(16 >> 4) << 16;
-  d |= (uint64_t)(1024 >> 4) << 32;
-  d |= (uint64_t)1 << 46;
-  d |= (uint64_t)2 << 61;
-  return d;
-}
-
-__device__ __forceinline__ constexpr uint32_t idesc_bf16(int N) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(QT >> 4) << 24);
-}
-
-__device__ __forceinline__ void mma(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
-  asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d),
-      "l"(a), "l"(b), "r"(idesc), "r"(acc));
-}
-
-__device__ __forceinline__ void commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   smem_u32(bar))
-               : "memory");
-}
-
-__device__ __forceinline__ void tma3(void* dst, const CUtensorMap* m, int x, int y, int z, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
-      "%4, %5}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
-      : "memory");
-}
-
-__device__ __forceinline__ void ld32(uint32_t taddr, float* v) {
-  uint32_t r[32];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
-      "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
-      "%30, %31}, [%32];\n"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
-        "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
-        "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
-
-__device__ __forceinline__ void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
 // shared memory plan (bytes), all tiles 1024-aligned
 template <int DH>
@@ -135,14 +81,11 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
     fence_mbar_init();
   }
   if (warp == 0) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_u32(&tmem_slot)),
-                 "r"(PL::TMEM_COLS));
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    tc::tmem_alloc(&tmem_slot, PL::TMEM_COLS);
   }
-  fence_before();
+  tc::fence_before();
   __syncthreads();
-  fence_after();
+  tc::fence_after();
   const uint32_t tmem = tmem_slot;
   const uint32_t tS = tmem, tO = tmem + KT;
   pdl_wait();
@@ -152,47 +95,47 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
       // Q tile (KB blocks of 64 dims), then K / V^T tiles through the ring
       mbar_arrive_expect_tx(&q_full, PL::Q_BYTES);
       for (int kb = 0; kb < PL::KB; ++kb)
-        tma3(sm + PL::OFF_Q + kb * QT * 128, &mQ, h * DH + kb * 64, q0, b, &q_full);
+        tc::tma_load_3d(sm + PL::OFF_Q + kb * QT * 128, &mQ, h * DH + kb * 64, q0, b, &q_full);
       for (int j = 0; j < ntiles; ++j) {
         const int s = j % PL::STAGES;
         if (j >= PL::STAGES) mbar_wait_bounded(&kv_empty[s], ((j / PL::STAGES) + 1) & 1, status);
         mbar_arrive_expect_tx(&kv_full[s], PL::K_BYTES + PL::VT_BYTES);
         for (int kb = 0; kb < PL::KB; ++kb)
-          tma3(sm + PL::OFF_K + s * PL::K_BYTES + kb * KT * 128, &mK, kb * 64, j * KT, bh, &kv_full[s]);
+          tc::tma_load_3d(sm + PL::OFF_K + s * PL::K_BYTES + kb * KT * 128, &mK, kb * 64, j * KT, bh, &kv_full[s]);
         for (int kb = 0; kb < KT / 64; ++kb)
-          tma3(sm + PL::OFF_VT + s * PL::VT_BYTES + kb * DH * 128, &mVt, j * KT + kb * 64, 0, bh,
+          tc::tma_load_3d(sm + PL::OFF_VT + s * PL::VT_BYTES + kb * DH * 128, &mVt, j * KT + kb * 64, 0, bh,
                &kv_full[s]);
       }
     }
   } else if (warp == 5) {
     if (lane == 0) {
-      constexpr uint32_t idS = idesc_bf16(KT), idO = idesc_bf16(DH);
+      constexpr uint32_t idS = tc::idesc_bf16_m128(KT), idO = tc::idesc_bf16_m128(DH);
       mbar_wait_bounded(&q_full, 0, status);
       for (int j = 0; j < ntiles; ++j) {
         const int s = j % PL::STAGES;
         // (S of tile j-1 was consumed before P of tile j-1 was published,
         // which this thread waited for before the previous P V)
         mbar_wait_bounded(&kv_full[s], (j / PL::STAGES) & 1, status);
-        fence_after();
+        tc::fence_after();
         // S = Q K^T over DH (KB blocks x 4 slices of 16)
         for (int kb = 0; kb < PL::KB; ++kb) {
-          const uint64_t dq = desc_sw128(smem_u32(sm + PL::OFF_Q + kb * QT * 128));
-          const uint64_t dk = desc_sw128(smem_u32(sm + PL::OFF_K + s * PL::K_BYTES + kb * KT * 128));
+          const uint64_t dq = tc::desc_sw128(smem_u32(sm + PL::OFF_Q + kb * QT * 128));
+          const uint64_t dk = tc::desc_sw128(smem_u32(sm + PL::OFF_K + s * PL::K_BYTES + kb * KT * 128));
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) mma(tS, dq + 2 * kk, dk + 2 * kk, idS, (kb | kk) ? 1u : 0u);
+          for (int kk = 0; kk < 4; ++kk) tc::mma_bf16(tS, dq + 2 * kk, dk + 2 * kk, idS, (kb | kk) ? 1u : 0u);
         }
-        commit(&s_full);
+        tc::commit(&s_full);
         // O_j = P V over the 128 keys (2 blocks x 4 slices of 16), once P is written
         mbar_wait_bounded(&p_full, j & 1, status);
-        fence_after();
+        tc::fence_after();
         for (int kb = 0; kb < KT / 64; ++kb) {
-          const uint64_t dp = desc_sw128(smem_u32(sm + PL::OFF_P + kb * QT * 128));
-          const uint64_t dv = desc_sw128(smem_u32(sm + PL::OFF_VT + s * PL::VT_BYTES + kb * DH * 128));
+          const uint64_t dp = tc::desc_sw128(smem_u32(sm + PL::OFF_P + kb * QT * 128));
+          const uint64_t dv = tc::desc_sw128(smem_u32(sm + PL::OFF_VT + s * PL::VT_BYTES + kb * DH * 128));
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) mma(tO, dp + 2 * kk, dv + 2 * kk, idO, (kb | kk) ? 1u : 0u);
+          for (int kk = 0; kk < 4; ++kk) tc::mma_bf16(tO, dp + 2 * kk, dv + 2 * kk, idO, (kb | kk) ? 1u : 0u);
         }
-        commit(&o_full);
-        commit(&kv_empty[s]);
+        tc::commit(&o_full);
+        tc::commit(&kv_empty[s]);
       }
     }
   } else {
@@ -207,14 +150,14 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
     uint8_t* prow = sm + PL::OFF_P;
     for (int j = 0; j < ntiles; ++j) {
       mbar_wait_bounded(&s_full, j & 1, status);
-      fence_after();
+      tc::fence_after();
       const int k0 = j * KT;
       // pass 1: row max over this tile (masked keys excluded), 32 columns at a time
       float tmax = -INFINITY;
 #pragma unroll
       for (int c = 0; c < KT; c += 32) {
         float sv[32];
-        ld32(tS + lane_base + c, sv);
+        tc::tmem_ld32(tS + lane_base + c, sv);
 #pragma unroll
         for (int u = 0; u < 32; ++u) {
           const int kj = k0 + c + u;
@@ -228,7 +171,7 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
 #pragma unroll
       for (int c = 0; c < KT; c += 32) {
         float sv[32];
-        ld32(tS + lane_base + c, sv);
+        tc::tmem_ld32(tS + lane_base + c, sv);
 #pragma unroll
         for (int c8 = 0; c8 < 4; ++c8) {
           float p[8];
@@ -250,15 +193,15 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
         }
       }
       fence_proxy_async();  // P visible to the tensor core
-      fence_before();
+      tc::fence_before();
       mbar_arrive(&p_full);
       // accumulate O_j with the rescale
       mbar_wait_bounded(&o_full, j & 1, status);
-      fence_after();
+      tc::fence_after();
 #pragma unroll
       for (int c = 0; c < DH; c += 32) {
         float ov[32];
-        ld32(tO + lane_base + c, ov);
+        tc::tmem_ld32(tO + lane_base + c, ov);
 #pragma unroll
         for (int u = 0; u < 32; ++u) o[c + u] = o[c + u] * corr + ov[u];
       }
@@ -281,11 +224,10 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
       }
     }
   }
-  fence_before();
+  tc::fence_before();
   __syncthreads();
   if (warp == 0)
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
-                 "r"(PL::TMEM_COLS));
+    tc::tmem_free(tmem, PL::TMEM_COLS);
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -324,12 +266,14 @@ bool map3(CUtensorMap* m, const void* base, long long x, long long y, long long 
 template <int DH>
 cudaError_t launch_tc(const void* q, int ldq, const void* kc, const void* vt, int vt_ld, int B,
                       int H, int cap, int n, void* out, int ld_out, int* status, cudaStream_t s) {
-  static bool prepared = false;
-  if (!prepared) {
+  // the attribute applies to the current device only
+  static bool prepared[MAX_DEVICES] = {};
+  const int dev = current_device();
+  if (dev < 0 || !prepared[dev]) {
     cudaError_t e = cudaFuncSetAttribute(attn_prefill_tc_kernel<DH>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, Plan<DH>::BYTES);
     if (e != cudaSuccess) return e;
-    prepared = true;
+    if (dev >= 0) prepared[dev] = true;
   }
   CUtensorMap mQ, mK, mVt;
   // Q rows b*n + i, dims (h*d + e): {ldq cols, n rows, B}

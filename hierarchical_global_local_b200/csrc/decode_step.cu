@@ -1259,13 +1259,16 @@ struct Device {
   bool ready = false;
 };
 
+// per device: kernel attributes apply to the current device only
 Device& device() {
-  static Device d;
+  static Device per_dev[MAX_DEVICES];
+  static Device none;
+  const int dev = current_device();
+  Device& d = dev >= 0 ? per_dev[dev] : none;
   if (!d.ready) {
-    int dev = 0, optin = 0;
+    int optin = 0;
     cudaFuncAttributes fa;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+    if (dev < 0 || cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
         cudaFuncGetAttributes(&fa, token_step_kernel<true>) != cudaSuccess)
       return d;

@@ -28,6 +28,7 @@
 #include "common.cuh"
 #include "epilogue.cuh"
 #include "kernels.h"
+#include "tc.cuh"
 
 namespace bt {
 
@@ -36,80 +37,6 @@ namespace {
 constexpr int BM = 128;  // MMA M (TMEM lanes)
 constexpr int BK = 64;   // K elements per stage = one 128-byte swizzle row
 constexpr size_t PART_BUDGET = 256;  // split-K reduces in distributed shared memory
-
-// ---- tcgen05 / TMA wrappers --------------------------------------------------
-__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
-  // K-major, 128-byte swizzle: rows of 128 B, 8-row groups 1024 B apart.
-  uint64_t d = 0;
-  d |= (uint64_t)((saddr & 0x3FFFF) >> 4);          // start address
-  d |= (uint64_t)(16 >> 4) << 16;                   // leading byte offset (unused)
-  d |= (uint64_t)(1024 >> 4) << 32;                 // stride byte offset
-  d |= (uint64_t)1 << 46;                           // descriptor version
-  d |= (uint64_t)2 << 61;                           // SWIZZLE_128B
-  return d;
-}
-
-template <int BN>
-__device__ __forceinline__ constexpr uint32_t instr_desc() {
-  // kind::f16: D fp32, A bf16, B bf16, both K-major, M = 128, N = BN.
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
-         ((uint32_t)(BM >> 4) << 24);
-}
-
-__device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc,
-                                         uint32_t accum) {
-  asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
-      "l"(a), "l"(b), "r"(idesc), "r"(accum));
-}
-
-__device__ __forceinline__ void mma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   smem_u32(bar))
-               : "memory");
-}
-
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
-                                            uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
-      "%4}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
-      : "memory");
-}
-
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
-  uint32_t r[16];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
-      "%12, %13, %14, %15}, [%16];\n"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
-}
-
-// cluster barrier halves (per thread, not warp-aligned)
-__device__ __forceinline__ void cluster_arrive_relaxed() {
-  asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_arrive_release() {
-  asm volatile("barrier.cluster.arrive.release;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_wait_acquire() {
-  asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
 
 constexpr int MAX_STAGES = 8;
 constexpr int THREADS = 192;  // warps 0-3 epilogue, warp 4 TMA producer, warp 5 MMA issuer
@@ -249,18 +176,15 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
     fence_mbar_init();
   }
   if (warp == 0) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_u32(&tmem_slot)),
-                 "r"(tmem_cols<BN>()));
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    tc::tmem_alloc(&tmem_slot, tmem_cols<BN>());
   }
-  tc_fence_before();
+  tc::fence_before();
   __syncthreads();
-  tc_fence_after();
+  tc::fence_after();
   const uint32_t tmem = tmem_slot;
   // split K: announce that this CTA is running; peers wait on it before
   // their first store into this CTA's shared memory
-  if (ks > 1) cluster_arrive_relaxed();
+  if (ks > 1) tc::cluster_arrive_relaxed();
 
   pdl_trigger();
   if (warp == 4) {
@@ -281,14 +205,14 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
       auto load_w = [&](int it, int s) {  // the weight operand
         int a0, b0, k, koff;
         coords(it, a0, b0, k, koff);
-        if (SWAP) tma_load_2d(sA + (size_t)s * BM * BK, &mapA, k, a0, &full[s]);
-        else tma_load_2d(sB + (size_t)s * BN * BK, &mapB, k, b0, &full[s]);
+        if (SWAP) tc::tma_load_2d(sA + (size_t)s * BM * BK, &mapA, k, a0, &full[s]);
+        else tc::tma_load_2d(sB + (size_t)s * BN * BK, &mapB, k, b0, &full[s]);
       };
       auto load_x = [&](int it, int s) {  // the activation operand
         int a0, b0, k, koff;
         coords(it, a0, b0, k, koff);
-        if (SWAP) tma_load_2d(sB + (size_t)s * BN * BK, &mapB, k + koff, b0, &full[s]);
-        else tma_load_2d(sA + (size_t)s * BM * BK, &mapA, k + koff, a0, &full[s]);
+        if (SWAP) tc::tma_load_2d(sB + (size_t)s * BN * BK, &mapB, k + koff, b0, &full[s]);
+        else tc::tma_load_2d(sA + (size_t)s * BM * BK, &mapA, k + koff, a0, &full[s]);
       };
       // weights do not depend on earlier kernels: fill the first ring with
       // them while the previous kernel finishes, then wait for it
@@ -311,25 +235,25 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
     // ---- MMA issuer ----
     pdl_wait();
     if (lane == 0) {
-      constexpr uint32_t idesc = instr_desc<BN>();
+      constexpr uint32_t idesc = tc::idesc_bf16_m128(BN);
       int it = 0, tl = 0;
       for (int t = t_first; t < ntiles; t += t_step, ++tl) {
         const int buf = tl & 1;
         if (tl >= 2) mbar_wait_bounded(&acc_empty[buf], ((tl >> 1) + 1) & 1, status);
-        tc_fence_after();
+        tc::fence_after();
         const uint32_t dt = tmem + (uint32_t)(buf * BN);
         for (int kb = kb_begin; kb < kb_end; ++kb, ++it) {
           const int s = it % stages;
           mbar_wait_bounded(&full[s], (it / stages) & 1, status);
-          tc_fence_after();
-          const uint64_t da = smem_desc_sw128(smem_u32(sA + (size_t)s * BM * BK));
-          const uint64_t db = smem_desc_sw128(smem_u32(sB + (size_t)s * BN * BK));
+          tc::fence_after();
+          const uint64_t da = tc::desc_sw128(smem_u32(sA + (size_t)s * BM * BK));
+          const uint64_t db = tc::desc_sw128(smem_u32(sB + (size_t)s * BN * BK));
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)  // 32 bytes per K slice: +2 in 16-byte units
-            mma_bf16(dt, da + 2 * kk, db + 2 * kk, idesc, (kb > kb_begin || kk > 0) ? 1u : 0u);
-          mma_commit(&empty[s]);
+            tc::mma_bf16(dt, da + 2 * kk, db + 2 * kk, idesc, (kb > kb_begin || kk > 0) ? 1u : 0u);
+          tc::commit(&empty[s]);
         }
-        mma_commit(&acc_full[buf]);
+        tc::commit(&acc_full[buf]);
       }
     }
   } else {
@@ -346,7 +270,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
       const int buf = tl & 1;
       const int a0 = (t % ntA) * BM, b0 = (t / ntA) * BN;
       mbar_wait_bounded(&acc_full[buf], (tl >> 1) & 1, status);
-      tc_fence_after();
+      tc::fence_after();
       const uint32_t tb = trow + (uint32_t)(buf * BN);
       if (ks > 1) {
         // push this CTA's partial columns to their owners: column c goes to
@@ -357,10 +281,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
         float* recv = reinterpret_cast<float*>(smem + (size_t)stages * stage_bytes<BN>());
         const int cpr = BN / ks;
         const int me = (int)cluster.block_rank();
-        cluster_wait_acquire();  // every CTA of the cluster has started
+        tc::cluster_wait_acquire();  // every CTA of the cluster has started
         for (int c0 = 0; c0 < BN; c0 += 16) {
           float v[16];
-          tmem_ld16(tb + c0, v);
+          tc::tmem_ld16(tb + c0, v);
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int c = c0 + j;
@@ -375,7 +299,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
         float* logits = reinterpret_cast<float*>(e.out0);
         for (int c0 = 0; c0 < BN; c0 += 16) {
           float v[16];
-          tmem_ld16(tb + c0, v);
+          tc::tmem_ld16(tb + c0, v);
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int m = b0 + c0 + j;
@@ -391,7 +315,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
             if (lane == 0) s_arg[warp][c0 + j] = make_float2(bv, __int_as_float(bi));
           }
         }
-        tc_fence_before();
+        tc::fence_before();
         mbar_arrive(&acc_empty[buf]);
         asm volatile("bar.sync 1, 128;" ::: "memory");  // the four epilogue warps
         if (r < BN && b0 + r < M) {
@@ -409,8 +333,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
         // drain the whole accumulator first, release it, then store
         float v[BN];
 #pragma unroll
-        for (int c0 = 0; c0 < BN; c0 += 16) tmem_ld16(tb + c0, v + c0);
-        tc_fence_before();
+        for (int c0 = 0; c0 < BN; c0 += 16) tc::tmem_ld16(tb + c0, v + c0);
+        tc::fence_before();
         mbar_arrive(&acc_empty[buf]);
 #pragma unroll
         for (int c = 0; c < BN; ++c) {
@@ -431,8 +355,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
         float* tile = reinterpret_cast<float*>(smem + (size_t)stages * stage_bytes<BN>()) + warp * 32 * 33;
         for (int c0 = 0; c0 < BN; c0 += 32) {
           float v[32];
-          tmem_ld16(tb + c0, v);
-          tmem_ld16(tb + c0 + 16, v + 16);
+          tc::tmem_ld16(tb + c0, v);
+          tc::tmem_ld16(tb + c0 + 16, v + 16);
 #pragma unroll
           for (int j = 0; j < 32; ++j) tile[lane * 33 + j] = v[j];
           __syncwarp();
@@ -443,12 +367,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
           }
           __syncwarp();
         }
-        tc_fence_before();
+        tc::fence_before();
         mbar_arrive(&acc_empty[buf]);
       } else {
         for (int c0 = 0; c0 < BN; c0 += 16) {
           float v[16];
-          tmem_ld16(tb + c0, v);
+          tc::tmem_ld16(tb + c0, v);
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int m = SWAP ? (b0 + c0 + j) : (a0 + r);
@@ -461,7 +385,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
             }
           }
         }
-        tc_fence_before();
+        tc::fence_before();
         mbar_arrive(&acc_empty[buf]);
         if (SWAP && e.ln_cnt) post_ln(e, b0, b0 + BN, M, N, ntA, s_rows, &s_nrows);
       }
@@ -476,9 +400,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
     // memory after the barrier, so no second barrier is needed.
     namespace cg = cooperative_groups;
     cg::cluster_group cluster = cg::this_cluster();
-    if (warp >= 4) cluster_wait_acquire();  // producer / MMA warps: first phase
-    cluster_arrive_release();               // second phase: all pushes done
-    cluster_wait_acquire();
+    if (warp >= 4) tc::cluster_wait_acquire();  // producer / MMA warps: first phase
+    tc::cluster_arrive_release();               // second phase: all pushes done
+    tc::cluster_wait_acquire();
     if (warp < 4) {
       const int r = warp * 32 + lane;
       const bool rope = SWAP && e.kind == EPI_QKV1_ROPE;
@@ -504,11 +428,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
     }
   }
 
-  tc_fence_before();
+  tc::fence_before();
   __syncthreads();
   if (warp == 0)
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
-                 "r"(tmem_cols<BN>()));
+    tc::tmem_free(tmem, tmem_cols<BN>());
 }
 
 // ---- host side -------------------------------------------------------------------
@@ -567,16 +490,7 @@ cudaError_t prepare_one() {
   return e;
 }
 
-int sm_count() {
-  static int n = 0;
-  if (!n) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
-  }
-  return n;
-}
+int sm_count() { return device_sm_count(); }
 
 template <int BN, bool SWAP>
 cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& mb, int M, int N, int nkb,
@@ -645,16 +559,17 @@ int swap_bn(int M) {
 }  // namespace
 
 cudaError_t gemm_tc_prepare() {
-  static bool done = false;
-  if (done) return cudaSuccess;
+  // kernel attributes apply to the current device only
+  static bool done[MAX_DEVICES] = {};
+  const int dev = current_device();
+  if (dev >= 0 && done[dev]) return cudaSuccess;
   cudaError_t e;
   if ((e = prepare_one<32, true>()) != cudaSuccess) return e;
   if ((e = prepare_one<64, true>()) != cudaSuccess) return e;
   if ((e = prepare_one<128, true>()) != cudaSuccess) return e;
   if ((e = prepare_one<256, true>()) != cudaSuccess) return e;
   if ((e = prepare_one<256, false>()) != cudaSuccess) return e;
-  sm_count();
-  done = true;
+  if (dev >= 0) done[dev] = true;
   return cudaSuccess;
 }
 

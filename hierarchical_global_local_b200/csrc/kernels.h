@@ -13,6 +13,17 @@ namespace bt {
 enum DType : int { DT_F32 = 0, DT_BF16 = 1 };
 inline size_t dt_size(int dt) { return dt == DT_F32 ? 4 : 2; }
 
+// ---- per-device one-time state ---------------------------------------------
+// Kernel attributes (cudaFuncSetAttribute) and device properties apply to the
+// device that is current when they are set or read, so one-time set-up is
+// kept per device.
+constexpr int MAX_DEVICES = 64;
+// Index of the current device, or -1 if it cannot be read or is >= MAX_DEVICES
+// (callers then redo their set-up on every call instead of caching it).
+int current_device();
+// Multiprocessor count of the current device (148 if it cannot be read).
+int device_sm_count();
+
 // ---- embedder / token ingest / step state --------------------------------
 // Prompt embedder: h[b*n + i, :] = concat_j blk_emb[tokens[b, i*L_B + j]].
 cudaError_t launch_embed_prompt(int dt, const int32_t* tokens, int B, int T, int L_B,
@@ -64,6 +75,14 @@ cudaError_t launch_rope_table(float2* tab, int n_pos, int rot, float base, cudaS
 // part / counters: scratch of attn_decode_scratch_bytes(); counters must be
 // zero before the first launch and are left zero.
 size_t attn_decode_scratch_bytes(int B, int H, int d, int cap, int dt);
+// The scratch layout behind it: merge counters for `pairs` (sequence, head)
+// pairs (padded to 256 bytes), then two partial slots of (d + 2) floats for
+// each of at most ATTN_DECODE_MAX_CTAS persistent CTAs.
+constexpr int ATTN_DECODE_MAX_CTAS = 4096;
+constexpr size_t attn_decode_scratch_bytes_for(long long pairs, int d) {
+  return (((size_t)pairs * sizeof(int) + 255) & ~(size_t)255) +
+         (size_t)2 * ATTN_DECODE_MAX_CTAS * (size_t)(d + 2) * sizeof(float);
+}
 // One-time setup of the decode-attention kernels (shared-memory limits).
 cudaError_t attn_prepare();
 int attn_decode_max_splits(int d, int cap, int dt);

@@ -24,7 +24,9 @@ namespace {
 // and d_head <= 128. Size: 8192 merge counters + the split partials, ~4.3 MB.
 constexpr int NOALLOC_MAX_PAIRS = 8192;
 constexpr int NOALLOC_MAX_D = 128;
-constexpr size_t NOALLOC_BYTES = 4456448;  // >= the scratch bytes of the largest problem
+constexpr size_t NOALLOC_BYTES = attn_decode_scratch_bytes_for(NOALLOC_MAX_PAIRS, NOALLOC_MAX_D);
+static_assert(NOALLOC_BYTES % 256 == 0 && NOALLOC_BYTES < (8u << 20),
+              "the fixed array covers the largest problem within the limits and stays modest");
 
 // Shared by every call on a device and kept between calls; every GPU that
 // loads the library holds it until the process exits.
