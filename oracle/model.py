@@ -29,6 +29,12 @@ Readings where the page is silent (each listed again in the design notes):
       pairing i <-> i + r/2, inv_freq_i = base^(-2i/r), base 10000),
       exact-erf GELU, 4x MLP, scores scaled by 1/sqrt(d_head), untied LM
       head without bias, no embedding norm.
+  R7  Inference left padding adds p = (-T) mod L_B pad tokens before the
+      prompt (at most L_B - 1, so that the prompt ends on a block boundary);
+      the pad id is the caller's choice.
+  R8  A prompt whose length is not a multiple of L_B without padding: its
+      trailing T mod L_B tokens form the incomplete current block and enter
+      the token decoder (the model's own definition of those positions).
 
 Pins (tests/test_oracle_*.py): HF GPTNeoX (an independent Pythia
 implementation) for the layer stack and the vanilla special case;
@@ -47,7 +53,7 @@ from scipy.special import erf
 
 __all__ = [
     "layer_norm", "gelu", "rotary", "attend", "pythia_layer", "embed_blocks",
-    "prefix_projection", "BlockTransformerOracle",
+    "prefix_projection", "left_pad", "BlockTransformerOracle", "ragged_generate_logits",
 ]
 
 
@@ -181,6 +187,18 @@ def prefix_projection(c: np.ndarray, w: np.ndarray, b: np.ndarray, P: int) -> np
     return out.reshape(*c.shape[:-1], P, D)
 
 
+def left_pad(tokens: np.ndarray, block_len: int, pad_id: int) -> np.ndarray:
+    """Inference left padding ([BT] §3.4 "The Embedder", prompts whose length
+    is not a multiple of L_B [orig. §2.2, App. H]): the first block is padded
+    on the left with pad tokens so that the prompt ends on a block boundary.
+
+    tokens: [T] -> [T + p], p = (-T) mod L_B in [0, L_B - 1] (reading R7).
+    """
+    tokens = np.asarray(tokens)
+    p = (-tokens.shape[0]) % block_len
+    return np.concatenate([np.full(p, pad_id, dtype=tokens.dtype), tokens])
+
+
 # --------------------------------------------------------------------------
 # the model
 # --------------------------------------------------------------------------
@@ -310,35 +328,46 @@ class OracleSession:
     def _token_rows(self, rows: np.ndarray, pos: np.ndarray) -> np.ndarray:
         return self.m.token_decoder(rows, pos, self.token_caches)
 
-    def _start_block(self, c: np.ndarray) -> np.ndarray:
-        """New token-decoder block: reset local KV, feed the P prefix rows;
-        return logits predicting the block's first token (row P-1)."""
+    def _start_block(self, c: np.ndarray, trailing: Optional[np.ndarray] = None) -> np.ndarray:
+        """New token-decoder block: reset local KV, feed the P prefix rows and
+        the tokens of the block already known (``trailing`` [B, r], r < L_B,
+        at local positions P..P+r-1); return logits of the last row fed,
+        which predict token r of the block."""
         s, m = self.s, self.m
         self.token_caches = m._fresh(m.token_layers)
-        pre = prefix_projection(c, m.g["w_prefix"], m.g["b_prefix"], s.prefix_len)
-        z = self._token_rows(pre, np.arange(s.prefix_len))
-        return z[:, s.prefix_len - 1]
+        rows = prefix_projection(c, m.g["w_prefix"], m.g["b_prefix"], s.prefix_len)
+        if trailing is not None and trailing.shape[1] > 0:
+            rows = np.concatenate([rows, m.g["tok_emb"][trailing]], axis=1)
+        z = self._token_rows(rows, np.arange(rows.shape[1]))
+        return z[:, -1]
 
     def prefill(self, tokens: np.ndarray) -> np.ndarray:
         """Process the prompt; return logits predicting token T.
 
         Only the most recent block enters the token decoder: its prefix comes
         from c_{n-1}; earlier blocks never do ([BT] §3.4 token-decoder cost
-        analysis, "prefill computation near zero" [orig. §2.4])."""
+        analysis, "prefill computation near zero" [orig. §2.4]). The block
+        decoder runs over the n = floor(T / L_B) complete blocks; when T is
+        not a multiple of L_B the r = T - n L_B trailing tokens are the first
+        tokens of the current block and enter the token decoder after the
+        prefix (reading R8), exactly as if they had been fed by r decode
+        calls."""
         s, m = self.s, self.m
         tokens = np.asarray(tokens)
         B, T = tokens.shape
         L = s.block_len
-        assert T % L == 0 and T >= L
+        assert T >= L
         n = T // L
+        r = T - n * L
         self.block_caches = m._fresh(m.block_layers)
-        e = embed_blocks(tokens, m.g["blk_emb"], L)
+        e = embed_blocks(tokens[:, :n * L], m.g["blk_emb"], L)
         c = m.block_decoder(e, np.arange(n), self.block_caches)[:, -1]   # c_{n-1}
         self.t = T
         self.cur_block = np.zeros((B, L), dtype=np.int64)
+        self.cur_block[:, :r] = tokens[:, n * L:]
         if not s.use_token_decoder:
             return c @ m.g["w_lm"].T
-        return self._start_block(c)
+        return self._start_block(c, tokens[:, n * L:])
 
     def decode(self, tok: np.ndarray) -> np.ndarray:
         """Feed token x_t (t = tokens seen so far); return logits for x_{t+1}.
@@ -373,3 +402,25 @@ class OracleSession:
         for i in range(steps - 1):
             out.append(self.decode(tokens[:, prompt_len + i]))
         return np.stack(out)
+
+
+def ragged_generate_logits(model: BlockTransformerOracle, prompts, continuations, steps: int,
+                           pad: bool = False, pad_id: int = 0) -> List[np.ndarray]:
+    """Teacher-forced runs of sequences with different prompt lengths, each
+    on its own (rows of a batch are independent: [BT] §3.2, every sequence
+    has its own block and token decoders' state).
+
+    prompts[b]: [T_b] token ids; continuations[b]: the tokens fed after the
+    prompt (at least steps - 1). pad = True left-pads every prompt to a
+    block boundary first (``left_pad``). Returns, per sequence, the logits
+    [steps, V] predicting the token after the prompt and after each fed
+    token.
+    """
+    out = []
+    for pr, cont in zip(prompts, continuations):
+        pr = np.asarray(pr)
+        if pad:
+            pr = left_pad(pr, model.s.block_len, pad_id)
+        seq = np.concatenate([pr, np.asarray(cont)[:steps - 1]])[None, :]
+        out.append(model.session().generate_logits(seq, pr.shape[0], steps)[:, 0])
+    return out

@@ -269,6 +269,43 @@ def pin_incremental_equals_full(om, shape=SMALL, T=8, G=11) -> float:
     return float(np.abs(inc - full[:, T:T + G].transpose(1, 0, 2)).max())
 
 
+def pin_left_padding(om) -> bool:
+    """Left padding: p = (-T) mod L_B pad ids in front, p = 0 for aligned
+    prompts; prefill of the padded prompt equals the full pass over the
+    padded sequence at the position after the prompt."""
+    L = SMALL.block_len
+    ok = True
+    for T in range(1, 13):
+        x = np.arange(100, 100 + T)
+        y = om.left_pad(x, L, 7)
+        p = (L - T % L) % L
+        ok &= y.shape[0] == T + p and (y.shape[0] % L == 0)
+        ok &= bool(np.all(y[:p] == 7)) and bool(np.array_equal(y[p:], x))
+    params = params_of(SMALL)
+    toks = tokens_of(SMALL, B=1, S=17)
+    o = om.BlockTransformerOracle(SMALL, params)
+    for T in (5, 7, 8):
+        padded = om.left_pad(toks[0, :T], L, 3)
+        seq = np.concatenate([padded, toks[0, T:]])[None]
+        z = o.session().prefill(padded[None])
+        full = o.forward_full(seq)
+        ok &= float(np.abs(z - full[:, padded.shape[0]]).max()) < 1e-10
+    return ok
+
+
+def pin_ragged_vs_batched(om) -> float:
+    """Ragged runs (one session per sequence) against the batched session:
+    equal prompt lengths give the batched logits row for row."""
+    params = params_of(SMALL)
+    o = om.BlockTransformerOracle(SMALL, params)
+    toks = tokens_of(SMALL, B=3, S=20)
+    T, G = 9, 6
+    batched = o.session().generate_logits(toks, T, G)           # [G, B, V]
+    rag = om.ragged_generate_logits(o, [toks[b, :T] for b in range(3)],
+                                    [toks[b, T:] for b in range(3)], G)
+    return float(max(np.abs(rag[b] - batched[:, b]).max() for b in range(3)))
+
+
 def pin_future_tokens_invisible(om) -> bool:
     """Invariant 2a: logits for x_t are bitwise unchanged when any x_t',
     t' >= t, is perturbed."""

@@ -32,6 +32,7 @@ def _first_failing_pin(mod):
         ("future_invisible", lambda: pins.pin_future_tokens_invisible(mod)),
         ("locality_nb0", lambda: pins.pin_locality_without_block_layers(mod)),
         ("incremental", lambda: pins.pin_incremental_equals_full(mod) < TOL),
+        ("incremental_partial", lambda: pins.pin_incremental_equals_full(mod, T=10, G=7) < TOL),
         ("hf_vanilla", lambda: pins.pin_vanilla_vs_hf(mod) < TOL),
         ("hf_block_model", lambda: pins.pin_block_model_vs_hf(mod) < TOL),
     ]
@@ -101,6 +102,31 @@ def _layer_serial_residual(h, p, pos, cache, H, r, eps, base):
     return h1 + ORIG["gelu"](m @ p["w_1"].T + p["b_1"]) @ p["w_2"].T + p["b_2"]
 
 
+_ORIG_START = om.OracleSession._start_block
+
+
+def _start_block_trailing_shifted(self, c, trailing=None):
+    # trailing prompt tokens one local position too far
+    if trailing is None or trailing.shape[1] == 0:
+        return _ORIG_START(self, c, trailing)
+    s, m = self.s, self.m
+    self.token_caches = m._fresh(m.token_layers)
+    pre = ORIG["prefix_projection"](c, m.g["w_prefix"], m.g["b_prefix"], s.prefix_len)
+    rows = np.concatenate([pre, m.g["tok_emb"][trailing]], axis=1)
+    pos = np.concatenate([np.arange(s.prefix_len), s.prefix_len + 1 + np.arange(trailing.shape[1])])
+    return self._token_rows(rows, pos)[:, -1]
+
+
+def _start_block_trailing_dropped(self, c, trailing=None):
+    return _ORIG_START(self, c, None)
+
+
+SESSION_MUTATIONS = {
+    "trailing_shifted": _start_block_trailing_shifted,
+    "trailing_dropped": _start_block_trailing_dropped,
+}
+
+
 MUTATIONS = {
     "rotary_sign": ("rotary", _rotary_wrong_sign),
     "rotary_freq": ("rotary", _rotary_wrong_freq),
@@ -123,6 +149,14 @@ def test_unmutated_oracle_passes_every_pin():
 def test_planted_mistake_is_caught(mutation, monkeypatch):
     name, fn = MUTATIONS[mutation]
     monkeypatch.setattr(om, name, fn)
+    caught_by = _first_failing_pin(om)
+    print(f"{mutation}: caught by {caught_by}")
+    assert caught_by is not None, f"no pin caught the planted mistake {mutation}"
+
+
+@pytest.mark.parametrize("mutation", sorted(SESSION_MUTATIONS))
+def test_planted_prefill_mistake_is_caught(mutation, monkeypatch):
+    monkeypatch.setattr(om.OracleSession, "_start_block", SESSION_MUTATIONS[mutation])
     caught_by = _first_failing_pin(om)
     print(f"{mutation}: caught by {caught_by}")
     assert caught_by is not None, f"no pin caught the planted mistake {mutation}"

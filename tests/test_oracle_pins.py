@@ -60,6 +60,26 @@ def test_incremental_equals_full_sequence(variant):
     assert pins.pin_incremental_equals_full(om, shape) < 1e-10
 
 
+@pytest.mark.parametrize("T", [5, 6, 7, 9, 10, 11])
+def test_incremental_equals_full_sequence_partial_block_prompt(T):
+    """Invariant 1 for prompts that end inside a block: the trailing tokens
+    prefilled into the token decoder give the full pass's logits."""
+    assert pins.pin_incremental_equals_full(om, pins.SMALL, T=T, G=9) < 1e-10
+
+
+def test_left_padding():
+    """Left padding adds (-T) mod L_B pad tokens (none for aligned prompts),
+    and a padded prompt is run as the aligned sequence it becomes."""
+    assert pins.pin_left_padding(om)
+
+
+def test_ragged_batch_equals_batched_rows():
+    """The per-sequence runs of a ragged batch agree with the batched session
+    on every row when the rows' prompt lengths are equal, and each row of a
+    ragged batch equals its own single-sequence run."""
+    assert pins.pin_ragged_vs_batched(om) < 1e-12
+
+
 def test_future_tokens_do_not_change_past_logits():
     """Invariant 2a."""
     assert pins.pin_future_tokens_invisible(om)
