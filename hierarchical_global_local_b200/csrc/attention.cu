@@ -87,6 +87,8 @@ attn_decode_kernel(const T* __restrict__ q, int ldq, const T* __restrict__ kc,
   pdl_trigger();
   pdl_wait();
   using C = DecCfg<T, DH>;
+  // chunks per pair from the longest sequence; a shorter sequence of a
+  // ragged batch (kvlen.row_lag) has empty trailing chunks
   const int n = pos_base(kvlen) + 1;
   const int nch = (n + C::CHUNK - 1) / C::CHUNK;
   const long long Ttot = (long long)pairs * nch;
@@ -125,13 +127,16 @@ attn_decode_kernel(const T* __restrict__ q, int ldq, const T* __restrict__ kc,
         const long long x = x0 + i;
         const int pr = (int)(x / nch), ci = (int)(x - (long long)pr * nch);
         const int r0 = ci * C::CHUNK;
-        const int rows = min(C::CHUNK, n - r0);
+        const int np = pos_base(kvlen, pr / H) + 1;  // this pair's entries
+        const int rows = max(0, min(C::CHUNK, np - r0));
         const uint32_t bytes = (uint32_t)rows * C::ROW_BYTES;
         const size_t off = ((size_t)pr * cap + r0) * DH;
         T* dk = sKV + (size_t)s * 2 * C::CHUNK * DH;
         mbar_arrive_expect_tx(&full[s], 2 * bytes);
-        bulk_g2s(dk, kc + off, bytes, &full[s]);
-        bulk_g2s(dk + C::CHUNK * DH, vc + off, bytes, &full[s]);
+        if (bytes) {
+          bulk_g2s(dk, kc + off, bytes, &full[s]);
+          bulk_g2s(dk + C::CHUNK * DH, vc + off, bytes, &full[s]);
+        }
       }
     }
     return;  // the copies complete on the mbarriers; consumers sync among themselves
@@ -147,6 +152,7 @@ attn_decode_kernel(const T* __restrict__ q, int ldq, const T* __restrict__ kc,
     const long long pend = (long long)(pr + 1) * nch;
     const int cnt = (int)((pend < x1 ? pend : x1) - (x0 + i));
     const int b = pr / H, h = pr - b * H;
+    const int np = pos_base(kvlen, b) + 1;  // this pair's entries (<= n)
     float M = -FLT_MAX, l = 0.f;
     float of[C::EPT];
 #pragma unroll
@@ -166,7 +172,7 @@ attn_decode_kernel(const T* __restrict__ q, int ldq, const T* __restrict__ kc,
         const T* sK = sKV + (size_t)s * 2 * C::CHUNK * DH;
         const T* sV = sK + C::CHUNK * DH;
         const long long x = x0 + ii;
-        const int rows = min(C::CHUNK, n - (int)(x - (long long)pr * nch) * C::CHUNK);
+        const int rows = min(C::CHUNK, np - (int)(x - (long long)pr * nch) * C::CHUNK);
         // uniform trip count over the warp: the row-group shuffles always
         // see the whole warp
         for (int rb = 0; rb < rows; rb += C::GROUPS) {

@@ -61,13 +61,24 @@ struct PosSpec {
   int mode;           // PosMode
   int add;            // constant added to the state-derived base
   int rows_per_seq;   // consecutive rows of one sequence
+  // POS_BLOCK only (may be null): per-sequence lag behind the longest
+  // sequence of a ragged batch; sequence b's block position is
+  // dstate[2] - row_lag[b]
+  const int* row_lag = nullptr;
 };
 
+// position base shared by every sequence (POS_BLOCK: the longest one's)
 __device__ __forceinline__ int pos_base(const PosSpec& p) {
   int b = 0;
   if (p.mode == POS_BLOCK) b = p.dstate[2];
   else if (p.mode == POS_LOCAL) b = p.dstate[1];
   return b + p.add;
+}
+
+// position base of sequence `seq`
+__device__ __forceinline__ int pos_base(const PosSpec& p, int seq) {
+  const int b = pos_base(p);
+  return (p.mode == POS_BLOCK && p.row_lag) ? b - p.row_lag[seq] : b;
 }
 
 // ---- mbarrier + bulk copy (PTX) -------------------------------------------

@@ -33,21 +33,49 @@ bool pdl_enabled() {
 template <typename T>
 __global__ void embed_prompt_kernel(const int32_t* __restrict__ tokens, int T_len, int n, int L_B,
                                     const T* __restrict__ table, int V, int D,
-                                    float* __restrict__ h, int* status) {
+                                    float* __restrict__ h, int* status, const int* __restrict__ row_pad,
+                                    const int* __restrict__ row_len, int pad_id) {
   pdl_trigger();
   pdl_wait();
   const int r = blockIdx.x;  // row = b * n + i
   const int b = r / n, i = r % n;
   const int De = D / L_B;
+  // ragged batch: sequence b is row_len[b] tokens preceded by row_pad[b]
+  // pad ids; blocks past its end read id 0 (their rows are never used)
+  const int pad = row_pad ? row_pad[b] : 0;
+  const int len = row_len ? row_len[b] : T_len;
   for (int x = threadIdx.x; x < D; x += blockDim.x) {
     const int j = x / De, e = x - j * De;
-    int tok = tokens[(size_t)b * T_len + (size_t)i * L_B + j];
+    const int src = i * L_B + j - pad;
+    int tok = src < 0 ? pad_id : (src < len ? tokens[(size_t)b * T_len + src] : 0);
     if (tok < 0 || tok >= V) {
       set_status(status, ST_BAD_TOKEN);
       tok = 0;
     }
     h[(size_t)r * D + x] = to_f(table[(size_t)tok * De + e]);
   }
+}
+
+// Trailing prompt tokens (prompt length not a multiple of L_B): token i < r
+// of row b, tokens[b * T_len + col0 + i], is recorded in block_tok[b, i] and
+// its token-decoder embedding becomes row b * rows_per_seq + row_off + i of h.
+template <typename T>
+__global__ void embed_tail_kernel(const int32_t* __restrict__ tokens, int T_len, int col0, int r,
+                                  int rows_per_seq, int row_off, const T* __restrict__ tok_emb, int V,
+                                  int D, float* __restrict__ h, int32_t* __restrict__ block_tok, int L_B,
+                                  int* status, const int* __restrict__ row_col0) {
+  pdl_trigger();
+  pdl_wait();
+  const int b = blockIdx.x / r, i = blockIdx.x % r;
+  const int c0 = row_col0 ? row_col0[b] : col0;
+  int tok = tokens[(size_t)b * T_len + c0 + i];
+  if (tok < 0 || tok >= V) {
+    if (threadIdx.x == 0) set_status(status, ST_BAD_TOKEN);
+    tok = 0;
+  }
+  if (threadIdx.x == 0) block_tok[b * L_B + i] = tok;
+  float* row = h + ((size_t)b * rows_per_seq + row_off + i) * D;
+  for (int x = threadIdx.x; x < D; x += blockDim.x) row[x] = to_f(tok_emb[(size_t)tok * D + x]);
 }
 
 template <typename T>
@@ -170,16 +198,32 @@ __global__ void advance_kernel(int* dstate, int L_B) {
 
 cudaError_t launch_embed_prompt(int dt, const int32_t* tokens, int B, int T, int L_B,
                                 const void* blk_emb, int V, int D, float* h, int* status,
-                                cudaStream_t s) {
-  const int n = T / L_B;
+                                cudaStream_t s, int n_blocks, const int* row_pad, const int* row_len,
+                                int pad_id) {
+  const int n = n_blocks >= 0 ? n_blocks : T / L_B;
   if (B * n == 0) return cudaSuccess;
   if (dt == DT_BF16) {
     BT_LAUNCH(embed_prompt_kernel<bf16>, dim3(B * n), dim3(256), 0, s, tokens, T, n, L_B, (const bf16*)blk_emb, V, D,
-                                                    h, status);
+              h, status, row_pad, row_len, pad_id);
   }
   else {
     BT_LAUNCH(embed_prompt_kernel<float>, dim3(B * n), dim3(256), 0, s, tokens, T, n, L_B, (const float*)blk_emb, V,
-                                                     D, h, status);
+              D, h, status, row_pad, row_len, pad_id);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_embed_tail(int dt, const int32_t* tokens, int B, int T_len, int col0, int r,
+                              int rows_per_seq, int row_off, const void* tok_emb, int V, int D, float* h,
+                              int32_t* block_tok, int L_B, int* status, cudaStream_t s,
+                              const int* row_col0) {
+  if (B * r == 0) return cudaSuccess;
+  if (dt == DT_BF16) {
+    BT_LAUNCH(embed_tail_kernel<bf16>, dim3(B * r), dim3(256), 0, s, tokens, T_len, col0, r, rows_per_seq,
+              row_off, (const bf16*)tok_emb, V, D, h, block_tok, L_B, status, row_col0);
+  } else {
+    BT_LAUNCH(embed_tail_kernel<float>, dim3(B * r), dim3(256), 0, s, tokens, T_len, col0, r, rows_per_seq,
+              row_off, (const float*)tok_emb, V, D, h, block_tok, L_B, status, row_col0);
   }
   return cudaGetLastError();
 }
@@ -299,14 +343,15 @@ template <typename T>
 __global__ void __launch_bounds__(LN_THREADS)
 ln_rows_kernel(const float* __restrict__ h, int row_step, int row_off, int D,
                const float* __restrict__ g, const float* __restrict__ b, float eps,
-               T* __restrict__ out) {
+               T* __restrict__ out, const int* __restrict__ row_lag) {
   pdl_trigger();
   pdl_wait();
   __shared__ float red[4];
   const int r = blockIdx.x;
   float4 v[LN_MAXV];
   float mu, rstd;
-  ln_row(h + ((size_t)r * row_step + row_off) * D, D, eps, v, mu, rstd, red);
+  const int off = row_lag ? row_off - row_lag[r] : row_off;
+  ln_row(h + ((size_t)r * row_step + off) * D, D, eps, v, mu, rstd, red);
   T* o = out + (size_t)r * D;
 #pragma unroll
   for (int u = 0; u < LN_MAXV; ++u) {
@@ -328,13 +373,16 @@ cudaError_t launch_ln_dual(int dt, const float* h, int M, int D, const float* g1
 }
 
 cudaError_t launch_ln_rows(int dt, const float* h, int R, int row_step, int row_off, int D,
-                           const float* g, const float* b, float eps, void* out, cudaStream_t s) {
+                           const float* g, const float* b, float eps, void* out, cudaStream_t s,
+                           const int* row_lag) {
   if (R == 0) return cudaSuccess;
   if (D > LN_THREADS * 4 * LN_MAXV || (D % 4)) return cudaErrorInvalidValue;
   if (dt == DT_BF16)
-    BT_LAUNCH(ln_rows_kernel<bf16>, dim3(R), dim3(LN_THREADS), 0, s, h, row_step, row_off, D, g, b, eps, (bf16*)out);
+    BT_LAUNCH(ln_rows_kernel<bf16>, dim3(R), dim3(LN_THREADS), 0, s, h, row_step, row_off, D, g, b, eps,
+              (bf16*)out, row_lag);
   else
-    BT_LAUNCH(ln_rows_kernel<float>, dim3(R), dim3(LN_THREADS), 0, s, h, row_step, row_off, D, g, b, eps, (float*)out);
+    BT_LAUNCH(ln_rows_kernel<float>, dim3(R), dim3(LN_THREADS), 0, s, h, row_step, row_off, D, g, b, eps,
+              (float*)out, row_lag);
   return cudaGetLastError();
 }
 
@@ -373,7 +421,7 @@ __global__ void rope_append_kernel(const T* __restrict__ qkv, int D, int H, int 
   const int d = D / H;
   const int half = rot >> 1;
   const int b = m / ps.rows_per_seq;
-  const int pos = pos_base(ps) + (m - b * ps.rows_per_seq);
+  const int pos = pos_base(ps, b) + (m - b * ps.rows_per_seq);
   const T* row = qkv + (size_t)m * 3 * D;
   for (int x = threadIdx.x; x < 3 * D; x += blockDim.x) {
     const int part = x / D;  // 0 q, 1 k, 2 v

@@ -49,7 +49,7 @@ __device__ __forceinline__ void epi_apply_rope(const Epi& e, int m, int n, float
   const int d = D / e.H;
   const int hh = c / d, dim = c - hh * d;
   const int b = m / e.pos.rows_per_seq;
-  const int pos = pos_base(e.pos) + (m - b * e.pos.rows_per_seq);
+  const int pos = pos_base(e.pos, b) + (m - b * e.pos.rows_per_seq);
   float out = v;
   if (part < 2 && dim < e.rot) {
     const int half = e.rot >> 1;

@@ -26,9 +26,22 @@ int device_sm_count();
 
 // ---- embedder / token ingest / step state --------------------------------
 // Prompt embedder: h[b*n + i, :] = concat_j blk_emb[tokens[b, i*L_B + j]].
+// Ragged batches (row_pad / row_len non-null): sequence b is the row_len[b]
+// tokens at the start of its row, preceded by row_pad[b] pad ids (pad_id);
+// n_blocks (>= 0) blocks per sequence are embedded (blocks past a sequence's
+// end read id 0).
 cudaError_t launch_embed_prompt(int dt, const int32_t* tokens, int B, int T, int L_B,
                                 const void* blk_emb, int V, int D, float* h, int* status,
-                                cudaStream_t s);
+                                cudaStream_t s, int n_blocks = -1, const int* row_pad = nullptr,
+                                const int* row_len = nullptr, int pad_id = 0);
+// Trailing prompt tokens of a prompt that ends inside a block: for b < B,
+// i < r, token tokens[b * T_len + col0 + i] is recorded in block_tok[b, i]
+// and its token-decoder embedding tok_emb[token] is written to row
+// b * rows_per_seq + row_off + i of h [.., D] (fp32).
+cudaError_t launch_embed_tail(int dt, const int32_t* tokens, int B, int T_len, int col0, int r,
+                              int rows_per_seq, int row_off, const void* tok_emb, int V, int D, float* h,
+                              int32_t* block_tok, int L_B, int* status, cudaStream_t s,
+                              const int* row_col0 = nullptr);  // per-sequence col0 (ragged)
 // Decode ingest of the fed token src[b] at position t = dstate[0]:
 // records it in block_tok[b, t % L_B]; block_step = 0 gathers
 // h[b] = tok_emb[src[b]]; block_step = 1 (the token completes its block)
@@ -54,8 +67,10 @@ cudaError_t launch_ln_dual(int dt, const float* h, int M, int D, const float* g1
                            const float* b1, const float* g2, const float* b2, float eps,
                            void* x1, cudaStream_t s);
 // out[r] = LN(h[r * row_step + row_off]; g, b) for r < R (act dtype).
+// row_lag (optional): row r reads h[r * row_step + row_off - row_lag[r]].
 cudaError_t launch_ln_rows(int dt, const float* h, int R, int row_step, int row_off, int D,
-                           const float* g, const float* b, float eps, void* out, cudaStream_t s);
+                           const float* g, const float* b, float eps, void* out, cudaStream_t s,
+                           const int* row_lag = nullptr);
 
 // ---- rotary + KV append ---------------------------------------------------
 // Row m of qkv [M, 3D] belongs to sequence m / rows_per_seq at position

@@ -100,7 +100,9 @@ int dims_of(const bt_config* c, Dims* o) {
   d.n_cap = (d.max_seq + d.L - 1) / d.L;
   d.l_cap = d.tokdec ? d.P + d.L - 1 : 1;
   const int rows_blk = d.Bmax * d.n_cap;
-  const int rows_tok = d.Bmax * (d.P > 1 ? d.P : 1);
+  // token-decoder rows of one call: P prefix rows plus up to L_B - 1
+  // trailing prompt tokens at prefill
+  const int rows_tok = d.Bmax * (d.tokdec ? d.P + d.L - 1 : 1);
   d.R = rows_blk > rows_tok ? rows_blk : rows_tok;
   d.tab_pos = d.n_cap > d.l_cap ? d.n_cap : d.l_cap;
   *o = d;
@@ -123,6 +125,11 @@ struct bt_model {
   float *h_b = nullptr, *h_t = nullptr, *logits = nullptr;
   void *x1 = nullptr, *qkv = nullptr, *qrot = nullptr, *a2 = nullptr, *xf = nullptr;
   int32_t *next = nullptr, *fed = nullptr, *block_tok = nullptr;
+  // per-sequence prefill layout of a ragged batch (zeros for a uniform one):
+  // row_lag [B_max] blocks behind the longest sequence, row_pad [B_max] left
+  // pad ids, row_len [B_max] prompt tokens, row_col0 [B_max] first trailing token
+  int *row_lag = nullptr, *row_pad = nullptr, *row_len = nullptr, *row_col0 = nullptr;
+  bool ragged = false;
   int *dstate = nullptr, *status = nullptr;
   float2* rope_tab = nullptr;
   void* attn_scratch = nullptr;
@@ -224,7 +231,7 @@ static size_t carve(bt_model* m, const Dims& d, void* ws) {
   // activations
   const size_t R = d.R;
   m->h_b = (float*)c.take(R * D * 4);
-  m->h_t = (float*)c.take((size_t)d.Bmax * (d.P > 1 ? d.P : 1) * D * 4);
+  m->h_t = (float*)c.take((size_t)d.Bmax * (d.tokdec ? d.P + d.L - 1 : 1) * D * 4);
   m->x1 = c.take(R * 2 * D * eb);
   m->qkv = c.take(R * 3 * D * eb);
   m->qrot = c.take(R * D * eb);
@@ -234,6 +241,10 @@ static size_t carve(bt_model* m, const Dims& d, void* ws) {
   m->next = (int32_t*)c.take((size_t)d.Bmax * 4);
   m->fed = (int32_t*)c.take((size_t)d.Bmax * 4);
   m->block_tok = (int32_t*)c.take((size_t)d.Bmax * d.L * 4);
+  m->row_lag = (int*)c.take((size_t)d.Bmax * 4 * sizeof(int));
+  m->row_pad = m->row_lag ? m->row_lag + d.Bmax : nullptr;
+  m->row_len = m->row_lag ? m->row_lag + 2 * d.Bmax : nullptr;
+  m->row_col0 = m->row_lag ? m->row_lag + 3 * d.Bmax : nullptr;
   m->dstate = (int*)c.take(64);
   m->status = (int*)c.take(64);
   m->rope_tab = (float2*)c.take((size_t)d.tab_pos * (d.rot / 2 > 0 ? d.rot / 2 : 1) * 8);
@@ -358,6 +369,7 @@ int bt_create(const bt_config* cfg, const bt_weights* w, void* ws, size_t ws_byt
   BT_TRYC(cudaMemsetAsync(m->attn_scratch, 0, attn_decode_scratch_bytes(d.Bmax, d.H, d.d, d.n_cap, d.dt), st));
   BT_TRYC(cudaMemsetAsync(m->gs.counters, 0, (size_t)m->gs.n_counters * 4, st));
   BT_TRYC(cudaMemsetAsync(m->block_tok, 0, (size_t)d.Bmax * d.L * 4, st));
+  BT_TRYC(cudaMemsetAsync(m->row_lag, 0, (size_t)d.Bmax * 4 * sizeof(int), st));
   BT_TRYC(cudaMemsetAsync(m->ln_cnt, 0, (size_t)d.Bmax * (d.P > 1 ? d.P : 1) * sizeof(int), st));
   if (m->ts_bar) BT_TRYC(cudaMemsetAsync(m->ts_bar, 0, 64, st));
   if (m->ts_cnt) BT_TRYC(cudaMemsetAsync(m->ts_cnt, 0, (size_t)d.Bmax * d.H * sizeof(int), st));
@@ -495,24 +507,39 @@ static int run_token_decoder(bt_model* m, int B, PosSpec pos, cudaStream_t s) {
   return BT_OK;
 }
 
+// Trailing prompt tokens entering the token decoder after the prefix rows.
+struct Tail {
+  const int32_t* tokens = nullptr;  // [B, T_len]
+  int T_len = 0, col0 = 0, r = 0;   // tokens col0 .. col0 + r - 1 of each row
+  const int* row_col0 = nullptr;    // per-sequence col0 (ragged batches)
+};
+
 // context rows (B rows of h_b, row r*row_step + row_off) -> LN_b -> either the
-// prefix projection and the token decoder over P rows, or (vanilla) xf.
-static int run_context_to_head_input(bt_model* m, int B, int row_step, int row_off, cudaStream_t s) {
+// prefix projection and the token decoder over P rows (plus the trailing
+// prompt tokens of `tail`), or (vanilla) xf.
+static int run_context_to_head_input(bt_model* m, int B, int row_step, int row_off, cudaStream_t s,
+                                     const Tail& tail = Tail(), const int* row_lag = nullptr) {
   const Dims& d = m->d;
   {
     ProfScope p(m, s, BT_K_LAYERNORM, B, d.D, 0);
     BT_CUDA(launch_ln_rows(d.dt, m->h_b, B, row_step, row_off, d.D, m->lnf_b_g, m->lnf_b_b,
-                           m->cfg.ln_eps, m->xf, s));
+                           m->cfg.ln_eps, m->xf, s, row_lag));
   }
   if (!d.tokdec) return BT_OK;
+  const int rows = d.P + tail.r;  // token-decoder rows per sequence
   {
-    // prefix rows: h_t[b*P + p, :] = (W_p c_b + b_p)[p*D:(p+1)*D]
+    // prefix rows: h_t[b*rows + p, :] = (W_p c_b + b_p)[p*D:(p+1)*D]
     ProfScope p(m, s, BT_K_GEMM, B, d.P * d.D, d.D);
-    Epi ep{EPI_F32, m->h_t, d.P * d.D, nullptr, 0, m->b_prefix, 0, d.D};
+    Epi ep{EPI_F32, m->h_t, rows * d.D, nullptr, 0, m->b_prefix, 0, d.D};
     BT_CUDA(launch_gemm(d.dt, m->xf, d.D, m->w_prefix, d.D, B, d.P * d.D, d.D, 1 << 30, 0, ep, m->gs,
                         m->status, s));
   }
-  PosSpec pos{nullptr, POS_ZERO, 0, d.P};
+  if (tail.r > 0) {
+    ProfScope p(m, s, BT_K_EMBED, B * tail.r, d.D, 0);
+    BT_CUDA(launch_embed_tail(d.dt, tail.tokens, B, tail.T_len, tail.col0, tail.r, rows, d.P, m->tok_emb, d.V,
+                              d.D, m->h_t, m->block_tok, d.L, m->status, s, tail.row_col0));
+  }
+  PosSpec pos{nullptr, POS_ZERO, 0, rows};
   return run_token_decoder(m, B, pos, s);
 }
 
@@ -584,7 +611,7 @@ static int enqueue_decode_fused(bt_model* m, bool block_step, bool greedy, bool 
     return BT_OK;
   };
   if (block_step) {
-    PosSpec pos{m->dstate, POS_BLOCK, 0, 1};
+    PosSpec pos{m->dstate, POS_BLOCK, 0, 1, m->row_lag};
     for (int l = 0; l < d.Nb; ++l) {
       const NextLN nx = (l + 1 < d.Nb) ? dual_ln(m, m->blk[l + 1]) : lnb;
       rc = run_layer(m, m->blk[l], m->h_b, B, pos, layer_ptr(m->kb, m->kb_layer, l, d.eb),
@@ -665,7 +692,8 @@ static bool block_step_fused(const bt_model* m, int B) {
   const Dims& d = m->d;
   const char* env = getenv("BT_DECODE_BLOCK_STEP");
   if (!env || strcmp(env, "fused") != 0) return false;
-  if (!m->ts_att || d.Nb < 1 || d.P != 1) return false;
+  // its attention phase assumes one cache length for the whole batch
+  if (!m->ts_att || d.Nb < 1 || d.P != 1 || m->ragged) return false;
   if (!token_step_block_supported(d.dt, B, d.D, d.H, d.rot, d.V, d.Nt, d.Nb, d.P, d.l_cap, d.n_cap, d.L))
     return false;
   const long long ls = d.Nt > 1 ? (long long)((uint8_t*)m->tok[1].w_qkv1 - (uint8_t*)m->tok[0].w_qkv1) : 0;
@@ -735,7 +763,7 @@ static int enqueue_decode_token_step(bt_model* m, bool block_step, bool greedy, 
     BT_CUDA(launch_ingest(d.dt, src, m->block_tok, m->dstate, B, d.L, d.V, d.D, 1, m->blk_emb,
                           m->tok_emb, m->h_b, m->status, s));
   }
-  PosSpec pos{m->dstate, POS_BLOCK, 0, 1};
+  PosSpec pos{m->dstate, POS_BLOCK, 0, 1, m->row_lag};
   for (int l = 0; l < d.Nb; ++l) {
     int rc = run_layer(m, m->blk[l], m->h_b, B, pos, layer_ptr(m->kb, m->kb_layer, l, d.eb),
                        layer_ptr(m->vb, m->kb_layer, l, d.eb), d.n_cap, ATT_DECODE, 0, s);
@@ -770,7 +798,7 @@ static int enqueue_decode(bt_model* m, bool block_step, bool greedy, bool want_l
   }
   int rc;
   if (block_step) {
-    PosSpec pos{m->dstate, POS_BLOCK, 0, 1};
+    PosSpec pos{m->dstate, POS_BLOCK, 0, 1, m->row_lag};
     for (int l = 0; l < d.Nb; ++l) {
       rc = run_layer(m, m->blk[l], m->h_b, B, pos, layer_ptr(m->kb, m->kb_layer, l, d.eb),
                      layer_ptr(m->vb, m->kb_layer, l, d.eb), d.n_cap, ATT_DECODE, 0, s);
@@ -801,18 +829,56 @@ static void drop_graphs(bt_model* m) {
 
 extern "C" {
 
-int bt_prefill(bt_model* m, const int32_t* tokens, int32_t B, int32_t T, float* logits,
-               int32_t* next) {
+}  // extern "C"
+
+// Prefill of B sequences whose prompts sit at the start of the rows of
+// tokens [B, T_stride]. lengths == nullptr: every prompt has T_stride tokens.
+// Otherwise lengths[b] (host) tokens each; pad_id >= 0 left-pads every prompt
+// to a block boundary with that id, pad_id < 0 requires the same remainder
+// mod L_B for every length.
+static int prefill_impl(bt_model* m, const int32_t* tokens, int T_stride, int B, const int32_t* lengths,
+                        int pad_id, float* logits, int32_t* next) {
   if (!m || !tokens) return BT_EINVAL;
   const Dims& d = m->d;
   if (B < 1 || B > d.Bmax) return BT_ECAPACITY;
-  if (T < d.L || T % d.L) return BT_EINVAL;
+  // per-sequence layout: padded length, complete blocks, lag behind the longest
+  std::vector<int> host(4 * (size_t)d.Bmax, 0);
+  int T = T_stride;  // the longest (padded) prompt
+  bool ragged = false;
+  if (lengths) {
+    if (pad_id >= d.V) return BT_EINVAL;
+    int rem = -1;
+    T = 0;
+    for (int b = 0; b < B; ++b) {
+      const int len = lengths[b];
+      if (len < 1 || len > T_stride) return BT_EINVAL;
+      const int pad = pad_id >= 0 ? (d.L - len % d.L) % d.L : 0;
+      const int Tb = len + pad;
+      if (Tb < d.L) return BT_EINVAL;
+      if (rem < 0) rem = Tb % d.L;
+      else if (Tb % d.L != rem) return BT_EINVAL;  // the token decoders must stay in step
+      host[d.Bmax + b] = pad;
+      host[2 * d.Bmax + b] = len;
+      if (Tb > T) T = Tb;
+      if (Tb != T_stride || pad) ragged = true;
+    }
+    for (int b = 0; b < B; ++b) {
+      const int Tb = host[2 * d.Bmax + b] + host[d.Bmax + b];
+      host[b] = (T - Tb) / d.L;                                    // lag in blocks
+      host[3 * d.Bmax + b] = (Tb / d.L) * d.L - host[d.Bmax + b];  // first trailing token
+    }
+  }
+  if (T < d.L) return BT_EINVAL;
   if (T >= d.max_seq) return BT_ECAPACITY;
   cudaStream_t s = m->stream;
   m->B = B;
   m->t = T;
-  const int n = T / d.L;
+  if (m->ragged != ragged) drop_graphs(m);  // the block-step schedule depends on it
+  m->ragged = ragged;
+  const int n = T / d.L;       // complete blocks of the longest sequence: block-decoder rows
+  const int r = T - n * d.L;   // trailing tokens: the current block so far
   const int M = B * n;
+  BT_CUDA(cudaMemcpyAsync(m->row_lag, host.data(), host.size() * sizeof(int), cudaMemcpyHostToDevice, s));
   // a new session: merge counters of the decode attention start from zero
   BT_CUDA(cudaMemsetAsync(m->attn_scratch, 0,
                           attn_decode_scratch_bytes(d.Bmax, d.H, d.d, d.n_cap, d.dt), s));
@@ -823,15 +889,22 @@ int bt_prefill(bt_model* m, const int32_t* tokens, int32_t B, int32_t T, float* 
   BT_CUDA(launch_set_state(m->dstate, T, d.L, s));
   {
     ProfScope p(m, s, BT_K_EMBED, M, d.D, 0);
-    BT_CUDA(launch_embed_prompt(d.dt, tokens, B, T, d.L, m->blk_emb, d.V, d.D, m->h_b, m->status, s));
+    BT_CUDA(launch_embed_prompt(d.dt, tokens, B, T_stride, d.L, m->blk_emb, d.V, d.D, m->h_b, m->status, s, n,
+                                ragged ? m->row_pad : nullptr, ragged ? m->row_len : nullptr,
+                                pad_id >= 0 ? pad_id : 0));
   }
+  // a shorter sequence's blocks sit at positions 0 .. n_b - 1 of its rows; the
+  // rows after them are computed but never read (causal attention)
   PosSpec pos{nullptr, POS_ZERO, 0, n};
   for (int l = 0; l < d.Nb; ++l) {
     int rc = run_layer(m, m->blk[l], m->h_b, M, pos, layer_ptr(m->kb, m->kb_layer, l, d.eb),
                        layer_ptr(m->vb, m->kb_layer, l, d.eb), d.n_cap, ATT_PREFILL, n, s);
     if (rc != BT_OK) return rc;
   }
-  int rc = run_context_to_head_input(m, B, n, n - 1, s);
+  Tail tail;
+  tail.tokens = tokens; tail.T_len = T_stride; tail.col0 = n * d.L; tail.r = r;
+  tail.row_col0 = ragged ? m->row_col0 : nullptr;
+  int rc = run_context_to_head_input(m, B, n, n - 1, s, tail, ragged ? m->row_lag : nullptr);
   if (rc != BT_OK) return rc;
   rc = run_head(m, B, logits != nullptr, s);
   if (rc != BT_OK) return rc;
@@ -839,6 +912,21 @@ int bt_prefill(bt_model* m, const int32_t* tokens, int32_t B, int32_t T, float* 
   m->prefilled = true;
   if (m->graph_B != B) { drop_graphs(m); m->graph_B = B; }
   return copy_outputs(m, logits, next);
+}
+
+extern "C" {
+
+int bt_prefill(bt_model* m, const int32_t* tokens, int32_t B, int32_t T, float* logits,
+               int32_t* next) {
+  if (!m || !tokens) return BT_EINVAL;
+  if (T < m->d.L) return BT_EINVAL;
+  return prefill_impl(m, tokens, T, B, nullptr, -1, logits, next);
+}
+
+int bt_prefill_ragged(bt_model* m, const int32_t* tokens, int32_t row_stride, const int32_t* lengths,
+                      int32_t B, int32_t pad_id, float* logits, int32_t* next) {
+  if (!m || !tokens || !lengths || row_stride < 1) return BT_EINVAL;
+  return prefill_impl(m, tokens, row_stride, B, lengths, pad_id, logits, next);
 }
 
 int bt_decode_step(bt_model* m, const int32_t* tokens, float* logits, int32_t* next) {

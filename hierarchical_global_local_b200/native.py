@@ -71,6 +71,8 @@ def lib() -> ctypes.CDLL:
             "bt_create": (c_int, [ctypes.POINTER(BtConfig), ctypes.POINTER(BtWeights), c_void_p,
                                   c_size_t, c_void_p, ctypes.POINTER(c_void_p)]),
             "bt_prefill": (c_int, [c_void_p, c_void_p, c_int32, c_int32, c_void_p, c_void_p]),
+            "bt_prefill_ragged": (c_int, [c_void_p, c_void_p, c_int32, ctypes.POINTER(c_int32), c_int32,
+                                          c_int32, c_void_p, c_void_p]),
             "bt_decode_step": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p]),
             "bt_sync": (c_int, [c_void_p]),
             "bt_position": (c_int, [c_void_p]),
@@ -112,7 +114,7 @@ def lib() -> ctypes.CDLL:
 def exported_symbols():
     """Names of the entry points the binding expects the library to export."""
     return [
-        "bt_workspace_bytes", "bt_create", "bt_prefill", "bt_decode_step", "bt_sync",
+        "bt_workspace_bytes", "bt_create", "bt_prefill", "bt_prefill_ragged", "bt_decode_step", "bt_sync",
         "bt_position", "bt_destroy", "bt_strerror", "bt_last_cuda_error",
         "bt_kernel_launches", "bt_profile_begin", "bt_profile_end",
         "bt_op_decode_attention_scratch_bytes", "bt_op_decode_attention",
@@ -227,6 +229,22 @@ class BlockTransformer:
             next_tokens = torch.empty(B, dtype=torch.int32, device="cuda")
         _check(lib().bt_prefill(self._h, tokens.data_ptr(), B, T, _ptr(logits),
                                 _ptr(next_tokens)), "bt_prefill")
+        self.batch = B
+        return logits, next_tokens
+
+    def prefill_ragged(self, tokens, lengths, pad_id: int = -1, logits=None,
+                       next_tokens=None) -> Tuple[object, object]:
+        """tokens: int32 CUDA [B, row_stride], sequence b's prompt in the first
+        lengths[b] entries of its row; pad_id >= 0 left-pads every prompt to a
+        block boundary (see bt_prefill_ragged)."""
+        import torch
+        B, stride = tokens.shape
+        assert tokens.dtype == torch.int32 and tokens.is_contiguous() and len(lengths) == B
+        if next_tokens is None:
+            next_tokens = torch.empty(B, dtype=torch.int32, device="cuda")
+        lens = (c_int32 * B)(*[int(x) for x in lengths])
+        _check(lib().bt_prefill_ragged(self._h, tokens.data_ptr(), stride, lens, B, int(pad_id),
+                                       _ptr(logits), _ptr(next_tokens)), "bt_prefill_ragged")
         self.batch = B
         return logits, next_tokens
 

@@ -132,17 +132,40 @@ BT_API int bt_create(const bt_config *cfg, const bt_weights *w, void *workspace_
 
 /* Prefill: process prompts tokens_dev [batch, prompt_len] (int32,
  * row-major, ids in [0, V)) for all `batch` sequences, resetting any earlier
- * state. Runs the embedder and the block decoder over the n = prompt_len/L_B
- * blocks (filling the block KV cache), then the prefix projection of the last
- * block's context and the token decoder over the P prefix rows (earlier
- * blocks never enter the token decoder, §3.4 token-decoder cost analysis).
- * Writes the logits predicting token prompt_len to logits_dev [batch, V]
- * fp32 (if non-NULL) and their greedy argmax (lowest id among ties) to
- * next_tokens_dev [batch] int32 (if non-NULL).
- * Requires 1 <= batch <= max_batch, prompt_len >= L_B, prompt_len % L_B == 0,
- * prompt_len < max_seq. */
+ * state. Runs the embedder and the block decoder over the n =
+ * floor(prompt_len / L_B) complete blocks (filling the block KV cache), then
+ * the prefix projection of the last complete block's context and the token
+ * decoder over the P prefix rows followed by the r = prompt_len mod L_B
+ * trailing tokens, which are the first tokens of the current block (earlier
+ * blocks never enter the token decoder, §3.4 token-decoder cost analysis;
+ * prompts that end inside a block, §3.4 "The Embedder"). Writes the logits
+ * predicting token prompt_len to logits_dev [batch, V] fp32 (if non-NULL)
+ * and their greedy argmax (lowest id among ties) to next_tokens_dev [batch]
+ * int32 (if non-NULL).
+ * Requires 1 <= batch <= max_batch, prompt_len >= L_B, prompt_len < max_seq. */
 BT_API int bt_prefill(bt_model *m, const int32_t *tokens_dev, int32_t batch,
                int32_t prompt_len, float *logits_dev, int32_t *next_tokens_dev);
+
+/* Prefill of a ragged batch: sequence b's prompt is the first lengths[b]
+ * tokens of row b of tokens_dev [batch, row_stride] (int32, device);
+ * `lengths` is a HOST array of `batch` entries, 1 <= lengths[b] <= row_stride.
+ *   pad_id >= 0: inference left padding (§3.4 "The Embedder", prompts whose
+ *     length is not a multiple of L_B): each prompt is preceded by
+ *     (-lengths[b]) mod L_B pad tokens of id pad_id, so that every sequence
+ *     ends on a block boundary.
+ *   pad_id < 0: no padding; every lengths[b] must leave the same remainder
+ *     mod L_B (the remainder's trailing tokens enter the token decoder as in
+ *     bt_prefill).
+ * Each sequence keeps its own number of blocks: the block decoder's KV cache
+ * of sequence b holds only its own blocks, and decode attention reads only
+ * them. Decode calls then run all sequences in step (the token decoders are
+ * at the same position of their blocks). bt_position reports the longest
+ * (padded) sequence's position; max_seq bounds it. Every padded length must
+ * be >= L_B. Errors as bt_prefill, and BT_EINVAL for lengths outside
+ * [1, row_stride], unequal remainders without padding, or pad_id >= V. */
+BT_API int bt_prefill_ragged(bt_model *m, const int32_t *tokens_dev, int32_t row_stride,
+                             const int32_t *lengths, int32_t batch, int32_t pad_id,
+                             float *logits_dev, int32_t *next_tokens_dev);
 
 /* Decode one token per sequence. tokens_dev [batch] int32 is the token fed
  * at position t (teacher forcing); NULL feeds the model's own greedy argmax

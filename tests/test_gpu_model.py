@@ -230,3 +230,107 @@ def test_fused_block_step_matches_oracle_and_chain(lb, B, monkeypatch):
         assert gh.rel_l2(gl[s], ol[s]) <= BF16_REL, (s, gh.rel_l2(gl[s], ol[s]))
         assert gh.rel_l2(gl[s], cl[s]) <= 1e-2, (s, gh.rel_l2(gl[s], cl[s]))
     assert np.array_equal(gn, gl.argmax(axis=-1))
+
+
+@pytest.mark.parametrize("lb,T,P", [(4, 49, 1), (4, 51, 1), (8, 61, 1), (2, 23, 2)])
+def test_prompt_ending_inside_a_block_bf16(lb, T, P):
+    """Prompt length not a multiple of L_B: the trailing tokens are prefilled
+    into the token decoder after the prefix; every following step (token and
+    block steps) matches the oracle."""
+    shape = synth.ModelShape(vocab=1000, d_model=256, n_heads=4, block_len=lb,
+                             n_block_layers=2, n_token_layers=2, prefix_len=P)
+    gl, gn, ol = _run(shape, B=3, T=T, G=2 * lb + 3, seed=7)
+    for s in range(gl.shape[0]):
+        assert gh.rel_l2(gl[s], ol[s]) <= BF16_REL, (s, gh.rel_l2(gl[s], ol[s]))
+    assert np.array_equal(gn, gl.argmax(axis=-1))
+
+
+def test_prompt_ending_inside_a_block_fp32():
+    """The fp32 workload shape with a prompt of 66 tokens (16 blocks + 2),
+    max |logit difference| <= 1e-4 at every step."""
+    wl = synth.WORKLOADS["tiny_fp32"]
+    gl, gn, ol = _run(wl.shape, B=2, T=66, G=11, seed=8)
+    err = np.abs(gl - ol).max(axis=(1, 2))
+    assert err.max() <= FP32_TOL, err
+
+
+def _ragged_run(shape, lengths, pad_id, G, seed):
+    """Ragged batch through bt_prefill_ragged + teacher-forced decode calls;
+    the oracle runs each sequence on its own."""
+    from oracle.model import BlockTransformerOracle, ragged_generate_logits
+    torch = gh.torch_mod()
+    B = len(lengths)
+    L = shape.block_len
+    w = synth.make_weights(shape, seed=1000 + seed)
+    stride = max(lengths) + G
+    toks = synth.make_tokens(batch=B, length=stride, vocab=shape.vocab, seed=2000 + seed)
+    padded = [n + ((L - n % L) % L if pad_id >= 0 else 0) for n in lengths]
+    model = gh.build_model(shape, w, max_batch=B, max_seq=max(padded) + G)
+    tok = torch.from_numpy(np.ascontiguousarray(toks)).cuda()
+    logits = torch.empty(G, B, shape.vocab, dtype=torch.float32, device="cuda")
+    nxt = torch.empty(G, B, dtype=torch.int32, device="cuda")
+    model.prefill_ragged(tok, lengths, pad_id, logits=logits[0], next_tokens=nxt[0])
+    for i in range(G - 1):
+        feed = torch.tensor([int(toks[b, lengths[b] + i]) for b in range(B)], dtype=torch.int32,
+                            device="cuda")
+        model.decode(feed, logits=logits[i + 1], next_tokens=nxt[i + 1])
+    model.sync()
+    assert model.position() == max(padded) + G - 1
+    gl, gn = logits.cpu().numpy(), nxt.cpu().numpy()
+    model.close()
+    o = BlockTransformerOracle(shape, {n: w.values(n) for n in w.names()})
+    ol = ragged_generate_logits(o, [toks[b, :lengths[b]] for b in range(B)],
+                                [toks[b, lengths[b]:] for b in range(B)], G,
+                                pad=pad_id >= 0, pad_id=max(pad_id, 0))
+    return gl, gn, ol
+
+
+@pytest.mark.parametrize("lb,pad_id,lengths", [
+    (4, 0, [37, 50, 64, 41]),        # left padding to a block boundary
+    (4, -1, [37, 41, 49, 53]),       # no padding, equal remainders (1)
+    (8, 11, [29, 64, 9, 40, 17]),    # left padding, L_B 8
+    (2, -1, [20, 34, 12]),           # no padding, aligned
+])
+def test_ragged_batch_matches_each_sequence_alone(lb, pad_id, lengths):
+    """Sequences of different prompt lengths in one batch: every sequence's
+    logits, at every step, match the oracle run on that sequence alone (its
+    own number of blocks in the block decoder's cache)."""
+    shape = synth.ModelShape(vocab=1000, d_model=256, n_heads=4, block_len=lb,
+                             n_block_layers=2, n_token_layers=2, prefix_len=1)
+    G = 2 * lb + 3
+    gl, gn, ol = _ragged_run(shape, lengths, pad_id, G, seed=9)
+    for b in range(len(lengths)):
+        for s in range(G):
+            e = gh.rel_l2(gl[s, b], ol[b][s])
+            assert e <= BF16_REL, (b, s, e)
+    assert np.array_equal(gn, gl.argmax(axis=-1))
+
+
+def test_ragged_batch_fp32_and_vanilla():
+    """fp32 (max |diff| <= 1e-4) ragged batch with padding, and the vanilla
+    L_B = 1 model on a ragged batch."""
+    wl = synth.WORKLOADS["tiny_fp32"]
+    gl, _, ol = _ragged_run(wl.shape, [33, 64, 50], 5, 9, seed=10)
+    for b in range(3):
+        assert np.abs(gl[:, b] - ol[b]).max() <= FP32_TOL, b
+    van = synth.ModelShape(vocab=800, d_model=256, n_heads=4, block_len=1, n_block_layers=3,
+                           n_token_layers=0, prefix_len=0, use_token_decoder=False)
+    gl, _, ol = _ragged_run(van, [21, 40, 33], -1, 6, seed=11)
+    for b in range(3):
+        for s in range(6):
+            assert gh.rel_l2(gl[s, b], ol[b][s]) <= BF16_REL, (b, s)
+
+
+def test_ragged_prefill_rejects_bad_lengths():
+    from hierarchical_global_local_b200 import native
+    torch = gh.torch_mod()
+    shape = synth.ModelShape(vocab=500, d_model=256, n_heads=4, block_len=4,
+                             n_block_layers=1, n_token_layers=1, prefix_len=1)
+    w = synth.make_weights(shape, seed=3)
+    m = gh.build_model(shape, w, 3, 80)
+    tok = torch.zeros(3, 40, dtype=torch.int32, device="cuda")
+    for lengths, pad in (([12, 13, 12], -1), ([0, 12, 12], 0), ([41, 12, 12], 0), ([12, 12, 12], 500)):
+        with pytest.raises(native.BtError) as ei:
+            m.prefill_ragged(tok, lengths, pad)
+        assert ei.value.code == native.BT_EINVAL, (lengths, pad)
+    m.close()
