@@ -275,7 +275,7 @@ def _ragged_run(shape, lengths, pad_id, G, seed):
                             device="cuda")
         model.decode(feed, logits=logits[i + 1], next_tokens=nxt[i + 1])
     model.sync()
-    assert model.position() == max(padded) + G - 1
+    assert model.position == max(padded) + G - 1
     gl, gn = logits.cpu().numpy(), nxt.cpu().numpy()
     model.close()
     o = BlockTransformerOracle(shape, {n: w.values(n) for n in w.names()})
