@@ -61,6 +61,7 @@
 #include <limits.h>
 
 #include "common.cuh"
+#include "gridsync.cuh"
 #include "kernels.h"
 #include "tc.cuh"
 
@@ -89,7 +90,6 @@ constexpr int ATT_SLOT_BYTES = 2 * ATT_CH * 64 * 2;              // K and V rows
 constexpr int ATT_BYTES = 4 * ATT_SLOTS * ATT_SLOT_BYTES;        // 96 KB
 constexpr int ATT_PART = 68;                                     // m, l, o[64], pad
 constexpr int ATT_MAX_CHUNKS = 32;                               // n_cap <= 1024
-constexpr long long BAR_CYCLES = 2000000000LL;  // ~1 s at 1.9 GHz
 constexpr int PRODUCER_SLEEP_NS = 128;  // back-off of the weight producer's slot waits
 constexpr int MMA_SLEEP_NS = 32;        // back-off of the MMA warp's waits (on the critical path)
 
@@ -106,11 +106,6 @@ struct Plan {
 
 __device__ __forceinline__ void wsync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
-__device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
-  unsigned v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
 
 template <typename T>
 __device__ __forceinline__ const T* layer_ptr(const T* base, int l, long long stride) {
@@ -121,7 +116,7 @@ __device__ __forceinline__ const T* layer_ptr(const T* base, int l, long long st
 // that the worker warps sharing their SM sub-partitions keep the issue
 // slots; gives up when the CTA has aborted
 __device__ bool wait_or_abort(uint64_t* bar, uint32_t parity, int* status, volatile int* s_abort,
-                              int sleep_ns) {
+                              int sleep_ns, long long limit) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   int n = 0;
@@ -129,7 +124,7 @@ __device__ bool wait_or_abort(uint64_t* bar, uint32_t parity, int* status, volat
     __nanosleep(sleep_ns);
     if ((++n & 63) == 0) {
       if (*s_abort) return false;
-      if (clock64() - t0 > BAR_CYCLES) {
+      if (clock64() - t0 > limit) {
         set_status(status, ST_WAIT_TIMEOUT);
         return false;
       }
@@ -138,33 +133,10 @@ __device__ bool wait_or_abort(uint64_t* bar, uint32_t parity, int* status, volat
   return true;
 }
 
-// Grid-wide barrier for the 128 worker threads of every CTA. `target` is
-// (barriers passed so far + 1) * gridDim.x. Returns false once the step has
-// been aborted (here or in another CTA).
-__device__ bool grid_sync(unsigned* bar, unsigned target, int* status, volatile int* s_abort) {
-  // activations written in this phase are read by TMA (async proxy) later
-  asm volatile("fence.proxy.async.global;" ::: "memory");
-  wsync();  // this CTA's writes of the phase are issued
-  if (threadIdx.x == 0 && !*s_abort) {
-    // release: this CTA's writes of the phase (ordered before by the CTA
-    // barrier above) are visible to any CTA that acquires the count
-    asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(&bar[0]) : "memory");
-    const long long t0 = clock64();
-    int n = 0;
-    while (ld_acquire(&bar[0]) < target) {
-      if ((++n & 63) == 0) {
-        if (ld_acquire(&bar[2]) != 0u) { *s_abort = 1; break; }
-        if (clock64() - t0 > BAR_CYCLES) {
-          atomicExch(&bar[2], 1u);
-          set_status(status, ST_WAIT_TIMEOUT);
-          *s_abort = 1;
-          break;
-        }
-      }
-    }
-  }
-  wsync();
-  return !*s_abort;
+// Grid-wide barrier for the 128 worker threads of every CTA (named barrier
+// 1), bounded by the launch's wait limit (gridsync.cuh).
+__device__ __forceinline__ bool grid_sync(const TokenStepArgs& a, unsigned target, volatile int* s_abort) {
+  return grid_barrier(a.bar, target, a.wait_cycles, a.status, s_abort, 1, 128);
 }
 
 // sum over the four worker warps (all 128 workers call it)
@@ -252,7 +224,7 @@ __device__ void ln_out(const float4* v, int D, float eps, const LnParams& p, bf1
 __device__ void producer(const CUtensorMap* mq, const CUtensorMap* mo, const CUtensorMap* ml,
                          const CUtensorMap* mqb, const CUtensorMap* mob, const CUtensorMap* mp,
                          const Plan& P, int Nt, int Nb, uint8_t* ring, uint64_t* full, uint64_t* empty,
-                         int* status, volatile int* s_abort) {
+                         int* status, volatile int* s_abort, long long limit) {
   const int G = gridDim.x, c = blockIdx.x;
   int it = 0;
   bool stop = false;
@@ -263,7 +235,7 @@ __device__ void producer(const CUtensorMap* mq, const CUtensorMap* mo, const CUt
   auto load = [&](const CUtensorMap* m, int x, int y, int z, bool three) {
     if (stop) return;
     const int s = it % P.stages;
-    if (it >= P.stages && !wait_or_abort(&empty[s], ((it / P.stages) + 1) & 1, status, s_abort, PRODUCER_SLEEP_NS)) {
+    if (it >= P.stages && !wait_or_abort(&empty[s], ((it / P.stages) + 1) & 1, status, s_abort, PRODUCER_SLEEP_NS, limit)) {
       stop = true;
       return;
     }
@@ -288,6 +260,14 @@ __device__ void producer(const CUtensorMap* mq, const CUtensorMap* mo, const CUt
       const int t = u % P.T2, sp = u / P.T2;
       for (int kb = 0; kb < P.nkbp; ++kb) load(mp, (sp * P.nkbp + kb) * 64, t * 128, 0, false);
     }
+  // The LM head's tiles of this CTA are prefetched into L2 while the
+  // token-decoder layers run (HBM is far from busy then), a share after each
+  // layer's loads, so that the LM-head phase streams them from L2.
+  uint64_t keep;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(keep));
+  const int my_lm = c < P.TL ? (P.TL - 1 - c) / G + 1 : 0;
+  const int lm_boxes = my_lm * P.nkbL;
+  int lm_done = 0;
   for (int l = 0; l < Nt && !stop; ++l) {
     for (int u = c; u < P.T1 * P.S1 && !stop; u += G) {
       const int t = u % P.T1, sp = u / P.T1;
@@ -296,6 +276,11 @@ __device__ void producer(const CUtensorMap* mq, const CUtensorMap* mo, const CUt
     for (int u = c; u < P.T2 * P.S2 && !stop; u += G) {
       const int t = u % P.T2, sp = u / P.T2;
       for (int kb = 0; kb < P.nkb2; ++kb) load(mo, (sp * P.nkb2 + kb) * 64, t * 128, l, true);
+    }
+    const int upto = (int)((long long)lm_boxes * (l + 1) / Nt);
+    for (; lm_done < upto && !stop; ++lm_done) {
+      const int t = c + (lm_done / P.nkbL) * G, kb = lm_done % P.nkbL;
+      tc::tma_prefetch_2d(ml, kb * 64, t * 128, keep);
     }
   }
   for (int t = c; t < P.TL && !stop; t += G)
@@ -388,16 +373,16 @@ __device__ void gemm_phase(const Plan& P, int T, int S, int nkb, const CUtensorM
 // MMA warp (one thread): the same unit sequence as the workers and the
 // producer. Waits for staged activations and a drained accumulator.
 __device__ void mma_issuer(const Plan& P, int Nt, int Nb, uint8_t* ring, const uint8_t* act, uint32_t tmem,
-                           const Sync& y, int* status, volatile int* s_abort) {
+                           const Sync& y, int* status, volatile int* s_abort, long long limit) {
   const int G = gridDim.x, c = blockIdx.x;
   int it = 0, na = 0, nu = 0;
   auto unit = [&](int nkb, bool need_act) -> bool {
     if (need_act) {
-      if (!wait_or_abort(y.act_full, na & 1, status, s_abort, MMA_SLEEP_NS)) return false;
+      if (!wait_or_abort(y.act_full, na & 1, status, s_abort, MMA_SLEEP_NS, limit)) return false;
       ++na;
     }
     const int buf = nu & 1;
-    if (nu >= 2 && !wait_or_abort(&y.acc_empty[buf], ((nu >> 1) + 1) & 1, status, s_abort, MMA_SLEEP_NS))
+    if (nu >= 2 && !wait_or_abort(&y.acc_empty[buf], ((nu >> 1) + 1) & 1, status, s_abort, MMA_SLEEP_NS, limit))
       return false;
     tc::fence_after();
     issue_unit(P, nkb, ring, act, tmem + (uint32_t)(buf * 64), y.full, y.empty, &y.acc_full[buf], it, status);
@@ -1108,9 +1093,10 @@ token_step_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
   if (warp == 4) {
     // weights do not depend on earlier kernels: no wait before streaming them
     if ((threadIdx.x & 31) == 0)
-      producer(&mq, &mo, &ml, &mqb, &mob, &mp, P, a.Nt, Nb, ring, full, empty, a.status, &s_abort);
+      producer(&mq, &mo, &ml, &mqb, &mob, &mp, P, a.Nt, Nb, ring, full, empty, a.status, &s_abort,
+               a.wait_cycles);
   } else if (warp == 5) {
-    if ((threadIdx.x & 31) == 0) mma_issuer(P, a.Nt, Nb, ring, act, tmem, y, a.status, &s_abort);
+    if ((threadIdx.x & 31) == 0) mma_issuer(P, a.Nt, Nb, ring, act, tmem, y, a.status, &s_abort, a.wait_cycles);
   } else {
     pdl_wait();
     const int G = gridDim.x;
@@ -1127,16 +1113,16 @@ token_step_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
       const int bpos = a.dstate[2];
       int katt = 0;
       block_ingest_phase(a, jb, red);
-      ok = grid_sync(a.bar, ++nb * G, a.status, &s_abort);
+      ok = grid_sync(a, ++nb * G, &s_abort);
       for (int l = 0; ok && l < Nb; ++l) {
         gemm_phase(P, P.T1, P.S1, P.nkb1, &mx1, [=](int t) { return t * 128 < 3 * D ? 0 : D; }, a.B, a.p1,
                    act, tmem, y, na, nu, a.status);
-        if (!(ok = grid_sync(a.bar, ++nb * G, a.status, &s_abort))) break;
+        if (!(ok = grid_sync(a, ++nb * G, &s_abort))) break;
         block_attention_phase(a, P, l, bpos, act, att_bar, q_s, katt);
-        if (!(ok = grid_sync(a.bar, ++nb * G, a.status, &s_abort))) break;
+        if (!(ok = grid_sync(a, ++nb * G, &s_abort))) break;
         gemm_phase(P, P.T2, P.S2, P.nkb2, &ma2, [](int) { return 0; }, a.B, a.p2, act, tmem, y, na, nu,
                    a.status);
-        if (!(ok = grid_sync(a.bar, ++nb * G, a.status, &s_abort))) break;
+        if (!(ok = grid_sync(a, ++nb * G, &s_abort))) break;
         if (l + 1 < Nb)
           reduce_ln(a, P, a.h_b, layer_ptr(a.bb_o2, l, a.layer_stride), P.S2, true,
                     layer_ptr(a.bln1_g, l + 1, a.layer_stride), layer_ptr(a.bln1_b, l + 1, a.layer_stride),
@@ -1145,37 +1131,37 @@ token_step_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
         else
           reduce_ln(a, P, a.h_b, layer_ptr(a.bb_o2, l, a.layer_stride), P.S2, true, a.lnb_g, a.lnb_b,
                     nullptr, nullptr, a.xf, red);
-        ok = grid_sync(a.bar, ++nb * G, a.status, &s_abort);
+        ok = grid_sync(a, ++nb * G, &s_abort);
       }
       if (ok) {
         gemm_phase(P, P.T2, P.Sp, P.nkbp, &mxf, [](int) { return 0; }, a.B, a.p2, act, tmem, y, na, nu,
                    a.status);
-        ok = grid_sync(a.bar, ++nb * G, a.status, &s_abort);
+        ok = grid_sync(a, ++nb * G, &s_abort);
       }
       if (ok) {
         reduce_ln(a, P, a.h, a.b_prefix, P.Sp, false, a.ln1_g, a.ln1_b, a.ln2_g, a.ln2_b, a.x1, red);
-        ok = grid_sync(a.bar, ++nb * G, a.status, &s_abort);
+        ok = grid_sync(a, ++nb * G, &s_abort);
       }
     } else {
       ingest_phase(a, jb, red);
-      ok = grid_sync(a.bar, ++nb * G, a.status, &s_abort);
+      ok = grid_sync(a, ++nb * G, &s_abort);
     }
     for (int l = 0; ok && l < a.Nt; ++l) {
       // G1: q|k|v tiles read LN1(h), fc1 tiles LN2(h)
       gemm_phase(P, P.T1, P.S1, P.nkb1, &mx1, [=](int t) { return t * 128 < 3 * D ? 0 : D; }, a.B, a.p1,
                  act, tmem, y, na, nu, a.status);
-      if (!(ok = grid_sync(a.bar, ++nb * G, a.status, &s_abort))) break;
+      if (!(ok = grid_sync(a, ++nb * G, &s_abort))) break;
       r1_phase(a, P, l, pos);
-      if (!(ok = grid_sync(a.bar, ++nb * G, a.status, &s_abort))) break;
+      if (!(ok = grid_sync(a, ++nb * G, &s_abort))) break;
       gemm_phase(P, P.T2, P.S2, P.nkb2, &ma2, [](int) { return 0; }, a.B, a.p2, act, tmem, y, na, nu,
                  a.status);
-      if (!(ok = grid_sync(a.bar, ++nb * G, a.status, &s_abort))) break;
+      if (!(ok = grid_sync(a, ++nb * G, &s_abort))) break;
       r2_phase(a, P, l, red);
-      ok = grid_sync(a.bar, ++nb * G, a.status, &s_abort);
+      ok = grid_sync(a, ++nb * G, &s_abort);
     }
     if (ok) {
       lm_phase(a, P, &mxf, act, tmem, y, na, nu, s_arg);
-      ok = grid_sync(a.bar, ++nb * G, a.status, &s_abort);
+      ok = grid_sync(a, ++nb * G, &s_abort);
     }
     if (ok) {
       argmax_phase(a, P);
@@ -1193,16 +1179,8 @@ token_step_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
   tc::fence_before();
   __syncthreads();
   if (warp == 0) tc::tmem_free(tmem, TMEM_COLS);
-  if (threadIdx.x == 0) {
-    // the last CTA out resets the barrier counter for the next launch: every
-    // CTA counts itself here only after its last barrier wait
-    __threadfence();
-    if (atomicAdd(&a.bar[1], 1u) == gridDim.x - 1) {
-      a.bar[0] = 0u;
-      a.bar[1] = 0u;
-      __threadfence();
-    }
-  }
+  // every CTA counts itself out only after its last barrier wait
+  if (threadIdx.x == 0) grid_exit(a.bar);
 }
 
 // ---- host side -----------------------------------------------------------------

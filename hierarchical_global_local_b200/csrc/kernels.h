@@ -234,6 +234,7 @@ struct TokenStepArgs {
   float *p1, *p2;    // split-K partials (token_step_scratch_floats)
   unsigned* bar;     // 3 words, zero before the first launch
   int* status;
+  long long wait_cycles;  // bound of every wait of the launch (SM clock cycles)
   // Block step (block = 1): the fed token completes a block. The block
   // embedding, every block-decoder layer (decode attention over the block
   // cache, the new entry appended at dstate[2]), LN_b and the prefix

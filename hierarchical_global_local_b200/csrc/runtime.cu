@@ -130,6 +130,9 @@ struct bt_model {
   // pad ids, row_len [B_max] prompt tokens, row_col0 [B_max] first trailing token
   int *row_lag = nullptr, *row_pad = nullptr, *row_len = nullptr, *row_col0 = nullptr;
   bool ragged = false;
+  // bound of the waits inside persistent kernels (SM clock cycles): ~1 s at
+  // B200 clocks; BT_WAIT_CYCLES (read at bt_create) overrides it
+  long long wait_cycles = 2000000000LL;
   int *dstate = nullptr, *status = nullptr;
   float2* rope_tab = nullptr;
   void* attn_scratch = nullptr;
@@ -335,6 +338,10 @@ int bt_create(const bt_config* cfg, const bt_weights* w, void* ws, size_t ws_byt
   if (ws_bytes < need) { delete m; return BT_EWORKSPACE; }
   const char* ng = getenv("BT_NO_GRAPH");
   m->use_graphs = !(ng && ng[0] == '1');
+  if (const char* wc = getenv("BT_WAIT_CYCLES")) {
+    const long long v = atoll(wc);
+    if (v > 0) m->wait_cycles = v;
+  }
   if (!w->blk_emb_dev || !w->lnf_b_g_dev || !w->lnf_b_b_dev || !w->w_lm_dev ||
       (d.Nb > 0 && !w->block_layers) || (d.Nt > 0 && !w->token_layers) ||
       (d.tokdec && (!w->w_prefix_dev || !w->b_prefix_dev || !w->tok_emb_dev ||
@@ -730,6 +737,7 @@ static int run_token_step(bt_model* m, int B, bool ingest, PosSpec pos, const in
   a.h = m->h_t; a.x1 = (bf16*)m->x1; a.a2 = (bf16*)m->a2; a.xf = (bf16*)m->xf;
   a.logits = want_logits ? m->logits : nullptr; a.next = m->next; a.arg_part = m->arg_part;
   a.p1 = m->ts_p1; a.p2 = m->ts_p2; a.bar = m->ts_bar; a.status = m->status;
+  a.wait_cycles = m->wait_cycles;
   const void *wqb = nullptr, *wob = nullptr;
   if (block) {
     const LayerW& b0 = m->blk[0];

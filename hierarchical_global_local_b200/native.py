@@ -102,6 +102,8 @@ def lib() -> ctypes.CDLL:
                                         c_float, c_void_p, c_void_p]),
             "bt_op_embed_prompt": (c_int, [c_int, c_void_p, c_int, c_int, c_int, c_void_p, c_int,
                                            c_int, c_void_p, c_void_p, c_void_p]),
+            "bt_op_grid_barrier_selftest": (c_int, [c_int, c_int, ctypes.c_longlong, c_void_p, c_void_p,
+                                                    c_void_p, c_void_p]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -121,7 +123,7 @@ def exported_symbols():
         "bt_op_decode_attention_noalloc",
         "bt_op_prefill_attention", "bt_op_prefill_attention_tc",
         "bt_op_linear_scratch_bytes", "bt_op_linear",
-        "bt_op_layernorm", "bt_op_embed_prompt"]
+        "bt_op_layernorm", "bt_op_embed_prompt", "bt_op_grid_barrier_selftest"]
 
 
 def _strerror(code: int) -> str:
@@ -380,3 +382,17 @@ def embed_prompt(tokens, table, L: int, D: int, status=None):
     _check(lib().bt_op_embed_prompt(_dt(table), tokens.data_ptr(), B, T, L, table.data_ptr(), V, D,
                                     h.data_ptr(), _ptr(status), _stream()), "bt_op_embed_prompt")
     return h
+
+
+def grid_barrier_selftest(rounds: int, withhold_cta: int = -1, wait_cycles: int = 2_000_000_000):
+    """Run the bounded grid-barrier self-test; returns (status word, barriers
+    passed summed over CTAs, the three barrier words) after synchronising."""
+    import torch
+    words = torch.zeros(3, dtype=torch.int32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    passed = torch.zeros(1, dtype=torch.int32, device="cuda")
+    _check(lib().bt_op_grid_barrier_selftest(rounds, withhold_cta, wait_cycles, words.data_ptr(),
+                                             status.data_ptr(), passed.data_ptr(), _stream()),
+           "bt_op_grid_barrier_selftest")
+    torch.cuda.synchronize()
+    return int(status.item()), int(passed.item()), [int(x) for x in words.tolist()]

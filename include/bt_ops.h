@@ -98,6 +98,24 @@ BT_API int bt_op_embed_prompt(int dtype, const int32_t *tokens_dev, int B, int T
                        const void *table_dev, int V, int D, float *h_dev, int32_t *status_dev,
                        void *stream);
 
+/* Self-test of the bounded grid-wide barrier that the persistent decode kernel
+ * uses between its phases (failure detection without a GPU fault; the pages
+ * have no counterpart). Launches one CTA per SM, cooperatively, each passing
+ * `rounds` barriers.
+ *   words_dev   3 uint32, zero before the call: arrival counter, exit counter,
+ *               abort word. The kernel leaves the counters zero; a timeout
+ *               leaves the abort word set (clear it before reusing the words).
+ *   withhold_cta -1, or a CTA index (< number of SMs) that does not arrive at
+ *               the first barrier: every CTA's wait then runs out after
+ *               wait_cycles SM clock cycles, ST_WAIT_TIMEOUT (2) is or-ed into
+ *               *status_dev, the abort word is set, and every CTA returns.
+ *   passed_dev  int, zero before the call; receives the sum over CTAs of the
+ *               barriers passed (rounds * number of SMs when nothing ran out).
+ * Returns BT_ENOTSUP if the device cannot launch cooperatively. */
+BT_API int bt_op_grid_barrier_selftest(int rounds, int withhold_cta, long long wait_cycles,
+                                       unsigned *words_dev, int *status_dev, int *passed_dev,
+                                       void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -95,3 +95,55 @@ def test_out_of_range_token_is_reported_once_and_the_model_recovers(where):
     f.sync()
     f.close()
     assert torch.equal(lg, lf)
+
+
+def test_grid_barrier_passes_every_round():
+    """The bounded grid barrier of the persistent decode kernel: 200 rounds
+    with every CTA arriving pass with a clean status and leave the counters
+    ready for the next launch."""
+    from hierarchical_global_local_b200 import native
+    torch = gh.torch_mod()
+    G = torch.cuda.get_device_properties(0).multi_processor_count
+    st, passed, words = native.grid_barrier_selftest(200)
+    assert st == 0 and passed == 200 * G and words == [0, 0, 0]
+
+
+def test_grid_barrier_wait_runs_out_without_a_fault():
+    """One CTA withholds its arrival: every wait runs out after ~1e5 cycles,
+    the kernel returns with ST_WAIT_TIMEOUT in the status word and the abort
+    word set, and the context stays usable (a clean run follows)."""
+    import time
+    from hierarchical_global_local_b200 import native
+    torch = gh.torch_mod()
+    G = torch.cuda.get_device_properties(0).multi_processor_count
+    t0 = time.perf_counter()
+    st, passed, words = native.grid_barrier_selftest(50, withhold_cta=G // 2, wait_cycles=100_000)
+    assert time.perf_counter() - t0 < 10.0
+    assert st & 2, st                        # ST_WAIT_TIMEOUT
+    assert passed == 0
+    assert words[2] == 1 and words[0] == 0 and words[1] == 0
+    st, passed, words = native.grid_barrier_selftest(100)
+    assert st == 0 and passed == 100 * G
+
+
+def test_model_runs_with_a_short_wait_bound(monkeypatch):
+    """BT_WAIT_CYCLES sets the bound of every wait inside the persistent
+    decode kernel; a bound far below a second (1e6 cycles) is still far
+    above any barrier of a healthy step, so logits are unchanged."""
+    torch = gh.torch_mod()
+    B, T = 2, 16
+    toks = synth.make_tokens(batch=B, length=T + 6, vocab=SHAPE.vocab, seed=53)
+    good = torch.from_numpy(np.ascontiguousarray(toks)).cuda()
+    out = []
+    for bound in (None, "1000000"):
+        if bound:
+            monkeypatch.setenv("BT_WAIT_CYCLES", bound)
+        m, _ = _model(B, 40)
+        lg = torch.empty(6, B, SHAPE.vocab, device="cuda")
+        m.prefill(good[:, :T].contiguous(), logits=lg[0])
+        for i in range(5):
+            m.decode(good[:, T + i].contiguous(), logits=lg[i + 1])
+        m.sync()
+        m.close()
+        out.append(lg)
+    assert torch.equal(out[0], out[1])
