@@ -235,6 +235,12 @@ struct TokenStepArgs {
   unsigned* bar;     // 3 words, zero before the first launch
   int* status;
   long long wait_cycles;  // bound of every wait of the launch (SM clock cycles)
+  // token_step2 only: per-(row, 128-feature tile) (mean, sum of squared
+  // deviations) of h [B][D/128]; the L2 persisting window over the local
+  // caches (bytes 0 = none)
+  float2* hstat;
+  void* l2_window_base;
+  size_t l2_window_bytes;
   // Block step (block = 1): the fed token completes a block. The block
   // embedding, every block-decoder layer (decode attention over the block
   // cache, the new entry appended at dstate[2]), LN_b and the prefix
@@ -263,6 +269,18 @@ size_t token_step_scratch_floats(int B, int D, int which, int H = 0, int n_cap =
 cudaError_t launch_token_step(const TokenStepArgs& a, const void* w_qkv1, const void* w_o2,
                               const void* w_lm, const void* w_qkv1_b, const void* w_o2_b,
                               const void* w_prefix, cudaStream_t s);
+
+// The token-decoder half of a decode step as one persistent kernel with no
+// grid-wide barrier (token_step.cu): bf16, B <= 64, d_head in {32, 64, 128},
+// rotary on none or the first d_head/4 dims, local window <= 16 rows, any
+// prefix length. a.bar: token_step2_counter_bytes(D) bytes, zero before the
+// first launch (a launch leaves them zero unless a wait ran out); a.p1, a.p2,
+// a.hstat: token_step2_scratch_floats(B, D, 1 | 2 | 3) floats.
+int token_step2_supported(int dt, int B, int D, int H, int rot, int V, int Nt, int l_cap);
+size_t token_step2_counter_bytes(int D);
+size_t token_step2_scratch_floats(int B, int D, int which);
+cudaError_t launch_token_step2(const TokenStepArgs& a, const void* w_qkv1, const void* w_o2, const void* w_lm,
+                               cudaStream_t s);
 
 // ---- LM head argmax ---------------------------------------------------------
 // next[b] = argmax_v logits[b, v] (lowest id among ties).

@@ -17,6 +17,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <algorithm>
 #include <string>
 #include <vector>
 
@@ -144,6 +145,10 @@ struct bt_model {
   unsigned* ts_bar = nullptr;                // fused token step: grid-barrier words
   float* ts_att = nullptr;                   // fused block step: decode-attention partials
   int* ts_cnt = nullptr;                     // fused block step: merge counters [B_max * H]
+  unsigned* ts2_ctr = nullptr;               // token_step2: counters
+  size_t ts2_ctr_bytes = 0;
+  float2* ts_hstat = nullptr;                // token_step2: per-(row, tile) statistics of h
+  size_t l2_window = 0;                      // bytes of the local caches kept in L2 (0: none)
   GemmScratch gs{};
   int B = 0, t = 0;
   bool prefilled = false;
@@ -255,11 +260,16 @@ static size_t carve(bt_model* m, const Dims& d, void* ws) {
   m->arg_part = (float2*)c.take((size_t)((d.V + 127) / 128) * d.Bmax * sizeof(float2));
   m->ln_cnt = (int*)c.take((size_t)d.Bmax * (d.P > 1 ? d.P : 1) * sizeof(int));
   if (d.tokdec && d.Bmax > 0) {
-    m->ts_p1 = (float*)c.take(token_step_scratch_floats(d.Bmax, d.D, 1) * 4);
-    m->ts_p2 = (float*)c.take(token_step_scratch_floats(d.Bmax, d.D, 2) * 4);
+    m->ts_p1 = (float*)c.take(std::max(token_step_scratch_floats(d.Bmax, d.D, 1),
+                                       token_step2_scratch_floats(d.Bmax, d.D, 1)) * 4);
+    m->ts_p2 = (float*)c.take(std::max(token_step_scratch_floats(d.Bmax, d.D, 2),
+                                       token_step2_scratch_floats(d.Bmax, d.D, 2)) * 4);
     m->ts_bar = (unsigned*)c.take(64);
     m->ts_att = (float*)c.take(token_step_scratch_floats(d.Bmax, d.D, 3, d.H, d.n_cap) * 4);
     m->ts_cnt = (int*)c.take((size_t)d.Bmax * d.H * sizeof(int));
+    m->ts2_ctr_bytes = token_step2_counter_bytes(d.D);
+    m->ts2_ctr = (unsigned*)c.take(m->ts2_ctr_bytes);
+    m->ts_hstat = (float2*)c.take(token_step2_scratch_floats(d.Bmax, d.D, 3) * 4);
   }
   m->vt_ld = (d.n_cap + 63) / 64 * 64;
   m->vtr = c.take((size_t)d.Bmax * D * m->vt_ld * eb);
@@ -380,6 +390,27 @@ int bt_create(const bt_config* cfg, const bt_weights* w, void* ws, size_t ws_byt
   BT_TRYC(cudaMemsetAsync(m->ln_cnt, 0, (size_t)d.Bmax * (d.P > 1 ? d.P : 1) * sizeof(int), st));
   if (m->ts_bar) BT_TRYC(cudaMemsetAsync(m->ts_bar, 0, 64, st));
   if (m->ts_cnt) BT_TRYC(cudaMemsetAsync(m->ts_cnt, 0, (size_t)d.Bmax * d.H * sizeof(int), st));
+  if (m->ts2_ctr) BT_TRYC(cudaMemsetAsync(m->ts2_ctr, 0, m->ts2_ctr_bytes, st));
+  {
+    // The token decoder's local caches (K and V of every layer, at most
+    // P + L_B - 1 rows per sequence and head) stay in L2 between the decode
+    // calls that read them: a persisting access-policy window on the fused
+    // token-step launches, with this context's persisting set-aside sized to
+    // it when the device allows (BT_L2_WINDOW=0 turns it off).
+    const char* env = getenv("BT_L2_WINDOW");
+    const size_t bytes = d.Nt > 0 ? 2 * m->kt_layer * d.Nt * d.eb : 0;
+    int dev = 0, max_persist = 0, max_window = 0;
+    if (bytes > 0 && !(env && env[0] == '0') && cudaGetDevice(&dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&max_persist, cudaDevAttrMaxPersistingL2CacheSize, dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&max_window, cudaDevAttrMaxAccessPolicyWindowSize, dev) == cudaSuccess &&
+        bytes <= (size_t)max_persist && bytes <= (size_t)max_window) {
+      size_t cur = 0;
+      if (cudaDeviceGetLimit(&cur, cudaLimitPersistingL2CacheSize) == cudaSuccess &&
+          (cur >= bytes || cudaDeviceSetLimit(cudaLimitPersistingL2CacheSize, bytes) == cudaSuccess))
+        m->l2_window = bytes;
+      cudaGetLastError();
+    }
+  }
   BT_TRYC(cudaStreamCreateWithFlags(&m->cap_stream, cudaStreamNonBlocking));
   if (d.dt == BT_BF16) BT_TRYC(gemm_tc_prepare());
   BT_TRYC(attn_prepare());
@@ -666,17 +697,12 @@ static int enqueue_decode_fused(bt_model* m, bool block_step, bool greedy, bool 
 // one persistent kernel where the shape allows; BT_DECODE_TOKEN_STEP=chain
 // keeps the kernel-per-operation schedule instead (read when a step kind is
 // first recorded).
-static bool token_step_fused(const bt_model* m, int B) {
-  const Dims& d = m->d;
-  const char* env = getenv("BT_DECODE_TOKEN_STEP");
-  if (env && strcmp(env, "chain") == 0) return false;
-  if (!d.tokdec || d.Nt < 1 || !m->ts_bar) return false;
-  if (!token_step_supported(d.dt, B, d.D, d.H, d.rot, d.V, d.Nt, d.P, d.l_cap)) return false;
-  // layer l's parameters at a fixed stride from layer 0's
-  const long long ls = d.Nt > 1 ? (long long)((uint8_t*)m->tok[1].w_qkv1 - (uint8_t*)m->tok[0].w_qkv1) : 0;
-  for (int l = 0; l < d.Nt; ++l) {
-    const LayerW& w = m->tok[l];
-    const LayerW& w0 = m->tok[0];
+// Layer l's parameters at a fixed stride from layer 0's (the fused kernels
+// address layers by that stride).
+static bool uniform_layers(const std::vector<LayerW>& v, long long ls) {
+  for (size_t l = 0; l < v.size(); ++l) {
+    const LayerW& w = v[l];
+    const LayerW& w0 = v[0];
     auto at = [&](const void* p, const void* p0) {
       return (const uint8_t*)p == (const uint8_t*)p0 + (long long)l * ls;
     };
@@ -687,6 +713,28 @@ static bool token_step_fused(const bt_model* m, int B) {
   }
   return true;
 }
+
+// Which fused kernel runs the token-decoder half of a decode call: 1 = the
+// grid-barrier kernel (decode_step.cu, prefix length 1), 2 = the
+// counter-synchronised kernel (token_step.cu, any prefix length), 0 = none
+// (kernel per operation). BT_DECODE_TOKEN_STEP=chain | v1 | v2 (read when a
+// step kind is first recorded) forces one of them.
+static int token_step_kind(const bt_model* m, int B) {
+  const Dims& d = m->d;
+  const char* env = getenv("BT_DECODE_TOKEN_STEP");
+  if (env && strcmp(env, "chain") == 0) return 0;
+  if (!d.tokdec || d.Nt < 1 || !m->ts_bar) return 0;
+  const long long ls = d.Nt > 1 ? (long long)((uint8_t*)m->tok[1].w_qkv1 - (uint8_t*)m->tok[0].w_qkv1) : 0;
+  if (!uniform_layers(m->tok, ls)) return 0;
+  const bool only1 = env && strcmp(env, "v1") == 0, only2 = env && strcmp(env, "v2") == 0;
+  const bool ok1 = token_step_supported(d.dt, B, d.D, d.H, d.rot, d.V, d.Nt, d.P, d.l_cap);
+  const bool ok2 = token_step2_supported(d.dt, B, d.D, d.H, d.rot, d.V, d.Nt, d.l_cap);
+  if (only1) return ok1 ? 1 : 0;
+  if (only2) return ok2 ? 2 : 0;
+  return ok1 ? 1 : (ok2 ? 2 : 0);
+}
+
+static bool token_step_fused(const bt_model* m, int B) { return token_step_kind(m, B) != 0; }
 
 // The block-step form of the same kernel (block embedding, block-decoder
 // layers with the decode attention as one of its phases, LN_b and the
@@ -753,6 +801,14 @@ static int run_token_step(bt_model* m, int B, bool ingest, PosSpec pos, const in
     wqb = b0.w_qkv1; wob = b0.w_o2;
   }
   ProfScope p(m, s, block ? BT_K_BLOCK_STEP : BT_K_TOKEN_STEP, B, d.V, d.D);
+  if (!block && token_step_kind(m, B) == 2) {
+    a.bar = m->ts2_ctr;
+    a.hstat = m->ts_hstat;
+    a.l2_window_base = m->kt;
+    a.l2_window_bytes = m->l2_window;
+    BT_CUDA(launch_token_step2(a, w0.w_qkv1, w0.w_o2, m->w_lm, s));
+    return BT_OK;
+  }
   BT_CUDA(launch_token_step(a, w0.w_qkv1, w0.w_o2, m->w_lm, wqb, wob, block ? m->w_prefix : nullptr, s));
   return BT_OK;
 }
@@ -782,13 +838,21 @@ static int enqueue_decode_token_step(bt_model* m, bool block_step, bool greedy, 
     BT_CUDA(launch_ln_rows(d.dt, m->h_b, B, 1, 0, d.D, m->lnf_b_g, m->lnf_b_b, m->cfg.ln_eps, m->xf, s));
   }
   {
-    // the prefix row h_t[b] = W_p c_b + b_p, then the token decoder over it
-    ProfScope p(m, s, BT_K_GEMM, B, d.D, d.D);
-    Epi ep{EPI_F32, m->h_t, d.D, nullptr, 0, m->b_prefix, 0, d.D};
-    BT_CUDA(launch_gemm(d.dt, m->xf, d.D, m->w_prefix, d.D, B, d.D, d.D, 1 << 30, 0, ep, m->gs,
+    // the prefix rows h_t[b * P + p] = (W_p c_b + b_p)[p D, (p + 1) D)
+    ProfScope p(m, s, BT_K_GEMM, B, d.P * d.D, d.D);
+    Epi ep{EPI_F32, m->h_t, d.P * d.D, nullptr, 0, m->b_prefix, 0, d.D};
+    BT_CUDA(launch_gemm(d.dt, m->xf, d.D, m->w_prefix, d.D, B, d.P * d.D, d.D, 1 << 30, 0, ep, m->gs,
                         m->status, s));
   }
-  return run_token_step(m, B, false, PosSpec{nullptr, POS_ZERO, 0, 1}, src, want_logits, s);
+  if (d.P == 1) return run_token_step(m, B, false, PosSpec{nullptr, POS_ZERO, 0, 1}, src, want_logits, s);
+  // several prefix rows: the token decoder over them as separate kernels
+  int rc = run_token_decoder(m, B, PosSpec{nullptr, POS_ZERO, 0, d.P}, s);
+  if (rc != BT_OK) return rc;
+  rc = run_head(m, B, want_logits, s);
+  if (rc != BT_OK) return rc;
+  ProfScope p(m, s, BT_K_OTHER, 1, 0, 0);
+  BT_CUDA(launch_advance(m->dstate, d.L, s));
+  return BT_OK;
 }
 
 // the body of one decode call (captured into a graph or run directly)
@@ -893,6 +957,7 @@ static int prefill_impl(bt_model* m, const int32_t* tokens, int T_stride, int B,
   // and the fused token step's barrier words (an aborted step leaves them set)
   if (m->ts_bar) BT_CUDA(cudaMemsetAsync(m->ts_bar, 0, 64, s));
   if (m->ts_cnt) BT_CUDA(cudaMemsetAsync(m->ts_cnt, 0, (size_t)d.Bmax * d.H * sizeof(int), s));
+  if (m->ts2_ctr) BT_CUDA(cudaMemsetAsync(m->ts2_ctr, 0, m->ts2_ctr_bytes, s));
   const long long k0 = launch_count();
   BT_CUDA(launch_set_state(m->dstate, T, d.L, s));
   {

@@ -160,13 +160,20 @@ def _launches(model):
     return int(native.lib().bt_kernel_launches(model._h))
 
 
-@pytest.mark.parametrize("lb,B", [(4, 3), (8, 17), (2, 64)])
-def test_fused_token_step_matches_oracle_and_chain(lb, B, monkeypatch):
-    """The token-decoder half of a decode step as one persistent kernel: a
-    token step is a single launch, its logits match the oracle, and they
-    agree with the kernel-per-operation schedule on the same inputs."""
-    shape = synth.ModelShape(vocab=3000, d_model=256, n_heads=4, block_len=lb,
-                             n_block_layers=2, n_token_layers=3, prefix_len=1)
+@pytest.mark.parametrize("lb,B,D,H,P,kind", [
+    (4, 3, 256, 4, 1, "v2"), (8, 17, 256, 4, 1, "v2"), (2, 64, 256, 4, 1, "v2"),
+    (4, 33, 512, 4, 2, "v2"),      # d_head 128, two prefix rows
+    (8, 64, 256, 8, 1, "v2"),      # d_head 32, window of 8 rows
+    (4, 5, 128, 4, 3, "v2"),       # one tile per GEMM row block, three prefix rows
+    (4, 3, 256, 4, 1, "v1"), (8, 17, 256, 4, 1, "v1")])
+def test_fused_token_step_matches_oracle_and_chain(lb, B, D, H, P, kind, monkeypatch):
+    """The token-decoder half of a decode step as one persistent kernel (v1:
+    grid barriers; v2: counter-synchronised, any prefix length): a token step is a
+    single launch, its logits match the oracle, and they agree with the
+    kernel-per-operation schedule on the same inputs."""
+    monkeypatch.setenv("BT_DECODE_TOKEN_STEP", kind)
+    shape = synth.ModelShape(vocab=3000, d_model=D, n_heads=H, block_len=lb,
+                             n_block_layers=2, n_token_layers=3, prefix_len=P)
     T, G = 6 * lb, 3 * lb + 2
     w = synth.make_weights(shape, seed=31)
     toks = synth.make_tokens(batch=B, length=T + G, vocab=shape.vocab, seed=32)
