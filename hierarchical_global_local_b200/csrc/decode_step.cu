@@ -241,6 +241,7 @@ __device__ void producer(const CUtensorMap* mq, const CUtensorMap* mo, const CUt
     }
     mbar_arrive_expect_tx(&full[s], TILE_BYTES);
     if (three) tc::tma_load_3d_hint(ring + (size_t)s * TILE_BYTES, m, x, y, z, &full[s], policy);
+    else if (m == ml) tc::tma_load_2d(ring + (size_t)s * TILE_BYTES, m, x, y, &full[s]);  // LM head: the launch's L2 window decides
     else tc::tma_load_2d_hint(ring + (size_t)s * TILE_BYTES, m, x, y, &full[s], policy);
     ++it;
   };
@@ -1390,13 +1391,25 @@ cudaError_t launch_token_step(const TokenStepArgs& a, const void* w_qkv1, const 
   cfg.stream = s;
   // cooperative: the driver guarantees that every CTA is resident at once
   // (the grid barriers rely on it) or refuses the launch
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeCooperative;
-  attr[0].val.cooperative = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[3];
+  int na = 0;
+  attr[na].id = cudaLaunchAttributeCooperative;
+  attr[na++].val.cooperative = 1;
+  if (pdl_enabled()) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na++].val.programmaticStreamSerializationAllowed = 1;
+  }
+  if (a.l2_window_bytes > 0) {
+    // the re-read regions (LM head, local caches) persist in L2
+    attr[na].id = cudaLaunchAttributeAccessPolicyWindow;
+    attr[na].val.accessPolicyWindow.base_ptr = a.l2_window_base;
+    attr[na].val.accessPolicyWindow.num_bytes = a.l2_window_bytes;
+    attr[na].val.accessPolicyWindow.hitRatio = a.l2_hit_ratio;
+    attr[na].val.accessPolicyWindow.hitProp = cudaAccessPropertyPersisting;
+    attr[na++].val.accessPolicyWindow.missProp = cudaAccessPropertyStreaming;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = pdl_enabled() ? 2 : 1;
+  cfg.numAttrs = na;
   if (a.block) e = cudaLaunchKernelEx(&cfg, token_step_kernel<true>, mq, mo, ml, mx1, ma2, mxf, mqb, mob, mp, a, P);
   else e = cudaLaunchKernelEx(&cfg, token_step_kernel<false>, mq, mo, ml, mx1, ma2, mxf, mqb, mob, mp, a, P);
   note_launch();

@@ -236,11 +236,12 @@ struct TokenStepArgs {
   int* status;
   long long wait_cycles;  // bound of every wait of the launch (SM clock cycles)
   // token_step2 only: per-(row, 128-feature tile) (mean, sum of squared
-  // deviations) of h [B][D/128]; the L2 persisting window over the local
-  // caches (bytes 0 = none)
+  // deviations) of h [B][D/128]. Both kernels: an L2 persisting access-policy
+  // window for the launch (bytes 0 = none)
   float2* hstat;
   void* l2_window_base;
   size_t l2_window_bytes;
+  float l2_hit_ratio;
   // Block step (block = 1): the fed token completes a block. The block
   // embedding, every block-decoder layer (decode attention over the block
   // cache, the new entry appended at dstate[2]), LN_b and the prefix

@@ -148,7 +148,9 @@ struct bt_model {
   unsigned* ts2_ctr = nullptr;               // token_step2: counters
   size_t ts2_ctr_bytes = 0;
   float2* ts_hstat = nullptr;                // token_step2: per-(row, tile) statistics of h
-  size_t l2_window = 0;                      // bytes of the local caches kept in L2 (0: none)
+  void* l2_base = nullptr;                   // L2 persisting window of the fused token step
+  size_t l2_window = 0;                      //   bytes (0: none)
+  float l2_hit = 0.f;                        //   hit ratio
   GemmScratch gs{};
   int B = 0, t = 0;
   bool prefilled = false;
@@ -228,14 +230,16 @@ static size_t carve(bt_model* m, const Dims& d, void* ws) {
     m->b_prefix = (float*)c.take((size_t)d.P * D * 4);
     m->lnf_t_g = (float*)c.take(D * 4); m->lnf_t_b = (float*)c.take(D * 4);
   }
+  // the LM head and the token decoder's local caches are adjacent: one L2
+  // persisting window can cover them (see bt_create)
   m->w_lm = c.take((size_t)d.V * D * eb);
   // caches: [layer][B][H][cap][d]
-  m->kb_layer = (size_t)d.Bmax * D * d.n_cap;
-  m->kb = c.take(m->kb_layer * d.Nb * eb);
-  m->vb = c.take(m->kb_layer * d.Nb * eb);
   m->kt_layer = (size_t)d.Bmax * D * d.l_cap;
   m->kt = c.take(m->kt_layer * (d.Nt > 0 ? d.Nt : 0) * eb);
   m->vt = c.take(m->kt_layer * (d.Nt > 0 ? d.Nt : 0) * eb);
+  m->kb_layer = (size_t)d.Bmax * D * d.n_cap;
+  m->kb = c.take(m->kb_layer * d.Nb * eb);
+  m->vb = c.take(m->kb_layer * d.Nb * eb);
   // activations
   const size_t R = d.R;
   m->h_b = (float*)c.take(R * D * 4);
@@ -392,22 +396,35 @@ int bt_create(const bt_config* cfg, const bt_weights* w, void* ws, size_t ws_byt
   if (m->ts_cnt) BT_TRYC(cudaMemsetAsync(m->ts_cnt, 0, (size_t)d.Bmax * d.H * sizeof(int), st));
   if (m->ts2_ctr) BT_TRYC(cudaMemsetAsync(m->ts2_ctr, 0, m->ts2_ctr_bytes, st));
   {
-    // The token decoder's local caches (K and V of every layer, at most
-    // P + L_B - 1 rows per sequence and head) stay in L2 between the decode
-    // calls that read them: a persisting access-policy window on the fused
-    // token-step launches, with this context's persisting set-aside sized to
-    // it when the device allows (BT_L2_WINDOW=0 turns it off).
+    // Decode calls re-read two regions every token step: the LM head and the
+    // token decoder's local caches (K and V of every layer, at most
+    // P + L_B - 1 rows per sequence and head). The fused token-step launches
+    // carry a persisting L2 access-policy window over both (adjacent in the
+    // workspace), and this context's persisting set-aside is sized to it as
+    // far as the device allows; when the window is larger than the set-aside
+    // the hit ratio keeps that fraction of it (BT_L2_WINDOW=0 turns it off).
     const char* env = getenv("BT_L2_WINDOW");
-    const size_t bytes = d.Nt > 0 ? 2 * m->kt_layer * d.Nt * d.eb : 0;
+    const size_t kv = d.Nt > 0 ? 2 * m->kt_layer * d.Nt * d.eb : 0;
+    const size_t bytes = kv > 0 ? (size_t)((uint8_t*)m->vt + kv / 2 - (uint8_t*)m->w_lm) : 0;
     int dev = 0, max_persist = 0, max_window = 0;
     if (bytes > 0 && !(env && env[0] == '0') && cudaGetDevice(&dev) == cudaSuccess &&
         cudaDeviceGetAttribute(&max_persist, cudaDevAttrMaxPersistingL2CacheSize, dev) == cudaSuccess &&
         cudaDeviceGetAttribute(&max_window, cudaDevAttrMaxAccessPolicyWindowSize, dev) == cudaSuccess &&
-        bytes <= (size_t)max_persist && bytes <= (size_t)max_window) {
+        max_persist > 0 && max_window > 0) {
+      void* base = m->w_lm;
+      size_t win = bytes;
+      if (win > (size_t)max_window) {  // the local caches alone
+        base = m->kt;
+        win = kv;
+      }
+      const size_t want = std::min(win, (size_t)max_persist);
       size_t cur = 0;
-      if (cudaDeviceGetLimit(&cur, cudaLimitPersistingL2CacheSize) == cudaSuccess &&
-          (cur >= bytes || cudaDeviceSetLimit(cudaLimitPersistingL2CacheSize, bytes) == cudaSuccess))
-        m->l2_window = bytes;
+      if (win <= (size_t)max_window && cudaDeviceGetLimit(&cur, cudaLimitPersistingL2CacheSize) == cudaSuccess &&
+          (cur >= want || cudaDeviceSetLimit(cudaLimitPersistingL2CacheSize, want) == cudaSuccess)) {
+        m->l2_base = base;
+        m->l2_window = win;
+        m->l2_hit = (float)std::min(1.0, (double)std::max(cur, want) / (double)win);
+      }
       cudaGetLastError();
     }
   }
@@ -786,6 +803,9 @@ static int run_token_step(bt_model* m, int B, bool ingest, PosSpec pos, const in
   a.logits = want_logits ? m->logits : nullptr; a.next = m->next; a.arg_part = m->arg_part;
   a.p1 = m->ts_p1; a.p2 = m->ts_p2; a.bar = m->ts_bar; a.status = m->status;
   a.wait_cycles = m->wait_cycles;
+  a.l2_window_base = m->l2_base;
+  a.l2_window_bytes = m->l2_window;
+  a.l2_hit_ratio = m->l2_hit;
   const void *wqb = nullptr, *wob = nullptr;
   if (block) {
     const LayerW& b0 = m->blk[0];
@@ -804,8 +824,6 @@ static int run_token_step(bt_model* m, int B, bool ingest, PosSpec pos, const in
   if (!block && token_step_kind(m, B) == 2) {
     a.bar = m->ts2_ctr;
     a.hstat = m->ts_hstat;
-    a.l2_window_base = m->kt;
-    a.l2_window_bytes = m->l2_window;
     BT_CUDA(launch_token_step2(a, w0.w_qkv1, w0.w_o2, m->w_lm, s));
     return BT_OK;
   }

@@ -62,12 +62,17 @@ constexpr int WORKERS = 128;               // warps 0-3 (TMEM lanes 0-127)
 constexpr int THREADS = WORKERS + 64;      // warp 4: TMA producer, warp 5: MMA issuer
 constexpr int BOX = 128 * 64 * 2;          // one weight box: 128 rows x 64 K (bf16)
 constexpr int MAX_STAGES = 16;
+constexpr int MAX_KB = 32;                 // K blocks of a staged activation operand (D / 64 <= 32)
 constexpr int MAX_B = 64;
 constexpr int MAX_WIN = 16;                // local-window rows (P + L_B - 1)
-constexpr int MAX_SPLIT = 16;              // K splits of a tile
-constexpr int TMEM_COLS = 128;             // two accumulators of up to 64 columns
+constexpr int TMEM_COLS = 512;             // two buffers of NCH accumulators of up to 64 columns
 constexpr int PRODUCER_SLEEP_NS = 128;
 constexpr int MMA_SLEEP_NS = 32;
+// K splits of a G1 tile (D / 128 blocks of 64 each) and of a G2 tile
+// (D / 128 blocks each): compile-time, so that the reductions over the
+// splits issue all their loads at once
+constexpr int S1 = 2;
+constexpr int S2 = 10;
 
 // counter slots (one 128-byte line each)
 enum : int {
@@ -94,6 +99,7 @@ struct Plan {
   int n_ing;              // CTAs that ingest rows (min(B, grid))
   int n_lm;               // CTAs with at least one vocabulary tile (min(TL, grid))
   int c_a2, c_g2p, n_slots;  // counter slots (see the enum)
+  int nch;                // independent accumulators per unit (K slices round-robin)
   int stages;             // weight ring depth
   int act_bytes;          // activation buffer
   float scale;            // log2(e) / sqrt(d_head)
@@ -145,10 +151,11 @@ __device__ __forceinline__ bool workers_wait(const TokenStepArgs& a, unsigned* c
   return !*s_abort;
 }
 
-// Workers' writes of a phase are done: every worker fences its own writes
-// (cumulative release through the barrier), then thread 0 signals.
+// Workers' writes of a phase are done: the worker barrier orders every
+// worker's writes before thread 0's release add (cumulative), which makes
+// them visible to whoever acquires the count.
 __device__ __forceinline__ void workers_signal(unsigned* c) {
-  __threadfence();
+  asm volatile("fence.proxy.async.global;" ::: "memory");  // consumers may read through TMA
   wsync();
   if (threadIdx.x == 0) signal(c);
 }
@@ -189,9 +196,16 @@ __device__ __forceinline__ uint2 pack_bf16x4(float a, float b, float c, float d)
 // (mean, sum of squared deviations) pairs over 128 features each (Chan's
 // pairwise combination; equal tile sizes).
 __device__ __forceinline__ void row_stats(const float2* hs, int T2, float eps, float& mu, float& rstd) {
+  constexpr int MAXT = 16;  // D <= 2048
+  float2 ps[MAXT];
+#pragma unroll
+  for (int t = 0; t < MAXT; ++t)
+    if (t < T2) ps[t] = __ldcg(hs + t);
   float m = 0.f, m2 = 0.f;
-  for (int t = 0; t < T2; ++t) {
-    const float2 p = __ldcg(hs + t);
+#pragma unroll
+  for (int t = 0; t < MAXT; ++t) {
+    if (t >= T2) break;
+    const float2 p = ps[t];
     const float n_a = 128.f * (float)t, n = n_a + 128.f;
     const float delta = p.x - m;
     m += delta * (128.f / n);
@@ -232,7 +246,7 @@ __device__ void producer(const CUtensorMap* mq, const CUtensorMap* mo, const CUt
     }
     mbar_arrive_expect_tx(&full[s], BOX);
     if (three) tc::tma_load_3d_hint(ring + (size_t)s * BOX, m, x, y, z, &full[s], first);
-    else tc::tma_load_2d_hint(ring + (size_t)s * BOX, m, x, y, &full[s], first);
+    else tc::tma_load_2d(ring + (size_t)s * BOX, m, x, y, &full[s]);  // LM head: the launch's L2 window decides
     ++it;
   };
   // the LM head's tiles of this CTA go to L2 while the layers run (HBM is
@@ -266,31 +280,57 @@ __device__ void producer(const CUtensorMap* mq, const CUtensorMap* mo, const CUt
 struct Sync {
   uint64_t* full;       // [stages] weight box landed
   uint64_t* empty;      // [stages] weight box consumed
-  uint64_t* act_full;   // activations of the unit staged (1 arrival + TMA bytes)
+  uint64_t* act_kb;     // [MAX_KB] K block kb of the unit's activations staged (1 arrival + TMA bytes)
   uint64_t* acc_full;   // [2] accumulator ready (tcgen05.commit)
   uint64_t* acc_empty;  // [2] accumulator drained (128 worker arrivals)
 };
 
 // One thread: the MMAs of one unit, `ntiles` row tiles of 128 accumulating
-// over nkb K blocks (ring boxes in tile-minor order per K block), into TMEM
-// columns tmem_d + i * Bp, then a commit to `done`.
-__device__ void issue_unit(const Plan& P, int nkb, int ntiles, uint8_t* ring, const uint8_t* act, uint32_t tmem_d,
-                           uint64_t* full, uint64_t* empty, uint64_t* done, int& it, const TokenStepArgs& a) {
+// over nkb K blocks (ring boxes in tile-minor order per K block). The 16-wide
+// K slices go round-robin to P.nch independent accumulators per tile (TMEM
+// columns tmem_d + (i * nch + ch) * Bp): consecutive MMAs into one
+// accumulator wait for each other, so independent chains keep the tensor
+// core busy at this small N. A commit to `done` follows.
+__device__ bool issue_unit(const Plan& P, int nkb, int ntiles, uint8_t* ring, const uint8_t* act, uint32_t tmem_d,
+                           const Sync& y, uint64_t* done, int& it, int* act_uses, bool need_act,
+                           const TokenStepArgs& a, volatile int* s_abort) {
   const uint32_t idesc = tc::idesc_bf16_m128(P.Bp);
   for (int kb = 0; kb < nkb; ++kb) {
+    // K block kb of the activations: MMAs start on the first block staged
+    if (need_act) {
+      if (!wait_or_abort(&y.act_kb[kb], act_uses[kb] & 1, a, s_abort, MMA_SLEEP_NS)) return false;
+      ++act_uses[kb];
+      tc::fence_after();
+    }
     const uint64_t db = tc::desc_sw128(smem_u32(act + (size_t)kb * P.Bp * 128));
     for (int i = 0; i < ntiles; ++i, ++it) {
       const int s = it % P.stages;
-      mbar_wait_bounded(&full[s], (it / P.stages) & 1, a.status, a.wait_cycles);
+      mbar_wait_bounded(&y.full[s], (it / P.stages) & 1, a.status, a.wait_cycles);
       tc::fence_after();
       const uint64_t da = tc::desc_sw128(smem_u32(ring + (size_t)s * BOX));
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk)  // 16-wide K slices: +32 bytes = +2 in descriptor units
-        tc::mma_bf16(tmem_d + (uint32_t)(i * P.Bp), da + 2 * kk, db + 2 * kk, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
-      tc::commit(&empty[s]);
+      for (int kk = 0; kk < 4; ++kk) {  // 16-wide K slices: +32 bytes = +2 in descriptor units
+        const int j = kb * 4 + kk, ch = j % P.nch;
+        tc::mma_bf16(tmem_d + (uint32_t)((i * P.nch + ch) * P.Bp), da + 2 * kk, db + 2 * kk, idesc,
+                     j >= P.nch ? 1u : 0u);
+      }
+      tc::commit(&y.empty[s]);
     }
   }
   tc::commit(done);
+  return true;
+}
+
+// Sum of the nch accumulators of one tile: 16 consecutive columns c0.. of
+// this warp's 32 TMEM lanes.
+__device__ __forceinline__ void acc_ld16(uint32_t trow, int nch, int Bp, int c0, float* v) {
+  tc::tmem_ld16(trow + c0, v);
+  for (int ch = 1; ch < nch; ++ch) {
+    float w[16];
+    tc::tmem_ld16(trow + ch * Bp + c0, w);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) v[j] += w[j];
+  }
 }
 
 // MMA warp (one thread): the unit sequence of the producer. Waits for the
@@ -298,16 +338,17 @@ __device__ void issue_unit(const Plan& P, int nkb, int ntiles, uint8_t* ring, co
 __device__ void mma_issuer(const Plan& P, int Nt, uint8_t* ring, const uint8_t* act, uint32_t tmem, const Sync& y,
                            const TokenStepArgs& a, volatile int* s_abort) {
   const int G = gridDim.x, c = blockIdx.x;
-  int it = 0, na = 0, nu = 0;
+  int it = 0, nu = 0;
+  int act_uses[MAX_KB];
+#pragma unroll
+  for (int k = 0; k < MAX_KB; ++k) act_uses[k] = 0;
   auto unit = [&](int nkb, int ntiles, bool need_act) -> bool {
-    if (need_act) {
-      if (!wait_or_abort(y.act_full, na & 1, a, s_abort, MMA_SLEEP_NS)) return false;
-      ++na;
-    }
     const int buf = nu & 1;
     if (nu >= 2 && !wait_or_abort(&y.acc_empty[buf], ((nu >> 1) + 1) & 1, a, s_abort, MMA_SLEEP_NS)) return false;
     tc::fence_after();
-    issue_unit(P, nkb, ntiles, ring, act, tmem + (uint32_t)(buf * 64), y.full, y.empty, &y.acc_full[buf], it, a);
+    if (!issue_unit(P, nkb, ntiles, ring, act, tmem + (uint32_t)(buf * P.nch * P.Bp), y, &y.acc_full[buf], it,
+                    act_uses, need_act, a, s_abort))
+      return false;
     ++nu;
     return true;
   };
@@ -316,13 +357,9 @@ __device__ void mma_issuer(const Plan& P, int Nt, uint8_t* ring, const uint8_t* 
     for (int w = first_g1(P, c); ok && w < P.N1; w += G) ok = unit(P.kb1, 1, true);
     for (int w = first_g2(P, c, G); ok && w < P.N2; w += G) ok = unit(P.kb2, 1, true);
   }
-  if (!ok) {
-    if (nu > 0) mbar_wait_bounded(&y.acc_full[(nu - 1) & 1], ((nu - 1) >> 1) & 1, a.status, a.wait_cycles);
-    return;
-  }
   bool first = true;
-  for (int t = c; t < P.TL; t += G) {
-    if (!unit(P.kbL, 1, first)) break;  // every vocabulary tile reads the same staged input
+  for (int t = c; ok && t < P.TL; t += G) {
+    ok = unit(P.kbL, 1, first);  // every vocabulary tile reads the same staged input
     first = false;
   }
   // MMAs still writing TMEM must finish before the accumulators are freed
@@ -334,13 +371,13 @@ __device__ void mma_issuer(const Plan& P, int Nt, uint8_t* ring, const uint8_t* 
 // accumulators; column b is batch row b.
 
 // Store the fp32 accumulator tile (128 features x B rows) to part[b][128].
-__device__ void store_partial(uint32_t tbuf, float* part, int B, int Bp) {
+__device__ void store_partial(uint32_t tbuf, float* part, int B, int Bp, int nch) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t trow = tbuf + ((uint32_t)(warp * 32) << 16);
   float* dst = part + warp * 32 + lane;
   for (int c0 = 0; c0 < Bp; c0 += 16) {
     float v[16];
-    tc::tmem_ld16(trow + c0, v);
+    acc_ld16(trow, nch, Bp, c0, v);
 #pragma unroll
     for (int j = 0; j < 16; ++j)
       if (c0 + j < B) __stcg(dst + (size_t)(c0 + j) * 128, v[j]);
@@ -383,39 +420,78 @@ __device__ void ingest_phase(const TokenStepArgs& a, const Plan& P, int jb) {
   }
 }
 
-// G1 activations: rows 0..Bp-1 of features [k0, k0 + 64 kb1) normalised
-// with (g, beta) -> bf16 in the swizzled K-major operand layout (rows >= B
-// are zero).
-__device__ void ln_to_operand(const TokenStepArgs& a, const Plan& P, int k0, const float* g, const float* beta,
-                              uint8_t* act) {
-  const int n_items = P.Bp * P.kb1;
-  for (int item = threadIdx.x; item < n_items; item += WORKERS) {
-    const int b = item / P.kb1, kb = item - b * P.kb1;
-    uint8_t* rowp = act + (size_t)kb * P.Bp * 128;
-    if (b >= a.B) {
-#pragma unroll
-      for (int ch = 0; ch < 8; ++ch)
-        *reinterpret_cast<uint4*>(rowp + tc::sw128_offset(b, ch)) = make_uint4(0, 0, 0, 0);
-      continue;
-    }
+// Per-row LayerNorm statistics (mean, 1 / std) of rows 0..B-1 and the
+// LayerNorm gain / shift of features [k0, k0 + 64 kb1) into shared memory.
+__device__ void ln_params_to_smem(const TokenStepArgs& a, const Plan& P, int k0, const float* g, const float* beta,
+                                  float* s_mu, float* s_rs, float* s_g, float* s_b) {
+  for (int b = threadIdx.x; b < a.B; b += WORKERS) {
     float mu, rstd;
     row_stats(a.hstat + (size_t)b * P.T2, P.T2, a.eps, mu, rstd);
-    const int f0 = k0 + kb * 64;
-    const float* hrow = a.h + (size_t)b * a.D + f0;
+    s_mu[b] = mu;
+    s_rs[b] = rstd;
+  }
+  for (int f = threadIdx.x * 4; f < P.kb1 * 64; f += WORKERS * 4) {
+    *reinterpret_cast<float4*>(s_g + f) = *reinterpret_cast<const float4*>(g + k0 + f);
+    *reinterpret_cast<float4*>(s_b + f) = *reinterpret_cast<const float4*>(beta + k0 + f);
+  }
+}
+
+// G1 activations: rows 0..Bp-1 of features [k0, k0 + 64 kb1) normalised
+// (statistics and parameters in shared memory) -> bf16 in the swizzled
+// K-major operand layout (rows >= B are zero), one K block at a time: block
+// kb is announced on bars[kb] (thread 0, after the worker barrier) so that
+// its MMAs start while the next block is normalised; the loads of block
+// kb + 1 are in flight while block kb is converted. Item = (row, 16-byte
+// chunk of 8 features) of a block; Bp * 8 <= 4 * WORKERS.
+__device__ void ln_to_operand(const TokenStepArgs& a, const Plan& P, int k0, const float* s_g, const float* s_b,
+                              const float* s_mu, const float* s_rs, uint8_t* act, uint64_t* bars, int* staged) {
+  constexpr int U = 4;
+  const int n_items = P.Bp * 8;
+  float4 cx0[U], cx1[U], nx0[U], nx1[U];
+  auto load = [&](int kb, float4* x0, float4* x1) {
 #pragma unroll
-    for (int ch = 0; ch < 8; ++ch) {
-      const float4 x0 = __ldcg(reinterpret_cast<const float4*>(hrow + ch * 8));
-      const float4 x1 = __ldcg(reinterpret_cast<const float4*>(hrow + ch * 8 + 4));
-      const float4 g0 = *reinterpret_cast<const float4*>(g + f0 + ch * 8);
-      const float4 g1 = *reinterpret_cast<const float4*>(g + f0 + ch * 8 + 4);
-      const float4 b0 = *reinterpret_cast<const float4*>(beta + f0 + ch * 8);
-      const float4 b1 = *reinterpret_cast<const float4*>(beta + f0 + ch * 8 + 4);
-      const uint2 lo = pack_bf16x4((x0.x - mu) * rstd * g0.x + b0.x, (x0.y - mu) * rstd * g0.y + b0.y,
-                                   (x0.z - mu) * rstd * g0.z + b0.z, (x0.w - mu) * rstd * g0.w + b0.w);
-      const uint2 hi = pack_bf16x4((x1.x - mu) * rstd * g1.x + b1.x, (x1.y - mu) * rstd * g1.y + b1.y,
-                                   (x1.z - mu) * rstd * g1.z + b1.z, (x1.w - mu) * rstd * g1.w + b1.w);
-      *reinterpret_cast<uint4*>(rowp + tc::sw128_offset(b, ch)) = make_uint4(lo.x, lo.y, hi.x, hi.y);
+    for (int u = 0; u < U; ++u) {
+      const int item = threadIdx.x + u * WORKERS;
+      const int b = item >> 3, ch = item & 7;
+      if (item < n_items && b < a.B) {
+        const float* src = a.h + (size_t)b * a.D + k0 + kb * 64 + ch * 8;
+        x0[u] = __ldcg(reinterpret_cast<const float4*>(src));
+        x1[u] = __ldcg(reinterpret_cast<const float4*>(src + 4));
+      }
     }
+  };
+  load(0, cx0, cx1);
+  for (int kb = 0; kb < P.kb1; ++kb) {
+    if (kb + 1 < P.kb1) load(kb + 1, nx0, nx1);
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int item = threadIdx.x + u * WORKERS;
+      if (item >= n_items) continue;
+      const int b = item >> 3, ch = item & 7;
+      uint4 out = make_uint4(0, 0, 0, 0);
+      if (b < a.B) {
+        const int f = kb * 64 + ch * 8;
+        const float mu = s_mu[b], rstd = s_rs[b];
+        const float4 g0 = *reinterpret_cast<const float4*>(s_g + f);
+        const float4 g1 = *reinterpret_cast<const float4*>(s_g + f + 4);
+        const float4 b0 = *reinterpret_cast<const float4*>(s_b + f);
+        const float4 b1 = *reinterpret_cast<const float4*>(s_b + f + 4);
+        const uint2 lo = pack_bf16x4((cx0[u].x - mu) * rstd * g0.x + b0.x, (cx0[u].y - mu) * rstd * g0.y + b0.y,
+                                     (cx0[u].z - mu) * rstd * g0.z + b0.z, (cx0[u].w - mu) * rstd * g0.w + b0.w);
+        const uint2 hi = pack_bf16x4((cx1[u].x - mu) * rstd * g1.x + b1.x, (cx1[u].y - mu) * rstd * g1.y + b1.y,
+                                     (cx1[u].z - mu) * rstd * g1.z + b1.z, (cx1[u].w - mu) * rstd * g1.w + b1.w);
+        out = make_uint4(lo.x, lo.y, hi.x, hi.y);
+      }
+      *reinterpret_cast<uint4*>(act + (size_t)kb * P.Bp * 128 + tc::sw128_offset(b, ch)) = out;
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    wsync();
+    if (threadIdx.x == 0) {
+      mbar_arrive(&bars[kb]);
+      ++staged[kb];
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) { cx0[u] = nx0[u]; cx1[u] = nx1[u]; }
   }
 }
 
@@ -471,13 +547,14 @@ __device__ void attention_items(const TokenStepArgs& a, const Plan& P, int l, in
       float4 sv = *reinterpret_cast<const float4*>(bias + 2 * a.D + fq);
       if (active) {
         const int f = hh * DH + e0 + e;  // feature within the tile
-        for (int sp = 0; sp < P.S1; ++sp) {
+#pragma unroll
+        for (int sp = 0; sp < S1; ++sp) {
           const size_t o = ((size_t)sp * a.B + r) * 128 + f;
-          sq = f4add(sq, __ldcg(reinterpret_cast<const float4*>(a.p1 + ((size_t)hg * P.S1) * a.B * 128 + o)));
+          sq = f4add(sq, __ldcg(reinterpret_cast<const float4*>(a.p1 + ((size_t)hg * S1) * a.B * 128 + o)));
           sk = f4add(sk, __ldcg(reinterpret_cast<const float4*>(
-                             a.p1 + ((size_t)(P.HG + hg) * P.S1) * a.B * 128 + o)));
+                             a.p1 + ((size_t)(P.HG + hg) * S1) * a.B * 128 + o)));
           sv = f4add(sv, __ldcg(reinterpret_cast<const float4*>(
-                             a.p1 + ((size_t)(2 * P.HG + hg) * P.S1) * a.B * 128 + o)));
+                             a.p1 + ((size_t)(2 * P.HG + hg) * S1) * a.B * 128 + o)));
         }
       }
       q[e] = sq.x; q[e + 1] = sq.y; q[e + 2] = sq.z; q[e + 3] = sq.w;
@@ -565,15 +642,31 @@ __device__ void attention_items(const TokenStepArgs& a, const Plan& P, int l, in
 __device__ void gelu_rows(const TokenStepArgs& a, const Plan& P, int l, int f, int r0, int r1) {
   const int t = 3 * P.HG + f;
   const float* bias = layer_ptr(a.b_qkv1, l, a.layer_stride) + 3 * a.D + f * 128;
-  const float* part = a.p1 + (size_t)t * P.S1 * a.B * 128;
+  const float* part = a.p1 + (size_t)t * S1 * a.B * 128;
   const int n = (r1 - r0) * 32;  // float4 groups
-  for (int i = threadIdx.x; i < n; i += WORKERS) {
-    const int r = r0 + i / 32, c = (i % 32) * 4;
-    float4 acc = *reinterpret_cast<const float4*>(bias + c);
-    for (int sp = 0; sp < P.S1; ++sp)
-      acc = f4add(acc, __ldcg(reinterpret_cast<const float4*>(part + ((size_t)sp * a.B + r) * 128 + c)));
-    *reinterpret_cast<uint2*>(a.a2 + (size_t)r * 5 * a.D + a.D + f * 128 + c) =
-        pack_bf16x4(gelu_erf(acc.x), gelu_erf(acc.y), gelu_erf(acc.z), gelu_erf(acc.w));
+  constexpr int U = 4;           // groups per thread in flight
+  for (int i0 = threadIdx.x; i0 < n; i0 += U * WORKERS) {
+    float4 acc[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i = i0 + u * WORKERS;
+      if (i < n) {
+        const int r = r0 + i / 32, c = (i % 32) * 4;
+        acc[u] = *reinterpret_cast<const float4*>(bias + c);
+#pragma unroll
+        for (int sp = 0; sp < S1; ++sp)
+          acc[u] = f4add(acc[u], __ldcg(reinterpret_cast<const float4*>(part + ((size_t)sp * a.B + r) * 128 + c)));
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i = i0 + u * WORKERS;
+      if (i < n) {
+        const int r = r0 + i / 32, c = (i % 32) * 4;
+        *reinterpret_cast<uint2*>(a.a2 + (size_t)r * 5 * a.D + a.D + f * 128 + c) =
+            pack_bf16x4(gelu_erf(acc[u].x), gelu_erf(acc[u].y), gelu_erf(acc[u].z), gelu_erf(acc[u].w));
+      }
+    }
   }
 }
 
@@ -584,12 +677,16 @@ __device__ void residual_rows(const TokenStepArgs& a, const Plan& P, int l, int 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int f = t2 * 128 + 4 * lane;
   const float4 bo = *reinterpret_cast<const float4*>(layer_ptr(a.b_o2, l, a.layer_stride) + f);
-  const float* part = a.p2 + (size_t)t2 * P.S2 * a.B * 128;
+  const float* part = a.p2 + (size_t)t2 * S2 * a.B * 128;
   for (int r = r0 + warp; r < r1; r += 4) {
     float* hrow = a.h + (size_t)r * a.D;
     float4 acc = f4add(__ldcg(reinterpret_cast<const float4*>(hrow + f)), bo);
-    for (int sp = 0; sp < P.S2; ++sp)
-      acc = f4add(acc, __ldcg(reinterpret_cast<const float4*>(part + ((size_t)sp * a.B + r) * 128 + 4 * lane)));
+    float4 ps[S2];
+#pragma unroll
+    for (int sp = 0; sp < S2; ++sp)
+      ps[sp] = __ldcg(reinterpret_cast<const float4*>(part + ((size_t)sp * a.B + r) * 128 + 4 * lane));
+#pragma unroll
+    for (int sp = 0; sp < S2; ++sp) acc = f4add(acc, ps[sp]);
     __stcg(reinterpret_cast<float4*>(hrow + f), acc);
     const float mean = warp_sum((acc.x + acc.y) + (acc.z + acc.w)) * (1.f / 128.f);
     const float dx = acc.x - mean, dy = acc.y - mean, dz = acc.z - mean, dw = acc.w - mean;
@@ -642,15 +739,15 @@ __device__ __forceinline__ void warp_argmax32(float* v, int* ix) {
 }
 
 // LM epilogue of vocabulary tile t: logits (optional) and the tile's argmax per row
-__device__ void lm_epilogue(uint32_t tbuf, int t, const TokenStepArgs& a, int Bp, float2 (*s_arg)[MAX_B]) {
+__device__ void lm_epilogue(uint32_t tbuf, int t, const TokenStepArgs& a, int Bp, int nch, float2 (*s_arg)[MAX_B]) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t trow = tbuf + ((uint32_t)(warp * 32) << 16);
   const int n = t * 128 + warp * 32 + lane;
   for (int c0 = 0; c0 < Bp; c0 += 32) {
     float v[32];
     int ix[32];
-    tc::tmem_ld16(trow + c0, v);
-    if (c0 + 16 < Bp) tc::tmem_ld16(trow + c0 + 16, v + 16);
+    acc_ld16(trow, nch, Bp, c0, v);
+    if (c0 + 16 < Bp) acc_ld16(trow, nch, Bp, c0 + 16, v + 16);
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
       const int m = c0 + j;
@@ -679,12 +776,19 @@ __device__ void lm_epilogue(uint32_t tbuf, int t, const TokenStepArgs& a, int Bp
 // Greedy id per row from the tile partials (lowest id on ties)
 __device__ void argmax_rows(const TokenStepArgs& a, const Plan& P) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int U = 16;  // tile partials per lane in flight (TL <= 512 * 32 / 32)
   for (int b = blockIdx.x * 4 + warp; b < a.B; b += 4 * gridDim.x) {
     float bv = -INFINITY;
     int bi = INT_MAX;
-    for (int t = lane; t < P.TL; t += 32) {
-      const float2 o = __ldcg(a.arg_part + (size_t)t * a.B + b);
-      better(bv, bi, o.x, __float_as_int(o.y));
+    for (int t0 = lane; t0 < P.TL; t0 += U * 32) {
+      float2 o[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int t = t0 + u * 32;
+        o[u] = t < P.TL ? __ldcg(a.arg_part + (size_t)t * a.B + b) : make_float2(-INFINITY, __int_as_float(INT_MAX));
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) better(bv, bi, o[u].x, __float_as_int(o[u].y));
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -697,12 +801,17 @@ __device__ void argmax_rows(const TokenStepArgs& a, const Plan& P) {
 }
 
 // TMA of nkb activation boxes (Bp rows x 64 columns, columns col0 + 64 kb)
-// into `act`, completion on `bar`. One thread; the rows were written through
-// the generic proxy by other CTAs before the counter this thread acquired.
-__device__ void load_act(const CUtensorMap* map, uint8_t* act, int col0, int nkb, int Bp, uint64_t* bar) {
+// into `act`, box kb completing on bars[kb]. One thread; the rows were
+// written through the generic proxy by other CTAs before the counter this
+// thread acquired.
+__device__ void load_act(const CUtensorMap* map, uint8_t* act, int col0, int nkb, int Bp, uint64_t* bars,
+                         int* staged) {
   asm volatile("fence.proxy.async.global;" ::: "memory");
-  mbar_arrive_expect_tx(bar, (uint32_t)(nkb * Bp * 128));
-  for (int kb = 0; kb < nkb; ++kb) tc::tma_load_2d(act + (size_t)kb * Bp * 128, map, col0 + kb * 64, 0, bar);
+  for (int kb = 0; kb < nkb; ++kb) {
+    mbar_arrive_expect_tx(&bars[kb], (uint32_t)(Bp * 128));
+    tc::tma_load_2d(act + (size_t)kb * Bp * 128, map, col0 + kb * 64, 0, &bars[kb]);
+    ++staged[kb];
+  }
 }
 
 template <int DH>
@@ -714,10 +823,11 @@ token_step2_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* ring = smem;
   uint8_t* act = smem + (size_t)P.stages * BOX;
-  __shared__ __align__(8) uint64_t full[MAX_STAGES], empty[MAX_STAGES], act_full, acc_full[2], acc_empty[2],
-      win_bar;
+  __shared__ __align__(8) uint64_t full[MAX_STAGES], empty[MAX_STAGES], act_kb[MAX_KB], acc_full[2],
+      acc_empty[2], win_bar;
   __shared__ uint32_t tmem_slot;
   __shared__ float2 s_arg[4][MAX_B];
+  __shared__ float s_mu[MAX_B], s_rs[MAX_B];
   __shared__ volatile int s_abort;
 
   const int warp = threadIdx.x >> 5;
@@ -726,7 +836,7 @@ token_step2_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
     }
-    mbar_init(&act_full, 1);
+    for (int i = 0; i < MAX_KB; ++i) mbar_init(&act_kb[i], 1);
     mbar_init(&win_bar, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&acc_full[i], 1);
@@ -740,7 +850,7 @@ token_step2_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
   __syncthreads();
   tc::fence_after();
   const uint32_t tmem = tmem_slot;
-  const Sync y{full, empty, &act_full, acc_full, acc_empty};
+  const Sync y{full, empty, act_kb, acc_full, acc_empty};
   pdl_trigger();
 
   if (warp == 4) {
@@ -757,7 +867,10 @@ token_step2_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
     unsigned* cb = a.bar;
     wsync();
     if (threadIdx.x == 0) signal(ctr(cb, C_ARRIVED));
-    int na = 0, nu = 0, nw = 0;
+    int nu = 0, nw = 0;
+    int staged[MAX_KB];  // worker-side uses of each activation barrier (thread 0)
+#pragma unroll
+    for (int k = 0; k < MAX_KB; ++k) staged[k] = 0;
     bool win_pending = false;
     bool ok = true;
     const int nh = 128 / DH;
@@ -774,11 +887,12 @@ token_step2_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
         const bool qkv = t < 3 * P.HG;
         const float* g = layer_ptr(qkv ? a.ln1_g : a.ln2_g, l, a.layer_stride);
         const float* be = layer_ptr(qkv ? a.ln1_b : a.ln2_b, l, a.layer_stride);
-        ln_to_operand(a, P, sp * P.kb1 * 64, g, be, act);
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        // LayerNorm parameters of the unit's K range after the operand
+        float* s_g = reinterpret_cast<float*>(act + (size_t)P.kb1 * P.Bp * 128);
+        float* s_b = s_g + P.kb1 * 64;
+        ln_params_to_smem(a, P, sp * P.kb1 * 64, g, be, s_mu, s_rs, s_g, s_b);
         wsync();
-        if (threadIdx.x == 0) mbar_arrive(&act_full);
-        ++na;
+        ln_to_operand(a, P, sp * P.kb1 * 64, s_g, s_b, s_mu, s_rs, act, act_kb, staged);
         const int buf = nu & 1;
         mbar_wait_bounded(&acc_full[buf], (nu >> 1) & 1, a.status, a.wait_cycles);
         tc::fence_after();
@@ -790,7 +904,7 @@ token_step2_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
           window_copies(a, l, hg, nh, ra0, ra1, pos, act, &win_bar);
           win_pending = true;
         }
-        store_partial(tmem + (uint32_t)(buf * 64), a.p1 + (size_t)(t * P.S1 + sp) * B * 128, B, P.Bp);
+        store_partial(tmem + (uint32_t)(buf * P.nch * P.Bp), a.p1 + (size_t)(t * P.S1 + sp) * B * 128, B, P.Bp, P.nch);
         tc::fence_before();
         mbar_arrive(&acc_empty[buf]);
         ++nu;
@@ -822,12 +936,11 @@ token_step2_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
             wait_count(a, ctr(cb, P.c_a2 + j), (unsigned)((l + 1) * (j < P.HG ? 3 * P.S1 : P.S1)), &s_abort);
         wsync();
         if (!(ok = !s_abort)) break;
-        if (threadIdx.x == 0) load_act(&ma2, act, col0, P.kb2, P.Bp, &act_full);
-        ++na;
+        if (threadIdx.x == 0) load_act(&ma2, act, col0, P.kb2, P.Bp, act_kb, staged);
         const int buf = nu & 1;
         mbar_wait_bounded(&acc_full[buf], (nu >> 1) & 1, a.status, a.wait_cycles);
         tc::fence_after();
-        store_partial(tmem + (uint32_t)(buf * 64), a.p2 + (size_t)(t2 * P.S2 + sp) * B * 128, B, P.Bp);
+        store_partial(tmem + (uint32_t)(buf * P.nch * P.Bp), a.p2 + (size_t)(t2 * P.S2 + sp) * B * 128, B, P.Bp, P.nch);
         tc::fence_before();
         mbar_arrive(&acc_empty[buf]);
         ++nu;
@@ -847,13 +960,12 @@ token_step2_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
     // LM head over this CTA's vocabulary tiles
     if (ok && c < P.TL) {
       if ((ok = workers_wait(a, ctr(cb, C_FINAL), (unsigned)P.n_ing, &s_abort))) {
-        if (threadIdx.x == 0) load_act(&mxf, act, 0, P.kbL, P.Bp, &act_full);
-        ++na;
+        if (threadIdx.x == 0) load_act(&mxf, act, 0, P.kbL, P.Bp, act_kb, staged);
         for (int t = c; t < P.TL; t += G) {
           const int buf = nu & 1;
           mbar_wait_bounded(&acc_full[buf], (nu >> 1) & 1, a.status, a.wait_cycles);
           tc::fence_after();
-          lm_epilogue(tmem + (uint32_t)(buf * 64), t, a, P.Bp, s_arg);
+          lm_epilogue(tmem + (uint32_t)(buf * P.nch * P.Bp), t, a, P.Bp, P.nch, s_arg);
           mbar_arrive(&acc_empty[buf]);  // lm_epilogue ended with the tcgen05 fence + barrier
           ++nu;
         }
@@ -876,7 +988,8 @@ token_step2_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
     // copies into shared memory still in flight must land before the CTA exits
     if (threadIdx.x == 0) {
       if (win_pending) mbar_wait_bounded(&win_bar, nw & 1, a.status, a.wait_cycles);
-      if (na > 0) mbar_wait_bounded(&act_full, (na - 1) & 1, a.status, a.wait_cycles);
+      for (int k = 0; k < MAX_KB; ++k)
+        if (staged[k] > 0) mbar_wait_bounded(&act_kb[k], (staged[k] - 1) & 1, a.status, a.wait_cycles);
     }
   }
 
@@ -975,8 +1088,6 @@ Device& device() {
   return d;
 }
 
-constexpr int S1_FIXED = 2;    // K splits of a G1 tile (kb1 = D / 128 blocks of 64)
-constexpr int S2_FIXED = 10;   // K splits of a G2 tile (kb2 = D / 128 blocks of 64)
 
 bool make_plan(int B, int D, int dh, int V, int l_cap, int sms, size_t smem_max, Plan* P, size_t* smem) {
   Plan p{};
@@ -985,8 +1096,8 @@ bool make_plan(int B, int D, int dh, int V, int l_cap, int sms, size_t smem_max,
   p.T1 = 7 * p.HG;
   p.T2 = p.HG;
   p.TL = (V + 127) / 128;
-  p.S1 = S1_FIXED;
-  p.S2 = S2_FIXED;
+  p.S1 = S1;
+  p.S2 = S2;
   p.kb1 = D / 64 / p.S1;
   p.kb2 = 5 * D / 64 / p.S2;
   p.kbL = D / 64;
@@ -998,8 +1109,11 @@ bool make_plan(int B, int D, int dh, int V, int l_cap, int sms, size_t smem_max,
   p.c_a2 = C_G1P + p.T1;
   p.c_g2p = p.c_a2 + 5 * p.HG;
   p.n_slots = p.c_g2p + p.T2;
+  // one accumulator per tile: tcgen05.mma costs ~156 cycles to issue on B200
+  // whatever its N (measured), so independent chains buy nothing here
+  p.nch = 1;
   // the activation buffer: the largest operand, or the attention windows
-  size_t act = (size_t)p.kb1 * p.Bp * 128;
+  size_t act = (size_t)p.kb1 * p.Bp * 128 + (size_t)p.kb1 * 64 * 2 * sizeof(float);  // + LayerNorm parameters
   act = act > (size_t)p.kb2 * p.Bp * 128 ? act : (size_t)p.kb2 * p.Bp * 128;
   act = act > (size_t)p.kbL * p.Bp * 128 ? act : (size_t)p.kbL * p.Bp * 128;
   const int rows_max = (B + 3 * p.S1 - 1) / (3 * p.S1);
@@ -1026,8 +1140,8 @@ size_t token_step2_counter_bytes(int D) {
 size_t token_step2_scratch_floats(int B, int D, int which) {
   if (B > MAX_B) B = MAX_B;
   const int hg = D / 128;
-  if (which == 1) return (size_t)7 * hg * S1_FIXED * B * 128;   // G1 partials
-  if (which == 2) return (size_t)hg * S2_FIXED * B * 128;       // G2 partials
+  if (which == 1) return (size_t)7 * hg * S1 * B * 128;   // G1 partials
+  if (which == 2) return (size_t)hg * S2 * B * 128;       // G2 partials
   return (size_t)B * hg * 2;                                     // per-(row, tile) statistics
 }
 
@@ -1037,7 +1151,7 @@ int token_step2_supported(int dt, int B, int D, int H, int rot, int V, int Nt, i
   const int dh = D / H;
   if (dh != 32 && dh != 64 && dh != 128) return 0;
   if (rot != 0 && rot != dh / 4) return 0;  // the rotary dims sit in one thread's quarter of the head
-  if ((5 * D / 64) % S2_FIXED || (D / 64) % S1_FIXED) return 0;
+  if ((5 * D / 64) % S2 || (D / 64) % S1) return 0;
   if (!encode_fn()) return 0;
   Device& d = device();
   if (!d.ready) return 0;
@@ -1084,11 +1198,11 @@ cudaError_t launch_token_step2(const TokenStepArgs& a, const void* w_qkv1, const
     attr[na++].val.programmaticStreamSerializationAllowed = 1;
   }
   if (a.l2_window_bytes > 0) {
-    // the local window (K and V of every token-decoder layer) persists in L2
+    // the re-read regions (LM head, local caches) persist in L2
     attr[na].id = cudaLaunchAttributeAccessPolicyWindow;
     attr[na].val.accessPolicyWindow.base_ptr = a.l2_window_base;
     attr[na].val.accessPolicyWindow.num_bytes = a.l2_window_bytes;
-    attr[na].val.accessPolicyWindow.hitRatio = 1.0f;
+    attr[na].val.accessPolicyWindow.hitRatio = a.l2_hit_ratio;
     attr[na].val.accessPolicyWindow.hitProp = cudaAccessPropertyPersisting;
     attr[na++].val.accessPolicyWindow.missProp = cudaAccessPropertyStreaming;
   }
