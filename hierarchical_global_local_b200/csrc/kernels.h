@@ -239,6 +239,7 @@ struct TokenStepArgs {
   // deviations) of h [B][D/128]. Both kernels: an L2 persisting access-policy
   // window for the launch (bytes 0 = none)
   float2* hstat;
+  bf16* hb;          // token_step2: bf16 copy of h [B, D] (the G1 units' TMA source)
   void* l2_window_base;
   size_t l2_window_bytes;
   float l2_hit_ratio;
@@ -276,7 +277,7 @@ cudaError_t launch_token_step(const TokenStepArgs& a, const void* w_qkv1, const 
 // rotary on none or the first d_head/4 dims, local window <= 16 rows, any
 // prefix length. a.bar: token_step2_counter_bytes(D) bytes, zero before the
 // first launch (a launch leaves them zero unless a wait ran out); a.p1, a.p2,
-// a.hstat: token_step2_scratch_floats(B, D, 1 | 2 | 3) floats.
+// a.hstat, a.hb: token_step2_scratch_floats(B, D, 1 | 2 | 3 | 4) floats.
 int token_step2_supported(int dt, int B, int D, int H, int rot, int V, int Nt, int l_cap);
 size_t token_step2_counter_bytes(int D);
 size_t token_step2_scratch_floats(int B, int D, int which);

@@ -148,6 +148,7 @@ struct bt_model {
   unsigned* ts2_ctr = nullptr;               // token_step2: counters
   size_t ts2_ctr_bytes = 0;
   float2* ts_hstat = nullptr;                // token_step2: per-(row, tile) statistics of h
+  bf16* ts_hb = nullptr;                     // token_step2: bf16 copy of h
   void* l2_base = nullptr;                   // L2 persisting window of the fused token step
   size_t l2_window = 0;                      //   bytes (0: none)
   float l2_hit = 0.f;                        //   hit ratio
@@ -274,6 +275,7 @@ static size_t carve(bt_model* m, const Dims& d, void* ws) {
     m->ts2_ctr_bytes = token_step2_counter_bytes(d.D);
     m->ts2_ctr = (unsigned*)c.take(m->ts2_ctr_bytes);
     m->ts_hstat = (float2*)c.take(token_step2_scratch_floats(d.Bmax, d.D, 3) * 4);
+    m->ts_hb = (bf16*)c.take(token_step2_scratch_floats(d.Bmax, d.D, 4) * 4);
   }
   m->vt_ld = (d.n_cap + 63) / 64 * 64;
   m->vtr = c.take((size_t)d.Bmax * D * m->vt_ld * eb);
@@ -824,6 +826,7 @@ static int run_token_step(bt_model* m, int B, bool ingest, PosSpec pos, const in
   if (!block && token_step_kind(m, B) == 2) {
     a.bar = m->ts2_ctr;
     a.hstat = m->ts_hstat;
+    a.hb = m->ts_hb;
     BT_CUDA(launch_token_step2(a, w0.w_qkv1, w0.w_o2, m->w_lm, s));
     return BT_OK;
   }

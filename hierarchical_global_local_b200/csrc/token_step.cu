@@ -65,7 +65,7 @@ constexpr int MAX_STAGES = 16;
 constexpr int MAX_KB = 32;                 // K blocks of a staged activation operand (D / 64 <= 32)
 constexpr int MAX_B = 64;
 constexpr int MAX_WIN = 16;                // local-window rows (P + L_B - 1)
-constexpr int TMEM_COLS = 512;             // two buffers of NCH accumulators of up to 64 columns
+constexpr int TMEM_COLS = 128;             // two accumulators of up to 64 columns
 constexpr int PRODUCER_SLEEP_NS = 128;
 constexpr int MMA_SLEEP_NS = 32;
 // K splits of a G1 tile (D / 128 blocks of 64 each) and of a G2 tile
@@ -99,7 +99,6 @@ struct Plan {
   int n_ing;              // CTAs that ingest rows (min(B, grid))
   int n_lm;               // CTAs with at least one vocabulary tile (min(TL, grid))
   int c_a2, c_g2p, n_slots;  // counter slots (see the enum)
-  int nch;                // independent accumulators per unit (K slices round-robin)
   int stages;             // weight ring depth
   int act_bytes;          // activation buffer
   float scale;            // log2(e) / sqrt(d_head)
@@ -286,11 +285,8 @@ struct Sync {
 };
 
 // One thread: the MMAs of one unit, `ntiles` row tiles of 128 accumulating
-// over nkb K blocks (ring boxes in tile-minor order per K block). The 16-wide
-// K slices go round-robin to P.nch independent accumulators per tile (TMEM
-// columns tmem_d + (i * nch + ch) * Bp): consecutive MMAs into one
-// accumulator wait for each other, so independent chains keep the tensor
-// core busy at this small N. A commit to `done` follows.
+// over nkb K blocks (ring boxes in tile-minor order per K block) into TMEM
+// columns tmem_d + i * Bp, then a commit to `done`.
 __device__ bool issue_unit(const Plan& P, int nkb, int ntiles, uint8_t* ring, const uint8_t* act, uint32_t tmem_d,
                            const Sync& y, uint64_t* done, int& it, int* act_uses, bool need_act,
                            const TokenStepArgs& a, volatile int* s_abort) {
@@ -309,11 +305,8 @@ __device__ bool issue_unit(const Plan& P, int nkb, int ntiles, uint8_t* ring, co
       tc::fence_after();
       const uint64_t da = tc::desc_sw128(smem_u32(ring + (size_t)s * BOX));
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {  // 16-wide K slices: +32 bytes = +2 in descriptor units
-        const int j = kb * 4 + kk, ch = j % P.nch;
-        tc::mma_bf16(tmem_d + (uint32_t)((i * P.nch + ch) * P.Bp), da + 2 * kk, db + 2 * kk, idesc,
-                     j >= P.nch ? 1u : 0u);
-      }
+      for (int kk = 0; kk < 4; ++kk)  // 16-wide K slices: +32 bytes = +2 in descriptor units
+        tc::mma_bf16(tmem_d + (uint32_t)(i * P.Bp), da + 2 * kk, db + 2 * kk, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
       tc::commit(&y.empty[s]);
     }
   }
@@ -321,17 +314,6 @@ __device__ bool issue_unit(const Plan& P, int nkb, int ntiles, uint8_t* ring, co
   return true;
 }
 
-// Sum of the nch accumulators of one tile: 16 consecutive columns c0.. of
-// this warp's 32 TMEM lanes.
-__device__ __forceinline__ void acc_ld16(uint32_t trow, int nch, int Bp, int c0, float* v) {
-  tc::tmem_ld16(trow + c0, v);
-  for (int ch = 1; ch < nch; ++ch) {
-    float w[16];
-    tc::tmem_ld16(trow + ch * Bp + c0, w);
-#pragma unroll
-    for (int j = 0; j < 16; ++j) v[j] += w[j];
-  }
-}
 
 // MMA warp (one thread): the unit sequence of the producer. Waits for the
 // staged activations and a drained accumulator.
@@ -346,7 +328,7 @@ __device__ void mma_issuer(const Plan& P, int Nt, uint8_t* ring, const uint8_t* 
     const int buf = nu & 1;
     if (nu >= 2 && !wait_or_abort(&y.acc_empty[buf], ((nu >> 1) + 1) & 1, a, s_abort, MMA_SLEEP_NS)) return false;
     tc::fence_after();
-    if (!issue_unit(P, nkb, ntiles, ring, act, tmem + (uint32_t)(buf * P.nch * P.Bp), y, &y.acc_full[buf], it,
+    if (!issue_unit(P, nkb, ntiles, ring, act, tmem + (uint32_t)(buf * 64), y, &y.acc_full[buf], it,
                     act_uses, need_act, a, s_abort))
       return false;
     ++nu;
@@ -371,13 +353,13 @@ __device__ void mma_issuer(const Plan& P, int Nt, uint8_t* ring, const uint8_t* 
 // accumulators; column b is batch row b.
 
 // Store the fp32 accumulator tile (128 features x B rows) to part[b][128].
-__device__ void store_partial(uint32_t tbuf, float* part, int B, int Bp, int nch) {
+__device__ void store_partial(uint32_t tbuf, float* part, int B, int Bp) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t trow = tbuf + ((uint32_t)(warp * 32) << 16);
   float* dst = part + warp * 32 + lane;
   for (int c0 = 0; c0 < Bp; c0 += 16) {
     float v[16];
-    acc_ld16(trow, nch, Bp, c0, v);
+    tc::tmem_ld16(trow + c0, v);
 #pragma unroll
     for (int j = 0; j < 16; ++j)
       if (c0 + j < B) __stcg(dst + (size_t)(c0 + j) * 128, v[j]);
@@ -412,6 +394,7 @@ __device__ void ingest_phase(const TokenStepArgs& a, const Plan& P, int jb) {
       } else {
         v = __ldcg(reinterpret_cast<const float4*>(hrow + f));
       }
+      *reinterpret_cast<uint2*>(a.hb + (size_t)b * D + f) = pack_bf16x4(v.x, v.y, v.z, v.w);
       const float mean = warp_sum((v.x + v.y) + (v.z + v.w)) * (1.f / 128.f);
       const float dx = v.x - mean, dy = v.y - mean, dz = v.z - mean, dw = v.w - mean;
       const float m2 = warp_sum((dx * dx + dy * dy) + (dz * dz + dw * dw));
@@ -436,53 +419,43 @@ __device__ void ln_params_to_smem(const TokenStepArgs& a, const Plan& P, int k0,
   }
 }
 
-// G1 activations: rows 0..Bp-1 of features [k0, k0 + 64 kb1) normalised
-// (statistics and parameters in shared memory) -> bf16 in the swizzled
-// K-major operand layout (rows >= B are zero), one K block at a time: block
-// kb is announced on bars[kb] (thread 0, after the worker barrier) so that
-// its MMAs start while the next block is normalised; the loads of block
-// kb + 1 are in flight while block kb is converted. Item = (row, 16-byte
-// chunk of 8 features) of a block; Bp * 8 <= 4 * WORKERS.
-__device__ void ln_to_operand(const TokenStepArgs& a, const Plan& P, int k0, const float* s_g, const float* s_b,
-                              const float* s_mu, const float* s_rs, uint8_t* act, uint64_t* bars, int* staged) {
+// G1 activations: rows 0..Bp-1 of features [k0, k0 + 64 kb1) of the bf16
+// copy of h, staged by TMA straight into the swizzled K-major operand layout
+// (box kb on staged_kb[kb]; rows >= B arrive as zeros), are normalised in
+// place: x = (h - mean) / std * g + beta with the rows' exact fp32
+// statistics, rounded to bf16 again. Block kb is announced on bars[kb]
+// (thread 0, after the worker barrier) as soon as it is done, so its MMAs
+// start while the next block is normalised. Item = (row, 16-byte chunk of 8
+// features) of a block; Bp * 8 <= 4 * WORKERS.
+__device__ void ln_to_operand(const TokenStepArgs& a, const Plan& P, const float* s_g, const float* s_b,
+                              const float* s_mu, const float* s_rs, uint8_t* act, uint64_t* staged_kb,
+                              uint32_t parity, uint64_t* bars, int* staged) {
   constexpr int U = 4;
   const int n_items = P.Bp * 8;
-  float4 cx0[U], cx1[U], nx0[U], nx1[U];
-  auto load = [&](int kb, float4* x0, float4* x1) {
+  for (int kb = 0; kb < P.kb1; ++kb) {
+    mbar_wait_bounded(&staged_kb[kb], parity, a.status, a.wait_cycles);
+    uint8_t* blk = act + (size_t)kb * P.Bp * 128;
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int item = threadIdx.x + u * WORKERS;
       const int b = item >> 3, ch = item & 7;
       if (item < n_items && b < a.B) {
-        const float* src = a.h + (size_t)b * a.D + k0 + kb * 64 + ch * 8;
-        x0[u] = __ldcg(reinterpret_cast<const float4*>(src));
-        x1[u] = __ldcg(reinterpret_cast<const float4*>(src + 4));
-      }
-    }
-  };
-  load(0, cx0, cx1);
-  for (int kb = 0; kb < P.kb1; ++kb) {
-    if (kb + 1 < P.kb1) load(kb + 1, nx0, nx1);
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int item = threadIdx.x + u * WORKERS;
-      if (item >= n_items) continue;
-      const int b = item >> 3, ch = item & 7;
-      uint4 out = make_uint4(0, 0, 0, 0);
-      if (b < a.B) {
+        uint4* cp = reinterpret_cast<uint4*>(blk + tc::sw128_offset(b, ch));
+        const uint4 w = *cp;
+        float x[8];
+        unpack16(w, x, (const bf16*)nullptr);
         const int f = kb * 64 + ch * 8;
         const float mu = s_mu[b], rstd = s_rs[b];
         const float4 g0 = *reinterpret_cast<const float4*>(s_g + f);
         const float4 g1 = *reinterpret_cast<const float4*>(s_g + f + 4);
         const float4 b0 = *reinterpret_cast<const float4*>(s_b + f);
         const float4 b1 = *reinterpret_cast<const float4*>(s_b + f + 4);
-        const uint2 lo = pack_bf16x4((cx0[u].x - mu) * rstd * g0.x + b0.x, (cx0[u].y - mu) * rstd * g0.y + b0.y,
-                                     (cx0[u].z - mu) * rstd * g0.z + b0.z, (cx0[u].w - mu) * rstd * g0.w + b0.w);
-        const uint2 hi = pack_bf16x4((cx1[u].x - mu) * rstd * g1.x + b1.x, (cx1[u].y - mu) * rstd * g1.y + b1.y,
-                                     (cx1[u].z - mu) * rstd * g1.z + b1.z, (cx1[u].w - mu) * rstd * g1.w + b1.w);
-        out = make_uint4(lo.x, lo.y, hi.x, hi.y);
+        const uint2 lo = pack_bf16x4((x[0] - mu) * rstd * g0.x + b0.x, (x[1] - mu) * rstd * g0.y + b0.y,
+                                     (x[2] - mu) * rstd * g0.z + b0.z, (x[3] - mu) * rstd * g0.w + b0.w);
+        const uint2 hi = pack_bf16x4((x[4] - mu) * rstd * g1.x + b1.x, (x[5] - mu) * rstd * g1.y + b1.y,
+                                     (x[6] - mu) * rstd * g1.z + b1.z, (x[7] - mu) * rstd * g1.w + b1.w);
+        *cp = make_uint4(lo.x, lo.y, hi.x, hi.y);
       }
-      *reinterpret_cast<uint4*>(act + (size_t)kb * P.Bp * 128 + tc::sw128_offset(b, ch)) = out;
     }
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     wsync();
@@ -490,8 +463,6 @@ __device__ void ln_to_operand(const TokenStepArgs& a, const Plan& P, int k0, con
       mbar_arrive(&bars[kb]);
       ++staged[kb];
     }
-#pragma unroll
-    for (int u = 0; u < U; ++u) { cx0[u] = nx0[u]; cx1[u] = nx1[u]; }
   }
 }
 
@@ -688,6 +659,7 @@ __device__ void residual_rows(const TokenStepArgs& a, const Plan& P, int l, int 
 #pragma unroll
     for (int sp = 0; sp < S2; ++sp) acc = f4add(acc, ps[sp]);
     __stcg(reinterpret_cast<float4*>(hrow + f), acc);
+    *reinterpret_cast<uint2*>(a.hb + (size_t)r * a.D + f) = pack_bf16x4(acc.x, acc.y, acc.z, acc.w);
     const float mean = warp_sum((acc.x + acc.y) + (acc.z + acc.w)) * (1.f / 128.f);
     const float dx = acc.x - mean, dy = acc.y - mean, dz = acc.z - mean, dw = acc.w - mean;
     const float m2 = warp_sum((dx * dx + dy * dy) + (dz * dz + dw * dw));
@@ -739,15 +711,15 @@ __device__ __forceinline__ void warp_argmax32(float* v, int* ix) {
 }
 
 // LM epilogue of vocabulary tile t: logits (optional) and the tile's argmax per row
-__device__ void lm_epilogue(uint32_t tbuf, int t, const TokenStepArgs& a, int Bp, int nch, float2 (*s_arg)[MAX_B]) {
+__device__ void lm_epilogue(uint32_t tbuf, int t, const TokenStepArgs& a, int Bp, float2 (*s_arg)[MAX_B]) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t trow = tbuf + ((uint32_t)(warp * 32) << 16);
   const int n = t * 128 + warp * 32 + lane;
   for (int c0 = 0; c0 < Bp; c0 += 32) {
     float v[32];
     int ix[32];
-    acc_ld16(trow, nch, Bp, c0, v);
-    if (c0 + 16 < Bp) acc_ld16(trow, nch, Bp, c0 + 16, v + 16);
+    tc::tmem_ld16(trow + c0, v);
+    if (c0 + 16 < Bp) tc::tmem_ld16(trow + c0 + 16, v + 16);
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
       const int m = c0 + j;
@@ -818,13 +790,14 @@ template <int DH>
 __global__ void __launch_bounds__(THREADS, 1)
 token_step2_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mo,
                    const __grid_constant__ CUtensorMap ml, const __grid_constant__ CUtensorMap ma2,
-                   const __grid_constant__ CUtensorMap mxf, const TokenStepArgs a, const Plan P) {
+                   const __grid_constant__ CUtensorMap mxf, const __grid_constant__ CUtensorMap mhb,
+                   const TokenStepArgs a, const Plan P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* ring = smem;
   uint8_t* act = smem + (size_t)P.stages * BOX;
-  __shared__ __align__(8) uint64_t full[MAX_STAGES], empty[MAX_STAGES], act_kb[MAX_KB], acc_full[2],
-      acc_empty[2], win_bar;
+  __shared__ __align__(8) uint64_t full[MAX_STAGES], empty[MAX_STAGES], act_kb[MAX_KB], hb_kb[MAX_KB],
+      acc_full[2], acc_empty[2], win_bar;
   __shared__ uint32_t tmem_slot;
   __shared__ float2 s_arg[4][MAX_B];
   __shared__ float s_mu[MAX_B], s_rs[MAX_B];
@@ -836,7 +809,10 @@ token_step2_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
     }
-    for (int i = 0; i < MAX_KB; ++i) mbar_init(&act_kb[i], 1);
+    for (int i = 0; i < MAX_KB; ++i) {
+      mbar_init(&act_kb[i], 1);
+      mbar_init(&hb_kb[i], 1);
+    }
     mbar_init(&win_bar, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&acc_full[i], 1);
@@ -867,7 +843,8 @@ token_step2_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
     unsigned* cb = a.bar;
     wsync();
     if (threadIdx.x == 0) signal(ctr(cb, C_ARRIVED));
-    int nu = 0, nw = 0;
+    int nu = 0, nw = 0, n_hb = 0;
+    bool hb_pending = false;
     int staged[MAX_KB];  // worker-side uses of each activation barrier (thread 0)
 #pragma unroll
     for (int k = 0; k < MAX_KB; ++k) staged[k] = 0;
@@ -885,14 +862,27 @@ token_step2_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
         const int t = w / P.S1, sp = w % P.S1;
         if (!(ok = workers_wait(a, ctr(cb, C_H), h_ready, &s_abort))) break;
         const bool qkv = t < 3 * P.HG;
+        const int k0 = sp * P.kb1 * 64;
+        // the unit's K range of every row (bf16 copy of h) into the operand
+        // buffer by TMA while the statistics and parameters are gathered
+        if (threadIdx.x == 0) {
+          asm volatile("fence.proxy.async.global;" ::: "memory");
+          for (int kb = 0; kb < P.kb1; ++kb) {
+            mbar_arrive_expect_tx(&hb_kb[kb], (uint32_t)(P.Bp * 128));
+            tc::tma_load_2d(act + (size_t)kb * P.Bp * 128, &mhb, k0 + kb * 64, 0, &hb_kb[kb]);
+          }
+          hb_pending = true;
+        }
         const float* g = layer_ptr(qkv ? a.ln1_g : a.ln2_g, l, a.layer_stride);
         const float* be = layer_ptr(qkv ? a.ln1_b : a.ln2_b, l, a.layer_stride);
         // LayerNorm parameters of the unit's K range after the operand
         float* s_g = reinterpret_cast<float*>(act + (size_t)P.kb1 * P.Bp * 128);
         float* s_b = s_g + P.kb1 * 64;
-        ln_params_to_smem(a, P, sp * P.kb1 * 64, g, be, s_mu, s_rs, s_g, s_b);
+        ln_params_to_smem(a, P, k0, g, be, s_mu, s_rs, s_g, s_b);
         wsync();
-        ln_to_operand(a, P, sp * P.kb1 * 64, s_g, s_b, s_mu, s_rs, act, act_kb, staged);
+        ln_to_operand(a, P, s_g, s_b, s_mu, s_rs, act, hb_kb, (uint32_t)(n_hb & 1), act_kb, staged);
+        ++n_hb;
+        if (threadIdx.x == 0) hb_pending = false;
         const int buf = nu & 1;
         mbar_wait_bounded(&acc_full[buf], (nu >> 1) & 1, a.status, a.wait_cycles);
         tc::fence_after();
@@ -904,7 +894,7 @@ token_step2_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
           window_copies(a, l, hg, nh, ra0, ra1, pos, act, &win_bar);
           win_pending = true;
         }
-        store_partial(tmem + (uint32_t)(buf * P.nch * P.Bp), a.p1 + (size_t)(t * P.S1 + sp) * B * 128, B, P.Bp, P.nch);
+        store_partial(tmem + (uint32_t)(buf * 64), a.p1 + (size_t)(t * P.S1 + sp) * B * 128, B, P.Bp);
         tc::fence_before();
         mbar_arrive(&acc_empty[buf]);
         ++nu;
@@ -940,7 +930,7 @@ token_step2_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
         const int buf = nu & 1;
         mbar_wait_bounded(&acc_full[buf], (nu >> 1) & 1, a.status, a.wait_cycles);
         tc::fence_after();
-        store_partial(tmem + (uint32_t)(buf * P.nch * P.Bp), a.p2 + (size_t)(t2 * P.S2 + sp) * B * 128, B, P.Bp, P.nch);
+        store_partial(tmem + (uint32_t)(buf * 64), a.p2 + (size_t)(t2 * P.S2 + sp) * B * 128, B, P.Bp);
         tc::fence_before();
         mbar_arrive(&acc_empty[buf]);
         ++nu;
@@ -965,7 +955,7 @@ token_step2_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
           const int buf = nu & 1;
           mbar_wait_bounded(&acc_full[buf], (nu >> 1) & 1, a.status, a.wait_cycles);
           tc::fence_after();
-          lm_epilogue(tmem + (uint32_t)(buf * P.nch * P.Bp), t, a, P.Bp, P.nch, s_arg);
+          lm_epilogue(tmem + (uint32_t)(buf * 64), t, a, P.Bp, s_arg);
           mbar_arrive(&acc_empty[buf]);  // lm_epilogue ended with the tcgen05 fence + barrier
           ++nu;
         }
@@ -988,6 +978,8 @@ token_step2_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
     // copies into shared memory still in flight must land before the CTA exits
     if (threadIdx.x == 0) {
       if (win_pending) mbar_wait_bounded(&win_bar, nw & 1, a.status, a.wait_cycles);
+      if (hb_pending)
+        for (int k = 0; k < P.kb1; ++k) mbar_wait_bounded(&hb_kb[k], n_hb & 1, a.status, a.wait_cycles);
       for (int k = 0; k < MAX_KB; ++k)
         if (staged[k] > 0) mbar_wait_bounded(&act_kb[k], (staged[k] - 1) & 1, a.status, a.wait_cycles);
     }
@@ -1109,9 +1101,6 @@ bool make_plan(int B, int D, int dh, int V, int l_cap, int sms, size_t smem_max,
   p.c_a2 = C_G1P + p.T1;
   p.c_g2p = p.c_a2 + 5 * p.HG;
   p.n_slots = p.c_g2p + p.T2;
-  // one accumulator per tile: tcgen05.mma costs ~156 cycles to issue on B200
-  // whatever its N (measured), so independent chains buy nothing here
-  p.nch = 1;
   // the activation buffer: the largest operand, or the attention windows
   size_t act = (size_t)p.kb1 * p.Bp * 128 + (size_t)p.kb1 * 64 * 2 * sizeof(float);  // + LayerNorm parameters
   act = act > (size_t)p.kb2 * p.Bp * 128 ? act : (size_t)p.kb2 * p.Bp * 128;
@@ -1142,7 +1131,8 @@ size_t token_step2_scratch_floats(int B, int D, int which) {
   const int hg = D / 128;
   if (which == 1) return (size_t)7 * hg * S1 * B * 128;   // G1 partials
   if (which == 2) return (size_t)hg * S2 * B * 128;       // G2 partials
-  return (size_t)B * hg * 2;                                     // per-(row, tile) statistics
+  if (which == 4) return (size_t)B * D / 2;               // bf16 copy of h (floats' worth)
+  return (size_t)B * hg * 2;                              // per-(row, tile) statistics
 }
 
 int token_step2_supported(int dt, int B, int D, int H, int rot, int V, int Nt, int l_cap) {
@@ -1167,16 +1157,17 @@ cudaError_t launch_token_step2(const TokenStepArgs& a, const void* w_qkv1, const
   Plan P;
   size_t smem;
   if (!make_plan(a.B, a.D, a.dh, a.V, a.l_cap, d.sms, d.smem_max, &P, &smem)) return cudaErrorNotSupported;
-  CUtensorMap mq, mo, ml, ma2, mxf;
+  CUtensorMap mq, mo, ml, ma2, mxf, mhb;
   // one layer: any stride at least the layer's own size satisfies the encoder
   const long long lsq = a.Nt > 1 ? a.layer_stride : 14LL * a.D * a.D;
   const long long lso = a.Nt > 1 ? a.layer_stride : 10LL * a.D * a.D;
   if (!weight_map(&mq, w_qkv1, a.D, 7LL * a.D, a.Nt, lsq) || !weight_map(&mo, w_o2, 5LL * a.D, a.D, a.Nt, lso) ||
       !weight_map(&ml, w_lm, a.D, a.V, 0, 0))
     return cudaErrorInvalidValue;
-  if (!act_map(&ma2, a.a2, a.B, 5LL * a.D, P.Bp) || !act_map(&mxf, a.xf, a.B, a.D, P.Bp))
+  if (!act_map(&ma2, a.a2, a.B, 5LL * a.D, P.Bp) || !act_map(&mxf, a.xf, a.B, a.D, P.Bp) ||
+      !act_map(&mhb, a.hb, a.B, a.D, P.Bp))
     return cudaErrorInvalidValue;
-  void (*kern)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, TokenStepArgs, Plan) =
+  void (*kern)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, TokenStepArgs, Plan) =
       a.dh == 32 ? token_step2_kernel<32> : (a.dh == 64 ? token_step2_kernel<64> : token_step2_kernel<128>);
   int per_sm = 0;
   cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, THREADS, smem);
@@ -1208,7 +1199,7 @@ cudaError_t launch_token_step2(const TokenStepArgs& a, const void* w_qkv1, const
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  e = cudaLaunchKernelEx(&cfg, kern, mq, mo, ml, ma2, mxf, a, P);
+  e = cudaLaunchKernelEx(&cfg, kern, mq, mo, ml, ma2, mxf, mhb, a, P);
   note_launch();
   return e;
 }
