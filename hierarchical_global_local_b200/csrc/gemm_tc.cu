@@ -39,6 +39,7 @@ constexpr int BK = 64;   // K elements per stage = one 128-byte swizzle row
 constexpr size_t PART_BUDGET = 256;  // split-K reduces in distributed shared memory
 
 constexpr int MAX_STAGES = 8;
+constexpr int MAX_KS = 16;  // K splits of one tile: CTAs of one (non-portable) cluster
 constexpr int THREADS = 192;  // warps 0-3 epilogue, warp 4 TMA producer, warp 5 MMA issuer
 
 template <int BN>
@@ -273,23 +274,26 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
       tc::fence_after();
       const uint32_t tb = trow + (uint32_t)(buf * BN);
       if (ks > 1) {
-        // push this CTA's partial columns to their owners: column c goes to
-        // rank c / (BN/ks), slot [my rank][c % (BN/ks)] of its receive
-        // buffer (remote stores do not wait for a round trip)
+        // push this CTA's partial columns to their owners, four columns per
+        // 16-byte store: column quad c..c+3 goes to rank c / (BN/ks), float4
+        // slot [my rank][(c % (BN/ks)) / 4][row] of its receive buffer
+        // (BN/ks is a multiple of 4; remote stores do not wait for a round
+        // trip)
         namespace cg = cooperative_groups;
         cg::cluster_group cluster = cg::this_cluster();
-        float* recv = reinterpret_cast<float*>(smem + (size_t)stages * stage_bytes<BN>());
-        const int cpr = BN / ks;
+        const uint32_t recv = smem_u32(smem + (size_t)stages * stage_bytes<BN>());
+        const int cpr = BN / ks, qpr = cpr / 4;
         const int me = (int)cluster.block_rank();
         tc::cluster_wait_acquire();  // every CTA of the cluster has started
         for (int c0 = 0; c0 < BN; c0 += 16) {
           float v[16];
           tc::tmem_ld16(tb + c0, v);
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int c = c0 + j;
-            float* dst = cluster.map_shared_rank(recv, c / cpr);
-            dst[((size_t)me * cpr + (c % cpr)) * BM + r] = v[j];
+          for (int u = 0; u < 4; ++u) {
+            const int c = c0 + 4 * u;
+            const uint32_t slot = recv + (uint32_t)((((me * qpr + (c % cpr) / 4) * BM) + r) * 16);
+            tc::st_cluster_v4(tc::map_rank(slot, (uint32_t)(c / cpr)), v[4 * u], v[4 * u + 1],
+                              v[4 * u + 2], v[4 * u + 3]);
           }
         }
       } else if (SWAP && BN <= 64 && e.kind == EPI_LOGITS_ARGMAX) {
@@ -336,15 +340,22 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
         for (int c0 = 0; c0 < BN; c0 += 16) tc::tmem_ld16(tb + c0, v + c0);
         tc::fence_before();
         mbar_arrive(&acc_empty[buf]);
+        if constexpr (SWAP) {
+          const int n = a0 + r;
 #pragma unroll
-        for (int c = 0; c < BN; ++c) {
-          const int m = SWAP ? (b0 + c) : (a0 + r);
-          const int n = SWAP ? (a0 + r) : (b0 + c);
-          if (rope) {
-            const float pv = __shfl_xor_sync(0xffffffffu, v[c], rhalf);
-            if (m < M && n < N) epi_apply_rope<bf16>(e, m, n, v[c], pv);
-          } else if (m < M && n < N) {
-            epi_apply<bf16>(e, m, n, v[c]);
+          for (int c0 = 0; c0 < BN; c0 += 16) {
+            float pv[16];
+            if (rope) {
+#pragma unroll
+              for (int j = 0; j < 16; ++j) pv[j] = __shfl_xor_sync(0xffffffffu, v[c0 + j], rhalf);
+            }
+            if (n < N && b0 + c0 < M) epi_cols<bf16, 16>(e, b0 + c0, 16, n, M, v + c0, pv);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < BN; ++c) {
+            const int m = a0 + r, n = b0 + c;
+            if (m < M && n < N) epi_apply<bf16>(e, m, n, v[c]);
           }
         }
         if (SWAP && e.ln_cnt) post_ln(e, b0, b0 + BN, M, N, ntA, s_rows, &s_nrows);
@@ -370,20 +381,16 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
         tc::fence_before();
         mbar_arrive(&acc_empty[buf]);
       } else {
+        // weights as A with BN > 64 (the activations-as-A path is above)
+        const int n = a0 + r;
         for (int c0 = 0; c0 < BN; c0 += 16) {
-          float v[16];
+          float v[16], pv[16];
           tc::tmem_ld16(tb + c0, v);
+          if (rope) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int m = SWAP ? (b0 + c0 + j) : (a0 + r);
-            const int n = SWAP ? (a0 + r) : (b0 + c0 + j);
-            if (rope) {
-              const float pv = __shfl_xor_sync(0xffffffffu, v[j], rhalf);
-              if (m < M && n < N) epi_apply_rope<bf16>(e, m, n, v[j], pv);
-            } else if (m < M && n < N) {
-              epi_apply<bf16>(e, m, n, v[j]);
-            }
+            for (int j = 0; j < 16; ++j) pv[j] = __shfl_xor_sync(0xffffffffu, v[j], rhalf);
           }
+          if (n < N && b0 + c0 < M) epi_cols<bf16, 16>(e, b0 + c0, 16, n, M, v, pv);
         }
         tc::fence_before();
         mbar_arrive(&acc_empty[buf]);
@@ -408,21 +415,45 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
       const bool rope = SWAP && e.kind == EPI_QKV1_ROPE;
       const int rhalf = e.rot >> 1;
       const int a0 = (t_first % ntA) * BM, b0 = (t_first / ntA) * BN;
-      const float* recv = reinterpret_cast<const float*>(smem + (size_t)stages * stage_bytes<BN>());
-      const int cpr = BN / ks;
+      const uint32_t recv = smem_u32(smem + (size_t)stages * stage_bytes<BN>());
+      const int cpr = BN / ks, qpr = cpr / 4;
       const int cbeg = (int)cluster.block_rank() * cpr;
-      for (int cc = 0; cc < cpr; ++cc) {
-        float acc = 0.f;
-        for (int p = 0; p < ks; ++p) acc += recv[((size_t)p * cpr + cc) * BM + r];
-        const int c = cbeg + cc;
-        const int m = SWAP ? (b0 + c) : (a0 + r);
-        const int n = SWAP ? (a0 + r) : (b0 + c);
-        if (rope) {
-          const float pv = __shfl_xor_sync(0xffffffffu, acc, rhalf);
-          if (m < M && n < N) epi_apply_rope<bf16>(e, m, n, acc, pv);
-        } else if (m < M && n < N) {
-          epi_apply<bf16>(e, m, n, acc);
+      // split K is weights-as-A only: feature n = a0 + r, rows b0 + c.
+      // Chunks of up to 16 rows: the partial sums first (shared-memory
+      // loads only), then the epilogue's loads, then its stores.
+      const int n = a0 + r;
+      for (int cc0 = 0; cc0 < cpr; cc0 += 16) {
+        const int cnt = (cpr - cc0 < 16) ? cpr - cc0 : 16;
+        float acc[16], pv[16];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          // the ks partials of column quad cc0/4 + u, all loads in flight,
+          // summed in rank order
+          float4 part[MAX_KS];
+          const int q = cc0 / 4 + u;
+#pragma unroll
+          for (int p = 0; p < MAX_KS; ++p)
+            if (p < ks && 4 * u < cnt) part[p] = tc::ld_shared_v4(recv + (uint32_t)(((p * qpr + q) * BM + r) * 16));
+          float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+          for (int p = 0; p < MAX_KS; ++p)
+            if (p < ks && 4 * u < cnt) {
+              t.x += part[p].x;
+              t.y += part[p].y;
+              t.z += part[p].z;
+              t.w += part[p].w;
+            }
+          acc[4 * u] = t.x;
+          acc[4 * u + 1] = t.y;
+          acc[4 * u + 2] = t.z;
+          acc[4 * u + 3] = t.w;
         }
+        if (rope) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) pv[j] = __shfl_xor_sync(0xffffffffu, acc[j], rhalf);
+        }
+        const int m0 = b0 + cbeg + cc0;
+        if (n < N && m0 < M) epi_cols<bf16, 16>(e, m0, cnt, n, M, acc, pv);
       }
       if (SWAP && e.ln_cnt) post_ln(e, b0 + cbeg, b0 + cbeg + cpr, M, N, ntA, s_rows, &s_nrows);
     }
@@ -486,19 +517,20 @@ cudaError_t prepare_one() {
   const size_t mx = (size_t)optin - fa.sharedSizeBytes;
   e = cudaFuncSetAttribute(gemm_tc_kernel<BN, SWAP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)mx);
+  // split-K clusters of up to 16 CTAs (above the portable 8)
+  if (e == cudaSuccess && SWAP)
+    e = cudaFuncSetAttribute(gemm_tc_kernel<BN, SWAP>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   if (e == cudaSuccess) dyn_smem_max<BN, SWAP>() = mx;
   return e;
 }
 
 int sm_count() { return device_sm_count(); }
 
+// Ring depth and dynamic shared memory of one launch with ks K splits.
 template <int BN, bool SWAP>
-cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& mb, int M, int N, int nkb,
-                       int ks, int ntA, int ntB, int xk_split, int xk_off, const Epi& e,
-                       int* status, cudaStream_t s) {
+size_t launch_smem(int nkb, int ks, int* stages_out) {
   constexpr size_t SB = stage_bytes<BN>();
   const size_t SMEM_MAX = dyn_smem_max<BN, SWAP>();
-  if (SMEM_MAX < 3 * SB) return cudaErrorInvalidConfiguration;
   const int nloc = (nkb + ks - 1) / ks;
   int stages = (int)((SMEM_MAX - 1024) / SB);
   if (stages > MAX_STAGES) stages = MAX_STAGES;
@@ -518,7 +550,66 @@ cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& mb, int M, int 
     if (stages > fit) stages = fit;
   }
   if (stages < 2) stages = 2;
-  const size_t smem = (size_t)stages * SB + recv_bytes + tr_bytes + 1024;
+  *stages_out = stages;
+  return (size_t)stages * SB + recv_bytes + tr_bytes + 1024;
+}
+
+// CTAs of ks-CTA clusters that fit on the device at once with this much
+// shared memory (the occupancy calculator's cluster count times ks), cached
+// per device, instantiation, split and size.
+template <int BN, bool SWAP>
+int resident_ctas(int ks, size_t smem) {
+  struct Entry { int dev, ks; size_t smem; int ctas; };
+  static Entry cache[64];
+  static int n_cache = 0;
+  const int dev = current_device();
+  for (int i = 0; i < n_cache; ++i)
+    if (cache[i].dev == dev && cache[i].ks == ks && cache[i].smem == smem) return cache[i].ctas;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(1, 1, ks);
+  cfg.blockDim = dim3(THREADS, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = ks;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int clusters = 0;
+  if (cudaOccupancyMaxActiveClusters(&clusters, gemm_tc_kernel<BN, SWAP>, &cfg) != cudaSuccess) {
+    cudaGetLastError();  // not sticky: clear it
+    clusters = 0;
+  }
+  const int ctas = clusters * ks;
+  if (n_cache < 64) cache[n_cache++] = Entry{dev, ks, smem, ctas};
+  return ctas;
+}
+
+// K splits of a weights-as-A launch with nt feature tiles and nkb K blocks:
+// the largest power of two <= 16 whose nt * ks CTAs all fit on the device
+// at once (one wave: the cluster shape limits residency below one CTA per
+// SM) with at least one K block per split; 1 (persistent over the tiles)
+// when even two splits do not fit.
+template <int BN>
+int plan_splits(int nt, int nkb) {
+  for (int ks = MAX_KS; ks >= 2; ks >>= 1) {
+    if (nkb < ks || BN / ks < 4) continue;  // a K block per split; column quads per rank
+    int stages = 0;
+    const size_t smem = launch_smem<BN, true>(nkb, ks, &stages);
+    if (nt * ks <= resident_ctas<BN, true>(ks, smem)) return ks;
+  }
+  return 1;
+}
+
+template <int BN, bool SWAP>
+cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& mb, int M, int N, int nkb,
+                       int ks, int ntA, int ntB, int xk_split, int xk_off, const Epi& e,
+                       int* status, cudaStream_t s) {
+  constexpr size_t SB = stage_bytes<BN>();
+  if (dyn_smem_max<BN, SWAP>() < 3 * SB) return cudaErrorInvalidConfiguration;
+  int stages = 0;
+  const size_t smem = launch_smem<BN, SWAP>(nkb, ks, &stages);
   const int ntiles = ntA * ntB;
   dim3 grid;
   if (ks > 1) {
@@ -611,12 +702,18 @@ cudaError_t launch_gemm_tc(int dt, const void* X, int ldx, const void* W, int ld
     const int nt = (N + BM - 1) / BM;
     if (!make_map(&ma, W, N, K, ldw, BM) || !make_map(&mb, X, M, xcols, ldx, BN))
       return cudaErrorInvalidValue;
-    // K splits (a power of two <= 8, the portable cluster size): the fewest
-    // that put a CTA on every SM, each split keeping >= 2 K blocks. Without
-    // a split the kernel runs persistent over the tiles.
+    // K splits: as many as fit in one wave (plan_splits); without a split
+    // the kernel runs persistent over the tiles. The argmax epilogue needs
+    // whole tiles.
     int ks = 1;
-    while (ks < 8 && nt * ks < sm_count() && nkb / (ks * 2) >= 2) ks *= 2;
-    if (e.kind == EPI_LOGITS_ARGMAX) ks = 1;  // the argmax epilogue needs whole tiles
+    if (e.kind != EPI_LOGITS_ARGMAX) {
+      switch (BN) {
+        case 32: ks = plan_splits<32>(nt, nkb); break;
+        case 64: ks = plan_splits<64>(nt, nkb); break;
+        case 128: ks = plan_splits<128>(nt, nkb); break;
+        default: ks = plan_splits<256>(nt, nkb); break;
+      }
+    }
     switch (BN) {
       case 32: return launch_one<32, true>(ma, mb, M, N, nkb, ks, nt, 1, xk_split, xk_off, e, status, s);
       case 64: return launch_one<64, true>(ma, mb, M, N, nkb, ks, nt, 1, xk_split, xk_off, e, status, s);
