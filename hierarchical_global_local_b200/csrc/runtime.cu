@@ -398,34 +398,27 @@ int bt_create(const bt_config* cfg, const bt_weights* w, void* ws, size_t ws_byt
   if (m->ts_cnt) BT_TRYC(cudaMemsetAsync(m->ts_cnt, 0, (size_t)d.Bmax * d.H * sizeof(int), st));
   if (m->ts2_ctr) BT_TRYC(cudaMemsetAsync(m->ts2_ctr, 0, m->ts2_ctr_bytes, st));
   {
-    // Decode calls re-read two regions every token step: the LM head and the
-    // token decoder's local caches (K and V of every layer, at most
-    // P + L_B - 1 rows per sequence and head). The fused token-step launches
-    // carry a persisting L2 access-policy window over both (adjacent in the
-    // workspace), and this context's persisting set-aside is sized to it as
-    // far as the device allows; when the window is larger than the set-aside
-    // the hit ratio keeps that fraction of it (BT_L2_WINDOW=0 turns it off).
+    // The token decoder's local caches (K and V of every layer, at most
+    // P + L_B - 1 rows per sequence and head) are written and re-read by
+    // every token step of a block: the fused token-step launches carry a
+    // persisting L2 access-policy window over them, and this context's
+    // persisting set-aside is sized to it as far as the device allows (hit
+    // ratio = the fraction that fits). The weights, LM head included, stream
+    // through with an evict-first hint. BT_L2_WINDOW=0 turns the window off.
     const char* env = getenv("BT_L2_WINDOW");
-    const size_t kv = d.Nt > 0 ? 2 * m->kt_layer * d.Nt * d.eb : 0;
-    const size_t bytes = kv > 0 ? (size_t)((uint8_t*)m->vt + kv / 2 - (uint8_t*)m->w_lm) : 0;
+    const size_t kv = d.Nt > 0 ? (size_t)((uint8_t*)m->vt + m->kt_layer * d.Nt * d.eb - (uint8_t*)m->kt) : 0;
     int dev = 0, max_persist = 0, max_window = 0;
-    if (bytes > 0 && !(env && env[0] == '0') && cudaGetDevice(&dev) == cudaSuccess &&
+    if (kv > 0 && !(env && env[0] == '0') && cudaGetDevice(&dev) == cudaSuccess &&
         cudaDeviceGetAttribute(&max_persist, cudaDevAttrMaxPersistingL2CacheSize, dev) == cudaSuccess &&
         cudaDeviceGetAttribute(&max_window, cudaDevAttrMaxAccessPolicyWindowSize, dev) == cudaSuccess &&
-        max_persist > 0 && max_window > 0) {
-      void* base = m->w_lm;
-      size_t win = bytes;
-      if (win > (size_t)max_window) {  // the local caches alone
-        base = m->kt;
-        win = kv;
-      }
-      const size_t want = std::min(win, (size_t)max_persist);
+        max_persist > 0 && max_window > 0 && kv <= (size_t)max_window) {
+      const size_t want = std::min(kv, (size_t)max_persist);
       size_t cur = 0;
-      if (win <= (size_t)max_window && cudaDeviceGetLimit(&cur, cudaLimitPersistingL2CacheSize) == cudaSuccess &&
+      if (cudaDeviceGetLimit(&cur, cudaLimitPersistingL2CacheSize) == cudaSuccess &&
           (cur >= want || cudaDeviceSetLimit(cudaLimitPersistingL2CacheSize, want) == cudaSuccess)) {
-        m->l2_base = base;
-        m->l2_window = win;
-        m->l2_hit = (float)std::min(1.0, (double)std::max(cur, want) / (double)win);
+        m->l2_base = m->kt;
+        m->l2_window = kv;
+        m->l2_hit = (float)std::min(1.0, (double)std::max(cur, want) / (double)kv);
       }
       cudaGetLastError();
     }

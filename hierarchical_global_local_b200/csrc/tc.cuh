@@ -164,14 +164,6 @@ __device__ __forceinline__ void tma_load_3d_hint(void* dst, const CUtensorMap* m
       : "memory");
 }
 
-// prefetch one tiled TMA box into L2 (nothing is written to shared memory and
-// no barrier is signalled), with an L2 cache policy
-__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int x, int y, uint64_t policy) {
-  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile.L2::cache_hint [%0, {%1, %2}], %3;" ::"l"(
-                   reinterpret_cast<uint64_t>(map)),
-               "r"(x), "r"(y), "l"(policy)
-               : "memory");
-}
 
 // byte offset of 16-byte chunk `c` (0..7) of row `r` in a 128-byte swizzled
 // K-major tile: the layout a TMA load with SWIZZLE_128B writes

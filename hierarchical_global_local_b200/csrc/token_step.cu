@@ -230,11 +230,11 @@ __device__ void producer(const CUtensorMap* mq, const CUtensorMap* mo, const CUt
   const int G = gridDim.x, c = blockIdx.x;
   int it = 0;
   bool stop = false;
-  uint64_t first, keep;
-  // weights are read once per step: keep them from evicting the activations,
-  // partial sums and the local window that the phases exchange through L2
+  uint64_t first;
+  // weights, LM head included, are read once per step: keep them from
+  // evicting the activations, partial sums and the local window that the
+  // phases exchange through L2
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(first));
-  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(keep));
   auto load = [&](const CUtensorMap* m, int x, int y, int z, bool three) {
     if (stop) return;
     const int s = it % P.stages;
@@ -245,14 +245,9 @@ __device__ void producer(const CUtensorMap* mq, const CUtensorMap* mo, const CUt
     }
     mbar_arrive_expect_tx(&full[s], BOX);
     if (three) tc::tma_load_3d_hint(ring + (size_t)s * BOX, m, x, y, z, &full[s], first);
-    else tc::tma_load_2d(ring + (size_t)s * BOX, m, x, y, &full[s]);  // LM head: the launch's L2 window decides
+    else tc::tma_load_2d_hint(ring + (size_t)s * BOX, m, x, y, &full[s], first);
     ++it;
   };
-  // the LM head's tiles of this CTA go to L2 while the layers run (HBM is
-  // far from busy then), a share after each layer's loads
-  const int my_lm = c < P.TL ? (P.TL - 1 - c) / G + 1 : 0;
-  const int lm_boxes = my_lm * P.kbL;
-  int lm_done = 0;
   for (int l = 0; l < Nt && !stop; ++l) {
     for (int w = first_g1(P, c); w < P.N1 && !stop; w += G) {
       const int t = w / P.S1, sp = w % P.S1;
@@ -261,11 +256,6 @@ __device__ void producer(const CUtensorMap* mq, const CUtensorMap* mo, const CUt
     for (int w = first_g2(P, c, G); w < P.N2 && !stop; w += G) {
       const int t = w / P.S2, sp = w % P.S2;
       for (int kb = 0; kb < P.kb2; ++kb) load(mo, (sp * P.kb2 + kb) * 64, t * 128, l, true);
-    }
-    const int upto = (int)((long long)lm_boxes * (l + 1) / Nt);
-    for (; lm_done < upto && !stop; ++lm_done) {
-      const int t = c + (lm_done / P.kbL) * G, kb = lm_done % P.kbL;
-      tc::tma_prefetch_2d(ml, kb * 64, t * 128, keep);
     }
   }
   for (int t = c; t < P.TL && !stop; t += G)
