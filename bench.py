@@ -280,6 +280,7 @@ def run_ours(args):
     if ws == 1 and not args.no_extra:
         with ClockSampler(local) as clk_x:
             line["runs_extra"] = run_extras(flush, hbm, tf_sus)
+            line["runs_extra"]["batch_sweep"] = run_batch_sweep(flush, hbm, tf_sus, cap=args.max_batch_cap)
         line["runs_extra"]["clocks"] = clk_x.summary()
         line["runs_extra"]["note"] = ("timed once each after an untimed run, outside value; the pages "
                                       "report 10-20x Block Transformer throughput over vanilla models of "
@@ -453,6 +454,80 @@ def run_extras(flush, hbm: float, tf_sus: float):
         for k in ("lb2", "lb4", "lb8"):
             if k in out:
                 out[k]["vs_vanilla"] = out[k]["tokens_per_s"] / v
+    return out
+
+
+SWEEP_RUNS = ("pythia160m_prefill_heavy", "pythia160m_decode_heavy")
+SWEEP_BATCHES = (1, 32, 256)
+SWEEP_MEMORY_FRACTION = 0.85  # of the device memory free when the sweep starts
+
+
+def run_batch_sweep(flush, hbm: float, tf_sus: float, cap: int = 0):
+    """Batch-size sensitivity and the maximum-throughput setting of the
+    method's evaluation: the pythia160m-scale prefill-heavy and decode-heavy
+    runs at batch 1, 32, 256 and the largest batch the device holds (every
+    model at its own memory-maximising batch, FlexGen's "maximum throughput"),
+    each timed once after an untimed run, plus memory per sample of the
+    Block Transformer against the vanilla L_B = 1 model. The largest batch is
+    the planner's (loader.max_batch_by_memory) for SWEEP_MEMORY_FRACTION of
+    the free device memory; cap > 0 bounds it."""
+    import torch
+    from hierarchical_global_local_b200 import costmodel as cm
+    from hierarchical_global_local_b200 import loader
+    stream = torch.cuda.current_stream()
+    free, total = torch.cuda.mem_get_info()
+    budget = int(free * SWEEP_MEMORY_FRACTION)
+    wl0 = synth.WORKLOADS[SWEEP_RUNS[0]]
+    shape, max_seq = wl0.shape, max(synth.WORKLOADS[r].max_seq for r in SWEEP_RUNS)
+    per_sample = loader.memory_per_sample(shape, max_seq)
+    ws1 = loader.workspace_bytes(shape, 1, max_seq)
+    b_mem = int((budget - ws1) // per_sample) + 1 if budget > ws1 else 0
+    b_max = loader.max_batch_by_memory(shape, max_seq, budget)
+    if cap > 0:
+        b_max = min(b_max, cap)
+    batches = sorted({b for b in SWEEP_BATCHES if b <= b_max} | {b_max})
+    out = {"budget_GB": budget / 1e9, "device_total_GB": total / 1e9,
+           "memory_per_sample_MB": per_sample / 1e6,
+           "max_batch_by_memory": b_mem,
+           "max_batch_run": b_max,
+           "max_batch_bound": "memory" if b_max >= b_mem else
+                              ("cap" if cap > 0 and b_max == cap else
+                               "32-bit buffer indexing (bt_config.max_batch)"),
+           "runs": {}}
+    model = loader.build_model(shape, synth.make_weights(wl0), b_max, max_seq)
+    for r in SWEEP_RUNS:
+        wl = synth.WORKLOADS[r]
+        toks = synth.make_tokens(wl, batch=b_max)
+        res = {}
+        for bs in batches:
+            prompt = torch.from_numpy(np.ascontiguousarray(toks[:bs, :wl.prompt_len])).cuda()
+            gen = torch.empty(wl.gen_len, bs, dtype=torch.int32, device="cuda")
+            generate(model, prompt, wl.gen_len, gen)
+            model.sync()
+            flush.fill_(4)
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            generate(model, prompt, wl.gen_len, gen)
+            b.record(stream)
+            model.sync()
+            ms = a.elapsed_time(b)
+            t_roof = cm.generate(cm.Shape.of(shape), bs, wl.prompt_len, wl.gen_len).roofline_seconds(hbm, tf_sus)
+            res[str(bs)] = {"ms": ms, "tokens_per_s": bs * wl.gen_len / (ms / 1e3),
+                            "roofline_ms": t_roof * 1e3, "frac_of_roofline": t_roof / (ms / 1e3)}
+            del prompt, gen
+        out["runs"][r] = res
+    model.close()
+    del model
+    torch.cuda.empty_cache()
+    # memory per sample across L_B at equal width and depth (the L_B sweep
+    # family, prompt 2,048 + 512 generated): L_B = 1 is the vanilla model
+    mem = {}
+    for lb in (1, 2, 4, 8):
+        w = synth.WORKLOADS[f"lb_sweep_L{lb}"]
+        mem[f"L_B={lb}"] = loader.memory_per_sample(w.shape, w.max_seq) / 1e6
+    out["lb_sweep_memory_per_sample_MB"] = mem
+    out["vanilla_over_lb4_memory_per_sample"] = mem["L_B=1"] / mem["L_B=4"]
     return out
 
 
@@ -662,11 +737,15 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-extra", action="store_true",
                     help="skip runs_extra (L_B sweep incl. vanilla, pythia410m-scale, long context)")
+    ap.add_argument("--max-batch-cap", type=int, default=0,
+                    help="bound on the largest batch of the batch sweep (0: the planner's, memory and "
+                         "buffer indexing only)")
     ap.add_argument("--cpu-seconds", type=float, default=20.0,
                     help="time budget of the cpu_baseline leg of our arm")
     ap.add_argument("--ref-seconds", type=float, default=60.0,
                     help="--impl reference: oracle time budget over all warm-up and timed steps")
-    ap.add_argument("--case", default=None, choices=["decode", "prefill", "decode_attention", "linear", "lb_sweep"],
+    ap.add_argument("--case", default=None, choices=["decode", "prefill", "decode_attention", "linear", "lb_sweep",
+                                                     "batch_sweep"],
                     help="instead of the benchmark, run a bounded case for profiler captures: decode "
                          "calls of the decode-heavy workload, or one op of the path")
     ap.add_argument("--case-steps", type=int, default=None,
@@ -683,6 +762,14 @@ def main():
     if args.case == "lb_sweep":
         args.case_steps = args.case_steps or 0
         run_lb_sweep(args)
+        return
+    if args.case == "batch_sweep":
+        import torch
+        torch.cuda.set_device(0)
+        flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+        hbm, _, tf_sus, _ = _peaks()
+        print(json.dumps({"case": "batch_sweep",
+                          **run_batch_sweep(flush, hbm, tf_sus, cap=args.max_batch_cap)}), flush=True)
         return
     if args.case is not None and args.case_steps is None:
         args.case_steps = 8

@@ -100,6 +100,18 @@ int dims_of(const bt_config* c, Dims* o) {
   d.eb = dt_size(d.dt);
   d.n_cap = (d.max_seq + d.L - 1) / d.L;
   d.l_cap = d.tokdec ? d.P + d.L - 1 : 1;
+  {
+    // every buffer's element count must stay below 2^31: kernels index
+    // within one buffer (one layer of a cache) with 32-bit arithmetic. The
+    // widest per-row activation buffer is [rows, 5D] (attention output |
+    // GELU(fc1), the out|fc2 GEMM's input)
+    const long long lim = 1LL << 31;
+    const long long B = d.Bmax, D = d.D;
+    const long long rows = B * (d.n_cap > d.l_cap ? d.n_cap : d.l_cap);
+    const long long vt_ld = (d.n_cap + 63) / 64 * 64;
+    if (rows * 5 * D >= lim || B * d.V >= lim || B * D * vt_ld >= lim || B * D * d.n_cap >= lim)
+      return BT_ENOTSUP;
+  }
   const int rows_blk = d.Bmax * d.n_cap;
   // token-decoder rows of one call: P prefix rows plus up to L_B - 1
   // trailing prompt tokens at prefill

@@ -69,3 +69,56 @@ def teacher_forced_logits(model: native.BlockTransformer, tokens: np.ndarray, T:
         model.decode(tok[:, T + i].contiguous(), logits=logits[i + 1], next_tokens=nxt[i + 1])
     model.sync()
     return logits.cpu().numpy(), nxt.cpu().numpy()
+
+
+# ---- memory planning: the maximum-throughput methodology --------------------
+# The method's throughput comparisons use, for every model, the largest batch
+# that fits in device memory (FlexGen's "maximum throughput" setting), and
+# report the memory one sequence costs. A model's device footprint is exactly
+# its workspace (bt_workspace_bytes: repacked weights, block and local KV
+# caches, activation buffers and scratch, all sized from the configuration);
+# the caller's original weight buffers are no longer read once bt_create's
+# copy has run. So both numbers follow from the workspace formula alone.
+
+def workspace_bytes(shape, max_batch: int, max_seq: int) -> int:
+    """Device bytes of a model with room for max_batch sequences of max_seq
+    tokens (0 if the configuration is invalid, for instance too large)."""
+    try:
+        return native.workspace_bytes(model_config(shape, max_batch, max_seq))
+    except native.BtError:
+        return 0
+
+
+def memory_per_sample(shape, max_seq: int) -> float:
+    """Bytes each additional sequence of max_seq tokens adds to the model's
+    footprint: the slope of the workspace in the batch capacity between 32
+    and 64 sequences (block and local KV caches, per-row activation buffers,
+    logits; a few scratch buffers follow the launch plan, so the slope
+    varies by under 1 % elsewhere)."""
+    lo, hi = 32, 64
+    a, b = workspace_bytes(shape, lo, max_seq), workspace_bytes(shape, hi, max_seq)
+    if a == 0 or b == 0:
+        raise ValueError("invalid configuration")
+    return (b - a) / (hi - lo)
+
+
+def max_batch_by_memory(shape, max_seq: int, budget_bytes: int, limit: int = 1 << 20) -> int:
+    """The largest batch capacity B <= limit whose workspace fits in
+    budget_bytes (0 if not even one sequence fits). The workspace grows with
+    B, so a doubling search followed by bisection finds it."""
+    def fits(b: int) -> bool:
+        n = workspace_bytes(shape, b, max_seq)
+        return 0 < n <= budget_bytes
+    if not fits(1):
+        return 0
+    lo, hi = 1, 2
+    while hi <= limit and fits(hi):
+        lo, hi = hi, hi * 2
+    hi = min(hi, limit + 1)
+    while hi - lo > 1:  # fits(lo), not fits(hi) (or hi past the limit)
+        mid = (lo + hi) // 2
+        if fits(mid):
+            lo = mid
+        else:
+            hi = mid
+    return lo

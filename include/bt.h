@@ -79,7 +79,12 @@ typedef struct bt_config {
   int32_t rotary_dims;       /* even, <= d_head                               */
   int32_t use_token_decoder; /* 0: vanilla model, requires block_len = 1; the
                                 LM head reads LN_b of the block decoder      */
-  int32_t max_batch;         /* B_max                                         */
+  int32_t max_batch;         /* B_max. Every device buffer must hold fewer
+                                than 2^31 elements (kernels index within one
+                                buffer in 32 bits): B_max * ceil(max_seq/L_B)
+                                * 5 d_model, B_max * vocab and B_max * d_model
+                                * ceil(max_seq/L_B) (rounded up to 64) must
+                                stay below 2^31, else BT_ENOTSUP            */
   int32_t max_seq;           /* prompt + generated tokens, per sequence       */
   int32_t dtype;             /* bt_dtype: storage and GEMM-input type; fp32
                                 accumulation and fp32 residual stream always  */

@@ -72,10 +72,37 @@ def test_pythia410m_decode_heavy_full_batch():
     _run("pythia410m_decode_heavy", G=G, check=set(range(0, G, 16)) | {1, 2, 3, G - 1}, n_rows=3)
 
 
+def test_pythia160m_decode_heavy_full_length():
+    """All 2,048 generated steps: the block cache reaches its full length
+    (n = 544 entries) through the model path."""
+    G = 2048
+    _run("pythia160m_decode_heavy", G=G, check=set(range(0, G, 64)) | {G - 4, G - 3, G - 2, G - 1},
+         n_rows=2)
+
+
+def test_pythia410m_decode_heavy_full_length():
+    G = 2048
+    _run("pythia410m_decode_heavy", G=G, check=set(range(0, G, 128)) | {G - 2, G - 1}, n_rows=2)
+
+
 @pytest.mark.parametrize("lb", [1, 2, 4, 8])
 def test_lb_sweep_full_batch_and_prompt(lb):
-    _run(f"lb_sweep_L{lb}", G=2 * max(lb, 2) + 1, check=set(range(2 * max(lb, 2) + 1)), n_rows=1)
+    _run(f"lb_sweep_L{lb}", G=2 * max(lb, 2) + 1, check=set(range(2 * max(lb, 2) + 1)), n_rows=2)
 
 
 def test_long_context_full_batch_and_prompt():
-    _run("long_context", G=5, check=set(range(5)), n_rows=1)
+    _run("long_context", G=5, check=set(range(5)), n_rows=2)
+
+
+def test_pythia160m_prefill_heavy_at_the_largest_batch():
+    """The maximum-throughput setting: the batch the memory planner allows
+    for 85 % of the free device memory (on a 180 GB B200 the 32-bit buffer
+    limit of bt_config.max_batch binds first, at 1,028), full prompt, sampled
+    rows against the oracle."""
+    from hierarchical_global_local_b200 import loader
+    torch = gh.torch_mod()
+    wl = synth.WORKLOADS["pythia160m_prefill_heavy"]
+    free, _ = torch.cuda.mem_get_info()
+    B = loader.max_batch_by_memory(wl.shape, wl.max_seq, int(0.85 * free))
+    assert B >= 256
+    _run("pythia160m_prefill_heavy", G=6, check=set(range(6)), n_rows=3, batch=B)
