@@ -35,6 +35,17 @@ Readings where the page is silent (each listed again in the design notes):
   R8  A prompt whose length is not a multiple of L_B without padding: its
       trailing T mod L_B tokens form the incomplete current block and enter
       the token decoder (the model's own definition of those positions).
+  R9  Summation injection ([BT] §3.4 "The Token Decoder", alternatives to
+      prefix tokens: MEGABYTE-style sum): Proj maps c to L_B vectors
+      s_0..s_{L_B-1} (W_s [L_B*D, D] + b_s, row-major as in R4); the token
+      decoder's input rows are s_0 (the position that predicts the block's
+      first token, where no token of the block is known yet) and
+      s_j + E(x_{j-1}) for j = 1..L_B-1, at positions 0..L_B-1.
+  R10 Window of previous context embeddings ([BT] §6 "Limitations",
+      App. B.3 direction): the prefix holds Proj(c) of the last w context
+      embeddings c_{i-w+1} .. c_i, oldest first, each through the same
+      projection (w*P rows); context embeddings before the first block are
+      zero vectors (their rows are b_p). w = 1 is the base model.
 
 Pins (tests/test_oracle_*.py): HF GPTNeoX (an independent Pythia
 implementation) for the layer stack and the vanilla special case;
@@ -217,6 +228,9 @@ class BlockTransformerOracle:
                  dtype=np.float64):
         self.s = shape
         self.dtype = dtype
+        self.sum_injection = getattr(shape, "injection", "prefix") == "sum"
+        self.window = int(getattr(shape, "context_window", 1))
+        assert self.window >= 1 and not (self.sum_injection and self.window > 1)
         get = (lambda n: np.asarray(params[n], dtype=dtype))
         gl = ["blk_emb", "lnf_b_g", "lnf_b_b", "w_lm"]
         if shape.use_token_decoder:
@@ -258,6 +272,34 @@ class BlockTransformerOracle:
     def _fresh(self, layers) -> List[KVCache]:
         return [KVCache() for _ in layers]
 
+    # ---- context injection (R4, R9, R10) ---------------------------------
+    @property
+    def n_ctx_rows(self) -> int:
+        """Rows in front of a block's tokens in the token decoder: w * P
+        projected prefix rows, or the one row s_0 of summation injection."""
+        return 1 if self.sum_injection else self.window * self.s.prefix_len
+
+    def context_input(self, c_win: np.ndarray) -> Tuple[np.ndarray, Optional[np.ndarray]]:
+        """c_win: [B, w, D] the window's context embeddings, oldest first.
+        Returns the context rows [B, n_ctx_rows, D] and, in summation
+        injection, the vectors added to the token rows 1..L_B-1
+        ([B, L_B - 1, D], else None)."""
+        B, w, D = c_win.shape
+        if self.sum_injection:
+            sv = prefix_projection(c_win[:, -1], self.g["w_prefix"], self.g["b_prefix"], self.s.block_len)
+            return sv[:, :1], sv[:, 1:]
+        rows = prefix_projection(c_win, self.g["w_prefix"], self.g["b_prefix"], self.s.prefix_len)
+        return rows.reshape(B, w * self.s.prefix_len, D), None
+
+    def token_rows(self, tok: np.ndarray, j: np.ndarray, add: Optional[np.ndarray]) -> np.ndarray:
+        """Input rows of tokens tok [B, r] at in-block offsets j [r] (token
+        j of the block is the input of row n_ctx + j): E(x), plus s_{j+1} in
+        summation injection."""
+        rows = self.g["tok_emb"][tok]
+        if add is not None:
+            rows = rows + add[:, j]
+        return rows
+
     # ---- full-sequence, teacher-forced layout ----------------------------
     def forward_full(self, tokens: np.ndarray) -> np.ndarray:
         """Teacher-forced logits for every predictable position.
@@ -282,18 +324,21 @@ class BlockTransformerOracle:
             assert L == 1
             pred[:, 1:n + 1] = c @ self.g["w_lm"].T
             return pred
-        P = s.prefix_len
+        P = self.n_ctx_rows
         D = s.d_model
-        # block k (1..n) is predicted from c_{k-1}
-        prefix = prefix_projection(c, self.g["w_prefix"], self.g["b_prefix"], P)
+        w = self.window
+        # block k (1..n) is predicted from c_{k-w} .. c_{k-1} (zeros before
+        # block 0, R10)
+        c_pad = np.concatenate([np.zeros((B, w - 1, D), dtype=dt), c], axis=1)
         nrows = P + L - 1
         u = np.zeros((B, n, nrows, D), dtype=dt)
-        u[:, :, :P] = prefix
         for k in range(1, n + 1):
+            rows, add = self.context_input(c_pad[:, k - 1:k - 1 + w])
+            u[:, k - 1, :P] = rows
             for j in range(L - 1):
                 t = k * L + j
                 if t < S:
-                    u[:, k - 1, P + j] = self.g["tok_emb"][tokens[:, t]]
+                    u[:, k - 1, P + j] = self.token_rows(tokens[:, t:t + 1], np.array([j]), add)[:, 0]
         # rows whose input token is unknown (t >= S) only feed later rows of
         # the same block; their logits are never used.
         uu = u.reshape(B * n, nrows, D)
@@ -323,21 +368,30 @@ class OracleSession:
         self.block_caches: List[KVCache] = []
         self.token_caches: List[KVCache] = []
         self.cur_block: Optional[np.ndarray] = None   # [B, L_B] tokens of the open block
-        self.c_last: Optional[np.ndarray] = None
+        self.c_win: Optional[np.ndarray] = None       # [B, w, D] last w context embeddings
+        self.add: Optional[np.ndarray] = None         # summation injection: s_1..s_{L_B-1}
 
     def _token_rows(self, rows: np.ndarray, pos: np.ndarray) -> np.ndarray:
         return self.m.token_decoder(rows, pos, self.token_caches)
 
-    def _start_block(self, c: np.ndarray, trailing: Optional[np.ndarray] = None) -> np.ndarray:
-        """New token-decoder block: reset local KV, feed the P prefix rows and
-        the tokens of the block already known (``trailing`` [B, r], r < L_B,
-        at local positions P..P+r-1); return logits of the last row fed,
-        which predict token r of the block."""
-        s, m = self.s, self.m
+    def _push_context(self, c: np.ndarray) -> None:
+        """c [B, D] becomes the newest context embedding of the window."""
+        if self.c_win is None:
+            B, D = c.shape
+            self.c_win = np.zeros((B, self.m.window, D), dtype=self.m.dtype)
+        self.c_win = np.concatenate([self.c_win[:, 1:], c[:, None]], axis=1)
+
+    def _start_block(self, trailing: Optional[np.ndarray] = None) -> np.ndarray:
+        """New token-decoder block: reset local KV, feed the context rows of
+        the window and the tokens of the block already known (``trailing``
+        [B, r], r < L_B, at local positions n_ctx..n_ctx+r-1); return logits
+        of the last row fed, which predict token r of the block."""
+        m = self.m
         self.token_caches = m._fresh(m.token_layers)
-        rows = prefix_projection(c, m.g["w_prefix"], m.g["b_prefix"], s.prefix_len)
+        rows, self.add = m.context_input(self.c_win)
         if trailing is not None and trailing.shape[1] > 0:
-            rows = np.concatenate([rows, m.g["tok_emb"][trailing]], axis=1)
+            r = trailing.shape[1]
+            rows = np.concatenate([rows, m.token_rows(trailing, np.arange(r), self.add)], axis=1)
         z = self._token_rows(rows, np.arange(rows.shape[1]))
         return z[:, -1]
 
@@ -361,13 +415,17 @@ class OracleSession:
         r = T - n * L
         self.block_caches = m._fresh(m.block_layers)
         e = embed_blocks(tokens[:, :n * L], m.g["blk_emb"], L)
-        c = m.block_decoder(e, np.arange(n), self.block_caches)[:, -1]   # c_{n-1}
+        c_all = m.block_decoder(e, np.arange(n), self.block_caches)       # c_0 .. c_{n-1}
+        c = c_all[:, -1]
+        self.c_win = None
+        for i in range(max(0, n - m.window), n):
+            self._push_context(c_all[:, i])
         self.t = T
         self.cur_block = np.zeros((B, L), dtype=np.int64)
         self.cur_block[:, :r] = tokens[:, n * L:]
         if not s.use_token_decoder:
             return c @ m.g["w_lm"].T
-        return self._start_block(c, tokens[:, n * L:])
+        return self._start_block(tokens[:, n * L:])
 
     def decode(self, tok: np.ndarray) -> np.ndarray:
         """Feed token x_t (t = tokens seen so far); return logits for x_{t+1}.
@@ -375,7 +433,7 @@ class OracleSession:
         If x_t completes block k = t // L_B, the block decoder appends e_k to
         its cache (position k) and a new token-decoder block starts from c_k;
         otherwise the token decoder appends one row at local position
-        P + (t mod L_B)."""
+        n_ctx_rows + (t mod L_B)."""
         s, m = self.s, self.m
         tok = np.asarray(tok)
         L = s.block_len
@@ -389,9 +447,10 @@ class OracleSession:
             c = m.block_decoder(e, np.array([k]), self.block_caches)[:, 0]
             if not s.use_token_decoder:
                 return c @ m.g["w_lm"].T
-            return self._start_block(c)
-        row = m.g["tok_emb"][tok][:, None, :]
-        z = self._token_rows(row, np.array([s.prefix_len + j]))
+            self._push_context(c)
+            return self._start_block()
+        row = m.token_rows(tok[:, None], np.array([j]), self.add)
+        z = self._token_rows(row, np.array([m.n_ctx_rows + j]))
         return z[:, 0]
 
     def generate_logits(self, tokens: np.ndarray, prompt_len: int,

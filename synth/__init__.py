@@ -49,6 +49,17 @@ class ModelShape:
     dtype: str = "bf16"     # "fp32" or "bf16": storage/compute type of the path
     ln_eps: float = 1e-5
     rope_base: float = 10000.0
+    # how the context embedding reaches the token decoder: "prefix" (P
+    # projected rows in front of the block's tokens) or "sum" (L_B projected
+    # vectors added to the token decoder's input rows, MEGABYTE-style)
+    injection: str = "prefix"
+    context_window: int = 1  # w: the last w context embeddings feed the prefix
+
+    @property
+    def proj_rows(self) -> int:
+        """Rows of D outputs of the context projection: P, or L_B in "sum"
+        injection."""
+        return self.block_len if self.injection == "sum" else self.prefix_len
 
     @property
     def d_head(self) -> int:
@@ -137,7 +148,7 @@ def layer_param_shapes(s: ModelShape) -> List[Tuple[str, Tuple[int, ...]]]:
 
 
 def global_param_shapes(s: ModelShape) -> List[Tuple[str, Tuple[int, ...]]]:
-    D, V, P = s.d_model, s.vocab, s.prefix_len
+    D, V, P = s.d_model, s.vocab, s.proj_rows
     out = [("blk_emb", (V, D // s.block_len)),
            ("lnf_b_g", (D,)), ("lnf_b_b", (D,))]
     if s.use_token_decoder:

@@ -17,6 +17,7 @@ the same pins against a deliberately broken copy.
 """
 from __future__ import annotations
 
+import dataclasses
 import math
 
 import numpy as np
@@ -377,3 +378,91 @@ def pin_batch_rows_independent(om) -> bool:
     x[1] = (x[1] + 3) % shape.vocab
     pert = o.forward_full(x)
     return bool(np.allclose(base[[0, 2]], pert[[0, 2]], rtol=0, atol=1e-12, equal_nan=True))
+
+
+# --------------------------------------------------------------------------
+# context injection variants: summation (reading R9) and a window of previous
+# context embeddings (reading R10)
+# --------------------------------------------------------------------------
+
+SUM = dataclasses.replace(SMALL, injection="sum", prefix_len=1)
+WIN = dataclasses.replace(SMALL, context_window=3)
+
+
+def pin_sum_injection_reduces_to_prefix(om) -> float:
+    """Summation injection whose vectors s_1..s_{L_B-1} are zero (projection
+    rows and bias beyond the first D) is the prefix model with P = 1 whose
+    projection is the first D rows."""
+    D = SUM.d_model
+    ps = params_of(SUM)
+    ps["w_prefix"] = ps["w_prefix"].copy()
+    ps["b_prefix"] = ps["b_prefix"].copy()
+    ps["w_prefix"][D:] = 0.0
+    ps["b_prefix"][D:] = 0.0
+    pp = dict(ps)
+    pp["w_prefix"] = ps["w_prefix"][:D]
+    pp["b_prefix"] = ps["b_prefix"][:D]
+    toks = tokens_of(SUM, S=22)
+    a = om.BlockTransformerOracle(SUM, ps).forward_full(toks)
+    b = om.BlockTransformerOracle(dataclasses.replace(SUM, injection="prefix"), pp).forward_full(toks)
+    return float(np.nanmax(np.abs(a - b)))
+
+
+def pin_sum_injection_slot_reach(om) -> bool:
+    """s_j is added to the input of in-block row j (row 0 holds s_0 alone):
+    under the causal token decoder, changing slot j of the projection's
+    bias changes exactly the predictions of in-block offsets j..L_B-1 of
+    every block, and none before."""
+    L, D = SUM.block_len, SUM.d_model
+    ps = params_of(SUM)
+    toks = tokens_of(SUM, S=20)
+    base = om.BlockTransformerOracle(SUM, ps).forward_full(toks)
+    ok = True
+    for j in range(L):
+        q = dict(ps)
+        q["b_prefix"] = ps["b_prefix"].copy()
+        q["b_prefix"][j * D:(j + 1) * D] += 0.5
+        got = om.BlockTransformerOracle(SUM, q).forward_full(toks)
+        for k in range(1, toks.shape[1] // L + 1):
+            for jj in range(L):
+                t = k * L + jj
+                if t > toks.shape[1]:
+                    continue
+                changed = bool(np.any(np.abs(got[:, t] - base[:, t]) > 1e-9))
+                ok &= changed == (jj >= j)
+    return ok
+
+
+def pin_window_assembly_bruteforce(om) -> float:
+    """The token decoder of block k sees the projections of c_{k-w} ..
+    c_{k-1}, oldest first, zero vectors before block 0, then the block's
+    tokens: rebuild that input by hand from the block decoder's outputs
+    (projection written out as a loop over the P output rows) and compare
+    with the full pass."""
+    w, P, L, D = WIN.context_window, WIN.prefix_len, WIN.block_len, WIN.d_model
+    ps = params_of(WIN)
+    toks = tokens_of(WIN, S=21)
+    o = om.BlockTransformerOracle(WIN, ps)
+    full = o.forward_full(toks)
+    B, S = toks.shape
+    n = S // L
+    e = om.embed_blocks(toks, o.g["blk_emb"], L)
+    c = o.block_decoder(e, np.arange(n), o._fresh(o.block_layers))
+    W, bias = o.g["w_prefix"], o.g["b_prefix"]
+    worst = 0.0
+    for k in range(1, n + 1):
+        rows = []
+        for i in range(k - w, k):
+            ci = c[:, i] if i >= 0 else np.zeros((B, D))
+            for r in range(P):
+                rows.append(ci @ W[r * D:(r + 1) * D].T + bias[r * D:(r + 1) * D])
+        for j in range(L - 1):
+            t = k * L + j
+            rows.append(o.g["tok_emb"][toks[:, min(t, S - 1)]])
+        u = np.stack(rows, axis=1)
+        z = o.token_decoder(u, np.arange(u.shape[1]), o._fresh(o.token_layers))
+        for j in range(L):
+            t = k * L + j  # predicted from the tokens before it: defined for t <= S
+            if t <= S:
+                worst = max(worst, float(np.abs(z[:, w * P - 1 + j] - full[:, t]).max()))
+    return worst

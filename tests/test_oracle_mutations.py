@@ -35,6 +35,11 @@ def _first_failing_pin(mod):
         ("incremental_partial", lambda: pins.pin_incremental_equals_full(mod, T=10, G=7) < TOL),
         ("hf_vanilla", lambda: pins.pin_vanilla_vs_hf(mod) < TOL),
         ("hf_block_model", lambda: pins.pin_block_model_vs_hf(mod) < TOL),
+        ("sum_reduces_to_prefix", lambda: pins.pin_sum_injection_reduces_to_prefix(mod) < TOL),
+        ("sum_slot_reach", lambda: pins.pin_sum_injection_slot_reach(mod)),
+        ("window_assembly", lambda: pins.pin_window_assembly_bruteforce(mod) < TOL),
+        ("incremental_sum", lambda: pins.pin_incremental_equals_full(mod, shape=pins.SUM, T=6, G=9) < TOL),
+        ("incremental_window", lambda: pins.pin_incremental_equals_full(mod, shape=pins.WIN, T=6, G=9) < TOL),
     ]
     for name, c in checks:
         if not c():
@@ -105,20 +110,22 @@ def _layer_serial_residual(h, p, pos, cache, H, r, eps, base):
 _ORIG_START = om.OracleSession._start_block
 
 
-def _start_block_trailing_shifted(self, c, trailing=None):
+def _start_block_trailing_shifted(self, trailing=None):
     # trailing prompt tokens one local position too far
     if trailing is None or trailing.shape[1] == 0:
-        return _ORIG_START(self, c, trailing)
-    s, m = self.s, self.m
+        return _ORIG_START(self, trailing)
+    m = self.m
     self.token_caches = m._fresh(m.token_layers)
-    pre = ORIG["prefix_projection"](c, m.g["w_prefix"], m.g["b_prefix"], s.prefix_len)
-    rows = np.concatenate([pre, m.g["tok_emb"][trailing]], axis=1)
-    pos = np.concatenate([np.arange(s.prefix_len), s.prefix_len + 1 + np.arange(trailing.shape[1])])
+    pre, add = m.context_input(self.c_win)
+    self.add = add
+    rows = np.concatenate([pre, m.token_rows(trailing, np.arange(trailing.shape[1]), add)], axis=1)
+    P = pre.shape[1]
+    pos = np.concatenate([np.arange(P), P + 1 + np.arange(trailing.shape[1])])
     return self._token_rows(rows, pos)[:, -1]
 
 
-def _start_block_trailing_dropped(self, c, trailing=None):
-    return _ORIG_START(self, c, None)
+def _start_block_trailing_dropped(self, trailing=None):
+    return _ORIG_START(self, None)
 
 
 SESSION_MUTATIONS = {
@@ -139,6 +146,60 @@ MUTATIONS = {
     "drop_b_o": ("pythia_layer", _layer_drop_bias_o),
     "serial_residual": ("pythia_layer", _layer_serial_residual),
 }
+
+
+# context injection variants (readings R9, R10): planted on the model class
+_ORIG_CTX = om.BlockTransformerOracle.context_input
+_ORIG_ROWS = om.BlockTransformerOracle.token_rows
+
+
+def _ctx_window_newest_first(self, c_win):
+    return _ORIG_CTX(self, c_win[:, ::-1])
+
+
+def _ctx_window_clamped(self, c_win):
+    # history before block 0 repeats the oldest known embedding instead of zeros
+    c = c_win.copy()
+    nz = np.abs(c).sum(axis=-1) > 0
+    for b in range(c.shape[0]):
+        idx = np.flatnonzero(nz[b])
+        if idx.size:
+            c[b, :idx[0]] = c[b, idx[0]]
+    return _ORIG_CTX(self, c)
+
+
+def _ctx_sum_slots_shifted(self, c_win):
+    rows, add = _ORIG_CTX(self, c_win)
+    if add is None:
+        return rows, add
+    # s_j added one row early: token rows get s_{j+2}, the last gets s_1
+    return rows, np.roll(add, -1, axis=1)
+
+
+def _rows_sum_own_slot(self, tok, j, add):
+    # token j of the block gets s_j instead of s_{j+1}
+    rows = self.g["tok_emb"][tok]
+    if add is not None:
+        full = np.concatenate([np.zeros_like(add[:, :1]), add], axis=1)
+        rows = rows + full[:, j]
+    return rows
+
+
+MODEL_MUTATIONS = {
+    "window_newest_first": ("context_input", _ctx_window_newest_first),
+    "window_clamped_history": ("context_input", _ctx_window_clamped),
+    "sum_slots_shifted": ("context_input", _ctx_sum_slots_shifted),
+    "sum_own_slot": ("token_rows", _rows_sum_own_slot),
+}
+
+
+@pytest.mark.parametrize("mutation", sorted(MODEL_MUTATIONS))
+def test_planted_injection_mistake_is_caught(mutation, monkeypatch):
+    name, fn = MODEL_MUTATIONS[mutation]
+    monkeypatch.setattr(om.BlockTransformerOracle, name, fn)
+    caught_by = _first_failing_pin(om)
+    print(f"{mutation}: caught by {caught_by}")
+    assert caught_by is not None, f"no pin caught the planted mistake {mutation}"
 
 
 def test_unmutated_oracle_passes_every_pin():

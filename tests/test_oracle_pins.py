@@ -97,3 +97,25 @@ def test_literal_locality_without_block_layers():
 
 def test_batch_rows_are_independent():
     assert pins.pin_batch_rows_independent(om)
+
+
+# ---- context injection variants (readings R9, R10) ------------------------
+
+def test_sum_injection_reduces_to_prefix_model():
+    assert pins.pin_sum_injection_reduces_to_prefix(om) < 1e-10
+
+
+def test_sum_injection_slot_j_reaches_rows_from_j():
+    assert pins.pin_sum_injection_slot_reach(om)
+
+
+def test_window_of_context_embeddings_matches_hand_assembly():
+    assert pins.pin_window_assembly_bruteforce(om) < 1e-10
+
+
+@pytest.mark.parametrize("shape_name", ["SUM", "WIN"])
+@pytest.mark.parametrize("T", [4, 6, 8, 13])
+def test_injection_variants_incremental_equals_full(shape_name, T):
+    """Invariant 1 for both variants, prompts shorter than the window (T = 4:
+    one block, two zero context slots) and ending inside a block."""
+    assert pins.pin_incremental_equals_full(om, shape=getattr(pins, shape_name), T=T, G=11) < 1e-10
