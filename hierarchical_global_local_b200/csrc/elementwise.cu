@@ -63,7 +63,8 @@ template <typename T>
 __global__ void embed_tail_kernel(const int32_t* __restrict__ tokens, int T_len, int col0, int r,
                                   int rows_per_seq, int row_off, const T* __restrict__ tok_emb, int V,
                                   int D, float* __restrict__ h, int32_t* __restrict__ block_tok, int L_B,
-                                  int* status, const int* __restrict__ row_col0) {
+                                  int* status, const int* __restrict__ row_col0,
+                                  const float* __restrict__ add) {
   pdl_trigger();
   pdl_wait();
   const int b = blockIdx.x / r, i = blockIdx.x % r;
@@ -75,7 +76,10 @@ __global__ void embed_tail_kernel(const int32_t* __restrict__ tokens, int T_len,
   }
   if (threadIdx.x == 0) block_tok[b * L_B + i] = tok;
   float* row = h + ((size_t)b * rows_per_seq + row_off + i) * D;
-  for (int x = threadIdx.x; x < D; x += blockDim.x) row[x] = to_f(tok_emb[(size_t)tok * D + x]);
+  // summation injection: token i of the block also receives s_{i+1}
+  const float* ad = add ? add + ((size_t)b * (L_B - 1) + i) * D : nullptr;
+  for (int x = threadIdx.x; x < D; x += blockDim.x)
+    row[x] = to_f(tok_emb[(size_t)tok * D + x]) + (ad ? ad[x] : 0.f);
 }
 
 template <typename T>
@@ -83,7 +87,7 @@ __global__ void ingest_kernel(const int32_t* __restrict__ src, int32_t* __restri
                               const int* __restrict__ dstate, int L_B, int V, int D,
                               int block_step, const T* __restrict__ blk_emb,
                               const T* __restrict__ tok_emb, float* __restrict__ h,
-                              int* status) {
+                              int* status, const float* __restrict__ add) {
   pdl_trigger();
   pdl_wait();
   const int b = blockIdx.x;
@@ -95,8 +99,10 @@ __global__ void ingest_kernel(const int32_t* __restrict__ src, int32_t* __restri
   }
   if (threadIdx.x == 0) block_tok[b * L_B + j] = tok;
   if (!block_step) {
+    // summation injection: token j of the block also receives s_{j+1}
+    const float* ad = add ? add + ((size_t)b * (L_B - 1) + j) * D : nullptr;
     for (int x = threadIdx.x; x < D; x += blockDim.x)
-      h[(size_t)b * D + x] = to_f(tok_emb[(size_t)tok * D + x]);
+      h[(size_t)b * D + x] = to_f(tok_emb[(size_t)tok * D + x]) + (ad ? ad[x] : 0.f);
   } else {
     const int De = D / L_B;
     for (int x = threadIdx.x; x < D; x += blockDim.x) {
@@ -216,30 +222,70 @@ cudaError_t launch_embed_prompt(int dt, const int32_t* tokens, int B, int T, int
 cudaError_t launch_embed_tail(int dt, const int32_t* tokens, int B, int T_len, int col0, int r,
                               int rows_per_seq, int row_off, const void* tok_emb, int V, int D, float* h,
                               int32_t* block_tok, int L_B, int* status, cudaStream_t s,
-                              const int* row_col0) {
+                              const int* row_col0, const float* add) {
   if (B * r == 0) return cudaSuccess;
   if (dt == DT_BF16) {
     BT_LAUNCH(embed_tail_kernel<bf16>, dim3(B * r), dim3(256), 0, s, tokens, T_len, col0, r, rows_per_seq,
-              row_off, (const bf16*)tok_emb, V, D, h, block_tok, L_B, status, row_col0);
+              row_off, (const bf16*)tok_emb, V, D, h, block_tok, L_B, status, row_col0, add);
   } else {
     BT_LAUNCH(embed_tail_kernel<float>, dim3(B * r), dim3(256), 0, s, tokens, T_len, col0, r, rows_per_seq,
-              row_off, (const float*)tok_emb, V, D, h, block_tok, L_B, status, row_col0);
+              row_off, (const float*)tok_emb, V, D, h, block_tok, L_B, status, row_col0, add);
   }
   return cudaGetLastError();
 }
 
 cudaError_t launch_ingest(int dt, const int32_t* src, int32_t* block_tok, const int* dstate,
                           int B, int L_B, int V, int D, int block_step, const void* blk_emb,
-                          const void* tok_emb, float* h, int* status, cudaStream_t s) {
+                          const void* tok_emb, float* h, int* status, cudaStream_t s, const float* add) {
   if (dt == DT_BF16) {
     BT_LAUNCH(ingest_kernel<bf16>, dim3(B), dim3(256), 0, s, src, block_tok, dstate, L_B, V, D, block_step,
-                                          (const bf16*)blk_emb, (const bf16*)tok_emb, h, status);
+                                          (const bf16*)blk_emb, (const bf16*)tok_emb, h, status, add);
   }
   else {
     BT_LAUNCH(ingest_kernel<float>, dim3(B), dim3(256), 0, s, src, block_tok, dstate, L_B, V, D, block_step,
                                            (const float*)blk_emb, (const float*)tok_emb, h,
-                                           status);
+                                           status, add);
   }
+  return cudaGetLastError();
+}
+
+// Context rows of the token decoder for the context-injection variants; one
+// CTA per (sequence, row), threads over the D features.
+//   CTX_WINDOW_SHIFT: h[b * h_rows + r] = r < (w-1)P ? ring[b][r + P]
+//                     : proj[b][r - (w-1)P], r < wP (the window moves on by
+//                     one context embedding, the newest projection last)
+//   CTX_WINDOW_SAVE:  ring[b][r] = h[b * h_rows + r], r < wP
+//   CTX_SUM_SPLIT:    h[b * h_rows] = proj[b][0] (s_0); add[b][j] =
+//                     proj[b][j + 1] (s_{j+1}), j < L_B - 1
+// ring [B, wP, D], proj [B, rows, D] (rows = P, or L_B for the split), fp32.
+__global__ void ctx_rows_kernel(int mode, const float* __restrict__ proj, float* __restrict__ ring,
+                                float* __restrict__ h, float* __restrict__ add, int nrows, int w, int P,
+                                int L_B, int D, int h_rows) {
+  pdl_trigger();
+  pdl_wait();
+  const int b = blockIdx.x / nrows, r = blockIdx.x % nrows;
+  const float* src;
+  float* dst;
+  if (mode == CTX_WINDOW_SHIFT) {
+    const int old = (w - 1) * P;
+    src = r < old ? ring + ((size_t)b * w * P + r + P) * D : proj + ((size_t)b * P + r - old) * D;
+    dst = h + ((size_t)b * h_rows + r) * D;
+  } else if (mode == CTX_WINDOW_SAVE) {
+    src = h + ((size_t)b * h_rows + r) * D;
+    dst = ring + ((size_t)b * w * P + r) * D;
+  } else {
+    src = proj + ((size_t)b * L_B + r) * D;
+    dst = r == 0 ? h + (size_t)b * h_rows * D : add + ((size_t)b * (L_B - 1) + r - 1) * D;
+  }
+  for (int x = threadIdx.x; x < D; x += blockDim.x) dst[x] = src[x];
+}
+
+cudaError_t launch_ctx_rows(int mode, const float* proj, float* ring, float* h, float* add, int B, int w,
+                            int P, int L_B, int D, int h_rows, cudaStream_t s) {
+  const int nrows = mode == CTX_SUM_SPLIT ? L_B : w * P;
+  if (B * nrows == 0) return cudaSuccess;
+  BT_LAUNCH(ctx_rows_kernel, dim3(B * nrows), dim3(256), 0, s, mode, proj, ring, h, add, nrows, w, P, L_B, D,
+            h_rows);
   return cudaGetLastError();
 }
 

@@ -36,19 +36,35 @@ cudaError_t launch_embed_prompt(int dt, const int32_t* tokens, int B, int T, int
                                 const int* row_len = nullptr, int pad_id = 0);
 // Trailing prompt tokens of a prompt that ends inside a block: for b < B,
 // i < r, token tokens[b * T_len + col0 + i] is recorded in block_tok[b, i]
-// and its token-decoder embedding tok_emb[token] is written to row
-// b * rows_per_seq + row_off + i of h [.., D] (fp32).
+// and its token-decoder embedding tok_emb[token] (+ add[b, i] when add is
+// not null: summation injection's s_{i+1}, add [B, L_B - 1, D] fp32) is
+// written to row b * rows_per_seq + row_off + i of h [.., D] (fp32).
 cudaError_t launch_embed_tail(int dt, const int32_t* tokens, int B, int T_len, int col0, int r,
                               int rows_per_seq, int row_off, const void* tok_emb, int V, int D, float* h,
                               int32_t* block_tok, int L_B, int* status, cudaStream_t s,
-                              const int* row_col0 = nullptr);  // per-sequence col0 (ragged)
+                              const int* row_col0 = nullptr,  // per-sequence col0 (ragged)
+                              const float* add = nullptr);
 // Decode ingest of the fed token src[b] at position t = dstate[0]:
 // records it in block_tok[b, t % L_B]; block_step = 0 gathers
-// h[b] = tok_emb[src[b]]; block_step = 1 (the token completes its block)
-// gathers h[b] = concat_j blk_emb[block_tok[b, j]].
+// h[b] = tok_emb[src[b]] (+ add[b, t % L_B] when add is not null:
+// summation injection's s_{j+1} for token j of the block); block_step = 1
+// (the token completes its block) gathers h[b] = concat_j blk_emb[block_tok[b, j]].
 cudaError_t launch_ingest(int dt, const int32_t* src, int32_t* block_tok, const int* dstate,
                           int B, int L_B, int V, int D, int block_step, const void* blk_emb,
-                          const void* tok_emb, float* h, int* status, cudaStream_t s);
+                          const void* tok_emb, float* h, int* status, cudaStream_t s,
+                          const float* add = nullptr);
+// Context rows of the token decoder for the context-injection variants
+// (one CTA per sequence and row, fp32):
+//   CTX_WINDOW_SHIFT  h[b * h_rows + r] = ring[b][r + P] for r < (w-1)P,
+//                     proj[b][r - (w-1)P] after: the window of the last w
+//                     projected context embeddings, oldest first
+//   CTX_WINDOW_SAVE   ring[b][r] = h[b * h_rows + r], r < wP
+//   CTX_SUM_SPLIT     h[b * h_rows] = proj[b][0]; add[b][j] = proj[b][j + 1]
+// ring [B, wP, D]; proj [B, P, D] (window) or [B, L_B, D] (summation);
+// add [B, L_B - 1, D].
+enum CtxMode { CTX_WINDOW_SHIFT = 0, CTX_WINDOW_SAVE = 1, CTX_SUM_SPLIT = 2 };
+cudaError_t launch_ctx_rows(int mode, const float* proj, float* ring, float* h, float* add, int B, int w,
+                            int P, int L_B, int D, int h_rows, cudaStream_t s);
 // Ingest plus the first LayerNorm(s) of the gathered row (bf16): g2 != null ->
 // x[b] = [LN1 | LN2] ([B, 2D]); else x[b] = LN(h[b]) ([B, D]).
 cudaError_t launch_ingest_ln(const int32_t* src, int32_t* block_tok, const int* dstate, int B,

@@ -67,6 +67,11 @@ struct Carver {
 
 struct Dims {
   int V, D, H, d, L, Nb, Nt, P, rot, Bmax, max_seq, dt, tokdec;
+  // context injection: inj 0 = prefix, 1 = summation; w = window of context
+  // embeddings; Pp = rows per projected context embedding (prefix_len);
+  // prows = output rows of the context projection (Pp, or L_B in
+  // summation). P above = the token decoder's context rows (w * Pp, or 1).
+  int inj, w, Pp, prows;
   size_t eb;
   int n_cap;   // block-cache entries per sequence
   int l_cap;   // local-cache rows per sequence
@@ -96,6 +101,13 @@ int dims_of(const bt_config* c, Dims* o) {
   } else if (d.L != 1) {
     return BT_EINVAL;  // vanilla mode is the L_B = 1 special case
   }
+  d.inj = d.tokdec ? c->context_injection : 0;
+  d.w = (d.tokdec && c->context_window > 0) ? c->context_window : 1;
+  if (d.inj != 0 && d.inj != 1) return BT_EINVAL;
+  if (d.inj == 1 && (d.P != 1 || d.w != 1)) return BT_EINVAL;
+  d.Pp = d.P;
+  d.prows = d.inj ? d.L : d.Pp;
+  if (d.tokdec && !d.inj) d.P = d.w * d.Pp;
   if (!(c->ln_eps > 0.f) || !(c->rope_base > 0.f)) return BT_EINVAL;
   d.eb = dt_size(d.dt);
   d.n_cap = (d.max_seq + d.L - 1) / d.L;
@@ -160,6 +172,9 @@ struct bt_model {
   unsigned* ts2_ctr = nullptr;               // token_step2: counters
   size_t ts2_ctr_bytes = 0;
   float2* ts_hstat = nullptr;                // token_step2: per-(row, tile) statistics of h
+  float* ctx_proj = nullptr;                 // context projection output [B, prows, D]
+  float* ctx_ring = nullptr;                 // window of projected context rows [B, w*Pp, D]
+  float* sum_add = nullptr;                  // summation vectors s_1.. [B, L_B - 1, D]
   bf16* ts_hb = nullptr;                     // token_step2: bf16 copy of h
   void* l2_base = nullptr;                   // L2 persisting window of the fused token step
   size_t l2_window = 0;                      //   bytes (0: none)
@@ -239,8 +254,8 @@ static size_t carve(bt_model* m, const Dims& d, void* ws) {
   m->lnf_b_g = (float*)c.take(D * 4); m->lnf_b_b = (float*)c.take(D * 4);
   if (d.tokdec) {
     m->tok_emb = c.take((size_t)d.V * D * eb);
-    m->w_prefix = c.take((size_t)d.P * D * D * eb);
-    m->b_prefix = (float*)c.take((size_t)d.P * D * 4);
+    m->w_prefix = c.take((size_t)d.prows * D * D * eb);
+    m->b_prefix = (float*)c.take((size_t)d.prows * D * 4);
     m->lnf_t_g = (float*)c.take(D * 4); m->lnf_t_b = (float*)c.take(D * 4);
   }
   // the LM head and the token decoder's local caches are adjacent: one L2
@@ -267,6 +282,13 @@ static size_t carve(bt_model* m, const Dims& d, void* ws) {
   m->fed = (int32_t*)c.take((size_t)d.Bmax * 4);
   m->block_tok = (int32_t*)c.take((size_t)d.Bmax * d.L * 4);
   m->row_lag = (int*)c.take((size_t)d.Bmax * 4 * sizeof(int));
+  if (d.tokdec && (d.inj || d.w > 1)) {
+    // context-injection variants: projection output, window ring, the
+    // summation vectors of the token rows
+    m->ctx_proj = (float*)c.take((size_t)d.Bmax * d.prows * D * 4);
+    if (d.w > 1) m->ctx_ring = (float*)c.take((size_t)d.Bmax * d.w * d.Pp * D * 4);
+    if (d.inj) m->sum_add = (float*)c.take((size_t)d.Bmax * (d.L > 1 ? d.L - 1 : 1) * D * 4);
+  }
   m->row_pad = m->row_lag ? m->row_lag + d.Bmax : nullptr;
   m->row_len = m->row_lag ? m->row_lag + 2 * d.Bmax : nullptr;
   m->row_col0 = m->row_lag ? m->row_lag + 3 * d.Bmax : nullptr;
@@ -391,9 +413,9 @@ int bt_create(const bt_config* cfg, const bt_weights* w, void* ws, size_t ws_byt
   if (d.tokdec) {
     BT_TRYC(cudaMemcpyAsync(m->tok_emb, w->tok_emb_dev, (size_t)d.V * D * eb,
                             cudaMemcpyDeviceToDevice, st));
-    BT_TRYC(cudaMemcpyAsync(m->w_prefix, w->w_prefix_dev, (size_t)d.P * D * D * eb,
+    BT_TRYC(cudaMemcpyAsync(m->w_prefix, w->w_prefix_dev, (size_t)d.prows * D * D * eb,
                             cudaMemcpyDeviceToDevice, st));
-    BT_TRYC(launch_convert_to_f32(d.dt, w->b_prefix_dev, m->b_prefix, (size_t)d.P * D, st));
+    BT_TRYC(launch_convert_to_f32(d.dt, w->b_prefix_dev, m->b_prefix, (size_t)d.prows * D, st));
     BT_TRYC(launch_convert_to_f32(d.dt, w->lnf_t_g_dev, m->lnf_t_g, D, st));
     BT_TRYC(launch_convert_to_f32(d.dt, w->lnf_t_b_dev, m->lnf_t_b, D, st));
   }
@@ -491,7 +513,7 @@ static bool fused_decode(const bt_model* m, int B) {
   const char* env = getenv("BT_DECODE_LN");
   if (!env || strcmp(env, "fused") != 0) return false;
   return d.dt == BT_BF16 && B <= 256 && d.D <= 2048 && (d.D % 128) == 0 &&
-         gemm_tc_supported(d.dt, B, d.D, 5 * d.D, 1 << 30, 0) && (!d.tokdec || d.P == 1);
+         gemm_tc_supported(d.dt, B, d.D, 5 * d.D, 1 << 30, 0) && (!d.tokdec || (d.P == 1 && !d.inj));
 }
 
 static int run_layer(bt_model* m, const LayerW& w, float* h, int M, PosSpec pos, void* kc,
@@ -580,7 +602,8 @@ struct Tail {
 // prefix projection and the token decoder over P rows (plus the trailing
 // prompt tokens of `tail`), or (vanilla) xf.
 static int run_context_to_head_input(bt_model* m, int B, int row_step, int row_off, cudaStream_t s,
-                                     const Tail& tail = Tail(), const int* row_lag = nullptr) {
+                                     const Tail& tail = Tail(), const int* row_lag = nullptr,
+                                     bool block_call = false) {
   const Dims& d = m->d;
   {
     ProfScope p(m, s, BT_K_LAYERNORM, B, d.D, 0);
@@ -589,17 +612,64 @@ static int run_context_to_head_input(bt_model* m, int B, int row_step, int row_o
   }
   if (!d.tokdec) return BT_OK;
   const int rows = d.P + tail.r;  // token-decoder rows per sequence
-  {
+  if (!d.inj && d.w == 1) {
     // prefix rows: h_t[b*rows + p, :] = (W_p c_b + b_p)[p*D:(p+1)*D]
     ProfScope p(m, s, BT_K_GEMM, B, d.P * d.D, d.D);
     Epi ep{EPI_F32, m->h_t, rows * d.D, nullptr, 0, m->b_prefix, 0, d.D};
     BT_CUDA(launch_gemm(d.dt, m->xf, d.D, m->w_prefix, d.D, B, d.P * d.D, d.D, 1 << 30, 0, ep, m->gs,
                         m->status, s));
+  } else if (d.inj) {
+    // summation: s = W_p c + b_p -> [B, L_B, D]; s_0 is the context row,
+    // s_1.. wait for the block's token rows
+    {
+      ProfScope p(m, s, BT_K_GEMM, B, d.prows * d.D, d.D);
+      Epi ep{EPI_F32, m->ctx_proj, d.prows * d.D, nullptr, 0, m->b_prefix, 0, d.D};
+      BT_CUDA(launch_gemm(d.dt, m->xf, d.D, m->w_prefix, d.D, B, d.prows * d.D, d.D, 1 << 30, 0, ep, m->gs,
+                          m->status, s));
+    }
+    ProfScope p(m, s, BT_K_OTHER, B, d.L, d.D);
+    BT_CUDA(launch_ctx_rows(CTX_SUM_SPLIT, m->ctx_proj, nullptr, m->h_t, m->sum_add, B, 1, 1, d.L, d.D, rows, s));
+  } else if (block_call) {
+    // window, block step: project the new context embedding, move the
+    // window on by one (oldest first) and keep it for the next block
+    {
+      ProfScope p(m, s, BT_K_GEMM, B, d.Pp * d.D, d.D);
+      Epi ep{EPI_F32, m->ctx_proj, d.Pp * d.D, nullptr, 0, m->b_prefix, 0, d.D};
+      BT_CUDA(launch_gemm(d.dt, m->xf, d.D, m->w_prefix, d.D, B, d.Pp * d.D, d.D, 1 << 30, 0, ep, m->gs,
+                          m->status, s));
+    }
+    ProfScope p(m, s, BT_K_OTHER, B, d.P, d.D);
+    BT_CUDA(launch_ctx_rows(CTX_WINDOW_SHIFT, m->ctx_proj, m->ctx_ring, m->h_t, nullptr, B, d.w, d.Pp, d.L, d.D,
+                            rows, s));
+    BT_CUDA(launch_ctx_rows(CTX_WINDOW_SAVE, nullptr, m->ctx_ring, m->h_t, nullptr, B, d.w, d.Pp, d.L, d.D, rows,
+                            s));
+  } else {
+    // window, prefill: the last w context embeddings of every sequence,
+    // oldest first, each projected into its Pp rows; zero vectors before the
+    // first block (their rows are b_p)
+    for (int q = 0; q < d.w; ++q) {
+      const int o = row_off - (d.w - 1 - q);
+      if (o >= 0) {
+        ProfScope p(m, s, BT_K_LAYERNORM, B, d.D, 0);
+        BT_CUDA(launch_ln_rows(d.dt, m->h_b, B, row_step, o, d.D, m->lnf_b_g, m->lnf_b_b, m->cfg.ln_eps, m->xf, s,
+                               row_lag));
+      } else {
+        BT_CUDA(cudaMemsetAsync(m->xf, 0, (size_t)B * d.D * d.eb, s));
+      }
+      ProfScope p(m, s, BT_K_GEMM, B, d.Pp * d.D, d.D);
+      Epi ep{EPI_F32, m->h_t + (size_t)q * d.Pp * d.D, rows * d.D, nullptr, 0, m->b_prefix, 0, d.D};
+      BT_CUDA(launch_gemm(d.dt, m->xf, d.D, m->w_prefix, d.D, B, d.Pp * d.D, d.D, 1 << 30, 0, ep, m->gs,
+                          m->status, s));
+    }
+    ProfScope p(m, s, BT_K_OTHER, B, d.P, d.D);
+    BT_CUDA(launch_ctx_rows(CTX_WINDOW_SAVE, nullptr, m->ctx_ring, m->h_t, nullptr, B, d.w, d.Pp, d.L, d.D, rows,
+                            s));
   }
   if (tail.r > 0) {
     ProfScope p(m, s, BT_K_EMBED, B * tail.r, d.D, 0);
     BT_CUDA(launch_embed_tail(d.dt, tail.tokens, B, tail.T_len, tail.col0, tail.r, rows, d.P, m->tok_emb, d.V,
-                              d.D, m->h_t, m->block_tok, d.L, m->status, s, tail.row_col0));
+                              d.D, m->h_t, m->block_tok, d.L, m->status, s, tail.row_col0,
+                              d.inj ? m->sum_add : nullptr));
   }
   PosSpec pos{nullptr, POS_ZERO, 0, rows};
   return run_token_decoder(m, B, pos, s);
@@ -748,6 +818,7 @@ static int token_step_kind(const bt_model* m, int B) {
   const char* env = getenv("BT_DECODE_TOKEN_STEP");
   if (env && strcmp(env, "chain") == 0) return 0;
   if (!d.tokdec || d.Nt < 1 || !m->ts_bar) return 0;
+  if (d.inj || d.w > 1) return 0;  // context-injection variants: kernel chain
   const long long ls = d.Nt > 1 ? (long long)((uint8_t*)m->tok[1].w_qkv1 - (uint8_t*)m->tok[0].w_qkv1) : 0;
   if (!uniform_layers(m->tok, ls)) return 0;
   const bool only1 = env && strcmp(env, "v1") == 0, only2 = env && strcmp(env, "v2") == 0;
@@ -772,7 +843,7 @@ static bool block_step_fused(const bt_model* m, int B) {
   const char* env = getenv("BT_DECODE_BLOCK_STEP");
   if (!env || strcmp(env, "fused") != 0) return false;
   // its attention phase assumes one cache length for the whole batch
-  if (!m->ts_att || d.Nb < 1 || d.P != 1 || m->ragged) return false;
+  if (!m->ts_att || d.Nb < 1 || d.P != 1 || d.inj || m->ragged) return false;
   if (!token_step_block_supported(d.dt, B, d.D, d.H, d.rot, d.V, d.Nt, d.Nb, d.P, d.l_cap, d.n_cap, d.L))
     return false;
   const long long ls = d.Nt > 1 ? (long long)((uint8_t*)m->tok[1].w_qkv1 - (uint8_t*)m->tok[0].w_qkv1) : 0;
@@ -892,7 +963,8 @@ static int enqueue_decode(bt_model* m, bool block_step, bool greedy, bool want_l
   {
     ProfScope p(m, s, BT_K_EMBED, B, d.D, 0);
     BT_CUDA(launch_ingest(d.dt, src, m->block_tok, m->dstate, B, d.L, d.V, d.D, block_step ? 1 : 0,
-                          m->blk_emb, m->tok_emb, block_step ? m->h_b : m->h_t, m->status, s));
+                          m->blk_emb, m->tok_emb, block_step ? m->h_b : m->h_t, m->status, s,
+                          d.inj ? m->sum_add : nullptr));
   }
   int rc;
   if (block_step) {
@@ -902,7 +974,7 @@ static int enqueue_decode(bt_model* m, bool block_step, bool greedy, bool want_l
                      layer_ptr(m->vb, m->kb_layer, l, d.eb), d.n_cap, ATT_DECODE, 0, s);
       if (rc != BT_OK) return rc;
     }
-    rc = run_context_to_head_input(m, B, 1, 0, s);
+    rc = run_context_to_head_input(m, B, 1, 0, s, Tail(), nullptr, true);
     if (rc != BT_OK) return rc;
   } else {
     PosSpec pos{m->dstate, POS_LOCAL, d.P, 1};
@@ -1025,6 +1097,7 @@ int bt_prefill(bt_model* m, const int32_t* tokens, int32_t B, int32_t T, float* 
 int bt_prefill_ragged(bt_model* m, const int32_t* tokens, int32_t row_stride, const int32_t* lengths,
                       int32_t B, int32_t pad_id, float* logits, int32_t* next) {
   if (!m || !tokens || !lengths || row_stride < 1) return BT_EINVAL;
+  if (m->d.w > 1) return BT_ENOTSUP;  // the window's missing slots would differ per sequence
   return prefill_impl(m, tokens, row_stride, B, lengths, pad_id, logits, next);
 }
 

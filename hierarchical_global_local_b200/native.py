@@ -36,7 +36,8 @@ class BtConfig(ctypes.Structure):
     _fields_ = [(n, c_int32) for n in (
         "vocab", "d_model", "n_heads", "block_len", "n_block_layers", "n_token_layers",
         "prefix_len", "rotary_dims", "use_token_decoder", "max_batch", "max_seq", "dtype")] + \
-        [("ln_eps", c_float), ("rope_base", c_float)]
+        [("ln_eps", c_float), ("rope_base", c_float),
+         ("context_injection", c_int32), ("context_window", c_int32)]
 
 
 LAYER_FIELDS = ("ln1_g", "ln1_b", "ln2_g", "ln2_b", "w_qkv", "b_qkv", "w_o", "b_o",
@@ -167,13 +168,16 @@ class ModelConfig:
     dtype: str = "bf16"       # "bf16" | "fp32"
     ln_eps: float = 1e-5
     rope_base: float = 10000.0
+    injection: str = "prefix"  # "prefix" | "sum"
+    context_window: int = 1
 
     def c(self) -> BtConfig:
         return BtConfig(self.vocab, self.d_model, self.n_heads, self.block_len,
                         self.n_block_layers, self.n_token_layers, self.prefix_len,
                         self.rotary_dims, 1 if self.use_token_decoder else 0, self.max_batch,
                         self.max_seq, BT_BF16 if self.dtype == "bf16" else BT_FP32,
-                        self.ln_eps, self.rope_base)
+                        self.ln_eps, self.rope_base, 1 if self.injection == "sum" else 0,
+                        self.context_window)
 
 
 def workspace_bytes(cfg: ModelConfig) -> int:

@@ -90,6 +90,19 @@ typedef struct bt_config {
                                 accumulation and fp32 residual stream always  */
   float ln_eps;              /* 1e-5 for Pythia                               */
   float rope_base;           /* 10000 for Pythia                              */
+  /* How the context embedding c reaches the token decoder (explainer page
+   * §3.4 "The Token Decoder" and its alternatives to prefix tokens; App. B.3
+   * for the window). 0 = prefix: the last context_window context embeddings
+   * are each projected to P rows (W_p [P*D, D], shared), oldest first, zero
+   * vectors before the first block; 1 = summation: c is projected to L_B
+   * vectors s_0..s_{L_B-1} (W_p [L_B*D, D]), s_0 is the token decoder's
+   * first row and s_{j+1} is added to the input row of token j of the block
+   * (requires prefix_len = 1 and context_window = 1). Both default to the
+   * base model when zero-initialised. Variants other than the base model
+   * run the token decoder as a chain of kernels; context_window > 1 does not
+   * support ragged batches (bt_prefill_ragged returns BT_ENOTSUP). */
+  int32_t context_injection;
+  int32_t context_window;    /* w >= 1 (0 is read as 1)                       */
 } bt_config;
 
 /* One Pythia layer. Matrices are row-major [out, in] (torch Linear layout) in

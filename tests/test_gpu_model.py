@@ -341,3 +341,52 @@ def test_ragged_prefill_rejects_bad_lengths():
             m.prefill_ragged(tok, lengths, pad)
         assert ei.value.code == native.BT_EINVAL, (lengths, pad)
     m.close()
+
+
+# ---- context-injection variants: summation (MEGABYTE-style) and a window of
+# previous context embeddings, against the oracle's readings of them
+
+@pytest.mark.parametrize("lb,T", [(4, 20), (4, 22), (2, 9), (8, 35)])
+def test_fp32_summation_injection_exact_tolerance(lb, T):
+    """Prompts ending on and inside a block (trailing tokens carry s_{j+1}),
+    decode across several blocks."""
+    shape = synth.ModelShape(vocab=300, d_model=128, n_heads=2, block_len=lb,
+                             n_block_layers=2, n_token_layers=2, prefix_len=1, dtype="fp32",
+                             injection="sum")
+    gl, gn, ol = _run(shape, B=3, T=T, G=3 * lb + 3)
+    assert np.abs(gl - ol).max() <= FP32_TOL
+
+
+@pytest.mark.parametrize("w,P,T", [(2, 1, 20), (3, 1, 4), (3, 2, 10), (4, 1, 13)])
+def test_fp32_context_window_exact_tolerance(w, P, T):
+    """Windows longer than the prompt's blocks (zero context slots) and
+    prompts ending inside a block; decode across several blocks so that the
+    window moves on."""
+    shape = synth.ModelShape(vocab=300, d_model=128, n_heads=2, block_len=4,
+                             n_block_layers=2, n_token_layers=2, prefix_len=P, dtype="fp32",
+                             context_window=w)
+    gl, gn, ol = _run(shape, B=3, T=T, G=15)
+    assert np.abs(gl - ol).max() <= FP32_TOL
+
+
+@pytest.mark.parametrize("variant", [{"injection": "sum"}, {"context_window": 3}])
+def test_bf16_context_variants(variant):
+    shape = synth.ModelShape(vocab=1000, d_model=256, n_heads=4, block_len=4,
+                             n_block_layers=2, n_token_layers=2, prefix_len=1, **variant)
+    gl, gn, ol = _run(shape, B=3, T=26, G=14)
+    for s in range(gl.shape[0]):
+        assert gh.rel_l2(gl[s], ol[s]) <= BF16_REL, (s, gh.rel_l2(gl[s], ol[s]))
+
+
+def test_context_window_refuses_ragged_batches():
+    from hierarchical_global_local_b200 import native
+    torch = gh.torch_mod()
+    shape = synth.ModelShape(vocab=300, d_model=128, n_heads=2, block_len=4,
+                             n_block_layers=1, n_token_layers=1, prefix_len=1, dtype="fp32",
+                             context_window=2)
+    model = gh.build_model(shape, synth.make_weights(shape, seed=3), 2, 32)
+    toks = torch.zeros(2, 12, dtype=torch.int32, device="cuda")
+    with pytest.raises(native.BtError) as e:
+        model.prefill_ragged(toks, [12, 9])
+    assert e.value.code == native.BT_ENOTSUP
+    model.close()
