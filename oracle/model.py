@@ -46,6 +46,12 @@ Readings where the page is silent (each listed again in the design notes):
       embeddings c_{i-w+1} .. c_i, oldest first, each through the same
       projection (w*P rows); context embeddings before the first block are
       zero vectors (their rows are b_p). w = 1 is the base model.
+  R11 Grouped-query attention in the block decoder ([BT] §3.4 "The Block
+      Decoder": standard attention, so multi-query / grouped-query
+      attention applies; §6 and App. D.2): H_kv key/value heads, query head
+      h reads key/value head floor(h / (H / H_kv)) (consecutive groups);
+      W_qkv rows are q (H d_head) | k (H_kv d_head) | v (H_kv d_head), the
+      cache holds H_kv heads. The token decoder keeps H_kv = H.
 
 Pins (tests/test_oracle_*.py): HF GPTNeoX (an independent Pythia
 implementation) for the layer stack and the vanilla special case;
@@ -146,27 +152,32 @@ class KVCache:
 
 def pythia_layer(h: np.ndarray, p: Mapping[str, np.ndarray], pos: np.ndarray,
                  cache: KVCache, n_heads: int, rotary_dims: int,
-                 eps: float, rope_base: float) -> np.ndarray:
+                 eps: float, rope_base: float, n_kv_heads: Optional[int] = None) -> np.ndarray:
     """One Pythia layer with parallel attention + MLP residual ([BT] §3.4,
     "The Block Decoder": standard causal self-attention and feed-forward
     layers; reading R6 for the Pythia form).
 
     h: [B, n, D] residual rows at positions ``pos`` (new rows); their keys and
     values are appended to ``cache`` and every new row attends causally over
-    the cache.
+    the cache. n_kv_heads < n_heads: grouped-query attention (reading R11).
     """
     B, n, D = h.shape
     d = D // n_heads
+    hk = n_heads if not n_kv_heads else n_kv_heads
+    Dk = hk * d
     a = layer_norm(h, p["ln1_g"], p["ln1_b"], eps)
     m = layer_norm(h, p["ln2_g"], p["ln2_b"], eps)
-    qkv = a @ p["w_qkv"].T + p["b_qkv"]                               # [B, n, 3D]
-    q = qkv[..., 0 * D:1 * D].reshape(B, n, n_heads, d)
-    k = qkv[..., 1 * D:2 * D].reshape(B, n, n_heads, d)
-    v = qkv[..., 2 * D:3 * D].reshape(B, n, n_heads, d)
+    qkv = a @ p["w_qkv"].T + p["b_qkv"]                               # [B, n, D + 2 Dk]
+    q = qkv[..., :D].reshape(B, n, n_heads, d)
+    k = qkv[..., D:D + Dk].reshape(B, n, hk, d)
+    v = qkv[..., D + Dk:D + 2 * Dk].reshape(B, n, hk, d)
     q = rotary(q, pos, rotary_dims, rope_base)
     k = rotary(k, pos, rotary_dims, rope_base)
     cache.append(k, v, pos)
-    att = attend(q, cache.k, cache.v, pos, cache.pos).reshape(B, n, D)
+    g = n_heads // hk                                                  # query heads per K/V head
+    kk = np.repeat(cache.k, g, axis=2)
+    vv = np.repeat(cache.v, g, axis=2)
+    att = attend(q, kk, vv, pos, cache.pos).reshape(B, n, D)
     mlp = gelu(m @ p["w_1"].T + p["b_1"]) @ p["w_2"].T + p["b_2"]
     return h + (att @ p["w_o"].T + p["b_o"]) + mlp
 
@@ -245,11 +256,11 @@ class BlockTransformerOracle:
                              for l in range(n_t)]
 
     # ---- stacks -----------------------------------------------------------
-    def _stack(self, h, layers, pos, caches):
+    def _stack(self, h, layers, pos, caches, n_kv_heads=None):
         s = self.s
         for lw, cache in zip(layers, caches):
             h = pythia_layer(h, lw, pos, cache, s.n_heads, s.rotary_dims,
-                             s.ln_eps, s.rope_base)
+                             s.ln_eps, s.rope_base, n_kv_heads)
         return h
 
     def block_decoder(self, e: np.ndarray, pos: np.ndarray,
@@ -257,7 +268,7 @@ class BlockTransformerOracle:
         """Causal transformer over block embeddings ([BT] §3.4 "The Block
         Decoder" [orig. §2.3]); returns the context embeddings
         c = LN_b(h) (reading R3)."""
-        h = self._stack(e, self.block_layers, pos, caches)
+        h = self._stack(e, self.block_layers, pos, caches, getattr(self.s, "n_kv_heads", 0) or None)
         return layer_norm(h, self.g["lnf_b_g"], self.g["lnf_b_b"], self.s.ln_eps)
 
     def token_decoder(self, u: np.ndarray, pos: np.ndarray,

@@ -54,6 +54,7 @@ class ModelShape:
     # vectors added to the token decoder's input rows, MEGABYTE-style)
     injection: str = "prefix"
     context_window: int = 1  # w: the last w context embeddings feed the prefix
+    n_kv_heads: int = 0      # block decoder's key/value heads (0: n_heads; < n_heads: GQA)
 
     @property
     def proj_rows(self) -> int:
@@ -136,11 +137,15 @@ def workload(name: str, **overrides) -> Workload:
 # parameter inventory (names, shapes; row-major [out, in] for matrices)
 # --------------------------------------------------------------------------
 
-def layer_param_shapes(s: ModelShape) -> List[Tuple[str, Tuple[int, ...]]]:
+def layer_param_shapes(s: ModelShape, block: bool = False) -> List[Tuple[str, Tuple[int, ...]]]:
+    """Parameters of one layer; block = True: a block-decoder layer, whose
+    q|k|v rows carry n_kv_heads key/value heads."""
     D = s.d_model
+    hk = (s.n_kv_heads or s.n_heads) if block else s.n_heads
+    Nq = D + 2 * hk * s.d_head
     return [
         ("ln1_g", (D,)), ("ln1_b", (D,)), ("ln2_g", (D,)), ("ln2_b", (D,)),
-        ("w_qkv", (3 * D, D)), ("b_qkv", (3 * D,)),
+        ("w_qkv", (Nq, D)), ("b_qkv", (Nq,)),
         ("w_o", (D, D)), ("b_o", (D,)),
         ("w_1", (4 * D, D)), ("b_1", (4 * D,)),
         ("w_2", (D, 4 * D)), ("b_2", (D,)),
@@ -162,7 +167,7 @@ def param_names(s: ModelShape) -> List[Tuple[str, Tuple[int, ...]]]:
     """Flat, ordered inventory: globals then block layers then token layers."""
     names = list(global_param_shapes(s))
     for l in range(s.n_block_layers):
-        names += [(f"block.{l}.{n}", sh) for n, sh in layer_param_shapes(s)]
+        names += [(f"block.{l}.{n}", sh) for n, sh in layer_param_shapes(s, block=True)]
     n_t = s.n_token_layers if s.use_token_decoder else 0
     for l in range(n_t):
         names += [(f"token.{l}.{n}", sh) for n, sh in layer_param_shapes(s)]

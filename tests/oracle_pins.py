@@ -466,3 +466,38 @@ def pin_window_assembly_bruteforce(om) -> float:
             if t <= S:
                 worst = max(worst, float(np.abs(z[:, w * P - 1 + j] - full[:, t]).max()))
     return worst
+
+
+# --------------------------------------------------------------------------
+# grouped-query attention in the block decoder (reading R11)
+# --------------------------------------------------------------------------
+
+GQA = dataclasses.replace(SMALL, n_kv_heads=2)
+
+
+def pin_gqa_equals_mha_with_shared_kv_rows(om) -> float:
+    """GQA with H_kv heads is multi-head attention whose query head h uses
+    copies of key/value head h // (H / H_kv): duplicate those projection
+    rows (a loop over the H query heads) into an MHA model and compare the
+    full pass."""
+    H, hk, D = GQA.n_heads, GQA.n_kv_heads, GQA.d_model
+    d, g = D // H, H // GQA.n_kv_heads
+    pg = params_of(GQA)
+    pm = dict(pg)
+    for l in range(GQA.n_block_layers):
+        w, b = pg[f"block.{l}.w_qkv"], pg[f"block.{l}.b_qkv"]
+        wk, wv = w[D:D + hk * d], w[D + hk * d:D + 2 * hk * d]
+        bk, bv = b[D:D + hk * d], b[D + hk * d:D + 2 * hk * d]
+        rk, rv, ck, cv = [], [], [], []
+        for h in range(H):
+            j = h // g
+            rk.append(wk[j * d:(j + 1) * d])
+            rv.append(wv[j * d:(j + 1) * d])
+            ck.append(bk[j * d:(j + 1) * d])
+            cv.append(bv[j * d:(j + 1) * d])
+        pm[f"block.{l}.w_qkv"] = np.concatenate([w[:D]] + rk + rv, axis=0)
+        pm[f"block.{l}.b_qkv"] = np.concatenate([b[:D]] + ck + cv, axis=0)
+    toks = tokens_of(GQA, S=22)
+    a = om.BlockTransformerOracle(GQA, pg).forward_full(toks)
+    m = om.BlockTransformerOracle(dataclasses.replace(GQA, n_kv_heads=0), pm).forward_full(toks)
+    return float(np.nanmax(np.abs(a - m)))

@@ -40,6 +40,8 @@ def _first_failing_pin(mod):
         ("window_assembly", lambda: pins.pin_window_assembly_bruteforce(mod) < TOL),
         ("incremental_sum", lambda: pins.pin_incremental_equals_full(mod, shape=pins.SUM, T=6, G=9) < TOL),
         ("incremental_window", lambda: pins.pin_incremental_equals_full(mod, shape=pins.WIN, T=6, G=9) < TOL),
+        ("gqa_vs_mha", lambda: pins.pin_gqa_equals_mha_with_shared_kv_rows(mod) < TOL),
+        ("incremental_gqa", lambda: pins.pin_incremental_equals_full(mod, shape=pins.GQA, T=6, G=9) < TOL),
     ]
     for name, c in checks:
         if not c():
@@ -91,18 +93,18 @@ def _prefix_colmajor(c, w, b, P):
     return np.swapaxes(out.reshape(*c.shape[:-1], D, P), -1, -2)
 
 
-def _layer_drop_bias_o(h, p, pos, cache, H, r, eps, base):
+def _layer_drop_bias_o(h, p, pos, cache, H, r, eps, base, hk=None):
     p2 = dict(p)
     p2["b_o"] = np.zeros_like(p["b_o"])
-    return ORIG["pythia_layer"](h, p2, pos, cache, H, r, eps, base)
+    return ORIG["pythia_layer"](h, p2, pos, cache, H, r, eps, base, hk)
 
 
-def _layer_serial_residual(h, p, pos, cache, H, r, eps, base):
+def _layer_serial_residual(h, p, pos, cache, H, r, eps, base, hk=None):
     # GPT-2 style sequential residual instead of Pythia's parallel form
     p_att = dict(p)
     for n in ("w_1", "b_1", "w_2", "b_2"):
         p_att[n] = np.zeros_like(p[n])
-    h1 = ORIG["pythia_layer"](h, p_att, pos, cache, H, r, eps, base)
+    h1 = ORIG["pythia_layer"](h, p_att, pos, cache, H, r, eps, base, hk)
     m = ORIG["layer_norm"](h1, p["ln2_g"], p["ln2_b"], eps)
     return h1 + ORIG["gelu"](m @ p["w_1"].T + p["b_1"]) @ p["w_2"].T + p["b_2"]
 
@@ -134,7 +136,29 @@ SESSION_MUTATIONS = {
 }
 
 
+def _layer_gqa_interleaved(h, p, pos, cache, H, r, eps, base, hk=None):
+    # query head h reads key/value head h % H_kv instead of h // (H / H_kv)
+    if not hk or hk == H:
+        return ORIG["pythia_layer"](h, p, pos, cache, H, r, eps, base, hk)
+    B, n, D = h.shape
+    d = D // H
+    Dk = hk * d
+    a = ORIG["layer_norm"](h, p["ln1_g"], p["ln1_b"], eps)
+    m = ORIG["layer_norm"](h, p["ln2_g"], p["ln2_b"], eps)
+    qkv = a @ p["w_qkv"].T + p["b_qkv"]
+    q = ORIG["rotary"](qkv[..., :D].reshape(B, n, H, d), pos, r, base)
+    k = ORIG["rotary"](qkv[..., D:D + Dk].reshape(B, n, hk, d), pos, r, base)
+    v = qkv[..., D + Dk:].reshape(B, n, hk, d)
+    cache.append(k, v, pos)
+    kk = np.tile(cache.k, (1, 1, H // hk, 1))
+    vv = np.tile(cache.v, (1, 1, H // hk, 1))
+    att = ORIG["attend"](q, kk, vv, pos, cache.pos).reshape(B, n, D)
+    mlp = ORIG["gelu"](m @ p["w_1"].T + p["b_1"]) @ p["w_2"].T + p["b_2"]
+    return h + (att @ p["w_o"].T + p["b_o"]) + mlp
+
+
 MUTATIONS = {
+    "gqa_interleaved": ("pythia_layer", _layer_gqa_interleaved),
     "rotary_sign": ("rotary", _rotary_wrong_sign),
     "rotary_freq": ("rotary", _rotary_wrong_freq),
     "ln_unbiased": ("layer_norm", _ln_unbiased),

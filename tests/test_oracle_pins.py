@@ -119,3 +119,14 @@ def test_injection_variants_incremental_equals_full(shape_name, T):
     """Invariant 1 for both variants, prompts shorter than the window (T = 4:
     one block, two zero context slots) and ending inside a block."""
     assert pins.pin_incremental_equals_full(om, shape=getattr(pins, shape_name), T=T, G=11) < 1e-10
+
+
+# ---- grouped-query attention in the block decoder (reading R11) ------------
+
+def test_gqa_equals_mha_with_shared_key_value_rows():
+    assert pins.pin_gqa_equals_mha_with_shared_kv_rows(om) < 1e-10
+
+
+@pytest.mark.parametrize("T", [8, 10])
+def test_gqa_incremental_equals_full(T):
+    assert pins.pin_incremental_equals_full(om, shape=pins.GQA, T=T, G=11) < 1e-10
