@@ -83,7 +83,7 @@ __global__ void __launch_bounds__(DecCfg<T, DH>::THREADS)
 attn_decode_kernel(const T* __restrict__ q, int ldq, const T* __restrict__ kc,
                    const T* __restrict__ vc, int pairs, int H, int cap, PosSpec kvlen,
                    T* __restrict__ out, int ld_out, float* __restrict__ part,
-                   int* __restrict__ counters, int* status, float qscale) {
+                   int* __restrict__ counters, int* status, float qscale, int qpk) {
   pdl_trigger();
   pdl_wait();
   using C = DecCfg<T, DH>;
@@ -130,7 +130,11 @@ attn_decode_kernel(const T* __restrict__ q, int ldq, const T* __restrict__ kc,
         const int np = pos_base(kvlen, pr / H) + 1;  // this pair's entries
         const int rows = max(0, min(C::CHUNK, np - r0));
         const uint32_t bytes = (uint32_t)rows * C::ROW_BYTES;
-        const size_t off = ((size_t)pr * cap + r0) * DH;
+        // key/value head of query head h: h / qpk (grouped-query attention;
+        // the qpk query heads of one key/value head are consecutive pairs, so
+        // their repeated reads of it come from L2)
+        const int kvp = (pr / H) * (H / qpk) + (pr % H) / qpk;
+        const size_t off = ((size_t)kvp * cap + r0) * DH;
         T* dk = sKV + (size_t)s * 2 * C::CHUNK * DH;
         mbar_arrive_expect_tx(&full[s], 2 * bytes);
         if (bytes) {
@@ -310,7 +314,7 @@ cudaError_t attn_prepare() {
 template <typename T, int DH>
 static cudaError_t launch_dec(const void* q, int ldq, const void* kc, const void* vc, int B,
                               int H, int cap, PosSpec kvlen, void* out, int ld_out,
-                              void* scratch, int* status, cudaStream_t s) {
+                              void* scratch, int* status, cudaStream_t s, int g) {
   using C = DecCfg<T, DH>;
   cudaError_t e = dec_prepare<T, DH>();
   if (e != cudaSuccess) return e;
@@ -323,17 +327,20 @@ static cudaError_t launch_dec(const void* q, int ldq, const void* kc, const void
   const float qscale = 1.4426950408889634f / sqrtf((float)DH);
   BT_LAUNCH(attn_decode_kernel<T, DH>, dim3(G), dim3(C::THREADS), C::SMEM, s, (const T*)q, ldq,
             (const T*)kc, (const T*)vc, pairs, H, cap, kvlen, (T*)out, ld_out, partp, counters,
-            status, qscale);
+            status, qscale, g);
   return cudaSuccess;
 }
 
 cudaError_t launch_attn_decode(int dt, const void* q, int ldq, const void* k_cache,
                                const void* v_cache, int B, int H, int d, int cap,
                                PosSpec kvlen, void* out, int ld_out, void* scratch,
-                               int* status, cudaStream_t s) {
+                               int* status, cudaStream_t s, int Hk) {
   if (B * H == 0) return cudaSuccess;
+  if (Hk <= 0) Hk = H;
+  if (H % Hk) return cudaErrorInvalidValue;
+  const int g = H / Hk;
 #define BT_DEC(T, DHV) \
-  return launch_dec<T, DHV>(q, ldq, k_cache, v_cache, B, H, cap, kvlen, out, ld_out, scratch, status, s)
+  return launch_dec<T, DHV>(q, ldq, k_cache, v_cache, B, H, cap, kvlen, out, ld_out, scratch, status, s, g)
   if (dt == DT_BF16) {
     if (d == 64) BT_DEC(bf16, 64);
     if (d == 128) BT_DEC(bf16, 128);
@@ -353,7 +360,7 @@ cudaError_t launch_attn_decode(int dt, const void* q, int ldq, const void* k_cac
 template <typename T, int DH>
 __global__ void attn_small_kernel(const T* __restrict__ q, int ldq, const T* __restrict__ kc,
                                   const T* __restrict__ vc, int B, int H, int cap, PosSpec qpos,
-                                  T* __restrict__ out, int ld_out, float scale) {
+                                  T* __restrict__ out, int ld_out, float scale, int g) {
   pdl_trigger();
   pdl_wait();
   constexpr int EPL = DH / 32;  // elements per lane
@@ -371,8 +378,9 @@ __global__ void attn_small_kernel(const T* __restrict__ q, int ldq, const T* __r
     qf[x] = to_f(q[(size_t)m * ldq + h * DH + lane + 32 * x]) * scale;
     of[x] = 0.f;
   }
-  const T* kb = kc + ((size_t)b * H + h) * cap * DH;
-  const T* vb = vc + ((size_t)b * H + h) * cap * DH;
+  // key/value head h / g of H / g (grouped-query attention)
+  const T* kb = kc + ((size_t)b * (H / g) + h / g) * cap * DH;
+  const T* vb = vc + ((size_t)b * (H / g) + h / g) * cap * DH;
   float mrun = -FLT_MAX, l = 0.f;
   for (int j = 0; j <= pos; ++j) {
     float s = 0.f;
@@ -392,15 +400,18 @@ __global__ void attn_small_kernel(const T* __restrict__ q, int ldq, const T* __r
 
 cudaError_t launch_attn_small(int dt, const void* q, int ldq, const void* k_cache,
                               const void* v_cache, int B, int H, int d, int cap, PosSpec qpos,
-                              void* out, int ld_out, cudaStream_t s) {
+                              void* out, int ld_out, cudaStream_t s, int Hk) {
   const int warps = B * qpos.rows_per_seq * H;
   if (warps == 0) return cudaSuccess;
+  if (Hk <= 0) Hk = H;
+  if (H % Hk) return cudaErrorInvalidValue;
+  const int g = H / Hk;
   const int grid = (warps + 3) / 4;
   const float scale = 1.4426950408889634f / sqrtf((float)d);
 #define BT_SMALL(T, DHV)                                                                      \
   BT_LAUNCH(attn_small_kernel<T, DHV>, dim3(grid), dim3(128), 0, s, (const T*)q, ldq, (const T*)k_cache,        \
                                                   (const T*)v_cache, B, H, cap, qpos, (T*)out, \
-                                                  ld_out, scale);                             \
+                                                  ld_out, scale, g);                          \
   return cudaGetLastError()
   if (dt == DT_BF16) {
     if (d == 32) { BT_SMALL(bf16, 32); }
@@ -419,9 +430,9 @@ cudaError_t launch_attn_small(int dt, const void* q, int ldq, const void* k_cach
 // positions; query i of a sequence sees cache entries 0..i).
 cudaError_t launch_attn_prefill(int dt, const void* q, int ldq, const void* k_cache,
                                 const void* v_cache, int B, int H, int d, int cap, int n,
-                                void* out, int ld_out, cudaStream_t s) {
+                                void* out, int ld_out, cudaStream_t s, int Hk) {
   PosSpec p{nullptr, POS_ZERO, 0, n};
-  return launch_attn_small(dt, q, ldq, k_cache, v_cache, B, H, d, cap, p, out, ld_out, s);
+  return launch_attn_small(dt, q, ldq, k_cache, v_cache, B, H, d, cap, p, out, ld_out, s, Hk);
 }
 
 }  // namespace bt

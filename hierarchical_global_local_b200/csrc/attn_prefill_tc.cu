@@ -53,7 +53,7 @@ template <int DH>
 __global__ void __launch_bounds__(THREADS, 1)
 attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
                        const __grid_constant__ CUtensorMap mVt, int H, int n, bf16* __restrict__ out,
-                       int ld_out, float scale_log2, int* status) {
+                       int ld_out, float scale_log2, int* status, int g) {
   using PL = Plan<DH>;
   pdl_trigger();
   extern __shared__ uint8_t smem_raw[];
@@ -65,6 +65,7 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
   const int qt = blockIdx.x % nqt;
   const int bh = blockIdx.x / nqt;  // b * H + h
   const int b = bh / H, h = bh - b * H;
+  const int kvh = b * (H / g) + h / g;  // key/value head (grouped-query attention)
   const int q0 = qt * QT;
   const int ntiles = (q0 + QT - 1) / KT + 1;  // key tiles intersecting the causal band
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -101,9 +102,9 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
         if (j >= PL::STAGES) mbar_wait_bounded(&kv_empty[s], ((j / PL::STAGES) + 1) & 1, status);
         mbar_arrive_expect_tx(&kv_full[s], PL::K_BYTES + PL::VT_BYTES);
         for (int kb = 0; kb < PL::KB; ++kb)
-          tc::tma_load_3d(sm + PL::OFF_K + s * PL::K_BYTES + kb * KT * 128, &mK, kb * 64, j * KT, bh, &kv_full[s]);
+          tc::tma_load_3d(sm + PL::OFF_K + s * PL::K_BYTES + kb * KT * 128, &mK, kb * 64, j * KT, kvh, &kv_full[s]);
         for (int kb = 0; kb < KT / 64; ++kb)
-          tc::tma_load_3d(sm + PL::OFF_VT + s * PL::VT_BYTES + kb * DH * 128, &mVt, j * KT + kb * 64, 0, bh,
+          tc::tma_load_3d(sm + PL::OFF_VT + s * PL::VT_BYTES + kb * DH * 128, &mVt, j * KT + kb * 64, 0, kvh,
                &kv_full[s]);
       }
     }
@@ -265,7 +266,7 @@ bool map3(CUtensorMap* m, const void* base, long long x, long long y, long long 
 
 template <int DH>
 cudaError_t launch_tc(const void* q, int ldq, const void* kc, const void* vt, int vt_ld, int B,
-                      int H, int cap, int n, void* out, int ld_out, int* status, cudaStream_t s) {
+                      int H, int cap, int n, void* out, int ld_out, int* status, cudaStream_t s, int Hk) {
   // the attribute applies to the current device only
   static bool prepared[MAX_DEVICES] = {};
   const int dev = current_device();
@@ -278,14 +279,14 @@ cudaError_t launch_tc(const void* q, int ldq, const void* kc, const void* vt, in
   CUtensorMap mQ, mK, mVt;
   // Q rows b*n + i, dims (h*d + e): {ldq cols, n rows, B}
   if (!map3(&mQ, q, ldq, n, B, ldq, (long long)n * ldq, QT)) return cudaErrorInvalidValue;
-  // K cache [B*H][cap][d], valid rows < n
-  if (!map3(&mK, kc, DH, n, (long long)B * H, DH, (long long)cap * DH, KT)) return cudaErrorInvalidValue;
-  // V^T [B*H][d][vt_ld], valid keys < n
-  if (!map3(&mVt, vt, n, DH, (long long)B * H, vt_ld, (long long)DH * vt_ld, DH)) return cudaErrorInvalidValue;
+  // K cache [B*Hk][cap][d], valid rows < n
+  if (!map3(&mK, kc, DH, n, (long long)B * Hk, DH, (long long)cap * DH, KT)) return cudaErrorInvalidValue;
+  // V^T [B*Hk][d][vt_ld], valid keys < n
+  if (!map3(&mVt, vt, n, DH, (long long)B * Hk, vt_ld, (long long)DH * vt_ld, DH)) return cudaErrorInvalidValue;
   const int nqt = (n + QT - 1) / QT;
   const float scale = 1.4426950408889634f / sqrtf((float)DH);
   BT_LAUNCH(attn_prefill_tc_kernel<DH>, dim3(B * H * nqt), dim3(THREADS), Plan<DH>::BYTES, s, mQ, mK,
-            mVt, H, n, (bf16*)out, ld_out, scale, status);
+            mVt, H, n, (bf16*)out, ld_out, scale, status, H / Hk);
   return cudaSuccess;
 }
 
@@ -300,10 +301,12 @@ int attn_prefill_tc_supported(int dt, int d, int ldq, int vt_ld) {
 
 cudaError_t launch_attn_prefill_tc(const void* q, int ldq, const void* k_cache, const void* vt,
                                    int vt_ld, int B, int H, int d, int cap, int n, void* out,
-                                   int ld_out, int* status, cudaStream_t s) {
+                                   int ld_out, int* status, cudaStream_t s, int Hk) {
   if (B * H * n == 0) return cudaSuccess;
-  if (d == 64) return launch_tc<64>(q, ldq, k_cache, vt, vt_ld, B, H, cap, n, out, ld_out, status, s);
-  if (d == 128) return launch_tc<128>(q, ldq, k_cache, vt, vt_ld, B, H, cap, n, out, ld_out, status, s);
+  if (Hk <= 0) Hk = H;
+  if (H % Hk) return cudaErrorInvalidValue;
+  if (d == 64) return launch_tc<64>(q, ldq, k_cache, vt, vt_ld, B, H, cap, n, out, ld_out, status, s, Hk);
+  if (d == 128) return launch_tc<128>(q, ldq, k_cache, vt, vt_ld, B, H, cap, n, out, ld_out, status, s, Hk);
   return cudaErrorInvalidValue;
 }
 

@@ -457,7 +457,7 @@ cudaError_t launch_rope_table(float2* tab, int n_pos, int rot, float base, cudaS
 }
 
 template <typename T>
-__global__ void rope_append_kernel(const T* __restrict__ qkv, int D, int H, int rot,
+__global__ void rope_append_kernel(const T* __restrict__ qkv, int D, int H, int Hk, int rot,
                                    const float2* __restrict__ tab, PosSpec ps,
                                    T* __restrict__ q_out, T* __restrict__ kc,
                                    T* __restrict__ vc, int cap, T* __restrict__ vt, int vt_ld) {
@@ -468,10 +468,12 @@ __global__ void rope_append_kernel(const T* __restrict__ qkv, int D, int H, int 
   const int half = rot >> 1;
   const int b = m / ps.rows_per_seq;
   const int pos = pos_base(ps, b) + (m - b * ps.rows_per_seq);
-  const T* row = qkv + (size_t)m * 3 * D;
-  for (int x = threadIdx.x; x < 3 * D; x += blockDim.x) {
-    const int part = x / D;  // 0 q, 1 k, 2 v
-    const int c = x - part * D;
+  // row: q (H heads) | k (Hk heads) | v (Hk heads)
+  const int Dk = Hk * d, W = D + 2 * Dk;
+  const T* row = qkv + (size_t)m * W;
+  for (int x = threadIdx.x; x < W; x += blockDim.x) {
+    const int part = x < D ? 0 : (x < D + Dk ? 1 : 2);  // 0 q, 1 k, 2 v
+    const int c = part == 0 ? x : (part == 1 ? x - D : x - D - Dk);
     const int hh = c / d, e = c - hh * d;
     float v = to_f(row[x]);
     if (part < 2 && e < rot) {
@@ -484,19 +486,20 @@ __global__ void rope_append_kernel(const T* __restrict__ qkv, int D, int H, int 
       q_out[(size_t)m * D + c] = from_f<T>(v);
     } else {
       T* cache = (part == 1) ? kc : vc;
-      cache[(((size_t)b * H + hh) * cap + pos) * d + e] = from_f<T>(v);
-      if (part == 2 && vt) vt[(((size_t)b * H + hh) * d + e) * vt_ld + pos] = from_f<T>(v);
+      cache[(((size_t)b * Hk + hh) * cap + pos) * d + e] = from_f<T>(v);
+      if (part == 2 && vt) vt[(((size_t)b * Hk + hh) * d + e) * vt_ld + pos] = from_f<T>(v);
     }
   }
 }
 
-// V^T [(b*H + h)*d + e][pos] for positions p0 + [0, 64) of one (sequence,
-// head): the tile goes through shared memory so that both the reads (along
-// the head dims of a row) and the writes (along positions) are coalesced.
-// Rows of a sequence are consecutive; row i has position pos0 + i.
+// V^T [(b*Hk + h)*d + e][pos] for positions p0 + [0, 64) of one (sequence,
+// key/value head): the tile goes through shared memory so that both the
+// reads (along the head dims of a row) and the writes (along positions) are
+// coalesced. Rows of a sequence are consecutive, W wide, V at column voff;
+// row i has position pos0 + i.
 template <typename T>
 __global__ void __launch_bounds__(256)
-vt_write_kernel(const T* __restrict__ qkv, int D, int H, int d, int rows, int pos0,
+vt_write_kernel(const T* __restrict__ qkv, int W, int voff, int H, int d, int rows, int pos0,
                 T* __restrict__ vt, int vt_ld) {
   pdl_trigger();
   pdl_wait();
@@ -508,7 +511,7 @@ vt_write_kernel(const T* __restrict__ qkv, int D, int H, int d, int rows, int po
     for (int x = threadIdx.x; x < 64 * ec; x += blockDim.x) {
       const int ii = x / ec, e = x - ii * ec;
       const int i = i0 + ii;
-      tile[ii][e] = (i < rows) ? to_f(qkv[((size_t)b * rows + i) * 3 * D + 2 * D + h * d + e0 + e]) : 0.f;
+      tile[ii][e] = (i < rows) ? to_f(qkv[((size_t)b * rows + i) * W + voff + h * d + e0 + e]) : 0.f;
     }
     __syncthreads();
     for (int x = threadIdx.x; x < 64 * ec; x += blockDim.x) {
@@ -522,27 +525,30 @@ vt_write_kernel(const T* __restrict__ qkv, int D, int H, int d, int rows, int po
 
 cudaError_t launch_rope_append(int dt, const void* qkv, int M, int D, int H, int rot,
                                const float2* rope_tab, PosSpec pos, void* q_out, void* k_cache,
-                               void* v_cache, int cap, cudaStream_t s, void* vt, int vt_ld) {
+                               void* v_cache, int cap, cudaStream_t s, void* vt, int vt_ld, int Hk) {
   if (M == 0) return cudaSuccess;
+  if (Hk <= 0) Hk = H;
+  if (H % Hk) return cudaErrorInvalidValue;
   // V^T is written for positions known on the host (prefill) only
   if (vt && pos.mode != POS_ZERO) return cudaErrorInvalidValue;
   if (dt == DT_BF16) {
-    BT_LAUNCH(rope_append_kernel<bf16>, dim3(M), dim3(256), 0, s, (const bf16*)qkv, D, H, rot, rope_tab, pos,
+    BT_LAUNCH(rope_append_kernel<bf16>, dim3(M), dim3(256), 0, s, (const bf16*)qkv, D, H, Hk, rot, rope_tab, pos,
                                                (bf16*)q_out, (bf16*)k_cache, (bf16*)v_cache, cap, (bf16*)nullptr, 0);
   }
   else {
-    BT_LAUNCH(rope_append_kernel<float>, dim3(M), dim3(256), 0, s, (const float*)qkv, D, H, rot, rope_tab, pos,
+    BT_LAUNCH(rope_append_kernel<float>, dim3(M), dim3(256), 0, s, (const float*)qkv, D, H, Hk, rot, rope_tab, pos,
                                                 (float*)q_out, (float*)k_cache, (float*)v_cache,
                                                 cap, (float*)nullptr, 0);
   }
   if (vt) {
     const int rows = pos.rows_per_seq, B = M / rows, d = D / H;
-    const dim3 grid((rows + 63) / 64, B * H);
+    const int W = D + 2 * Hk * d, voff = D + Hk * d;
+    const dim3 grid((rows + 63) / 64, B * Hk);
     if (dt == DT_BF16)
-      BT_LAUNCH(vt_write_kernel<bf16>, grid, dim3(256), 0, s, (const bf16*)qkv, D, H, d, rows, pos.add,
+      BT_LAUNCH(vt_write_kernel<bf16>, grid, dim3(256), 0, s, (const bf16*)qkv, W, voff, Hk, d, rows, pos.add,
                 (bf16*)vt, vt_ld);
     else
-      BT_LAUNCH(vt_write_kernel<float>, grid, dim3(256), 0, s, (const float*)qkv, D, H, d, rows, pos.add,
+      BT_LAUNCH(vt_write_kernel<float>, grid, dim3(256), 0, s, (const float*)qkv, W, voff, Hk, d, rows, pos.add,
                 (float*)vt, vt_ld);
   }
   return cudaGetLastError();

@@ -41,12 +41,14 @@ __device__ __forceinline__ void epi_apply_rope(const Epi& e, int m, int n, float
                                                float partner) {
   const float v = acc + e.bias[n];
   const int D = e.D;
-  if (n >= 3 * D) {
-    reinterpret_cast<T*>(e.out1)[(size_t)m * e.ld1 + D + (n - 3 * D)] = from_f<T>(gelu_erf(v));
+  const int d = D / e.H;
+  const int Dk = (e.Hk > 0 ? e.Hk : e.H) * d;
+  if (n >= D + 2 * Dk) {
+    reinterpret_cast<T*>(e.out1)[(size_t)m * e.ld1 + D + (n - D - 2 * Dk)] = from_f<T>(gelu_erf(v));
     return;
   }
-  const int part = n / D, c = n - part * D;
-  const int d = D / e.H;
+  const int part = n < D ? 0 : (n < D + Dk ? 1 : 2);
+  const int c = part == 0 ? n : (part == 1 ? n - D : n - D - Dk);
   const int hh = c / d, dim = c - hh * d;
   const int b = m / e.pos.rows_per_seq;
   const int pos = pos_base(e.pos, b) + (m - b * e.pos.rows_per_seq);
@@ -61,7 +63,7 @@ __device__ __forceinline__ void epi_apply_rope(const Epi& e, int m, int n, float
     reinterpret_cast<T*>(e.out0)[(size_t)m * e.ld0 + c] = from_f<T>(out);
   } else {
     T* cache = reinterpret_cast<T*>(part == 1 ? e.kc : e.vc);
-    cache[(((size_t)b * e.H + hh) * e.cap + pos) * d + dim] = from_f<T>(out);
+    cache[(((size_t)b * (Dk / d) + hh) * e.cap + pos) * d + dim] = from_f<T>(out);
   }
 }
 
@@ -80,15 +82,18 @@ __device__ __forceinline__ void epi_cols(const Epi& e, int m0, int cnt, int n, i
     case EPI_QKV1_ROPE: {
       const float bn = e.bias[n];
       const int D = e.D;
-      if (n >= 3 * D) {
-        T* o = reinterpret_cast<T*>(e.out1) + D + (n - 3 * D);
+      const int d = D / e.H;
+      const int Hk = e.Hk > 0 ? e.Hk : e.H, Dk = Hk * d;
+      if (n >= D + 2 * Dk) {
+        T* o = reinterpret_cast<T*>(e.out1) + D + (n - D - 2 * Dk);
 #pragma unroll
         for (int j = 0; j < CH; ++j)
           if (j < lim) o[(size_t)(m0 + j) * e.ld1] = from_f<T>(gelu_erf(v[j] + bn));
         return;
       }
-      const int part = n / D, c = n - part * D;
-      const int d = D / e.H;
+      // q (H heads) | k (Hk heads) | v (Hk heads)
+      const int part = n < D ? 0 : (n < D + Dk ? 1 : 2);
+      const int c = part == 0 ? n : (part == 1 ? n - D : n - D - Dk);
       const int hh = c / d, dim = c - hh * d;
       const int half = e.rot >> 1;
       const bool rot = part < 2 && dim < e.rot;
@@ -118,7 +123,7 @@ __device__ __forceinline__ void epi_cols(const Epi& e, int m0, int cnt, int n, i
           reinterpret_cast<T*>(e.out0)[(size_t)(m0 + j) * e.ld0 + c] = from_f<T>(out);
         } else {
           T* cache = reinterpret_cast<T*>(part == 1 ? e.kc : e.vc);
-          cache[(((size_t)seq[j] * e.H + hh) * e.cap + pos[j]) * d + dim] = from_f<T>(out);
+          cache[(((size_t)seq[j] * Hk + hh) * e.cap + pos[j]) * d + dim] = from_f<T>(out);
         }
       }
       return;

@@ -97,7 +97,7 @@ cudaError_t launch_ln_rows(int dt, const float* h, int R, int row_step, int row_
 cudaError_t launch_rope_append(int dt, const void* qkv, int M, int D, int H, int rot,
                                const float2* rope_tab, PosSpec pos, void* q_out, void* k_cache,
                                void* v_cache, int cap, cudaStream_t s, void* vt = nullptr,
-                               int vt_ld = 0);
+                               int vt_ld = 0, int Hk = 0);  // Hk: key/value heads (0 = H)
 cudaError_t launch_rope_table(float2* tab, int n_pos, int rot, float base, cudaStream_t s);
 
 // ---- attention --------------------------------------------------------------
@@ -117,26 +117,29 @@ constexpr size_t attn_decode_scratch_bytes_for(long long pairs, int d) {
 // One-time setup of the decode-attention kernels (shared-memory limits).
 cudaError_t attn_prepare();
 int attn_decode_max_splits(int d, int cap, int dt);
+// Hk: key/value heads of the caches ([B][Hk][cap][d]); query head h reads
+// head h / (H / Hk) (grouped-query attention; 0 = H). Same in the attention
+// launchers below.
 cudaError_t launch_attn_decode(int dt, const void* q, int ldq, const void* k_cache,
                                const void* v_cache, int B, int H, int d, int cap,
                                PosSpec kvlen, void* out, int ld_out, void* scratch,
-                               int* status, cudaStream_t s);
+                               int* status, cudaStream_t s, int Hk = 0);
 // Small causal attention: rows_per_seq queries per sequence at positions
 // pos_base(qpos) + i; query at position p attends to cache entries 0..p.
 cudaError_t launch_attn_small(int dt, const void* q, int ldq, const void* k_cache,
                               const void* v_cache, int B, int H, int d, int cap, PosSpec qpos,
-                              void* out, int ld_out, cudaStream_t s);
+                              void* out, int ld_out, cudaStream_t s, int Hk = 0);
 // Tensor-core prefill attention (bf16, d in {64, 128}): as launch_attn_prefill
 // but V is read through its transpose vt [B*H][d][vt_ld] (keys contiguous).
 int attn_prefill_tc_supported(int dt, int d, int ldq, int vt_ld);
 cudaError_t launch_attn_prefill_tc(const void* q, int ldq, const void* k_cache, const void* vt,
                                    int vt_ld, int B, int H, int d, int cap, int n, void* out,
-                                   int ld_out, int* status, cudaStream_t s);
+                                   int ld_out, int* status, cudaStream_t s, int Hk = 0);
 // Prefill causal attention over n positions 0..n-1 of every sequence:
 // q rows b*n + i of q [B*n, ldq]; out rows likewise.
 cudaError_t launch_attn_prefill(int dt, const void* q, int ldq, const void* k_cache,
                                 const void* v_cache, int B, int H, int d, int cap, int n,
-                                void* out, int ld_out, cudaStream_t s);
+                                void* out, int ld_out, cudaStream_t s, int Hk = 0);
 
 // ---- GEMM -----------------------------------------------------------------
 enum EpiKind : int {
@@ -188,6 +191,9 @@ struct Epi {
   int ln_step;
   int ln_off;
   float ln_eps;
+  // EPI_QKV1_ROPE: key/value heads (0 = H): output features are q (D) |
+  // k (Hk d) | v (Hk d) | fc1 (4D), the caches [B][Hk][cap][d]
+  int Hk;
 };
 // True when launch_gemm runs EPI_LOGITS_ARGMAX for this shape.
 int gemm_argmax_fusable(int dt, int M, int N, int K);

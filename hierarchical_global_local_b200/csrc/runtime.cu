@@ -45,9 +45,11 @@ void bt::note_cuda_error(const char* what, cudaError_t e) {
 namespace {
 
 struct LayerW {
-  void* w_qkv1 = nullptr;  // [7D, D]   rows q | k | v | fc1
+  void* w_qkv1 = nullptr;  // [Nq + 4D, D] rows q | k | v | fc1
   void* w_o2 = nullptr;    // [D, 5D]   cols W_o | W_2
-  float* b_qkv1 = nullptr; // [7D]
+  float* b_qkv1 = nullptr; // [Nq + 4D]
+  int Hk = 0;              // key/value heads (block decoder: H_kv; token decoder: H)
+  int Nq = 0;              // q | k | v width: D + 2 Hk d_head (3D without GQA)
   float* b_o2 = nullptr;   // [D]       b_o + b_2
   float *ln1_g = nullptr, *ln1_b = nullptr, *ln2_g = nullptr, *ln2_b = nullptr;
 };
@@ -72,6 +74,7 @@ struct Dims {
   // prows = output rows of the context projection (Pp, or L_B in
   // summation). P above = the token decoder's context rows (w * Pp, or 1).
   int inj, w, Pp, prows;
+  int Hkb;     // block decoder's key/value heads (grouped-query attention when < H)
   size_t eb;
   int n_cap;   // block-cache entries per sequence
   int l_cap;   // local-cache rows per sequence
@@ -107,6 +110,8 @@ int dims_of(const bt_config* c, Dims* o) {
   if (d.inj == 1 && (d.P != 1 || d.w != 1)) return BT_EINVAL;
   d.Pp = d.P;
   d.prows = d.inj ? d.L : d.Pp;
+  d.Hkb = c->n_kv_heads > 0 ? c->n_kv_heads : d.H;
+  if (d.H % d.Hkb) return BT_EINVAL;
   if (d.tokdec && !d.inj) d.P = d.w * d.Pp;
   if (!(c->ln_eps > 0.f) || !(c->rope_base > 0.f)) return BT_EINVAL;
   d.eb = dt_size(d.dt);
@@ -238,18 +243,20 @@ static size_t carve(bt_model* m, const Dims& d, void* ws) {
   Carver c(ws);
   const size_t eb = d.eb;
   const size_t D = d.D;
-  auto layer = [&](LayerW& w) {
-    w.w_qkv1 = c.take(7 * D * D * eb);
+  auto layer = [&](LayerW& w, int Hk) {
+    w.Hk = Hk;
+    w.Nq = (int)(D + 2 * (size_t)Hk * d.d);
+    w.w_qkv1 = c.take((w.Nq + 4 * D) * D * eb);
     w.w_o2 = c.take(5 * D * D * eb);
-    w.b_qkv1 = (float*)c.take(7 * D * 4);
+    w.b_qkv1 = (float*)c.take((w.Nq + 4 * D) * 4);
     w.b_o2 = (float*)c.take(D * 4);
     w.ln1_g = (float*)c.take(D * 4); w.ln1_b = (float*)c.take(D * 4);
     w.ln2_g = (float*)c.take(D * 4); w.ln2_b = (float*)c.take(D * 4);
   };
   m->blk.assign(d.Nb, LayerW());
   m->tok.assign(d.Nt, LayerW());
-  for (auto& w : m->blk) layer(w);
-  for (auto& w : m->tok) layer(w);
+  for (auto& w : m->blk) layer(w, d.Hkb);
+  for (auto& w : m->tok) layer(w, d.H);
   m->blk_emb = c.take((size_t)d.V * (D / d.L) * eb);
   m->lnf_b_g = (float*)c.take(D * 4); m->lnf_b_b = (float*)c.take(D * 4);
   if (d.tokdec) {
@@ -265,7 +272,7 @@ static size_t carve(bt_model* m, const Dims& d, void* ws) {
   m->kt_layer = (size_t)d.Bmax * D * d.l_cap;
   m->kt = c.take(m->kt_layer * (d.Nt > 0 ? d.Nt : 0) * eb);
   m->vt = c.take(m->kt_layer * (d.Nt > 0 ? d.Nt : 0) * eb);
-  m->kb_layer = (size_t)d.Bmax * D * d.n_cap;
+  m->kb_layer = (size_t)d.Bmax * d.Hkb * d.d * d.n_cap;
   m->kb = c.take(m->kb_layer * d.Nb * eb);
   m->vb = c.take(m->kb_layer * d.Nb * eb);
   // activations
@@ -354,16 +361,17 @@ static int copy_layer(bt_model* m, const LayerW& w, const bt_layer_weights& s) {
       !s.b_1_dev || !s.b_2_dev || !s.ln1_g_dev || !s.ln1_b_dev || !s.ln2_g_dev || !s.ln2_b_dev)
     return BT_EINVAL;
   uint8_t* q1 = (uint8_t*)w.w_qkv1;
-  BT_CUDA(cudaMemcpyAsync(q1, s.w_qkv_dev, 3 * D * D * eb, cudaMemcpyDeviceToDevice, st));
-  BT_CUDA(cudaMemcpyAsync(q1 + 3 * D * D * eb, s.w_1_dev, 4 * D * D * eb,
+  const size_t Nq = w.Nq;
+  BT_CUDA(cudaMemcpyAsync(q1, s.w_qkv_dev, Nq * D * eb, cudaMemcpyDeviceToDevice, st));
+  BT_CUDA(cudaMemcpyAsync(q1 + Nq * D * eb, s.w_1_dev, 4 * D * D * eb,
                           cudaMemcpyDeviceToDevice, st));
   uint8_t* o2 = (uint8_t*)w.w_o2;
   BT_CUDA(cudaMemcpy2DAsync(o2, 5 * D * eb, s.w_o_dev, D * eb, D * eb, D,
                             cudaMemcpyDeviceToDevice, st));
   BT_CUDA(cudaMemcpy2DAsync(o2 + D * eb, 5 * D * eb, s.w_2_dev, 4 * D * eb, 4 * D * eb, D,
                             cudaMemcpyDeviceToDevice, st));
-  BT_CUDA(launch_convert_to_f32(d.dt, s.b_qkv_dev, w.b_qkv1, 3 * D, st));
-  BT_CUDA(launch_convert_to_f32(d.dt, s.b_1_dev, w.b_qkv1 + 3 * D, 4 * D, st));
+  BT_CUDA(launch_convert_to_f32(d.dt, s.b_qkv_dev, w.b_qkv1, Nq, st));
+  BT_CUDA(launch_convert_to_f32(d.dt, s.b_1_dev, w.b_qkv1 + Nq, 4 * D, st));
   BT_CUDA(launch_add_to_f32(d.dt, s.b_o_dev, s.b_2_dev, w.b_o2, D, st));
   BT_CUDA(launch_convert_to_f32(d.dt, s.ln1_g_dev, w.ln1_g, D, st));
   BT_CUDA(launch_convert_to_f32(d.dt, s.ln1_b_dev, w.ln1_b, D, st));
@@ -528,39 +536,42 @@ static int run_layer(bt_model* m, const LayerW& w, float* h, int M, PosSpec pos,
   // the fused rotary epilogue does not write V^T, which the tensor-core
   // prefill attention reads: prefill takes the separate rotary kernel then
   const bool pf_tc = ak == ATT_PREFILL && attn_prefill_tc_supported(d.dt, d.d, D, m->vt_ld);
-  if (!pf_tc && gemm_rope_fusable(d.dt, M, 7 * D, D, 3 * D, D, d.d, d.rot)) {
+  const int Nq = w.Nq, N1 = w.Nq + 4 * D;  // q|k|v width (w.Hk key/value heads), + fc1
+  if (!pf_tc && gemm_rope_fusable(d.dt, M, N1, D, Nq, D, d.d, d.rot)) {
     // q|k|v|fc1 GEMM with rotary and the KV-cache append in its epilogue
-    ProfScope p(m, s, BT_K_GEMM, M, 7 * D, D);
-    Epi e1{EPI_QKV1_ROPE, m->qrot, D, m->a2, 5 * D, w.b_qkv1, 3 * D, D,
+    ProfScope p(m, s, BT_K_GEMM, M, N1, D);
+    Epi e1{EPI_QKV1_ROPE, m->qrot, D, m->a2, 5 * D, w.b_qkv1, Nq, D,
            m->rope_tab, d.rot, d.H, kc, vc, cap, pos};
-    BT_CUDA(launch_gemm(d.dt, m->x1, 2 * D, w.w_qkv1, D, M, 7 * D, D, 3 * D, D, e1, m->gs, m->status, s));
+    e1.Hk = w.Hk;
+    BT_CUDA(launch_gemm(d.dt, m->x1, 2 * D, w.w_qkv1, D, M, N1, D, Nq, D, e1, m->gs, m->status, s));
   } else {
     {
-      ProfScope p(m, s, BT_K_GEMM, M, 7 * D, D);
-      Epi e1{EPI_QKV1, m->qkv, 3 * D, m->a2, 5 * D, w.b_qkv1, 3 * D, D};
-      BT_CUDA(launch_gemm(d.dt, m->x1, 2 * D, w.w_qkv1, D, M, 7 * D, D, 3 * D, D, e1, m->gs, m->status, s));
+      ProfScope p(m, s, BT_K_GEMM, M, N1, D);
+      Epi e1{EPI_QKV1, m->qkv, Nq, m->a2, 5 * D, w.b_qkv1, Nq, D};
+      BT_CUDA(launch_gemm(d.dt, m->x1, 2 * D, w.w_qkv1, D, M, N1, D, Nq, D, e1, m->gs, m->status, s));
     }
-    ProfScope p(m, s, BT_K_ROPE_APPEND, M, 3 * D, 0);
+    ProfScope p(m, s, BT_K_ROPE_APPEND, M, Nq, 0);
     // the tensor-core prefill attention reads V through its transpose
     BT_CUDA(launch_rope_append(d.dt, m->qkv, M, D, d.H, d.rot, m->rope_tab, pos, m->qrot, kc, vc,
-                               cap, s, pf_tc ? m->vtr : nullptr, m->vt_ld));
+                               cap, s, pf_tc ? m->vtr : nullptr, m->vt_ld, w.Hk));
   }
   const int Bseq = M / pos.rows_per_seq;
   if (ak == ATT_PREFILL) {
     ProfScope p(m, s, BT_K_ATTN_PREFILL, Bseq * d.H, n_prefill, d.d);
     if (attn_prefill_tc_supported(d.dt, d.d, D, m->vt_ld))
       BT_CUDA(launch_attn_prefill_tc(m->qrot, D, kc, m->vtr, m->vt_ld, Bseq, d.H, d.d, cap, n_prefill,
-                                     m->a2, 5 * D, m->status, s));
+                                     m->a2, 5 * D, m->status, s, w.Hk));
     else
-      BT_CUDA(launch_attn_prefill(d.dt, m->qrot, D, kc, vc, Bseq, d.H, d.d, cap, n_prefill, m->a2, 5 * D, s));
+      BT_CUDA(launch_attn_prefill(d.dt, m->qrot, D, kc, vc, Bseq, d.H, d.d, cap, n_prefill, m->a2, 5 * D, s,
+                                  w.Hk));
   } else if (ak == ATT_DECODE) {
     // entries read: the block index of the fed token + 1 (known on the host)
     ProfScope p(m, s, BT_K_ATTN_DECODE, Bseq * d.H, m->t / d.L + 1, d.d);
     BT_CUDA(launch_attn_decode(d.dt, m->qrot, D, kc, vc, Bseq, d.H, d.d, cap, pos, m->a2, 5 * D,
-                               m->attn_scratch, m->status, s));
+                               m->attn_scratch, m->status, s, w.Hk));
   } else {
     ProfScope p(m, s, BT_K_ATTN_LOCAL, M * d.H, cap, d.d);
-    BT_CUDA(launch_attn_small(d.dt, m->qrot, D, kc, vc, Bseq, d.H, d.d, cap, pos, m->a2, 5 * D, s));
+    BT_CUDA(launch_attn_small(d.dt, m->qrot, D, kc, vc, Bseq, d.H, d.d, cap, pos, m->a2, 5 * D, s, w.Hk));
   }
   {
     ProfScope p(m, s, BT_K_GEMM, M, D, 5 * D);
@@ -843,7 +854,7 @@ static bool block_step_fused(const bt_model* m, int B) {
   const char* env = getenv("BT_DECODE_BLOCK_STEP");
   if (!env || strcmp(env, "fused") != 0) return false;
   // its attention phase assumes one cache length for the whole batch
-  if (!m->ts_att || d.Nb < 1 || d.P != 1 || d.inj || m->ragged) return false;
+  if (!m->ts_att || d.Nb < 1 || d.P != 1 || d.inj || d.Hkb != d.H || m->ragged) return false;
   if (!token_step_block_supported(d.dt, B, d.D, d.H, d.rot, d.V, d.Nt, d.Nb, d.P, d.l_cap, d.n_cap, d.L))
     return false;
   const long long ls = d.Nt > 1 ? (long long)((uint8_t*)m->tok[1].w_qkv1 - (uint8_t*)m->tok[0].w_qkv1) : 0;

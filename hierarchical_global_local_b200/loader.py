@@ -46,7 +46,7 @@ def model_config(shape, max_batch: int, max_seq: int) -> native.ModelConfig:
         rotary_dims=shape.rotary_dims, use_token_decoder=shape.use_token_decoder,
         max_batch=max_batch, max_seq=max_seq, dtype=shape.dtype, ln_eps=shape.ln_eps,
         rope_base=shape.rope_base, injection=getattr(shape, "injection", "prefix"),
-        context_window=getattr(shape, "context_window", 1))
+        context_window=getattr(shape, "context_window", 1), n_kv_heads=getattr(shape, "n_kv_heads", 0))
 
 
 def build_model(shape, params, max_batch: int, max_seq: int) -> native.BlockTransformer:

@@ -37,7 +37,7 @@ class BtConfig(ctypes.Structure):
         "vocab", "d_model", "n_heads", "block_len", "n_block_layers", "n_token_layers",
         "prefix_len", "rotary_dims", "use_token_decoder", "max_batch", "max_seq", "dtype")] + \
         [("ln_eps", c_float), ("rope_base", c_float),
-         ("context_injection", c_int32), ("context_window", c_int32)]
+         ("context_injection", c_int32), ("context_window", c_int32), ("n_kv_heads", c_int32)]
 
 
 LAYER_FIELDS = ("ln1_g", "ln1_b", "ln2_g", "ln2_b", "w_qkv", "b_qkv", "w_o", "b_o",
@@ -170,6 +170,7 @@ class ModelConfig:
     rope_base: float = 10000.0
     injection: str = "prefix"  # "prefix" | "sum"
     context_window: int = 1
+    n_kv_heads: int = 0        # block decoder (0: n_heads)
 
     def c(self) -> BtConfig:
         return BtConfig(self.vocab, self.d_model, self.n_heads, self.block_len,
@@ -177,7 +178,7 @@ class ModelConfig:
                         self.rotary_dims, 1 if self.use_token_decoder else 0, self.max_batch,
                         self.max_seq, BT_BF16 if self.dtype == "bf16" else BT_FP32,
                         self.ln_eps, self.rope_base, 1 if self.injection == "sum" else 0,
-                        self.context_window)
+                        self.context_window, self.n_kv_heads)
 
 
 def workspace_bytes(cfg: ModelConfig) -> int:

@@ -103,11 +103,18 @@ typedef struct bt_config {
    * support ragged batches (bt_prefill_ragged returns BT_ENOTSUP). */
   int32_t context_injection;
   int32_t context_window;    /* w >= 1 (0 is read as 1)                       */
+  /* Key/value heads of the block decoder's attention (grouped-query
+   * attention, explainer page §3.4 "The Block Decoder": standard attention,
+   * so MQA/GQA apply); query head h reads key/value head h / (H / H_kv);
+   * 0 = n_heads; must divide n_heads. The token decoder keeps H heads. */
+  int32_t n_kv_heads;
 } bt_config;
 
 /* One Pythia layer. Matrices are row-major [out, in] (torch Linear layout) in
  * the config dtype; vectors are in the config dtype too.
  *   w_qkv [3D, D] rows ordered q | k | v, each head-major [H, d_head]; b_qkv [3D]
+ *     (block-decoder layers with n_kv_heads = H_kv: [D + 2 H_kv d_head, D],
+ *     k and v with H_kv heads each)
  *   w_o [D, D], b_o [D]; w_1 [4D, D], b_1 [4D]; w_2 [D, 4D], b_2 [D]
  *   ln1_* feeds attention, ln2_* feeds the MLP (parallel residual). */
 typedef struct bt_layer_weights {

@@ -390,3 +390,25 @@ def test_context_window_refuses_ragged_batches():
         model.prefill_ragged(toks, [12, 9])
     assert e.value.code == native.BT_ENOTSUP
     model.close()
+
+
+# ---- grouped-query attention in the block decoder ---------------------------
+
+@pytest.mark.parametrize("hk", [1, 2])
+def test_fp32_gqa_block_decoder_exact_tolerance(hk):
+    shape = synth.ModelShape(vocab=300, d_model=128, n_heads=4, block_len=4,
+                             n_block_layers=2, n_token_layers=2, prefix_len=1, dtype="fp32",
+                             n_kv_heads=hk)
+    gl, gn, ol = _run(shape, B=3, T=22, G=14)
+    assert np.abs(gl - ol).max() <= FP32_TOL
+
+
+@pytest.mark.parametrize("H,hk", [(4, 1), (4, 2), (2, 1)])
+def test_bf16_gqa_block_decoder(H, hk):
+    """d_head 64 and 128: tensor-core prefill attention and the decode
+    attention kernel read key/value head h / (H / H_kv)."""
+    shape = synth.ModelShape(vocab=1000, d_model=256, n_heads=H, block_len=4,
+                             n_block_layers=2, n_token_layers=2, prefix_len=1, n_kv_heads=hk)
+    gl, gn, ol = _run(shape, B=3, T=64, G=14)
+    for s in range(gl.shape[0]):
+        assert gh.rel_l2(gl[s], ol[s]) <= BF16_REL, (s, gh.rel_l2(gl[s], ol[s]))
