@@ -274,6 +274,7 @@ def run_ours(args):
     if prof:
         line["roofline"] = prof["dominant"]
         line["roofline_decode_attention"] = prof.get("attn_decode")
+        line["roofline_decode_attention_n300"] = prof.get("attn_decode_n300")
         line["roofline_decode_gemm"] = prof.get("gemm_decode")
         line["kernel_time_shares"] = prof["shares"]
         line["roofline"]["peak_source"] = peak_src
@@ -303,8 +304,8 @@ def run_ours(args):
 # the source is unchanged; after a change the traffic is null until it is
 # captured again.
 NCU_TRAFFIC = {
-    "token_step": {"bytes": 172.09e6, "source": "hierarchical_global_local_b200/csrc/decode_step.cu",
-                   "sha16": "fa7b915618c4d566"},
+    "token_step": {"bytes": 172.24e6, "source": "hierarchical_global_local_b200/csrc/decode_step.cu",
+                   "sha16": "3ad7db2bece3a80b"},
 }
 
 
@@ -362,6 +363,12 @@ def profile_step(model, prompts, gens, flush):
             c["flops"] += 2.0 * rc.m * rc.n * rc.k
         elif k == "attn_decode":
             c["bytes"] += rc.m * (2.0 * rc.n * rc.k * 2 + 2.0 * rc.k * 2)
+            if rc.n >= 300:
+                # launches over caches of >= 300 entries, on their own
+                cl = cls.setdefault("attn_decode_n300", {"ms": 0.0, "launches": 0, "bytes": 0.0, "flops": 0.0})
+                cl["ms"] += rc.ms
+                cl["launches"] += 1
+                cl["bytes"] += rc.m * (2.0 * rc.n * rc.k * 2 + 2.0 * rc.k * 2)
         elif k == "block_step":
             # block-decoder, prefix, token-decoder and LM-head weights (the
             # block KV read is not in the record and is left out)
@@ -372,6 +379,7 @@ def profile_step(model, prompts, gens, flush):
             # and the LM head, once per launch; activations stay in L2
             c["bytes"] += 2.0 * (Nt * 12 * rc.k * rc.k + rc.n * rc.k)
             c["flops"] += 2.0 * rc.m * (Nt * 12 * rc.k * rc.k + rc.n * rc.k)
+    long_attn = cls.pop("attn_decode_n300", None)
     total = sum(c["ms"] for c in cls.values())
     shares = {k: round(c["ms"] / total, 4) for k, c in sorted(cls.items(), key=lambda kv: -kv[1]["ms"])}
     dom_name = max(cls, key=lambda k: cls[k]["ms"])
@@ -396,6 +404,9 @@ def profile_step(model, prompts, gens, flush):
            "shares": shares}
     if "attn_decode" in cls:
         out["attn_decode"] = roof("attn_decode")
+    if long_attn is not None:
+        cls["attn_decode_n300"] = long_attn
+        out["attn_decode_n300"] = roof("attn_decode_n300")
     if "gemm_decode" in cls:
         out["gemm_decode"] = roof("gemm_decode")
     return out
@@ -629,6 +640,33 @@ def run_decode_case(args):
     model.close()
 
 
+def run_variants_case(args):
+    """A bounded case for profiler captures of the context-injection variants'
+    kernels: pythia160m-scale models with summation injection and with a
+    window of w = 3 context embeddings, batch 64, a 130-token prompt (two
+    trailing tokens inside the current block), then --case-steps greedy
+    decode calls each."""
+    import dataclasses
+    import torch
+    from hierarchical_global_local_b200.loader import build_model
+    torch.cuda.set_device(0)
+    base = synth.WORKLOADS[RUNS[1]]
+    for variant in ({"injection": "sum"}, {"context_window": 3}):
+        shape = dataclasses.replace(base.shape, **variant)
+        T = 130
+        model = build_model(shape, synth.make_weights(shape, seed=base.weight_seed), base.batch,
+                            T + args.case_steps + 1)
+        toks = synth.make_tokens(base, length=T)
+        out = torch.empty(args.case_steps + 1, base.batch, dtype=torch.int32, device="cuda")
+        model.prefill(torch.from_numpy(np.ascontiguousarray(toks)).cuda(), next_tokens=out[0])
+        for i in range(1, args.case_steps + 1):
+            model.decode(None, next_tokens=out[i])
+        model.sync()
+        model.close()
+        print(json.dumps({"case": "variants", "variant": variant, "prompt": T, "decode_calls": args.case_steps}),
+              flush=True)
+
+
 def run_prefill_case(args):
     """A bounded prefill-only case for profiler captures: --case-steps
     prefills of the prefill-heavy run (batch 64, prompt 2048)."""
@@ -745,7 +783,7 @@ def main():
     ap.add_argument("--ref-seconds", type=float, default=60.0,
                     help="--impl reference: oracle time budget over all warm-up and timed steps")
     ap.add_argument("--case", default=None, choices=["decode", "prefill", "decode_attention", "linear", "lb_sweep",
-                                                     "batch_sweep"],
+                                                     "batch_sweep", "variants"],
                     help="instead of the benchmark, run a bounded case for profiler captures: decode "
                          "calls of the decode-heavy workload, or one op of the path")
     ap.add_argument("--case-steps", type=int, default=None,
@@ -778,6 +816,9 @@ def main():
         return
     if args.case == "prefill":
         run_prefill_case(args)
+        return
+    if args.case == "variants":
+        run_variants_case(args)
         return
     if args.case in ("decode_attention", "linear"):
         run_kernel_case(args)
