@@ -371,10 +371,17 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
 #pragma unroll
           for (int j = 0; j < 32; ++j) tile[lane * 33 + j] = v[j];
           __syncwarp();
+          // the lane's column n is fixed over the block's 32 rows: the
+          // chunked epilogue issues a 16-row chunk's loads (bias, residual)
+          // before its stores
           const int n = b0 + c0 + lane;
-          for (int rr = 0; rr < 32; ++rr) {
-            const int m = a0 + warp * 32 + rr;
-            if (m < M && n < N) epi_apply<bf16>(e, m, n, tile[rr * 33 + lane]);
+          const int m0 = a0 + warp * 32;
+#pragma unroll
+          for (int rr0 = 0; rr0 < 32; rr0 += 16) {
+            float vv[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) vv[j] = tile[(rr0 + j) * 33 + lane];
+            if (n < N && m0 + rr0 < M) epi_cols<bf16, 16>(e, m0 + rr0, 16, n, M, vv, nullptr);
           }
           __syncwarp();
         }
