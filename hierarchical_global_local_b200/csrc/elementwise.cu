@@ -456,6 +456,14 @@ cudaError_t launch_rope_table(float2* tab, int n_pos, int rot, float base, cudaS
   return cudaGetLastError();
 }
 
+__device__ __forceinline__ uint2 pack_bf16x4_ew(float a, float b, float c, float d) {
+  __nv_bfloat162 lo = __floats2bfloat162_rn(a, b), hi = __floats2bfloat162_rn(c, d);
+  uint2 u;
+  u.x = *reinterpret_cast<uint32_t*>(&lo);
+  u.y = *reinterpret_cast<uint32_t*>(&hi);
+  return u;
+}
+
 template <typename T>
 __global__ void rope_append_kernel(const T* __restrict__ qkv, int D, int H, int Hk, int rot,
                                    const float2* __restrict__ tab, PosSpec ps,
@@ -489,6 +497,53 @@ __global__ void rope_append_kernel(const T* __restrict__ qkv, int D, int H, int 
       cache[(((size_t)b * Hk + hh) * cap + pos) * d + e] = from_f<T>(v);
       if (part == 2 && vt) vt[(((size_t)b * Hk + hh) * d + e) * vt_ld + pos] = from_f<T>(v);
     }
+  }
+}
+
+// The same in 16-byte pieces (bf16, d and rot / 2 multiples of 8): one
+// thread per 8 consecutive features of a row, so that part, head and
+// position are computed once per piece and every access is a 16-byte load
+// or store; the rotate-half partner of a piece inside the rotary span is the
+// aligned piece rot / 2 features away in the same head.
+__global__ void rope_append_vec_kernel(const bf16* __restrict__ qkv, int M, int D, int H, int Hk, int rot,
+                                       const float2* __restrict__ tab, PosSpec ps, bf16* __restrict__ q_out,
+                                       bf16* __restrict__ kc, bf16* __restrict__ vc, int cap) {
+  pdl_trigger();
+  pdl_wait();
+  const int d = D / H;
+  const int half = rot >> 1;
+  const int Dk = Hk * d, W = D + 2 * Dk;
+  const int pieces = W / 8;
+  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (long long)M * pieces) return;
+  const int m = (int)(idx / pieces);
+  const int x = (int)(idx - (long long)m * pieces) * 8;
+  const int b = m / ps.rows_per_seq;
+  const int pos = pos_base(ps, b) + (m - b * ps.rows_per_seq);
+  const bf16* row = qkv + (size_t)m * W;
+  const int part = x < D ? 0 : (x < D + Dk ? 1 : 2);
+  const int c = part == 0 ? x : (part == 1 ? x - D : x - D - Dk);
+  const int hh = c / d, e = c - hh * d;
+  float v[8];
+  unpack16(*reinterpret_cast<const uint4*>(row + x), v, (const bf16*)nullptr);
+  if (part < 2 && e < rot) {
+    const bool lo = e < half;
+    float pv[8];
+    unpack16(*reinterpret_cast<const uint4*>(row + (lo ? x + half : x - half)), pv, (const bf16*)nullptr);
+    const int i0 = lo ? e : e - half;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float2 cs = tab[(size_t)pos * half + i0 + j];
+      v[j] = lo ? v[j] * cs.x - pv[j] * cs.y : v[j] * cs.x + pv[j] * cs.y;
+    }
+  }
+  const uint2 lo4 = pack_bf16x4_ew(v[0], v[1], v[2], v[3]), hi4 = pack_bf16x4_ew(v[4], v[5], v[6], v[7]);
+  const uint4 out = make_uint4(lo4.x, lo4.y, hi4.x, hi4.y);
+  if (part == 0) {
+    *reinterpret_cast<uint4*>(q_out + (size_t)m * D + c) = out;
+  } else {
+    bf16* cache = part == 1 ? kc : vc;
+    *reinterpret_cast<uint4*>(cache + (((size_t)b * Hk + hh) * cap + pos) * d + e) = out;
   }
 }
 
@@ -531,7 +586,12 @@ cudaError_t launch_rope_append(int dt, const void* qkv, int M, int D, int H, int
   if (H % Hk) return cudaErrorInvalidValue;
   // V^T is written for positions known on the host (prefill) only
   if (vt && pos.mode != POS_ZERO) return cudaErrorInvalidValue;
-  if (dt == DT_BF16) {
+  const int dh = D / H;
+  if (dt == DT_BF16 && dh % 8 == 0 && (rot / 2) % 8 == 0) {
+    const long long n = (long long)M * ((D + 2 * Hk * dh) / 8);
+    BT_LAUNCH(rope_append_vec_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, (const bf16*)qkv, M, D, H,
+              Hk, rot, rope_tab, pos, (bf16*)q_out, (bf16*)k_cache, (bf16*)v_cache, cap);
+  } else if (dt == DT_BF16) {
     BT_LAUNCH(rope_append_kernel<bf16>, dim3(M), dim3(256), 0, s, (const bf16*)qkv, D, H, Hk, rot, rope_tab, pos,
                                                (bf16*)q_out, (bf16*)k_cache, (bf16*)v_cache, cap, (bf16*)nullptr, 0);
   }
