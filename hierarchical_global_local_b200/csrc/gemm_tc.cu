@@ -40,7 +40,18 @@ constexpr size_t PART_BUDGET = 256;  // split-K reduces in distributed shared me
 
 constexpr int MAX_STAGES = 8;
 constexpr int MAX_KS = 16;  // K splits of one tile: CTAs of one (non-portable) cluster
-constexpr int THREADS = 192;  // warps 0-3 epilogue, warp 4 TMA producer, warp 5 MMA issuer
+// Warp roles: EPI epilogue warps, then the TMA producer warp and the MMA
+// issuer warp. The activations-as-A orientation (prefill) runs eight
+// epilogue warps: two per quarter of the TMEM lanes, each taking half of the
+// tile's columns (its epilogue -- GELU and stores of every output -- is the
+// bound there, not the tensor pipe); weights-as-A (decode) runs four.
+template <bool SWAP>
+struct Roles {
+  static constexpr int EPI = SWAP ? 4 : 8;
+  static constexpr int THREADS = EPI * 32 + 64;
+  static constexpr int PRODUCER = EPI, MMA = EPI + 1;
+};
+constexpr int THREADS = Roles<true>::THREADS;  // decode orientation (split-K planning)
 
 template <int BN>
 __host__ __device__ constexpr size_t stage_bytes() {
@@ -142,7 +153,7 @@ __device__ void post_ln(const Epi& e, int m_lo, int m_hi, int M, int N, int nfea
 // ks > 1: one tile per CTA, K split over the cluster's ks CTAs, partial
 //   tiles reduce-scattered over distributed shared memory.
 template <int BN, bool SWAP>
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__(Roles<SWAP>::THREADS, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
                int M, int N, int nkb, int ks, int stages, int ntA, int ntB, int xk_split,
                int xk_off, Epi e, int* status) {
@@ -172,7 +183,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_empty[i], 128);
+      mbar_init(&acc_empty[i], Roles<SWAP>::EPI * 32);
     }
     fence_mbar_init();
   }
@@ -188,7 +199,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
   if (ks > 1) tc::cluster_arrive_relaxed();
 
   pdl_trigger();
-  if (warp == 4) {
+  if (warp == Roles<SWAP>::PRODUCER) {
     // ---- TMA producer ----
     if (lane == 0) {
       const uint32_t bytes = (uint32_t)stage_bytes<BN>();
@@ -232,7 +243,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
         load_x(it, s);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == Roles<SWAP>::MMA) {
     // ---- MMA issuer ----
     pdl_wait();
     if (lane == 0) {
@@ -258,10 +269,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
       }
     }
   } else {
-    // ---- epilogue warps 0-3: TMEM lanes 32w..32w+31 ----
+    // ---- epilogue warps: TMEM lanes 32 (w % 4) .. 32 (w % 4) + 31 ----
     pdl_wait();  // outputs may still be read by earlier kernels
-    const int r = warp * 32 + lane;  // row of A = TMEM lane
-    const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+    const int quarter = warp & 3;     // TMEM lane quarter
+    const int r = quarter * 32 + lane;  // row of A = TMEM lane
+    const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
     // fused rotary: the rotate-half partner of feature f is f ^ (rot/2), held
     // by lane ^ (rot/2) of the same warp (heads are 32-feature aligned)
     const bool rope = SWAP && e.kind == EPI_QKV1_ROPE;
@@ -364,7 +376,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
         // through this warp's shared-memory tile so that one store
         // instruction covers 32 consecutive output columns of one row
         float* tile = reinterpret_cast<float*>(smem + (size_t)stages * stage_bytes<BN>()) + warp * 32 * 33;
-        for (int c0 = 0; c0 < BN; c0 += 32) {
+        // the two warps of a lane quarter take the two halves of the columns
+        constexpr int CW = BN / (Roles<SWAP>::EPI / 4);
+        const int cbeg = (warp >> 2) * CW;
+        for (int c0 = cbeg; c0 < cbeg + CW; c0 += 32) {
           float v[32];
           tc::tmem_ld16(tb + c0, v);
           tc::tmem_ld16(tb + c0 + 16, v + 16);
@@ -375,7 +390,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
           // chunked epilogue issues a 16-row chunk's loads (bias, residual)
           // before its stores
           const int n = b0 + c0 + lane;
-          const int m0 = a0 + warp * 32;
+          const int m0 = a0 + quarter * 32;
 #pragma unroll
           for (int rr0 = 0; rr0 < 32; rr0 += 16) {
             float vv[16];
@@ -414,10 +429,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
     // memory after the barrier, so no second barrier is needed.
     namespace cg = cooperative_groups;
     cg::cluster_group cluster = cg::this_cluster();
-    if (warp >= 4) tc::cluster_wait_acquire();  // producer / MMA warps: first phase
+    if (warp >= Roles<SWAP>::EPI) tc::cluster_wait_acquire();  // producer / MMA warps: first phase
     tc::cluster_arrive_release();               // second phase: all pushes done
     tc::cluster_wait_acquire();
-    if (warp < 4) {
+    if (warp < Roles<SWAP>::EPI) {
       const int r = warp * 32 + lane;
       const bool rope = SWAP && e.kind == EPI_QKV1_ROPE;
       const int rhalf = e.rot >> 1;
@@ -551,7 +566,7 @@ size_t launch_smem(int nkb, int ks, int* stages_out) {
     if (stages > fit) stages = fit;
   }
   // activations as A: per-warp 32 x 33 fp32 transpose tiles for the epilogue
-  const size_t tr_bytes = SWAP ? 0 : (size_t)4 * 32 * 33 * 4;
+  const size_t tr_bytes = SWAP ? 0 : (size_t)Roles<SWAP>::EPI * 32 * 33 * 4;
   if (!SWAP) {
     int fit = (int)((SMEM_MAX - 1024 - tr_bytes) / SB);
     if (stages > fit) stages = fit;
@@ -574,7 +589,7 @@ int resident_ctas(int ks, size_t smem) {
     if (cache[i].dev == dev && cache[i].ks == ks && cache[i].smem == smem) return cache[i].ctas;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(1, 1, ks);
-  cfg.blockDim = dim3(THREADS, 1, 1);
+  cfg.blockDim = dim3(Roles<SWAP>::THREADS, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -623,14 +638,14 @@ cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& mb, int M, int 
     grid = dim3(ntiles, 1, ks);
   } else {
     int per_sm = 0;
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gemm_tc_kernel<BN, SWAP>, THREADS, smem);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gemm_tc_kernel<BN, SWAP>, Roles<SWAP>::THREADS, smem);
     if (per_sm < 1) per_sm = 1;
     const int slots = sm_count() * per_sm;
     grid = dim3(ntiles < slots ? ntiles : slots, 1, 1);
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
-  cfg.blockDim = dim3(THREADS, 1, 1);
+  cfg.blockDim = dim3(Roles<SWAP>::THREADS, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[2];
