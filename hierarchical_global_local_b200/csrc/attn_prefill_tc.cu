@@ -45,12 +45,22 @@ struct Plan {
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
   static constexpr int OFF_VT = OFF_K + STAGES * K_BYTES;
   static constexpr int OFF_P = OFF_VT + STAGES * VT_BYTES;
-  static constexpr int BYTES = OFF_P + P_BYTES + 1024;  // + alignment slack
+  static constexpr int OFF_BAR = OFF_P + P_BYTES;     // mbarriers and the TMEM slot
+  static constexpr int BAR_BYTES = 128;
+  // CTAs per SM: two for d_head 64 (their shared memory, with the 1 KB the
+  // system keeps per block, fits the SM's 228 KB only without static shared
+  // variables -- hence the barriers in the dynamic allocation), else one
+  static constexpr int CTAS = DH == 64 ? 2 : 1;
+  static constexpr int LIMIT = 233472 / CTAS - 1024;
+  static constexpr int NEED = OFF_BAR + BAR_BYTES;
+  static constexpr int BYTES = NEED + 1024 < LIMIT ? NEED + 1024 : LIMIT;
+  static constexpr int SLACK = BYTES - NEED;           // room for aligning the base to 1024
   static constexpr int TMEM_COLS = 256;               // S: 128 columns, O: DH columns
+  static_assert(SLACK >= 0, "shared-memory plan");
 };
 
 template <int DH>
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__(THREADS, Plan<DH>::CTAS)
 attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
                        const __grid_constant__ CUtensorMap mVt, int H, int n, bf16* __restrict__ out,
                        int ld_out, float scale_log2, int* status, int g) {
@@ -58,8 +68,21 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
   pdl_trigger();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-  __shared__ __align__(8) uint64_t q_full, kv_full[PL::STAGES], kv_empty[PL::STAGES], s_full, p_full, o_full;
-  __shared__ uint32_t tmem_slot;
+  // the plan leaves SLACK bytes for aligning the base; a base further off
+  // (none in practice: the kernel has no static shared variables) is
+  // reported instead of overrunning the allocation
+  if ((size_t)(sm - smem_raw) > (size_t)PL::SLACK) {
+    if (threadIdx.x == 0) set_status(status, ST_BAD_ARGS);
+    return;
+  }
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + PL::OFF_BAR);
+  uint64_t* q_full = bars;
+  uint64_t* kv_full = bars + 1;
+  uint64_t* kv_empty = bars + 1 + PL::STAGES;
+  uint64_t* s_full = bars + 1 + 2 * PL::STAGES;
+  uint64_t* p_full = s_full + 1;
+  uint64_t* o_full = s_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_full + 3);
 
   const int nqt = (n + QT - 1) / QT;
   const int qt = blockIdx.x % nqt;
@@ -71,32 +94,32 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    mbar_init(&q_full, 1);
+    mbar_init(q_full, 1);
     for (int s = 0; s < PL::STAGES; ++s) {
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], 1);
     }
-    mbar_init(&s_full, 1);
-    mbar_init(&p_full, 128);
-    mbar_init(&o_full, 1);
+    mbar_init(s_full, 1);
+    mbar_init(p_full, 128);
+    mbar_init(o_full, 1);
     fence_mbar_init();
   }
   if (warp == 0) {
-    tc::tmem_alloc(&tmem_slot, PL::TMEM_COLS);
+    tc::tmem_alloc(tmem_slot, PL::TMEM_COLS);
   }
   tc::fence_before();
   __syncthreads();
   tc::fence_after();
-  const uint32_t tmem = tmem_slot;
+  const uint32_t tmem = *tmem_slot;
   const uint32_t tS = tmem, tO = tmem + KT;
   pdl_wait();
 
   if (warp == 4) {
     if (lane == 0) {
       // Q tile (KB blocks of 64 dims), then K / V^T tiles through the ring
-      mbar_arrive_expect_tx(&q_full, PL::Q_BYTES);
+      mbar_arrive_expect_tx(q_full, PL::Q_BYTES);
       for (int kb = 0; kb < PL::KB; ++kb)
-        tc::tma_load_3d(sm + PL::OFF_Q + kb * QT * 128, &mQ, h * DH + kb * 64, q0, b, &q_full);
+        tc::tma_load_3d(sm + PL::OFF_Q + kb * QT * 128, &mQ, h * DH + kb * 64, q0, b, q_full);
       for (int j = 0; j < ntiles; ++j) {
         const int s = j % PL::STAGES;
         if (j >= PL::STAGES) mbar_wait_bounded(&kv_empty[s], ((j / PL::STAGES) + 1) & 1, status);
@@ -111,7 +134,7 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
   } else if (warp == 5) {
     if (lane == 0) {
       constexpr uint32_t idS = tc::idesc_bf16_m128(KT), idO = tc::idesc_bf16_m128(DH);
-      mbar_wait_bounded(&q_full, 0, status);
+      mbar_wait_bounded(q_full, 0, status);
       for (int j = 0; j < ntiles; ++j) {
         const int s = j % PL::STAGES;
         // (S of tile j-1 was consumed before P of tile j-1 was published,
@@ -125,17 +148,19 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) tc::mma_bf16(tS, dq + 2 * kk, dk + 2 * kk, idS, (kb | kk) ? 1u : 0u);
         }
-        tc::commit(&s_full);
-        // O_j = P V over the 128 keys (2 blocks x 4 slices of 16), once P is written
-        mbar_wait_bounded(&p_full, j & 1, status);
+        tc::commit(s_full);
+        // O += P_j V_j over the 128 keys (2 blocks x 4 slices of 16), once P is
+        // written (and O rescaled where the running max moved); O accumulates
+        // in TMEM across the key tiles
+        mbar_wait_bounded(p_full, j & 1, status);
         tc::fence_after();
         for (int kb = 0; kb < KT / 64; ++kb) {
           const uint64_t dp = tc::desc_sw128(smem_u32(sm + PL::OFF_P + kb * QT * 128));
           const uint64_t dv = tc::desc_sw128(smem_u32(sm + PL::OFF_VT + s * PL::VT_BYTES + kb * DH * 128));
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) tc::mma_bf16(tO, dp + 2 * kk, dv + 2 * kk, idO, (kb | kk) ? 1u : 0u);
+          for (int kk = 0; kk < 4; ++kk) tc::mma_bf16(tO, dp + 2 * kk, dv + 2 * kk, idO, (j | kb | kk) ? 1u : 0u);
         }
-        tc::commit(&o_full);
+        tc::commit(o_full);
         tc::commit(&kv_empty[s]);
       }
     }
@@ -145,12 +170,9 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
     const int qi = q0 + r;
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
     float m = -INFINITY, l = 0.f;
-    float o[DH];
-#pragma unroll
-    for (int e = 0; e < DH; ++e) o[e] = 0.f;
     uint8_t* prow = sm + PL::OFF_P;
     for (int j = 0; j < ntiles; ++j) {
-      mbar_wait_bounded(&s_full, j & 1, status);
+      mbar_wait_bounded(s_full, j & 1, status);
       tc::fence_after();
       const int k0 = j * KT;
       // pass 1: row max over this tile (masked keys excluded), 32 columns at a time
@@ -166,7 +188,25 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
         }
       }
       const float mn = fmaxf(m, tmax);
-      const float corr = (mn == -INFINITY) ? 1.f : exp2f(m - mn);
+      const float corr = (mn == -INFINITY || m == -INFINITY) ? 1.f : exp2f(m - mn);
+      if (j > 0) {
+        // O holds sum_{i<j} P_i V_i at the old maxima: once P_{j-1} V_{j-1}
+        // is in, rescale the rows whose maximum moved (warp-uniform: the
+        // TMEM accesses are warp-collective), before P_j V_j accumulates
+        mbar_wait_bounded(o_full, (j - 1) & 1, status);
+        tc::fence_after();
+        if (__any_sync(0xffffffffu, corr != 1.f)) {
+#pragma unroll
+          for (int c = 0; c < DH; c += 16) {
+            float ov[16];
+            tc::tmem_ld16(tO + lane_base + c, ov);
+#pragma unroll
+            for (int u = 0; u < 16; ++u) ov[u] *= corr;
+            tc::tmem_st16(tO + lane_base + c, ov);
+          }
+          tc::tmem_wait_st();
+        }
+      }
       // pass 2: P = exp2(s - mn) as bf16 into the swizzled K-major tile
       float lt = 0.f;
 #pragma unroll
@@ -195,33 +235,31 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
       }
       fence_proxy_async();  // P visible to the tensor core
       tc::fence_before();
-      mbar_arrive(&p_full);
-      // accumulate O_j with the rescale
-      mbar_wait_bounded(&o_full, j & 1, status);
-      tc::fence_after();
-#pragma unroll
-      for (int c = 0; c < DH; c += 32) {
-        float ov[32];
-        tc::tmem_ld32(tO + lane_base + c, ov);
-#pragma unroll
-        for (int u = 0; u < 32; ++u) o[c + u] = o[c + u] * corr + ov[u];
-      }
+      mbar_arrive(p_full);
       l = l * corr + lt;
       m = mn;
     }
-    if (qi < n) {
-      const float inv = 1.f / l;
-      bf16* dst = out + ((size_t)b * n + qi) * ld_out + h * DH;
+    // the last P V is in: O / l, read from TMEM 16 columns at a time
+    mbar_wait_bounded(o_full, (ntiles - 1) & 1, status);
+    tc::fence_after();
+    const float inv = (qi < n && l > 0.f) ? 1.f / l : 0.f;
+    bf16* dst = out + ((size_t)b * n + qi) * ld_out + h * DH;
 #pragma unroll
-      for (int e = 0; e < DH; e += 8) {
-        __nv_bfloat162 h0 = __floats2bfloat162_rn(o[e] * inv, o[e + 1] * inv);
-        __nv_bfloat162 h1 = __floats2bfloat162_rn(o[e + 2] * inv, o[e + 3] * inv);
-        __nv_bfloat162 h2 = __floats2bfloat162_rn(o[e + 4] * inv, o[e + 5] * inv);
-        __nv_bfloat162 h3 = __floats2bfloat162_rn(o[e + 6] * inv, o[e + 7] * inv);
-        uint4 w;
-        w.x = *reinterpret_cast<uint32_t*>(&h0); w.y = *reinterpret_cast<uint32_t*>(&h1);
-        w.z = *reinterpret_cast<uint32_t*>(&h2); w.w = *reinterpret_cast<uint32_t*>(&h3);
-        *reinterpret_cast<uint4*>(dst + e) = w;
+    for (int c = 0; c < DH; c += 16) {
+      float ov[16];
+      tc::tmem_ld16(tO + lane_base + c, ov);
+      if (qi < n) {
+#pragma unroll
+        for (int e = 0; e < 16; e += 8) {
+          __nv_bfloat162 h0 = __floats2bfloat162_rn(ov[e] * inv, ov[e + 1] * inv);
+          __nv_bfloat162 h1 = __floats2bfloat162_rn(ov[e + 2] * inv, ov[e + 3] * inv);
+          __nv_bfloat162 h2 = __floats2bfloat162_rn(ov[e + 4] * inv, ov[e + 5] * inv);
+          __nv_bfloat162 h3 = __floats2bfloat162_rn(ov[e + 6] * inv, ov[e + 7] * inv);
+          uint4 w;
+          w.x = *reinterpret_cast<uint32_t*>(&h0); w.y = *reinterpret_cast<uint32_t*>(&h1);
+          w.z = *reinterpret_cast<uint32_t*>(&h2); w.w = *reinterpret_cast<uint32_t*>(&h3);
+          *reinterpret_cast<uint4*>(dst + c + e) = w;
+        }
       }
     }
   }
