@@ -84,9 +84,13 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
   uint64_t* o_full = s_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_full + 3);
 
+  // longest first: CTAs are numbered q-tile-major from the last (causal)
+  // q-tile down, so the tiles with the most key tiles start first and the
+  // one-key-tile ones fill the tail
   const int nqt = (n + QT - 1) / QT;
-  const int qt = blockIdx.x % nqt;
-  const int bh = blockIdx.x / nqt;  // b * H + h
+  const int BH = gridDim.x / nqt;
+  const int qt = nqt - 1 - (int)(blockIdx.x / BH);
+  const int bh = blockIdx.x % BH;  // b * H + h
   const int b = bh / H, h = bh - b * H;
   const int kvh = b * (H / g) + h / g;  // key/value head (grouped-query attention)
   const int q0 = qt * QT;
