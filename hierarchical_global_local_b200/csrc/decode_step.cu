@@ -73,11 +73,13 @@ constexpr int WORKERS = 128;                 // warps 0-3 (TMEM lanes 0-127)
 constexpr int THREADS = WORKERS + 64;        // warp 4: TMA producer, warp 5: MMA issuer
 constexpr int TILE_BYTES = 128 * 64 * 2;     // one weight box: 128 rows x 64 K (bf16)
 constexpr int MAX_STAGES = 12;
-// K splits: as many as fill the SMs up to these caps (fewer splits mean
-// fewer partial sums for the reduction phases; measured on B200 at D = 768:
-// 2 and 12 beat 3 / 15 and 1 / 12)
+// K splits: as many as fill the SMs up to these caps. q|k|v|fc1: fewer
+// splits mean fewer partial sums for the reduction phase (measured on B200
+// at D = 768: 2 beats 1 and 3). [W_o | W_2]: the token layers add their
+// splits into h with L2 reductions, so more splits only add reductions
+// (D = 768: 20 splits 170.5 us per token step, 15: 174.4, 12: 174.7).
 constexpr int MAX_S1 = 2;                    // K splits of the q|k|v|fc1 GEMM
-constexpr int MAX_S2 = 12;                   // K splits of the [W_o | W_2] GEMM
+constexpr int MAX_S2 = 24;                   // K splits of the [W_o | W_2] GEMM
 constexpr int MAX_B = 64;
 constexpr int MAX_WIN = 8;                   // local-window slots (P + L_B - 1)
 constexpr int TMEM_COLS = 128;               // two accumulators of up to 64 columns
@@ -327,6 +329,24 @@ __device__ void store_partial(uint32_t tbuf, float* part, int u, int B, int Bp) 
   }
 }
 
+// The same accumulator added into the fp32 rows h [B][D] (features
+// t*128 .. t*128+127) with L2 reductions: the K splits' sum lands in h
+// directly, so the phase after the next grid barrier reads one value per
+// element instead of one per split. The order of the splits' additions
+// varies from run to run (fp32 rounding only).
+__device__ void red_partial(uint32_t tbuf, float* h, int t, int B, int Bp, int D) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t trow = tbuf + ((uint32_t)(warp * 32) << 16);
+  float* dst = h + (size_t)t * 128 + warp * 32 + lane;
+  for (int c0 = 0; c0 < Bp; c0 += 16) {
+    float v[16];
+    tc::tmem_ld16(trow + c0, v);
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      if (c0 + j < B) atomicAdd(dst + (size_t)(c0 + j) * D, v[j]);
+  }
+}
+
 // Shared-memory barriers of the worker / MMA hand-off.
 struct Sync {
   uint64_t* full;       // [stages] weight tile landed
@@ -343,7 +363,7 @@ struct Sync {
 template <typename ColOf>
 __device__ void gemm_phase(const Plan& P, int T, int S, int nkb, const CUtensorMap* map, ColOf col_of,
                            int B, float* part, uint8_t* act, uint32_t tmem, const Sync& y, int& na,
-                           int& nu, int* status) {
+                           int& nu, int* status, float* red_h = nullptr, int D = 0) {
   for (int u = blockIdx.x; u < T * S; u += gridDim.x) {
     const int t = u % T, sp = u / T;
     // act is free: the previous unit's MMAs (its last readers) completed
@@ -353,7 +373,8 @@ __device__ void gemm_phase(const Plan& P, int T, int S, int nkb, const CUtensorM
     const int buf = nu & 1;
     mbar_wait_bounded(&y.acc_full[buf], (nu >> 1) & 1, status);
     tc::fence_after();
-    store_partial(tmem + (uint32_t)(buf * 64), part, u, B, P.Bp);
+    if (red_h) red_partial(tmem + (uint32_t)(buf * 64), red_h, t, B, P.Bp, D);
+    else store_partial(tmem + (uint32_t)(buf * 64), part, u, B, P.Bp);
     tc::fence_before();
     mbar_arrive(&y.acc_empty[buf]);
     ++nu;
@@ -565,8 +586,9 @@ __device__ void gelu_fc1(const TokenStepArgs& a, const Plan& P, const float* bq)
   }
 }
 
-// R2: h += sum of the K splits + (b_o + b_2); LayerNorm of the new row for
-// layer l + 1 (LN1 | LN2 -> x1) or the final LayerNorm (-> xf).
+// R2: h += (b_o + b_2) -- the out|fc2 units already added their K splits'
+// products into h -- then the LayerNorm of the new row for layer l + 1
+// (LN1 | LN2 -> x1) or the final LayerNorm (-> xf).
 __device__ void r2_phase(const TokenStepArgs& a, const Plan& P, int l, float* red) {
   const int D = a.D, B = a.B;
   const float* bo = layer_ptr(a.b_o2, l, a.layer_stride);
@@ -587,14 +609,8 @@ __device__ void r2_phase(const TokenStepArgs& a, const Plan& P, int l, float* re
       const int f = (threadIdx.x + u * WORKERS) * 4;
       hv[u] = make_float4(0.f, 0.f, 0.f, 0.f);
       if (f < D) {
-        float4 acc = f4add(__ldcg(reinterpret_cast<const float4*>(hrow + f)),
-                           *reinterpret_cast<const float4*>(bo + f));
-        const int t = f >> 7, off = f & 127;
-#pragma unroll
-        for (int s = 0; s < MAX_S2; ++s)
-          if (s < P.S2)
-            acc = f4add(acc, __ldcg(reinterpret_cast<const float4*>(
-                                 a.p2 + ((size_t)(s * P.T2 + t) * B + b) * 128 + off)));
+        const float4 acc = f4add(__ldcg(reinterpret_cast<const float4*>(hrow + f)),
+                                 *reinterpret_cast<const float4*>(bo + f));
         hv[u] = acc;
         __stcg(reinterpret_cast<float4*>(hrow + f), acc);
       }
@@ -1110,16 +1126,17 @@ token_step_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
         if (!(ok = grid_sync(a, ++nb * G, &s_abort))) break;
         block_attention_phase(a, P, l, bpos, act, att_bar, q_s, katt);
         if (!(ok = grid_sync(a, ++nb * G, &s_abort))) break;
+        // the out|fc2 splits go into the block residual rows by L2 reductions
         gemm_phase(P, P.T2, P.S2, P.nkb2, &ma2, [](int) { return 0; }, a.B, a.p2, act, tmem, y, na, nu,
-                   a.status);
+                   a.status, a.h_b, D);
         if (!(ok = grid_sync(a, ++nb * G, &s_abort))) break;
         if (l + 1 < Nb)
-          reduce_ln(a, P, a.h_b, layer_ptr(a.bb_o2, l, a.layer_stride), P.S2, true,
+          reduce_ln(a, P, a.h_b, layer_ptr(a.bb_o2, l, a.layer_stride), 0, true,
                     layer_ptr(a.bln1_g, l + 1, a.layer_stride), layer_ptr(a.bln1_b, l + 1, a.layer_stride),
                     layer_ptr(a.bln2_g, l + 1, a.layer_stride), layer_ptr(a.bln2_b, l + 1, a.layer_stride),
                     a.x1, red);
         else
-          reduce_ln(a, P, a.h_b, layer_ptr(a.bb_o2, l, a.layer_stride), P.S2, true, a.lnb_g, a.lnb_b,
+          reduce_ln(a, P, a.h_b, layer_ptr(a.bb_o2, l, a.layer_stride), 0, true, a.lnb_g, a.lnb_b,
                     nullptr, nullptr, a.xf, red);
         ok = grid_sync(a, ++nb * G, &s_abort);
       }
@@ -1144,7 +1161,7 @@ token_step_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
       r1_phase(a, P, l, pos);
       if (!(ok = grid_sync(a, ++nb * G, &s_abort))) break;
       gemm_phase(P, P.T2, P.S2, P.nkb2, &ma2, [](int) { return 0; }, a.B, a.p2, act, tmem, y, na, nu,
-                 a.status);
+                 a.status, a.h, D);
       if (!(ok = grid_sync(a, ++nb * G, &s_abort))) break;
       r2_phase(a, P, l, red);
       ok = grid_sync(a, ++nb * G, &s_abort);
