@@ -329,22 +329,39 @@ __device__ void store_partial(uint32_t tbuf, float* part, int u, int B, int Bp) 
   }
 }
 
-// The same accumulator added into the fp32 rows h [B][D] (features
-// t*128 .. t*128+127) with L2 reductions: the K splits' sum lands in h
-// directly, so the phase after the next grid barrier reads one value per
-// element instead of one per split. The order of the splits' additions
-// varies from run to run (fp32 rounding only).
-__device__ void red_partial(uint32_t tbuf, float* h, int t, int B, int Bp, int D) {
+// Fixed-point scale of the split-K sums: a partial v is added as the
+// 64-bit integer round(v * 2^32). Integer addition is associative, so the
+// sum does not depend on the order in which the splits arrive, and the
+// result is the same bit for bit from run to run (which fp32 additions in
+// arrival order are not). Resolution 2^-32; |sums| below 2^31.
+constexpr float FX_ONE = 4294967296.0f;            // 2^32
+constexpr float FX_INV = 2.3283064365386963e-10f;  // 2^-32
+
+// The same accumulator added into the int64 accumulators fx [B][D]
+// (features t*128 .. t*128+127) with L2 reductions: the phase after the
+// next grid barrier reads one value per element instead of one per split,
+// and stores zero back.
+__device__ void red_partial(uint32_t tbuf, long long* fx, int t, int B, int Bp, int D) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t trow = tbuf + ((uint32_t)(warp * 32) << 16);
-  float* dst = h + (size_t)t * 128 + warp * 32 + lane;
+  unsigned long long* dst = reinterpret_cast<unsigned long long*>(fx) + (size_t)t * 128 + warp * 32 + lane;
   for (int c0 = 0; c0 < Bp; c0 += 16) {
     float v[16];
     tc::tmem_ld16(trow + c0, v);
 #pragma unroll
     for (int j = 0; j < 16; ++j)
-      if (c0 + j < B) atomicAdd(dst + (size_t)(c0 + j) * D, v[j]);
+      if (c0 + j < B) atomicAdd(dst + (size_t)(c0 + j) * D, (unsigned long long)__float2ll_rn(v[j] * FX_ONE));
   }
+}
+
+// four consecutive fixed-point sums as floats; the accumulators are cleared
+__device__ __forceinline__ float4 fx_take4(long long* p) {
+  longlong2* q = reinterpret_cast<longlong2*>(p);
+  const longlong2 a = __ldcg(q), b = __ldcg(q + 1);
+  __stcg(q, make_longlong2(0, 0));
+  __stcg(q + 1, make_longlong2(0, 0));
+  return make_float4(__ll2float_rn(a.x) * FX_INV, __ll2float_rn(a.y) * FX_INV, __ll2float_rn(b.x) * FX_INV,
+                     __ll2float_rn(b.y) * FX_INV);
 }
 
 // Shared-memory barriers of the worker / MMA hand-off.
@@ -363,7 +380,7 @@ struct Sync {
 template <typename ColOf>
 __device__ void gemm_phase(const Plan& P, int T, int S, int nkb, const CUtensorMap* map, ColOf col_of,
                            int B, float* part, uint8_t* act, uint32_t tmem, const Sync& y, int& na,
-                           int& nu, int* status, float* red_h = nullptr, int D = 0) {
+                           int& nu, int* status, long long* red_fx = nullptr, int D = 0) {
   for (int u = blockIdx.x; u < T * S; u += gridDim.x) {
     const int t = u % T, sp = u / T;
     // act is free: the previous unit's MMAs (its last readers) completed
@@ -373,7 +390,7 @@ __device__ void gemm_phase(const Plan& P, int T, int S, int nkb, const CUtensorM
     const int buf = nu & 1;
     mbar_wait_bounded(&y.acc_full[buf], (nu >> 1) & 1, status);
     tc::fence_after();
-    if (red_h) red_partial(tmem + (uint32_t)(buf * 64), red_h, t, B, P.Bp, D);
+    if (red_fx) red_partial(tmem + (uint32_t)(buf * 64), red_fx, t, B, P.Bp, D);
     else store_partial(tmem + (uint32_t)(buf * 64), part, u, B, P.Bp);
     tc::fence_before();
     mbar_arrive(&y.acc_empty[buf]);
@@ -530,7 +547,7 @@ __device__ void attend_item(const TokenStepArgs& a, const Plan& P, const float* 
 __device__ void gelu_fc1(const TokenStepArgs& a, const Plan& P, const float* bq);
 
 __device__ void r1_phase(const TokenStepArgs& a, const Plan& P, int l, int pos) {
-  const int D = a.D, B = a.B;
+  const int B = a.B;
   const float* bq = layer_ptr(a.b_qkv1, l, a.layer_stride);
   bf16* kc = a.kt + (size_t)l * a.kt_layer;
   bf16* vc = a.vt + (size_t)l * a.kt_layer;
@@ -586,8 +603,8 @@ __device__ void gelu_fc1(const TokenStepArgs& a, const Plan& P, const float* bq)
   }
 }
 
-// R2: h += (b_o + b_2) -- the out|fc2 units already added their K splits'
-// products into h -- then the LayerNorm of the new row for layer l + 1
+// R2: h += (the out|fc2 units' K-split sum, from the fixed-point
+// accumulators) + (b_o + b_2), then the LayerNorm of the new row for layer l + 1
 // (LN1 | LN2 -> x1) or the final LayerNorm (-> xf).
 __device__ void r2_phase(const TokenStepArgs& a, const Plan& P, int l, float* red) {
   const int D = a.D, B = a.B;
@@ -604,12 +621,13 @@ __device__ void r2_phase(const TokenStepArgs& a, const Plan& P, int l, float* re
   for (int b = blockIdx.x; b < B; b += gridDim.x) {
     float4 hv[4];
     float* hrow = a.h + (size_t)b * D;
+    long long* frow = a.fx + (size_t)b * D;
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int f = (threadIdx.x + u * WORKERS) * 4;
       hv[u] = make_float4(0.f, 0.f, 0.f, 0.f);
       if (f < D) {
-        const float4 acc = f4add(__ldcg(reinterpret_cast<const float4*>(hrow + f)),
+        const float4 acc = f4add(f4add(__ldcg(reinterpret_cast<const float4*>(hrow + f)), fx_take4(frow + f)),
                                  *reinterpret_cast<const float4*>(bo + f));
         hv[u] = acc;
         __stcg(reinterpret_cast<float4*>(hrow + f), acc);
@@ -664,7 +682,8 @@ __device__ void ingest_phase(const TokenStepArgs& a, int jb, float* red) {
 }
 
 // Row reduction for the out|fc2 and prefix GEMMs: h[b] = (residual ? h[b] : 0)
-// + bias + the S K-split partials (T tiles), then a LayerNorm of the new row:
+// + bias + the S K-split partials (T tiles) or, with S = 0, the fixed-point
+// sums in a.fx (cleared as they are read), then a LayerNorm of the new row:
 // LN1 | LN2 -> out (row stride 2D) when lp holds two, else one LN -> out
 // (row stride D). One CTA per row.
 __device__ void reduce_ln(const TokenStepArgs& a, const Plan& P, float* h, const float* bias, int S,
@@ -683,6 +702,7 @@ __device__ void reduce_ln(const TokenStepArgs& a, const Plan& P, float* h, const
       if (f < D) {
         float4 acc = *reinterpret_cast<const float4*>(bias + f);
         if (residual) acc = f4add(acc, __ldcg(reinterpret_cast<const float4*>(hrow + f)));
+        if (S == 0) acc = f4add(acc, fx_take4(a.fx + (size_t)b * D + f));
         const int t = f >> 7, off = f & 127;
 #pragma unroll
         for (int sp = 0; sp < MAX_S2; ++sp)
@@ -1126,9 +1146,9 @@ token_step_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
         if (!(ok = grid_sync(a, ++nb * G, &s_abort))) break;
         block_attention_phase(a, P, l, bpos, act, att_bar, q_s, katt);
         if (!(ok = grid_sync(a, ++nb * G, &s_abort))) break;
-        // the out|fc2 splits go into the block residual rows by L2 reductions
+        // the out|fc2 splits go into the fixed-point accumulators by L2 reductions
         gemm_phase(P, P.T2, P.S2, P.nkb2, &ma2, [](int) { return 0; }, a.B, a.p2, act, tmem, y, na, nu,
-                   a.status, a.h_b, D);
+                   a.status, a.fx, D);
         if (!(ok = grid_sync(a, ++nb * G, &s_abort))) break;
         if (l + 1 < Nb)
           reduce_ln(a, P, a.h_b, layer_ptr(a.bb_o2, l, a.layer_stride), 0, true,
@@ -1161,7 +1181,7 @@ token_step_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
       r1_phase(a, P, l, pos);
       if (!(ok = grid_sync(a, ++nb * G, &s_abort))) break;
       gemm_phase(P, P.T2, P.S2, P.nkb2, &ma2, [](int) { return 0; }, a.B, a.p2, act, tmem, y, na, nu,
-                 a.status, a.h, D);
+                 a.status, a.fx, D);
       if (!(ok = grid_sync(a, ++nb * G, &s_abort))) break;
       r2_phase(a, P, l, red);
       ok = grid_sync(a, ++nb * G, &s_abort);
@@ -1360,6 +1380,7 @@ cudaError_t launch_token_step(const TokenStepArgs& a, const void* w_qkv1, const 
                   !token_step_block_supported(DT_BF16, a.B, a.D, a.H, a.rot, a.V, a.Nt, a.Nb, 1, a.l_cap,
                                               a.n_cap, a.L_B)))
     return cudaErrorNotSupported;
+  if (!a.fx || (reinterpret_cast<uintptr_t>(a.fx) & 15)) return cudaErrorInvalidValue;
   Device& d = device();
   Plan P;
   size_t smem;

@@ -51,7 +51,6 @@ struct Roles {
   static constexpr int THREADS = EPI * 32 + 64;
   static constexpr int PRODUCER = EPI, MMA = EPI + 1;
 };
-constexpr int THREADS = Roles<true>::THREADS;  // decode orientation (split-K planning)
 
 template <int BN>
 __host__ __device__ constexpr size_t stage_bytes() {

@@ -254,6 +254,8 @@ struct TokenStepArgs {
   int32_t* next;
   float2* arg_part;  // [ceil(V/128), B]
   float *p1, *p2;    // split-K partials (token_step_scratch_floats)
+  long long* fx;     // token_step: [B, D] int64 fixed-point split-K sums (units of 2^-32),
+                     // zero between launches (each launch clears what it adds)
   unsigned* bar;     // 3 words, zero before the first launch
   int* status;
   long long wait_cycles;  // bound of every wait of the launch (SM clock cycles)

@@ -171,6 +171,7 @@ struct bt_model {
   float2* arg_part = nullptr;  // LM-head per-tile argmax partials
   int* ln_cnt = nullptr;       // per-row counters of the LayerNorm fused into GEMM epilogues
   float *ts_p1 = nullptr, *ts_p2 = nullptr;  // fused token step: split-K partials
+  long long* ts_fx = nullptr;                // fused token step: fixed-point split-K sums [Bmax][D]
   unsigned* ts_bar = nullptr;                // fused token step: grid-barrier words
   float* ts_att = nullptr;                   // fused block step: decode-attention partials
   int* ts_cnt = nullptr;                     // fused block step: merge counters [B_max * H]
@@ -311,6 +312,7 @@ static size_t carve(bt_model* m, const Dims& d, void* ws) {
     m->ts_p2 = (float*)c.take(std::max(token_step_scratch_floats(d.Bmax, d.D, 2),
                                        token_step2_scratch_floats(d.Bmax, d.D, 2)) * 4);
     m->ts_bar = (unsigned*)c.take(64);
+    m->ts_fx = (long long*)c.take((size_t)d.Bmax * d.D * sizeof(long long));
     m->ts_att = (float*)c.take(token_step_scratch_floats(d.Bmax, d.D, 3, d.H, d.n_cap) * 4);
     m->ts_cnt = (int*)c.take((size_t)d.Bmax * d.H * sizeof(int));
     m->ts2_ctr_bytes = token_step2_counter_bytes(d.D);
@@ -437,6 +439,7 @@ int bt_create(const bt_config* cfg, const bt_weights* w, void* ws, size_t ws_byt
   BT_TRYC(cudaMemsetAsync(m->row_lag, 0, (size_t)d.Bmax * 4 * sizeof(int), st));
   BT_TRYC(cudaMemsetAsync(m->ln_cnt, 0, (size_t)d.Bmax * (d.P > 1 ? d.P : 1) * sizeof(int), st));
   if (m->ts_bar) BT_TRYC(cudaMemsetAsync(m->ts_bar, 0, 64, st));
+  if (m->ts_fx) BT_TRYC(cudaMemsetAsync(m->ts_fx, 0, (size_t)d.Bmax * d.D * sizeof(long long), st));
   if (m->ts_cnt) BT_TRYC(cudaMemsetAsync(m->ts_cnt, 0, (size_t)d.Bmax * d.H * sizeof(int), st));
   if (m->ts2_ctr) BT_TRYC(cudaMemsetAsync(m->ts2_ctr, 0, m->ts2_ctr_bytes, st));
   {
@@ -890,7 +893,7 @@ static int run_token_step(bt_model* m, int B, bool ingest, PosSpec pos, const in
   a.rope_tab = m->rope_tab; a.lnf_g = m->lnf_t_g; a.lnf_b = m->lnf_t_b;
   a.h = m->h_t; a.x1 = (bf16*)m->x1; a.a2 = (bf16*)m->a2; a.xf = (bf16*)m->xf;
   a.logits = want_logits ? m->logits : nullptr; a.next = m->next; a.arg_part = m->arg_part;
-  a.p1 = m->ts_p1; a.p2 = m->ts_p2; a.bar = m->ts_bar; a.status = m->status;
+  a.p1 = m->ts_p1; a.p2 = m->ts_p2; a.fx = m->ts_fx; a.bar = m->ts_bar; a.status = m->status;
   a.wait_cycles = m->wait_cycles;
   a.l2_window_base = m->l2_base;
   a.l2_window_bytes = m->l2_window;
@@ -1065,6 +1068,8 @@ static int prefill_impl(bt_model* m, const int32_t* tokens, int T_stride, int B,
                           attn_decode_scratch_bytes(d.Bmax, d.H, d.d, d.n_cap, d.dt), s));
   // and the fused token step's barrier words (an aborted step leaves them set)
   if (m->ts_bar) BT_CUDA(cudaMemsetAsync(m->ts_bar, 0, 64, s));
+  // and its fixed-point accumulators (an aborted step can leave sums in them)
+  if (m->ts_fx) BT_CUDA(cudaMemsetAsync(m->ts_fx, 0, (size_t)d.Bmax * d.D * sizeof(long long), s));
   if (m->ts_cnt) BT_CUDA(cudaMemsetAsync(m->ts_cnt, 0, (size_t)d.Bmax * d.H * sizeof(int), s));
   if (m->ts2_ctr) BT_CUDA(cudaMemsetAsync(m->ts2_ctr, 0, m->ts2_ctr_bytes, s));
   const long long k0 = launch_count();
