@@ -24,21 +24,21 @@ namespace bt {
 // split-K decode attention
 // ---------------------------------------------------------------------------
 // A work unit is one (sequence, head) pair and a contiguous range of its
-// cached rows, streamed in CHUNK-row pieces (8 KB of K + 8 KB of V) through a
+// cached rows, streamed in CHUNK-row pieces (4 KB of K + 4 KB of V) through a
 // STAGES-deep ring of 1-D bulk copies, with an online softmax across chunks.
 // Pairs are split into several units only when there are too few pairs to
 // keep every SM busy; split units are merged by the last one to finish.
 template <typename T, int DH>
 struct DecCfg {
   static constexpr int ROW_BYTES = DH * (int)sizeof(T);
-  static constexpr int CHUNK = 8192 / ROW_BYTES;         // rows per chunk (8 KB of K)
-  static constexpr int STAGES = 3;
+  static constexpr int CHUNK = 4096 / ROW_BYTES;         // rows per chunk (4 KB of K)
+  static constexpr int STAGES = 4;
   static constexpr int TPR = ROW_BYTES / 16;             // threads per row, 16 B each
   static constexpr int CWARPS = 4;                       // consumer warps
   static constexpr int THREADS = (CWARPS + 1) * 32;      // + one producer warp
   static constexpr int GROUPS = CWARPS * 32 / TPR;       // row groups (each owns rows)
   static constexpr int EPT = 16 / (int)sizeof(T);        // elements per thread
-  static constexpr int SMEM = STAGES * 2 * CHUNK * ROW_BYTES + GROUPS * (DH + 2) * 4;
+  static constexpr int SMEM = STAGES * 2 * CHUNK * ROW_BYTES + CWARPS * (DH + 2) * 4;
   static_assert(TPR >= 1 && TPR <= 32 && (32 % TPR) == 0, "row split");
   static_assert(DH <= CWARPS * 32, "one thread per output dim in the final reduction");
 };
@@ -64,11 +64,16 @@ __device__ __forceinline__ float block_reduce_sum128(float v, float* red) {
   return v;
 }
 
-// Persistent, stream-K over the flattened list of (pair, chunk) work: CTA c of
-// G handles chunks [floor(c*T/G), floor((c+1)*T/G)) of the T = pairs * nch
-// chunks, its copy ring running straight across pair boundaries. A pair whose
-// chunks span several CTAs gets one partial (m, l, o) from each; the last to
-// finish (atomic counter, no waiting) merges them in CTA order.
+// Two partitions of the flattened list of (pair, chunk) work, the copy ring
+// of a CTA running straight across pair boundaries:
+// * whole pairs (whole = 1, when there are at least half as many pairs as
+//   resident CTAs): CTA c of G handles pairs [floor(c*pairs/G),
+//   floor((c+1)*pairs/G)), so no pair is split and no CTA merges partials
+//   or waits on a counter at its end;
+// * stream-K (whole = 0): CTA c of G handles chunks [floor(c*T/G),
+//   floor((c+1)*T/G)) of the T = pairs * nch chunks. A pair whose chunks
+//   span several CTAs gets one partial (m, l, o) from each; the last to
+//   finish (atomic counter, no waiting) merges them in CTA order.
 __device__ __forceinline__ int dec_owner(long long x, int G, long long T) {
   // the CTA whose chunk range contains chunk x
   return (int)(((x + 1) * G + T - 1) / T) - 1;
@@ -83,7 +88,7 @@ __global__ void __launch_bounds__(DecCfg<T, DH>::THREADS)
 attn_decode_kernel(const T* __restrict__ q, int ldq, const T* __restrict__ kc,
                    const T* __restrict__ vc, int pairs, int H, int cap, PosSpec kvlen,
                    T* __restrict__ out, int ld_out, float* __restrict__ part,
-                   int* __restrict__ counters, int* status, float qscale, int qpk) {
+                   int* __restrict__ counters, int* status, float qscale, int qpk, int whole) {
   pdl_trigger();
   pdl_wait();
   using C = DecCfg<T, DH>;
@@ -92,12 +97,14 @@ attn_decode_kernel(const T* __restrict__ q, int ldq, const T* __restrict__ kc,
   const int n = pos_base(kvlen) + 1;
   const int nch = (n + C::CHUNK - 1) / C::CHUNK;
   const long long Ttot = (long long)pairs * nch;
-  // effective grid <= chunks, so that every CTA's range is non-empty and the
-  // CTAs sharing a pair are consecutive
-  const int G = (int)((long long)gridDim.x < Ttot ? (long long)gridDim.x : Ttot);
+  // effective grid <= chunks (stream-K) or <= pairs (whole pairs), so that
+  // every CTA's range is non-empty and the CTAs sharing a pair are consecutive
+  const long long units = whole ? (long long)pairs : Ttot;
+  const int G = (int)((long long)gridDim.x < units ? (long long)gridDim.x : units);
   const int c = blockIdx.x;
   if (c >= G) return;
-  const long long x0 = (long long)c * Ttot / G, x1 = (long long)(c + 1) * Ttot / G;
+  const long long x0 = whole ? (long long)c * pairs / G * nch : (long long)c * Ttot / G;
+  const long long x1 = whole ? (long long)(c + 1) * pairs / G * nch : (long long)(c + 1) * Ttot / G;
   const int nc = (int)(x1 - x0);
 
   extern __shared__ __align__(128) uint8_t smem[];
@@ -151,6 +158,13 @@ attn_decode_kernel(const T* __restrict__ q, int ldq, const T* __restrict__ kc,
   const int g = tid / C::TPR;  // valid for consumer warps
   const int e0 = (tid % C::TPR) * C::EPT;
   const int first_pair = (int)(x0 / nch);
+  // q of the CTA's first pair; the next pair's q is loaded while the current
+  // pair is combined
+  uint4 qn;
+  {
+    const int b = first_pair / H, h = first_pair - b * H;
+    qn = *reinterpret_cast<const uint4*>(q + (size_t)b * ldq + h * DH + e0);
+  }
   int i = 0;
   for (int pr = first_pair; i < nc; ++pr) {
     const long long pend = (long long)(pr + 1) * nch;
@@ -163,12 +177,9 @@ attn_decode_kernel(const T* __restrict__ q, int ldq, const T* __restrict__ kc,
     for (int e = 0; e < C::EPT; ++e) of[e] = 0.f;
     {
       float qf[C::EPT];
-      {
-        const uint4 u = *reinterpret_cast<const uint4*>(q + (size_t)b * ldq + h * DH + e0);
-        unpack16(u, qf, (const T*)nullptr);
+      unpack16(qn, qf, (const T*)nullptr);
 #pragma unroll
-        for (int e = 0; e < C::EPT; ++e) qf[e] *= qscale;
-      }
+      for (int e = 0; e < C::EPT; ++e) qf[e] *= qscale;
       for (int k = 0; k < cnt; ++k) {
         const int ii = i + k;
         const int s = ii % C::STAGES;
@@ -207,27 +218,49 @@ attn_decode_kernel(const T* __restrict__ q, int ldq, const T* __restrict__ kc,
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);  // this warp is done with stage s
       }
-      // park this group's (M, l, o slice) for the combination
-      float* gr = sR + (size_t)g * (DH + 2);
-#pragma unroll
-      for (int e = 0; e < C::EPT; ++e) gr[2 + e0 + e] = of[e];
-      if ((tid % C::TPR) == 0) { gr[0] = M; gr[1] = l; }
     }
     i += cnt;
+    if (i < nc) {
+      const int b1 = (pr + 1) / H, h1 = (pr + 1) - b1 * H;
+      qn = *reinterpret_cast<const uint4*>(q + (size_t)b1 * ldq + h1 * DH + e0);
+    }
+    // the warp's row groups merged by shuffles: lanes t, t + TPR, ... hold
+    // the same output slice (a group without rows has M = -FLT_MAX, l = 0)
+#pragma unroll
+    for (int o = C::TPR; o < 32; o <<= 1) {
+      const float Mo = __shfl_xor_sync(0xffffffffu, M, o);
+      const float lo = __shfl_xor_sync(0xffffffffu, l, o);
+      const float Mn = fmaxf(M, Mo);
+      const float wa = exp2f(M - Mn), wb = exp2f(Mo - Mn);
+      l = l * wa + lo * wb;
+#pragma unroll
+      for (int e = 0; e < C::EPT; ++e) of[e] = of[e] * wa + __shfl_xor_sync(0xffffffffu, of[e], o) * wb;
+      M = Mn;
+    }
+    // park each warp's (M, l, o) for the combination across warps
+    if (lane < C::TPR) {
+      float* gr = sR + (size_t)warp * (DH + 2);
+#pragma unroll
+      for (int e = 0; e < C::EPT; ++e) gr[2 + e0 + e] = of[e];
+      if (lane == 0) { gr[0] = M; gr[1] = l; }
+    }
     cons_sync();
-    // combine the groups: thread t < DH owns output dim t
+    // combine the warps: thread t < DH owns output dim t
     float Mg = -FLT_MAX, Lg = 0.f, og = 0.f;
     if (tid < DH) {
-      for (int gg = 0; gg < C::GROUPS; ++gg) Mg = fmaxf(Mg, sR[(size_t)gg * (DH + 2)]);
-      for (int gg = 0; gg < C::GROUPS; ++gg) {
-        const float* gr = sR + (size_t)gg * (DH + 2);
-        const float w = exp2f(gr[0] - Mg);
-        Lg = fmaf(w, gr[1], Lg);
-        og = fmaf(w, gr[2 + tid], og);
+#pragma unroll
+      for (int w = 0; w < C::CWARPS; ++w) Mg = fmaxf(Mg, sR[(size_t)w * (DH + 2)]);
+#pragma unroll
+      for (int w = 0; w < C::CWARPS; ++w) {
+        const float* gr = sR + (size_t)w * (DH + 2);
+        const float wt = exp2f(gr[0] - Mg);
+        Lg = fmaf(wt, gr[1], Lg);
+        og = fmaf(wt, gr[2 + tid], og);
       }
     }
     const long long pbeg = (long long)pr * nch;
-    const int first = dec_owner(pbeg, G, Ttot), last = dec_owner(pbeg + nch - 1, G, Ttot);
+    const int first = whole ? c : dec_owner(pbeg, G, Ttot);
+    const int last = whole ? c : dec_owner(pbeg + nch - 1, G, Ttot);
     if (first == last) {
       if (ok && tid < DH) out[(size_t)b * ld_out + h * DH + tid] = from_f<T>(og / Lg);
     } else {
@@ -235,12 +268,18 @@ attn_decode_kernel(const T* __restrict__ q, int ldq, const T* __restrict__ kc,
       float* my = part + ((size_t)2 * c + (pr == first_pair ? 0 : 1)) * (DH + 2);
       if (tid < DH) my[2 + tid] = og;
       if (tid == 0) { my[0] = Mg; my[1] = Lg; }
-      __threadfence();
+      // the consumers' barrier orders their partial writes before thread 0's
+      // gpu-scope fence and counter update (release); the fence after the
+      // update orders the last arriver's reads of the other partials after
+      // it (acquire)
       cons_sync();
-      if (tid == 0) s_last = (atomicAdd(&counters[pr], 1) == last - first);
+      if (tid == 0) {
+        __threadfence();
+        s_last = (atomicAdd(&counters[pr], 1) == last - first);
+        __threadfence();
+      }
       cons_sync();
       if (s_last) {
-        __threadfence();
         float M2 = -FLT_MAX;
         for (int cc = first; cc <= last; ++cc) {
           const int first_of_cc = (int)(((long long)cc * Ttot / G) / nch);
@@ -267,20 +306,35 @@ static int dec_sm_count() { return device_sm_count(); }
 
 template <typename T>
 static int dec_chunk(int d) {
-  return 8192 / (d * (int)sizeof(T));
+  return 4096 / (d * (int)sizeof(T));
 }
 
-constexpr int DEC_CTAS_PER_SM = 4;
+// resident CTAs per SM: 6 x (32 KB ring + the combine slots) of shared
+// memory, 6 x 160 threads x 64 registers
+constexpr int DEC_CTAS_PER_SM = 6;
 
-// Persistent grid: DEC_CTAS_PER_SM CTAs per SM, never more than the chunks.
-static int dec_grid(int pairs, int d, int cap, int dt) {
+// Persistent grid, at most DEC_CTAS_PER_SM CTAs per SM. With at least half as
+// many (sequence, head) pairs as resident CTAs each CTA takes whole pairs,
+// k or k - 1 of them for k = ceil(pairs / resident) (*whole = 1); with fewer
+// pairs the chunks are spread over every resident CTA (stream-K, never more
+// CTAs than chunks at the capacity).
+static int dec_grid(int pairs, int d, int cap, int dt, int* whole) {
   const int chunk = dt == DT_BF16 ? dec_chunk<bf16>(d) : dec_chunk<float>(d);
+  const long long slots = (long long)DEC_CTAS_PER_SM * dec_sm_count();
+  if (2LL * pairs >= slots) {
+    *whole = 1;
+    const long long k = (pairs + slots - 1) / slots;
+    return (int)((pairs + k - 1) / k);
+  }
+  *whole = 0;
   const long long max_chunks = (long long)pairs * ((cap + chunk - 1) / chunk);
-  const long long g = (long long)DEC_CTAS_PER_SM * dec_sm_count();
-  return (int)(g < max_chunks ? g : max_chunks);
+  return (int)(slots < max_chunks ? slots : max_chunks);
 }
 
-int attn_decode_max_splits(int d, int cap, int dt) { return dec_grid(1, d, cap, dt); }
+int attn_decode_max_splits(int d, int cap, int dt) {
+  int whole;
+  return dec_grid(1, d, cap, dt, &whole);
+}
 
 // scratch layout: [merge counters: B*H ints, 256-aligned][partials: two
 // slots of (d + 2) floats per CTA of the grid]; counters sit at offset 0.
@@ -319,7 +373,8 @@ static cudaError_t launch_dec(const void* q, int ldq, const void* kc, const void
   cudaError_t e = dec_prepare<T, DH>();
   if (e != cudaSuccess) return e;
   const int pairs = B * H;
-  int G = dec_grid(pairs, DH, cap, sizeof(T) == 2 ? DT_BF16 : DT_F32);
+  int whole = 0;
+  int G = dec_grid(pairs, DH, cap, sizeof(T) == 2 ? DT_BF16 : DT_F32, &whole);
   if (G > DEC_UNITS_SLACK) G = DEC_UNITS_SLACK;  // partial slots in the scratch
   int* counters = reinterpret_cast<int*>(scratch);
   float* partp = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(scratch) +
@@ -327,7 +382,7 @@ static cudaError_t launch_dec(const void* q, int ldq, const void* kc, const void
   const float qscale = 1.4426950408889634f / sqrtf((float)DH);
   BT_LAUNCH(attn_decode_kernel<T, DH>, dim3(G), dim3(C::THREADS), C::SMEM, s, (const T*)q, ldq,
             (const T*)kc, (const T*)vc, pairs, H, cap, kvlen, (T*)out, ld_out, partp, counters,
-            status, qscale, g);
+            status, qscale, g, whole);
   return cudaSuccess;
 }
 

@@ -156,10 +156,13 @@ def test_linear_tensor_cores_match_fp64(M, N, K):
 
 
 @pytest.mark.parametrize("B,H,d,n,cap", [(64, 12, 64, 300, 544), (8, 16, 128, 2100, 2176),
-                                         (256, 16, 64, 37, 544), (1, 1, 64, 1, 8)])
+                                         (256, 16, 64, 37, 544), (1, 1, 64, 1, 8),
+                                         (100, 10, 64, 200, 208), (48, 12, 128, 77, 80)])
 def test_decode_attention_bench_shapes(B, H, d, n, cap):
-    """Stream-K decode attention at the workloads' shapes (pairs split across
-    CTAs and merged) against the oracle's attention in fp64."""
+    """Decode attention at the workloads' shapes against the oracle's
+    attention in fp64, in both partitions: whole (sequence, head) pairs per
+    CTA (one, or an uneven two per CTA at 1,000 pairs) and stream-K (few
+    pairs: pairs split across CTAs and merged)."""
     from hierarchical_global_local_b200 import native
     torch = gh.torch_mod()
     g = torch.Generator(device="cuda").manual_seed(B * 7 + n)
