@@ -275,6 +275,8 @@ def run_ours(args):
         line["roofline"] = prof["dominant"]
         line["roofline_decode_attention"] = prof.get("attn_decode")
         line["roofline_decode_attention_n300"] = prof.get("attn_decode_n300")
+        if line["roofline_decode_attention_n300"] is not None and ws == 1:
+            line["roofline_decode_attention_n300"]["graph_replay"] = decode_attention_replay(hbm)
         line["roofline_decode_gemm"] = prof.get("gemm_decode")
         line["kernel_time_shares"] = prof["shares"]
         line["roofline"]["peak_source"] = peak_src
@@ -304,8 +306,8 @@ def run_ours(args):
 # the source is unchanged; after a change the traffic is null until it is
 # captured again.
 NCU_TRAFFIC = {
-    "token_step": {"bytes": 172.24e6, "source": "hierarchical_global_local_b200/csrc/decode_step.cu",
-                   "sha16": "3ad7db2bece3a80b"},
+    "token_step": {"bytes": 171.20e6, "source": "hierarchical_global_local_b200/csrc/decode_step.cu",
+                   "sha16": "5d27b7f429b0acb0"},
 }
 
 
@@ -322,6 +324,61 @@ def ncu_traffic(kind: str):
     except OSError:
         return None
     return e["bytes"] if sha == e["sha16"] else None
+
+
+def decode_attention_replay(hbm: float, ns=(300, 420, 545)):
+    """The block decoder's decode attention alone at the decode-heavy
+    workload's shapes (B 64, H 12, d_head 64, bf16, cache capacity 576):
+    32 launches per n, captured in one CUDA graph, cycling through 8 K/V
+    sets (8 x 113 MB, past L2) so that every launch reads its cache from
+    HBM; CUDA events around the replays. Unlike the in-model figure (an
+    event pair around every launch, which also times each launch's start
+    without the overlap programmatic dependent launch gives inside the
+    decode graphs) this is the kernel's duration in a launch sequence."""
+    import torch
+    from hierarchical_global_local_b200 import native
+    shape = synth.WORKLOADS["pythia160m_decode_heavy"].shape
+    B, H, d, cap, R = 64, shape.n_heads, shape.d_model // shape.n_heads, 576, 8
+    g = torch.Generator(device="cuda").manual_seed(3)
+    qs = [torch.randn(B, H * d, device="cuda", generator=g).bfloat16() for _ in range(R)]
+    ks = [torch.randn(B, H, cap, d, device="cuda", generator=g).bfloat16() for _ in range(R)]
+    vs = [torch.randn(B, H, cap, d, device="cuda", generator=g).bfloat16() for _ in range(R)]
+    out = torch.empty(B, H * d, device="cuda", dtype=torch.bfloat16)
+    scr = native.decode_attention_scratch(native.BT_BF16, B, H, d, cap)
+    st = torch.cuda.Stream()
+    res, tot_b, tot_us = {}, 0.0, 0.0
+    with torch.cuda.stream(st):
+        for n in ns:
+            for i in range(R):
+                native.decode_attention(qs[i], ks[i], vs[i], n, out=out, scratch=scr)
+            st.synchronize()
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, stream=st):
+                for _ in range(4):
+                    for i in range(R):
+                        native.decode_attention(qs[i], ks[i], vs[i], n, out=out, scratch=scr)
+            for _ in range(3):
+                gr.replay()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            st.synchronize()
+            a.record(st)
+            for _ in range(5):
+                gr.replay()
+            b.record(st)
+            st.synchronize()
+            us = a.elapsed_time(b) * 1e3 / (5 * 4 * R)
+            by = B * H * (2.0 * n * d * 2 + 2.0 * d * 2)
+            res[str(n)] = {"us": us, "GB/s": by / us / 1e3, "frac": by / us / 1e3 / hbm}
+            tot_b += by
+            tot_us += us
+            del gr
+    ach = tot_b / tot_us / 1e3
+    del qs, ks, vs
+    torch.cuda.empty_cache()
+    return {"kernel": "attn_decode", "bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s",
+            "frac": ach / hbm, "per_n": res,
+            "case": f"B {B} H {H} d {d} bf16, n {list(ns)}, 8 K/V sets past L2, CUDA-graph replay"}
 
 
 def profile_step(model, prompts, gens, flush):

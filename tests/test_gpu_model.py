@@ -201,16 +201,18 @@ def test_fused_token_step_matches_oracle_and_chain(lb, B, D, H, P, kind, monkeyp
     assert np.array_equal(gn, gl.argmax(axis=-1))
 
 
-@pytest.mark.parametrize("lb,B", [(4, 5), (8, 64), (2, 33)])
-def test_fused_block_step_matches_oracle_and_chain(lb, B, monkeypatch):
+@pytest.mark.parametrize("lb,B,nbp", [(4, 5, 12), (8, 64, 12), (2, 33, 12), (2, 40, 70), (4, 64, 40)])
+def test_fused_block_step_matches_oracle_and_chain(lb, B, nbp, monkeypatch):
     """A block step (block decoder with decode attention over the block cache,
     LN_b, the prefix projection, then the token decoder and the LM head) as
     one persistent kernel (opt-in): one launch per block step, logits match
-    the oracle and agree with the kernel-per-operation block step."""
+    the oracle and agree with the kernel-per-operation block step. nbp prompt
+    blocks: block caches of one unit of 32 entries and of several with a
+    ragged last one, whose (sequence, head) runs are merged across warps."""
     monkeypatch.setenv("BT_DECODE_BLOCK_STEP", "fused")
     shape = synth.ModelShape(vocab=3000, d_model=256, n_heads=4, block_len=lb,
                              n_block_layers=3, n_token_layers=2, prefix_len=1)
-    T, G = 12 * lb, 4 * lb + 3
+    T, G = nbp * lb, 4 * lb + 3
     w = synth.make_weights(shape, seed=41)
     toks = synth.make_tokens(batch=B, length=T + G, vocab=shape.vocab, seed=42)
     torch = gh.torch_mod()
