@@ -448,22 +448,27 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
         float acc[16], pv[16];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          // the ks partials of column quad cc0/4 + u, all loads in flight,
-          // summed in rank order
-          float4 part[MAX_KS];
+          // the ks partials of column quad cc0/4 + u, summed in rank order,
+          // four ranks' loads in flight at a time
           const int q = cc0 / 4 + u;
-#pragma unroll
-          for (int p = 0; p < MAX_KS; ++p)
-            if (p < ks && 4 * u < cnt) part[p] = tc::ld_shared_v4(recv + (uint32_t)(((p * qpr + q) * BM + r) * 16));
           float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-          for (int p = 0; p < MAX_KS; ++p)
-            if (p < ks && 4 * u < cnt) {
-              t.x += part[p].x;
-              t.y += part[p].y;
-              t.z += part[p].z;
-              t.w += part[p].w;
-            }
+          for (int p0 = 0; p0 < MAX_KS; p0 += 4) {
+            if (p0 >= ks) break;
+            float4 part[4];
+#pragma unroll
+            for (int p = 0; p < 4; ++p)
+              if (p0 + p < ks && 4 * u < cnt)
+                part[p] = tc::ld_shared_v4(recv + (uint32_t)((((p0 + p) * qpr + q) * BM + r) * 16));
+#pragma unroll
+            for (int p = 0; p < 4; ++p)
+              if (p0 + p < ks && 4 * u < cnt) {
+                t.x += part[p].x;
+                t.y += part[p].y;
+                t.z += part[p].z;
+                t.w += part[p].w;
+              }
+          }
           acc[4 * u] = t.x;
           acc[4 * u + 1] = t.y;
           acc[4 * u + 2] = t.z;
