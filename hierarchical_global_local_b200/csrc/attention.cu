@@ -45,6 +45,10 @@ struct DecCfg {
 
 constexpr int DEC_UNITS_SLACK = ATTN_DECODE_MAX_CTAS;  // partial slots in the scratch (grid cap)
 
+// resident CTAs per SM: 6 x (32 KB ring + the combine slots) of shared
+// memory, 6 x 160 threads x at most 64 registers (the launch bound)
+constexpr int DEC_CTAS_PER_SM = 6;
+
 __device__ __forceinline__ float block_reduce_max128(float v, float* red) {
   v = warp_max(v);
   const int w = threadIdx.x >> 5;
@@ -84,7 +88,7 @@ __device__ __forceinline__ int dec_owner(long long x, int G, long long T) {
 __device__ __forceinline__ void cons_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 template <typename T, int DH>
-__global__ void __launch_bounds__(DecCfg<T, DH>::THREADS)
+__global__ void __launch_bounds__(DecCfg<T, DH>::THREADS, DEC_CTAS_PER_SM)
 attn_decode_kernel(const T* __restrict__ q, int ldq, const T* __restrict__ kc,
                    const T* __restrict__ vc, int pairs, int H, int cap, PosSpec kvlen,
                    T* __restrict__ out, int ld_out, float* __restrict__ part,
@@ -188,30 +192,45 @@ attn_decode_kernel(const T* __restrict__ q, int ldq, const T* __restrict__ kc,
         const T* sV = sK + C::CHUNK * DH;
         const long long x = x0 + ii;
         const int rows = min(C::CHUNK, np - (int)(x - (long long)pr * nch) * C::CHUNK);
-        // uniform trip count over the warp: the row-group shuffles always
-        // see the whole warp
-        for (int rb = 0; rb < rows; rb += C::GROUPS) {
-          const int r = rb + g;
-          const bool valid = r < rows;
-          float sc = 0.f;
-          float vf[C::EPT];
-          if (valid) {
-            const uint4 uk = *reinterpret_cast<const uint4*>(sK + r * DH + e0);
-            const uint4 uv = *reinterpret_cast<const uint4*>(sV + r * DH + e0);
+        // a chunk holds 2 * GROUPS rows: row group g takes rows g and
+        // g + GROUPS and folds both into its softmax with one rescale. All
+        // lanes run the shuffles (an empty row scores -FLT_MAX, weight 0).
+        static_assert(C::CHUNK == 2 * C::GROUPS, "two rows per row group and chunk");
+        {
+          const int r0 = g, r1 = g + C::GROUPS;
+          const bool v0 = r0 < rows, v1 = r1 < rows;
+          float s0 = 0.f, s1 = 0.f;
+          float vf0[C::EPT], vf1[C::EPT];
+          if (v0) {
             float kf[C::EPT];
-            unpack16(uk, kf, (const T*)nullptr);
-            unpack16(uv, vf, (const T*)nullptr);
+            unpack16(*reinterpret_cast<const uint4*>(sK + r0 * DH + e0), kf, (const T*)nullptr);
+            unpack16(*reinterpret_cast<const uint4*>(sV + r0 * DH + e0), vf0, (const T*)nullptr);
 #pragma unroll
-            for (int e = 0; e < C::EPT; ++e) sc = fmaf(qf[e], kf[e], sc);
+            for (int e = 0; e < C::EPT; ++e) s0 = fmaf(qf[e], kf[e], s0);
+          }
+          if (v1) {
+            float kf[C::EPT];
+            unpack16(*reinterpret_cast<const uint4*>(sK + r1 * DH + e0), kf, (const T*)nullptr);
+            unpack16(*reinterpret_cast<const uint4*>(sV + r1 * DH + e0), vf1, (const T*)nullptr);
+#pragma unroll
+            for (int e = 0; e < C::EPT; ++e) s1 = fmaf(qf[e], kf[e], s1);
           }
 #pragma unroll
-          for (int o = C::TPR / 2; o > 0; o >>= 1) sc += __shfl_xor_sync(0xffffffffu, sc, o);
-          if (valid) {
-            const float Mn = fmaxf(M, sc);
-            const float cs = exp2f(M - Mn), p = exp2f(sc - Mn);
-            l = l * cs + p;
+          for (int o = C::TPR / 2; o > 0; o >>= 1) {
+            s0 += __shfl_xor_sync(0xffffffffu, s0, o);
+            s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+          }
+          if (v0) {
+            if (!v1) s1 = -FLT_MAX;
+            const float Mn = fmaxf(M, fmaxf(s0, s1));
+            const float cs = exp2f(M - Mn), p0 = exp2f(s0 - Mn), p1 = v1 ? exp2f(s1 - Mn) : 0.f;
+            l = l * cs + (p0 + p1);
 #pragma unroll
-            for (int e = 0; e < C::EPT; ++e) of[e] = fmaf(p, vf[e], of[e] * cs);
+            for (int e = 0; e < C::EPT; ++e) {
+              float t = of[e] * cs;
+              t = fmaf(p0, vf0[e], t);
+              of[e] = v1 ? fmaf(p1, vf1[e], t) : t;
+            }
             M = Mn;
           }
         }
@@ -309,9 +328,6 @@ static int dec_chunk(int d) {
   return 4096 / (d * (int)sizeof(T));
 }
 
-// resident CTAs per SM: 6 x (32 KB ring + the combine slots) of shared
-// memory, 6 x 160 threads x 64 registers
-constexpr int DEC_CTAS_PER_SM = 6;
 
 // Persistent grid, at most DEC_CTAS_PER_SM CTAs per SM. With at least half as
 // many (sequence, head) pairs as resident CTAs each CTA takes whole pairs,
