@@ -544,38 +544,54 @@ __device__ void attend_item(const TokenStepArgs& a, const Plan& P, const float* 
   }
 }
 
-__device__ void gelu_fc1(const TokenStepArgs& a, const Plan& P, const float* bq);
+__device__ void gelu_fc1(const TokenStepArgs& a, const Plan& P, const float* bq, int c0 = 0, int nc = 0);
 
 __device__ void r1_phase(const TokenStepArgs& a, const Plan& P, int l, int pos) {
   const int B = a.B;
   const float* bq = layer_ptr(a.b_qkv1, l, a.layer_stride);
   bf16* kc = a.kt + (size_t)l * a.kt_layer;
   bf16* vc = a.vt + (size_t)l * a.kt_layer;
-  // (sequence, head) items over the half-warps of the grid; both halves of
-  // a warp run the shuffles together, an idle half with active = false
+  // (sequence, head) items over the half-warps of the first CA CTAs; both
+  // halves of a warp run the shuffles together, an idle half with
+  // active = false. When one item per half-warp leaves CTAs without items,
+  // and those can take GELU(fc1) in at most two batches of four float4 per
+  // thread, they do it meanwhile (two latency chains side by side instead
+  // of one after the other); else every CTA does GELU after its items.
+  const int G = gridDim.x;
   const int hw = threadIdx.x >> 4;
   const int n_items = B * a.H;
-  for (int i0 = blockIdx.x * 8 + (hw & ~1); i0 < n_items; i0 += 8 * gridDim.x) {
-    const int i = i0 + (hw & 1);
-    const bool active = i < n_items;
-    const int b = active ? i / a.H : 0, h = active ? i - b * a.H : 0;
-    if (a.dh == 32) attend_item<32>(a, P, bq, kc, vc, b, h, pos, active);
-    else if (a.dh == 64) attend_item<64>(a, P, bq, kc, vc, b, h, pos, active);
-    else attend_item<128>(a, P, bq, kc, vc, b, h, pos, active);
+  const int A = min(G, (n_items + 7) / 8);
+  const bool split = A < G && (long long)B * a.D <= (long long)(G - A) * WORKERS * 8;
+  const int CA = split ? A : G;
+  if ((int)blockIdx.x < CA) {
+    for (int i0 = blockIdx.x * 8 + (hw & ~1); i0 < n_items; i0 += 8 * CA) {
+      const int i = i0 + (hw & 1);
+      const bool active = i < n_items;
+      const int b = active ? i / a.H : 0, h = active ? i - b * a.H : 0;
+      if (a.dh == 32) attend_item<32>(a, P, bq, kc, vc, b, h, pos, active);
+      else if (a.dh == 64) attend_item<64>(a, P, bq, kc, vc, b, h, pos, active);
+      else attend_item<128>(a, P, bq, kc, vc, b, h, pos, active);
+    }
   }
-  gelu_fc1(a, P, bq);
+  gelu_fc1(a, P, bq, split ? A : 0, split ? G - A : 0);
 }
 
 // GELU(fc1): features 3D + c, c < 4D, of the first GEMM (its K splits + the
 // bias) -> a2[:, D + c], four at a time (a group never crosses a 128-feature
-// tile)
-__device__ void gelu_fc1(const TokenStepArgs& a, const Plan& P, const float* bq) {
+// tile), over the nc CTAs c0 .. c0 + nc - 1 (nc = 0: the whole grid)
+__device__ void gelu_fc1(const TokenStepArgs& a, const Plan& P, const float* bq, int c0, int nc) {
+  if (nc <= 0) {
+    c0 = 0;
+    nc = gridDim.x;
+  }
+  const int rank = (int)blockIdx.x - c0;
+  if (rank < 0 || rank >= nc) return;
   const int D = a.D, B = a.B;
   const int W4 = D;  // float4 groups per row
   const int E = B * W4;
-  const int nthr = gridDim.x * WORKERS;
+  const int nthr = nc * WORKERS;
   constexpr int BATCH = 4;
-  for (int e0 = blockIdx.x * WORKERS + threadIdx.x; e0 < E; e0 += BATCH * nthr) {
+  for (int e0 = rank * WORKERS + threadIdx.x; e0 < E; e0 += BATCH * nthr) {
     float4 acc[BATCH];
 #pragma unroll
     for (int j = 0; j < BATCH; ++j) {

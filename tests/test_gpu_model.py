@@ -165,7 +165,8 @@ def _launches(model):
     (4, 33, 512, 4, 2, "v2"),      # d_head 128, two prefix rows
     (8, 64, 256, 8, 1, "v2"),      # d_head 32, window of 8 rows
     (4, 5, 128, 4, 3, "v2"),       # one tile per GEMM row block, three prefix rows
-    (4, 3, 256, 4, 1, "v1"), (8, 17, 256, 4, 1, "v1")])
+    (4, 3, 256, 4, 1, "v1"), (8, 17, 256, 4, 1, "v1"),
+    (2, 64, 1024, 16, 1, "v1")])    # too few CTAs left without items for GELU
 def test_fused_token_step_matches_oracle_and_chain(lb, B, D, H, P, kind, monkeypatch):
     """The token-decoder half of a decode step as one persistent kernel (v1:
     grid barriers; v2: counter-synchronised, any prefix length): a token step is a
