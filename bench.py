@@ -306,8 +306,8 @@ def run_ours(args):
 # the source is unchanged; after a change the traffic is null until it is
 # captured again.
 NCU_TRAFFIC = {
-    "token_step": {"bytes": 171.20e6, "source": "hierarchical_global_local_b200/csrc/decode_step.cu",
-                   "sha16": "5d27b7f429b0acb0"},
+    "token_step": {"bytes": 171.21e6, "source": "hierarchical_global_local_b200/csrc/decode_step.cu",
+                   "sha16": "0a13c8aec57d57e4"},
 }
 
 
@@ -781,8 +781,9 @@ def run_lb_sweep(args):
 
 def run_kernel_case(args):
     """One op of the path through the op-level C-ABI, a few launches, for
-    profiler captures: decode attention (B, H, d, n) or a dense projection
-    (M, N, K) on the tensor-core path."""
+    profiler captures: decode attention (B, H, d, n), the tensor-core
+    prefill attention (B, H, d, n: causal over n block rows per sequence) or
+    a dense projection (M, N, K) on the tensor-core path."""
     import torch
     from hierarchical_global_local_b200 import native
     torch.cuda.set_device(0)
@@ -796,6 +797,13 @@ def run_kernel_case(args):
         out = torch.empty(B, H * d, device="cuda", dtype=torch.bfloat16)
         scr = native.decode_attention_scratch(native.BT_BF16, B, H, d, n)
         run = lambda: native.decode_attention(q, k, v, n, out=out, scratch=scr)  # noqa: E731
+    elif args.case == "prefill_attention":
+        B, H, d, n = dims
+        q = torch.randn(B * n, H * d, device="cuda", generator=g).bfloat16()
+        k = torch.randn(B, H, n, d, device="cuda", generator=g).bfloat16()
+        v = torch.randn(B, H, n, d, device="cuda", generator=g).bfloat16()
+        out = torch.empty(B * n, H * d, device="cuda", dtype=torch.bfloat16)
+        run = lambda: native.prefill_attention_tc(q, k, v, n, out=out)  # noqa: E731
     else:
         M, N, K = dims
         x = torch.randn(M, K, device="cuda", generator=g).bfloat16()
@@ -839,7 +847,8 @@ def main():
                     help="time budget of the cpu_baseline leg of our arm")
     ap.add_argument("--ref-seconds", type=float, default=60.0,
                     help="--impl reference: oracle time budget over all warm-up and timed steps")
-    ap.add_argument("--case", default=None, choices=["decode", "prefill", "decode_attention", "linear", "lb_sweep",
+    ap.add_argument("--case", default=None, choices=["decode", "prefill", "decode_attention", "prefill_attention",
+                                                     "linear", "lb_sweep",
                                                      "batch_sweep", "variants"],
                     help="instead of the benchmark, run a bounded case for profiler captures: decode "
                          "calls of the decode-heavy workload, or one op of the path")
@@ -847,7 +856,7 @@ def main():
                     help="decode calls / launches of the case (default 8); lb_sweep: generated "
                          "tokens (default: the configured 512)")
     ap.add_argument("--case-shape", default="128,16,64,640",
-                    help="decode_attention: B,H,d,n; linear: M,N,K")
+                    help="decode_attention, prefill_attention: B,H,d,n; linear: M,N,K")
     args = ap.parse_args()
     if args.gpus > 1 and "WORLD_SIZE" not in os.environ and args.case is None:
         relaunch_distributed(args.gpus)
@@ -877,7 +886,7 @@ def main():
     if args.case == "variants":
         run_variants_case(args)
         return
-    if args.case in ("decode_attention", "linear"):
+    if args.case in ("decode_attention", "prefill_attention", "linear"):
         run_kernel_case(args)
         return
     if args.impl == "reference":

@@ -26,6 +26,15 @@
 
 namespace bt {
 
+// 2^x by the special-function unit's approximation (PTX ex2.approx.ftz.f32;
+// subnormal results flush to zero, so a softmax weight below 2^-126 of the
+// row's largest counts as 0)
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 namespace {
 
 constexpr int QT = 128;   // queries per CTA (MMA M)
@@ -179,16 +188,32 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
       mbar_wait_bounded(s_full, j & 1, status);
       tc::fence_after();
       const int k0 = j * KT;
+      // every key of the tile is visible to every query row of the CTA (left
+      // of the diagonal, inside n): no per-element masking (warp-uniform)
+      const bool full = (k0 + KT - 1 <= q0) && (k0 + KT <= n);
       // pass 1: row max over this tile (masked keys excluded), 32 columns at a time
       float tmax = -INFINITY;
+      if (full) {
+        // the scale is positive: scale the raw maximum once
+        float rmax = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < KT; c += 32) {
-        float sv[32];
-        tc::tmem_ld32(tS + lane_base + c, sv);
+        for (int c = 0; c < KT; c += 32) {
+          float sv[32];
+          tc::tmem_ld32(tS + lane_base + c, sv);
 #pragma unroll
-        for (int u = 0; u < 32; ++u) {
-          const int kj = k0 + c + u;
-          if (kj <= qi && kj < n) tmax = fmaxf(tmax, sv[u] * scale_log2);
+          for (int u = 0; u < 32; ++u) rmax = fmaxf(rmax, sv[u]);
+        }
+        tmax = rmax * scale_log2;
+      } else {
+#pragma unroll
+        for (int c = 0; c < KT; c += 32) {
+          float sv[32];
+          tc::tmem_ld32(tS + lane_base + c, sv);
+#pragma unroll
+          for (int u = 0; u < 32; ++u) {
+            const int kj = k0 + c + u;
+            if (kj <= qi && kj < n) tmax = fmaxf(tmax, sv[u] * scale_log2);
+          }
         }
       }
       const float mn = fmaxf(m, tmax);
@@ -220,11 +245,19 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
 #pragma unroll
         for (int c8 = 0; c8 < 4; ++c8) {
           float p[8];
+          if (full) {
 #pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const int kj = k0 + c + c8 * 8 + u;
-            p[u] = (kj <= qi && kj < n) ? exp2f(sv[c8 * 8 + u] * scale_log2 - mn) : 0.f;
-            lt += p[u];
+            for (int u = 0; u < 8; ++u) {
+              p[u] = ex2_approx(fmaf(sv[c8 * 8 + u], scale_log2, -mn));
+              lt += p[u];
+            }
+          } else {
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const int kj = k0 + c + c8 * 8 + u;
+              p[u] = (kj <= qi && kj < n) ? ex2_approx(fmaf(sv[c8 * 8 + u], scale_log2, -mn)) : 0.f;
+              lt += p[u];
+            }
           }
           __nv_bfloat162 h0 = __floats2bfloat162_rn(p[0], p[1]), h1 = __floats2bfloat162_rn(p[2], p[3]);
           __nv_bfloat162 h2 = __floats2bfloat162_rn(p[4], p[5]), h3 = __floats2bfloat162_rn(p[6], p[7]);
