@@ -192,18 +192,20 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
       // of the diagonal, inside n): no per-element masking (warp-uniform)
       const bool full = (k0 + KT - 1 <= q0) && (k0 + KT <= n);
       // pass 1: row max over this tile (masked keys excluded), 32 columns at a time
-      float tmax = -INFINITY;
+      // (eight independent max chains: two softmax warps share a scheduler,
+      // so one 128-long dependency chain per row would leave it idle)
+      float mx[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) mx[u] = -INFINITY;
       if (full) {
         // the scale is positive: scale the raw maximum once
-        float rmax = -INFINITY;
 #pragma unroll
         for (int c = 0; c < KT; c += 32) {
           float sv[32];
           tc::tmem_ld32(tS + lane_base + c, sv);
 #pragma unroll
-          for (int u = 0; u < 32; ++u) rmax = fmaxf(rmax, sv[u]);
+          for (int u = 0; u < 32; ++u) mx[u & 7] = fmaxf(mx[u & 7], sv[u]);
         }
-        tmax = rmax * scale_log2;
       } else {
 #pragma unroll
         for (int c = 0; c < KT; c += 32) {
@@ -212,10 +214,13 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
 #pragma unroll
           for (int u = 0; u < 32; ++u) {
             const int kj = k0 + c + u;
-            if (kj <= qi && kj < n) tmax = fmaxf(tmax, sv[u] * scale_log2);
+            if (kj <= qi && kj < n) mx[u & 7] = fmaxf(mx[u & 7], sv[u]);
           }
         }
       }
+      float tmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                         fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      if (tmax != -INFINITY) tmax *= scale_log2;
       const float mn = fmaxf(m, tmax);
       const float corr = (mn == -INFINITY || m == -INFINITY) ? 1.f : exp2f(m - mn);
       if (j > 0) {
@@ -237,7 +242,10 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
         }
       }
       // pass 2: P = exp2(s - mn) as bf16 into the swizzled K-major tile
-      float lt = 0.f;
+      // (eight partial row sums, one per position in an 8-key chunk)
+      float ls[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) ls[u] = 0.f;
 #pragma unroll
       for (int c = 0; c < KT; c += 32) {
         float sv[32];
@@ -249,14 +257,14 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
               p[u] = ex2_approx(fmaf(sv[c8 * 8 + u], scale_log2, -mn));
-              lt += p[u];
+              ls[u] += p[u];
             }
           } else {
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
               const int kj = k0 + c + c8 * 8 + u;
               p[u] = (kj <= qi && kj < n) ? ex2_approx(fmaf(sv[c8 * 8 + u], scale_log2, -mn)) : 0.f;
-              lt += p[u];
+              ls[u] += p[u];
             }
           }
           __nv_bfloat162 h0 = __floats2bfloat162_rn(p[0], p[1]), h1 = __floats2bfloat162_rn(p[2], p[3]);
@@ -273,6 +281,7 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
       fence_proxy_async();  // P visible to the tensor core
       tc::fence_before();
       mbar_arrive(p_full);
+      const float lt = ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
       l = l * corr + lt;
       m = mn;
     }
