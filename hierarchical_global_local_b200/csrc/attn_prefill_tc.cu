@@ -148,13 +148,12 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
     if (lane == 0) {
       constexpr uint32_t idS = tc::idesc_bf16_m128(KT), idO = tc::idesc_bf16_m128(DH);
       mbar_wait_bounded(q_full, 0, status);
-      for (int j = 0; j < ntiles; ++j) {
+      // S = Q K^T of key tile j (stage j % STAGES) over DH (KB blocks x 4
+      // slices of 16) into the S columns
+      auto issue_s = [&](int j) {
         const int s = j % PL::STAGES;
-        // (S of tile j-1 was consumed before P of tile j-1 was published,
-        // which this thread waited for before the previous P V)
         mbar_wait_bounded(&kv_full[s], (j / PL::STAGES) & 1, status);
         tc::fence_after();
-        // S = Q K^T over DH (KB blocks x 4 slices of 16)
         for (int kb = 0; kb < PL::KB; ++kb) {
           const uint64_t dq = tc::desc_sw128(smem_u32(sm + PL::OFF_Q + kb * QT * 128));
           const uint64_t dk = tc::desc_sw128(smem_u32(sm + PL::OFF_K + s * PL::K_BYTES + kb * KT * 128));
@@ -162,11 +161,18 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
           for (int kk = 0; kk < 4; ++kk) tc::mma_bf16(tS, dq + 2 * kk, dk + 2 * kk, idS, (kb | kk) ? 1u : 0u);
         }
         tc::commit(s_full);
-        // O += P_j V_j over the 128 keys (2 blocks x 4 slices of 16), once P is
-        // written (and O rescaled where the running max moved); O accumulates
-        // in TMEM across the key tiles
+      };
+      issue_s(0);
+      for (int j = 0; j < ntiles; ++j) {
+        const int s = j % PL::STAGES;
+        // P_j is written (the softmax is done reading S_j, and O has been
+        // rescaled where the running max moved): S_{j+1} goes first, so the
+        // softmax's max pass over tile j+1 overlaps P_j V_j
         mbar_wait_bounded(p_full, j & 1, status);
         tc::fence_after();
+        if (j + 1 < ntiles) issue_s(j + 1);
+        // O += P_j V_j over the 128 keys (2 blocks x 4 slices of 16); O
+        // accumulates in TMEM across the key tiles
         for (int kb = 0; kb < KT / 64; ++kb) {
           const uint64_t dp = tc::desc_sw128(smem_u32(sm + PL::OFF_P + kb * QT * 128));
           const uint64_t dv = tc::desc_sw128(smem_u32(sm + PL::OFF_VT + s * PL::VT_BYTES + kb * DH * 128));
