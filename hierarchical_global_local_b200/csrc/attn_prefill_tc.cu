@@ -8,10 +8,14 @@
 // One CTA per (sequence, head, 128-query tile), flash-attention style:
 //   S = Q K^T           tcgen05.mma, M = 128 queries, N = 128 keys, into TMEM
 //   P = softmax pieces  4 warps, one query row per thread (tcgen05.ld), online
-//                       max / sum, causal + tail masking, P written to shared
-//                       memory in the 128-byte-swizzled K-major layout
-//   O_j = P V           tcgen05.mma, M = 128, N = d, K = 128 keys, into TMEM;
-//                       accumulated (with the softmax rescale) in registers
+//                       max / sum, causal + tail masking (only on the
+//                       diagonal and tail tiles), P written to shared memory
+//                       in the 128-byte-swizzled K-major layout
+//   O += P V            tcgen05.mma, M = 128, N = d, K = 128 keys: O stays in
+//                       TMEM across the key tiles and is rescaled there when
+//                       a row's running max grows by more than 8 (log2)
+// The MMA warp issues S of tile j+1 before P_j V_j, so the softmax's max pass
+// over the next tile overlaps P V.
 // Operands come in by TMA with 3-D tensor maps bounded per (sequence, head),
 // so keys / queries past n read as zeros (no stale cache bytes reach the
 // products). V is read through its transpose V^T [B*H][d][n_pad] (written
@@ -227,11 +231,16 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
       float tmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                          fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
       if (tmax != -INFINITY) tmax *= scale_log2;
-      const float mn = fmaxf(m, tmax);
-      const float corr = (mn == -INFINITY || m == -INFINITY) ? 1.f : exp2f(m - mn);
+      // the running max m moves only when the tile's exceeds it by more than
+      // 8 (log2 units): the weights exp2(s - m) then stay below 2^8, which
+      // bf16 holds at the same relative precision, and l uses the same m, so
+      // O / l is unchanged while most tiles skip rescaling O
+      const bool grow = (m == -INFINITY) || (tmax > m + 8.f);
+      const float mn = grow ? fmaxf(m, tmax) : m;
+      const float corr = (!grow || mn == -INFINITY || m == -INFINITY) ? 1.f : exp2f(m - mn);
       if (j > 0) {
         // O holds sum_{i<j} P_i V_i at the old maxima: once P_{j-1} V_{j-1}
-        // is in, rescale the rows whose maximum moved (warp-uniform: the
+        // is in, rescale the rows whose running max moved (warp-uniform: the
         // TMEM accesses are warp-collective), before P_j V_j accumulates
         mbar_wait_bounded(o_full, (j - 1) & 1, status);
         tc::fence_after();
