@@ -73,11 +73,11 @@ constexpr int WORKERS = 128;                 // warps 0-3 (TMEM lanes 0-127)
 constexpr int THREADS = WORKERS + 64;        // warp 4: TMA producer, warp 5: MMA issuer
 constexpr int TILE_BYTES = 128 * 64 * 2;     // one weight box: 128 rows x 64 K (bf16)
 constexpr int MAX_STAGES = 12;
-// K splits: as many as fill the SMs up to these caps. q|k|v|fc1: fewer
-// splits mean fewer partial sums for the reduction phase (measured on B200
-// at D = 768: 2 beats 1 and 3). [W_o | W_2]: the token layers add their
-// splits into h with L2 reductions, so more splits only add reductions
-// (D = 768: 20 splits 170.5 us per token step, 15: 174.4, 12: 174.7).
+// K splits: as many as fill the SMs up to these caps. q|k|v|fc1: fewer splits
+// mean fewer partial sums for the reduction phase (B200, D = 768: 2 beats 1
+// and 3). [W_o | W_2]: the token layers add their splits into fixed-point
+// accumulators by L2 reductions, so more splits only add reductions (D = 768:
+// 20 splits 178.6 us per token step, 15: 178.7, 12: 180.6, 10: 182.6).
 constexpr int MAX_S1 = 2;                    // K splits of the q|k|v|fc1 GEMM
 constexpr int MAX_S2 = 24;                   // K splits of the [W_o | W_2] GEMM
 constexpr int MAX_B = 64;
