@@ -1016,6 +1016,15 @@ __device__ __forceinline__ void warp_argmax32(float* v, int* ix) {
 }
 
 // GL epilogue of vocab tile t: logits (optional) and the tile's argmax per row
+// Greedy argmax through one 64-bit atomicMax per row and vocabulary tile: the
+// logit's order-preserving bits above (-0 counted as +0), 2^32 - 1 - id below,
+// so the largest logit wins and the lowest id among equal ones.
+__device__ __forceinline__ unsigned long long argmax_key(float v, int id) {
+  const unsigned u = __float_as_uint(v + 0.0f);
+  const unsigned ord = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  return ((unsigned long long)ord << 32) | (unsigned long long)(0xFFFFFFFFu - (unsigned)id);
+}
+
 __device__ void lm_epilogue(uint32_t tbuf, int t, const TokenStepArgs& a, int Bp, float2 (*s_arg)[MAX_B]) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t trow = tbuf + ((uint32_t)(warp * 32) << 16);
@@ -1045,7 +1054,7 @@ __device__ void lm_epilogue(uint32_t tbuf, int t, const TokenStepArgs& a, int Bp
       const float2 o = s_arg[w][r];
       if (o.x > best.x || (o.x == best.x && __float_as_int(o.y) < __float_as_int(best.y))) best = o;
     }
-    __stcg(a.arg_part + (size_t)t * a.B + r, best);
+    atomicMax(a.arg_key + r, argmax_key(best.x, __float_as_int(best.y)));
   }
   wsync();  // s_arg is reused by the next tile
 }
@@ -1067,23 +1076,20 @@ __device__ void lm_phase(const TokenStepArgs& a, const Plan& P, const CUtensorMa
 }
 
 // AR: greedy id per row from the tile partials (lowest id on ties)
-__device__ void argmax_phase(const TokenStepArgs& a, const Plan& P) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int b = blockIdx.x * 4 + warp; b < a.B; b += 4 * gridDim.x) {
-    float bv = -INFINITY;
-    int bi = INT_MAX;
-    for (int t = lane; t < P.TL; t += 32) {
-      const float2 o = __ldcg(a.arg_part + (size_t)t * a.B + b);
-      const int oi = __float_as_int(o.y);
-      if (o.x > bv || (o.x == bv && oi < bi)) { bv = o.x; bi = oi; }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
-    }
-    if (lane == 0) a.next[b] = bi;
+// The last CTA out of a completed step: each row's id from its argmax key (the
+// keys reset for the next launch), then the position advances. After an abort
+// only the keys are reset.
+__device__ void finish_step(const TokenStepArgs& a) {
+  const bool aborted = *reinterpret_cast<volatile unsigned*>(&a.bar[2]) != 0u;
+  for (int b = threadIdx.x; b < a.B; b += blockDim.x) {
+    const unsigned long long k = atomicExch(a.arg_key + b, 0ull);
+    if (!aborted) a.next[b] = (int)(0xFFFFFFFFu - (unsigned)(k & 0xFFFFFFFFull));
+  }
+  if (threadIdx.x == 0 && !aborted) {
+    const int t = a.dstate[0] + 1;
+    a.dstate[0] = t;
+    a.dstate[1] = t % a.L_B;
+    a.dstate[2] = t / a.L_B;
   }
 }
 
@@ -1105,6 +1111,7 @@ token_step_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
   __shared__ float red[4];
   __shared__ float2 s_arg[4][MAX_B];
   __shared__ volatile int s_abort;
+  __shared__ int s_last;
   __shared__ __align__(8) uint64_t att_bar[4 * ATT_SLOTS];  // block-step attention slots
   __shared__ float q_s[4 * 64];
 
@@ -1202,19 +1209,9 @@ token_step_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
       r2_phase(a, P, l, red);
       ok = grid_sync(a, ++nb * G, &s_abort);
     }
-    if (ok) {
-      lm_phase(a, P, &mxf, act, tmem, y, na, nu, s_arg);
-      ok = grid_sync(a, ++nb * G, &s_abort);
-    }
-    if (ok) {
-      argmax_phase(a, P);
-      if (blockIdx.x == 0 && threadIdx.x == 0) {
-        const int t = a.dstate[0] + 1;
-        a.dstate[0] = t;
-        a.dstate[1] = t % a.L_B;
-        a.dstate[2] = t / a.L_B;
-      }
-    }
+    // the LM tiles' epilogues fold each row's best (logit, id) into
+    // a.arg_key; the last CTA out turns the keys into ids (finish_step)
+    if (ok) lm_phase(a, P, &mxf, act, tmem, y, na, nu, s_arg);
     // workers that stop early (abort) release the MMA warp's waits
     if (!ok && threadIdx.x == 0) s_abort = 1;
   }
@@ -1222,8 +1219,11 @@ token_step_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
   tc::fence_before();
   __syncthreads();
   if (warp == 0) tc::tmem_free(tmem, TMEM_COLS);
-  // every CTA counts itself out only after its last barrier wait
-  if (threadIdx.x == 0) grid_exit(a.bar);
+  // every CTA counts itself out only after its last barrier wait and its
+  // argmax updates (ordered before thread 0 by the CTA barrier above)
+  if (threadIdx.x == 0) s_last = grid_exit(a.bar) ? 1 : 0;
+  __syncthreads();
+  if (s_last) finish_step(a);
 }
 
 // ---- host side -----------------------------------------------------------------
@@ -1396,7 +1396,7 @@ cudaError_t launch_token_step(const TokenStepArgs& a, const void* w_qkv1, const 
                   !token_step_block_supported(DT_BF16, a.B, a.D, a.H, a.rot, a.V, a.Nt, a.Nb, 1, a.l_cap,
                                               a.n_cap, a.L_B)))
     return cudaErrorNotSupported;
-  if (!a.fx || (reinterpret_cast<uintptr_t>(a.fx) & 15)) return cudaErrorInvalidValue;
+  if (!a.fx || (reinterpret_cast<uintptr_t>(a.fx) & 15) || !a.arg_key) return cudaErrorInvalidValue;
   Device& d = device();
   Plan P;
   size_t smem;

@@ -57,16 +57,20 @@ __device__ __forceinline__ bool grid_barrier(unsigned* bar, unsigned target, lon
   return !*s_abort;
 }
 
-// Called once by thread 0 of every CTA after its last barrier wait: the last
+// Called once by thread 0 of every CTA after its last barrier wait (and
+// after a CTA barrier that orders the CTA's other writes before it): the last
 // CTA out resets the arrival and exit counters for the next launch (the abort
-// word stays set until the host clears it).
-__device__ __forceinline__ void grid_exit(unsigned* bar) {
+// word stays set until the host clears it) and gets true; every CTA's writes
+// before its exit are then visible to it.
+__device__ __forceinline__ bool grid_exit(unsigned* bar) {
   __threadfence();
   if (atomicAdd(&bar[1], 1u) == gridDim.x - 1) {
     bar[0] = 0u;
     bar[1] = 0u;
     __threadfence();
+    return true;
   }
+  return false;
 }
 
 }  // namespace bt

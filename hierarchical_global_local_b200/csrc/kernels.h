@@ -253,6 +253,7 @@ struct TokenStepArgs {
   float* logits;
   int32_t* next;
   float2* arg_part;  // [ceil(V/128), B]
+  unsigned long long* arg_key;  // token_step: [B] argmax keys, zero between launches (the last CTA resets them)
   float *p1, *p2;    // split-K partials (token_step_scratch_floats)
   long long* fx;     // token_step: [B, D] int64 fixed-point split-K sums (units of 2^-32),
                      // zero between launches (each launch clears what it adds)

@@ -172,6 +172,7 @@ struct bt_model {
   int* ln_cnt = nullptr;       // per-row counters of the LayerNorm fused into GEMM epilogues
   float *ts_p1 = nullptr, *ts_p2 = nullptr;  // fused token step: split-K partials
   long long* ts_fx = nullptr;                // fused token step: fixed-point split-K sums [Bmax][D]
+  unsigned long long* ts_key = nullptr;      // fused token step: argmax keys [Bmax]
   unsigned* ts_bar = nullptr;                // fused token step: grid-barrier words
   float* ts_att = nullptr;                   // fused block step: decode-attention partials
   int* ts_cnt = nullptr;                     // fused block step: merge counters [B_max * H]
@@ -313,6 +314,7 @@ static size_t carve(bt_model* m, const Dims& d, void* ws) {
                                        token_step2_scratch_floats(d.Bmax, d.D, 2)) * 4);
     m->ts_bar = (unsigned*)c.take(64);
     m->ts_fx = (long long*)c.take((size_t)d.Bmax * d.D * sizeof(long long));
+    m->ts_key = (unsigned long long*)c.take((size_t)d.Bmax * sizeof(unsigned long long));
     m->ts_att = (float*)c.take(token_step_scratch_floats(d.Bmax, d.D, 3, d.H, d.n_cap) * 4);
     m->ts_cnt = (int*)c.take((size_t)d.Bmax * d.H * sizeof(int));
     m->ts2_ctr_bytes = token_step2_counter_bytes(d.D);
@@ -440,6 +442,7 @@ int bt_create(const bt_config* cfg, const bt_weights* w, void* ws, size_t ws_byt
   BT_TRYC(cudaMemsetAsync(m->ln_cnt, 0, (size_t)d.Bmax * (d.P > 1 ? d.P : 1) * sizeof(int), st));
   if (m->ts_bar) BT_TRYC(cudaMemsetAsync(m->ts_bar, 0, 64, st));
   if (m->ts_fx) BT_TRYC(cudaMemsetAsync(m->ts_fx, 0, (size_t)d.Bmax * d.D * sizeof(long long), st));
+  if (m->ts_key) BT_TRYC(cudaMemsetAsync(m->ts_key, 0, (size_t)d.Bmax * sizeof(unsigned long long), st));
   if (m->ts_cnt) BT_TRYC(cudaMemsetAsync(m->ts_cnt, 0, (size_t)d.Bmax * d.H * sizeof(int), st));
   if (m->ts2_ctr) BT_TRYC(cudaMemsetAsync(m->ts2_ctr, 0, m->ts2_ctr_bytes, st));
   {
@@ -893,7 +896,8 @@ static int run_token_step(bt_model* m, int B, bool ingest, PosSpec pos, const in
   a.rope_tab = m->rope_tab; a.lnf_g = m->lnf_t_g; a.lnf_b = m->lnf_t_b;
   a.h = m->h_t; a.x1 = (bf16*)m->x1; a.a2 = (bf16*)m->a2; a.xf = (bf16*)m->xf;
   a.logits = want_logits ? m->logits : nullptr; a.next = m->next; a.arg_part = m->arg_part;
-  a.p1 = m->ts_p1; a.p2 = m->ts_p2; a.fx = m->ts_fx; a.bar = m->ts_bar; a.status = m->status;
+  a.p1 = m->ts_p1; a.p2 = m->ts_p2; a.fx = m->ts_fx; a.arg_key = m->ts_key; a.bar = m->ts_bar;
+  a.status = m->status;
   a.wait_cycles = m->wait_cycles;
   a.l2_window_base = m->l2_base;
   a.l2_window_bytes = m->l2_window;
@@ -1070,6 +1074,7 @@ static int prefill_impl(bt_model* m, const int32_t* tokens, int T_stride, int B,
   if (m->ts_bar) BT_CUDA(cudaMemsetAsync(m->ts_bar, 0, 64, s));
   // and its fixed-point accumulators (an aborted step can leave sums in them)
   if (m->ts_fx) BT_CUDA(cudaMemsetAsync(m->ts_fx, 0, (size_t)d.Bmax * d.D * sizeof(long long), s));
+  if (m->ts_key) BT_CUDA(cudaMemsetAsync(m->ts_key, 0, (size_t)d.Bmax * sizeof(unsigned long long), s));
   if (m->ts_cnt) BT_CUDA(cudaMemsetAsync(m->ts_cnt, 0, (size_t)d.Bmax * d.H * sizeof(int), s));
   if (m->ts2_ctr) BT_CUDA(cudaMemsetAsync(m->ts2_ctr, 0, m->ts2_ctr_bytes, s));
   const long long k0 = launch_count();
