@@ -3,11 +3,12 @@
 // * Block-decoder decode attention: one new block per sequence attends over
 //   its n cached block entries ("Block Transformer: Global-to-Local Language
 //   Modeling for Fast Inference", §3.4 "The Block Decoder": the KV cache is
-//   L_B times shorter and read once per L_B tokens). Split-K flash decoding:
-//   each CTA streams one chunk of K and V rows of one (sequence, head) into
-//   shared memory with a 1-D bulk copy, computes chunk-local softmax
-//   statistics (m, l) and o, and the last CTA of a (sequence, head) merges
-//   the chunks: o = sum_s e^{m_s - M} o_s / sum_s e^{m_s - M} l_s. No CTA
+//   L_B times shorter and read once per L_B tokens). Flash decoding: a
+//   persistent grid streams chunks of K and V rows into shared memory with
+//   1-D bulk copies and keeps an online softmax (m, l, o). With enough
+//   (sequence, head) pairs each CTA takes whole pairs; with few, a pair's
+//   chunks are split over several CTAs and the last of them merges the
+//   partials: o = sum_s e^{m_s - M} o_s / sum_s e^{m_s - M} l_s. No CTA
 //   waits for another (last-arriver merge through an atomic counter).
 // * Token-decoder local attention: each new row attends over at most
 //   P + L_B - 1 rows of its own block (§3.4 "The Token Decoder"); one warp per
